@@ -1,0 +1,344 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each check comes from the mathematics, a library routine the oracle does not call
+(numpy, torch, transformers' Llama), a closed form, or a worked example in
+tests/golden.  They are chosen so that a dropped term, a wrong sign or index, a
+transposed operand or a wrong head grouping in the oracle fails at least one.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import mk_inputs as mi
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_splitmix64_matches_published_values():
+    import ctypes
+    want = [int(l, 16) for l in open(os.path.join(GOLDEN, "splitmix64_state0.txt")) if l.startswith("0x")]
+    st = ctypes.c_uint64(0)
+    got = [mi.lib().mki_splitmix64_next(st) for _ in want]
+    assert got == want
+
+
+def test_generator_is_counter_based_and_normal():
+    a = mi.normal_bf16(0, 77, (3_000_001,), sigma=0.02)
+    b = mi.normal_bf16(0, 77, (1000,), sigma=0.02)
+    assert np.array_equal(a[:1000], b)  # prefix property: element i depends only on i
+    f = mi.bf16_to_f32(a).astype(np.float64)
+    assert abs(f.mean()) < 1e-4 and abs(f.std() - 0.02) < 1e-4
+    t = mi.tokens(0, 5, 10000, 1000)
+    assert t.min() >= 0 and t.max() < 1000 and len(np.unique(t)) > 990
+
+
+# ---------------------------------------------------------------- RMSNorm
+
+def test_rmsnorm_constant_vector_closed_form():
+    # RMSNorm(c * 1) = c / sqrt(c^2 + eps) * g
+    for c, eps in [(3.0, 1e-6), (-0.5, 1e-5), (1e-3, 1e-5)]:
+        g = np.linspace(0.5, 2.0, 64)
+        y = oracle.rmsnorm(np.full(64, c), g, eps)
+        assert np.allclose(y, c / math.sqrt(c * c + eps) * g, rtol=1e-14, atol=0)
+
+
+def test_rmsnorm_matches_torch_and_is_scale_invariant():
+    rng = np.random.default_rng(1)
+    x, g = rng.normal(size=300), rng.normal(size=300)
+    y = oracle.rmsnorm(x, g, 1e-5)
+    ref = torch.nn.functional.rms_norm(torch.tensor(x), (300,), torch.tensor(g), eps=1e-5).numpy()
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-14)
+    # RMSNorm(a x) = RMSNorm(x) up to the eps term: relative change <= eps / (2 mean(x^2))
+    assert np.allclose(oracle.rmsnorm(1000 * x, g, 1e-5), y, rtol=1e-5 / np.mean(x * x))
+
+
+# ---------------------------------------------------------------- matvec
+
+def test_matvec_matches_numpy_on_non_square_shapes():
+    w = mi.normal_bf16(3, 9, (37, 53), sigma=0.5)
+    x = np.random.default_rng(2).normal(size=53)
+    ref = mi.bf16_to_f32(w).astype(np.float64) @ x
+    assert np.allclose(oracle.matvec_bf16(w, x), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_norm_then_linear_equals_linear_then_divide():
+    # Mirage article, "Case 1: Normalization + Linear": RMSNorm(x) W = ((x * g) W) / rms(x).
+    rng = np.random.default_rng(3)
+    H, N, eps = 128, 40, 1e-5
+    x, g = rng.normal(size=H), rng.normal(size=H)
+    w = mi.normal_bf16(0, 11, (N, H), sigma=0.1)
+    lhs = oracle.matvec_bf16(w, oracle.rmsnorm(x, g, eps))
+    rms = math.sqrt(np.mean(x * x) + eps)
+    rhs = oracle.matvec_bf16(w, x * g) / rms
+    assert np.allclose(lhs, rhs, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- RoPE
+
+def test_rope_position_zero_is_identity():
+    v = np.random.default_rng(4).normal(size=128)
+    assert np.array_equal(oracle.rope(v, 0, 5e5), v)
+
+
+def test_rope_two_dims_is_plane_rotation():
+    # d = 2: one pair with inverse frequency theta^0 = 1, so position p rotates by p radians.
+    for p in (1, 2, 7):
+        out = oracle.rope(np.array([1.0, 0.0]), p, 1e4)
+        assert np.allclose(out, [math.cos(p), math.sin(p)], atol=1e-15)
+
+
+def test_rope_pairs_i_with_i_plus_half():
+    # a one-hot at index 1 of a 8-dim head must rotate into index 1 + 4 (rotate-half pairing),
+    # with the angle of pair 1: p * theta^(-2/8).
+    d, p, theta = 8, 3, 100.0
+    e = np.zeros(d)
+    e[1] = 1.0
+    out = oracle.rope(e, p, theta)
+    ang = p * theta ** (-2.0 / d)
+    want = np.zeros(d)
+    want[1], want[5] = math.cos(ang), math.sin(ang)
+    assert np.allclose(out, want, atol=1e-15)
+
+
+def test_rope_preserves_pair_norms_and_is_relative():
+    rng = np.random.default_rng(5)
+    d = 64
+    q, k = rng.normal(size=d), rng.normal(size=d)
+    rq = oracle.rope(q, 11, 1e4)
+    half = d // 2
+    assert np.allclose(rq[:half] ** 2 + rq[half:] ** 2, q[:half] ** 2 + q[half:] ** 2, rtol=1e-12)
+    # <R_m q, R_n k> depends on m - n only
+    a = oracle.rope(q, 17, 1e4) @ oracle.rope(k, 5, 1e4)
+    b = oracle.rope(q, 112, 1e4) @ oracle.rope(k, 100, 1e4)
+    assert abs(a - b) < 1e-10
+
+
+# ---------------------------------------------------------------- attention
+
+def _golden_attention():
+    rows = {}
+    for line in open(os.path.join(GOLDEN, "attention_two_keys.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        key, *vals = line.split()
+        rows.setdefault(key, []).append([float(v) for v in vals])
+    return rows
+
+
+def test_attention_worked_example():
+    g = _golden_attention()
+    o, p = oracle.attention_head(np.array(g["q"][0]), np.array(g["k"]), np.array(g["v"]), 1.0)
+    assert np.allclose(p, g["probs"][0], atol=1e-15)
+    assert np.allclose(o, g["o"][0], atol=1e-14)
+
+
+def test_attention_single_key_returns_v_and_equal_keys_return_mean():
+    rng = np.random.default_rng(6)
+    q, v = rng.normal(size=16), rng.normal(size=(5, 16))
+    o, p = oracle.attention_head(q, rng.normal(size=(1, 16)), v[:1], 0.25)
+    assert np.allclose(o, v[0], atol=1e-15) and p[0] == 1.0
+    k = np.repeat(rng.normal(size=(1, 16)), 5, axis=0)
+    o, p = oracle.attention_head(q, k, v, 0.25)
+    assert np.allclose(o, v.mean(axis=0), atol=1e-14)
+    assert np.allclose(p, 0.2, atol=1e-15)
+
+
+def test_attention_matches_torch_sdpa_and_probs_sum_to_one():
+    rng = np.random.default_rng(7)
+    for L, d, scale in [(1, 8, 1.0), (37, 64, 0.125), (300, 128, 1 / math.sqrt(128))]:
+        q, k, v = rng.normal(size=d), rng.normal(size=(L, d)), rng.normal(size=(L, d))
+        o, p = oracle.attention_head(q, k, v, scale)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q)[None, None, None], torch.tensor(k)[None, None], torch.tensor(v)[None, None],
+            scale=scale)[0, 0, 0].numpy()
+        assert np.allclose(o, ref, rtol=1e-12, atol=1e-13)
+        assert abs(p.sum() - 1.0) < 1e-12
+
+
+def test_standalone_attention_f16_matches_torch_sdpa():
+    # The Mirage example's form: fp16 inputs, K given transposed [BH, d, L], no scaling.
+    BH, d, L = 3, 128, 200
+    q = mi.normal_f16(0, 1, (BH, d))
+    kt = mi.normal_f16(0, 2, (BH, d, L))
+    v = mi.normal_f16(0, 3, (BH, L, d))
+    o = oracle.attention_decode_f16(q, kt, v, 1.0)
+    qt = torch.tensor(mi.f16_to_f32(q), dtype=torch.float64)
+    kk = torch.tensor(mi.f16_to_f32(kt), dtype=torch.float64).transpose(1, 2)
+    vv = torch.tensor(mi.f16_to_f32(v), dtype=torch.float64)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt[:, None], kk, vv, scale=1.0)[:, 0].numpy()
+    assert np.allclose(o, ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- SiLU
+
+def test_silu_special_values_and_torch():
+    assert oracle.silu(0.0) == 0.0
+    assert abs(oracle.silu(40.0) - 40.0) < 1e-12
+    assert abs(oracle.silu(-40.0)) < 1e-15
+    z = np.linspace(-8, 8, 33)
+    ref = torch.nn.functional.silu(torch.tensor(z)).numpy()
+    assert np.allclose([oracle.silu(t) for t in z], ref, rtol=1e-14, atol=1e-15)
+
+
+def test_argmax_ties_take_lowest_index():
+    x = np.array([0.0, 3.0, -1.0, 3.0, 2.0], dtype=np.float32)
+    assert oracle.argmax(x) == 1
+
+
+# ---------------------------------------------------------------- whole decoder
+
+def _hf_llama(w):
+    """transformers' Llama (an independent implementation), float64, same weights."""
+    from transformers import LlamaConfig, LlamaForCausalLM
+    s = w.shape
+    cfg = LlamaConfig(vocab_size=s.vocab, hidden_size=s.hidden, intermediate_size=s.ffn,
+                      num_hidden_layers=s.n_layers, num_attention_heads=s.n_q_heads,
+                      num_key_value_heads=s.n_kv_heads, head_dim=s.head_dim, rms_norm_eps=s.rms_eps,
+                      rope_theta=s.rope_theta, max_position_embeddings=4096, tie_word_embeddings=False,
+                      attention_bias=False, mlp_bias=False)
+    cfg._attn_implementation = "eager"
+    m = LlamaForCausalLM(cfg).to(torch.float64).eval()
+
+    def t(a):
+        return torch.tensor(mi.bf16_to_f32(a), dtype=torch.float64)
+
+    with torch.no_grad():
+        m.model.embed_tokens.weight.copy_(t(w.embed))
+        m.lm_head.weight.copy_(t(w.lm_head))
+        m.model.norm.weight.copy_(t(w.final_norm))
+        for l, layer in enumerate(m.model.layers):
+            layer.input_layernorm.weight.copy_(t(w.attn_norm[l]))
+            layer.post_attention_layernorm.weight.copy_(t(w.mlp_norm[l]))
+            layer.self_attn.q_proj.weight.copy_(t(w.wq[l]))
+            layer.self_attn.k_proj.weight.copy_(t(w.wk[l]))
+            layer.self_attn.v_proj.weight.copy_(t(w.wv[l]))
+            layer.self_attn.o_proj.weight.copy_(t(w.wo[l]))
+            layer.mlp.gate_proj.weight.copy_(t(w.wg[l]))
+            layer.mlp.up_proj.weight.copy_(t(w.wu[l]))
+            layer.mlp.down_proj.weight.copy_(t(w.wd[l]))
+    return m
+
+
+def _random_gains(w, seed=9):
+    # gains are 1 in every config; random gains here make a dropped gain visible
+    H = w.shape.hidden
+    w.final_norm = mi.normal_bf16(seed, 50, (H,), sigma=0.3, mean=1.0)
+    for l in range(w.shape.n_layers):
+        w.attn_norm[l] = mi.normal_bf16(seed, 51 + 2 * l, (H,), sigma=0.3, mean=1.0)
+        w.mlp_norm[l] = mi.normal_bf16(seed, 52 + 2 * l, (H,), sigma=0.3, mean=1.0)
+    return w
+
+
+@pytest.fixture(scope="module")
+def tiny_weights():
+    return _random_gains(mi.make_weights(mi.TINY, seed=0, sigma=0.05))
+
+
+def test_decoder_matches_transformers_llama(tiny_weights):
+    w = tiny_weights
+    T = 12
+    toks = mi.prompt(0, 0, T + 3, w.shape.vocab)
+    m = _hf_llama(w)
+    with torch.no_grad():
+        ref = m(torch.tensor(toks[None].astype(np.int64)), use_cache=False).logits[0].numpy()
+    d = oracle.Decoder(w, 1, 64, f64=True, kv_round=False)
+    got = [d.prefill(toks[:T])[0]]
+    for t in range(T, T + 3):
+        got.append(d.decode_f64(toks[t:t + 1])[0])
+    got = np.stack(got)
+    want = ref[T - 1:]
+    # transformers computes RoPE angles, the norm and the softmax in fp32
+    assert np.max(np.abs(got - want)) < 2e-5 * np.max(np.abs(want))
+
+
+def test_gqa_equals_mha_with_replicated_kv_heads(tiny_weights):
+    # GQA with kv head floor(h*nkv/nq) == MHA whose K/V weight rows repeat each kv head nq/nkv times.
+    w = tiny_weights
+    s = w.shape
+    rep = s.n_q_heads // s.n_kv_heads
+    import copy
+    w2 = copy.copy(w)
+    w2.shape = mi.Shape("tiny-mha", s.n_layers, s.hidden, s.n_q_heads, s.n_q_heads, s.head_dim, s.ffn, s.vocab,
+                        s.rms_eps, s.rope_theta)
+    D = s.head_dim
+    w2.wk = [np.ascontiguousarray(np.repeat(a.reshape(s.n_kv_heads, D, s.hidden), rep, axis=0).reshape(-1, s.hidden))
+             for a in w.wk]
+    w2.wv = [np.ascontiguousarray(np.repeat(a.reshape(s.n_kv_heads, D, s.hidden), rep, axis=0).reshape(-1, s.hidden))
+             for a in w.wv]
+    toks = mi.prompt(0, 1, 9, s.vocab)
+    a = oracle.Decoder(w, 1, 32, f64=True, kv_round=False).prefill(toks)
+    b = oracle.Decoder(w2, 1, 32, f64=True, kv_round=False).prefill(toks)
+    assert np.allclose(a, b, rtol=1e-13, atol=1e-13)
+
+
+def test_prefill_equals_token_by_token_decode(tiny_weights):
+    w = tiny_weights
+    toks = mi.prompt(0, 2, 10, w.shape.vocab)
+    a = oracle.Decoder(w, 1, 32, f64=True).prefill(toks)
+    d = oracle.Decoder(w, 1, 32, f64=True)
+    d.prefill(toks[:1])
+    for t in range(1, 10):
+        b = d.decode_f64(toks[t:t + 1])
+    # prefill hands back fp32 logits; the decode path keeps fp64
+    assert np.allclose(a, b, rtol=1e-6, atol=1e-7)
+
+
+def test_fp32_mode_tracks_fp64_mode(tiny_weights):
+    w = tiny_weights
+    toks = mi.prompt(0, 3, 16, w.shape.vocab)
+    a = oracle.Decoder(w, 1, 64, f64=False, kv_round=False)
+    b = oracle.Decoder(w, 1, 64, f64=True, kv_round=False)
+    la, lb = a.prefill(toks), b.prefill(toks)
+    for t in range(4):
+        tok = np.array([oracle.argmax(lb[0])], dtype=np.int32)
+        la, lb = a.decode(tok), b.decode_f64(tok)
+        assert np.max(np.abs(la - lb)) < 1e-5 * max(1.0, np.max(np.abs(lb)))
+
+
+def test_kv_cache_holds_bf16_rounded_keys_and_values(tiny_weights):
+    w = tiny_weights
+    toks = mi.prompt(0, 4, 8, w.shape.vocab)
+    a = oracle.Decoder(w, 1, 16, f64=True, kv_round=True)
+    b = oracle.Decoder(w, 1, 16, f64=True, kv_round=False)
+    a.prefill(toks)
+    b.prefill(toks)
+    ca, cb = mi.bf16_to_f32(a.get_cache(8)), mi.bf16_to_f32(b.get_cache(8))
+    # the first layer sees identical inputs, so its K/V differ only by the storage rounding
+    assert np.array_equal(ca[0], cb[0])
+    assert not np.all(ca == 0)
+
+
+def test_batch_rows_are_independent(tiny_weights):
+    w = tiny_weights
+    p0, p1 = mi.prompt(0, 5, 6, w.shape.vocab), mi.prompt(0, 6, 6, w.shape.vocab)
+    both = oracle.Decoder(w, 2, 16).prefill(np.stack([p0, p1]))
+    one = oracle.Decoder(w, 1, 16).prefill(p1)
+    assert np.array_equal(both[1], one[0])
+
+
+def test_set_cache_then_decode_equals_prefill_then_decode(tiny_weights):
+    w = tiny_weights
+    toks = mi.prompt(0, 7, 9, w.shape.vocab)
+    a = oracle.Decoder(w, 1, 16)
+    a.prefill(toks[:8])
+    kv = a.get_cache(8)
+    want = a.decode(toks[8:9])
+    b = oracle.Decoder(w, 1, 16)
+    b.set_cache(kv, 8)
+    assert b.position(0) == 8
+    assert np.array_equal(b.decode(toks[8:9]), want)
+
+
+def test_thread_count_does_not_change_results(tiny_weights):
+    w = mi.make_weights(mi.TINY.with_layers(1), seed=1)
+    toks = mi.prompt(0, 8, 5, w.shape.vocab)
+    oracle.set_threads(1)
+    a = oracle.Decoder(w, 1, 8).prefill(toks)
+    oracle.set_threads(7)
+    b = oracle.Decoder(w, 1, 8).prefill(toks)
+    oracle.set_threads(0)
+    assert np.array_equal(a, b)
