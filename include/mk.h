@@ -1,0 +1,187 @@
+/*
+ * mk.h -- C ABI of the persistent decode megakernel for B200 (sm_100a).
+ *
+ * One Llama-style decoder step (RMSNorm, QKV projection + RoPE, KV-cache append, decode
+ * attention, O-projection + residual, SwiGLU MLP, final norm + LM head) is lowered on the
+ * host into a task graph of tiles linked by dependency events, and one persistent kernel
+ * with one CTA per SM runs the whole step.  The method is the one described in
+ * "Compiler des LLM en MegaKernel pour obtenir une inference a faible latence"
+ * (fr.news.hada.io summary of the Mirage Persistent Kernel post): Part 1 "Compilateur"
+ * (computation graph -> task graph of tasks and events), Part 2 "Runtime" (workers,
+ * schedulers, event-driven execution).  The per-op definitions follow the Mirage article
+ * (iaiol.com): the attention example O = softmax(Q K) V, "Case 1: Normalization + Linear"
+ * and "Case 3: Gated MLP".
+ *
+ * Conventions for every entry point:
+ *   - Plain C types only.  `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *     default stream).  Device pointers are raw CUDA device addresses the CALLER owns
+ *     (allocated e.g. with torch); the library never frees them.
+ *   - Calls that take a stream are asynchronous and stream-ordered.
+ *   - Every int-returning function returns MK_OK (0) or a negative MK_ERR_* code and never
+ *     aborts or throws.  mk_last_error() then holds a one-line description.
+ *   - Device-side timeouts (a dependency wait that ran out) are reported by the next
+ *     mk_sync_status() on the stream that ran the step.
+ *   - bf16 / fp16 values are passed as uint16_t bit patterns.
+ */
+#ifndef MK_H
+#define MK_H
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MK_OK 0
+#define MK_ERR_INVALID_ARG (-1)    /* a pointer, size or config field is out of range */
+#define MK_ERR_CUDA (-2)           /* a CUDA runtime call failed (text in mk_last_error) */
+#define MK_ERR_DEVICE_TIMEOUT (-3) /* a device-side dependency wait exceeded its limit */
+#define MK_ERR_NOT_RESIDENT (-4)   /* the persistent grid cannot be co-resident on the GPU */
+#define MK_ERR_STATE (-5)          /* call out of order (e.g. decode before load) */
+#define MK_ERR_UNSUPPORTED (-6)    /* valid config this build has no kernel instantiation for */
+
+/* Model and capacity.  Decoder shape as in the pages' workloads (Llama-3-8B shape for the
+ * MPK decode benchmark, "Valeur cle de MPK"; Chameleon-7B / Llama-3-8B shapes in the Mirage
+ * article's end-to-end figure).  Requirements checked by mk_build_taskgraph:
+ * hidden == n_q_heads * head_dim; n_q_heads % n_kv_heads == 0; head_dim in {64, 128};
+ * hidden and ffn multiples of 8; max_batch in [1, MK_MAX_BATCH]; tie_embeddings == 0. */
+typedef struct mk_config {
+  int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
+  float rms_eps, rope_theta;
+  int max_batch, max_seq;
+  int tie_embeddings; /* must be 0: separate LM-head matrix */
+} mk_config;
+
+#define MK_MAX_BATCH 16
+
+/* Host weights: bf16 bit patterns, canonical [out, in] row-major; per-layer arrays hold
+ * n_layers pointers.  Read once by mk_load_weights; the caller keeps ownership. */
+typedef struct mk_host_weights {
+  const uint16_t* embed;      /* [vocab, hidden] */
+  const uint16_t* lm_head;    /* [vocab, hidden] */
+  const uint16_t* final_norm; /* [hidden] */
+  const uint16_t* const* attn_norm; /* [hidden] */
+  const uint16_t* const* wq;  /* [n_q_heads*head_dim, hidden] */
+  const uint16_t* const* wk;  /* [n_kv_heads*head_dim, hidden] */
+  const uint16_t* const* wv;  /* [n_kv_heads*head_dim, hidden] */
+  const uint16_t* const* wo;  /* [hidden, n_q_heads*head_dim] */
+  const uint16_t* const* mlp_norm; /* [hidden] */
+  const uint16_t* const* wg;  /* [ffn, hidden] */
+  const uint16_t* const* wu;  /* [ffn, hidden] */
+  const uint16_t* const* wd;  /* [hidden, ffn] */
+} mk_host_weights;
+
+typedef struct mk_ctx mk_ctx; /* opaque, library-owned host object */
+
+/* Lower one decoder step of `cfg` into the task graph for `device` (Part 1 "Compilateur":
+ * every op split into per-SM tile tasks; events with thresholds equal to their producer
+ * counts; per-SM queues in a topological order), validate it on the CPU (acyclic, counts
+ * consistent, every read ordered after its writes, no queue can deadlock) and size the
+ * arenas.  Allocates no device memory.  *out receives the context (NULL on error). */
+int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out);
+
+/* Sizes (bytes) of the three device buffers the caller allocates.  The weight arena holds
+ * the packed bf16 weights; the workspace holds the task graph, event counters, activations
+ * and prefill scratch; the KV cache is bf16 in the layout
+ * [layer][K=0|V=1][max_batch][n_kv_heads][max_seq][head_dim].  All need 256-byte alignment. */
+size_t mk_weight_arena_bytes(const mk_ctx* ctx);
+size_t mk_workspace_bytes(const mk_ctx* ctx);
+size_t mk_kv_cache_bytes(const mk_ctx* ctx);
+
+/* Pack the host weights into tile order (QKV rows grouped per KV head with RoPE pairs
+ * adjacent; gate/up rows interleaved) and copy them to `weight_arena`; upload the task
+ * graph and RoPE table into `workspace` and zero its event counters.  Both buffers must
+ * stay allocated and unmoved until mk_destroy.  Synchronises `stream` before returning. */
+int mk_load_weights(mk_ctx* ctx, const mk_host_weights* w, void* weight_arena, void* workspace, void* stream);
+
+/* Prefill (the hybrid arrangement of "Ada-MK: Adaptive MegaKernel Optimization via
+ * Automated DAG-based Search for LLM Inference", section 3: prompt on ordinary kernels,
+ * decode on the megakernel).  tokens: device int32 [B][T]; fills positions 0..T-1 of
+ * the cache for sequences 0..B-1 and sets their positions to T.  last_logits: device fp32
+ * [B][vocab] for the last prompt token, or NULL.  B <= max_batch, T <= max_seq. */
+int mk_prefill(mk_ctx* ctx, const int32_t* tokens, int B, int T, void* kv_cache, float* last_logits,
+               void* stream);
+
+/* Declare that the caller filled the cache itself: sequence b (b < B) has host_pos[b]
+ * valid positions.  Sets the active batch to B. */
+int mk_set_positions(mk_ctx* ctx, const int32_t* host_pos, int B);
+/* Current positions of the active batch (host copy kept by the library); returns B. */
+int mk_get_positions(const mk_ctx* ctx, int32_t* host_pos, int capacity);
+
+/* One decode step of the active batch: one launch of the persistent megakernel.
+ * tokens: device int32 [B], token b goes in at position pos[b]; logits: device fp32
+ * [B][vocab]; next_tokens: device int32 [B] (greedy argmax, lowest index on ties) or NULL.
+ * Appends K/V at pos[b] and advances every position by one. */
+int mk_decode_step(mk_ctx* ctx, const int32_t* tokens, void* kv_cache, float* logits, int32_t* next_tokens,
+                   void* stream);
+
+/* Synchronise `stream` and report the device status of the steps run on it:
+ * MK_OK, or MK_ERR_DEVICE_TIMEOUT (the event counters are then reset so the context
+ * stays usable; the cache contents of the failed step are undefined). */
+int mk_sync_status(mk_ctx* ctx, void* stream);
+
+/* Limit of every device-side wait, in nanoseconds (default 2e9).  Must be > 0. */
+int mk_set_wait_timeout_ns(mk_ctx* ctx, uint64_t ns);
+
+/* Test hook for failure detection: while `on` is nonzero, the next decode steps skip the
+ * notify of event `event_id` (as if its producer never finished), so every task waiting
+ * on it times out after the wait limit and the step reports MK_ERR_DEVICE_TIMEOUT.
+ * Nothing faults or traps. */
+int mk_debug_drop_notify(mk_ctx* ctx, int event_id, int on);
+
+/* Tracing (per-task timing of the next decode steps).  device_buffer: n_tasks * 6 uint64
+ * records (n_tasks from mk_get_graph_info), or NULL to switch tracing off.  Record of task i
+ * (global-timer ns): [0] worker starts waiting for the task's inputs, [1] inputs released by
+ * the scheduler, [2] task done, [3] low 32 bits: worker ns blocked on weight-ring stages,
+ * high 32 bits: SM, [4] producer ns blocked on a full ring while issuing the task's weight
+ * stages, [5] time of the task's first weight issue.  Each step overwrites the records. */
+int mk_set_trace(mk_ctx* ctx, void* device_buffer);
+
+/* Task-graph introspection (for tests and the bench). */
+typedef struct mk_graph_info {
+  int n_sms;         /* workers = resident CTAs of the persistent grid */
+  int n_tasks, n_events;
+  int attn_chunks;   /* split-KV chunks per (sequence, KV head) */
+  int kernel_variant;/* index of the compiled instantiation chosen for this shape */
+  uint64_t weight_bytes_per_step; /* bf16 weights streamed by one decode step */
+  uint64_t smem_bytes;            /* dynamic shared memory per CTA */
+} mk_graph_info;
+int mk_get_graph_info(const mk_ctx* ctx, mk_graph_info* out);
+
+/* Flat copy of the task graph: per task {kind, layer, sm, row0, nrows, n_wait, wait0,
+ * wait1, n_notify, notify0, notify1} as 11 int32; per event its per-step count.  Returns
+ * the number of tasks (or a negative error); either buffer may be NULL to query sizes. */
+int mk_export_taskgraph(const mk_ctx* ctx, int32_t* tasks, int task_capacity, int32_t* event_counts,
+                        int event_capacity);
+
+/* Validate an exported-and-edited task graph with the same CPU checks mk_build_taskgraph
+ * runs (used to show that corrupted graphs are rejected).  Returns MK_OK or
+ * MK_ERR_INVALID_ARG with the reason in mk_last_error(ctx). */
+int mk_validate_taskgraph(mk_ctx* ctx, const int32_t* tasks, int n_tasks, const int32_t* event_counts,
+                          int n_events);
+
+/* Standalone decode attention in the Mirage article's example form (attention code sample:
+ * Q [64,1,128], K [64,128,4096] pre-transposed, V [64,4096,128], fp16, O = softmax(Q K) V):
+ *   q [BH][d], k_t [BH][d][L] (key index fastest), v [BH][L][d]: fp16 device arrays;
+ *   o [BH][d]: fp32 device output; o[h] = sum_j softmax_j(scale * q[h].k_t[h][:,j]) v[h][j].
+ * Accumulation and softmax in fp32, split-KV over all SMs with an online-softmax merge.
+ * d must be 64 or 128; L >= 1; scale = 1.0 reproduces the example (no scaling).
+ * workspace: device scratch of mk_attention_workspace_bytes(BH, d, L) bytes, 256-byte
+ * aligned; its counter words must be zero before the first call (e.g. cudaMemset once);
+ * every call leaves them zero again.  Calls sharing a workspace must not overlap. */
+size_t mk_attention_workspace_bytes(int BH, int d, int L);
+int mk_attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d, int L,
+                        float scale, void* workspace, void* stream);
+/* Synchronise `stream` and report whether an mk_attention_decode call with these sizes
+ * and this workspace had a device wait run out (MK_ERR_DEVICE_TIMEOUT; the workspace is
+ * then re-zeroed) or finished normally (MK_OK). */
+int mk_attention_status(void* workspace, int BH, int d, int L, void* stream);
+
+/* Last error text for ctx (or the thread's last context-free error when ctx is NULL). */
+const char* mk_last_error(const mk_ctx* ctx);
+void mk_destroy(mk_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MK_H */

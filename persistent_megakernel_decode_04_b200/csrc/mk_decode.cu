@@ -1,0 +1,751 @@
+// mk_decode.cu -- the persistent decode megakernel (one launch per decode step).
+//
+// Runtime of the MPK summary "Compiler des LLM en MegaKernel ..." Part 2 "Runtime":
+// one CTA per SM runs the tasks of its queue in order ("Workers": fetch, execute, notify,
+// repeat); a scheduler role watches the event counters ("Schedulers", "Execution pilotee
+// par evenements": a finished task increments an event counter; once the counter reaches
+// its threshold the dependent tasks may run).  Roles inside each CTA:
+//   warps 0-7  worker:    GEMV / attention / epilogues of the current task
+//   warp 8     producer:  streams the queue's weight tiles into a 6-stage shared-memory ring
+//                         with 1-D TMA bulk copies; weights never depend on activations, so
+//                         it runs ahead across dependency waits (the cross-layer overlap of
+//                         the same summary's "Valeur cle" / Part 2)
+//   warp 9     scheduler: acquires the events the next tasks wait on and releases them to the
+//                         workers through a shared-memory counter
+// Every wait is bounded by a global-timer limit; a wait that runs out records an error word,
+// raises a global abort flag that every CTA polls, and all roles return (the producer first
+// waits, bounded, for its copies in flight).
+//
+// GEMV tiles: a task is up to 32 rows x full K.  Each of the 256 worker threads owns 8 K
+// elements of every 2048-element segment, so x (times the norm gain) sits in registers for
+// the whole task and each weight byte is read from shared memory once; partial sums are
+// reduced across lanes with a transposed butterfly of shuffles (lane r ends with row r) and
+// across warps through shared memory.  RMSNorm is fused by the "Normalization + Linear"
+// identity of the Mirage article (Case 1): dot(W, x*g) * rsqrt(mean(x^2) + eps).
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "mk_internal.h"
+#include "mk_ptx.cuh"
+
+namespace mk {
+
+struct DSmem {
+  uint8_t ring[kStages][kSlotBytes];
+  float red[kWorkerWarps][32];
+  float tot[kRMax];
+  float ssw[kWorkerWarps];
+  float am[kWorkerWarps][4];
+  float al[kWorkerWarps][4];
+  float aacc[kWorkerWarps][4][128];
+  float lmv[kWorkerWarps];
+  int lmi[kWorkerWarps];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint32_t ready;            // tasks [0, ready) of this queue have their inputs
+  uint32_t cabort;           // worker-role abort: written before, read after a worker barrier
+  volatile uint32_t abort;   // any role gave up: stop waiting
+  uint32_t flag;             // worker broadcast (last-arriver decisions)
+};
+
+size_t decode_smem_bytes() { return sizeof(DSmem) + 1024; }
+
+__device__ __forceinline__ void worker_bar() { named_bar_sync(1, kWorkerThreads); }
+
+__device__ __forceinline__ void raise_error(const DecodeParams& P, DSmem& S, uint32_t code, uint32_t where,
+                                            uint32_t task) {
+  S.abort = 1u;
+  if (atomicCAS(&P.err[ERR_CODE], 0u, code) == 0u) {
+    P.err[ERR_WHERE] = where;
+    P.err[ERR_TASK] = task;
+  }
+  atomicExch(&P.err[ERR_ABORT], 1u);
+}
+
+// Bounded mbarrier wait (see header comment).  False once the limit passed or a role aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_t limit_ns, DSmem* S) {
+  uint64_t t0 = 0;
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_test(bar, parity)) return true;
+    if ((n & 127u) == 0) {
+      if (S && S->abort) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > limit_ns) return false;
+    }
+  }
+}
+
+struct Pipe {
+  int stage;
+  uint32_t phase;
+  __device__ __forceinline__ void advance() {
+    if (++stage == kStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+__device__ __forceinline__ float dot8(const uint4 w, const float* x, float acc) {
+  acc = fmaf(bf16lo(w.x), x[0], acc);
+  acc = fmaf(bf16hi(w.x), x[1], acc);
+  acc = fmaf(bf16lo(w.y), x[2], acc);
+  acc = fmaf(bf16hi(w.y), x[3], acc);
+  acc = fmaf(bf16lo(w.z), x[4], acc);
+  acc = fmaf(bf16hi(w.z), x[5], acc);
+  acc = fmaf(bf16lo(w.w), x[6], acc);
+  acc = fmaf(bf16hi(w.w), x[7], acc);
+  return acc;
+}
+
+__device__ __forceinline__ uint16_t f2bf(float f) {
+  // round to nearest even
+  uint32_t u = __float_as_uint(f);
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return (uint16_t)(u >> 16);
+}
+
+// Which stream a GEMV task reads: arena offset and row length (bytes) for the task's op.
+__device__ __forceinline__ void gemv_source(const DecodeParams& P, const Task& t, uint64_t* off, uint32_t* row_bytes) {
+  const LayerOff& lo = P.loff[t.layer < P.L ? t.layer : 0];
+  switch (t.kind) {
+    case TK_QKV: *off = lo.qkv; *row_bytes = (uint32_t)P.H * 2u; break;
+    case TK_OPROJ: *off = lo.o; *row_bytes = (uint32_t)P.H * 2u; break;
+    case TK_GATEUP: *off = lo.gu; *row_bytes = (uint32_t)P.H * 2u; break;
+    case TK_DOWN: *off = lo.d; *row_bytes = (uint32_t)P.F * 2u; break;
+    default: *off = P.off_lm; *row_bytes = (uint32_t)P.H * 2u; break;
+  }
+}
+
+__device__ __forceinline__ bool is_gemv(uint8_t k) {
+  return k == TK_QKV || k == TK_OPROJ || k == TK_GATEUP || k == TK_DOWN || k == TK_LMHEAD;
+}
+
+// ---------------------------------------------------------------------------------------
+// GEMV core: acc[r] = sum_k W[row0 + r][k] * x[k] * g[k] for r < nrows, rows streamed through
+// the ring RPS rows per stage.  Writes the per-row totals to S.tot and returns (via S.ssw) the
+// sum of squares of x for the fused norm.  Returns false if a wait ran out (uniform).
+template <int NSEG, int RPS>
+__device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe& pp, const float* __restrict__ xsrc,
+                                          const uint16_t* __restrict__ gain, int K, int nrows, uint32_t row_bytes,
+                                          uint32_t task_id, uint32_t& stall_ns) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  float x[NSEG][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int s = 0; s < NSEG; ++s) {
+    const int k = s * kSegElems + tid * 8;
+    if (k < K) {
+      const float4 a = __ldcg(reinterpret_cast<const float4*>(xsrc + k));
+      const float4 b = __ldcg(reinterpret_cast<const float4*>(xsrc + k + 4));
+      x[s][0] = a.x; x[s][1] = a.y; x[s][2] = a.z; x[s][3] = a.w;
+      x[s][4] = b.x; x[s][5] = b.y; x[s][6] = b.z; x[s][7] = b.w;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss = fmaf(x[s][i], x[s][i], ss);
+      if (gain) {
+        const uint4 g = __ldg(reinterpret_cast<const uint4*>(gain + k));
+        x[s][0] *= bf16lo(g.x); x[s][1] *= bf16hi(g.x);
+        x[s][2] *= bf16lo(g.y); x[s][3] *= bf16hi(g.y);
+        x[s][4] *= bf16lo(g.z); x[s][5] *= bf16hi(g.z);
+        x[s][6] *= bf16lo(g.w); x[s][7] *= bf16hi(g.w);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[s][i] = 0.f;
+    }
+  }
+  float acc[kRMax];
+#pragma unroll
+  for (int r = 0; r < kRMax; ++r) acc[r] = 0.f;
+  bool ok = true;
+#pragma unroll
+  for (int r = 0; r < kRMax; ++r) {
+    if (r < nrows) {
+      if (r % RPS == 0) {
+        const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
+        if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
+          if (ok) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
+          ok = false;
+          S.cabort = 1u;
+        }
+        if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
+      }
+      const uint8_t* row = S.ring[pp.stage] + (r % RPS) * row_bytes;
+#pragma unroll
+      for (int s = 0; s < NSEG; ++s) {
+        if (s * kSegElems + tid * 8 < K) {
+          const uint4 w = *reinterpret_cast<const uint4*>(row + s * kSegBytes + tid * 16);
+          acc[r] = dot8(w, x[s], acc[r]);
+        }
+      }
+      if (r % RPS == RPS - 1 || r == nrows - 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
+        pp.advance();
+      }
+    }
+  }
+  // transposed butterfly: afterwards lane l holds the warp's sum for row l
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? acc[i] : acc[i + off];
+      const float keep = upper ? acc[i + off] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  S.red[warp][lane] = acc[0];
+  if (lane == 0) S.ssw[warp] = ss;
+  worker_bar();
+  if (S.cabort) return false;
+  if (tid < nrows) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWorkerWarps; ++w) t += S.red[w][tid];
+    S.tot[tid] = t;
+  }
+  worker_bar();
+  return true;
+}
+
+__device__ __forceinline__ float norm_factor(const DSmem& S, int K, float eps) {
+  float ss = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWorkerWarps; ++w) ss += S.ssw[w];
+  return 1.0f / sqrtf(ss / (float)K + eps);
+}
+
+// ---------------------------------------------------------------------------------------
+// Epilogues (thread t < nrows handles row row0 + t).
+__device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, const Task& t, float r) {
+  const int tid = threadIdx.x;
+  if (tid >= (int)t.nrows) return;
+  const int D = P.D, G = P.nq / P.nkv, half = D / 2;
+  const int rpg = (G + 2) * D;
+  const int R = (int)t.row0 + tid;
+  const int grp = R / rpg, rr = R % rpg;
+  const float v = S.tot[tid] * r;
+  const int b = 0;
+  const int pos = P.pos[b];
+  const size_t head_stride = (size_t)P.max_seq * D;
+  const size_t kv_layer = (size_t)P.max_batch * P.nkv * head_stride;  // one of K or V, one layer
+  if (rr < (G + 1) * D) {
+    // q or k: rows come in RoPE pairs (i, i + D/2) at packed positions (2i, 2i+1)
+    const int pd = (rr < G * D) ? (rr % D) : (rr - G * D);
+    const int i = pd >> 1, hi = pd & 1;
+    const float other = S.tot[tid ^ 1] * r;
+    const float2 cs = P.rope[(size_t)pos * half + i];
+    float outv;
+    int dim;
+    if (hi == 0) {
+      outv = v * cs.x - other * cs.y;
+      dim = i;
+    } else {
+      outv = v * cs.x + other * cs.y;
+      dim = i + half;
+    }
+    if (rr < G * D) {
+      const int hq = grp * G + rr / D;
+      P.qbuf[((size_t)t.layer * P.B + b) * P.nq * D + (size_t)hq * D + dim] = outv;
+    } else {
+      uint16_t* kc = P.kv + ((size_t)t.layer * 2 + 0) * kv_layer + ((size_t)b * P.nkv + grp) * head_stride;
+      kc[(size_t)pos * D + dim] = f2bf(outv);
+    }
+  } else {
+    const int dim = rr - (G + 1) * D;
+    uint16_t* vc = P.kv + ((size_t)t.layer * 2 + 1) * kv_layer + ((size_t)b * P.nkv + grp) * head_stride;
+    vc[(size_t)pos * D + dim] = f2bf(v);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Split-KV attention chunk for one (sequence, KV head): scores of its G query heads over the
+// chunk's keys, per-warp online softmax, merged across warps into one partial (m, l, acc).
+// The last chunk to arrive merges all partials of the (sequence, KV head) into o.
+template <int D>
+__device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, const Task& t, uint32_t task_id) {
+  constexpr int DL = D / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = P.nq / P.nkv;
+  const int b = (int)t.row0 / P.nkv, g = (int)t.row0 % P.nkv;
+  const int c = t.aux;
+  const int Lk = P.pos[b] + 1;
+  const int cl = (Lk + P.nch - 1) / P.nch;
+  const int j0 = c * cl, j1 = min(Lk, j0 + cl);
+  const size_t head_stride = (size_t)P.max_seq * D;
+  const size_t kv_layer = (size_t)P.max_batch * P.nkv * head_stride;
+  const uint16_t* kc = P.kv + ((size_t)t.layer * 2 + 0) * kv_layer + ((size_t)b * P.nkv + g) * head_stride;
+  const uint16_t* vc = P.kv + ((size_t)t.layer * 2 + 1) * kv_layer + ((size_t)b * P.nkv + g) * head_stride;
+  const float* qsrc = P.qbuf + ((size_t)t.layer * P.B + b) * P.nq * D + (size_t)g * G * D;
+
+  float qv[4][DL], m[4], l[4], acc[4][DL];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    m[h] = -INFINITY;
+    l[h] = 0.f;
+#pragma unroll
+    for (int i = 0; i < DL; ++i) {
+      qv[h][i] = (h < G) ? __ldcg(qsrc + h * D + lane * DL + i) * P.attn_scale : 0.f;
+      acc[h][i] = 0.f;
+    }
+  }
+  for (int j = j0 + warp; j < j1; j += kWorkerWarps) {
+    float kf[DL], vf[DL];
+    if (DL == 4) {
+      const uint2 kw = __ldcg(reinterpret_cast<const uint2*>(kc + (size_t)j * D + lane * 4));
+      const uint2 vw = __ldcg(reinterpret_cast<const uint2*>(vc + (size_t)j * D + lane * 4));
+      kf[0] = bf16lo(kw.x); kf[1] = bf16hi(kw.x); kf[2 % DL] = bf16lo(kw.y); kf[3 % DL] = bf16hi(kw.y);
+      vf[0] = bf16lo(vw.x); vf[1] = bf16hi(vw.x); vf[2 % DL] = bf16lo(vw.y); vf[3 % DL] = bf16hi(vw.y);
+    } else {
+      const uint32_t kw = __ldcg(reinterpret_cast<const unsigned int*>(kc + (size_t)j * D + lane * 2));
+      const uint32_t vw = __ldcg(reinterpret_cast<const unsigned int*>(vc + (size_t)j * D + lane * 2));
+      kf[0] = bf16lo(kw); kf[1 % DL] = bf16hi(kw);
+      vf[0] = bf16lo(vw); vf[1 % DL] = bf16hi(vw);
+    }
+    float s[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float a = 0.f;
+#pragma unroll
+      for (int i = 0; i < DL; ++i) a = fmaf(qv[h][i], kf[i], a);
+      s[h] = a;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+      for (int h = 0; h < 4; ++h) s[h] += __shfl_xor_sync(0xffffffffu, s[h], off);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      if (h < G) {
+        const float mn = fmaxf(m[h], s[h]);
+        const float a = expf(m[h] - mn);
+        const float p = expf(s[h] - mn);
+        l[h] = l[h] * a + p;
+#pragma unroll
+        for (int i = 0; i < DL; ++i) acc[h][i] = fmaf(acc[h][i], a, p * vf[i]);
+        m[h] = mn;
+      }
+    }
+  }
+  // cross-warp merge of the chunk
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    if (h < G) {
+      if (lane == 0) {
+        S.am[warp][h] = m[h];
+        S.al[warp][h] = l[h];
+      }
+#pragma unroll
+      for (int i = 0; i < DL; ++i) S.aacc[warp][h][lane * DL + i] = acc[h][i];
+    }
+  }
+  worker_bar();
+  const int nq = P.nq;
+  float* part_base = P.part + (((size_t)t.layer * P.B + b) * nq) * (size_t)P.nch * (D + 2);
+  for (int e = tid; e < G * D; e += kWorkerThreads) {
+    const int h = e / D, d = e % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWorkerWarps; ++w) M = fmaxf(M, S.am[w][h]);
+    float ls = 0.f, as = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWorkerWarps; ++w) {
+        const float f = expf(S.am[w][h] - M);
+        ls += f * S.al[w][h];
+        as += f * S.aacc[w][h][d];
+      }
+    }
+    float* pp = part_base + ((size_t)(g * G + h) * P.nch + c) * (D + 2);
+    pp[2 + d] = as;
+    if (d == 0) {
+      pp[0] = M;
+      pp[1] = ls;
+    }
+  }
+  worker_bar();
+  if (tid == 0) {
+    __threadfence();
+    uint32_t* cnt = P.acnt + ((size_t)t.layer * P.B + b) * P.nkv + g;
+    const uint32_t old = atom_acq_rel_gpu_add(cnt, 1u);
+    S.flag = (old + 1u == P.epoch * (uint32_t)P.nch) ? 1u : 0u;
+  }
+  worker_bar();
+  if (S.flag) {
+    __threadfence();
+    float* o = P.obuf + ((size_t)t.layer * P.B + b) * nq * D + (size_t)g * G * D;
+    for (int e = tid; e < G * D; e += kWorkerThreads) {
+      const int h = e / D, d = e % D;
+      const float* ph = part_base + (size_t)(g * G + h) * P.nch * (D + 2);
+      float M = -INFINITY;
+      for (int cc = 0; cc < P.nch; ++cc) M = fmaxf(M, __ldcg(ph + (size_t)cc * (D + 2)));
+      float num = 0.f, den = 0.f;
+      for (int cc = 0; cc < P.nch; ++cc) {
+        const float* pc = ph + (size_t)cc * (D + 2);
+        const float mc = __ldcg(pc);
+        if (mc == -INFINITY) continue;
+        const float f = expf(mc - M);
+        den += f * __ldcg(pc + 1);
+        num += f * __ldcg(pc + 2 + d);
+      }
+      o[(size_t)h * D + d] = num / den;
+    }
+    worker_bar();
+    if (tid == 0 && (int)t.notify[0] != P.drop_event) {
+      __threadfence();
+      red_release_gpu_add(&P.ev[t.notify[0]], 1u);
+    }
+  }
+  (void)task_id;
+  return true;
+}
+
+// LM-head epilogue: logits and this task's (max, index) partial; the last LM task picks the token.
+__device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, const Task& t, float r) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int b = 0;
+  if (tid < 32) {
+    float v = -INFINITY;
+    int idx = 0x7fffffff;
+    if (tid < (int)t.nrows) {
+      v = S.tot[tid] * r;
+      idx = (int)t.row0 + tid;
+      P.logits[(size_t)b * P.V + idx] = v;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, v, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
+      if (ov > v || (ov == v && oi < idx)) {
+        v = ov;
+        idx = oi;
+      }
+    }
+    if (lane == 0) {
+      P.lm_val[(size_t)t.index * P.B + b] = v;
+      P.lm_idx[(size_t)t.index * P.B + b] = idx;
+    }
+  }
+  worker_bar();
+  if (tid == 0) {
+    __threadfence();
+    const uint32_t old = atom_acq_rel_gpu_add(&P.ev[P.ev_lm], 1u);
+    S.flag = (old + 1u == P.epoch * (uint32_t)P.n_lm) ? 1u : 0u;
+  }
+  worker_bar();
+  if (S.flag && P.next_tokens) {
+    __threadfence();
+    float v = -INFINITY;
+    int idx = 0x7fffffff;
+    for (int i = tid; i < P.n_lm; i += kWorkerThreads) {
+      const float ov = __ldcg(P.lm_val + (size_t)i * P.B + b);
+      const int oi = __ldcg(P.lm_idx + (size_t)i * P.B + b);
+      if (ov > v || (ov == v && oi < idx)) {
+        v = ov;
+        idx = oi;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, v, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
+      if (ov > v || (ov == v && oi < idx)) {
+        v = ov;
+        idx = oi;
+      }
+    }
+    if (lane == 0) {
+      S.lmv[tid >> 5] = v;
+      S.lmi[tid >> 5] = idx;
+    }
+    worker_bar();
+    if (tid == 0) {
+      for (int w = 1; w < kWorkerWarps; ++w)
+        if (S.lmv[w] > v || (S.lmv[w] == v && S.lmi[w] < idx)) {
+          v = S.lmv[w];
+          idx = S.lmi[w];
+        }
+      P.next_tokens[b] = idx;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F>
+__global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  DSmem& S = *reinterpret_cast<DSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t qb = P.qbegin[blockIdx.x], qe = P.qbegin[blockIdx.x + 1];
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], kWorkerWarps);
+    }
+    S.ready = 0;
+    S.cabort = 0;
+    S.abort = 0;
+    S.flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kProducerWarp) {
+    // ------------------------------- producer -------------------------------
+    if (lane != 0) return;
+    const uint64_t pol = policy_evict_first();
+    Pipe pp{0, 0};
+    int issued = 0;
+    bool ok = true;
+    for (uint32_t i = qb; i < qe && ok; ++i) {
+      const Task t = P.tasks[i];
+      if (!is_gemv(t.kind)) continue;
+      uint64_t off;
+      uint32_t rb;
+      gemv_source(P, t, &off, &rb);
+      const int rps = (t.kind == TK_DOWN) ? RPS_F : RPS_H;
+      const uint8_t* src = P.arena + off + (uint64_t)t.row0 * rb;
+      uint64_t blocked = 0, first = 0;
+      for (uint32_t r0 = 0; r0 < t.nrows; r0 += (uint32_t)rps) {
+        const uint32_t nr = min((uint32_t)rps, t.nrows - r0);
+        const uint64_t tw = P.trace ? globaltimer_ns() : 0;
+        if (!wait_bar(&S.empty[pp.stage], pp.phase ^ 1u, P.timeout_ns, &S)) {
+          if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, i);
+          ok = false;
+          break;
+        }
+        if (P.trace) {
+          const uint64_t now = globaltimer_ns();
+          blocked += now - tw;
+          if (r0 == 0) first = now;
+        }
+        mbar_arrive_expect_tx(&S.full[pp.stage], nr * rb);
+        bulk_g2s(S.ring[pp.stage], src + (uint64_t)r0 * rb, nr * rb, &S.full[pp.stage], pol);
+        ++issued;
+        pp.advance();
+      }
+      if (P.trace) {
+        P.trace[(size_t)i * kTraceWords + 4] = blocked;
+        P.trace[(size_t)i * kTraceWords + 5] = first;
+      }
+    }
+    // leave no copy in flight: wait (bounded) for the last issued stages to land
+    for (int k = 1; k <= (issued < kStages ? issued : kStages); ++k) {
+      int s = pp.stage - k;
+      uint32_t ph = pp.phase;
+      if (s < 0) {
+        s += kStages;
+        ph ^= 1u;
+      }
+      wait_bar(&S.full[s], ph, P.timeout_ns, nullptr);
+    }
+    return;
+  }
+
+  if (warp == kSchedWarp) {
+    // ------------------------------- scheduler ------------------------------
+    if (lane != 0) return;
+    for (uint32_t i = qb; i < qe; ++i) {
+      const Task t = P.tasks[i];
+      for (int w = 0; w < t.n_wait; ++w) {
+        const uint32_t e = t.wait[w];
+        const uint32_t target = P.epoch * P.ev_count[e];
+        uint64_t t0 = 0;
+        for (uint32_t n = 1;; ++n) {
+          if ((int32_t)(ld_acquire_gpu(&P.ev[e]) - target) >= 0) break;
+          if ((n & 63u) == 0) {
+            if (S.abort || *(volatile uint32_t*)&P.err[ERR_ABORT]) {
+              S.abort = 1u;
+              return;
+            }
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > P.timeout_ns) {
+              raise_error(P, S, DEV_ERR_WAIT_EVENT, e, i);
+              return;
+            }
+          }
+        }
+      }
+      st_release_cta_shared(&S.ready, i - qb + 1u);
+    }
+    return;
+  }
+
+  // --------------------------------- workers ---------------------------------
+  Pipe pp{0, 0};
+  for (uint32_t i = qb; i < qe; ++i) {
+    const uint64_t t_wait = (P.trace && tid == 0) ? globaltimer_ns() : 0;
+    uint32_t stall = 0;
+    // wait for the scheduler to release task i (bounded, abort-aware, then uniform decision)
+    {
+      uint64_t t0 = 0;
+      for (uint32_t n = 1;; ++n) {
+        if (ld_acquire_cta_shared(&S.ready) > i - qb) break;
+        if ((n & 63u) == 0) {
+          if (S.abort) {
+            S.cabort = 1u;
+            break;
+          }
+          const uint64_t now = globaltimer_ns();
+          if (t0 == 0) t0 = now;
+          else if (now - t0 > P.timeout_ns + 1000000000ull) {  // the scheduler reports first
+            raise_error(P, S, DEV_ERR_WAIT_READY, blockIdx.x, i);
+            S.cabort = 1u;
+            break;
+          }
+        }
+      }
+      worker_bar();
+      if (S.cabort) break;
+    }
+    const uint64_t t_ready = (P.trace && tid == 0) ? globaltimer_ns() : 0;
+    const Task t = P.tasks[i];
+    bool notify = true;
+    switch (t.kind) {
+      case TK_EMBED: {
+        const int b = 0;
+        int tok = __ldcg(P.tokens + b);
+        if (tok < 0 || tok >= P.V) {  // never read outside the table: record and use row 0
+          if (tid == 0 && t.row0 == 0) atomicCAS(&P.err[ERR_CODE], 0u, (uint32_t)DEV_ERR_BAD_TOKEN);
+          tok = 0;
+        }
+        const uint16_t* e = reinterpret_cast<const uint16_t*>(P.arena + P.off_embed) + (size_t)tok * P.H;
+        for (uint32_t r = tid; r < t.nrows; r += kWorkerThreads)
+          P.x_in[(size_t)b * P.H + t.row0 + r] = __uint_as_float((uint32_t)e[t.row0 + r] << 16);
+        break;
+      }
+      case TK_QKV: {
+        const LayerOff& lo = P.loff[t.layer];
+        const float* xs = P.x_in + (size_t)t.layer * P.B * P.H;
+        if (!gemv_tile<NSEG_H, RPS_H>(P, S, pp, xs, reinterpret_cast<const uint16_t*>(P.arena + lo.attn_norm), P.H,
+                                      (int)t.nrows, (uint32_t)P.H * 2u, i, stall))
+          goto out;
+        epi_qkv(P, S, t, norm_factor(S, P.H, P.eps));
+        break;
+      }
+      case TK_ATTN: {
+        notify = false;  // the merging chunk notifies
+        if (P.D == 128) attention_task<128>(P, S, t, i);
+        else attention_task<64>(P, S, t, i);
+        break;
+      }
+      case TK_OPROJ: {
+        const float* os = P.obuf + (size_t)t.layer * P.B * P.nq * P.D;
+        if (!gemv_tile<NSEG_H, RPS_H>(P, S, pp, os, nullptr, P.H, (int)t.nrows, (uint32_t)P.H * 2u, i, stall)) goto out;
+        if (tid < (int)t.nrows) {
+          const size_t r = (size_t)t.row0 + tid;
+          const float* xi = P.x_in + (size_t)t.layer * P.B * P.H;
+          P.x_mid[(size_t)t.layer * P.B * P.H + r] = __ldcg(xi + r) + S.tot[tid];
+        }
+        break;
+      }
+      case TK_GATEUP: {
+        const LayerOff& lo = P.loff[t.layer];
+        const float* xs = P.x_mid + (size_t)t.layer * P.B * P.H;
+        if (!gemv_tile<NSEG_H, RPS_H>(P, S, pp, xs, reinterpret_cast<const uint16_t*>(P.arena + lo.mlp_norm), P.H,
+                                      (int)t.nrows, (uint32_t)P.H * 2u, i, stall))
+          goto out;
+        const float r = norm_factor(S, P.H, P.eps);
+        if (tid < (int)t.nrows && (tid & 1) == 0) {
+          const float gv = S.tot[tid] * r, uv = S.tot[tid + 1] * r;
+          const float sg = gv / (1.f + expf(-gv));
+          P.hbuf[(size_t)t.layer * P.B * P.F + (t.row0 + tid) / 2] = sg * uv;
+        }
+        break;
+      }
+      case TK_DOWN: {
+        const float* hs = P.hbuf + (size_t)t.layer * P.B * P.F;
+        if (!gemv_tile<NSEG_F, RPS_F>(P, S, pp, hs, nullptr, P.F, (int)t.nrows, (uint32_t)P.F * 2u, i, stall)) goto out;
+        if (tid < (int)t.nrows) {
+          const size_t r = (size_t)t.row0 + tid;
+          const float* xm = P.x_mid + (size_t)t.layer * P.B * P.H;
+          P.x_in[(size_t)(t.layer + 1) * P.B * P.H + r] = __ldcg(xm + r) + S.tot[tid];
+        }
+        break;
+      }
+      case TK_LMHEAD: {
+        notify = false;
+        const float* xs = P.x_in + (size_t)P.L * P.B * P.H;
+        if (!gemv_tile<NSEG_H, RPS_H>(P, S, pp, xs, reinterpret_cast<const uint16_t*>(P.arena + P.off_fnorm), P.H,
+                                      (int)t.nrows, (uint32_t)P.H * 2u, i, stall))
+          goto out;
+        epi_lmhead(P, S, t, norm_factor(S, P.H, P.eps));
+        break;
+      }
+      default:
+        break;
+    }
+    if (P.trace && tid == 0) {
+      uint64_t* rec = P.trace + (size_t)i * kTraceWords;
+      rec[0] = t_wait;
+      rec[1] = t_ready;
+      rec[2] = globaltimer_ns();
+      rec[3] = (uint64_t)stall | ((uint64_t)blockIdx.x << 32);
+    }
+    if (notify) {
+      worker_bar();
+      if (tid == 0) {
+        __threadfence();
+        for (int k = 0; k < t.n_notify; ++k)
+          if ((int)t.notify[k] != P.drop_event) red_release_gpu_add(&P.ev[t.notify[k]], 1u);
+      }
+    }
+  }
+out:
+  return;
+}
+
+// ---------------------------------------------------------------------------------------
+// Instantiations: (segments, rows per stage) for K = hidden and K = ffn.
+static const Variant kVariants[] = {
+    {2, 4, 7, 1, 1},   // Llama-3-8B shape: hidden 4096, ffn 14336
+    {2, 4, 6, 1, 1},   // Chameleon-7B shape: hidden 4096, ffn 11008
+    {1, 32, 1, 16, 1}, // tiny: hidden 256, ffn 768
+    {1, 32, 1, 32, 1}, // small test shapes: hidden <= 256, ffn <= 512
+    {2, 4, 2, 4, 1},   // hidden 4096, ffn <= 4096
+    {1, 32, 2, 4, 1},  // hidden <= 256... ffn in (2048, 4096]
+};
+
+typedef void (*DecodeFn)(DecodeParams);
+
+static const void* kFns[] = {
+    (const void*)decode_kernel<2, 4, 7, 1>,  (const void*)decode_kernel<2, 4, 6, 1>,
+    (const void*)decode_kernel<1, 32, 1, 16>, (const void*)decode_kernel<1, 32, 1, 32>,
+    (const void*)decode_kernel<2, 4, 2, 4>,  (const void*)decode_kernel<1, 32, 2, 4>,
+};
+
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int batch) {
+  for (int i = 0; i < (int)(sizeof(kVariants) / sizeof(kVariants[0])); ++i) {
+    const Variant& v = kVariants[i];
+    if (v.nseg_h == nseg_h && v.rps_h == rps_h && v.nseg_f == nseg_f && v.rps_f == rps_f && v.batch == batch)
+      return i;
+  }
+  return -1;
+}
+
+const void* decode_kernel_ptr(int variant) { return kFns[variant]; }
+
+int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t stream, std::string* err) {
+  const void* fn = kFns[variant];
+  const size_t smem = decode_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) {
+    void* args[] = {const_cast<DecodeParams*>(&p)};
+    e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kBlockThreads), args, smem, stream);
+  }
+  if (e != cudaSuccess) {
+    *err = std::string("decode launch: ") + cudaGetErrorString(e);
+    return e == cudaErrorCooperativeLaunchTooLarge ? MK_ERR_NOT_RESIDENT : MK_ERR_CUDA;
+  }
+  return MK_OK;
+}
+
+}  // namespace mk

@@ -1,0 +1,1039 @@
+// mk_host.cpp -- host side of the C ABI: config checks, task-graph lowering and validation,
+// weight packing, arena layout, launches.
+//
+// Lowering follows Part 1 "Compilateur" of the MPK summary ("Compiler des LLM en MegaKernel
+// ..."): every op of the decode step becomes per-SM tile tasks, edges follow the actual data
+// each tile reads (attention of KV head g waits only for the QKV tiles of head group g), and
+// events carry thresholds equal to their producer counts.  Queues are static and in one
+// global topological order (the precomputed schedule of "Ada-MK ...", section 2, "offline
+// DAG search -> fixed schedule"), which is what lets the producer warp prefetch the next
+// task's weights before its inputs exist.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "mk_internal.h"
+
+using namespace mk;
+
+namespace {
+
+thread_local std::string g_err;
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct TaskRec {  // host-side task with its SM
+  Task t;
+  int sm;
+};
+
+struct Graph {
+  std::vector<TaskRec> tasks;  // in queue order, grouped by SM (SM 0 first)
+  std::vector<uint32_t> ev_count;
+  int n_sms = 0;
+};
+
+}  // namespace
+
+struct mk_ctx {
+  mk_config cfg;
+  int device = -1;
+  int n_sms = 148;
+  int variant = -1;
+  int G = 1, rows_qkv = 0, rows_gu = 0, nch = 1, n_lm = 0;
+  int nseg_h = 0, rps_h = 0, nseg_f = 0, rps_f = 0;
+  // events
+  int n_events = 0, ev_lm = 0;
+  Graph g;
+  std::vector<uint32_t> qbegin;
+  // arena layout
+  std::vector<LayerOff> loff;
+  uint64_t off_embed = 0, off_lm = 0, off_fnorm = 0, arena_bytes = 0;
+  // workspace layout
+  size_t ws_tasks = 0, ws_qbegin = 0, ws_evcount = 0, ws_ev = 0, ws_acnt = 0, ws_err = 0, ws_loff = 0, ws_rope = 0,
+         ws_xin = 0, ws_xmid = 0, ws_q = 0, ws_o = 0, ws_h = 0, ws_part = 0, ws_lmval = 0, ws_lmidx = 0,
+         ws_pf = 0, ws_bytes = 0;
+  size_t ev_bytes = 0, acnt_bytes = 0;
+  int pf_rows = 0;
+  size_t kv_bytes = 0;
+  uint64_t weight_bytes_per_step = 0;
+  // runtime
+  uint8_t* arena = nullptr;
+  uint8_t* ws = nullptr;
+  bool loaded = false;
+  int B = 0;
+  std::vector<int> pos;
+  uint32_t epoch = 0;
+  uint64_t timeout_ns = 2000000000ull;
+  int drop_event = -1;
+  uint64_t* trace = nullptr;
+  std::string err;
+};
+
+namespace {
+
+int fail(mk_ctx* c, int code, const std::string& msg) {
+  if (c) c->err = msg;
+  g_err = msg;
+  return code;
+}
+
+int pow2_floor(int x) {
+  int p = 1;
+  while (p * 2 <= x) p *= 2;
+  return p;
+}
+
+// ---------------------------------------------------------------------------------------
+// Event ids
+int ev_embed() { return 0; }
+int ev_base(const mk_ctx* c, int l) { return 1 + l * (c->cfg.n_kv_heads + 4); }
+int ev_qkv(const mk_ctx* c, int l, int g) { return ev_base(c, l) + g; }
+int ev_attn(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads; }
+int ev_o(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads + 1; }
+int ev_gu(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads + 2; }
+int ev_down(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads + 3; }
+
+// Split `total` rows over n_sms SMs in contiguous, balanced ranges (multiples of gran), and
+// each range into tasks of at most kRMax rows.
+std::vector<std::vector<std::pair<int, int>>> partition_rows(int total, int gran, int n_sms) {
+  std::vector<std::vector<std::pair<int, int>>> out(n_sms);
+  for (int s = 0; s < n_sms; ++s) {
+    int a = (int)(((long long)total * s / n_sms) / gran * gran);
+    int b = (s + 1 == n_sms) ? total : (int)(((long long)total * (s + 1) / n_sms) / gran * gran);
+    int n = b - a;
+    if (n <= 0) continue;
+    int nt = (n + kRMax - 1) / kRMax;
+    for (;;) {
+      bool ok = true;
+      std::vector<std::pair<int, int>> parts;
+      for (int i = 0; i < nt; ++i) {
+        int lo = (int)(((long long)n * i / nt) / gran * gran);
+        int hi = (i + 1 == nt) ? n : (int)(((long long)n * (i + 1) / nt) / gran * gran);
+        if (hi - lo > kRMax) ok = false;
+        if (hi > lo) parts.push_back({a + lo, hi - lo});
+      }
+      if (ok) {
+        out[s] = parts;
+        break;
+      }
+      ++nt;
+    }
+  }
+  return out;
+}
+
+Task make_task(uint8_t kind, int layer, int row0, int nrows) {
+  Task t;
+  std::memset(&t, 0, sizeof(t));
+  t.kind = kind;
+  t.layer = (uint16_t)layer;
+  t.row0 = (uint32_t)row0;
+  t.nrows = (uint32_t)nrows;
+  return t;
+}
+
+void add_wait(Task& t, int e) { t.wait[t.n_wait++] = (uint32_t)e; }
+void add_notify(Task& t, int e) { t.notify[t.n_notify++] = (uint32_t)e; }
+
+// ---------------------------------------------------------------------------------------
+// Validation of a task graph (used at build time and by mk_validate_taskgraph).
+struct VTask {
+  int kind, layer, sm, row0, nrows, n_wait, wait[2], n_notify, notify[2];
+};
+
+int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>& cnt) {
+  const mk_config& f = c->cfg;
+  const int L = f.n_layers, nkv = f.n_kv_heads, nE = (int)cnt.size();
+  const int rpg = c->rows_qkv / nkv;
+  const int B = f.max_batch;
+  char buf[256];
+  // (a) ids
+  for (size_t i = 0; i < T.size(); ++i) {
+    const VTask& t = T[i];
+    if (t.sm < 0 || t.sm >= c->n_sms || t.n_wait < 0 || t.n_wait > 2 || t.n_notify < 0 || t.n_notify > 2 ||
+        t.layer < 0 || t.layer > L)
+      return fail(c, MK_ERR_INVALID_ARG, "task " + std::to_string(i) + ": field out of range");
+    for (int k = 0; k < t.n_wait; ++k)
+      if (t.wait[k] < 0 || t.wait[k] >= nE) return fail(c, MK_ERR_INVALID_ARG, "task wait event out of range");
+    for (int k = 0; k < t.n_notify; ++k)
+      if (t.notify[k] < 0 || t.notify[k] >= nE)
+        return fail(c, MK_ERR_INVALID_ARG, "task notify event out of range");
+  }
+  // (b) thresholds equal producer counts (an attention group notifies once, from its merge)
+  std::vector<uint32_t> produced(nE, 0);
+  {
+    std::vector<std::vector<char>> seen(nE);
+    for (const VTask& t : T) {
+      if (t.kind == TK_ATTN) {
+        for (int k = 0; k < t.n_notify; ++k) {
+          auto& s = seen[t.notify[k]];
+          size_t key = (size_t)t.layer * B * nkv + t.row0;
+          if (s.size() <= key) s.resize(key + 1, 0);
+          if (!s[key]) {
+            s[key] = 1;
+            produced[t.notify[k]]++;
+          }
+        }
+      } else {
+        for (int k = 0; k < t.n_notify; ++k) produced[t.notify[k]]++;
+      }
+    }
+    for (const VTask& t : T)
+      if (t.kind == TK_LMHEAD) produced[c->ev_lm]++;
+  }
+  for (int e = 0; e < nE; ++e)
+    if (produced[e] != cnt[e]) {
+      snprintf(buf, sizeof buf, "event %d: threshold %u but %u producers per step", e, cnt[e], produced[e]);
+      return fail(c, MK_ERR_INVALID_ARG, buf);
+    }
+  // (c) every op's rows covered exactly once
+  auto rows_of = [&](int kind) -> int {
+    switch (kind) {
+      case TK_EMBED: return f.hidden;
+      case TK_QKV: return c->rows_qkv;
+      case TK_OPROJ: return f.hidden;
+      case TK_GATEUP: return c->rows_gu;
+      case TK_DOWN: return f.hidden;
+      case TK_LMHEAD: return f.vocab;
+    }
+    return 0;
+  };
+  std::vector<std::vector<int>> cover((size_t)8 * (L + 1));
+  std::vector<std::vector<int>> attn_cover((size_t)L * B * nkv);
+  for (const VTask& t : T) {
+    if (t.kind == TK_ATTN) {
+      if (t.row0 < 0 || t.row0 >= B * nkv || t.layer >= L)
+        return fail(c, MK_ERR_INVALID_ARG, "attention task outside the (sequence, KV head) range");
+      auto& v = attn_cover[(size_t)t.layer * B * nkv + t.row0];
+      v.push_back(t.nrows);  // chunk index travels in nrows of the export
+      continue;
+    }
+    if (t.kind < TK_EMBED || t.kind > TK_LMHEAD) return fail(c, MK_ERR_INVALID_ARG, "unknown task kind");
+    int rows = rows_of(t.kind);
+    if (t.nrows <= 0 || t.nrows > kRMax || t.row0 < 0 || t.row0 + t.nrows > rows)
+      return fail(c, MK_ERR_INVALID_ARG, "task rows out of range");
+    if ((t.kind == TK_QKV || t.kind == TK_GATEUP) && ((t.row0 | t.nrows) & 1))
+      return fail(c, MK_ERR_INVALID_ARG, "QKV/gate-up tasks must hold whole row pairs");
+    int lay = (t.kind == TK_EMBED || t.kind == TK_LMHEAD) ? L : t.layer;
+    auto& v = cover[(size_t)t.kind * (L + 1) + lay];
+    if (v.empty()) v.assign(rows, 0);
+    for (int r = t.row0; r < t.row0 + t.nrows; ++r) v[r]++;
+  }
+  for (int kind = TK_EMBED; kind <= TK_LMHEAD; ++kind) {
+    if (kind == TK_ATTN) continue;
+    for (int l = 0; l <= L; ++l) {
+      bool per_layer = !(kind == TK_EMBED || kind == TK_LMHEAD);
+      if (per_layer == (l == L)) continue;
+      auto& v = cover[(size_t)kind * (L + 1) + l];
+      int rows = rows_of(kind);
+      if ((int)v.size() != rows) return fail(c, MK_ERR_INVALID_ARG, "an op has no tasks");
+      for (int r = 0; r < rows; ++r)
+        if (v[r] != 1) {
+          snprintf(buf, sizeof buf, "op kind %d layer %d: row %d covered %d times", kind, l, r, v[r]);
+          return fail(c, MK_ERR_INVALID_ARG, buf);
+        }
+    }
+  }
+  for (int l = 0; l < L; ++l)
+    for (int bg = 0; bg < B * nkv; ++bg) {
+      auto v = attn_cover[(size_t)l * B * nkv + bg];
+      std::sort(v.begin(), v.end());
+      bool ok = (int)v.size() == c->nch;
+      for (int i = 0; ok && i < (int)v.size(); ++i) ok = v[i] == i;
+      if (!ok) return fail(c, MK_ERR_INVALID_ARG, "attention chunks of a (sequence, KV head) incomplete");
+    }
+  // (d) simulate the queues: deadlock-freedom; (e) every read after its writes
+  // categories: 0 embed; per layer: qkv-group g, qkv, attn, o, gu, down; last: lm
+  const int CPL = nkv + 5;
+  auto cat_qkvg = [&](int l, int g) { return 1 + l * CPL + g; };
+  auto cat_of = [&](int kind, int l) {
+    switch (kind) {
+      case TK_QKV: return 1 + l * CPL + nkv;
+      case TK_ATTN: return 1 + l * CPL + nkv + 1;
+      case TK_OPROJ: return 1 + l * CPL + nkv + 2;
+      case TK_GATEUP: return 1 + l * CPL + nkv + 3;
+      case TK_DOWN: return 1 + l * CPL + nkv + 4;
+      case TK_LMHEAD: return 1 + L * CPL;
+    }
+    return 0;
+  };
+  const int NC = 2 + L * CPL;
+  const int W = (NC + 63) / 64;
+  std::vector<int> cat_size(NC, 0);
+  auto cats_of_task = [&](const VTask& t, std::vector<int>& out) {
+    out.clear();
+    out.push_back(cat_of(t.kind, t.layer));
+    if (t.kind == TK_QKV) {
+      for (int g = t.row0 / rpg; g <= (t.row0 + t.nrows - 1) / rpg; ++g) out.push_back(cat_qkvg(t.layer, g));
+    }
+  };
+  std::vector<int> tmp;
+  for (const VTask& t : T) {
+    cats_of_task(t, tmp);
+    for (int x : tmp) cat_size[x]++;
+  }
+  // per-SM queues in array order
+  std::vector<std::vector<int>> q(c->n_sms);
+  for (size_t i = 0; i < T.size(); ++i) q[T[i].sm].push_back((int)i);
+  std::vector<size_t> head(c->n_sms, 0);
+  std::vector<uint32_t> ctr(nE, 0);
+  std::vector<uint64_t> Gb(T.size() * W, 0);   // categories complete before the task starts
+  std::vector<uint64_t> Fe((size_t)nE * W, 0);  // categories complete when the event is active
+  std::vector<std::vector<int>> ev_cat_done(nE, std::vector<int>());
+  std::vector<int> cat_done(NC, 0);
+  std::vector<int> attn_arrive((size_t)L * B * nkv, 0);
+  std::vector<uint64_t> attn_acc((size_t)L * B * nkv * W, 0);
+  auto setbit = [&](uint64_t* bs, int x) { bs[x >> 6] |= 1ull << (x & 63); };
+  auto hasbit = [&](const uint64_t* bs, int x) { return (bs[x >> 6] >> (x & 63)) & 1ull; };
+  std::vector<int> ev_ncat((size_t)nE * NC, 0);  // notifiers of e per category (for "all of C done")
+  size_t executed = 0;
+  std::vector<uint64_t> prevG(W);
+  std::vector<std::vector<uint64_t>> smG(c->n_sms, std::vector<uint64_t>(W, 0));
+  auto fire = [&](int e, const uint64_t* contrib, const std::vector<int>& cats_done) {
+    ctr[e]++;
+    for (int w = 0; w < W; ++w) Fe[(size_t)e * W + w] |= contrib[w];
+    for (int x : cats_done) {
+      int& n = ev_ncat[(size_t)e * NC + x];
+      n++;
+      if (n == cat_size[x]) setbit(&Fe[(size_t)e * W], x);
+    }
+  };
+  bool progress = true;
+  while (progress) {
+    progress = false;
+    for (int s = 0; s < c->n_sms; ++s) {
+      while (head[s] < q[s].size()) {
+        const int i = q[s][head[s]];
+        const VTask& t = T[i];
+        bool ready = true;
+        for (int k = 0; k < t.n_wait; ++k)
+          if (ctr[t.wait[k]] < cnt[t.wait[k]]) ready = false;
+        if (!ready) break;
+        // categories complete before t: its queue predecessor's view plus the waited events'
+        uint64_t* gi = &Gb[(size_t)i * W];
+        for (int w = 0; w < W; ++w) gi[w] = smG[s][w];
+        for (int k = 0; k < t.n_wait; ++k)
+          for (int w = 0; w < W; ++w) gi[w] |= Fe[(size_t)t.wait[k] * W + w];
+        // required inputs
+        std::vector<int> need;
+        const int l = t.layer;
+        switch (t.kind) {
+          case TK_QKV: need.push_back(l == 0 ? 0 : cat_of(TK_DOWN, l - 1)); break;
+          case TK_ATTN: need.push_back(cat_qkvg(l, t.row0 % nkv)); break;
+          case TK_OPROJ:
+            need.push_back(cat_of(TK_ATTN, l));
+            need.push_back(l == 0 ? 0 : cat_of(TK_DOWN, l - 1));
+            break;
+          case TK_GATEUP: need.push_back(cat_of(TK_OPROJ, l)); break;
+          case TK_DOWN:
+            need.push_back(cat_of(TK_GATEUP, l));
+            need.push_back(cat_of(TK_OPROJ, l));
+            break;
+          case TK_LMHEAD: need.push_back(cat_of(TK_DOWN, L - 1)); break;
+        }
+        for (int x : need)
+          if (!hasbit(gi, x)) {
+            snprintf(buf, sizeof buf, "task %d (kind %d layer %d) may read data before its producers finish", i,
+                     t.kind, l);
+            return fail(c, MK_ERR_INVALID_ARG, buf);
+          }
+        // execute
+        cats_of_task(t, tmp);
+        for (int x : tmp) {
+          if (++cat_done[x] == cat_size[x]) { /* completion is only visible through events */ }
+        }
+        if (t.kind == TK_ATTN) {
+          size_t key = (size_t)l * B * nkv + t.row0;
+          uint64_t* acc = &attn_acc[key * W];
+          for (int w = 0; w < W; ++w) acc[w] |= gi[w];
+          if (++attn_arrive[key] == c->nch) {
+            // the merge runs after every chunk of the group: all their views hold, and the
+            // group's chunks are done
+            std::vector<int> done_cats;
+            for (int r = 0; r < c->nch; ++r) done_cats.push_back(cat_of(TK_ATTN, l));
+            for (int k = 0; k < t.n_notify; ++k) fire(t.notify[k], acc, done_cats);
+          }
+        } else {
+          for (int k = 0; k < t.n_notify; ++k) fire(t.notify[k], gi, tmp);
+        }
+        if (t.kind == TK_LMHEAD) ctr[c->ev_lm]++;
+        head[s]++;
+        executed++;
+        progress = true;
+      }
+    }
+  }
+  if (executed != T.size()) {
+    for (int s = 0; s < c->n_sms; ++s)
+      if (head[s] < q[s].size()) {
+        snprintf(buf, sizeof buf, "deadlock: SM %d blocked at its task %zu (graph task %d)", s, head[s],
+                 q[s][head[s]]);
+        return fail(c, MK_ERR_INVALID_ARG, buf);
+      }
+  }
+  return MK_OK;
+}
+
+std::vector<VTask> to_vtasks(const Graph& g) {
+  std::vector<VTask> v;
+  for (const TaskRec& r : g.tasks) {
+    VTask t;
+    t.kind = r.t.kind;
+    t.layer = r.t.layer;
+    t.sm = r.sm;
+    t.row0 = (int)r.t.row0;
+    t.nrows = r.t.kind == TK_ATTN ? (int)r.t.aux : (int)r.t.nrows;
+    t.n_wait = r.t.n_wait;
+    t.wait[0] = (int)r.t.wait[0];
+    t.wait[1] = (int)r.t.wait[1];
+    t.n_notify = r.t.n_notify;
+    t.notify[0] = (int)r.t.notify[0];
+    t.notify[1] = (int)r.t.notify[1];
+    v.push_back(t);
+  }
+  return v;
+}
+
+// ---------------------------------------------------------------------------------------
+int build_graph(mk_ctx* c) {
+  const mk_config& f = c->cfg;
+  const int L = f.n_layers, nkv = f.n_kv_heads, D = f.head_dim, n = c->n_sms;
+  const int B = f.max_batch;
+  c->n_events = 1 + L * (nkv + 4) + 1;
+  c->ev_lm = c->n_events - 1;
+  std::vector<uint32_t> evc(c->n_events, 0);
+  std::vector<std::vector<Task>> q(n);
+  const int rpg = (c->G + 2) * D;
+
+  // embedding slices
+  {
+    auto parts = partition_rows(f.hidden, 1, n);
+    for (int s = 0; s < n; ++s)
+      for (auto& p : parts[s]) {
+        Task t = make_task(TK_EMBED, 0, p.first, p.second);
+        add_notify(t, ev_embed());
+        evc[ev_embed()]++;
+        q[s].push_back(t);
+      }
+  }
+  auto qkv_parts = partition_rows(c->rows_qkv, 2, n);
+  auto o_parts = partition_rows(f.hidden, 1, n);
+  auto gu_parts = partition_rows(c->rows_gu, 2, n);
+  auto d_parts = partition_rows(f.hidden, 1, n);
+  const int n_attn = B * nkv * c->nch;
+  for (int l = 0; l < L; ++l) {
+    for (int s = 0; s < n; ++s)
+      for (auto& p : qkv_parts[s]) {
+        Task t = make_task(TK_QKV, l, p.first, p.second);
+        add_wait(t, l == 0 ? ev_embed() : ev_down(c, l - 1));
+        int g0 = p.first / rpg, g1 = (p.first + p.second - 1) / rpg;
+        if (g1 - g0 > 1) return fail(c, MK_ERR_UNSUPPORTED, "QKV tile spans more than two KV groups");
+        for (int g = g0; g <= g1; ++g) {
+          add_notify(t, ev_qkv(c, l, g));
+          evc[ev_qkv(c, l, g)]++;
+        }
+        q[s].push_back(t);
+      }
+    for (int idx = 0; idx < n_attn; ++idx) {
+      const int bg = idx / c->nch, ch = idx % c->nch;
+      const int g = bg % nkv;
+      Task t = make_task(TK_ATTN, l, bg, 0);
+      t.aux = (uint16_t)ch;
+      add_wait(t, ev_qkv(c, l, g));
+      add_notify(t, ev_attn(c, l));
+      const int s = (int)(((long long)idx * n / n_attn + (long long)l * 37) % n);
+      q[s].push_back(t);
+    }
+    evc[ev_attn(c, l)] = (uint32_t)(B * nkv);
+    for (int s = 0; s < n; ++s)
+      for (auto& p : o_parts[s]) {
+        Task t = make_task(TK_OPROJ, l, p.first, p.second);
+        add_wait(t, ev_attn(c, l));
+        add_notify(t, ev_o(c, l));
+        evc[ev_o(c, l)]++;
+        q[s].push_back(t);
+      }
+    for (int s = 0; s < n; ++s)
+      for (auto& p : gu_parts[s]) {
+        Task t = make_task(TK_GATEUP, l, p.first, p.second);
+        add_wait(t, ev_o(c, l));
+        add_notify(t, ev_gu(c, l));
+        evc[ev_gu(c, l)]++;
+        q[s].push_back(t);
+      }
+    for (int s = 0; s < n; ++s)
+      for (auto& p : d_parts[s]) {
+        Task t = make_task(TK_DOWN, l, p.first, p.second);
+        add_wait(t, ev_gu(c, l));
+        add_notify(t, ev_down(c, l));
+        evc[ev_down(c, l)]++;
+        q[s].push_back(t);
+      }
+  }
+  {
+    auto parts = partition_rows(f.vocab, 1, n);
+    int idx = 0;
+    for (int s = 0; s < n; ++s)
+      for (auto& p : parts[s]) {
+        Task t = make_task(TK_LMHEAD, L, p.first, p.second);
+        t.layer = (uint16_t)L;
+        add_wait(t, ev_down(c, L - 1));
+        t.index = (uint32_t)idx++;
+        q[s].push_back(t);
+      }
+    c->n_lm = idx;
+    evc[c->ev_lm] = (uint32_t)idx;
+  }
+  c->g.tasks.clear();
+  c->qbegin.assign(n + 1, 0);
+  uint64_t wbytes = 0;
+  for (int s = 0; s < n; ++s) {
+    c->qbegin[s] = (uint32_t)c->g.tasks.size();
+    for (auto& t : q[s]) {
+      c->g.tasks.push_back({t, s});
+      switch (t.kind) {
+        case TK_QKV: case TK_OPROJ: case TK_GATEUP: case TK_LMHEAD: wbytes += (uint64_t)t.nrows * f.hidden * 2; break;
+        case TK_DOWN: wbytes += (uint64_t)t.nrows * f.ffn * 2; break;
+      }
+    }
+  }
+  c->qbegin[n] = (uint32_t)c->g.tasks.size();
+  c->g.ev_count = evc;
+  c->g.n_sms = n;
+  c->weight_bytes_per_step = wbytes;
+  return validate(c, to_vtasks(c->g), evc);
+}
+
+void layout(mk_ctx* c) {
+  const mk_config& f = c->cfg;
+  const int L = f.n_layers, H = f.hidden, F = f.ffn, D = f.head_dim, nq = f.n_q_heads, nkv = f.n_kv_heads;
+  const int B = f.max_batch;
+  // weight arena
+  uint64_t o = 0;
+  c->loff.resize(L);
+  c->off_embed = o;
+  o = align256(o + (uint64_t)f.vocab * H * 2);
+  for (int l = 0; l < L; ++l) {
+    LayerOff& lo = c->loff[l];
+    lo.qkv = o;
+    o = align256(o + (uint64_t)c->rows_qkv * H * 2);
+    lo.o = o;
+    o = align256(o + (uint64_t)H * nq * D * 2);
+    lo.gu = o;
+    o = align256(o + (uint64_t)c->rows_gu * H * 2);
+    lo.d = o;
+    o = align256(o + (uint64_t)H * F * 2);
+    lo.attn_norm = o;
+    o = align256(o + (uint64_t)H * 2);
+    lo.mlp_norm = o;
+    o = align256(o + (uint64_t)H * 2);
+  }
+  c->off_lm = o;
+  o = align256(o + (uint64_t)f.vocab * H * 2);
+  c->off_fnorm = o;
+  o = align256(o + (uint64_t)H * 2);
+  c->arena_bytes = o;
+  // workspace
+  size_t w = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = w;
+    w = align256(w + bytes);
+    return at;
+  };
+  c->ws_tasks = take(c->g.tasks.size() * sizeof(Task));
+  c->ws_qbegin = take((c->n_sms + 1) * sizeof(uint32_t));
+  c->ws_evcount = take(c->n_events * sizeof(uint32_t));
+  c->ev_bytes = c->n_events * sizeof(uint32_t);
+  c->ws_ev = take(c->ev_bytes);
+  c->acnt_bytes = (size_t)L * B * nkv * sizeof(uint32_t);
+  c->ws_acnt = take(c->acnt_bytes);
+  c->ws_err = take(4 * sizeof(uint32_t));
+  c->ws_loff = take(L * sizeof(LayerOff));
+  c->ws_rope = take((size_t)f.max_seq * (D / 2) * sizeof(float2));
+  c->ws_xin = take((size_t)(L + 1) * B * H * 4);
+  c->ws_xmid = take((size_t)L * B * H * 4);
+  c->ws_q = take((size_t)L * B * nq * D * 4);
+  c->ws_o = take((size_t)L * B * nq * D * 4);
+  c->ws_h = take((size_t)L * B * F * 4);
+  c->ws_part = take((size_t)L * B * nq * c->nch * (D + 2) * 4);
+  c->ws_lmval = take((size_t)c->n_lm * B * 4);
+  c->ws_lmidx = take((size_t)c->n_lm * B * 4);
+  // prefill scratch: X, XN, Y, Q, O, HH per row
+  const long long ycols = std::max<long long>(std::max(c->rows_qkv, c->rows_gu), H);
+  c->pf_rows = (int)std::min<long long>(1024, (long long)B * f.max_seq);
+  const long long per_row = (long long)H * 2 + ycols + (long long)nq * D * 2 + F;
+  c->ws_pf = take((size_t)c->pf_rows * per_row * 4);
+  c->ws_bytes = w;
+  c->kv_bytes = (size_t)L * 2 * B * nkv * f.max_seq * D * 2;
+}
+
+int check_config(const mk_config* f, std::string* why) {
+  auto bad = [&](const char* m) {
+    *why = m;
+    return MK_ERR_INVALID_ARG;
+  };
+  if (!f) return bad("config is NULL");
+  if (f->n_layers < 1 || f->n_layers > 1024) return bad("n_layers out of range");
+  if (f->hidden < 8 || f->hidden % 8) return bad("hidden must be a positive multiple of 8");
+  if (f->ffn < 8 || f->ffn % 8) return bad("ffn must be a positive multiple of 8");
+  if (f->head_dim != 64 && f->head_dim != 128) return bad("head_dim must be 64 or 128");
+  if (f->n_q_heads < 1 || f->n_kv_heads < 1 || f->n_q_heads % f->n_kv_heads) return bad("bad head counts");
+  if (f->n_q_heads / f->n_kv_heads > 4) return bad("more than 4 query heads per KV head");
+  if (f->n_q_heads * f->head_dim != f->hidden) return bad("hidden must equal n_q_heads * head_dim");
+  if (f->vocab < 2) return bad("vocab too small");
+  if (!(f->rms_eps > 0) || !(f->rope_theta > 0)) return bad("rms_eps and rope_theta must be > 0");
+  if (f->max_batch < 1 || f->max_batch > MK_MAX_BATCH) return bad("max_batch out of range");
+  if (f->max_seq < 1 || f->max_seq > (1 << 20)) return bad("max_seq out of range");
+  if (f->tie_embeddings != 0) return bad("tied embeddings are not supported");
+  if (f->hidden > 4 * kSegElems || f->ffn > 8 * kSegElems) return bad("hidden or ffn too large");
+  return MK_OK;
+}
+
+// RoPE table: cos/sin of pos * theta^(-2i/D), computed in double and rounded to fp32.
+void rope_table(const mk_config& f, std::vector<float2>& out) {
+  const int half = f.head_dim / 2;
+  out.resize((size_t)f.max_seq * half);
+  for (int i = 0; i < half; ++i) {
+    const double inv = std::pow((double)f.rope_theta, -2.0 * i / f.head_dim);
+    for (int p = 0; p < f.max_seq; ++p) {
+      const double a = (double)p * inv;
+      out[(size_t)p * half + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+    }
+  }
+}
+
+bool cuda_ok(mk_ctx* c, cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return true;
+  fail(c, MK_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return false;
+}
+
+}  // namespace
+
+namespace mk {
+TensorMapEncodeFn get_tensor_map_encoder() {
+  static TensorMapEncodeFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<TensorMapEncodeFn>(p);
+  }
+  return fn;
+}
+}  // namespace mk
+
+// =========================================================================================
+extern "C" {
+
+int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
+  if (!out) return fail(nullptr, MK_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  std::string why;
+  int rc = check_config(cfg, &why);
+  if (rc) return fail(nullptr, rc, why);
+  mk_ctx* c = new mk_ctx();
+  c->cfg = *cfg;
+  c->device = device;
+  if (device >= 0) {
+    int n = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
+    if (e != cudaSuccess) {
+      delete c;
+      return fail(nullptr, MK_ERR_CUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
+    }
+    c->n_sms = n;
+  } else {
+    c->n_sms = 148;  // planning without a device: a B200's SM count
+  }
+  const mk_config& f = c->cfg;
+  c->G = f.n_q_heads / f.n_kv_heads;
+  c->rows_qkv = (f.n_q_heads + 2 * f.n_kv_heads) * f.head_dim;
+  c->rows_gu = 2 * f.ffn;
+  // split-KV chunks: fill the SMs with (sequence, KV head, chunk) tasks, chunks of >= 16 keys
+  {
+    int per = std::max(1, c->n_sms / (f.max_batch * f.n_kv_heads));
+    int by_len = std::max(1, (f.max_seq + 15) / 16);
+    c->nch = std::min(per, by_len);
+  }
+  c->nseg_h = (f.hidden + kSegElems - 1) / kSegElems;
+  c->nseg_f = (f.ffn + kSegElems - 1) / kSegElems;
+  c->rps_h = pow2_floor(std::min(kRMax, kSlotBytes / (f.hidden * 2)));
+  c->rps_f = pow2_floor(std::min(kRMax, kSlotBytes / (f.ffn * 2)));
+  if (f.ffn * 2 > kSlotBytes || f.hidden * 2 > kSlotBytes) {
+    delete c;
+    return fail(nullptr, MK_ERR_UNSUPPORTED, "a weight row does not fit one ring stage");
+  }
+  c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, 1);
+  rc = build_graph(c);
+  if (rc) {
+    std::string m = c->err;
+    delete c;
+    return fail(nullptr, rc, m);
+  }
+  layout(c);
+  c->pos.assign(f.max_batch, 0);
+  *out = c;
+  return MK_OK;
+}
+
+size_t mk_weight_arena_bytes(const mk_ctx* c) { return c ? c->arena_bytes : 0; }
+size_t mk_workspace_bytes(const mk_ctx* c) { return c ? c->ws_bytes : 0; }
+size_t mk_kv_cache_bytes(const mk_ctx* c) { return c ? c->kv_bytes : 0; }
+
+int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, void* workspace, void* stream) {
+  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!w || !weight_arena || !workspace) return fail(c, MK_ERR_INVALID_ARG, "NULL weights or buffers");
+  if (c->device < 0) return fail(c, MK_ERR_STATE, "context was planned without a device");
+  if ((reinterpret_cast<uintptr_t>(weight_arena) | reinterpret_cast<uintptr_t>(workspace)) & 255)
+    return fail(c, MK_ERR_INVALID_ARG, "arena and workspace must be 256-byte aligned");
+  const mk_config& f = c->cfg;
+  const int L = f.n_layers, H = f.hidden, F = f.ffn, D = f.head_dim, nq = f.n_q_heads, nkv = f.n_kv_heads;
+  if (!w->embed || !w->lm_head || !w->final_norm || !w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo ||
+      !w->mlp_norm || !w->wg || !w->wu || !w->wd)
+    return fail(c, MK_ERR_INVALID_ARG, "a weight pointer is NULL");
+  for (int l = 0; l < L; ++l)
+    if (!w->attn_norm[l] || !w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->mlp_norm[l] || !w->wg[l] ||
+        !w->wu[l] || !w->wd[l])
+      return fail(c, MK_ERR_INVALID_ARG, "a per-layer weight pointer is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!cuda_ok(c, cudaSetDevice(c->device), "cudaSetDevice")) return MK_ERR_CUDA;
+  uint8_t* A = static_cast<uint8_t*>(weight_arena);
+  auto put = [&](uint64_t off, const void* src, size_t bytes) {
+    return cuda_ok(c, cudaMemcpyAsync(A + off, src, bytes, cudaMemcpyHostToDevice, s), "weight copy");
+  };
+  if (!put(c->off_embed, w->embed, (size_t)f.vocab * H * 2)) return MK_ERR_CUDA;
+  if (!put(c->off_lm, w->lm_head, (size_t)f.vocab * H * 2)) return MK_ERR_CUDA;
+  if (!put(c->off_fnorm, w->final_norm, (size_t)H * 2)) return MK_ERR_CUDA;
+  std::vector<uint16_t> qkv((size_t)c->rows_qkv * H), gu((size_t)c->rows_gu * H);
+  const int G = c->G, half = D / 2;
+  for (int l = 0; l < L; ++l) {
+    // QKV rows grouped per KV head g: [q heads g*G.., k head g, v head g]; q and k rows of a
+    // head in RoPE pairs (i, i + D/2) -> packed (2i, 2i + 1); v rows in natural order
+    size_t r = 0;
+    auto copy_row = [&](const uint16_t* src, int row) {
+      std::memcpy(&qkv[r * H], src + (size_t)row * H, (size_t)H * 2);
+      ++r;
+    };
+    for (int g = 0; g < nkv; ++g) {
+      for (int hq = g * G; hq < (g + 1) * G; ++hq)
+        for (int i = 0; i < half; ++i) {
+          copy_row(w->wq[l], hq * D + i);
+          copy_row(w->wq[l], hq * D + i + half);
+        }
+      for (int i = 0; i < half; ++i) {
+        copy_row(w->wk[l], g * D + i);
+        copy_row(w->wk[l], g * D + i + half);
+      }
+      for (int i = 0; i < D; ++i) copy_row(w->wv[l], g * D + i);
+    }
+    for (int i = 0; i < F; ++i) {
+      std::memcpy(&gu[(size_t)(2 * i) * H], w->wg[l] + (size_t)i * H, (size_t)H * 2);
+      std::memcpy(&gu[(size_t)(2 * i + 1) * H], w->wu[l] + (size_t)i * H, (size_t)H * 2);
+    }
+    const LayerOff& lo = c->loff[l];
+    // synchronous copies: the staging vectors are reused for the next layer
+    if (!cuda_ok(c, cudaMemcpy(A + lo.qkv, qkv.data(), qkv.size() * 2, cudaMemcpyHostToDevice), "qkv copy"))
+      return MK_ERR_CUDA;
+    if (!cuda_ok(c, cudaMemcpy(A + lo.gu, gu.data(), gu.size() * 2, cudaMemcpyHostToDevice), "gate/up copy"))
+      return MK_ERR_CUDA;
+    if (!put(lo.o, w->wo[l], (size_t)H * nq * D * 2) || !put(lo.d, w->wd[l], (size_t)H * F * 2) ||
+        !put(lo.attn_norm, w->attn_norm[l], (size_t)H * 2) || !put(lo.mlp_norm, w->mlp_norm[l], (size_t)H * 2))
+      return MK_ERR_CUDA;
+  }
+  // workspace: task graph, counts, zeroed counters, offsets, RoPE table
+  uint8_t* W = static_cast<uint8_t*>(workspace);
+  std::vector<Task> tv;
+  for (auto& r : c->g.tasks) tv.push_back(r.t);
+  std::vector<float2> rope;
+  rope_table(f, rope);
+  if (!cuda_ok(c, cudaMemcpy(W + c->ws_tasks, tv.data(), tv.size() * sizeof(Task), cudaMemcpyHostToDevice),
+               "task upload") ||
+      !cuda_ok(c, cudaMemcpy(W + c->ws_qbegin, c->qbegin.data(), c->qbegin.size() * 4, cudaMemcpyHostToDevice),
+               "queue upload") ||
+      !cuda_ok(c, cudaMemcpy(W + c->ws_evcount, c->g.ev_count.data(), c->g.ev_count.size() * 4,
+                             cudaMemcpyHostToDevice),
+               "event upload") ||
+      !cuda_ok(c, cudaMemcpy(W + c->ws_loff, c->loff.data(), c->loff.size() * sizeof(LayerOff),
+                             cudaMemcpyHostToDevice),
+               "offset upload") ||
+      !cuda_ok(c, cudaMemcpy(W + c->ws_rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice),
+               "rope upload") ||
+      !cuda_ok(c, cudaMemset(W + c->ws_ev, 0, c->ev_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(W + c->ws_acnt, 0, c->acnt_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(W + c->ws_err, 0, 16), "error reset") ||
+      !cuda_ok(c, cudaStreamSynchronize(s), "load sync"))
+    return MK_ERR_CUDA;
+  c->arena = A;
+  c->ws = W;
+  c->loaded = true;
+  c->epoch = 0;
+  return MK_OK;
+}
+
+int mk_prefill(mk_ctx* c, const int32_t* tokens, int B, int T, void* kv_cache, float* last_logits, void* stream) {
+  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!c->loaded) return fail(c, MK_ERR_STATE, "weights not loaded");
+  if (!tokens || !kv_cache) return fail(c, MK_ERR_INVALID_ARG, "NULL tokens or cache");
+  if (B < 1 || B > c->cfg.max_batch || T < 1 || T > c->cfg.max_seq)
+    return fail(c, MK_ERR_INVALID_ARG, "B or T out of range");
+  const mk_config& f = c->cfg;
+  PrefillParams p;
+  p.arena = c->arena;
+  p.loff_host = c->loff.data();
+  p.off_embed = c->off_embed;
+  p.off_lm = c->off_lm;
+  p.off_fnorm = c->off_fnorm;
+  p.rope = reinterpret_cast<const float2*>(c->ws + c->ws_rope);
+  p.kv = static_cast<uint16_t*>(kv_cache);
+  const long long ycols = std::max<long long>(std::max(c->rows_qkv, c->rows_gu), f.hidden);
+  float* base = reinterpret_cast<float*>(c->ws + c->ws_pf);
+  const size_t R = (size_t)c->pf_rows;
+  p.X = base;
+  p.XN = p.X + R * f.hidden;
+  p.Y = p.XN + R * f.hidden;
+  p.Q = p.Y + R * ycols;
+  p.O = p.Q + R * f.n_q_heads * f.head_dim;
+  p.HH = p.O + R * f.n_q_heads * f.head_dim;
+  p.rows_cap = c->pf_rows;
+  p.H = f.hidden;
+  p.nq = f.n_q_heads;
+  p.nkv = f.n_kv_heads;
+  p.D = f.head_dim;
+  p.F = f.ffn;
+  p.V = f.vocab;
+  p.L = f.n_layers;
+  p.max_seq = f.max_seq;
+  p.max_batch = f.max_batch;
+  p.eps = f.rms_eps;
+  p.attn_scale = 1.0f / std::sqrt((float)f.head_dim);
+  std::string err;
+  int rc = run_prefill(p, tokens, B, T, last_logits, reinterpret_cast<cudaStream_t>(stream), &err);
+  if (rc) return fail(c, rc, err);
+  c->B = B;
+  for (int b = 0; b < B; ++b) c->pos[b] = T;
+  return MK_OK;
+}
+
+int mk_set_positions(mk_ctx* c, const int32_t* host_pos, int B) {
+  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!host_pos || B < 1 || B > c->cfg.max_batch) return fail(c, MK_ERR_INVALID_ARG, "bad positions");
+  for (int b = 0; b < B; ++b)
+    if (host_pos[b] < 0 || host_pos[b] >= c->cfg.max_seq) return fail(c, MK_ERR_INVALID_ARG, "position out of range");
+  c->B = B;
+  for (int b = 0; b < B; ++b) c->pos[b] = host_pos[b];
+  return MK_OK;
+}
+
+int mk_get_positions(const mk_ctx* c, int32_t* host_pos, int capacity) {
+  if (!c || (capacity > 0 && !host_pos)) return MK_ERR_INVALID_ARG;
+  for (int b = 0; b < c->B && b < capacity; ++b) host_pos[b] = c->pos[b];
+  return c->B;
+}
+
+int mk_decode_step(mk_ctx* c, const int32_t* tokens, void* kv_cache, float* logits, int32_t* next_tokens,
+                   void* stream) {
+  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!c->loaded) return fail(c, MK_ERR_STATE, "weights not loaded");
+  if (c->B < 1) return fail(c, MK_ERR_STATE, "no active batch (call mk_prefill or mk_set_positions)");
+  if (!tokens || !kv_cache || !logits) return fail(c, MK_ERR_INVALID_ARG, "NULL tokens, cache or logits");
+  if (c->variant < 0 || c->B > kMaxDecodeBatch)
+    return fail(c, MK_ERR_UNSUPPORTED, "no decode kernel instantiation for this shape / batch");
+  const mk_config& f = c->cfg;
+  for (int b = 0; b < c->B; ++b)
+    if (c->pos[b] >= f.max_seq) return fail(c, MK_ERR_INVALID_ARG, "sequence is full (max_seq reached)");
+  DecodeParams P;
+  std::memset(&P, 0, sizeof(P));
+  uint8_t* W = c->ws;
+  P.tasks = reinterpret_cast<const Task*>(W + c->ws_tasks);
+  P.qbegin = reinterpret_cast<const uint32_t*>(W + c->ws_qbegin);
+  P.ev_count = reinterpret_cast<const uint32_t*>(W + c->ws_evcount);
+  P.ev = reinterpret_cast<uint32_t*>(W + c->ws_ev);
+  P.acnt = reinterpret_cast<uint32_t*>(W + c->ws_acnt);
+  P.err = reinterpret_cast<uint32_t*>(W + c->ws_err);
+  P.arena = c->arena;
+  P.loff = reinterpret_cast<const LayerOff*>(W + c->ws_loff);
+  P.off_embed = c->off_embed;
+  P.off_lm = c->off_lm;
+  P.off_fnorm = c->off_fnorm;
+  P.rope = reinterpret_cast<const float2*>(W + c->ws_rope);
+  P.kv = static_cast<uint16_t*>(kv_cache);
+  P.x_in = reinterpret_cast<float*>(W + c->ws_xin);
+  P.x_mid = reinterpret_cast<float*>(W + c->ws_xmid);
+  P.qbuf = reinterpret_cast<float*>(W + c->ws_q);
+  P.obuf = reinterpret_cast<float*>(W + c->ws_o);
+  P.hbuf = reinterpret_cast<float*>(W + c->ws_h);
+  P.part = reinterpret_cast<float*>(W + c->ws_part);
+  P.lm_val = reinterpret_cast<float*>(W + c->ws_lmval);
+  P.lm_idx = reinterpret_cast<int32_t*>(W + c->ws_lmidx);
+  P.tokens = tokens;
+  P.logits = logits;
+  P.next_tokens = next_tokens;
+  for (int b = 0; b < c->B; ++b) P.pos[b] = c->pos[b];
+  P.B = f.max_batch;  // buffer strides use the capacity; the kernel serves sequence 0.. of it
+  P.H = f.hidden;
+  P.nq = f.n_q_heads;
+  P.nkv = f.n_kv_heads;
+  P.D = f.head_dim;
+  P.F = f.ffn;
+  P.V = f.vocab;
+  P.L = f.n_layers;
+  P.nch = c->nch;
+  P.max_seq = f.max_seq;
+  P.max_batch = f.max_batch;
+  P.n_lm = c->n_lm;
+  P.eps = f.rms_eps;
+  P.attn_scale = 1.0f / std::sqrt((float)f.head_dim);
+  P.epoch = c->epoch + 1;
+  P.ev_lm = (uint32_t)c->ev_lm;
+  P.drop_event = c->drop_event;
+  P.timeout_ns = c->timeout_ns;
+  P.trace = c->trace;
+  std::string err;
+  int rc = launch_decode(c->variant, P, c->n_sms, reinterpret_cast<cudaStream_t>(stream), &err);
+  if (rc) return fail(c, rc, err);
+  c->epoch += 1;
+  for (int b = 0; b < c->B; ++b) c->pos[b] += 1;
+  return MK_OK;
+}
+
+int mk_sync_status(mk_ctx* c, void* stream) {
+  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!cuda_ok(c, cudaStreamSynchronize(s), "stream sync")) return MK_ERR_CUDA;
+  if (!c->loaded) return MK_OK;
+  uint32_t e[4];
+  if (!cuda_ok(c, cudaMemcpy(e, c->ws + c->ws_err, 16, cudaMemcpyDeviceToHost), "error read")) return MK_ERR_CUDA;
+  if (e[ERR_CODE] == 0) return MK_OK;
+  if (e[ERR_CODE] == DEV_ERR_BAD_TOKEN && e[ERR_ABORT] == 0) {
+    cudaMemset(c->ws + c->ws_err, 0, 16);
+    return fail(c, MK_ERR_INVALID_ARG, "a token id was outside [0, vocab); row 0 was used");
+  }
+  char buf[160];
+  snprintf(buf, sizeof buf, "device wait timed out (kind %u, at %u, task %u)", e[ERR_CODE], e[ERR_WHERE],
+           e[ERR_TASK]);
+  // reset counters so the context stays usable
+  if (!cuda_ok(c, cudaMemset(c->ws + c->ws_ev, 0, c->ev_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(c->ws + c->ws_acnt, 0, c->acnt_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(c->ws + c->ws_err, 0, 16), "error reset") ||
+      !cuda_ok(c, cudaDeviceSynchronize(), "reset sync"))
+    return MK_ERR_CUDA;
+  c->epoch = 0;
+  return fail(c, MK_ERR_DEVICE_TIMEOUT, buf);
+}
+
+int mk_set_wait_timeout_ns(mk_ctx* c, uint64_t ns) {
+  if (!c || ns == 0) return fail(c, MK_ERR_INVALID_ARG, "timeout must be > 0");
+  c->timeout_ns = ns;
+  return MK_OK;
+}
+
+int mk_debug_drop_notify(mk_ctx* c, int event_id, int on) {
+  if (!c || event_id < 0 || event_id >= c->n_events) return fail(c, MK_ERR_INVALID_ARG, "bad event id");
+  c->drop_event = on ? event_id : -1;
+  return MK_OK;
+}
+
+int mk_set_trace(mk_ctx* c, void* device_buffer) {
+  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (device_buffer && (reinterpret_cast<uintptr_t>(device_buffer) & 7))
+    return fail(c, MK_ERR_INVALID_ARG, "trace buffer must be 8-byte aligned");
+  c->trace = static_cast<uint64_t*>(device_buffer);
+  return MK_OK;
+}
+
+int mk_get_graph_info(const mk_ctx* c, mk_graph_info* out) {
+  if (!c || !out) return MK_ERR_INVALID_ARG;
+  out->n_sms = c->n_sms;
+  out->n_tasks = (int)c->g.tasks.size();
+  out->n_events = c->n_events;
+  out->attn_chunks = c->nch;
+  out->kernel_variant = c->variant;
+  out->weight_bytes_per_step = c->weight_bytes_per_step;
+  out->smem_bytes = decode_smem_bytes();
+  return MK_OK;
+}
+
+int mk_export_taskgraph(const mk_ctx* c, int32_t* tasks, int task_capacity, int32_t* event_counts,
+                        int event_capacity) {
+  if (!c) return MK_ERR_INVALID_ARG;
+  std::vector<VTask> v = to_vtasks(c->g);
+  if (tasks)
+    for (int i = 0; i < (int)v.size() && i < task_capacity; ++i) {
+      const VTask& t = v[i];
+      int32_t* o = tasks + (size_t)i * 11;
+      o[0] = t.kind; o[1] = t.layer; o[2] = t.sm; o[3] = t.row0; o[4] = t.nrows; o[5] = t.n_wait;
+      o[6] = t.wait[0]; o[7] = t.wait[1]; o[8] = t.n_notify; o[9] = t.notify[0]; o[10] = t.notify[1];
+    }
+  if (event_counts)
+    for (int e = 0; e < c->n_events && e < event_capacity; ++e) event_counts[e] = (int32_t)c->g.ev_count[e];
+  return (int)v.size();
+}
+
+int mk_validate_taskgraph(mk_ctx* c, const int32_t* tasks, int n_tasks, const int32_t* event_counts, int n_events) {
+  if (!c || !tasks || !event_counts || n_tasks < 0 || n_events != c->n_events)
+    return fail(c, MK_ERR_INVALID_ARG, "bad arguments to mk_validate_taskgraph");
+  std::vector<VTask> v(n_tasks);
+  for (int i = 0; i < n_tasks; ++i) {
+    const int32_t* o = tasks + (size_t)i * 11;
+    v[i] = VTask{o[0], o[1], o[2], o[3], o[4], o[5], {o[6], o[7]}, o[8], {o[9], o[10]}};
+  }
+  std::vector<uint32_t> cnt(n_events);
+  for (int e = 0; e < n_events; ++e) cnt[e] = (uint32_t)std::max(0, event_counts[e]);
+  return validate(c, v, cnt);
+}
+
+size_t mk_attention_workspace_bytes(int BH, int d, int L) {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return attention_workspace_bytes(BH, d, L, n);
+}
+
+int mk_attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d, int L,
+                        float scale, void* workspace, void* stream) {
+  if (!q || !k_t || !v || !o) return fail(nullptr, MK_ERR_INVALID_ARG, "NULL operand");
+  if (BH < 1 || L < 1 || (d != 64 && d != 128)) return fail(nullptr, MK_ERR_INVALID_ARG, "bad BH, d or L");
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return fail(nullptr, MK_ERR_CUDA, "no CUDA device");
+  std::string err;
+  int rc = attention_decode(q, k_t, v, o, BH, d, L, scale, workspace, reinterpret_cast<cudaStream_t>(stream), n,
+                            2000000000ull, &err);
+  if (rc) return fail(nullptr, rc, err);
+  return MK_OK;
+}
+
+int mk_attention_status(void* workspace, int BH, int d, int L, void* stream) {
+  if (!workspace || BH < 1 || L < 1 || (d != 64 && d != 128)) return fail(nullptr, MK_ERR_INVALID_ARG, "bad arguments");
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return fail(nullptr, MK_ERR_CUDA, "stream sync failed");
+  if (L % 8 != 0) return MK_OK;  // the plain-load path has no waits and no workspace
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  uint32_t* word = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) +
+                                               attention_error_word_offset(BH, d, L, n));
+  uint32_t e = 0;
+  if (cudaMemcpy(&e, word, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return fail(nullptr, MK_ERR_CUDA, "read failed");
+  if (e == 0) return MK_OK;
+  // a timed-out call may leave arrival counts behind: clear them with the error word
+  size_t bytes = attention_workspace_bytes(BH, d, L, n);
+  cudaMemset(workspace, 0, bytes);
+  cudaDeviceSynchronize();
+  return fail(nullptr, MK_ERR_DEVICE_TIMEOUT, "attention wait timed out");
+}
+
+const char* mk_last_error(const mk_ctx* c) { return c ? c->err.c_str() : g_err.c_str(); }
+
+void mk_destroy(mk_ctx* c) { delete c; }
+
+}  // extern "C"

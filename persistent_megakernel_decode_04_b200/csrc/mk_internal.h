@@ -1,0 +1,139 @@
+// mk_internal.h -- structures shared by the library's host code and its kernels.
+//
+// Task graph (Part 1 "Compilateur" of the MPK summary "Compiler des LLM en MegaKernel ..."):
+// a task is one tile of one op assigned to one SM (worker); an event is a counter in device
+// memory with a per-step threshold.  A task waits on up to two events and notifies up to
+// two.  Thresholds are epoch-based: during decode step e (1, 2, ...) event v is active once
+// its counter reaches e * count[v], so nothing is reset between steps.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "mk.h"
+
+namespace mk {
+
+// ---- persistent decode kernel geometry ----
+constexpr int kWorkerWarps = 8;                      // compute role (the "worker" of Part 2)
+constexpr int kWorkerThreads = kWorkerWarps * 32;    // 256
+constexpr int kProducerWarp = kWorkerWarps;          // TMA weight streaming
+constexpr int kSchedWarp = kWorkerWarps + 1;         // event polling (the "scheduler" role)
+constexpr int kBlockThreads = (kWorkerWarps + 2) * 32;
+constexpr int kSegElems = kWorkerThreads * 8;        // K elements one pass of all workers covers
+constexpr int kSegBytes = kSegElems * 2;
+constexpr int kRMax = 32;                            // rows per GEMV task (one per lane after reduction)
+constexpr int kSlotBytes = 32 * 1024;                // one ring stage
+constexpr int kStages = 6;                           // ring depth
+constexpr int kMaxDecodeBatch = 1;                   // CUDA-core path instantiations
+
+enum TaskKind : uint8_t {
+  TK_EMBED = 1,   // x_0 = E[token] for a slice of rows
+  TK_QKV = 2,     // q,k,v rows of W_qkv . RMSNorm(x); RoPE; K/V append
+  TK_ATTN = 3,    // split-KV chunk of one (sequence, KV head); last arriver merges
+  TK_OPROJ = 4,   // x_mid = x + W_o o
+  TK_GATEUP = 5,  // h = silu(W_g xn) * (W_u xn), rows interleaved (g_i, u_i)
+  TK_DOWN = 6,    // x_next = x_mid + W_d h
+  TK_LMHEAD = 7,  // logits rows of W_lm . RMSNorm(x); per-task argmax partial
+};
+
+struct Task {
+  uint8_t kind, n_wait, n_notify, pad0;
+  uint16_t layer, aux;  // ATTN: aux = chunk index
+  uint32_t row0;        // GEMV: first (packed) row; ATTN: b * n_kv_heads + kv head; EMBED: first row
+  uint32_t nrows;       // GEMV / EMBED: row count; ATTN: 0
+  uint32_t wait[2];
+  uint32_t notify[2];   // ATTN: notify[0] is raised by the merging (last) chunk only
+  uint32_t index;       // LMHEAD: ordinal among LM-head tasks (argmax partial slot)
+  uint32_t pad1;
+};
+static_assert(sizeof(Task) == 40, "Task layout");
+
+// Byte offsets of one layer's tensors in the weight arena.
+struct LayerOff {
+  uint64_t qkv, o, gu, d;   // packed matrices
+  uint64_t attn_norm, mlp_norm;
+};
+
+struct DecodeParams {
+  const Task* tasks;
+  const uint32_t* qbegin;     // [n_sms + 1]
+  const uint32_t* ev_count;   // [n_events]
+  uint32_t* ev;               // [n_events] counters
+  uint32_t* acnt;             // [L][B][nkv] attention chunk arrivals
+  uint32_t* err;              // [4]: code, where, task, global abort flag
+  const uint8_t* arena;
+  const LayerOff* loff;       // [L]
+  uint64_t off_embed, off_lm, off_fnorm;
+  const float2* rope;         // [max_seq][D/2] (cos, sin)
+  uint16_t* kv;               // [L][2][max_batch][nkv][max_seq][D]
+  float* x_in;                // [L+1][B][H]
+  float* x_mid;               // [L][B][H]
+  float* qbuf;                // [L][B][nq*D]
+  float* obuf;                // [L][B][nq*D]
+  float* hbuf;                // [L][B][F]
+  float* part;                // [L][B][nq][nch][D+2]
+  float* lm_val;              // [n_lm][B]
+  int32_t* lm_idx;            // [n_lm][B]
+  const int32_t* tokens;      // [B]
+  float* logits;              // [B][V]
+  int32_t* next_tokens;       // [B] or null
+  int pos[MK_MAX_BATCH];
+  int B, H, nq, nkv, D, F, V, L, nch, max_seq, max_batch, n_lm;
+  float eps, attn_scale;
+  uint32_t epoch;
+  uint32_t ev_lm;             // event counting finished LM-head tasks (last one picks the token)
+  int drop_event;             // test hook: notify skipped for this event id (-1 = none)
+  uint64_t timeout_ns;
+  uint64_t* trace;            // optional [n_tasks][kTraceWords] timing records (null = off)
+};
+
+// Trace record per task (global-timer ns): worker start of the wait for inputs, inputs
+// released, task done; worker ns blocked on ring stages | SM id << 32; producer ns blocked
+// on a full ring while issuing this task's stages; producer time of the task's first issue.
+constexpr int kTraceWords = 6;
+
+// Error word layout in the workspace.
+enum { ERR_CODE = 0, ERR_WHERE = 1, ERR_TASK = 2, ERR_ABORT = 3 };
+enum { DEV_ERR_WAIT_EVENT = 1, DEV_ERR_WAIT_READY = 2, DEV_ERR_WAIT_FULL = 3, DEV_ERR_WAIT_EMPTY = 4,
+       DEV_ERR_BAD_TOKEN = 5 };
+
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+TensorMapEncodeFn get_tensor_map_encoder();
+
+// Kernel variants: one instantiation per (segments, rows per stage) of the two K sizes.
+struct Variant {
+  int nseg_h, rps_h, nseg_f, rps_f, batch;
+};
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int batch);
+const void* decode_kernel_ptr(int variant);
+size_t decode_smem_bytes();
+int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t stream, std::string* err);
+
+// Standalone attention (mk_attention.cu).
+size_t attention_workspace_bytes(int BH, int d, int L, int n_sms);
+size_t attention_error_word_offset(int BH, int d, int L, int n_sms);
+int attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d, int L,
+                     float scale, void* workspace, cudaStream_t stream, int n_sms, uint64_t timeout_ns,
+                     std::string* err);
+
+// Prefill (mk_prefill.cu).
+struct PrefillParams {
+  const uint8_t* arena;
+  const LayerOff* loff_host;  // host copy of per-layer offsets
+  uint64_t off_embed, off_lm, off_fnorm;
+  const float2* rope;
+  uint16_t* kv;
+  float *X, *XN, *Y, *Q, *O, *HH;  // scratch [rows][...]
+  int rows_cap;
+  int H, nq, nkv, D, F, V, L, max_seq, max_batch;
+  float eps, attn_scale;
+};
+int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, float* last_logits,
+                cudaStream_t stream, std::string* err);
+
+}  // namespace mk

@@ -1,0 +1,135 @@
+"""C-ABI library: loads without a GPU, exports every entry point of include/mk.h, checks
+configs, and its task-graph validator accepts the built graphs and rejects corrupted ones."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import mk_inputs as mi
+import persistent_megakernel_decode_04_b200 as mk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "mk.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mk_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_entry_point():
+    names = header_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(mk._lib, n), f"libmk.so lacks {n}"
+    assert set(names) == set(mk.exported_symbols())
+
+
+def _cfg(**kw):
+    c = mk.Config.from_shape(mi.TINY, 1, 64)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("field,value", [("head_dim", 96), ("hidden", 250), ("n_kv_heads", 3), ("max_batch", 0),
+                                         ("max_batch", 17), ("max_seq", 0), ("rms_eps", 0.0), ("vocab", 1)])
+def test_bad_configs_are_rejected(field, value):
+    with pytest.raises(mk.MkError) as e:
+        mk.mk_build_taskgraph(_cfg(**{field: value}).c(), -1)
+    assert e.value.code == mk.MK_ERR_INVALID_ARG
+
+
+def test_null_context_calls_fail_cleanly():
+    assert mk._lib.mk_decode_step(None, None, None, None, None, None) == mk.MK_ERR_INVALID_ARG
+    assert mk._lib.mk_prefill(None, None, 1, 1, None, None, None) == mk.MK_ERR_INVALID_ARG
+    assert mk.mk_last_error(None)
+
+
+def test_decode_before_load_is_a_state_error():
+    ctx = mk.mk_build_taskgraph(_cfg().c(), -1)
+    try:
+        rc = mk._lib.mk_decode_step(ctx, 1, 1, 1, None, None)
+        assert rc == mk.MK_ERR_STATE
+    finally:
+        mk.mk_destroy(ctx)
+
+
+@pytest.fixture(params=["tiny", "llama3-8b", "chameleon-7b-b1"])
+def graph(request):
+    shape, ms = {"tiny": (mi.TINY, 64), "llama3-8b": (mi.LLAMA8B, 1024),
+                 "chameleon-7b-b1": (mi.CHAMELEON7B, 1280)}[request.param]
+    ctx = mk.mk_build_taskgraph(mk.Config.from_shape(shape, 1, ms).c(), -1)
+    tasks, counts = mk.mk_export_taskgraph(ctx)
+    yield ctx, tasks, counts, shape
+    mk.mk_destroy(ctx)
+
+
+def test_built_graph_validates_and_balances_bytes(graph):
+    ctx, tasks, counts, shape = graph
+    assert mk.mk_validate_taskgraph(ctx, tasks, counts) == 0
+    info = mk.mk_get_graph_info(ctx)
+    # weight bytes streamed per step = every projection once (plain definition of the step)
+    s = shape
+    per_layer = ((s.n_q_heads + 2 * s.n_kv_heads) * s.head_dim * s.hidden + s.hidden * s.n_q_heads * s.head_dim
+                 + 2 * s.ffn * s.hidden + s.hidden * s.ffn) * 2
+    assert info["weight_bytes_per_step"] == s.n_layers * per_layer + s.vocab * s.hidden * 2
+    # each SM streams nearly the same number of weight bytes (within 3 %)
+    K = {2: s.hidden, 4: s.hidden, 5: s.hidden, 6: s.ffn, 7: s.hidden}
+    per_sm = np.zeros(info["n_sms"])
+    for t in tasks:
+        if t[0] in K:
+            per_sm[t[2]] += t[4] * K[t[0]] * 2
+    if s.hidden >= 4096:
+        assert per_sm.max() / per_sm.mean() < 1.03
+
+
+def _reject(ctx, tasks, counts, needle):
+    rc = mk.mk_validate_taskgraph(ctx, tasks, counts)
+    assert rc == mk.MK_ERR_INVALID_ARG
+    assert needle in mk.mk_last_error(ctx), mk.mk_last_error(ctx)
+
+
+def test_validator_rejects_a_dropped_notify(graph):
+    ctx, tasks, counts, _ = graph
+    t = tasks.copy()
+    i = int(np.nonzero(t[:, 0] == 4)[0][0])  # an O-projection task
+    t[i, 8] = 0
+    _reject(ctx, t, counts, "producers per step")
+
+
+def test_validator_rejects_a_missing_dependency(graph):
+    ctx, tasks, counts, _ = graph
+    t = tasks.copy()
+    i = int(np.nonzero(t[:, 0] == 3)[0][-1])  # an attention task loses its wait on QKV
+    t[i, 5] = 0
+    _reject(ctx, t, counts, "before its producers finish")
+
+
+def test_validator_rejects_a_queue_that_deadlocks(graph):
+    ctx, tasks, counts, _ = graph
+    t = tasks.copy()
+    # move SM 0's first down-projection task in front of its first gate/up task
+    sm0 = np.nonzero(t[:, 2] == 0)[0]
+    gu = [i for i in sm0 if t[i, 0] == 5][0]
+    dn = [i for i in sm0 if t[i, 0] == 6][0]
+    order = list(range(len(t)))
+    order.remove(dn)
+    order.insert(order.index(gu), dn)
+    _reject(ctx, t[order], counts, "deadlock")
+
+
+def test_validator_rejects_overlapping_rows(graph):
+    ctx, tasks, counts, _ = graph
+    t = tasks.copy()
+    i = int(np.nonzero(t[:, 0] == 7)[0][3])
+    t[i, 3] -= 2  # LM-head tile shifted onto its neighbour's rows
+    _reject(ctx, t, counts, "covered")
+
+
+def test_validator_rejects_a_wrong_threshold(graph):
+    ctx, tasks, counts, _ = graph
+    c = counts.copy()
+    c[1] += 1
+    _reject(ctx, tasks, c, "threshold")
