@@ -129,6 +129,11 @@ int mk_set_wait_timeout_ns(mk_ctx* ctx, uint64_t ns);
  * Nothing faults or traps. */
 int mk_debug_drop_notify(mk_ctx* ctx, int event_id, int on);
 
+/* Weight prefetch depth: besides the shared-memory ring (6 stages of 32 KB per SM), each
+ * SM's producer prefetches the next `stages` weight stages of its queue into L2, so HBM keeps
+ * streaming while the ring is full (default 0 = off, which measured fastest on B200; at most 64). */
+int mk_set_l2_prefetch(mk_ctx* ctx, int stages);
+
 /* Tracing (per-task timing of the next decode steps).  device_buffer: n_tasks * 6 uint64
  * records (n_tasks from mk_get_graph_info), or NULL to switch tracing off.  Record of task i
  * (global-timer ns): [0] worker starts waiting for the task's inputs, [1] inputs released by

@@ -79,6 +79,7 @@ _SIGS = {
     "mk_sync_status": ([_vp, _vp], _i32),
     "mk_set_wait_timeout_ns": ([_vp, _u64], _i32),
     "mk_debug_drop_notify": ([_vp, _i32, _i32], _i32),
+    "mk_set_l2_prefetch": ([_vp, _i32], _i32),
     "mk_set_trace": ([_vp, _vp], _i32),
     "mk_get_graph_info": ([_vp, ctypes.POINTER(mk_graph_info)], _i32),
     "mk_export_taskgraph": ([_vp, _vp, _i32, _vp, _i32], _i32),
@@ -205,6 +206,10 @@ def mk_set_wait_timeout_ns(ctx, ns: int):
 
 def mk_debug_drop_notify(ctx, event_id: int, on: bool):
     _check(_lib.mk_debug_drop_notify(ctx, int(event_id), int(bool(on))), ctx)
+
+
+def mk_set_l2_prefetch(ctx, stages: int):
+    _check(_lib.mk_set_l2_prefetch(ctx, int(stages)), ctx)
 
 
 def mk_set_trace(ctx, device_buffer):

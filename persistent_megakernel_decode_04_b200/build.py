@@ -32,14 +32,21 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > so_t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, csrc: str | None = None, out: str | None = None,
+          defines=()) -> str:
+    """Compile every .cu/.cpp of `csrc` (default: this package's csrc/) into `out`
+    (default: libmk.so next to this file).  `defines`: extra -D macros."""
+    so = out or SO
+    if not force and out is None and not _stale():
         return SO
-    objdir = os.path.join(HERE, "_build")
+    src_dir = csrc or CSRC
+    objdir = os.path.join(os.path.dirname(so), "_build")
     os.makedirs(objdir, exist_ok=True)
     objs, report = [], []
-    common = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"), "-I", CSRC]
-    for src in sources():
+    common = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"), "-I", src_dir]
+    common += [f"-D{d}" for d in defines]
+    srcs = sorted(glob.glob(os.path.join(src_dir, "*.cu")) + glob.glob(os.path.join(src_dir, "*.cpp")))
+    for src in srcs:
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [NVCC, *ARCH, *common, "-lineinfo", "-c", src, "-o", obj]
         if src.endswith(".cu"):
@@ -50,10 +57,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
             sys.stderr.write(r.stderr)
             raise RuntimeError(f"nvcc failed on {src}")
         objs.append(obj)
-    tmp = SO + ".tmp"
+    tmp = so + ".tmp"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lrt", "-lpthread"])
-    os.replace(tmp, SO)
-    with open(os.path.join(HERE, "libmk.ptxas.txt"), "w") as f:
+    os.replace(tmp, so)
+    with open(os.path.join(os.path.dirname(so), "libmk.ptxas.txt"), "w") as f:
         f.write("\n".join(report))
     if verbose:
         print("\n".join(report))

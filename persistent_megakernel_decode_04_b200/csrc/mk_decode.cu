@@ -33,12 +33,15 @@ namespace mk {
 
 struct DSmem {
   uint8_t ring[kStages][kSlotBytes];
-  float red[kWorkerWarps][32];
-  float tot[kRMax];
+  union {
+    float red[kWorkerWarps][kTaskRows];  // GEMV: per-warp row sums of the current task
+    float aacc[kAttnWarps][4][128];      // attention: per-warp partial outputs
+  };
+  float tot[kTaskRows];                  // row totals of the current task
   float ssw[kWorkerWarps];
-  float am[kWorkerWarps][4];
-  float al[kWorkerWarps][4];
-  float aacc[kWorkerWarps][4][128];
+  float am[kAttnWarps][4];
+  float al[kAttnWarps][4];
+  float mm[4 * kMaxChunks], ll[4 * kMaxChunks], ww[4 * kMaxChunks];  // split-KV merge
   float lmv[kWorkerWarps];
   int lmi[kWorkerWarps];
   uint64_t full[kStages];
@@ -124,20 +127,54 @@ __device__ __forceinline__ bool is_gemv(uint8_t k) {
 }
 
 // ---------------------------------------------------------------------------------------
-// GEMV core: acc[r] = sum_k W[row0 + r][k] * x[k] * g[k] for r < nrows, rows streamed through
-// the ring RPS rows per stage.  Writes the per-row totals to S.tot and returns (via S.ssw) the
-// sum of squares of x for the fused norm.  Returns false if a wait ran out (uniform).
+// Warp reduction of the V (power of two) row partials a[0..V) of one ring stage: transposed
+// butterfly (each exchange halves the live values), then a plain butterfly over the lanes
+// left; lane l with l % (32/V) == 0 ends with the warp's sum for row r(l).
+__host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v / 2); }
+
+template <int V>
+__device__ __forceinline__ void warp_reduce_rows(float (&a)[V], float* out, int lane, int valid) {
+  constexpr int LV = ilog2(V);
+#pragma unroll
+  for (int k = 0; k < LV; ++k) {
+    const int off = 16 >> k, half = (V >> k) >> 1;
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? a[i] : a[i + half];
+      const float keep = upper ? a[i + half] : a[i];
+      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+#pragma unroll
+  for (int off = 16 >> LV; off >= 1; off >>= 1) a[0] += __shfl_xor_sync(0xffffffffu, a[0], off);
+  if ((lane & ((32 >> LV) - 1)) == 0) {
+    int r = 0;
+#pragma unroll
+    for (int k = 0; k < LV; ++k) r += ((lane >> (4 - k)) & 1) * ((V >> k) >> 1);
+    if (r < valid) out[r] = a[0];
+  }
+}
+
+// GEMV core: tot[r] = sum_k W[row0 + r][k] * x[k] * g[k] for r < nrows (<= kTaskRows), rows
+// streamed through the ring RPS rows per stage.  The stage loop is a runtime loop and only
+// one stage's rows are unrolled, so the code stays small; each stage's rows are reduced
+// across lanes right away into S.red[warp][row], and across warps at the end into S.tot.
+// Also leaves the per-warp sums of x^2 in S.ssw for the fused norm.  Returns false (for
+// every worker thread alike) if a wait ran out.
 template <int NSEG, int RPS>
 __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe& pp, const float* __restrict__ xsrc,
                                           const uint16_t* __restrict__ gain, int K, int nrows, uint32_t row_bytes,
                                           uint32_t task_id, uint32_t& stall_ns) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // only the last segment can be partial: K > (NSEG - 1) * kSegElems by construction
+  const bool last_ok = (NSEG - 1) * kSegElems + tid * 8 < K;
   float x[NSEG][8];
   float ss = 0.f;
 #pragma unroll
   for (int s = 0; s < NSEG; ++s) {
     const int k = s * kSegElems + tid * 8;
-    if (k < K) {
+    if (s < NSEG - 1 || last_ok) {
       const float4 a = __ldcg(reinterpret_cast<const float4*>(xsrc + k));
       const float4 b = __ldcg(reinterpret_cast<const float4*>(xsrc + k + 4));
       x[s][0] = a.x; x[s][1] = a.y; x[s][2] = a.z; x[s][3] = a.w;
@@ -156,59 +193,50 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
       for (int i = 0; i < 8; ++i) x[s][i] = 0.f;
     }
   }
-  float acc[kRMax];
-#pragma unroll
-  for (int r = 0; r < kRMax; ++r) acc[r] = 0.f;
+  float* red = S.red[warp];
   bool ok = true;
+  for (int r0 = 0; r0 < nrows; r0 += RPS) {
+    const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
+    if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
+      if (ok) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
+      ok = false;
+      S.cabort = 1u;
+    }
+    if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
+    const uint8_t* base = S.ring[pp.stage] + tid * 16;
+    float a[RPS], b[RPS];  // two partial sums per row: shorter dependency chains
 #pragma unroll
-  for (int r = 0; r < kRMax; ++r) {
-    if (r < nrows) {
-      if (r % RPS == 0) {
-        const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
-        if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
-          if (ok) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
-          ok = false;
-          S.cabort = 1u;
-        }
-        if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
-      }
-      const uint8_t* row = S.ring[pp.stage] + (r % RPS) * row_bytes;
+    for (int rr = 0; rr < RPS; ++rr) {
+      a[rr] = 0.f;
+      b[rr] = 0.f;
+      if (RPS == 1 || r0 + rr < nrows) {
 #pragma unroll
-      for (int s = 0; s < NSEG; ++s) {
-        if (s * kSegElems + tid * 8 < K) {
-          const uint4 w = *reinterpret_cast<const uint4*>(row + s * kSegBytes + tid * 16);
-          acc[r] = dot8(w, x[s], acc[r]);
+        for (int s = 0; s < NSEG; ++s) {
+          if (s < NSEG - 1 || last_ok) {
+            const uint4 w = *reinterpret_cast<const uint4*>(base + rr * row_bytes + s * kSegBytes);
+            if (s & 1) b[rr] = dot8(w, x[s], b[rr]);
+            else a[rr] = dot8(w, x[s], a[rr]);
+          }
         }
-      }
-      if (r % RPS == RPS - 1 || r == nrows - 1) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
-        pp.advance();
       }
     }
-  }
-  // transposed butterfly: afterwards lane l holds the warp's sum for row l
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
+    pp.advance();
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
-    const bool upper = (lane & off) != 0;
-#pragma unroll
-    for (int i = 0; i < off; ++i) {
-      const float send = upper ? acc[i] : acc[i + off];
-      const float keep = upper ? acc[i + off] : acc[i];
-      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-    }
+    for (int rr = 0; rr < RPS; ++rr) a[rr] += b[rr];
+    warp_reduce_rows<RPS>(a, red + r0, lane, nrows - r0);
   }
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  S.red[warp][lane] = acc[0];
   if (lane == 0) S.ssw[warp] = ss;
   worker_bar();
   if (S.cabort) return false;
-  if (tid < nrows) {
-    float t = 0.f;
+  for (int t = tid; t < nrows; t += kWorkerThreads) {
+    float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWorkerWarps; ++w) t += S.red[w][tid];
-    S.tot[tid] = t;
+    for (int w2 = 0; w2 < kWorkerWarps; ++w2) v += S.red[w2][t];
+    S.tot[t] = v;
   }
   worker_bar();
   return true;
@@ -267,7 +295,10 @@ __device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, c
 // ---------------------------------------------------------------------------------------
 // Split-KV attention chunk for one (sequence, KV head): scores of its G query heads over the
 // chunk's keys, per-warp online softmax, merged across warps into one partial (m, l, acc).
-// The last chunk to arrive merges all partials of the (sequence, KV head) into o.
+// At the current length only nch_eff = ceil(L / kMinChunkKeys) (at most nch) chunks hold keys;
+// the other chunk tasks only count their arrival.  The last task of the (sequence, KV head)
+// to arrive merges the partials into o (FlashDecoding-style online-softmax merge) and
+// notifies; with a single chunk in use that chunk writes o directly and nothing is merged.
 template <int D>
 __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, const Task& t, uint32_t task_id) {
   constexpr int DL = D / 32;
@@ -276,203 +307,196 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
   const int b = (int)t.row0 / P.nkv, g = (int)t.row0 % P.nkv;
   const int c = t.aux;
   const int Lk = P.pos[b] + 1;
-  const int cl = (Lk + P.nch - 1) / P.nch;
+  const int nch_eff = max(1, min(P.nch, (Lk + kMinChunkKeys - 1) / kMinChunkKeys));
+  const int cl = (Lk + nch_eff - 1) / nch_eff;
   const int j0 = c * cl, j1 = min(Lk, j0 + cl);
   const size_t head_stride = (size_t)P.max_seq * D;
   const size_t kv_layer = (size_t)P.max_batch * P.nkv * head_stride;
   const uint16_t* kc = P.kv + ((size_t)t.layer * 2 + 0) * kv_layer + ((size_t)b * P.nkv + g) * head_stride;
   const uint16_t* vc = P.kv + ((size_t)t.layer * 2 + 1) * kv_layer + ((size_t)b * P.nkv + g) * head_stride;
   const float* qsrc = P.qbuf + ((size_t)t.layer * P.B + b) * P.nq * D + (size_t)g * G * D;
+  // partial of (head h, chunk cc) of this sequence at part_base + (h * nch + cc) * (D + 2)
+  float* part_base = P.part + ((size_t)t.layer * P.B + b) * P.nq * (size_t)P.nch * (D + 2);
+  float* o = P.obuf + ((size_t)t.layer * P.B + b) * P.nq * D + (size_t)g * G * D;
 
-  float qv[4][DL], m[4], l[4], acc[4][DL];
-#pragma unroll
-  for (int h = 0; h < 4; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-#pragma unroll
-    for (int i = 0; i < DL; ++i) {
-      qv[h][i] = (h < G) ? __ldcg(qsrc + h * D + lane * DL + i) * P.attn_scale : 0.f;
-      acc[h][i] = 0.f;
-    }
-  }
-  for (int j = j0 + warp; j < j1; j += kWorkerWarps) {
-    float kf[DL], vf[DL];
-    if (DL == 4) {
-      const uint2 kw = __ldcg(reinterpret_cast<const uint2*>(kc + (size_t)j * D + lane * 4));
-      const uint2 vw = __ldcg(reinterpret_cast<const uint2*>(vc + (size_t)j * D + lane * 4));
-      kf[0] = bf16lo(kw.x); kf[1] = bf16hi(kw.x); kf[2 % DL] = bf16lo(kw.y); kf[3 % DL] = bf16hi(kw.y);
-      vf[0] = bf16lo(vw.x); vf[1] = bf16hi(vw.x); vf[2 % DL] = bf16lo(vw.y); vf[3 % DL] = bf16hi(vw.y);
-    } else {
-      const uint32_t kw = __ldcg(reinterpret_cast<const unsigned int*>(kc + (size_t)j * D + lane * 2));
-      const uint32_t vw = __ldcg(reinterpret_cast<const unsigned int*>(vc + (size_t)j * D + lane * 2));
-      kf[0] = bf16lo(kw); kf[1 % DL] = bf16hi(kw);
-      vf[0] = bf16lo(vw); vf[1 % DL] = bf16hi(vw);
-    }
-    float s[4];
+  if (c < nch_eff) {  // uniform across the CTA
+    float qv[4][DL], m[4], l[4], acc[4][DL];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      float a = 0.f;
+      m[h] = -INFINITY;
+      l[h] = 0.f;
 #pragma unroll
-      for (int i = 0; i < DL; ++i) a = fmaf(qv[h][i], kf[i], a);
-      s[h] = a;
+      for (int i = 0; i < DL; ++i) {
+        qv[h][i] = (h < G) ? __ldcg(qsrc + h * D + lane * DL + i) * P.attn_scale : 0.f;
+        acc[h][i] = 0.f;
+      }
     }
+    for (int j = j0 + warp; warp < kAttnWarps && j < j1; j += kAttnWarps) {
+      float kf[DL], vf[DL];
+      if (DL == 4) {
+        const uint2 kw = __ldcg(reinterpret_cast<const uint2*>(kc + (size_t)j * D + lane * 4));
+        const uint2 vw = __ldcg(reinterpret_cast<const uint2*>(vc + (size_t)j * D + lane * 4));
+        kf[0] = bf16lo(kw.x); kf[1] = bf16hi(kw.x); kf[2 % DL] = bf16lo(kw.y); kf[3 % DL] = bf16hi(kw.y);
+        vf[0] = bf16lo(vw.x); vf[1] = bf16hi(vw.x); vf[2 % DL] = bf16lo(vw.y); vf[3 % DL] = bf16hi(vw.y);
+      } else {
+        const uint32_t kw = __ldcg(reinterpret_cast<const unsigned int*>(kc + (size_t)j * D + lane * 2));
+        const uint32_t vw = __ldcg(reinterpret_cast<const unsigned int*>(vc + (size_t)j * D + lane * 2));
+        kf[0] = bf16lo(kw); kf[1 % DL] = bf16hi(kw);
+        vf[0] = bf16lo(vw); vf[1 % DL] = bf16hi(vw);
+      }
+      float sc[4];
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1)
+      for (int h = 0; h < 4; ++h) {
+        float a = 0.f;
 #pragma unroll
-      for (int h = 0; h < 4; ++h) s[h] += __shfl_xor_sync(0xffffffffu, s[h], off);
+        for (int i = 0; i < DL; ++i) a = fmaf(qv[h][i], kf[i], a);
+        sc[h] = a;
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1)
+#pragma unroll
+        for (int h = 0; h < 4; ++h) sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], off);
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        if (h < G) {
+          const float mn = fmaxf(m[h], sc[h]);
+          const float a = expf(m[h] - mn);
+          const float p = expf(sc[h] - mn);
+          l[h] = l[h] * a + p;
+#pragma unroll
+          for (int i = 0; i < DL; ++i) acc[h][i] = fmaf(acc[h][i], a, p * vf[i]);
+          m[h] = mn;
+        }
+      }
+    }
+    // cross-warp merge of this chunk
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      if (h < G) {
-        const float mn = fmaxf(m[h], s[h]);
-        const float a = expf(m[h] - mn);
-        const float p = expf(s[h] - mn);
-        l[h] = l[h] * a + p;
+      if (h < G && warp < kAttnWarps) {
+        if (lane == 0) {
+          S.am[warp][h] = m[h];
+          S.al[warp][h] = l[h];
+        }
 #pragma unroll
-        for (int i = 0; i < DL; ++i) acc[h][i] = fmaf(acc[h][i], a, p * vf[i]);
-        m[h] = mn;
+        for (int i = 0; i < DL; ++i) S.aacc[warp][h][lane * DL + i] = acc[h][i];
       }
     }
-  }
-  // cross-warp merge of the chunk
+    worker_bar();
+    for (int e = tid; e < G * D; e += kWorkerThreads) {
+      const int h = e / D, d = e % D;
+      float M = -INFINITY;
 #pragma unroll
-  for (int h = 0; h < 4; ++h) {
-    if (h < G) {
-      if (lane == 0) {
-        S.am[warp][h] = m[h];
-        S.al[warp][h] = l[h];
+      for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, S.am[w][h]);
+      float ls = 0.f, as = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) {
+          const float f = expf(S.am[w][h] - M);
+          ls += f * S.al[w][h];
+          as += f * S.aacc[w][h][d];
+        }
       }
-#pragma unroll
-      for (int i = 0; i < DL; ++i) S.aacc[warp][h][lane * DL + i] = acc[h][i];
-    }
-  }
-  worker_bar();
-  const int nq = P.nq;
-  float* part_base = P.part + (((size_t)t.layer * P.B + b) * nq) * (size_t)P.nch * (D + 2);
-  for (int e = tid; e < G * D; e += kWorkerThreads) {
-    const int h = e / D, d = e % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWorkerWarps; ++w) M = fmaxf(M, S.am[w][h]);
-    float ls = 0.f, as = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kWorkerWarps; ++w) {
-        const float f = expf(S.am[w][h] - M);
-        ls += f * S.al[w][h];
-        as += f * S.aacc[w][h][d];
+      if (nch_eff == 1) {
+        o[(size_t)h * D + d] = as / ls;  // the only chunk in use: final output, nothing to merge
+      } else {
+        float* pc = part_base + ((size_t)(g * G + h) * P.nch + c) * (D + 2);
+        pc[2 + d] = as;
+        if (d == 0) {
+          pc[0] = M;
+          pc[1] = ls;
+        }
       }
-    }
-    float* pp = part_base + ((size_t)(g * G + h) * P.nch + c) * (D + 2);
-    pp[2 + d] = as;
-    if (d == 0) {
-      pp[0] = M;
-      pp[1] = ls;
     }
   }
   worker_bar();
   if (tid == 0) {
-    __threadfence();
     uint32_t* cnt = P.acnt + ((size_t)t.layer * P.B + b) * P.nkv + g;
     const uint32_t old = atom_acq_rel_gpu_add(cnt, 1u);
     S.flag = (old + 1u == P.epoch * (uint32_t)P.nch) ? 1u : 0u;
   }
   worker_bar();
-  if (S.flag) {
-    __threadfence();
-    float* o = P.obuf + ((size_t)t.layer * P.B + b) * nq * D + (size_t)g * G * D;
+  if (S.flag && nch_eff > 1) {
+    // (m, l) of every used chunk of this group's heads, loaded in parallel
+    for (int e = tid; e < G * nch_eff; e += kWorkerThreads) {
+      const int h = e / nch_eff, cc = e % nch_eff;
+      const float* pc = part_base + ((size_t)(g * G + h) * P.nch + cc) * (D + 2);
+      S.mm[e] = __ldcg(pc);
+      S.ll[e] = __ldcg(pc + 1);
+    }
+    worker_bar();
+    for (int e = tid; e < G * nch_eff; e += kWorkerThreads) {
+      const int h = e / nch_eff;
+      float M = -INFINITY;
+      for (int cc = 0; cc < nch_eff; ++cc) M = fmaxf(M, S.mm[h * nch_eff + cc]);
+      S.ww[e] = (S.mm[e] == -INFINITY) ? 0.f : expf(S.mm[e] - M);
+    }
+    worker_bar();
     for (int e = tid; e < G * D; e += kWorkerThreads) {
       const int h = e / D, d = e % D;
-      const float* ph = part_base + (size_t)(g * G + h) * P.nch * (D + 2);
-      float M = -INFINITY;
-      for (int cc = 0; cc < P.nch; ++cc) M = fmaxf(M, __ldcg(ph + (size_t)cc * (D + 2)));
+      const float* ph = part_base + (size_t)(g * G + h) * P.nch * (D + 2) + 2 + d;
       float num = 0.f, den = 0.f;
-      for (int cc = 0; cc < P.nch; ++cc) {
-        const float* pc = ph + (size_t)cc * (D + 2);
-        const float mc = __ldcg(pc);
-        if (mc == -INFINITY) continue;
-        const float f = expf(mc - M);
-        den += f * __ldcg(pc + 1);
-        num += f * __ldcg(pc + 2 + d);
+#pragma unroll 8
+      for (int cc = 0; cc < nch_eff; ++cc) {
+        const float w = S.ww[h * nch_eff + cc];
+        num = fmaf(w, __ldcg(ph + (size_t)cc * (D + 2)), num);
+        den = fmaf(w, S.ll[h * nch_eff + cc], den);
       }
       o[(size_t)h * D + d] = num / den;
     }
     worker_bar();
-    if (tid == 0 && (int)t.notify[0] != P.drop_event) {
-      __threadfence();
-      red_release_gpu_add(&P.ev[t.notify[0]], 1u);
-    }
   }
+  if (S.flag && tid == 0 && (int)t.notify[0] != P.drop_event) red_release_gpu_add(&P.ev[t.notify[0]], 1u);
   (void)task_id;
   return true;
 }
 
 // LM-head epilogue: logits and this task's (max, index) partial; the last LM task picks the token.
-__device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, const Task& t, float r) {
+__device__ __forceinline__ void argmax_merge(float& v, int& idx, float ov, int oi) {
+  if (ov > v || (ov == v && oi < idx)) {
+    v = ov;
+    idx = oi;
+  }
+}
+
+__device__ __forceinline__ void block_argmax(DSmem& S, float& v, int& idx) {
   const int tid = threadIdx.x, lane = tid & 31;
-  const int b = 0;
-  if (tid < 32) {
-    float v = -INFINITY;
-    int idx = 0x7fffffff;
-    if (tid < (int)t.nrows) {
-      v = S.tot[tid] * r;
-      idx = (int)t.row0 + tid;
-      P.logits[(size_t)b * P.V + idx] = v;
-    }
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, v, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
-      if (ov > v || (ov == v && oi < idx)) {
-        v = ov;
-        idx = oi;
-      }
-    }
-    if (lane == 0) {
-      P.lm_val[(size_t)t.index * P.B + b] = v;
-      P.lm_idx[(size_t)t.index * P.B + b] = idx;
-    }
+  for (int off = 16; off >= 1; off >>= 1)
+    argmax_merge(v, idx, __shfl_xor_sync(0xffffffffu, v, off), __shfl_xor_sync(0xffffffffu, idx, off));
+  if (lane == 0) {
+    S.lmv[tid >> 5] = v;
+    S.lmi[tid >> 5] = idx;
   }
   worker_bar();
+  if (tid == 0)
+    for (int w = 1; w < kWorkerWarps; ++w) argmax_merge(v, idx, S.lmv[w], S.lmi[w]);
+}
+
+__device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, const Task& t, float r) {
+  const int tid = threadIdx.x;
+  const int b = 0;
+  float v = -INFINITY;
+  int idx = 0x7fffffff;
+  for (int i = tid; i < (int)t.nrows; i += kWorkerThreads) {
+    const float lv = S.tot[i] * r;
+    P.logits[(size_t)b * P.V + t.row0 + i] = lv;
+    argmax_merge(v, idx, lv, (int)t.row0 + i);
+  }
+  block_argmax(S, v, idx);
   if (tid == 0) {
-    __threadfence();
+    P.lm_val[(size_t)t.index * P.B + b] = v;
+    P.lm_idx[(size_t)t.index * P.B + b] = idx;
     const uint32_t old = atom_acq_rel_gpu_add(&P.ev[P.ev_lm], 1u);
     S.flag = (old + 1u == P.epoch * (uint32_t)P.n_lm) ? 1u : 0u;
   }
   worker_bar();
   if (S.flag && P.next_tokens) {
-    __threadfence();
-    float v = -INFINITY;
-    int idx = 0x7fffffff;
-    for (int i = tid; i < P.n_lm; i += kWorkerThreads) {
-      const float ov = __ldcg(P.lm_val + (size_t)i * P.B + b);
-      const int oi = __ldcg(P.lm_idx + (size_t)i * P.B + b);
-      if (ov > v || (ov == v && oi < idx)) {
-        v = ov;
-        idx = oi;
-      }
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, v, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
-      if (ov > v || (ov == v && oi < idx)) {
-        v = ov;
-        idx = oi;
-      }
-    }
-    if (lane == 0) {
-      S.lmv[tid >> 5] = v;
-      S.lmi[tid >> 5] = idx;
-    }
-    worker_bar();
-    if (tid == 0) {
-      for (int w = 1; w < kWorkerWarps; ++w)
-        if (S.lmv[w] > v || (S.lmv[w] == v && S.lmi[w] < idx)) {
-          v = S.lmv[w];
-          idx = S.lmi[w];
-        }
-      P.next_tokens[b] = idx;
-    }
+    v = -INFINITY;
+    idx = 0x7fffffff;
+    for (int i = tid; i < P.n_lm; i += kWorkerThreads)
+      argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
+    block_argmax(S, v, idx);
+    if (tid == 0) P.next_tokens[b] = idx;
   }
 }
 
@@ -501,6 +525,30 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     // ------------------------------- producer -------------------------------
     if (lane != 0) return;
     const uint64_t pol = policy_evict_first();
+    // L2 lookahead: a second cursor over this queue's weight stages runs l2_ahead stages in
+    // front of the ring cursor and prefetches them into L2, so HBM keeps streaming while the
+    // ring is full (e.g. while the workers wait for a dependency).
+    uint32_t la_task = qb, la_row = 0;
+    int la_lead = 0;  // stages the lookahead cursor is ahead of the ring cursor
+    auto la_step = [&]() {  // prefetch the stage under the lookahead cursor and advance it
+      while (la_task < qe) {
+        const Task lt = P.tasks[la_task];
+        if (!is_gemv(lt.kind) || la_row >= lt.nrows) {
+          ++la_task;
+          la_row = 0;
+          continue;
+        }
+        uint64_t off;
+        uint32_t rb;
+        gemv_source(P, lt, &off, &rb);
+        const uint32_t rps = (lt.kind == TK_DOWN) ? (uint32_t)RPS_F : (uint32_t)RPS_H;
+        const uint32_t nr = min(rps, lt.nrows - la_row);
+        prefetch_l2(P.arena + off + (uint64_t)(lt.row0 + la_row) * rb, nr * rb);
+        la_row += rps;
+        ++la_lead;
+        return;
+      }
+    };
     Pipe pp{0, 0};
     int issued = 0;
     bool ok = true;
@@ -515,6 +563,8 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
       uint64_t blocked = 0, first = 0;
       for (uint32_t r0 = 0; r0 < t.nrows; r0 += (uint32_t)rps) {
         const uint32_t nr = min((uint32_t)rps, t.nrows - r0);
+        // keep the lookahead l2_ahead stages in front of the stage about to enter the ring
+        while (la_lead < P.l2_ahead && la_task < qe) la_step();
         const uint64_t tw = P.trace ? globaltimer_ns() : 0;
         if (!wait_bar(&S.empty[pp.stage], pp.phase ^ 1u, P.timeout_ns, &S)) {
           if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, i);
@@ -529,6 +579,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
         mbar_arrive_expect_tx(&S.full[pp.stage], nr * rb);
         bulk_g2s(S.ring[pp.stage], src + (uint64_t)r0 * rb, nr * rb, &S.full[pp.stage], pol);
         ++issued;
+        if (P.l2_ahead > 0) --la_lead;  // this stage was prefetched while it was ahead
         pp.advance();
       }
       if (P.trace) {
@@ -693,7 +744,6 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     if (notify) {
       worker_bar();
       if (tid == 0) {
-        __threadfence();
         for (int k = 0; k < t.n_notify; ++k)
           if ((int)t.notify[k] != P.drop_event) red_release_gpu_add(&P.ev[t.notify[k]], 1u);
       }
@@ -705,21 +755,26 @@ out:
 
 // ---------------------------------------------------------------------------------------
 // Instantiations: (segments, rows per stage) for K = hidden and K = ffn.
+// One instantiation per weight-row shape class: (segments, rows per ring stage) of the
+// K = hidden and K = ffn GEMVs, computed from representative sizes.
+__host__ __device__ constexpr int seg_count(int K) { return (K + kSegElems - 1) / kSegElems; }
+__host__ __device__ constexpr int pow2_floor_c(int x) { return x < 2 ? 1 : 2 * pow2_floor_c(x / 2); }
+__host__ __device__ constexpr int stage_rows(int K) {
+  return pow2_floor_c((kSlotBytes / (2 * K)) < kRpsMax ? (kSlotBytes / (2 * K)) : kRpsMax);
+}
+#define MK_VARIANT(H, F) {seg_count(H), stage_rows(H), seg_count(F), stage_rows(F), 1}
+#define MK_KERNEL(H, F) (const void*)decode_kernel<seg_count(H), stage_rows(H), seg_count(F), stage_rows(F)>
 static const Variant kVariants[] = {
-    {2, 4, 7, 1, 1},   // Llama-3-8B shape: hidden 4096, ffn 14336
-    {2, 4, 6, 1, 1},   // Chameleon-7B shape: hidden 4096, ffn 11008
-    {1, 32, 1, 16, 1}, // tiny: hidden 256, ffn 768
-    {1, 32, 1, 32, 1}, // small test shapes: hidden <= 256, ffn <= 512
-    {2, 4, 2, 4, 1},   // hidden 4096, ffn <= 4096
-    {1, 32, 2, 4, 1},  // hidden <= 256... ffn in (2048, 4096]
+    MK_VARIANT(4096, 14336),  // Llama-3-8B shape
+    MK_VARIANT(4096, 11008),  // Chameleon-7B shape
+    MK_VARIANT(256, 768),     // tiny decoder
+    MK_VARIANT(4096, 4096),
+    MK_VARIANT(2048, 4096),
+    MK_VARIANT(256, 256),
 };
-
-typedef void (*DecodeFn)(DecodeParams);
-
 static const void* kFns[] = {
-    (const void*)decode_kernel<2, 4, 7, 1>,  (const void*)decode_kernel<2, 4, 6, 1>,
-    (const void*)decode_kernel<1, 32, 1, 16>, (const void*)decode_kernel<1, 32, 1, 32>,
-    (const void*)decode_kernel<2, 4, 2, 4>,  (const void*)decode_kernel<1, 32, 2, 4>,
+    MK_KERNEL(4096, 14336), MK_KERNEL(4096, 11008), MK_KERNEL(256, 768),
+    MK_KERNEL(4096, 4096),  MK_KERNEL(2048, 4096),  MK_KERNEL(256, 256),
 };
 
 int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int batch) {

@@ -72,6 +72,7 @@ struct mk_ctx {
   uint64_t timeout_ns = 2000000000ull;
   int drop_event = -1;
   uint64_t* trace = nullptr;
+  int l2_ahead = 0;
   std::string err;
 };
 
@@ -100,7 +101,7 @@ int ev_gu(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads + 2
 int ev_down(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads + 3; }
 
 // Split `total` rows over n_sms SMs in contiguous, balanced ranges (multiples of gran), and
-// each range into tasks of at most kRMax rows.
+// each range into tasks of at most kTaskRows rows.
 std::vector<std::vector<std::pair<int, int>>> partition_rows(int total, int gran, int n_sms) {
   std::vector<std::vector<std::pair<int, int>>> out(n_sms);
   for (int s = 0; s < n_sms; ++s) {
@@ -108,14 +109,14 @@ std::vector<std::vector<std::pair<int, int>>> partition_rows(int total, int gran
     int b = (s + 1 == n_sms) ? total : (int)(((long long)total * (s + 1) / n_sms) / gran * gran);
     int n = b - a;
     if (n <= 0) continue;
-    int nt = (n + kRMax - 1) / kRMax;
+    int nt = (n + kTaskRows - 1) / kTaskRows;
     for (;;) {
       bool ok = true;
       std::vector<std::pair<int, int>> parts;
       for (int i = 0; i < nt; ++i) {
         int lo = (int)(((long long)n * i / nt) / gran * gran);
         int hi = (i + 1 == nt) ? n : (int)(((long long)n * (i + 1) / nt) / gran * gran);
-        if (hi - lo > kRMax) ok = false;
+        if (hi - lo > kTaskRows) ok = false;
         if (hi > lo) parts.push_back({a + lo, hi - lo});
       }
       if (ok) {
@@ -216,7 +217,7 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
     }
     if (t.kind < TK_EMBED || t.kind > TK_LMHEAD) return fail(c, MK_ERR_INVALID_ARG, "unknown task kind");
     int rows = rows_of(t.kind);
-    if (t.nrows <= 0 || t.nrows > kRMax || t.row0 < 0 || t.row0 + t.nrows > rows)
+    if (t.nrows <= 0 || t.nrows > kTaskRows || t.row0 < 0 || t.row0 + t.nrows > rows)
       return fail(c, MK_ERR_INVALID_ARG, "task rows out of range");
     if ((t.kind == TK_QKV || t.kind == TK_GATEUP) && ((t.row0 | t.nrows) & 1))
       return fail(c, MK_ERR_INVALID_ARG, "QKV/gate-up tasks must hold whole row pairs");
@@ -663,12 +664,12 @@ int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
   {
     int per = std::max(1, c->n_sms / (f.max_batch * f.n_kv_heads));
     int by_len = std::max(1, (f.max_seq + 15) / 16);
-    c->nch = std::min(per, by_len);
+    c->nch = std::min(std::min(per, by_len), kMaxChunks);
   }
   c->nseg_h = (f.hidden + kSegElems - 1) / kSegElems;
   c->nseg_f = (f.ffn + kSegElems - 1) / kSegElems;
-  c->rps_h = pow2_floor(std::min(kRMax, kSlotBytes / (f.hidden * 2)));
-  c->rps_f = pow2_floor(std::min(kRMax, kSlotBytes / (f.ffn * 2)));
+  c->rps_h = pow2_floor(std::min(kRpsMax, kSlotBytes / (f.hidden * 2)));
+  c->rps_f = pow2_floor(std::min(kRpsMax, kSlotBytes / (f.ffn * 2)));
   if (f.ffn * 2 > kSlotBytes || f.hidden * 2 > kSlotBytes) {
     delete c;
     return fail(nullptr, MK_ERR_UNSUPPORTED, "a weight row does not fit one ring stage");
@@ -898,6 +899,7 @@ int mk_decode_step(mk_ctx* c, const int32_t* tokens, void* kv_cache, float* logi
   P.drop_event = c->drop_event;
   P.timeout_ns = c->timeout_ns;
   P.trace = c->trace;
+  P.l2_ahead = c->l2_ahead;
   std::string err;
   int rc = launch_decode(c->variant, P, c->n_sms, reinterpret_cast<cudaStream_t>(stream), &err);
   if (rc) return fail(c, rc, err);
@@ -940,6 +942,12 @@ int mk_set_wait_timeout_ns(mk_ctx* c, uint64_t ns) {
 int mk_debug_drop_notify(mk_ctx* c, int event_id, int on) {
   if (!c || event_id < 0 || event_id >= c->n_events) return fail(c, MK_ERR_INVALID_ARG, "bad event id");
   c->drop_event = on ? event_id : -1;
+  return MK_OK;
+}
+
+int mk_set_l2_prefetch(mk_ctx* c, int stages) {
+  if (!c || stages < 0 || stages > 64) return fail(c, MK_ERR_INVALID_ARG, "stages must be in [0, 64]");
+  c->l2_ahead = stages;
   return MK_OK;
 }
 

@@ -17,14 +17,20 @@
 namespace mk {
 
 // ---- persistent decode kernel geometry ----
-constexpr int kWorkerWarps = 8;                      // compute role (the "worker" of Part 2)
+#ifndef MK_WORKER_WARPS
+#define MK_WORKER_WARPS 8
+#endif
+constexpr int kWorkerWarps = MK_WORKER_WARPS;        // compute role (the "worker" of Part 2)
+constexpr int kAttnWarps = 8;                        // workers that walk keys in an attention task
 constexpr int kWorkerThreads = kWorkerWarps * 32;    // 256
 constexpr int kProducerWarp = kWorkerWarps;          // TMA weight streaming
 constexpr int kSchedWarp = kWorkerWarps + 1;         // event polling (the "scheduler" role)
 constexpr int kBlockThreads = (kWorkerWarps + 2) * 32;
 constexpr int kSegElems = kWorkerThreads * 8;        // K elements one pass of all workers covers
 constexpr int kSegBytes = kSegElems * 2;
-constexpr int kRMax = 32;                            // rows per GEMV task (one per lane after reduction)
+constexpr int kTaskRows = 256;                       // rows per GEMV task (one per worker thread)
+constexpr int kRpsMax = 32;                          // rows per ring stage (unrolled in the GEMV loop)
+constexpr int kMaxChunks = 64;                       // split-KV chunks per (sequence, KV head)
 constexpr int kSlotBytes = 32 * 1024;                // one ring stage
 constexpr int kStages = 6;                           // ring depth
 constexpr int kMaxDecodeBatch = 1;                   // CUDA-core path instantiations
@@ -88,7 +94,9 @@ struct DecodeParams {
   int drop_event;             // test hook: notify skipped for this event id (-1 = none)
   uint64_t timeout_ns;
   uint64_t* trace;            // optional [n_tasks][kTraceWords] timing records (null = off)
+  int l2_ahead;               // weight stages the producer prefetches into L2 beyond the ring
 };
+constexpr int kMinChunkKeys = 32;  // split-KV chunks hold at least this many keys
 
 // Trace record per task (global-timer ns): worker start of the wait for inputs, inputs
 // released, task done; worker ns blocked on ring stages | SM id << 32; producer ns blocked
