@@ -1,0 +1,369 @@
+"""Benchmark: 8B-shaped batch-1 decode on the persistent megakernel (one B200 per rank).
+
+Workload (one "step" = one decode step = one launch of the megakernel): Llama-3-8B-shaped
+decoder (32 layers, hidden 4096, 32/8 heads x 128, SwiGLU 14336, vocab 128256), seeded
+random bf16 weights N(0, 0.02) (16 GB), a 39-token seeded prompt prefilled into the bf16
+KV cache, then greedy decode with the next token fed back on the device.  W warm-up steps
+and K timed steps follow the prompt, so positions 39 .. 39+W+K-1 are decoded (the default
+W=8, K=504 is the 512-step run of that workload).  The weights stream from HBM every step
+(15 GB > the 126 MB L2), so no L2 flush is needed between steps.
+
+Multi-GPU (torchrun, one process per GPU): independent replicas, no collective on the data
+path; the timed region is bracketed by a barrier and a device synchronise on every rank and
+the slowest rank's time is reported.  `--impl reference` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode ms/token + achieved HBM GB/s (% of peak), 8B-shape bs=1, 1 B200"
+PROMPT_LEN = 39
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=504)
+    p.add_argument("--warmup", type=int, default=8)
+    p.add_argument("--impl", default="mk", choices=["mk", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=64)
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(shape, positions):
+    """Bytes one decode step must read from HBM: every weight once (projections, norms, LM
+    head), one embedding row, and the K/V actually attended (positions 0..p inclusive)."""
+    s = shape
+    D = s.head_dim
+    per_layer = ((s.n_q_heads + 2 * s.n_kv_heads) * D * s.hidden + s.hidden * s.n_q_heads * D
+                 + 2 * s.ffn * s.hidden + s.hidden * s.ffn + 2 * s.hidden) * 2
+    weights = s.n_layers * per_layer + (s.vocab * s.hidden + s.hidden) * 2 + s.hidden * 2
+    kv = [s.n_layers * 2 * s.n_kv_heads * (p + 1) * D * 2 for p in positions]
+    return weights, kv
+
+
+def kernel_source_hash():
+    src = os.path.join(ROOT, "persistent_megakernel_decode_04_b200", "csrc", "mk_decode.cu")
+    with open(src, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(per_step_alg_bytes):
+    """DRAM bytes per launch from the committed ncu summary, scaled to this launch's
+    algorithmic bytes; None if the summary is missing or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "decode_kernel_llama8b_traffic.txt")
+    try:
+        kv = {}
+        for line in open(path):
+            if "=" in line and not line.startswith("#"):
+                k, v = line.split("=", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None, "kernel changed since the ncu capture"
+        ratio = float(kv["dram_bytes"]) / float(kv["algorithmic_bytes"])
+        return ratio * per_step_alg_bytes, kv.get("how", "")
+    except Exception:
+        return None, "no ncu summary"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.uuid = uuid
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu=uuid,{self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        mhz, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            if self.uuid and parts[0] != self.uuid:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------------------- CPU oracle
+
+def oracle_ms_per_token(weights_full, shape, budget_s=20.0):
+    """Time the CPU oracle on a bounded sample of the same workload: decode steps of the
+    8B shape truncated to one layer (full LM head) after a synthetic 39-position cache;
+    ms/token is scaled to the full model by weight bytes (the oracle's work is proportional
+    to the weights it reads)."""
+    import mk_inputs as mi
+    import oracle
+    one = mi.Weights(shape.with_layers(1), weights_full.embed, weights_full.lm_head, weights_full.final_norm,
+                     weights_full.attn_norm[:1], weights_full.wq[:1], weights_full.wk[:1], weights_full.wv[:1],
+                     weights_full.wo[:1], weights_full.mlp_norm[:1], weights_full.wg[:1], weights_full.wu[:1],
+                     weights_full.wd[:1])
+    d = oracle.Decoder(one, 1, PROMPT_LEN + 64)
+    d.set_cache(mi.kv_cache_values(0, one.shape, 1, PROMPT_LEN, sigma=1.0), PROMPT_LEN)
+    tok = np.array([1], dtype=np.int32)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        d.decode(tok)
+        n += 1
+        if time.perf_counter() - t0 > budget_s or n >= 64:
+            break
+    dt = (time.perf_counter() - t0) / n
+    full_w, _ = algorithmic_bytes(shape, [PROMPT_LEN])
+    one_w, _ = algorithmic_bytes(one.shape, [PROMPT_LEN])
+    cores = int(os.environ.get("OR_THREADS", os.cpu_count() or 1))
+    return dt * 1e3 * full_w / one_w, cores, n
+
+
+# ------------------------------------------------------------------------------- arms
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import mk_inputs as mi
+    shape = mi.LLAMA8B
+    t = time.perf_counter()
+    w1 = mi.make_weights(shape.with_layers(1), seed=0)
+    import oracle
+    d = oracle.Decoder(w1, 1, PROMPT_LEN + args.warmup + args.steps + 1)
+    d.set_cache(mi.kv_cache_values(0, w1.shape, 1, PROMPT_LEN, sigma=1.0), PROMPT_LEN)
+    tok = np.array([1], dtype=np.int32)
+    for _ in range(args.warmup):
+        tok = np.array([oracle.argmax(d.decode(tok)[0])], dtype=np.int32)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        tok = np.array([oracle.argmax(d.decode(tok)[0])], dtype=np.int32)
+    dt = (time.perf_counter() - t0) / args.steps
+    full_w, _ = algorithmic_bytes(shape, [PROMPT_LEN])
+    one_w, _ = algorithmic_bytes(w1.shape, [PROMPT_LEN])
+    ms = dt * 1e3 * full_w / one_w
+    cores = int(os.environ.get("OR_THREADS", os.cpu_count() or 1))
+    sample = (f"each step: one oracle decode step of the 8B shape truncated to 1 layer (full LM head), "
+              f"scaled to 32 layers by weight bytes ({full_w / one_w:.2f}x)")
+    out = {"impl": "reference", "metric": METRIC, "value": ms, "unit": "ms/token", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": False,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded random weights)",
+           "config": {"workload": "llama3-8b-shape decode, batch 1, 39-token prompt, greedy",
+                      "prompt_len": PROMPT_LEN, "parallelism": "replicas", "weights": "bf16"},
+           "cpu_baseline": {"value": ms, "unit": "ms/token", "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": ms, "unit": "ms/token", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           "setup_s": time.perf_counter() - t}
+    print(json.dumps(out), flush=True)
+
+
+def run_mk(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+    import mk_inputs as mi
+    import persistent_megakernel_decode_04_b200 as mk
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600),
+                                device_id=dev)
+    shape = mi.LLAMA8B
+    total_steps = args.warmup + args.steps
+    max_seq = PROMPT_LEN + total_steps + args.e2e_steps + 8
+    os.environ.setdefault("MK_INPUT_THREADS", str(max(1, (os.cpu_count() or 1) // max(1, world))))
+    weights = mi.make_weights(shape, seed=0)
+    stream = torch.cuda.current_stream(dev)
+    m = mk.Megakernel(mk.Config.from_shape(shape, 1, max_seq), weights, local, stream=stream)
+    info = m.info()
+    keep_weights = rank == 0 and not args.no_cpu_baseline
+    if not keep_weights:
+        del weights
+    prompt = torch.from_numpy(mi.prompt(0, 0, PROMPT_LEN, shape.vocab)[None].astype(np.int32)).to(dev)
+    logits = m.prefill(prompt)
+    tok = torch.argmax(logits[0]).to(torch.int32).reshape(1)
+    for _ in range(args.warmup):
+        _, nt = m.decode(tok)
+        tok = nt.clone()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    pos0 = m.positions()[0]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clk:
+        start.record(stream)
+        for a, b in ev:
+            a.record(stream)
+            _, nt = m.decode(tok)
+            b.record(stream)
+            tok = nt  # next step reads this step's greedy token on the device
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    status = m.sync_status()
+    if status != mk.MK_OK:
+        raise SystemExit(f"decode reported status {status}: {mk.mk_last_error(m.ctx)}")
+    elapsed_ms = start.elapsed_time(stop)
+    step_ms = np.array([a.elapsed_time(b) for a, b in ev])
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    max_ms = float(t.item())
+
+    # end to end through the C ABI with host buffers: token in from pinned host memory,
+    # logits and next token back to pinned host memory, every step
+    host_tok = torch.zeros(1, dtype=torch.int32, pin_memory=True)
+    host_logits = torch.empty(shape.vocab, dtype=torch.float32, pin_memory=True)
+    host_next = torch.zeros(1, dtype=torch.int32, pin_memory=True)
+    dev_tok = torch.zeros(1, dtype=torch.int32, device=dev)
+    host_tok[0] = int(tok.item())
+    m.set_positions([pos0 + args.steps])
+    n_e2e = min(args.e2e_steps, max_seq - (pos0 + args.steps) - 1)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        dev_tok.copy_(host_tok, non_blocking=True)
+        lg, nt = m.decode(dev_tok)
+        host_logits.copy_(lg[0], non_blocking=True)
+        host_next.copy_(nt, non_blocking=True)
+        stream.synchronize()
+        host_tok[0] = host_next[0]
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_max = float(te.item())
+    if m.sync_status() != mk.MK_OK:
+        raise SystemExit("decode reported an error in the end-to-end loop")
+
+    if rank == 0:
+        positions = list(range(pos0, pos0 + args.steps))
+        wbytes, kvbytes = algorithmic_bytes(shape, positions)
+        alg = wbytes + float(np.mean(kvbytes))
+        mean_ms = float(step_ms.mean())
+        peak, peak_kind = measured_peaks()
+        achieved = alg / (mean_ms * 1e-3) / 1e9
+        traffic, traffic_note = profiled_traffic(alg)
+        value = max_ms / (args.steps * world)  # whole job: slowest rank's time over all ranks' tokens
+        out = {
+            "metric": METRIC, "value": value, "unit": "ms/token", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded random weights)",
+            "config": {"workload": "llama3-8b-shape decode, batch 1, 39-token prompt, greedy",
+                       "prompt_len": PROMPT_LEN, "decode_positions": [pos0, pos0 + args.steps - 1],
+                       "global_batch": world, "parallelism": "replicas", "weights": "bf16",
+                       "l2": "inputs larger than L2 (15 GB of weights streamed per step)"},
+            "ms_per_token_p50": float(np.median(step_ms)), "tokens_per_s": 1e3 / (max_ms / args.steps) * world,
+            "hbm_gbs": achieved, "hbm_frac_of_measured": achieved / peak, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
+            "bound_ms_at_8tbs": alg / NOMINAL_HBM_GBS / 1e6,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": alg, "traffic_note": traffic_note},
+            "e2e": {"value": e2e_max / max(1, n_e2e), "unit": "ms/token", "h2d_bytes_per_step": 4,
+                    "d2h_bytes_per_step": shape.vocab * 4 + 4, "steps": n_e2e},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+            "kernel": {"n_sms": info["n_sms"], "n_tasks": info["n_tasks"], "smem_bytes": info["smem_bytes"]},
+        }
+        if not args.no_cpu_baseline:
+            ms, cores, n = oracle_ms_per_token(weights, shape)
+            out["cpu_baseline"] = {
+                "value": ms, "unit": "ms/token", "cores": cores, "kind": "oracle",
+                "sample": f"{n} oracle decode steps of the 8B shape truncated to 1 layer (full LM head), "
+                          f"39-position synthetic cache, scaled to 32 layers by weight bytes"}
+        print(json.dumps(out), flush=True)
+    m.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.gpus != world and world == 1 and args.gpus > 1:
+        print(json.dumps({"error": f"--gpus {args.gpus} needs torchrun with {args.gpus} processes"}))
+        sys.exit(2)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_mk(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()
