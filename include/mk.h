@@ -182,6 +182,22 @@ int mk_attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* 
  * then re-zeroed) or finished normally (MK_OK). */
 int mk_attention_status(void* workspace, int BH, int d, int L, void* stream);
 
+/* mk_attention_decode without a workspace argument, for callers that may not allocate device
+ * memory: e.g. a serving process whose own allocator reserved the GPU's memory up front, or a
+ * latency-critical loop where cudaMalloc / cudaFree would block and synchronise the device.
+ * (No counterpart in the pages: an addition for such callers.)  Same operands, layouts,
+ * arithmetic and result as mk_attention_decode; the scratch is a fixed 4 MiB array inside
+ * the library that every GPU loading the library keeps until the process exits.  Sizes whose
+ * scratch (mk_attention_workspace_bytes(BH, d, L)) exceeds 4 MiB are rejected with
+ * MK_ERR_INVALID_ARG and a message.  The first call on a device looks up the array's device
+ * address (once, with that device current); make that first call before any stream capture.
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library routine); it
+ * zeroes the array's arrival counts and error word on `stream` before the kernel.  All calls
+ * share the one array, so calls that overlap on the GPU (other streams, other threads) race:
+ * order them on one stream. */
+int mk_attention_decode_noalloc(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d,
+                                int L, float scale, void* stream);
+
 /* Last error text for ctx (or the thread's last context-free error when ctx is NULL). */
 const char* mk_last_error(const mk_ctx* ctx);
 void mk_destroy(mk_ctx* ctx);

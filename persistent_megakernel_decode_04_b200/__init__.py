@@ -87,6 +87,7 @@ _SIGS = {
     "mk_attention_workspace_bytes": ([_i32, _i32, _i32], _sz),
     "mk_attention_decode": ([_vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.c_float, _vp, _vp], _i32),
     "mk_attention_status": ([_vp, _i32, _i32, _i32, _vp], _i32),
+    "mk_attention_decode_noalloc": ([_vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.c_float, _vp], _i32),
     "mk_last_error": ([_vp], ctypes.c_char_p),
     "mk_destroy": ([_vp], None),
 }
@@ -247,6 +248,13 @@ def mk_attention_workspace_bytes(BH: int, d: int, L: int) -> int:
 def mk_attention_decode(q, k_t, v, o, BH: int, d: int, L: int, scale: float, workspace, stream=None):
     _check(_lib.mk_attention_decode(_ptr(q), _ptr(k_t), _ptr(v), _ptr(o), int(BH), int(d), int(L), float(scale),
                                     _ptr(workspace), _stream(stream)))
+
+
+def mk_attention_decode_noalloc(q, k_t, v, o, BH: int, d: int, L: int, scale: float, stream=None):
+    """Same as mk_attention_decode for callers that may not allocate: the scratch is a fixed
+    4 MiB array inside libmk.so (sizes needing more are rejected)."""
+    _check(_lib.mk_attention_decode_noalloc(_ptr(q), _ptr(k_t), _ptr(v), _ptr(o), int(BH), int(d), int(L),
+                                            float(scale), _stream(stream)))
 
 
 def mk_attention_status(workspace, BH: int, d: int, L: int, stream=None) -> int:

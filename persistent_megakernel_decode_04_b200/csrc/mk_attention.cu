@@ -20,6 +20,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "mk_internal.h"
 #include "mk_ptx.cuh"
 
@@ -410,6 +412,12 @@ size_t attention_workspace_bytes(int BH, int d, int L, int n_sms) {
   return part + (((size_t)BH * sizeof(uint32_t) + 255) & ~(size_t)255) + 256;
 }
 
+size_t attention_counter_offset(int BH, int d, int L, int n_sms) {
+  int nu, U, G, maxc;
+  attn_geometry(BH, d, L, n_sms, &nu, &U, &G, &maxc);
+  return ((size_t)BH * maxc * (d + 2) * sizeof(float) + 255) & ~(size_t)255;
+}
+
 size_t attention_error_word_offset(int BH, int d, int L, int n_sms) {
   return attention_workspace_bytes(BH, d, L, n_sms) - 256;
 }
@@ -489,6 +497,67 @@ int attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, 
     return MK_ERR_CUDA;
   }
   return MK_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant.  Some callers may not call cudaMalloc: a serving process whose own
+// allocator reserved the device memory up front (a library allocation would fail or fragment
+// it), or a latency-critical loop where cudaMalloc/cudaFree would block and synchronise the
+// device.  For them the scratch of the split-KV attention (per-head partials, arrival counts,
+// error word) lives in one fixed array in the library's device image instead of a caller
+// buffer.  Every GPU that loads the library holds the array until the process exits.
+constexpr size_t kNoAllocScratchBytes = 4u << 20;  // 4 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+}  // namespace
+
+size_t attention_noalloc_capacity() { return kNoAllocScratchBytes; }
+
+int attention_decode_noalloc(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d,
+                             int L, float scale, cudaStream_t stream, std::string* err) {
+  int dev = 0, n_sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices ||
+      cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    *err = "no usable CUDA device";
+    return MK_ERR_CUDA;
+  }
+  const size_t need = attention_workspace_bytes(BH, d, L, n_sms);
+  if (need > kNoAllocScratchBytes) {
+    *err = "mk_attention_decode_noalloc: these sizes need " + std::to_string(need) +
+           " bytes of scratch; the fixed array holds " + std::to_string(kNoAllocScratchBytes) +
+           " (use mk_attention_decode with a caller workspace)";
+    return MK_ERR_INVALID_ARG;
+  }
+  void* scratch = nullptr;
+  {
+    // once per device, with that device current: the array's device address (the symbol
+    // itself is only a host-side stand-in)
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess || !p) {
+        *err = std::string("cudaGetSymbolAddress(noalloc scratch): ") + cudaGetErrorString(e);
+        return MK_ERR_CUDA;
+      }
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  if (L % 8 == 0) {
+    // the array keeps the previous call's contents: zero the arrival counts and error word
+    const size_t counters = attention_counter_offset(BH, d, L, n_sms);
+    const cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(scratch) + counters, 0, need - counters, stream);
+    if (e != cudaSuccess) {
+      *err = std::string("clearing the noalloc counters: ") + cudaGetErrorString(e);
+      return MK_ERR_CUDA;
+    }
+  }
+  return attention_decode(q, k_t, v, o, BH, d, L, scale, scratch, stream, n_sms, 2000000000ull, err);
 }
 
 }  // namespace mk

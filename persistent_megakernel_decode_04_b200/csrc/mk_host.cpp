@@ -1020,6 +1020,16 @@ int mk_attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* 
   return MK_OK;
 }
 
+int mk_attention_decode_noalloc(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d,
+                                int L, float scale, void* stream) {
+  if (!q || !k_t || !v || !o) return fail(nullptr, MK_ERR_INVALID_ARG, "NULL operand");
+  if (BH < 1 || L < 1 || (d != 64 && d != 128)) return fail(nullptr, MK_ERR_INVALID_ARG, "bad BH, d or L");
+  std::string err;
+  int rc = attention_decode_noalloc(q, k_t, v, o, BH, d, L, scale, reinterpret_cast<cudaStream_t>(stream), &err);
+  if (rc) return fail(nullptr, rc, err);
+  return MK_OK;
+}
+
 int mk_attention_status(void* workspace, int BH, int d, int L, void* stream) {
   if (!workspace || BH < 1 || L < 1 || (d != 64 && d != 128)) return fail(nullptr, MK_ERR_INVALID_ARG, "bad arguments");
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)

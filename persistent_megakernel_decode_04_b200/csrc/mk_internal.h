@@ -128,6 +128,10 @@ size_t attention_error_word_offset(int BH, int d, int L, int n_sms);
 int attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d, int L,
                      float scale, void* workspace, cudaStream_t stream, int n_sms, uint64_t timeout_ns,
                      std::string* err);
+size_t attention_counter_offset(int BH, int d, int L, int n_sms);
+size_t attention_noalloc_capacity();
+int attention_decode_noalloc(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d,
+                             int L, float scale, cudaStream_t stream, std::string* err);
 
 // Prefill (mk_prefill.cu).
 struct PrefillParams {
