@@ -42,6 +42,11 @@ def parse():
     p.add_argument("--impl", default="mk", choices=["mk", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=64)
+    p.add_argument("--no-calibrate", action="store_true",
+                   help="keep equal rows per SM instead of the schedule calibrated during warm-up")
+    p.add_argument("--layers", type=int, default=0,
+                   help="truncate the decoder to this many layers (profiling captures of a small case); "
+                        "0 = the full 32-layer workload")
     return p.parse_args()
 
 
@@ -231,7 +236,7 @@ def run_mk(args, rank, world, local):
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600),
                                 device_id=dev)
-    shape = mi.LLAMA8B
+    shape = mi.LLAMA8B if args.layers <= 0 else mi.LLAMA8B.with_layers(args.layers)
     total_steps = args.warmup + args.steps
     max_seq = PROMPT_LEN + total_steps + args.e2e_steps + 8
     os.environ.setdefault("MK_INPUT_THREADS", str(max(1, (os.cpu_count() or 1) // max(1, world))))
@@ -245,7 +250,14 @@ def run_mk(args, rank, world, local):
     prompt = torch.from_numpy(mi.prompt(0, 0, PROMPT_LEN, shape.vocab)[None].astype(np.int32)).to(dev)
     logits = m.prefill(prompt)
     tok = torch.argmax(logits[0]).to(torch.int32).reshape(1)
-    for _ in range(args.warmup):
+    warm = args.warmup
+    calibrated = False
+    if not args.no_calibrate and warm >= 6:
+        # measure per-SM streaming speed on warm-up steps and re-partition rows (3 rounds x 2 steps)
+        m.calibrate(tok, steps=2, rounds=3)
+        warm -= 6
+        calibrated = True
+    for _ in range(warm):
         _, nt = m.decode(tok)
         tok = nt.clone()
     if world > 1:
@@ -324,9 +336,11 @@ def run_mk(args, rank, world, local):
             "metric": METRIC, "value": value, "unit": "ms/token", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded random weights)",
-            "config": {"workload": "llama3-8b-shape decode, batch 1, 39-token prompt, greedy",
+            "config": {"workload": "llama3-8b-shape decode, batch 1, 39-token prompt, greedy"
+                                   + ("" if args.layers <= 0 else f" (truncated to {args.layers} layers)"),
                        "prompt_len": PROMPT_LEN, "decode_positions": [pos0, pos0 + args.steps - 1],
                        "global_batch": world, "parallelism": "replicas", "weights": "bf16",
+                       "schedule": "calibrated per-SM rows" if calibrated else "equal rows per SM",
                        "l2": "inputs larger than L2 (15 GB of weights streamed per step)"},
             "ms_per_token_p50": float(np.median(step_ms)), "tokens_per_s": 1e3 / (max_ms / args.steps) * world,
             "hbm_gbs": achieved, "hbm_frac_of_measured": achieved / peak, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
@@ -334,7 +348,7 @@ def run_mk(args, rank, world, local):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": alg, "traffic_note": traffic_note},
-            "e2e": {"value": e2e_max / max(1, n_e2e), "unit": "ms/token", "h2d_bytes_per_step": 4,
+            "e2e": {"value": (e2e_max / n_e2e) if n_e2e > 0 else None, "unit": "ms/token", "h2d_bytes_per_step": 4,
                     "d2h_bytes_per_step": shape.vocab * 4 + 4, "steps": n_e2e},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),

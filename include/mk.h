@@ -129,6 +129,17 @@ int mk_set_wait_timeout_ns(mk_ctx* ctx, uint64_t ns);
  * Nothing faults or traps. */
 int mk_debug_drop_notify(mk_ctx* ctx, int event_id, int on);
 
+/* Calibrated static schedule: re-partition every projection's rows over the SMs in
+ * proportion to weights[s] (relative streaming speed of SM s, n = mk_get_graph_info().n_sms;
+ * equal weights = equal bytes per SM, the default).  On this GPU some SMs stream measurably
+ * slower, and with equal shares every phase waits for them; weights measured from traced
+ * steps (see the binding's Megakernel.calibrate) fix the schedule offline, as the fixed
+ * schedule found ahead of time in "Ada-MK ..." section 2.  The new graph is validated like
+ * the first one; if weights are already loaded it is uploaded at once (after synchronising
+ * `stream`) and the event counters restart.  Returns MK_ERR_UNSUPPORTED if the new graph
+ * does not fit the workspace reserve (the old graph then stays). */
+int mk_set_sm_weights(mk_ctx* ctx, const float* weights, int n, void* stream);
+
 /* Weight prefetch depth: besides the shared-memory ring (6 stages of 32 KB per SM), each
  * SM's producer prefetches the next `stages` weight stages of its queue into L2, so HBM keeps
  * streaming while the ring is full (default 0 = off, which measured fastest on B200; at most 64). */
@@ -146,6 +157,7 @@ int mk_set_trace(mk_ctx* ctx, void* device_buffer);
 typedef struct mk_graph_info {
   int n_sms;         /* workers = resident CTAs of the persistent grid */
   int n_tasks, n_events;
+  int task_capacity; /* tasks the workspace can hold (re-partitioning headroom) */
   int attn_chunks;   /* split-KV chunks per (sequence, KV head) */
   int kernel_variant;/* index of the compiled instantiation chosen for this shape */
   uint64_t weight_bytes_per_step; /* bf16 weights streamed by one decode step */

@@ -61,7 +61,7 @@ class mk_host_weights(ctypes.Structure):
 
 class mk_graph_info(ctypes.Structure):
     _fields_ = [("n_sms", ctypes.c_int), ("n_tasks", ctypes.c_int), ("n_events", ctypes.c_int),
-                ("attn_chunks", ctypes.c_int), ("kernel_variant", ctypes.c_int),
+                ("task_capacity", ctypes.c_int), ("attn_chunks", ctypes.c_int), ("kernel_variant", ctypes.c_int),
                 ("weight_bytes_per_step", ctypes.c_uint64), ("smem_bytes", ctypes.c_uint64)]
 
 
@@ -80,6 +80,7 @@ _SIGS = {
     "mk_set_wait_timeout_ns": ([_vp, _u64], _i32),
     "mk_debug_drop_notify": ([_vp, _i32, _i32], _i32),
     "mk_set_l2_prefetch": ([_vp, _i32], _i32),
+    "mk_set_sm_weights": ([_vp, _vp, _i32, _vp], _i32),
     "mk_set_trace": ([_vp, _vp], _i32),
     "mk_get_graph_info": ([_vp, ctypes.POINTER(mk_graph_info)], _i32),
     "mk_export_taskgraph": ([_vp, _vp, _i32, _vp, _i32], _i32),
@@ -209,6 +210,12 @@ def mk_debug_drop_notify(ctx, event_id: int, on: bool):
     _check(_lib.mk_debug_drop_notify(ctx, int(event_id), int(bool(on))), ctx)
 
 
+def mk_set_sm_weights(ctx, weights, stream=None):
+    import numpy as np
+    w = np.ascontiguousarray(weights, dtype=np.float32)
+    _check(_lib.mk_set_sm_weights(ctx, w.ctypes.data, w.size, _stream(stream)), ctx)
+
+
 def mk_set_l2_prefetch(ctx, stages: int):
     _check(_lib.mk_set_l2_prefetch(ctx, int(stages)), ctx)
 
@@ -334,6 +341,34 @@ class Megakernel:
         B = tokens.shape[0]
         mk_decode_step(self.ctx, tokens, self.kv, self.logits, self.next_tokens, self.stream)
         return self.logits[:B], self.next_tokens[:B]
+
+    def calibrate(self, tokens, steps: int = 2, rounds: int = 3):
+        """Measure each SM's busy time on the projection tasks over `steps` traced decode steps
+        (decoding `tokens`, which advances the positions) and re-partition the rows so that
+        every SM finishes together; `rounds` measure/re-partition passes.  Returns the weights."""
+        import numpy as np
+        import torch
+        info = self.info()
+        n = info["n_sms"]
+        w = np.ones(n)
+        trace = torch.zeros(info["task_capacity"] * 6, dtype=torch.int64, device=tokens.device)
+        for _ in range(rounds):
+            tasks, _ = mk_export_taskgraph(self.ctx)
+            mk_set_trace(self.ctx, trace)
+            busy = np.zeros(n)
+            for _ in range(steps):
+                self.decode(tokens)
+                self.sync_status()
+                T = trace[: tasks.shape[0] * 6].view(-1, 6).cpu().numpy()
+                gemv = np.isin(tasks[:, 0], (2, 4, 5, 6, 7))
+                np.add.at(busy, tasks[gemv, 2], (T[gemv, 2] - T[gemv, 1]).astype(np.float64))
+            mk_set_trace(self.ctx, None)
+            if busy.min() <= 0:
+                break
+            w = w * busy.mean() / busy  # slower SMs (more busy time) get fewer rows
+            w = w / w.mean()
+            mk_set_sm_weights(self.ctx, w, self.stream)
+        return w
 
     def set_positions(self, positions):
         mk_set_positions(self.ctx, positions)

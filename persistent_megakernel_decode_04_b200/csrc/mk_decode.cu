@@ -68,6 +68,7 @@ __device__ __forceinline__ void raise_error(const DecodeParams& P, DSmem& S, uin
 
 // Bounded mbarrier wait (see header comment).  False once the limit passed or a role aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_t limit_ns, DSmem* S) {
+  if (mbar_test_now(bar, parity)) return true;  // common case: already complete
   uint64_t t0 = 0;
   for (uint32_t n = 1;; ++n) {
     if (mbar_test(bar, parity)) return true;
@@ -91,16 +92,13 @@ struct Pipe {
   }
 };
 
-__device__ __forceinline__ float dot8(const uint4 w, const float* x, float acc) {
-  acc = fmaf(bf16lo(w.x), x[0], acc);
-  acc = fmaf(bf16hi(w.x), x[1], acc);
-  acc = fmaf(bf16lo(w.y), x[2], acc);
-  acc = fmaf(bf16hi(w.y), x[3], acc);
-  acc = fmaf(bf16lo(w.z), x[4], acc);
-  acc = fmaf(bf16hi(w.z), x[5], acc);
-  acc = fmaf(bf16lo(w.w), x[6], acc);
-  acc = fmaf(bf16hi(w.w), x[7], acc);
-  return acc;
+// acc (even/odd partial sums packed in one register pair) += the 8 bf16 weights of w times
+// the packed x pairs: each 32-bit word holds weights (2j, 2j+1) and meets x pair j.
+__device__ __forceinline__ void dot8(const uint4 w, const uint64_t* x2, uint64_t& acc) {
+  fma2_bf16w(acc, w.x, x2[0]);
+  fma2_bf16w(acc, w.y, x2[1]);
+  fma2_bf16w(acc, w.z, x2[2]);
+  fma2_bf16w(acc, w.w, x2[3]);
 }
 
 __device__ __forceinline__ uint16_t f2bf(float f) {
@@ -193,6 +191,11 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
       for (int i = 0; i < 8; ++i) x[s][i] = 0.f;
     }
   }
+  uint64_t x2[NSEG][4];
+#pragma unroll
+  for (int s = 0; s < NSEG; ++s)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) x2[s][j] = pack2(x[s][2 * j], x[s][2 * j + 1]);
   float* red = S.red[warp];
   bool ok = true;
   for (int r0 = 0; r0 < nrows; r0 += RPS) {
@@ -204,18 +207,16 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
     }
     if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
     const uint8_t* base = S.ring[pp.stage] + tid * 16;
-    float a[RPS], b[RPS];  // two partial sums per row: shorter dependency chains
+    uint64_t acc[RPS];  // per row: (even, odd) partial sums
 #pragma unroll
     for (int rr = 0; rr < RPS; ++rr) {
-      a[rr] = 0.f;
-      b[rr] = 0.f;
+      acc[rr] = 0ull;
       if (RPS == 1 || r0 + rr < nrows) {
 #pragma unroll
         for (int s = 0; s < NSEG; ++s) {
           if (s < NSEG - 1 || last_ok) {
             const uint4 w = *reinterpret_cast<const uint4*>(base + rr * row_bytes + s * kSegBytes);
-            if (s & 1) b[rr] = dot8(w, x[s], b[rr]);
-            else a[rr] = dot8(w, x[s], a[rr]);
+            dot8(w, x2[s], acc[rr]);
           }
         }
       }
@@ -223,8 +224,12 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
     pp.advance();
+    float a[RPS];
 #pragma unroll
-    for (int rr = 0; rr < RPS; ++rr) a[rr] += b[rr];
+    for (int rr = 0; rr < RPS; ++rr) {
+      const float2 v = unpack2(acc[rr]);
+      a[rr] = v.x + v.y;
+    }
     warp_reduce_rows<RPS>(a, red + r0, lane, nrows - r0);
   }
 #pragma unroll
@@ -299,21 +304,87 @@ __device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, c
 // the other chunk tasks only count their arrival.  The last task of the (sequence, KV head)
 // to arrive merges the partials into o (FlashDecoding-style online-softmax merge) and
 // notifies; with a single chunk in use that chunk writes o directly and nothing is merged.
+//
+// Latency: keys before the current position were written by earlier steps, so each warp
+// loads its first block of kAttnBlock keys (raw bf16 words in registers) before the task's
+// inputs are released (attn_preload); after the release only q and the key/value at the
+// current position are fetched.  Each lane holds DL = D/32 dims of every head; the KB x 4
+// (key, head) partial dot products of a block are summed across lanes with one transposed
+// butterfly (each exchange halves the live values) and broadcast back with shuffles.
+constexpr int kAttnBlock = 8;  // keys per warp per block
+
+struct AttnGeom {
+  int b, g, c, Lk, nch_eff, j0, j1;
+};
+
+__device__ __forceinline__ AttnGeom attn_geom(const DecodeParams& P, const Task& t) {
+  AttnGeom a;
+  a.b = (int)t.row0 / P.nkv;
+  a.g = (int)t.row0 % P.nkv;
+  a.c = t.aux;
+  a.Lk = P.pos[a.b] + 1;
+  a.nch_eff = max(1, min(P.nch, (a.Lk + kMinChunkKeys - 1) / kMinChunkKeys));
+  const int cl = (a.Lk + a.nch_eff - 1) / a.nch_eff;
+  a.j0 = a.c * cl;
+  a.j1 = (a.c < a.nch_eff) ? min(a.Lk, a.j0 + cl) : a.j0;
+  return a;
+}
+
 template <int D>
-__device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, const Task& t, uint32_t task_id) {
-  constexpr int DL = D / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = P.nq / P.nkv;
-  const int b = (int)t.row0 / P.nkv, g = (int)t.row0 % P.nkv;
-  const int c = t.aux;
-  const int Lk = P.pos[b] + 1;
-  const int nch_eff = max(1, min(P.nch, (Lk + kMinChunkKeys - 1) / kMinChunkKeys));
-  const int cl = (Lk + nch_eff - 1) / nch_eff;
-  const int j0 = c * cl, j1 = min(Lk, j0 + cl);
+struct AttnRegs {
+  static constexpr int W = D / 64;  // 32-bit words of K (or V) per lane per key: 2 (D=128) or 1
+  uint32_t k[kAttnBlock][W], v[kAttnBlock][W];
+};
+
+template <int D>
+__device__ __forceinline__ const uint16_t* attn_cache(const DecodeParams& P, const Task& t, const AttnGeom& a,
+                                                       int kind) {
   const size_t head_stride = (size_t)P.max_seq * D;
   const size_t kv_layer = (size_t)P.max_batch * P.nkv * head_stride;
-  const uint16_t* kc = P.kv + ((size_t)t.layer * 2 + 0) * kv_layer + ((size_t)b * P.nkv + g) * head_stride;
-  const uint16_t* vc = P.kv + ((size_t)t.layer * 2 + 1) * kv_layer + ((size_t)b * P.nkv + g) * head_stride;
+  return P.kv + ((size_t)t.layer * 2 + kind) * kv_layer + ((size_t)a.b * P.nkv + a.g) * head_stride;
+}
+
+template <int D>
+__device__ __forceinline__ void attn_load_key(const uint16_t* kc, const uint16_t* vc, int j, int lane,
+                                              uint32_t (&kw)[D / 64], uint32_t (&vw)[D / 64]) {
+  if (D == 128) {
+    const uint2 a = __ldcg(reinterpret_cast<const uint2*>(kc + (size_t)j * D + lane * 4));
+    const uint2 b = __ldcg(reinterpret_cast<const uint2*>(vc + (size_t)j * D + lane * 4));
+    kw[0] = a.x; kw[(D / 64) - 1] = a.y;
+    vw[0] = b.x; vw[(D / 64) - 1] = b.y;
+  } else {
+    kw[0] = __ldcg(reinterpret_cast<const unsigned int*>(kc + (size_t)j * D + lane * 2));
+    vw[0] = __ldcg(reinterpret_cast<const unsigned int*>(vc + (size_t)j * D + lane * 2));
+  }
+}
+
+// Before the release: this warp's first block of keys, positions < pos only.
+template <int D>
+__device__ __forceinline__ void attn_preload(const DecodeParams& P, const Task& t, AttnRegs<D>& R) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const AttnGeom a = attn_geom(P, t);
+  if (warp >= kAttnWarps) return;
+  const uint16_t* kc = attn_cache<D>(P, t, a, 0);
+  const uint16_t* vc = attn_cache<D>(P, t, a, 1);
+  const int pos = a.Lk - 1;
+#pragma unroll
+  for (int u = 0; u < kAttnBlock; ++u) {
+    const int j = a.j0 + warp + u * kAttnWarps;
+    if (j < a.j1 && j < pos) attn_load_key<D>(kc, vc, j, lane, R.k[u], R.v[u]);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, const Task& t, AttnRegs<D>& R,
+                                               uint32_t task_id) {
+  constexpr int DL = D / 32;
+  constexpr int W = D / 64;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = P.nq / P.nkv;
+  const AttnGeom a = attn_geom(P, t);
+  const int g = a.g, b = a.b, c = a.c, nch_eff = a.nch_eff, pos = a.Lk - 1;
+  const uint16_t* kc = attn_cache<D>(P, t, a, 0);
+  const uint16_t* vc = attn_cache<D>(P, t, a, 1);
   const float* qsrc = P.qbuf + ((size_t)t.layer * P.B + b) * P.nq * D + (size_t)g * G * D;
   // partial of (head h, chunk cc) of this sequence at part_base + (h * nch + cc) * (D + 2)
   float* part_base = P.part + ((size_t)t.layer * P.B + b) * P.nq * (size_t)P.nch * (D + 2);
@@ -321,6 +392,12 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
 
   if (c < nch_eff) {  // uniform across the CTA
     float qv[4][DL], m[4], l[4], acc[4][DL];
+    // the key/value at the current position were written in this step: load them now
+#pragma unroll
+    for (int u = 0; u < kAttnBlock; ++u) {
+      const int j = a.j0 + warp + u * kAttnWarps;
+      if (warp < kAttnWarps && j == pos) attn_load_key<D>(kc, vc, j, lane, R.k[u], R.v[u]);
+    }
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       m[h] = -INFINITY;
@@ -331,41 +408,72 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
         acc[h][i] = 0.f;
       }
     }
-    for (int j = j0 + warp; warp < kAttnWarps && j < j1; j += kAttnWarps) {
-      float kf[DL], vf[DL];
-      if (DL == 4) {
-        const uint2 kw = __ldcg(reinterpret_cast<const uint2*>(kc + (size_t)j * D + lane * 4));
-        const uint2 vw = __ldcg(reinterpret_cast<const uint2*>(vc + (size_t)j * D + lane * 4));
-        kf[0] = bf16lo(kw.x); kf[1] = bf16hi(kw.x); kf[2 % DL] = bf16lo(kw.y); kf[3 % DL] = bf16hi(kw.y);
-        vf[0] = bf16lo(vw.x); vf[1] = bf16hi(vw.x); vf[2 % DL] = bf16lo(vw.y); vf[3 % DL] = bf16hi(vw.y);
-      } else {
-        const uint32_t kw = __ldcg(reinterpret_cast<const unsigned int*>(kc + (size_t)j * D + lane * 2));
-        const uint32_t vw = __ldcg(reinterpret_cast<const unsigned int*>(vc + (size_t)j * D + lane * 2));
-        kf[0] = bf16lo(kw); kf[1 % DL] = bf16hi(kw);
-        vf[0] = bf16lo(vw); vf[1 % DL] = bf16hi(vw);
+    for (int jb = a.j0 + warp; warp < kAttnWarps && jb < a.j1; jb += kAttnBlock * kAttnWarps) {
+      if (jb != a.j0 + warp) {  // later blocks (long chunks): load them now
+#pragma unroll
+        for (int u = 0; u < kAttnBlock; ++u) {
+          const int j = jb + u * kAttnWarps;
+          if (j < a.j1) attn_load_key<D>(kc, vc, j, lane, R.k[u], R.v[u]);
+        }
       }
-      float sc[4];
+      // partial dots of the block: slot u * 4 + h
+      float sc[kAttnBlock * 4];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        float a = 0.f;
+      for (int u = 0; u < kAttnBlock; ++u) {
+        float kf[DL];
 #pragma unroll
-        for (int i = 0; i < DL; ++i) a = fmaf(qv[h][i], kf[i], a);
-        sc[h] = a;
+        for (int w = 0; w < W; ++w) {
+          kf[2 * w] = bf16lo(R.k[u][w]);
+          kf[2 * w + 1] = bf16hi(R.k[u][w]);
+        }
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          float s = 0.f;
+#pragma unroll
+          for (int i = 0; i < DL; ++i) s = fmaf(qv[h][i], kf[i], s);
+          sc[u * 4 + h] = s;
+        }
       }
+      // transposed butterfly: lane l ends with the warp's sum of slot l ...
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1)
+      for (int off = 16; off >= 1; off >>= 1) {
+        const bool upper = (lane & off) != 0;
 #pragma unroll
-        for (int h = 0; h < 4; ++h) sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], off);
+        for (int i = 0; i < off; ++i) {
+          const float send = upper ? sc[i] : sc[i + off];
+          const float keep = upper ? sc[i + off] : sc[i];
+          sc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      const float mine = sc[0];
+      // ... and every lane gets every slot back
+#pragma unroll
+      for (int i = 0; i < kAttnBlock * 4; ++i) sc[i] = __shfl_sync(0xffffffffu, mine, i);
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         if (h < G) {
-          const float mn = fmaxf(m[h], sc[h]);
-          const float a = expf(m[h] - mn);
-          const float p = expf(sc[h] - mn);
-          l[h] = l[h] * a + p;
+          float mx = m[h];
 #pragma unroll
-          for (int i = 0; i < DL; ++i) acc[h][i] = fmaf(acc[h][i], a, p * vf[i]);
-          m[h] = mn;
+          for (int u = 0; u < kAttnBlock; ++u)
+            if (jb + u * kAttnWarps < a.j1) mx = fmaxf(mx, sc[u * 4 + h]);
+          const float alpha = expf(m[h] - mx);  // 0 on the first block (m = -inf)
+          float ls = 0.f;
+#pragma unroll
+          for (int i = 0; i < DL; ++i) acc[h][i] *= alpha;
+#pragma unroll
+          for (int u = 0; u < kAttnBlock; ++u) {
+            if (jb + u * kAttnWarps < a.j1) {
+              const float p = expf(sc[u * 4 + h] - mx);
+              ls += p;
+#pragma unroll
+              for (int w = 0; w < W; ++w) {
+                acc[h][2 * w] = fmaf(p, bf16lo(R.v[u][w]), acc[h][2 * w]);
+                acc[h][2 * w + 1] = fmaf(p, bf16hi(R.v[u][w]), acc[h][2 * w + 1]);
+              }
+            }
+          }
+          l[h] = l[h] * alpha + ls;
+          m[h] = mx;
         }
       }
     }
@@ -424,6 +532,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       S.ll[e] = __ldcg(pc + 1);
     }
     worker_bar();
+    // merge weights w_c = exp(m_c - M) per (head, chunk)
     for (int e = tid; e < G * nch_eff; e += kWorkerThreads) {
       const int h = e / nch_eff;
       float M = -INFINITY;
@@ -431,15 +540,24 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       S.ww[e] = (S.mm[e] == -INFINITY) ? 0.f : expf(S.mm[e] - M);
     }
     worker_bar();
+    // o[h][d] = sum_c w_c acc_c[d] / sum_c w_c l_c: all loads of a block of 16 chunks are
+    // issued before any is used (one L2 round trip per 16 chunks)
     for (int e = tid; e < G * D; e += kWorkerThreads) {
       const int h = e / D, d = e % D;
       const float* ph = part_base + (size_t)(g * G + h) * P.nch * (D + 2) + 2 + d;
       float num = 0.f, den = 0.f;
-#pragma unroll 8
-      for (int cc = 0; cc < nch_eff; ++cc) {
-        const float w = S.ww[h * nch_eff + cc];
-        num = fmaf(w, __ldcg(ph + (size_t)cc * (D + 2)), num);
-        den = fmaf(w, S.ll[h * nch_eff + cc], den);
+      for (int c0 = 0; c0 < nch_eff; c0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = (c0 + k < nch_eff) ? __ldcg(ph + (size_t)(c0 + k) * (D + 2)) : 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          if (c0 + k < nch_eff) {
+            const float w = S.ww[h * nch_eff + c0 + k];
+            num = fmaf(w, v[k], num);
+            den = fmaf(w, S.ll[h * nch_eff + c0 + k], den);
+          }
+        }
       }
       o[(size_t)h * D + d] = num / den;
     }
@@ -501,7 +619,7 @@ __device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, cons
 }
 
 // ---------------------------------------------------------------------------------------
-template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F>
+template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD>
 __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   DSmem& S = *reinterpret_cast<DSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -525,29 +643,33 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     // ------------------------------- producer -------------------------------
     if (lane != 0) return;
     const uint64_t pol = policy_evict_first();
-    // L2 lookahead: a second cursor over this queue's weight stages runs l2_ahead stages in
-    // front of the ring cursor and prefetches them into L2, so HBM keeps streaming while the
-    // ring is full (e.g. while the workers wait for a dependency).
+    // L2 lookahead for dependency stalls: a second cursor over this queue's weight stages.
+    // While the ring is full and the producer has been blocked for over kStallPrefetchNs (the
+    // workers wait for a dependency, so HBM would idle), it prefetches up to l2_ahead stages
+    // beyond the ring into L2; a stage it prefetched later loads from L2.  In steady
+    // streaming (short blocks) it prefetches nothing, so it never competes with the ring.
     uint32_t la_task = qb, la_row = 0;
-    int la_lead = 0;  // stages the lookahead cursor is ahead of the ring cursor
-    auto la_step = [&]() {  // prefetch the stage under the lookahead cursor and advance it
+    int la_lead = 0;  // stages the lookahead cursor is in front of the next ring stage
+    Task la_t = P.tasks[qb < qe ? qb : 0];  // descriptor under the cursor, cached in registers
+    auto la_advance = [&](bool prefetch) {  // move the lookahead cursor one stage on
       while (la_task < qe) {
-        const Task lt = P.tasks[la_task];
-        if (!is_gemv(lt.kind) || la_row >= lt.nrows) {
-          ++la_task;
+        if (!is_gemv(la_t.kind) || la_row >= la_t.nrows) {
+          if (++la_task < qe) la_t = P.tasks[la_task];
           la_row = 0;
           continue;
         }
-        uint64_t off;
-        uint32_t rb;
-        gemv_source(P, lt, &off, &rb);
-        const uint32_t rps = (lt.kind == TK_DOWN) ? (uint32_t)RPS_F : (uint32_t)RPS_H;
-        const uint32_t nr = min(rps, lt.nrows - la_row);
-        prefetch_l2(P.arena + off + (uint64_t)(lt.row0 + la_row) * rb, nr * rb);
+        const uint32_t rps = (la_t.kind == TK_DOWN) ? (uint32_t)RPS_F : (uint32_t)RPS_H;
+        if (prefetch) {
+          uint64_t off;
+          uint32_t rb;
+          gemv_source(P, la_t, &off, &rb);
+          const uint32_t nr = min(rps, la_t.nrows - la_row);
+          prefetch_l2(P.arena + off + (uint64_t)(la_t.row0 + la_row) * rb, nr * rb);
+        }
         la_row += rps;
-        ++la_lead;
-        return;
+        return true;
       }
+      return false;
     };
     Pipe pp{0, 0};
     int issued = 0;
@@ -563,9 +685,20 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
       uint64_t blocked = 0, first = 0;
       for (uint32_t r0 = 0; r0 < t.nrows; r0 += (uint32_t)rps) {
         const uint32_t nr = min((uint32_t)rps, t.nrows - r0);
-        // keep the lookahead l2_ahead stages in front of the stage about to enter the ring
-        while (la_lead < P.l2_ahead && la_task < qe) la_step();
-        const uint64_t tw = P.trace ? globaltimer_ns() : 0;
+        const uint64_t tw = (P.trace || P.l2_ahead > 0) ? globaltimer_ns() : 0;
+        if (P.l2_ahead > 0 && !mbar_test_now(&S.empty[pp.stage], pp.phase ^ 1u)) {
+          // blocked: after kStallPrefetchNs, prefetch while still blocked
+          uint64_t t0 = tw;
+          for (uint32_t n = 1;; ++n) {
+            if (mbar_test(&S.empty[pp.stage], pp.phase ^ 1u)) break;
+            const uint64_t now = globaltimer_ns();
+            if (now - t0 > kStallPrefetchNs && la_lead < P.l2_ahead && la_advance(true)) {
+              ++la_lead;
+              t0 = now - kStallPrefetchNs + kStallPrefetchGapNs;  // next prefetch after a short gap
+            }
+            if ((n & 127u) == 0 && (S.abort || now - tw > P.timeout_ns)) break;
+          }
+        }
         if (!wait_bar(&S.empty[pp.stage], pp.phase ^ 1u, P.timeout_ns, &S)) {
           if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, i);
           ok = false;
@@ -579,7 +712,11 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
         mbar_arrive_expect_tx(&S.full[pp.stage], nr * rb);
         bulk_g2s(S.ring[pp.stage], src + (uint64_t)r0 * rb, nr * rb, &S.full[pp.stage], pol);
         ++issued;
-        if (P.l2_ahead > 0) --la_lead;  // this stage was prefetched while it was ahead
+        // the lookahead cursor stays at or in front of the next ring stage
+        if (P.l2_ahead > 0) {
+          if (la_lead > 0) --la_lead;
+          else la_advance(false);
+        }
         pp.advance();
       }
       if (P.trace) {
@@ -605,6 +742,20 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     if (lane != 0) return;
     for (uint32_t i = qb; i < qe; ++i) {
       const Task t = P.tasks[i];
+      if (t.kind == TK_ATTN) {
+        // positions before pos were written by earlier steps: start their journey from HBM
+        // now, while this task still waits for the QKV tiles of its head group
+        const AttnGeom a = attn_geom(P, t);
+        const int j1 = min(a.j1, a.Lk - 1);  // old positions only
+        if (a.c < a.nch_eff && j1 > a.j0) {
+          const size_t head_stride = (size_t)P.max_seq * P.D;
+          const size_t kv_layer = (size_t)P.max_batch * P.nkv * head_stride;
+          const size_t off = ((size_t)a.b * P.nkv + a.g) * head_stride + (size_t)a.j0 * P.D;
+          const uint32_t bytes = (uint32_t)(j1 - a.j0) * (uint32_t)P.D * 2u;
+          prefetch_l2(P.kv + ((size_t)t.layer * 2 + 0) * kv_layer + off, bytes);
+          prefetch_l2(P.kv + ((size_t)t.layer * 2 + 1) * kv_layer + off, bytes);
+        }
+      }
       for (int w = 0; w < t.n_wait; ++w) {
         const uint32_t e = t.wait[w];
         const uint32_t target = P.epoch * P.ev_count[e];
@@ -632,7 +783,16 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
 
   // --------------------------------- workers ---------------------------------
   Pipe pp{0, 0};
+  // descriptor (and layer offsets) of the next task are loaded while the worker still waits
+  // for that task's inputs, so only the activation loads remain after the release
+  Task t_next = P.tasks[qb < qe ? qb : 0];
   for (uint32_t i = qb; i < qe; ++i) {
+    const Task t = t_next;
+    const LayerOff lo = P.loff[t.layer < P.L ? t.layer : 0];
+    if (i + 1 < qe) t_next = P.tasks[i + 1];
+    // attention: keys of earlier steps can be loaded before this step's q, k, v exist
+    AttnRegs<HD> ar;
+    if (t.kind == TK_ATTN) attn_preload<HD>(P, t, ar);
     const uint64_t t_wait = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     uint32_t stall = 0;
     // wait for the scheduler to release task i (bounded, abort-aware, then uniform decision)
@@ -658,81 +818,76 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
       if (S.cabort) break;
     }
     const uint64_t t_ready = (P.trace && tid == 0) ? globaltimer_ns() : 0;
-    const Task t = P.tasks[i];
     bool notify = true;
-    switch (t.kind) {
-      case TK_EMBED: {
-        const int b = 0;
-        int tok = __ldcg(P.tokens + b);
-        if (tok < 0 || tok >= P.V) {  // never read outside the table: record and use row 0
-          if (tid == 0 && t.row0 == 0) atomicCAS(&P.err[ERR_CODE], 0u, (uint32_t)DEV_ERR_BAD_TOKEN);
-          tok = 0;
-        }
-        const uint16_t* e = reinterpret_cast<const uint16_t*>(P.arena + P.off_embed) + (size_t)tok * P.H;
-        for (uint32_t r = tid; r < t.nrows; r += kWorkerThreads)
-          P.x_in[(size_t)b * P.H + t.row0 + r] = __uint_as_float((uint32_t)e[t.row0 + r] << 16);
-        break;
+    if (is_gemv(t.kind)) {
+      // operands of the task's GEMV: x source, norm gain (null = no norm) and K
+      const float* xs;
+      const uint16_t* gain = nullptr;
+      int K = P.H;
+      const size_t lay = (size_t)t.layer * P.B;
+      switch (t.kind) {
+        case TK_QKV:
+          xs = P.x_in + lay * P.H;
+          gain = reinterpret_cast<const uint16_t*>(P.arena + lo.attn_norm);
+          break;
+        case TK_OPROJ: xs = P.obuf + lay * P.nq * P.D; break;
+        case TK_GATEUP:
+          xs = P.x_mid + lay * P.H;
+          gain = reinterpret_cast<const uint16_t*>(P.arena + lo.mlp_norm);
+          break;
+        case TK_DOWN:
+          xs = P.hbuf + lay * P.F;
+          K = P.F;
+          break;
+        default:  // LM head
+          xs = P.x_in + (size_t)P.L * P.B * P.H;
+          gain = reinterpret_cast<const uint16_t*>(P.arena + P.off_fnorm);
+          break;
       }
-      case TK_QKV: {
-        const LayerOff& lo = P.loff[t.layer];
-        const float* xs = P.x_in + (size_t)t.layer * P.B * P.H;
-        if (!gemv_tile<NSEG_H, RPS_H>(P, S, pp, xs, reinterpret_cast<const uint16_t*>(P.arena + lo.attn_norm), P.H,
-                                      (int)t.nrows, (uint32_t)P.H * 2u, i, stall))
-          goto out;
-        epi_qkv(P, S, t, norm_factor(S, P.H, P.eps));
-        break;
+      const bool ok = (t.kind == TK_DOWN)
+                          ? gemv_tile<NSEG_F, RPS_F>(P, S, pp, xs, gain, K, (int)t.nrows, (uint32_t)K * 2u, i, stall)
+                          : gemv_tile<NSEG_H, RPS_H>(P, S, pp, xs, gain, K, (int)t.nrows, (uint32_t)K * 2u, i, stall);
+      if (!ok) goto out;
+      const float r = gain ? norm_factor(S, K, P.eps) : 1.f;
+      switch (t.kind) {
+        case TK_QKV: epi_qkv(P, S, t, r); break;
+        case TK_OPROJ:
+          if (tid < (int)t.nrows) {
+            const size_t row = (size_t)t.row0 + tid;
+            P.x_mid[lay * P.H + row] = __ldcg(P.x_in + lay * P.H + row) + S.tot[tid];
+          }
+          break;
+        case TK_GATEUP:
+          if (tid < (int)t.nrows && (tid & 1) == 0) {
+            const float gv = S.tot[tid] * r, uv = S.tot[tid + 1] * r;
+            const float sg = gv / (1.f + expf(-gv));
+            P.hbuf[lay * P.F + (t.row0 + tid) / 2] = sg * uv;
+          }
+          break;
+        case TK_DOWN:
+          if (tid < (int)t.nrows) {
+            const size_t row = (size_t)t.row0 + tid;
+            P.x_in[(lay + P.B) * P.H + row] = __ldcg(P.x_mid + lay * P.H + row) + S.tot[tid];
+          }
+          break;
+        default:
+          notify = false;
+          epi_lmhead(P, S, t, r);
+          break;
       }
-      case TK_ATTN: {
-        notify = false;  // the merging chunk notifies
-        if (P.D == 128) attention_task<128>(P, S, t, i);
-        else attention_task<64>(P, S, t, i);
-        break;
+    } else if (t.kind == TK_EMBED) {
+      const int b = 0;
+      int tok = __ldcg(P.tokens + b);
+      if (tok < 0 || tok >= P.V) {  // never read outside the table: record and use row 0
+        if (tid == 0 && t.row0 == 0) atomicCAS(&P.err[ERR_CODE], 0u, (uint32_t)DEV_ERR_BAD_TOKEN);
+        tok = 0;
       }
-      case TK_OPROJ: {
-        const float* os = P.obuf + (size_t)t.layer * P.B * P.nq * P.D;
-        if (!gemv_tile<NSEG_H, RPS_H>(P, S, pp, os, nullptr, P.H, (int)t.nrows, (uint32_t)P.H * 2u, i, stall)) goto out;
-        if (tid < (int)t.nrows) {
-          const size_t r = (size_t)t.row0 + tid;
-          const float* xi = P.x_in + (size_t)t.layer * P.B * P.H;
-          P.x_mid[(size_t)t.layer * P.B * P.H + r] = __ldcg(xi + r) + S.tot[tid];
-        }
-        break;
-      }
-      case TK_GATEUP: {
-        const LayerOff& lo = P.loff[t.layer];
-        const float* xs = P.x_mid + (size_t)t.layer * P.B * P.H;
-        if (!gemv_tile<NSEG_H, RPS_H>(P, S, pp, xs, reinterpret_cast<const uint16_t*>(P.arena + lo.mlp_norm), P.H,
-                                      (int)t.nrows, (uint32_t)P.H * 2u, i, stall))
-          goto out;
-        const float r = norm_factor(S, P.H, P.eps);
-        if (tid < (int)t.nrows && (tid & 1) == 0) {
-          const float gv = S.tot[tid] * r, uv = S.tot[tid + 1] * r;
-          const float sg = gv / (1.f + expf(-gv));
-          P.hbuf[(size_t)t.layer * P.B * P.F + (t.row0 + tid) / 2] = sg * uv;
-        }
-        break;
-      }
-      case TK_DOWN: {
-        const float* hs = P.hbuf + (size_t)t.layer * P.B * P.F;
-        if (!gemv_tile<NSEG_F, RPS_F>(P, S, pp, hs, nullptr, P.F, (int)t.nrows, (uint32_t)P.F * 2u, i, stall)) goto out;
-        if (tid < (int)t.nrows) {
-          const size_t r = (size_t)t.row0 + tid;
-          const float* xm = P.x_mid + (size_t)t.layer * P.B * P.H;
-          P.x_in[(size_t)(t.layer + 1) * P.B * P.H + r] = __ldcg(xm + r) + S.tot[tid];
-        }
-        break;
-      }
-      case TK_LMHEAD: {
-        notify = false;
-        const float* xs = P.x_in + (size_t)P.L * P.B * P.H;
-        if (!gemv_tile<NSEG_H, RPS_H>(P, S, pp, xs, reinterpret_cast<const uint16_t*>(P.arena + P.off_fnorm), P.H,
-                                      (int)t.nrows, (uint32_t)P.H * 2u, i, stall))
-          goto out;
-        epi_lmhead(P, S, t, norm_factor(S, P.H, P.eps));
-        break;
-      }
-      default:
-        break;
+      const uint16_t* e = reinterpret_cast<const uint16_t*>(P.arena + P.off_embed) + (size_t)tok * P.H;
+      for (uint32_t r = tid; r < t.nrows; r += kWorkerThreads)
+        P.x_in[(size_t)b * P.H + t.row0 + r] = __uint_as_float((uint32_t)e[t.row0 + r] << 16);
+    } else if (t.kind == TK_ATTN) {
+      notify = false;  // the last chunk to arrive notifies
+      attention_task<HD>(P, S, t, ar, i);
     }
     if (P.trace && tid == 0) {
       uint64_t* rec = P.trace + (size_t)i * kTraceWords;
@@ -762,25 +917,25 @@ __host__ __device__ constexpr int pow2_floor_c(int x) { return x < 2 ? 1 : 2 * p
 __host__ __device__ constexpr int stage_rows(int K) {
   return pow2_floor_c((kSlotBytes / (2 * K)) < kRpsMax ? (kSlotBytes / (2 * K)) : kRpsMax);
 }
-#define MK_VARIANT(H, F) {seg_count(H), stage_rows(H), seg_count(F), stage_rows(F), 1}
-#define MK_KERNEL(H, F) (const void*)decode_kernel<seg_count(H), stage_rows(H), seg_count(F), stage_rows(F)>
+#define MK_VARIANT(H, F, D) {seg_count(H), stage_rows(H), seg_count(F), stage_rows(F), D}
+#define MK_KERNEL(H, F, D) (const void*)decode_kernel<seg_count(H), stage_rows(H), seg_count(F), stage_rows(F), D>
 static const Variant kVariants[] = {
-    MK_VARIANT(4096, 14336),  // Llama-3-8B shape
-    MK_VARIANT(4096, 11008),  // Chameleon-7B shape
-    MK_VARIANT(256, 768),     // tiny decoder
-    MK_VARIANT(4096, 4096),
-    MK_VARIANT(2048, 4096),
-    MK_VARIANT(256, 256),
+    MK_VARIANT(4096, 14336, 128),  // Llama-3-8B shape
+    MK_VARIANT(4096, 11008, 128),  // Chameleon-7B shape
+    MK_VARIANT(256, 768, 64),      // tiny decoder
+    MK_VARIANT(4096, 4096, 128),
+    MK_VARIANT(2048, 4096, 128),
+    MK_VARIANT(256, 256, 64),
 };
 static const void* kFns[] = {
-    MK_KERNEL(4096, 14336), MK_KERNEL(4096, 11008), MK_KERNEL(256, 768),
-    MK_KERNEL(4096, 4096),  MK_KERNEL(2048, 4096),  MK_KERNEL(256, 256),
+    MK_KERNEL(4096, 14336, 128), MK_KERNEL(4096, 11008, 128), MK_KERNEL(256, 768, 64),
+    MK_KERNEL(4096, 4096, 128),  MK_KERNEL(2048, 4096, 128),  MK_KERNEL(256, 256, 64),
 };
 
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int batch) {
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim) {
   for (int i = 0; i < (int)(sizeof(kVariants) / sizeof(kVariants[0])); ++i) {
     const Variant& v = kVariants[i];
-    if (v.nseg_h == nseg_h && v.rps_h == rps_h && v.nseg_f == nseg_f && v.rps_f == rps_f && v.batch == batch)
+    if (v.nseg_h == nseg_h && v.rps_h == rps_h && v.nseg_f == nseg_f && v.rps_f == rps_f && v.head_dim == head_dim)
       return i;
   }
   return -1;

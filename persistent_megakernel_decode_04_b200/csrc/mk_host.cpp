@@ -73,6 +73,8 @@ struct mk_ctx {
   int drop_event = -1;
   uint64_t* trace = nullptr;
   int l2_ahead = 0;
+  std::vector<double> sm_weights;  // relative streaming speed per SM (partition weights)
+  size_t task_cap = 0, lm_cap = 0; // workspace capacity for re-partitioned graphs
   std::string err;
 };
 
@@ -100,13 +102,21 @@ int ev_o(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads + 1;
 int ev_gu(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads + 2; }
 int ev_down(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads + 3; }
 
-// Split `total` rows over n_sms SMs in contiguous, balanced ranges (multiples of gran), and
-// each range into tasks of at most kTaskRows rows.
-std::vector<std::vector<std::pair<int, int>>> partition_rows(int total, int gran, int n_sms) {
+// Split `total` rows over the SMs in contiguous ranges (multiples of gran) proportional to
+// the per-SM weights (equal weights: balanced), and each range into tasks of at most
+// kTaskRows rows.
+std::vector<std::vector<std::pair<int, int>>> partition_rows(int total, int gran, const std::vector<double>& w) {
+  const int n_sms = (int)w.size();
   std::vector<std::vector<std::pair<int, int>>> out(n_sms);
+  std::vector<double> cum(n_sms + 1, 0.0);
+  for (int s = 0; s < n_sms; ++s) cum[s + 1] = cum[s] + w[s];
+  auto bound = [&](int s) -> int {
+    if (s == n_sms) return total;
+    return (int)((long long)std::llround((double)total * cum[s] / cum[n_sms]) / gran * gran);
+  };
   for (int s = 0; s < n_sms; ++s) {
-    int a = (int)(((long long)total * s / n_sms) / gran * gran);
-    int b = (s + 1 == n_sms) ? total : (int)(((long long)total * (s + 1) / n_sms) / gran * gran);
+    int a = bound(s);
+    int b = bound(s + 1);
     int n = b - a;
     if (n <= 0) continue;
     int nt = (n + kTaskRows - 1) / kTaskRows;
@@ -414,7 +424,7 @@ int build_graph(mk_ctx* c) {
 
   // embedding slices
   {
-    auto parts = partition_rows(f.hidden, 1, n);
+    auto parts = partition_rows(f.hidden, 1, c->sm_weights);
     for (int s = 0; s < n; ++s)
       for (auto& p : parts[s]) {
         Task t = make_task(TK_EMBED, 0, p.first, p.second);
@@ -423,10 +433,10 @@ int build_graph(mk_ctx* c) {
         q[s].push_back(t);
       }
   }
-  auto qkv_parts = partition_rows(c->rows_qkv, 2, n);
-  auto o_parts = partition_rows(f.hidden, 1, n);
-  auto gu_parts = partition_rows(c->rows_gu, 2, n);
-  auto d_parts = partition_rows(f.hidden, 1, n);
+  auto qkv_parts = partition_rows(c->rows_qkv, 2, c->sm_weights);
+  auto o_parts = partition_rows(f.hidden, 1, c->sm_weights);
+  auto gu_parts = partition_rows(c->rows_gu, 2, c->sm_weights);
+  auto d_parts = partition_rows(f.hidden, 1, c->sm_weights);
   const int n_attn = B * nkv * c->nch;
   for (int l = 0; l < L; ++l) {
     for (int s = 0; s < n; ++s)
@@ -478,7 +488,7 @@ int build_graph(mk_ctx* c) {
       }
   }
   {
-    auto parts = partition_rows(f.vocab, 1, n);
+    auto parts = partition_rows(f.vocab, 1, c->sm_weights);
     int idx = 0;
     for (int s = 0; s < n; ++s)
       for (auto& p : parts[s]) {
@@ -547,7 +557,10 @@ void layout(mk_ctx* c) {
     w = align256(w + bytes);
     return at;
   };
-  c->ws_tasks = take(c->g.tasks.size() * sizeof(Task));
+  // room for re-partitioned graphs (mk_set_sm_weights) without changing the workspace size
+  c->task_cap = c->g.tasks.size() * 2 + (size_t)c->n_sms * 16;
+  c->lm_cap = (size_t)c->n_lm * 2 + (size_t)c->n_sms * 4;
+  c->ws_tasks = take(c->task_cap * sizeof(Task));
   c->ws_qbegin = take((c->n_sms + 1) * sizeof(uint32_t));
   c->ws_evcount = take(c->n_events * sizeof(uint32_t));
   c->ev_bytes = c->n_events * sizeof(uint32_t);
@@ -563,8 +576,8 @@ void layout(mk_ctx* c) {
   c->ws_o = take((size_t)L * B * nq * D * 4);
   c->ws_h = take((size_t)L * B * F * 4);
   c->ws_part = take((size_t)L * B * nq * c->nch * (D + 2) * 4);
-  c->ws_lmval = take((size_t)c->n_lm * B * 4);
-  c->ws_lmidx = take((size_t)c->n_lm * B * 4);
+  c->ws_lmval = take(c->lm_cap * B * 4);
+  c->ws_lmidx = take(c->lm_cap * B * 4);
   // prefill scratch: X, XN, Y, Q, O, HH per row
   const long long ycols = std::max<long long>(std::max(c->rows_qkv, c->rows_gu), H);
   c->pf_rows = (int)std::min<long long>(1024, (long long)B * f.max_seq);
@@ -613,6 +626,25 @@ bool cuda_ok(mk_ctx* c, cudaError_t e, const char* what) {
   if (e == cudaSuccess) return true;
   fail(c, MK_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
   return false;
+}
+
+// Copy the task graph (tasks, queue offsets, event counts) into the workspace and zero the
+// event and arrival counters (the epoch restarts at 1 with the next step).
+int upload_graph(mk_ctx* c, uint8_t* W) {
+  std::vector<Task> tv;
+  for (auto& r : c->g.tasks) tv.push_back(r.t);
+  if (!cuda_ok(c, cudaMemcpy(W + c->ws_tasks, tv.data(), tv.size() * sizeof(Task), cudaMemcpyHostToDevice),
+               "task upload") ||
+      !cuda_ok(c, cudaMemcpy(W + c->ws_qbegin, c->qbegin.data(), c->qbegin.size() * 4, cudaMemcpyHostToDevice),
+               "queue upload") ||
+      !cuda_ok(c, cudaMemcpy(W + c->ws_evcount, c->g.ev_count.data(), c->g.ev_count.size() * 4,
+                             cudaMemcpyHostToDevice),
+               "event upload") ||
+      !cuda_ok(c, cudaMemset(W + c->ws_ev, 0, c->ev_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(W + c->ws_acnt, 0, c->acnt_bytes), "counter reset"))
+    return MK_ERR_CUDA;
+  c->epoch = 0;
+  return MK_OK;
 }
 
 }  // namespace
@@ -674,7 +706,8 @@ int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
     delete c;
     return fail(nullptr, MK_ERR_UNSUPPORTED, "a weight row does not fit one ring stage");
   }
-  c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, 1);
+  c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim);
+  c->sm_weights.assign(c->n_sms, 1.0);
   rc = build_graph(c);
   if (rc) {
     std::string m = c->err;
@@ -753,18 +786,10 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
   }
   // workspace: task graph, counts, zeroed counters, offsets, RoPE table
   uint8_t* W = static_cast<uint8_t*>(workspace);
-  std::vector<Task> tv;
-  for (auto& r : c->g.tasks) tv.push_back(r.t);
   std::vector<float2> rope;
   rope_table(f, rope);
-  if (!cuda_ok(c, cudaMemcpy(W + c->ws_tasks, tv.data(), tv.size() * sizeof(Task), cudaMemcpyHostToDevice),
-               "task upload") ||
-      !cuda_ok(c, cudaMemcpy(W + c->ws_qbegin, c->qbegin.data(), c->qbegin.size() * 4, cudaMemcpyHostToDevice),
-               "queue upload") ||
-      !cuda_ok(c, cudaMemcpy(W + c->ws_evcount, c->g.ev_count.data(), c->g.ev_count.size() * 4,
-                             cudaMemcpyHostToDevice),
-               "event upload") ||
-      !cuda_ok(c, cudaMemcpy(W + c->ws_loff, c->loff.data(), c->loff.size() * sizeof(LayerOff),
+  if (upload_graph(c, W) != MK_OK) return MK_ERR_CUDA;
+  if (!cuda_ok(c, cudaMemcpy(W + c->ws_loff, c->loff.data(), c->loff.size() * sizeof(LayerOff),
                              cudaMemcpyHostToDevice),
                "offset upload") ||
       !cuda_ok(c, cudaMemcpy(W + c->ws_rope, rope.data(), rope.size() * sizeof(float2), cudaMemcpyHostToDevice),
@@ -945,6 +970,37 @@ int mk_debug_drop_notify(mk_ctx* c, int event_id, int on) {
   return MK_OK;
 }
 
+int mk_set_sm_weights(mk_ctx* c, const float* weights, int n, void* stream) {
+  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!weights || n != c->n_sms) return fail(c, MK_ERR_INVALID_ARG, "need one weight per SM");
+  std::vector<double> w(n);
+  for (int i = 0; i < n; ++i) {
+    if (!(weights[i] > 0.f) || !std::isfinite(weights[i]) || weights[i] > 1e3f)
+      return fail(c, MK_ERR_INVALID_ARG, "weights must be finite and in (0, 1000]");
+    w[i] = weights[i];
+  }
+  if (c->loaded && !cuda_ok(c, cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "stream sync"))
+    return MK_ERR_CUDA;
+  std::vector<double> old = c->sm_weights;
+  Graph old_g = c->g;
+  std::vector<uint32_t> old_q = c->qbegin;
+  const int old_lm = c->n_lm;
+  c->sm_weights = w;
+  int rc = build_graph(c);
+  if (rc == MK_OK && (c->g.tasks.size() > c->task_cap || (size_t)c->n_lm > c->lm_cap))
+    rc = fail(c, MK_ERR_UNSUPPORTED, "re-partitioned graph exceeds the workspace reserve");
+  if (rc != MK_OK) {
+    std::string m = c->err;
+    c->sm_weights = old;
+    c->g = old_g;
+    c->qbegin = old_q;
+    c->n_lm = old_lm;
+    return fail(c, rc, m);
+  }
+  if (c->loaded && upload_graph(c, c->ws) != MK_OK) return MK_ERR_CUDA;
+  return MK_OK;
+}
+
 int mk_set_l2_prefetch(mk_ctx* c, int stages) {
   if (!c || stages < 0 || stages > 64) return fail(c, MK_ERR_INVALID_ARG, "stages must be in [0, 64]");
   c->l2_ahead = stages;
@@ -963,6 +1019,7 @@ int mk_get_graph_info(const mk_ctx* c, mk_graph_info* out) {
   if (!c || !out) return MK_ERR_INVALID_ARG;
   out->n_sms = c->n_sms;
   out->n_tasks = (int)c->g.tasks.size();
+  out->task_capacity = (int)c->task_cap;
   out->n_events = c->n_events;
   out->attn_chunks = c->nch;
   out->kernel_variant = c->variant;

@@ -29,10 +29,16 @@ constexpr int kBlockThreads = (kWorkerWarps + 2) * 32;
 constexpr int kSegElems = kWorkerThreads * 8;        // K elements one pass of all workers covers
 constexpr int kSegBytes = kSegElems * 2;
 constexpr int kTaskRows = 256;                       // rows per GEMV task (one per worker thread)
-constexpr int kRpsMax = 32;                          // rows per ring stage (unrolled in the GEMV loop)
+constexpr int kRpsMax = 8;                           // rows per ring stage (unrolled in the GEMV loop)
 constexpr int kMaxChunks = 64;                       // split-KV chunks per (sequence, KV head)
-constexpr int kSlotBytes = 32 * 1024;                // one ring stage
-constexpr int kStages = 6;                           // ring depth
+#ifndef MK_SLOT_KB
+#define MK_SLOT_KB 32
+#endif
+#ifndef MK_STAGES
+#define MK_STAGES 6
+#endif
+constexpr int kSlotBytes = MK_SLOT_KB * 1024;        // one ring stage
+constexpr int kStages = MK_STAGES;                   // ring depth (kStages x kSlotBytes per SM)
 constexpr int kMaxDecodeBatch = 1;                   // CUDA-core path instantiations
 
 enum TaskKind : uint8_t {
@@ -96,7 +102,12 @@ struct DecodeParams {
   uint64_t* trace;            // optional [n_tasks][kTraceWords] timing records (null = off)
   int l2_ahead;               // weight stages the producer prefetches into L2 beyond the ring
 };
-constexpr int kMinChunkKeys = 32;  // split-KV chunks hold at least this many keys
+constexpr uint64_t kStallPrefetchNs = 1000;    // producer blocked this long: prefetch ahead into L2
+constexpr uint64_t kStallPrefetchGapNs = 100;   // then one more stage per this interval
+#ifndef MK_MIN_CHUNK_KEYS
+#define MK_MIN_CHUNK_KEYS 64
+#endif
+constexpr int kMinChunkKeys = MK_MIN_CHUNK_KEYS;  // split-KV chunks hold at least this many keys
 
 // Trace record per task (global-timer ns): worker start of the wait for inputs, inputs
 // released, task done; worker ns blocked on ring stages | SM id << 32; producer ns blocked
@@ -115,9 +126,9 @@ TensorMapEncodeFn get_tensor_map_encoder();
 
 // Kernel variants: one instantiation per (segments, rows per stage) of the two K sizes.
 struct Variant {
-  int nseg_h, rps_h, nseg_f, rps_f, batch;
+  int nseg_h, rps_h, nseg_f, rps_f, head_dim;
 };
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int batch);
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim);
 const void* decode_kernel_ptr(int variant);
 size_t decode_smem_bytes();
 int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t stream, std::string* err);

@@ -133,3 +133,28 @@ def test_validator_rejects_a_wrong_threshold(graph):
     c = counts.copy()
     c[1] += 1
     _reject(ctx, tasks, c, "threshold")
+
+
+def test_weighted_partition_follows_the_sm_weights():
+    ctx = mk.mk_build_taskgraph(mk.Config.from_shape(mi.LLAMA8B, 1, 1024).c(), -1)
+    try:
+        info = mk.mk_get_graph_info(ctx)
+        n = info["n_sms"]
+        w = np.random.default_rng(0).uniform(0.6, 1.4, n).astype(np.float32)
+        mk.mk_set_sm_weights(ctx, w)
+        tasks, counts = mk.mk_export_taskgraph(ctx)
+        assert mk.mk_validate_taskgraph(ctx, tasks, counts) == 0
+        assert len(tasks) <= mk.mk_get_graph_info(ctx)["task_capacity"]
+        K = {2: 4096, 4: 4096, 5: 4096, 6: 14336, 7: 4096}
+        per_sm = np.zeros(n)
+        for t in tasks:
+            if t[0] in K:
+                per_sm[t[2]] += t[4] * K[t[0]] * 2
+        share = per_sm / per_sm.sum()
+        assert np.allclose(share, w / w.sum(), rtol=0.02)
+        with pytest.raises(mk.MkError):
+            mk.mk_set_sm_weights(ctx, np.zeros(n, dtype=np.float32))
+        with pytest.raises(mk.MkError):
+            mk.mk_set_sm_weights(ctx, np.ones(n - 1, dtype=np.float32))
+    finally:
+        mk.mk_destroy(ctx)

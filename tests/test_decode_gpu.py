@@ -121,3 +121,25 @@ def test_dependency_wait_times_out_cleanly():
     assert m.sync_status() == mk.MK_OK
     logits_close(gl[0].cpu().numpy(), rl, "after recovery")
     assert info["n_sms"] > 0
+
+
+def test_calibrated_schedule_keeps_parity():
+    # re-partitioned rows (per-SM weights measured from traced steps) must not change results
+    w = mi.make_weights(mi.TINY, seed=4)
+    prompt = mi.prompt(4, 0, 12, w.shape.vocab)
+    ref = oracle.Decoder(w, 1, 64)
+    m = gpu_model(w, 64)
+    ref.prefill(prompt)
+    m.prefill(torch.from_numpy(prompt[None].astype(np.int32)).to(DEV))
+    tok = 3
+    # calibration decodes real steps: mirror them on the oracle
+    weights = m.calibrate(torch.tensor([tok], dtype=torch.int32, device=DEV), steps=1, rounds=2)
+    for _ in range(2):
+        ref.decode(np.array([tok], dtype=np.int32))
+    assert weights.shape[0] == m.info()["n_sms"]
+    for i in range(4):
+        rl = ref.decode(np.array([tok], dtype=np.int32))[0]
+        gl, _ = m.decode(torch.tensor([tok], dtype=torch.int32, device=DEV))
+        logits_close(gl[0].cpu().numpy(), rl, f"step {i}")
+        tok = oracle.argmax(rl)
+    assert m.sync_status() == mk.MK_OK
