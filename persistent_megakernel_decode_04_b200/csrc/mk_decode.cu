@@ -456,14 +456,14 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
 #pragma unroll
           for (int u = 0; u < kAttnBlock; ++u)
             if (jb + u * kAttnWarps < a.j1) mx = fmaxf(mx, sc[u * 4 + h]);
-          const float alpha = expf(m[h] - mx);  // 0 on the first block (m = -inf)
+          const float alpha = __expf(m[h] - mx);  // 0 on the first block (m = -inf)
           float ls = 0.f;
 #pragma unroll
           for (int i = 0; i < DL; ++i) acc[h][i] *= alpha;
 #pragma unroll
           for (int u = 0; u < kAttnBlock; ++u) {
             if (jb + u * kAttnWarps < a.j1) {
-              const float p = expf(sc[u * 4 + h] - mx);
+              const float p = __expf(sc[u * 4 + h] - mx);
               ls += p;
 #pragma unroll
               for (int w = 0; w < W; ++w) {
@@ -499,7 +499,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       if (M != -INFINITY) {
 #pragma unroll
         for (int w = 0; w < kAttnWarps; ++w) {
-          const float f = expf(S.am[w][h] - M);
+          const float f = __expf(S.am[w][h] - M);
           ls += f * S.al[w][h];
           as += f * S.aacc[w][h][d];
         }
@@ -524,43 +524,54 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
   }
   worker_bar();
   if (S.flag && nch_eff > 1) {
-    // (m, l) of every used chunk of this group's heads, loaded in parallel
-    for (int e = tid; e < G * nch_eff; e += kWorkerThreads) {
-      const int h = e / nch_eff, cc = e % nch_eff;
-      const float* pc = part_base + ((size_t)(g * G + h) * P.nch + cc) * (D + 2);
-      S.mm[e] = __ldcg(pc);
-      S.ll[e] = __ldcg(pc + 1);
-    }
-    worker_bar();
-    // merge weights w_c = exp(m_c - M) per (head, chunk)
-    for (int e = tid; e < G * nch_eff; e += kWorkerThreads) {
-      const int h = e / nch_eff;
-      float M = -INFINITY;
-      for (int cc = 0; cc < nch_eff; ++cc) M = fmaxf(M, S.mm[h * nch_eff + cc]);
-      S.ww[e] = (S.mm[e] == -INFINITY) ? 0.f : expf(S.mm[e] - M);
-    }
-    worker_bar();
-    // o[h][d] = sum_c w_c acc_c[d] / sum_c w_c l_c: all loads of a block of 16 chunks are
-    // issued before any is used (one L2 round trip per 16 chunks)
-    for (int e = tid; e < G * D; e += kWorkerThreads) {
-      const int h = e / D, d = e % D;
-      const float* ph = part_base + (size_t)(g * G + h) * P.nch * (D + 2) + 2 + d;
-      float num = 0.f, den = 0.f;
-      for (int c0 = 0; c0 < nch_eff; c0 += 16) {
-        float v[16];
+    // Merge in one L2 round trip: every thread issues the partial-accumulator loads of its
+    // (up to two) output elements together with the (m, l) loads, then weighs each chunk by
+    // exp(m_c - M) itself.  Blocks of 16 chunks (one block up to nch_eff = 16).
+    const int e0 = tid, e1 = tid + kWorkerThreads;
+    const bool has0 = e0 < G * D, has1 = e1 < G * D;
+    const int h0 = e0 / D, d0 = e0 % D, h1 = e1 / D, d1 = e1 % D;
+    const float* ph0 = part_base + (size_t)(g * G + (has0 ? h0 : 0)) * P.nch * (D + 2) + 2 + d0;
+    const float* ph1 = part_base + (size_t)(g * G + (has1 ? h1 : 0)) * P.nch * (D + 2) + 2 + d1;
+    float num0 = 0.f, den0 = 0.f, num1 = 0.f, den1 = 0.f;
+    for (int c0 = 0; c0 < nch_eff; c0 += 16) {
+      float v0[16], v1[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = (c0 + k < nch_eff) ? __ldcg(ph + (size_t)(c0 + k) * (D + 2)) : 0.f;
+      for (int k = 0; k < 16; ++k) {
+        const bool ok = c0 + k < nch_eff;
+        v0[k] = (ok && has0) ? __ldcg(ph0 + (size_t)(c0 + k) * (D + 2)) : 0.f;
+        v1[k] = (ok && has1) ? __ldcg(ph1 + (size_t)(c0 + k) * (D + 2)) : 0.f;
+      }
+      if (c0 == 0) {
+        for (int e = tid; e < G * nch_eff; e += kWorkerThreads) {
+          const int h = e / nch_eff, cc = e % nch_eff;
+          const float* pc = part_base + ((size_t)(g * G + h) * P.nch + cc) * (D + 2);
+          S.mm[e] = __ldcg(pc);
+          S.ll[e] = __ldcg(pc + 1);
+        }
+        worker_bar();
+      }
+      const float* mm0 = S.mm + (has0 ? h0 : 0) * nch_eff;
+      const float* mm1 = S.mm + (has1 ? h1 : 0) * nch_eff;
+      float M0 = -INFINITY, M1 = -INFINITY;
+      for (int cc = 0; cc < nch_eff; ++cc) {
+        M0 = fmaxf(M0, mm0[cc]);
+        M1 = fmaxf(M1, mm1[cc]);
+      }
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          if (c0 + k < nch_eff) {
-            const float w = S.ww[h * nch_eff + c0 + k];
-            num = fmaf(w, v[k], num);
-            den = fmaf(w, S.ll[h * nch_eff + c0 + k], den);
-          }
+      for (int k = 0; k < 16; ++k) {
+        if (c0 + k < nch_eff) {
+          const int cc = c0 + k;
+          const float w0 = (mm0[cc] == -INFINITY) ? 0.f : __expf(mm0[cc] - M0);
+          const float w1 = (mm1[cc] == -INFINITY) ? 0.f : __expf(mm1[cc] - M1);
+          num0 = fmaf(w0, v0[k], num0);
+          den0 = fmaf(w0, S.ll[(has0 ? h0 : 0) * nch_eff + cc], den0);
+          num1 = fmaf(w1, v1[k], num1);
+          den1 = fmaf(w1, S.ll[(has1 ? h1 : 0) * nch_eff + cc], den1);
         }
       }
-      o[(size_t)h * D + d] = num / den;
     }
+    if (has0) o[(size_t)h0 * D + d0] = num0 / den0;
+    if (has1) o[(size_t)h1 * D + d1] = num1 / den1;
     worker_bar();
   }
   if (S.flag && tid == 0 && (int)t.notify[0] != P.drop_event) red_release_gpu_add(&P.ev[t.notify[0]], 1u);
