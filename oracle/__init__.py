@@ -61,6 +61,7 @@ def lib():
         L.or_decode_f64.argtypes = [vp, vp, vp]
         L.or_set_cache.argtypes = [vp, vp, i32]
         L.or_get_cache.argtypes = [vp, vp, i32]
+        L.or_set_positions.argtypes = [vp, vp]
         L.or_position.argtypes = [vp, i32]
         L.or_argmax.argtypes = [vp, i32]
         L.or_rmsnorm.argtypes = [vp, vp, i32, dbl, vp]
@@ -164,6 +165,11 @@ class Decoder:
         if lib().or_get_cache(self._h, _ptr(out), int(length)) != 0:
             raise ValueError("or_get_cache rejected its arguments")
         return out
+
+    def set_positions(self, positions) -> None:
+        pos = _c(np.asarray(positions), np.int32)
+        if pos.size != self.batch or lib().or_set_positions(self._h, _ptr(pos)) != 0:
+            raise ValueError("or_set_positions rejected its arguments")
 
     def position(self, b: int = 0) -> int:
         return lib().or_position(self._h, b)

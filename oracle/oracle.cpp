@@ -380,6 +380,14 @@ int or_get_cache(const or_state* s, uint16_t* kv, int length) {
   return 0;
 }
 
+int or_set_positions(or_state* s, const int32_t* pos) {
+  if (!s || !pos) return -1;
+  for (int b = 0; b < s->impl->batch; ++b)
+    if (pos[b] < 0 || pos[b] > s->impl->max_seq) return -1;
+  for (int b = 0; b < s->impl->batch; ++b) s->impl->pos[b] = pos[b];
+  return 0;
+}
+
 int or_position(const or_state* s, int b) {
   if (!s || b < 0 || b >= s->impl->batch) return -1;
   return s->impl->pos[b];

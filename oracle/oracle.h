@@ -74,6 +74,9 @@ int or_set_cache(or_state* s, const uint16_t* kv, int length);
 /* Copy the cache out as bf16 bits (fp32 values rounded RNE; exact when kv_round = 1),
  * same layout with `length` positions. */
 int or_get_cache(const or_state* s, uint16_t* kv, int length);
+/* Set each sequence's position (0..max_seq): the next token of sequence b goes to pos[b] and
+ * attends to cache entries 0..pos[b].  Entries at or past pos[b] are ignored and overwritten. */
+int or_set_positions(or_state* s, const int32_t* pos);
 int or_position(const or_state* s, int b);
 /* Greedy pick: index of the largest logit, the lowest index among equal values. */
 int or_argmax(const float* logits, int n);

@@ -34,11 +34,11 @@ namespace mk {
 struct DSmem {
   uint8_t ring[kStages][kSlotBytes];
   union {
-    float red[kWorkerWarps][kTaskRows];  // GEMV: per-warp row sums of the current task
+    float red[kWorkerWarps][kTaskRows];  // GEMV: per-warp sums of the current task, [row][seq]
     float aacc[kAttnWarps][4][128];      // attention: per-warp partial outputs
   };
-  float tot[kTaskRows];                  // row totals of the current task
-  float ssw[kWorkerWarps];
+  float tot[kTaskRows];                  // totals of the current task, [row][seq]
+  float ssw[kWorkerWarps][kMaxDecodeBatch];  // per-warp sums of x^2 per sequence
   float am[kAttnWarps][4];
   float al[kAttnWarps][4];
   float mm[4 * kMaxChunks], ll[4 * kMaxChunks], ww[4 * kMaxChunks];  // split-KV merge
@@ -115,7 +115,13 @@ __device__ __forceinline__ void gemv_source(const DecodeParams& P, const Task& t
     case TK_QKV: *off = lo.qkv; *row_bytes = (uint32_t)P.H * 2u; break;
     case TK_OPROJ: *off = lo.o; *row_bytes = (uint32_t)P.H * 2u; break;
     case TK_GATEUP: *off = lo.gu; *row_bytes = (uint32_t)P.H * 2u; break;
-    case TK_DOWN: *off = lo.d; *row_bytes = (uint32_t)P.F * 2u; break;
+    case TK_DOWN: {  // K chunk t.aux of W_down: chunk-major, rows of kc = min(kdc, F - k0) weights
+      const uint32_t k0 = (uint32_t)t.aux * (uint32_t)P.kdc;
+      const uint32_t kc = min((uint32_t)P.kdc, (uint32_t)P.F - k0);
+      *off = lo.d + (uint64_t)k0 * P.H * 2u;
+      *row_bytes = kc * 2u;
+      break;
+    }
     default: *off = P.off_lm; *row_bytes = (uint32_t)P.H * 2u; break;
   }
 }
@@ -154,48 +160,53 @@ __device__ __forceinline__ void warp_reduce_rows(float (&a)[V], float* out, int 
   }
 }
 
-// GEMV core: tot[r] = sum_k W[row0 + r][k] * x[k] * g[k] for r < nrows (<= kTaskRows), rows
-// streamed through the ring RPS rows per stage.  The stage loop is a runtime loop and only
-// one stage's rows are unrolled, so the code stays small; each stage's rows are reduced
-// across lanes right away into S.red[warp][row], and across warps at the end into S.tot.
-// Also leaves the per-warp sums of x^2 in S.ssw for the fused norm.  Returns false (for
-// every worker thread alike) if a wait ran out.
-template <int NSEG, int RPS>
+// GEMV core: tot[r * BM + b] = sum_k W[row0 + r][k] * x_b[k] * g[k] for r < nrows and the
+// nb (<= BM) sequences b, where x_b = xsrc + b * xstride; nrows * BM <= kTaskRows.  Rows are
+// streamed through the ring RPS rows per stage, so each weight is read from shared memory
+// once and meets all BM activation vectors.  The stage loop is a runtime loop and only one
+// stage's rows are unrolled, so the code stays small; each stage's RPS x BM sums are reduced
+// across lanes right away into S.red[warp][row * BM + b], and across warps at the end into
+// S.tot.  Also leaves the per-warp sums of x_b^2 in S.ssw for the fused norm.  Returns false
+// (for every worker thread alike) if a wait ran out.
+template <int NSEG, int RPS, int BM>
 __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe& pp, const float* __restrict__ xsrc,
-                                          const uint16_t* __restrict__ gain, int K, int nrows, uint32_t row_bytes,
-                                          uint32_t task_id, uint32_t& stall_ns) {
+                                          int xstride, int nb, const uint16_t* __restrict__ gain, int K, int nrows,
+                                          uint32_t row_bytes, uint32_t task_id, uint32_t& stall_ns) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // only the last segment can be partial: K > (NSEG - 1) * kSegElems by construction
+  // only the last segment can be partial or empty: K > (NSEG - 2) * kSegElems by construction
   const bool last_ok = (NSEG - 1) * kSegElems + tid * 8 < K;
-  float x[NSEG][8];
-  float ss = 0.f;
+  uint64_t x2[BM][NSEG][4];
+  float ss[BM];
 #pragma unroll
-  for (int s = 0; s < NSEG; ++s) {
-    const int k = s * kSegElems + tid * 8;
-    if (s < NSEG - 1 || last_ok) {
-      const float4 a = __ldcg(reinterpret_cast<const float4*>(xsrc + k));
-      const float4 b = __ldcg(reinterpret_cast<const float4*>(xsrc + k + 4));
-      x[s][0] = a.x; x[s][1] = a.y; x[s][2] = a.z; x[s][3] = a.w;
-      x[s][4] = b.x; x[s][5] = b.y; x[s][6] = b.z; x[s][7] = b.w;
+  for (int b = 0; b < BM; ++b) {
+    ss[b] = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ss = fmaf(x[s][i], x[s][i], ss);
-      if (gain) {
-        const uint4 g = __ldg(reinterpret_cast<const uint4*>(gain + k));
-        x[s][0] *= bf16lo(g.x); x[s][1] *= bf16hi(g.x);
-        x[s][2] *= bf16lo(g.y); x[s][3] *= bf16hi(g.y);
-        x[s][4] *= bf16lo(g.z); x[s][5] *= bf16hi(g.z);
-        x[s][6] *= bf16lo(g.w); x[s][7] *= bf16hi(g.w);
+    for (int s = 0; s < NSEG; ++s) {
+      const int k = s * kSegElems + tid * 8;
+      float x[8];
+      if ((s < NSEG - 1 || last_ok) && (BM == 1 || b < nb)) {
+        const float* xb = xsrc + (size_t)b * xstride;
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(xb + k));
+        const float4 c = __ldcg(reinterpret_cast<const float4*>(xb + k + 4));
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss[b] = fmaf(x[i], x[i], ss[b]);
+        if (gain) {
+          const uint4 g = __ldg(reinterpret_cast<const uint4*>(gain + k));
+          x[0] *= bf16lo(g.x); x[1] *= bf16hi(g.x);
+          x[2] *= bf16lo(g.y); x[3] *= bf16hi(g.y);
+          x[4] *= bf16lo(g.z); x[5] *= bf16hi(g.z);
+          x[6] *= bf16lo(g.w); x[7] *= bf16hi(g.w);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = 0.f;
       }
-    } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[s][i] = 0.f;
+      for (int j = 0; j < 4; ++j) x2[b][s][j] = pack2(x[2 * j], x[2 * j + 1]);
     }
   }
-  uint64_t x2[NSEG][4];
-#pragma unroll
-  for (int s = 0; s < NSEG; ++s)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) x2[s][j] = pack2(x[s][2 * j], x[s][2 * j + 1]);
   float* red = S.red[warp];
   bool ok = true;
   for (int r0 = 0; r0 < nrows; r0 += RPS) {
@@ -207,16 +218,28 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
     }
     if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
     const uint8_t* base = S.ring[pp.stage] + tid * 16;
-    uint64_t acc[RPS];  // per row: (even, odd) partial sums
+    uint64_t acc[RPS][BM];  // per (row, sequence): (even, odd) partial sums
 #pragma unroll
     for (int rr = 0; rr < RPS; ++rr) {
-      acc[rr] = 0ull;
+#pragma unroll
+      for (int b = 0; b < BM; ++b) acc[rr][b] = 0ull;
       if (RPS == 1 || r0 + rr < nrows) {
 #pragma unroll
         for (int s = 0; s < NSEG; ++s) {
           if (s < NSEG - 1 || last_ok) {
             const uint4 w = *reinterpret_cast<const uint4*>(base + rr * row_bytes + s * kSegBytes);
-            dot8(w, x2[s], acc[rr]);
+            if (BM == 1) {
+              dot8(w, x2[0][s], acc[rr][0]);
+            } else {
+              const uint64_t wp[4] = {widen_bf16w(w.x), widen_bf16w(w.y), widen_bf16w(w.z), widen_bf16w(w.w)};
+#pragma unroll
+              for (int b = 0; b < BM; ++b) {
+                if (b < nb) {
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) fma2_pair(acc[rr][b], wp[j], x2[b][s][j]);
+                }
+              }
+            }
           }
         }
       }
@@ -224,20 +247,25 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
     pp.advance();
-    float a[RPS];
+    float a[RPS * BM];
 #pragma unroll
-    for (int rr = 0; rr < RPS; ++rr) {
-      const float2 v = unpack2(acc[rr]);
-      a[rr] = v.x + v.y;
-    }
-    warp_reduce_rows<RPS>(a, red + r0, lane, nrows - r0);
+    for (int rr = 0; rr < RPS; ++rr)
+#pragma unroll
+      for (int b = 0; b < BM; ++b) {
+        const float2 v = unpack2(acc[rr][b]);
+        a[rr * BM + b] = v.x + v.y;
+      }
+    warp_reduce_rows<RPS * BM>(a, red + r0 * BM, lane, (nrows - r0) * BM);
   }
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-  if (lane == 0) S.ssw[warp] = ss;
+  for (int b = 0; b < BM; ++b) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss[b] += __shfl_xor_sync(0xffffffffu, ss[b], off);
+    if (lane == 0) S.ssw[warp][b] = ss[b];
+  }
   worker_bar();
   if (S.cabort) return false;
-  for (int t = tid; t < nrows; t += kWorkerThreads) {
+  for (int t = tid; t < nrows * BM; t += kWorkerThreads) {
     float v = 0.f;
 #pragma unroll
     for (int w2 = 0; w2 < kWorkerWarps; ++w2) v += S.red[w2][t];
@@ -247,24 +275,26 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
   return true;
 }
 
-__device__ __forceinline__ float norm_factor(const DSmem& S, int K, float eps) {
+__device__ __forceinline__ float norm_factor(const DSmem& S, int K, float eps, int b) {
   float ss = 0.f;
 #pragma unroll
-  for (int w = 0; w < kWorkerWarps; ++w) ss += S.ssw[w];
+  for (int w = 0; w < kWorkerWarps; ++w) ss += S.ssw[w][b];
   return 1.0f / sqrtf(ss / (float)K + eps);
 }
 
 // ---------------------------------------------------------------------------------------
-// Epilogues (thread t < nrows handles row row0 + t).
+// Epilogues: thread e < nrows * BM handles row row0 + e / BM of sequence b = e % BM, whose
+// GEMV total is S.tot[e] (sequences b >= nb are skipped).
+template <int BM>
 __device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, const Task& t, float r) {
   const int tid = threadIdx.x;
-  if (tid >= (int)t.nrows) return;
+  const int b = tid % BM;
+  if (tid >= (int)t.nrows * BM || b >= P.nb) return;
   const int D = P.D, G = P.nq / P.nkv, half = D / 2;
   const int rpg = (G + 2) * D;
-  const int R = (int)t.row0 + tid;
+  const int R = (int)t.row0 + tid / BM;
   const int grp = R / rpg, rr = R % rpg;
   const float v = S.tot[tid] * r;
-  const int b = 0;
   const int pos = P.pos[b];
   const size_t head_stride = (size_t)P.max_seq * D;
   const size_t kv_layer = (size_t)P.max_batch * P.nkv * head_stride;  // one of K or V, one layer
@@ -272,7 +302,7 @@ __device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, c
     // q or k: rows come in RoPE pairs (i, i + D/2) at packed positions (2i, 2i+1)
     const int pd = (rr < G * D) ? (rr % D) : (rr - G * D);
     const int i = pd >> 1, hi = pd & 1;
-    const float other = S.tot[tid ^ 1] * r;
+    const float other = S.tot[tid ^ BM] * r;  // the RoPE partner row, same sequence
     const float2 cs = P.rope[(size_t)pos * half + i];
     float outv;
     int dim;
@@ -323,6 +353,11 @@ __device__ __forceinline__ AttnGeom attn_geom(const DecodeParams& P, const Task&
   a.g = (int)t.row0 % P.nkv;
   a.c = t.aux;
   a.Lk = P.pos[a.b] + 1;
+  if (a.b >= P.nb) {  // sequence not in the active batch: its tasks only count their arrival
+    a.nch_eff = 0;
+    a.j0 = a.j1 = 0;
+    return a;
+  }
   a.nch_eff = max(1, min(P.nch, (a.Lk + kMinChunkKeys - 1) / kMinChunkKeys));
   const int cl = (a.Lk + a.nch_eff - 1) / a.nch_eff;
   a.j0 = a.c * cl;
@@ -601,36 +636,45 @@ __device__ __forceinline__ void block_argmax(DSmem& S, float& v, int& idx) {
     for (int w = 1; w < kWorkerWarps; ++w) argmax_merge(v, idx, S.lmv[w], S.lmi[w]);
 }
 
-__device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, const Task& t, float r) {
+template <int BM>
+__device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, const Task& t, int K) {
   const int tid = threadIdx.x;
-  const int b = 0;
-  float v = -INFINITY;
-  int idx = 0x7fffffff;
-  for (int i = tid; i < (int)t.nrows; i += kWorkerThreads) {
-    const float lv = S.tot[i] * r;
-    P.logits[(size_t)b * P.V + t.row0 + i] = lv;
-    argmax_merge(v, idx, lv, (int)t.row0 + i);
+  for (int b = 0; b < P.nb; ++b) {
+    const float r = norm_factor(S, K, P.eps, b);
+    float v = -INFINITY;
+    int idx = 0x7fffffff;
+    for (int i = tid; i < (int)t.nrows; i += kWorkerThreads) {
+      const float lv = S.tot[i * BM + b] * r;
+      P.logits[(size_t)b * P.V + t.row0 + i] = lv;
+      argmax_merge(v, idx, lv, (int)t.row0 + i);
+    }
+    block_argmax(S, v, idx);
+    if (tid == 0) {
+      P.lm_val[(size_t)t.index * P.B + b] = v;
+      P.lm_idx[(size_t)t.index * P.B + b] = idx;
+    }
+    worker_bar();  // S.lmv / S.lmi are reused by the next sequence
   }
-  block_argmax(S, v, idx);
   if (tid == 0) {
-    P.lm_val[(size_t)t.index * P.B + b] = v;
-    P.lm_idx[(size_t)t.index * P.B + b] = idx;
     const uint32_t old = atom_acq_rel_gpu_add(&P.ev[P.ev_lm], 1u);
     S.flag = (old + 1u == P.epoch * (uint32_t)P.n_lm) ? 1u : 0u;
   }
   worker_bar();
   if (S.flag && P.next_tokens) {
-    v = -INFINITY;
-    idx = 0x7fffffff;
-    for (int i = tid; i < P.n_lm; i += kWorkerThreads)
-      argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
-    block_argmax(S, v, idx);
-    if (tid == 0) P.next_tokens[b] = idx;
+    for (int b = 0; b < P.nb; ++b) {
+      float v = -INFINITY;
+      int idx = 0x7fffffff;
+      for (int i = tid; i < P.n_lm; i += kWorkerThreads)
+        argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
+      block_argmax(S, v, idx);
+      if (tid == 0) P.next_tokens[b] = idx;
+      worker_bar();
+    }
   }
 }
 
 // ---------------------------------------------------------------------------------------
-template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD>
+template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM>
 __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   DSmem& S = *reinterpret_cast<DSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -831,71 +875,91 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     const uint64_t t_ready = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     bool notify = true;
     if (is_gemv(t.kind)) {
-      // operands of the task's GEMV: x source, norm gain (null = no norm) and K
+      // operands of the task's GEMV: x source of sequence 0 and the stride to the next, norm
+      // gain (null = no norm) and K
       const float* xs;
       const uint16_t* gain = nullptr;
-      int K = P.H;
+      int K = P.H, xstride = P.H;
       const size_t lay = (size_t)t.layer * P.B;
       switch (t.kind) {
         case TK_QKV:
           xs = P.x_in + lay * P.H;
           gain = reinterpret_cast<const uint16_t*>(P.arena + lo.attn_norm);
           break;
-        case TK_OPROJ: xs = P.obuf + lay * P.nq * P.D; break;
+        case TK_OPROJ:
+          xs = P.obuf + lay * P.nq * P.D;
+          xstride = P.nq * P.D;
+          break;
         case TK_GATEUP:
           xs = P.x_mid + lay * P.H;
           gain = reinterpret_cast<const uint16_t*>(P.arena + lo.mlp_norm);
           break;
-        case TK_DOWN:
-          xs = P.hbuf + lay * P.F;
-          K = P.F;
+        case TK_DOWN: {
+          const int k0 = (int)t.aux * P.kdc;  // K chunk of the down projection
+          xs = P.hbuf + lay * P.F + k0;
+          xstride = P.F;
+          K = min(P.kdc, P.F - k0);
           break;
+        }
         default:  // LM head
           xs = P.x_in + (size_t)P.L * P.B * P.H;
           gain = reinterpret_cast<const uint16_t*>(P.arena + P.off_fnorm);
           break;
       }
+      uint32_t rb;
+      {
+        uint64_t off_unused;
+        gemv_source(P, t, &off_unused, &rb);
+      }
       const bool ok = (t.kind == TK_DOWN)
-                          ? gemv_tile<NSEG_F, RPS_F>(P, S, pp, xs, gain, K, (int)t.nrows, (uint32_t)K * 2u, i, stall)
-                          : gemv_tile<NSEG_H, RPS_H>(P, S, pp, xs, gain, K, (int)t.nrows, (uint32_t)K * 2u, i, stall);
+                          ? gemv_tile<NSEG_F, RPS_F, BM>(P, S, pp, xs, xstride, P.nb, gain, K, (int)t.nrows, rb, i, stall)
+                          : gemv_tile<NSEG_H, RPS_H, BM>(P, S, pp, xs, xstride, P.nb, gain, K, (int)t.nrows, rb, i, stall);
       if (!ok) goto out;
-      const float r = gain ? norm_factor(S, K, P.eps) : 1.f;
+      // this thread's (row, sequence) in the epilogues
+      const int eb = tid % BM, er = tid / BM;
+      const bool mine = er < (int)t.nrows && eb < P.nb;
+      const float r = gain ? norm_factor(S, K, P.eps, eb) : 1.f;
       switch (t.kind) {
-        case TK_QKV: epi_qkv(P, S, t, r); break;
+        case TK_QKV: epi_qkv<BM>(P, S, t, r); break;
         case TK_OPROJ:
-          if (tid < (int)t.nrows) {
-            const size_t row = (size_t)t.row0 + tid;
-            P.x_mid[lay * P.H + row] = __ldcg(P.x_in + lay * P.H + row) + S.tot[tid];
+          if (mine) {
+            const size_t at = (lay + eb) * P.H + t.row0 + er;
+            P.x_mid[at] = __ldcg(P.x_in + at) + S.tot[tid];
           }
           break;
         case TK_GATEUP:
-          if (tid < (int)t.nrows && (tid & 1) == 0) {
-            const float gv = S.tot[tid] * r, uv = S.tot[tid + 1] * r;
+          if (mine && (er & 1) == 0) {
+            const float gv = S.tot[tid] * r, uv = S.tot[tid + BM] * r;
             const float sg = gv / (1.f + expf(-gv));
-            P.hbuf[lay * P.F + (t.row0 + tid) / 2] = sg * uv;
+            P.hbuf[(lay + eb) * P.F + (t.row0 + er) / 2] = sg * uv;
           }
           break;
         case TK_DOWN:
-          if (tid < (int)t.nrows) {
-            const size_t row = (size_t)t.row0 + tid;
-            P.x_in[(lay + P.B) * P.H + row] = __ldcg(P.x_mid + lay * P.H + row) + S.tot[tid];
+          if (mine) {
+            // K chunk 0 starts from the residual; later chunks of the same rows ran earlier
+            // in this queue, on this thread, and add to what it stored
+            const size_t at = (lay + eb) * P.H + t.row0 + er;
+            float* dst = P.x_in + P.B * P.H + at;
+            const float base = (t.aux == 0) ? __ldcg(P.x_mid + at) : *dst;
+            *dst = base + S.tot[tid];
           }
           break;
         default:
           notify = false;
-          epi_lmhead(P, S, t, r);
+          epi_lmhead<BM>(P, S, t, K);
           break;
       }
     } else if (t.kind == TK_EMBED) {
-      const int b = 0;
-      int tok = __ldcg(P.tokens + b);
-      if (tok < 0 || tok >= P.V) {  // never read outside the table: record and use row 0
-        if (tid == 0 && t.row0 == 0) atomicCAS(&P.err[ERR_CODE], 0u, (uint32_t)DEV_ERR_BAD_TOKEN);
-        tok = 0;
+      for (int b = 0; b < P.nb; ++b) {
+        int tok = __ldcg(P.tokens + b);
+        if (tok < 0 || tok >= P.V) {  // never read outside the table: record and use row 0
+          if (tid == 0 && t.row0 == 0) atomicCAS(&P.err[ERR_CODE], 0u, (uint32_t)DEV_ERR_BAD_TOKEN);
+          tok = 0;
+        }
+        const uint16_t* e = reinterpret_cast<const uint16_t*>(P.arena + P.off_embed) + (size_t)tok * P.H;
+        for (uint32_t r = tid; r < t.nrows; r += kWorkerThreads)
+          P.x_in[(size_t)b * P.H + t.row0 + r] = __uint_as_float((uint32_t)e[t.row0 + r] << 16);
       }
-      const uint16_t* e = reinterpret_cast<const uint16_t*>(P.arena + P.off_embed) + (size_t)tok * P.H;
-      for (uint32_t r = tid; r < t.nrows; r += kWorkerThreads)
-        P.x_in[(size_t)b * P.H + t.row0 + r] = __uint_as_float((uint32_t)e[t.row0 + r] << 16);
     } else if (t.kind == TK_ATTN) {
       notify = false;  // the last chunk to arrive notifies
       attention_task<HD>(P, S, t, ar, i);
@@ -928,25 +992,38 @@ __host__ __device__ constexpr int pow2_floor_c(int x) { return x < 2 ? 1 : 2 * p
 __host__ __device__ constexpr int stage_rows(int K) {
   return pow2_floor_c((kSlotBytes / (2 * K)) < kRpsMax ? (kSlotBytes / (2 * K)) : kRpsMax);
 }
-#define MK_VARIANT(H, F, D) {seg_count(H), stage_rows(H), seg_count(F), stage_rows(F), D}
-#define MK_KERNEL(H, F, D) (const void*)decode_kernel<seg_count(H), stage_rows(H), seg_count(F), stage_rows(F), D>
+// Batch width 1 streams W_down whole (K = ffn); batch width 4 streams it in K chunks of
+// kDownChunk columns, so the K = ffn class is the chunk's.
+__host__ __device__ constexpr int down_k(int F, int BM) { return BM == 1 ? F : (F < kDownChunk ? F : kDownChunk); }
+#define MK_VARIANT(H, F, D, BM) {seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, BM}
+#define MK_KERNEL(H, F, D, BM)                                                                                   \
+  (const void*)decode_kernel<seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, \
+                             BM>
 static const Variant kVariants[] = {
-    MK_VARIANT(4096, 14336, 128),  // Llama-3-8B shape
-    MK_VARIANT(4096, 11008, 128),  // Chameleon-7B shape
-    MK_VARIANT(256, 768, 64),      // tiny decoder
-    MK_VARIANT(4096, 4096, 128),
-    MK_VARIANT(2048, 4096, 128),
-    MK_VARIANT(256, 256, 64),
+    MK_VARIANT(4096, 14336, 128, 1),  // Llama-3-8B shape
+    MK_VARIANT(4096, 11008, 128, 1),  // Chameleon-7B shape
+    MK_VARIANT(256, 768, 64, 1),      // tiny decoder
+    MK_VARIANT(4096, 4096, 128, 1),
+    MK_VARIANT(2048, 4096, 128, 1),
+    MK_VARIANT(256, 256, 64, 1),
+    MK_VARIANT(4096, 4096, 128, 4),   // hidden 4096, any ffn >= 4096 (Llama-3-8B, Chameleon-7B), 2..4 sequences
+    MK_VARIANT(256, 768, 64, 4),      // tiny decoder, 2..4 sequences
+    MK_VARIANT(2048, 4096, 128, 4),
+    MK_VARIANT(256, 256, 64, 4),
 };
 static const void* kFns[] = {
-    MK_KERNEL(4096, 14336, 128), MK_KERNEL(4096, 11008, 128), MK_KERNEL(256, 768, 64),
-    MK_KERNEL(4096, 4096, 128),  MK_KERNEL(2048, 4096, 128),  MK_KERNEL(256, 256, 64),
+    MK_KERNEL(4096, 14336, 128, 1), MK_KERNEL(4096, 11008, 128, 1), MK_KERNEL(256, 768, 64, 1),
+    MK_KERNEL(4096, 4096, 128, 1),  MK_KERNEL(2048, 4096, 128, 1),  MK_KERNEL(256, 256, 64, 1),
+    MK_KERNEL(4096, 4096, 128, 4),  MK_KERNEL(256, 768, 64, 4),     MK_KERNEL(2048, 4096, 128, 4),
+    MK_KERNEL(256, 256, 64, 4),
 };
+static_assert(sizeof(kVariants) / sizeof(kVariants[0]) == sizeof(kFns) / sizeof(kFns[0]), "variant table");
 
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim) {
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm) {
   for (int i = 0; i < (int)(sizeof(kVariants) / sizeof(kVariants[0])); ++i) {
     const Variant& v = kVariants[i];
-    if (v.nseg_h == nseg_h && v.rps_h == rps_h && v.nseg_f == nseg_f && v.rps_f == rps_f && v.head_dim == head_dim)
+    if (v.nseg_h == nseg_h && v.rps_h == rps_h && v.nseg_f == nseg_f && v.rps_f == rps_f && v.head_dim == head_dim &&
+        v.bm == bm)
       return i;
   }
   return -1;

@@ -47,6 +47,9 @@ struct mk_ctx {
   int variant = -1;
   int G = 1, rows_qkv = 0, rows_gu = 0, nch = 1, n_lm = 0;
   int nseg_h = 0, rps_h = 0, nseg_f = 0, rps_f = 0;
+  int bm = 1;              // batch width of the decode kernel (1, or 4 with masking)
+  int kdc = 0, ndc = 1;    // down-projection K chunk and chunk count (ndc > 1 when bm > 1)
+  int task_rows = kTaskRows;  // rows per GEMV task (kTaskRows / bm)
   // events
   int n_events = 0, ev_lm = 0;
   Graph g;
@@ -105,7 +108,8 @@ int ev_down(const mk_ctx* c, int l) { return ev_base(c, l) + c->cfg.n_kv_heads +
 // Split `total` rows over the SMs in contiguous ranges (multiples of gran) proportional to
 // the per-SM weights (equal weights: balanced), and each range into tasks of at most
 // kTaskRows rows.
-std::vector<std::vector<std::pair<int, int>>> partition_rows(int total, int gran, const std::vector<double>& w) {
+std::vector<std::vector<std::pair<int, int>>> partition_rows(int total, int gran, const std::vector<double>& w,
+                                                             int max_rows) {
   const int n_sms = (int)w.size();
   std::vector<std::vector<std::pair<int, int>>> out(n_sms);
   std::vector<double> cum(n_sms + 1, 0.0);
@@ -119,14 +123,14 @@ std::vector<std::vector<std::pair<int, int>>> partition_rows(int total, int gran
     int b = bound(s + 1);
     int n = b - a;
     if (n <= 0) continue;
-    int nt = (n + kTaskRows - 1) / kTaskRows;
+    int nt = (n + max_rows - 1) / max_rows;
     for (;;) {
       bool ok = true;
       std::vector<std::pair<int, int>> parts;
       for (int i = 0; i < nt; ++i) {
         int lo = (int)(((long long)n * i / nt) / gran * gran);
         int hi = (i + 1 == nt) ? n : (int)(((long long)n * (i + 1) / nt) / gran * gran);
-        if (hi - lo > kTaskRows) ok = false;
+        if (hi - lo > max_rows) ok = false;
         if (hi > lo) parts.push_back({a + lo, hi - lo});
       }
       if (ok) {
@@ -227,7 +231,7 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
     }
     if (t.kind < TK_EMBED || t.kind > TK_LMHEAD) return fail(c, MK_ERR_INVALID_ARG, "unknown task kind");
     int rows = rows_of(t.kind);
-    if (t.nrows <= 0 || t.nrows > kTaskRows || t.row0 < 0 || t.row0 + t.nrows > rows)
+    if (t.nrows <= 0 || t.nrows > c->task_rows || t.row0 < 0 || t.row0 + t.nrows > rows)
       return fail(c, MK_ERR_INVALID_ARG, "task rows out of range");
     if ((t.kind == TK_QKV || t.kind == TK_GATEUP) && ((t.row0 | t.nrows) & 1))
       return fail(c, MK_ERR_INVALID_ARG, "QKV/gate-up tasks must hold whole row pairs");
@@ -244,8 +248,9 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
       auto& v = cover[(size_t)kind * (L + 1) + l];
       int rows = rows_of(kind);
       if ((int)v.size() != rows) return fail(c, MK_ERR_INVALID_ARG, "an op has no tasks");
+      const int want = (kind == TK_DOWN) ? c->ndc : 1;  // one down task per K chunk
       for (int r = 0; r < rows; ++r)
-        if (v[r] != 1) {
+        if (v[r] != want) {
           snprintf(buf, sizeof buf, "op kind %d layer %d: row %d covered %d times", kind, l, r, v[r]);
           return fail(c, MK_ERR_INVALID_ARG, buf);
         }
@@ -424,7 +429,7 @@ int build_graph(mk_ctx* c) {
 
   // embedding slices
   {
-    auto parts = partition_rows(f.hidden, 1, c->sm_weights);
+    auto parts = partition_rows(f.hidden, 1, c->sm_weights, c->task_rows);
     for (int s = 0; s < n; ++s)
       for (auto& p : parts[s]) {
         Task t = make_task(TK_EMBED, 0, p.first, p.second);
@@ -433,10 +438,10 @@ int build_graph(mk_ctx* c) {
         q[s].push_back(t);
       }
   }
-  auto qkv_parts = partition_rows(c->rows_qkv, 2, c->sm_weights);
-  auto o_parts = partition_rows(f.hidden, 1, c->sm_weights);
-  auto gu_parts = partition_rows(c->rows_gu, 2, c->sm_weights);
-  auto d_parts = partition_rows(f.hidden, 1, c->sm_weights);
+  auto qkv_parts = partition_rows(c->rows_qkv, 2, c->sm_weights, c->task_rows);
+  auto o_parts = partition_rows(f.hidden, 1, c->sm_weights, c->task_rows);
+  auto gu_parts = partition_rows(c->rows_gu, 2, c->sm_weights, c->task_rows);
+  auto d_parts = partition_rows(f.hidden, 1, c->sm_weights, c->task_rows);
   const int n_attn = B * nkv * c->nch;
   for (int l = 0; l < L; ++l) {
     for (int s = 0; s < n; ++s)
@@ -479,16 +484,18 @@ int build_graph(mk_ctx* c) {
         q[s].push_back(t);
       }
     for (int s = 0; s < n; ++s)
-      for (auto& p : d_parts[s]) {
-        Task t = make_task(TK_DOWN, l, p.first, p.second);
-        add_wait(t, ev_gu(c, l));
-        add_notify(t, ev_down(c, l));
-        evc[ev_down(c, l)]++;
-        q[s].push_back(t);
-      }
+      for (auto& p : d_parts[s])
+        for (int kc = 0; kc < c->ndc; ++kc) {  // K chunks of the same rows run back to back
+          Task t = make_task(TK_DOWN, l, p.first, p.second);
+          t.aux = (uint16_t)kc;
+          add_wait(t, ev_gu(c, l));
+          add_notify(t, ev_down(c, l));
+          evc[ev_down(c, l)]++;
+          q[s].push_back(t);
+        }
   }
   {
-    auto parts = partition_rows(f.vocab, 1, c->sm_weights);
+    auto parts = partition_rows(f.vocab, 1, c->sm_weights, c->task_rows);
     int idx = 0;
     for (int s = 0; s < n; ++s)
       for (auto& p : parts[s]) {
@@ -510,7 +517,11 @@ int build_graph(mk_ctx* c) {
       c->g.tasks.push_back({t, s});
       switch (t.kind) {
         case TK_QKV: case TK_OPROJ: case TK_GATEUP: case TK_LMHEAD: wbytes += (uint64_t)t.nrows * f.hidden * 2; break;
-        case TK_DOWN: wbytes += (uint64_t)t.nrows * f.ffn * 2; break;
+        case TK_DOWN: {
+          const int k0 = t.aux * c->kdc;
+          wbytes += (uint64_t)t.nrows * std::min(c->kdc, f.ffn - k0) * 2;
+          break;
+        }
       }
     }
   }
@@ -698,15 +709,23 @@ int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
     int by_len = std::max(1, (f.max_seq + 15) / 16);
     c->nch = std::min(std::min(per, by_len), kMaxChunks);
   }
+  // batch width: 1, or 4 (sequences beyond the active batch masked); with 4 the
+  // down projection runs in K chunks of kDownChunk so its activations fit in registers
+  c->bm = (f.max_batch > 1) ? 4 : 1;
+  c->task_rows = kTaskRows / c->bm;
+  c->kdc = (c->bm > 1) ? std::min(f.ffn, kDownChunk) : f.ffn;
+  c->ndc = (f.ffn + c->kdc - 1) / c->kdc;
   c->nseg_h = (f.hidden + kSegElems - 1) / kSegElems;
-  c->nseg_f = (f.ffn + kSegElems - 1) / kSegElems;
+  c->nseg_f = (c->kdc + kSegElems - 1) / kSegElems;
   c->rps_h = pow2_floor(std::min(kRpsMax, kSlotBytes / (f.hidden * 2)));
-  c->rps_f = pow2_floor(std::min(kRpsMax, kSlotBytes / (f.ffn * 2)));
-  if (f.ffn * 2 > kSlotBytes || f.hidden * 2 > kSlotBytes) {
+  c->rps_f = pow2_floor(std::min(kRpsMax, kSlotBytes / (c->kdc * 2)));
+  // the GEMV takes every segment but the last of a K chunk as full
+  const bool ragged_chunk = c->ndc > 1 && f.ffn - (c->ndc - 1) * c->kdc < (c->nseg_f - 1) * kSegElems;
+  if ((f.max_batch == 1 && f.ffn * 2 > kSlotBytes) || f.hidden * 2 > kSlotBytes || ragged_chunk) {
     delete c;
     return fail(nullptr, MK_ERR_UNSUPPORTED, "a weight row does not fit one ring stage");
   }
-  c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim);
+  c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm);
   c->sm_weights.assign(c->n_sms, 1.0);
   rc = build_graph(c);
   if (rc) {
@@ -780,7 +799,22 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
       return MK_ERR_CUDA;
     if (!cuda_ok(c, cudaMemcpy(A + lo.gu, gu.data(), gu.size() * 2, cudaMemcpyHostToDevice), "gate/up copy"))
       return MK_ERR_CUDA;
-    if (!put(lo.o, w->wo[l], (size_t)H * nq * D * 2) || !put(lo.d, w->wd[l], (size_t)H * F * 2) ||
+    if (c->ndc > 1) {
+      // W_down chunk-major: chunk k holds columns [k*kdc, k*kdc + kc) of every row, contiguous
+      std::vector<uint16_t> dk((size_t)H * c->kdc);
+      for (int k = 0; k < c->ndc; ++k) {
+        const int k0 = k * c->kdc, kc = std::min(c->kdc, F - k0);
+        for (int r = 0; r < H; ++r)
+          std::memcpy(&dk[(size_t)r * kc], w->wd[l] + (size_t)r * F + k0, (size_t)kc * 2);
+        if (!cuda_ok(c, cudaMemcpy(A + lo.d + (size_t)H * k0 * 2, dk.data(), (size_t)H * kc * 2,
+                                   cudaMemcpyHostToDevice),
+                     "down chunk copy"))
+          return MK_ERR_CUDA;
+      }
+    } else if (!put(lo.d, w->wd[l], (size_t)H * F * 2)) {
+      return MK_ERR_CUDA;
+    }
+    if (!put(lo.o, w->wo[l], (size_t)H * nq * D * 2) ||
         !put(lo.attn_norm, w->attn_norm[l], (size_t)H * 2) || !put(lo.mlp_norm, w->mlp_norm[l], (size_t)H * 2))
       return MK_ERR_CUDA;
   }
@@ -842,6 +876,8 @@ int mk_prefill(mk_ctx* c, const int32_t* tokens, int B, int T, void* kv_cache, f
   p.max_batch = f.max_batch;
   p.eps = f.rms_eps;
   p.attn_scale = 1.0f / std::sqrt((float)f.head_dim);
+  p.kdc = c->kdc;
+  p.ndc = c->ndc;
   std::string err;
   int rc = run_prefill(p, tokens, B, T, last_logits, reinterpret_cast<cudaStream_t>(stream), &err);
   if (rc) return fail(c, rc, err);
@@ -872,7 +908,7 @@ int mk_decode_step(mk_ctx* c, const int32_t* tokens, void* kv_cache, float* logi
   if (!c->loaded) return fail(c, MK_ERR_STATE, "weights not loaded");
   if (c->B < 1) return fail(c, MK_ERR_STATE, "no active batch (call mk_prefill or mk_set_positions)");
   if (!tokens || !kv_cache || !logits) return fail(c, MK_ERR_INVALID_ARG, "NULL tokens, cache or logits");
-  if (c->variant < 0 || c->B > kMaxDecodeBatch)
+  if (c->variant < 0 || c->B > c->bm)
     return fail(c, MK_ERR_UNSUPPORTED, "no decode kernel instantiation for this shape / batch");
   const mk_config& f = c->cfg;
   for (int b = 0; b < c->B; ++b)
@@ -919,6 +955,9 @@ int mk_decode_step(mk_ctx* c, const int32_t* tokens, void* kv_cache, float* logi
   P.n_lm = c->n_lm;
   P.eps = f.rms_eps;
   P.attn_scale = 1.0f / std::sqrt((float)f.head_dim);
+  P.nb = c->B;
+  P.kdc = c->kdc;
+  P.ndc = c->ndc;
   P.epoch = c->epoch + 1;
   P.ev_lm = (uint32_t)c->ev_lm;
   P.drop_event = c->drop_event;

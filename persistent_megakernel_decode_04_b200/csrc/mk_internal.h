@@ -39,7 +39,8 @@ constexpr int kMaxChunks = 64;                       // split-KV chunks per (seq
 #endif
 constexpr int kSlotBytes = MK_SLOT_KB * 1024;        // one ring stage
 constexpr int kStages = MK_STAGES;                   // ring depth (kStages x kSlotBytes per SM)
-constexpr int kMaxDecodeBatch = 1;                   // CUDA-core path instantiations
+constexpr int kMaxDecodeBatch = 4;                   // CUDA-core path: batch width 1 or 4
+constexpr int kDownChunk = 4096;                     // down-projection K chunk for batch width 4
 
 enum TaskKind : uint8_t {
   TK_EMBED = 1,   // x_0 = E[token] for a slice of rows
@@ -101,6 +102,8 @@ struct DecodeParams {
   uint64_t timeout_ns;
   uint64_t* trace;            // optional [n_tasks][kTraceWords] timing records (null = off)
   int l2_ahead;               // weight stages the producer prefetches into L2 beyond the ring
+  int nb;                     // active sequences (<= the kernel's batch width)
+  int kdc, ndc;               // down-projection K chunk and chunk count
 };
 constexpr uint64_t kStallPrefetchNs = 1000;    // producer blocked this long: prefetch ahead into L2
 constexpr uint64_t kStallPrefetchGapNs = 100;   // then one more stage per this interval
@@ -126,9 +129,9 @@ TensorMapEncodeFn get_tensor_map_encoder();
 
 // Kernel variants: one instantiation per (segments, rows per stage) of the two K sizes.
 struct Variant {
-  int nseg_h, rps_h, nseg_f, rps_f, head_dim;
+  int nseg_h, rps_h, nseg_f, rps_f, head_dim, bm;
 };
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim);
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm);
 const void* decode_kernel_ptr(int variant);
 size_t decode_smem_bytes();
 int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t stream, std::string* err);
@@ -155,6 +158,7 @@ struct PrefillParams {
   int rows_cap;
   int H, nq, nkv, D, F, V, L, max_seq, max_batch;
   float eps, attn_scale;
+  int kdc, ndc;  // W_down stored in ndc chunk-major K chunks of kdc columns
 };
 int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, float* last_logits,
                 cudaStream_t stream, std::string* err);

@@ -54,11 +54,12 @@ __global__ void rmsnorm(const float* X, const uint16_t* g, float* Y, int H, floa
   for (int i = threadIdx.x; i < H; i += blockDim.x) Y[(size_t)row * H + i] = x[i] * r * bf(g[i]);
 }
 
-// Y[n][N] (row stride ldy) = A[n][K] (fp32) . W[N][K]^T (bf16), fp32 accumulation.
-// 64 x 64 output tile per block, 256 threads x (4 x 4) outputs, K tile 32.
+// Y[n][N] (row stride ldy) (+)= A[n][K] (fp32, row stride lda) . W[N][K]^T (bf16), fp32
+// accumulation.  64 x 64 output tile per block, 256 threads x (4 x 4) outputs, K tile 32.
 constexpr int BM = 64, BN = 64, BK = 32;
 __global__ void __launch_bounds__(256) gemm(const float* __restrict__ A, const uint16_t* __restrict__ W,
-                                            float* __restrict__ Y, int n, int N, int K, int ldy) {
+                                            float* __restrict__ Y, int n, int N, int K, int lda, int ldy,
+                                            int accumulate) {
   __shared__ float As[BK][BM + 4];
   __shared__ float Ws[BK][BN + 4];
   const int tid = threadIdx.x;
@@ -70,7 +71,7 @@ __global__ void __launch_bounds__(256) gemm(const float* __restrict__ A, const u
     for (int e = tid; e < BM * BK; e += 256) {
       const int r = e / BK, k = e % BK;
       const int gr = m0 + r, gk = k0 + k;
-      As[k][r] = (gr < n && gk < K) ? A[(size_t)gr * K + gk] : 0.f;
+      As[k][r] = (gr < n && gk < K) ? A[(size_t)gr * lda + gk] : 0.f;
     }
     for (int e = tid; e < BN * BK; e += 256) {
       const int r = e / BK, k = e % BK;
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(256) gemm(const float* __restrict__ A, const u
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int gc = n0 + tx * 4 + j;
-      if (gc < N) Y[(size_t)gr * ldy + gc] = acc[i][j];
+      if (gc < N) Y[(size_t)gr * ldy + gc] = accumulate ? Y[(size_t)gr * ldy + gc] + acc[i][j] : acc[i][j];
     }
   }
 }
@@ -218,9 +219,10 @@ static bool ck(cudaError_t e, const char* what, std::string* err) {
   return false;
 }
 
-static void gemm(const float* A, const uint16_t* W, float* Y, int n, int N, int K, int ldy, cudaStream_t s) {
+static void gemm(const float* A, const uint16_t* W, float* Y, int n, int N, int K, int ldy, cudaStream_t s,
+                 int lda = -1, int accumulate = 0) {
   dim3 grid((N + pf::BN - 1) / pf::BN, (n + pf::BM - 1) / pf::BM);
-  pf::gemm<<<grid, 256, 0, s>>>(A, W, Y, n, N, K, ldy);
+  pf::gemm<<<grid, 256, 0, s>>>(A, W, Y, n, N, K, lda < 0 ? K : lda, ldy, accumulate);
 }
 
 int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, float* last_logits, cudaStream_t s,
@@ -256,7 +258,10 @@ int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, flo
       pf::rmsnorm<<<n, 256, 0, s>>>(p.X, mn, p.XN, H, p.eps, 1, 0);
       gemm(p.XN, reinterpret_cast<const uint16_t*>(p.arena + lo.gu), p.Y, n, 2 * F, H, 2 * F, s);
       pf::swiglu<<<n, 256, 0, s>>>(p.Y, p.HH, F);
-      gemm(p.HH, reinterpret_cast<const uint16_t*>(p.arena + lo.d), p.Y, n, H, F, H, s);
+      for (int k = 0; k < p.ndc; ++k) {  // W_down in chunk-major K chunks (one chunk when unsplit)
+        const int k0 = k * p.kdc, kc = (F - k0) < p.kdc ? (F - k0) : p.kdc;
+        gemm(p.HH + k0, reinterpret_cast<const uint16_t*>(p.arena + lo.d) + (size_t)H * k0, p.Y, n, H, kc, H, s, F, k);
+      }
       pf::residual_add<<<256, 256, 0, s>>>(p.X, p.Y, (size_t)n * H);
     }
     if (!ck(cudaGetLastError(), "prefill chunk", err)) return MK_ERR_CUDA;

@@ -170,6 +170,22 @@ __device__ __forceinline__ void fma2_bf16w(uint64_t& acc, uint32_t w, uint64_t x
       : "r"(w), "l"(xpair));
 }
 
+// The two bf16 weights of word w widened exactly into an fp32 pair (for reuse across rows of x).
+__device__ __forceinline__ uint64_t widen_bf16w(uint32_t w) {
+  uint64_t r;
+  asm("{\n\t.reg .b32 lo, hi;\n\t"
+      "shl.b32 lo, %1, 16;\n\t"
+      "and.b32 hi, %1, 0xffff0000;\n\t"
+      "mov.b64 %0, {lo, hi};\n\t}"
+      : "=l"(r)
+      : "r"(w));
+  return r;
+}
+// acc += wp * xpair, both fp32 pairs.
+__device__ __forceinline__ void fma2_pair(uint64_t& acc, uint64_t wp, uint64_t xpair) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(wp), "l"(xpair));
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 

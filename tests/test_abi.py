@@ -56,11 +56,12 @@ def test_decode_before_load_is_a_state_error():
         mk.mk_destroy(ctx)
 
 
-@pytest.fixture(params=["tiny", "llama3-8b", "chameleon-7b-b1"])
+@pytest.fixture(params=["tiny", "llama3-8b", "chameleon-7b-b1", "tiny-b4", "llama3-8b-b4", "chameleon-7b-b4"])
 def graph(request):
+    name, B = (request.param[:-3], 4) if request.param.endswith("-b4") else (request.param, 1)
     shape, ms = {"tiny": (mi.TINY, 64), "llama3-8b": (mi.LLAMA8B, 1024),
-                 "chameleon-7b-b1": (mi.CHAMELEON7B, 1280)}[request.param]
-    ctx = mk.mk_build_taskgraph(mk.Config.from_shape(shape, 1, ms).c(), -1)
+                 "chameleon-7b-b1": (mi.CHAMELEON7B, 1280), "chameleon-7b": (mi.CHAMELEON7B, 1280)}[name]
+    ctx = mk.mk_build_taskgraph(mk.Config.from_shape(shape, B, ms).c(), -1)
     tasks, counts = mk.mk_export_taskgraph(ctx)
     yield ctx, tasks, counts, shape
     mk.mk_destroy(ctx)
@@ -75,8 +76,11 @@ def test_built_graph_validates_and_balances_bytes(graph):
     per_layer = ((s.n_q_heads + 2 * s.n_kv_heads) * s.head_dim * s.hidden + s.hidden * s.n_q_heads * s.head_dim
                  + 2 * s.ffn * s.hidden + s.hidden * s.ffn) * 2
     assert info["weight_bytes_per_step"] == s.n_layers * per_layer + s.vocab * s.hidden * 2
-    # each SM streams nearly the same number of weight bytes (within 3 %)
-    K = {2: s.hidden, 4: s.hidden, 5: s.hidden, 6: s.ffn, 7: s.hidden}
+    # each SM streams nearly the same number of weight bytes (within 3 %); with more than one
+    # sequence the down projection runs in K chunks, one task per chunk of the same rows
+    down = tasks[tasks[:, 0] == 6]
+    ndc = len(down) // len({(int(t[1]), int(t[3])) for t in down})
+    K = {2: s.hidden, 4: s.hidden, 5: s.hidden, 6: s.ffn / ndc, 7: s.hidden}
     per_sm = np.zeros(info["n_sms"])
     for t in tasks:
         if t[0] in K:

@@ -40,3 +40,31 @@ def test_llama8b_prompt39_decode(w8b):
     n = 39 + steps
     kv_close(m.kv_view()[:, :, :1, :, :n, :].cpu().numpy(), ref.get_cache(n), "kv cache")
     m.close()
+
+
+def test_llama8b_4096_context(w8b):
+    """Long context: 4096 cached positions (a seeded synthetic cache standing in for the
+    4096-token prompt), 2 decode steps; split-KV attention spans every chunk."""
+    w = w8b
+    s = w.shape
+    L, steps, max_seq = 4096, 2, 4112
+    kv = mi.kv_cache_values(4, s, 1, L, sigma=1.0)
+    ref = oracle.Decoder(w, 1, max_seq)
+    ref.set_cache(kv, L)
+    m = mk.Megakernel(mk.Config.from_shape(s, 1, max_seq), w, 0)
+    m.kv_view()[:, :, :1, :, :L, :] = torch.from_numpy(kv.view(np.int16)).to(DEV)
+    del kv
+    m.set_positions([L])
+    tok = int(mi.prompt(4, 0, 1, s.vocab)[0])
+    for i in range(steps):
+        rl = ref.decode(np.array([tok], dtype=np.int32))[0]
+        g, nt = m.decode(torch.tensor([tok], dtype=torch.int32, device=DEV))
+        g = g[0].cpu().numpy()
+        logits_close(g, rl, f"step {i}")
+        assert argmax_agrees(g, rl, int(nt[0].item()))
+        tok = oracle.argmax(rl)
+    assert m.sync_status() == mk.MK_OK
+    n = L + steps
+    got = m.kv_view()[:, :, :1, :, L:n, :].cpu().numpy()
+    kv_close(got, ref.get_cache(n)[:, :, :, :, L:n], "kv cache (appended positions)")
+    m.close()

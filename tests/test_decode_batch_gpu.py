@@ -1,0 +1,124 @@
+"""Batched decode (2..4 sequences per step) against the CPU oracle, teacher-forced per
+sequence on the oracle's tokens: per-step logits of every sequence, argmax, the bf16 KV
+cache, masking of sequences outside the active batch and per-sequence positions."""
+import numpy as np
+import pytest
+import torch
+
+import mk_inputs as mi
+import oracle
+import persistent_megakernel_decode_04_b200 as mk
+from _parity import argmax_agrees, kv_close, logits_close
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+
+
+def _model(weights, max_batch, max_seq):
+    return mk.Megakernel(mk.Config.from_shape(weights.shape, max_batch, max_seq), weights, 0)
+
+
+def _step_both(ref, m, toks, label):
+    """One decode step on both sides with the same per-sequence tokens; returns the oracle's picks."""
+    B = len(toks)
+    rl = ref.decode(np.array(toks, dtype=np.int32))
+    gl, nt = m.decode(torch.tensor(toks, dtype=torch.int32, device=DEV))
+    gl, nt = gl[:B].cpu().numpy(), nt[:B].cpu().numpy()
+    for b in range(B):
+        logits_close(gl[b], rl[b], f"{label} seq {b}")
+        assert argmax_agrees(gl[b], rl[b], int(nt[b])), f"{label} seq {b}: argmax differs with a clear margin"
+    return [oracle.argmax(rl[b]) for b in range(B)]
+
+
+def _teacher_forced_batch(w, B, max_batch, T, steps, max_seq, seed):
+    prompts = np.stack([mi.prompt(seed, b, T, w.shape.vocab) for b in range(B)])
+    ref = oracle.Decoder(w, B, max_seq)
+    m = _model(w, max_batch, max_seq)
+    rl = ref.prefill(prompts)
+    gl = m.prefill(torch.from_numpy(prompts.astype(np.int32)).to(DEV)).cpu().numpy()
+    for b in range(B):
+        logits_close(gl[b], rl[b], f"prefill seq {b}")
+    toks = [oracle.argmax(rl[b]) for b in range(B)]
+    for i in range(steps):
+        toks = _step_both(ref, m, toks, f"step {i}")
+    assert m.sync_status() == mk.MK_OK
+    n = T + steps
+    kv_close(m.kv_view()[:, :, :B, :, :n, :].cpu().numpy(), ref.get_cache(n), "kv cache")
+    m.close()
+
+
+def test_tiny_batch4_prefill_and_16_steps():
+    w = mi.make_weights(mi.TINY, seed=5)
+    _teacher_forced_batch(w, B=4, max_batch=4, T=12, steps=16, max_seq=64, seed=5)
+
+
+@pytest.mark.parametrize("B", [1, 2, 3])
+def test_tiny_partial_batch_is_masked(B):
+    # the batch-4 kernel serving fewer sequences: the unused slots compute nothing visible
+    w = mi.make_weights(mi.TINY, seed=6)
+    _teacher_forced_batch(w, B=B, max_batch=4, T=9, steps=6, max_seq=32, seed=6 + B)
+
+
+def test_tiny_batch4_ragged_positions():
+    # every sequence at its own position: RoPE angle, cache slot and attention length per sequence
+    w = mi.make_weights(mi.TINY, seed=7)
+    s = w.shape
+    L = 50
+    kv = mi.kv_cache_values(7, s, 4, L, sigma=1.0)
+    pos = [50, 17, 33, 1]
+    ref = oracle.Decoder(w, 4, 64)
+    ref.set_cache(kv, L)
+    ref.set_positions(pos)
+    m = _model(w, 4, 64)
+    m.kv_view()[:, :, :4, :, :L, :] = torch.from_numpy(kv.view(np.int16)).to(DEV)
+    m.set_positions(pos)
+    toks = [3, 99, 512, 1000]
+    for i in range(6):
+        toks = _step_both(ref, m, toks, f"step {i}")
+    assert m.sync_status() == mk.MK_OK
+    got = m.kv_view()[:, :, :4, :, :57, :].cpu().numpy()
+    want = ref.get_cache(57)
+    for b in range(4):  # compare each sequence over the positions it has written or read
+        n = pos[b] + 6
+        kv_close(got[:, :, b : b + 1, :, :n], want[:, :, b : b + 1, :, :n], f"kv cache seq {b}")
+
+
+def test_batch_beyond_kernel_width_is_rejected():
+    # 5..16 sequences need the tensor-core projection path; the CUDA-core kernel refuses them
+    w = mi.make_weights(mi.TINY, seed=8)
+    m = _model(w, 8, 16)
+    prompts = np.stack([mi.prompt(8, b, 4, w.shape.vocab) for b in range(8)])
+    m.prefill(torch.from_numpy(prompts.astype(np.int32)).to(DEV))
+    with pytest.raises(mk.MkError) as e:
+        m.decode(torch.zeros(8, dtype=torch.int32, device=DEV))
+    assert e.value.code == mk.MK_ERR_UNSUPPORTED
+    m.close()
+
+
+@pytest.fixture(scope="module")
+def w_chameleon():
+    return mi.make_weights(mi.CHAMELEON7B, seed=0)
+
+
+@pytest.mark.parametrize("B", [1, 4])
+def test_chameleon7b_1024_context(w_chameleon, B):
+    """Chameleon-7B-shaped MHA decoder, every sequence at 1024 cached positions (a seeded
+    synthetic cache standing in for the 1024-token prompts), 2 decode steps."""
+    w = w_chameleon
+    s = w.shape
+    L, steps, max_seq = 1024, 2, 1040
+    kv = mi.kv_cache_values(11, s, B, L, sigma=1.0)
+    ref = oracle.Decoder(w, B, max_seq)
+    ref.set_cache(kv, L)
+    m = _model(w, B, max_seq)
+    m.kv_view()[:, :, :B, :, :L, :] = torch.from_numpy(kv.view(np.int16)).to(DEV)
+    del kv
+    m.set_positions([L] * B)
+    toks = [int(t) for t in mi.prompt(11, 0, B, s.vocab)]
+    for i in range(steps):
+        toks = _step_both(ref, m, toks, f"step {i}")
+    assert m.sync_status() == mk.MK_OK
+    n = L + steps
+    got = m.kv_view()[:, :, :B, :, L:n, :].cpu().numpy()
+    kv_close(got, ref.get_cache(n)[:, :, :, :, L:n], "kv cache (appended positions)")
+    m.close()

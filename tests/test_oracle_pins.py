@@ -333,6 +333,26 @@ def test_set_cache_then_decode_equals_prefill_then_decode(tiny_weights):
     assert np.array_equal(b.decode(toks[8:9]), want)
 
 
+def test_per_sequence_positions_equal_separate_decoders(tiny_weights):
+    # two sequences at different positions in one batch: each row equals a one-sequence
+    # decoder whose prompt ends at that position (entries past a position are ignored)
+    w = tiny_weights
+    pa, pb = mi.prompt(0, 9, 10, w.shape.vocab), mi.prompt(0, 10, 4, w.shape.vocab)
+    ra, rb = oracle.Decoder(w, 1, 16), oracle.Decoder(w, 1, 16)
+    ra.prefill(pa[:-1])
+    rb.prefill(pb[:-1])
+    kva, kvb = ra.get_cache(9), rb.get_cache(9)  # rb's entries 3..8 are zero padding
+    both = oracle.Decoder(w, 2, 16)
+    both.set_cache(np.concatenate([kva, kvb], axis=2), 9)
+    both.set_positions([9, 3])
+    assert (both.position(0), both.position(1)) == (9, 3)
+    got = both.decode(np.array([pa[-1], pb[-1]], dtype=np.int32))
+    assert np.array_equal(got[0], ra.decode(pa[-1:])[0])
+    assert np.array_equal(got[1], rb.decode(pb[-1:])[0])
+    with pytest.raises(ValueError):
+        both.set_positions([17, 0])  # beyond max_seq
+
+
 def test_thread_count_does_not_change_results(tiny_weights):
     w = mi.make_weights(mi.TINY.with_layers(1), seed=1)
     toks = mi.prompt(0, 8, 5, w.shape.vocab)
