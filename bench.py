@@ -8,6 +8,13 @@ and K timed steps follow the prompt, so positions 39 .. 39+W+K-1 are decoded (th
 W=8, K=504 is the 512-step run of that workload).  The weights stream from HBM every step
 (15 GB > the 126 MB L2), so no L2 flush is needed between steps.
 
+Other workloads of the same decoder family (`--workload`, each printing its own line; the
+default is the one above): `llama8b-ctx4096` (8B shape, batch 1, every step attending over
+4096+ cached positions) and `chameleon7b-b1` / `-b4` / `-b16` (Chameleon-7B-shaped MHA
+decoder, 1, 4 or 16 sequences each at 1024+ cached positions; 16 sequences run the
+projections on the tensor cores).  Their caches are seeded synthetic values standing in for
+the prefilled prompts.
+
 Multi-GPU (torchrun, one process per GPU): independent replicas, no collective on the data
 path; the timed region is bracketed by a barrier and a device synchronise on every rank and
 the slowest rank's time is reported.  `--impl reference` times the CPU oracle instead.
@@ -34,6 +41,24 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 
 
+# name: (shape name, sequences, cached positions before decoding (0 = prefill the 39-token prompt))
+WORKLOADS = {
+    "llama8b": ("LLAMA8B", 1, 0),
+    "llama8b-ctx4096": ("LLAMA8B", 1, 4096),
+    "chameleon7b-b1": ("CHAMELEON7B", 1, 1024),
+    "chameleon7b-b4": ("CHAMELEON7B", 4, 1024),
+    "chameleon7b-b16": ("CHAMELEON7B", 16, 1024),
+}
+WORKLOAD_TEXT = {
+    "llama8b": "llama3-8b-shape decode, batch 1, 39-token prompt, greedy",
+    "llama8b-ctx4096": "llama3-8b-shape decode, batch 1, 4096 cached positions (synthetic), greedy",
+    "chameleon7b-b1": "chameleon-7b-shape MHA decode, batch 1, 1024 cached positions (synthetic), greedy",
+    "chameleon7b-b4": "chameleon-7b-shape MHA decode, batch 4, 1024 cached positions each (synthetic), greedy",
+    "chameleon7b-b16": "chameleon-7b-shape MHA decode, batch 16 (tensor-core projections), 1024 cached positions "
+                       "each (synthetic), greedy",
+}
+
+
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -44,6 +69,7 @@ def parse():
     p.add_argument("--e2e-steps", type=int, default=64)
     p.add_argument("--no-calibrate", action="store_true",
                    help="keep equal rows per SM instead of the schedule calibrated during warm-up")
+    p.add_argument("--workload", default="llama8b", choices=sorted(WORKLOADS))
     p.add_argument("--layers", type=int, default=0,
                    help="truncate the decoder to this many layers (profiling captures of a small case); "
                         "0 = the full 32-layer workload")
@@ -77,6 +103,12 @@ def algorithmic_bytes(shape, positions):
     weights = s.n_layers * per_layer + (s.vocab * s.hidden + s.hidden) * 2 + s.hidden * 2
     kv = [s.n_layers * 2 * s.n_kv_heads * (p + 1) * D * 2 for p in positions]
     return weights, kv
+
+
+def workload_metric(name):
+    if name == "llama8b":
+        return METRIC
+    return f"decode ms/step + achieved HBM GB/s (% of peak), {name}, 1 B200"
 
 
 def kernel_source_hash():
@@ -236,20 +268,34 @@ def run_mk(args, rank, world, local):
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600),
                                 device_id=dev)
-    shape = mi.LLAMA8B if args.layers <= 0 else mi.LLAMA8B.with_layers(args.layers)
+    shape_name, B, ctx0 = WORKLOADS[args.workload]
+    base = getattr(mi, shape_name)
+    shape = base if args.layers <= 0 else base.with_layers(args.layers)
     total_steps = args.warmup + args.steps
-    max_seq = PROMPT_LEN + total_steps + args.e2e_steps + 8
+    max_seq = (ctx0 or PROMPT_LEN) + total_steps + args.e2e_steps + 8
     os.environ.setdefault("MK_INPUT_THREADS", str(max(1, (os.cpu_count() or 1) // max(1, world))))
     weights = mi.make_weights(shape, seed=0)
     stream = torch.cuda.current_stream(dev)
-    m = mk.Megakernel(mk.Config.from_shape(shape, 1, max_seq), weights, local, stream=stream)
+    m = mk.Megakernel(mk.Config.from_shape(shape, B, max_seq), weights, local, stream=stream)
     info = m.info()
-    keep_weights = rank == 0 and not args.no_cpu_baseline
-    if not keep_weights:
+    cpu_baseline = rank == 0 and not args.no_cpu_baseline and args.workload == "llama8b"
+    if not cpu_baseline:
         del weights
-    prompt = torch.from_numpy(mi.prompt(0, 0, PROMPT_LEN, shape.vocab)[None].astype(np.int32)).to(dev)
-    logits = m.prefill(prompt)
-    tok = torch.argmax(logits[0]).to(torch.int32).reshape(1)
+    if ctx0 == 0:
+        prompt = torch.from_numpy(mi.prompt(0, 0, PROMPT_LEN, shape.vocab)[None].astype(np.int32)).to(dev)
+        logits = m.prefill(prompt)
+        tok = torch.argmax(logits[0]).to(torch.int32).reshape(1)
+    else:
+        # seeded synthetic cache standing in for the prefilled prompts, filled layer by layer
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1234)
+        kvv = m.kv_view()
+        for l in range(shape.n_layers):
+            vals = torch.randn((2, B, shape.n_kv_heads, ctx0, shape.head_dim), generator=gen, device=dev)
+            kvv[l, :, :B, :, :ctx0, :] = vals.to(torch.bfloat16).view(torch.int16)
+            del vals
+        m.set_positions([ctx0] * B)
+        tok = torch.from_numpy(mi.prompt(0, 0, B, shape.vocab).astype(np.int32)).to(dev)
     warm = args.warmup
     calibrated = False
     if not args.no_calibrate and warm >= 6:
@@ -293,12 +339,12 @@ def run_mk(args, rank, world, local):
 
     # end to end through the C ABI with host buffers: token in from pinned host memory,
     # logits and next token back to pinned host memory, every step
-    host_tok = torch.zeros(1, dtype=torch.int32, pin_memory=True)
-    host_logits = torch.empty(shape.vocab, dtype=torch.float32, pin_memory=True)
-    host_next = torch.zeros(1, dtype=torch.int32, pin_memory=True)
-    dev_tok = torch.zeros(1, dtype=torch.int32, device=dev)
-    host_tok[0] = int(tok.item())
-    m.set_positions([pos0 + args.steps])
+    host_tok = torch.zeros(B, dtype=torch.int32, pin_memory=True)
+    host_logits = torch.empty((B, shape.vocab), dtype=torch.float32, pin_memory=True)
+    host_next = torch.zeros(B, dtype=torch.int32, pin_memory=True)
+    dev_tok = torch.zeros(B, dtype=torch.int32, device=dev)
+    host_tok.copy_(tok.cpu())
+    m.set_positions([pos0 + args.steps] * B)
     n_e2e = min(args.e2e_steps, max_seq - (pos0 + args.steps) - 1)
     if world > 1:
         dist.barrier()
@@ -309,10 +355,10 @@ def run_mk(args, rank, world, local):
     for _ in range(n_e2e):
         dev_tok.copy_(host_tok, non_blocking=True)
         lg, nt = m.decode(dev_tok)
-        host_logits.copy_(lg[0], non_blocking=True)
+        host_logits.copy_(lg, non_blocking=True)
         host_next.copy_(nt, non_blocking=True)
         stream.synchronize()
-        host_tok[0] = host_next[0]
+        host_tok.copy_(host_next)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
@@ -326,35 +372,38 @@ def run_mk(args, rank, world, local):
     if rank == 0:
         positions = list(range(pos0, pos0 + args.steps))
         wbytes, kvbytes = algorithmic_bytes(shape, positions)
-        alg = wbytes + float(np.mean(kvbytes))
+        alg = wbytes + B * float(np.mean(kvbytes))  # every sequence attends over its own cache
         mean_ms = float(step_ms.mean())
         peak, peak_kind = measured_peaks()
         achieved = alg / (mean_ms * 1e-3) / 1e9
-        traffic, traffic_note = profiled_traffic(alg)
-        value = max_ms / (args.steps * world)  # whole job: slowest rank's time over all ranks' tokens
+        traffic, traffic_note = profiled_traffic(alg) if args.workload == "llama8b" else (None, "no ncu summary")
+        # whole job: slowest rank's time over all ranks' steps (replicas decode concurrently)
+        value = max_ms / (args.steps * world)
         out = {
-            "metric": METRIC, "value": value, "unit": "ms/token", "n_gpus": world, "steps": args.steps,
+            "metric": workload_metric(args.workload), "value": value,
+            "unit": "ms/token" if B == 1 else "ms/step", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded random weights)",
-            "config": {"workload": "llama3-8b-shape decode, batch 1, 39-token prompt, greedy"
+            "config": {"workload": WORKLOAD_TEXT[args.workload]
                                    + ("" if args.layers <= 0 else f" (truncated to {args.layers} layers)"),
-                       "prompt_len": PROMPT_LEN, "decode_positions": [pos0, pos0 + args.steps - 1],
-                       "global_batch": world, "parallelism": "replicas", "weights": "bf16",
+                       "prompt_len": PROMPT_LEN if ctx0 == 0 else None, "cached_positions": ctx0 or None,
+                       "decode_positions": [pos0, pos0 + args.steps - 1], "batch_per_gpu": B,
+                       "global_batch": world * B, "parallelism": "replicas", "weights": "bf16",
                        "schedule": "calibrated per-SM rows" if calibrated else "equal rows per SM",
                        "l2": "inputs larger than L2 (15 GB of weights streamed per step)"},
-            "ms_per_token_p50": float(np.median(step_ms)), "tokens_per_s": 1e3 / (max_ms / args.steps) * world,
+            "ms_per_step_p50": float(np.median(step_ms)), "tokens_per_s": 1e3 / (max_ms / args.steps) * world * B,
             "hbm_gbs": achieved, "hbm_frac_of_measured": achieved / peak, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,
             "bound_ms_at_8tbs": alg / NOMINAL_HBM_GBS / 1e6,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": alg, "traffic_note": traffic_note},
-            "e2e": {"value": (e2e_max / n_e2e) if n_e2e > 0 else None, "unit": "ms/token", "h2d_bytes_per_step": 4,
-                    "d2h_bytes_per_step": shape.vocab * 4 + 4, "steps": n_e2e},
+            "e2e": {"value": (e2e_max / n_e2e) if n_e2e > 0 else None, "unit": "ms/token" if B == 1 else "ms/step",
+                    "h2d_bytes_per_step": 4 * B, "d2h_bytes_per_step": B * (shape.vocab * 4 + 4), "steps": n_e2e},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
             "kernel": {"n_sms": info["n_sms"], "n_tasks": info["n_tasks"], "smem_bytes": info["smem_bytes"]},
         }
-        if not args.no_cpu_baseline:
+        if cpu_baseline:
             ms, cores, n = oracle_ms_per_token(weights, shape)
             out["cpu_baseline"] = {
                 "value": ms, "unit": "ms/token", "cores": cores, "kind": "oracle",

@@ -31,11 +31,13 @@
 
 namespace mk {
 
+// Dynamic shared memory: the weight ring (nst stages of kSlotBytes, 1024-aligned), then for
+// the tensor-core kernel the activation operand (kTcBopBytes), then DSmem.
 struct DSmem {
-  uint8_t ring[kStages][kSlotBytes];
   union {
     float red[kWorkerWarps][kTaskRows];  // GEMV: per-warp sums of the current task, [row][seq]
     float aacc[kAttnWarps][4][128];      // attention: per-warp partial outputs
+    float tile[kTcRecFloats];            // tensor-core tile: summed partial records
   };
   float tot[kTaskRows];                  // totals of the current task, [row][seq]
   float ssw[kWorkerWarps][kMaxDecodeBatch];  // per-warp sums of x^2 per sequence
@@ -44,15 +46,21 @@ struct DSmem {
   float mm[4 * kMaxChunks], ll[4 * kMaxChunks], ww[4 * kMaxChunks];  // split-KV merge
   float lmv[kWorkerWarps];
   int lmi[kWorkerWarps];
+  float tss[kTcBatch];       // tensor-core task: per-sequence sum of x^2 over its K range
   uint64_t full[kStages];
   uint64_t empty[kStages];
+  uint64_t mma_done;         // tensor-core task: its MMAs completed
+  uint32_t tmem;             // tensor-memory accumulator address
   uint32_t ready;            // tasks [0, ready) of this queue have their inputs
   uint32_t cabort;           // worker-role abort: written before, read after a worker barrier
   volatile uint32_t abort;   // any role gave up: stop waiting
   uint32_t flag;             // worker broadcast (last-arriver decisions)
 };
 
-size_t decode_smem_bytes() { return sizeof(DSmem) + 1024; }
+__host__ __device__ constexpr int ring_stages(bool tc) { return tc ? kTcStages : kStages; }
+__host__ __device__ constexpr size_t ring_bytes(bool tc) {
+  return (size_t)ring_stages(tc) * kSlotBytes + (tc ? (size_t)kTcBopBytes : 0);
+}
 
 __device__ __forceinline__ void worker_bar() { named_bar_sync(1, kWorkerThreads); }
 
@@ -84,8 +92,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_
 struct Pipe {
   int stage;
   uint32_t phase;
+  int nst;  // ring depth
   __device__ __forceinline__ void advance() {
-    if (++stage == kStages) {
+    if (++stage == nst) {
       stage = 0;
       phase ^= 1u;
     }
@@ -108,9 +117,22 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
   return (uint16_t)(u >> 16);
 }
 
-// Which stream a GEMV task reads: arena offset and row length (bytes) for the task's op.
+// Which stream a GEMV task reads: arena offset and row length (bytes) for the task's op.  A
+// tensor-core task streams whole weight blocks: row0 counts blocks of kSlotBytes.
+template <bool TC>
 __device__ __forceinline__ void gemv_source(const DecodeParams& P, const Task& t, uint64_t* off, uint32_t* row_bytes) {
   const LayerOff& lo = P.loff[t.layer < P.L ? t.layer : 0];
+  if (TC) {
+    switch (t.kind) {
+      case TK_QKV: *off = lo.qkv; break;
+      case TK_OPROJ: *off = lo.o; break;
+      case TK_GATEUP: *off = lo.gu; break;
+      case TK_DOWN: *off = lo.d; break;
+      default: *off = P.off_lm; break;
+    }
+    *row_bytes = (uint32_t)kSlotBytes;
+    return;
+  }
   switch (t.kind) {
     case TK_QKV: *off = lo.qkv; *row_bytes = (uint32_t)P.H * 2u; break;
     case TK_OPROJ: *off = lo.o; *row_bytes = (uint32_t)P.H * 2u; break;
@@ -169,7 +191,8 @@ __device__ __forceinline__ void warp_reduce_rows(float (&a)[V], float* out, int 
 // S.tot.  Also leaves the per-warp sums of x_b^2 in S.ssw for the fused norm.  Returns false
 // (for every worker thread alike) if a wait ran out.
 template <int NSEG, int RPS, int BM>
-__device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe& pp, const float* __restrict__ xsrc,
+__device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe& pp, const uint8_t* ring,
+                                          const float* __restrict__ xsrc,
                                           int xstride, int nb, const uint16_t* __restrict__ gain, int K, int nrows,
                                           uint32_t row_bytes, uint32_t task_id, uint32_t& stall_ns) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -217,7 +240,7 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
       S.cabort = 1u;
     }
     if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
-    const uint8_t* base = S.ring[pp.stage] + tid * 16;
+    const uint8_t* base = ring + (size_t)pp.stage * kSlotBytes + tid * 16;
     uint64_t acc[RPS][BM];  // per (row, sequence): (even, odd) partial sums
 #pragma unroll
     for (int rr = 0; rr < RPS; ++rr) {
@@ -285,16 +308,12 @@ __device__ __forceinline__ float norm_factor(const DSmem& S, int K, float eps, i
 // ---------------------------------------------------------------------------------------
 // Epilogues: thread e < nrows * BM handles row row0 + e / BM of sequence b = e % BM, whose
 // GEMV total is S.tot[e] (sequences b >= nb are skipped).
-template <int BM>
-__device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, const Task& t, float r) {
-  const int tid = threadIdx.x;
-  const int b = tid % BM;
-  if (tid >= (int)t.nrows * BM || b >= P.nb) return;
+// Packed QKV row R of sequence b (value v; other = its RoPE partner row R ^ 1): q rows go to
+// qbuf after RoPE, k rows after RoPE and v rows as they are into the bf16 cache at pos[b].
+__device__ __forceinline__ void qkv_out(const DecodeParams& P, int layer, int R, int b, float v, float other) {
   const int D = P.D, G = P.nq / P.nkv, half = D / 2;
   const int rpg = (G + 2) * D;
-  const int R = (int)t.row0 + tid / BM;
   const int grp = R / rpg, rr = R % rpg;
-  const float v = S.tot[tid] * r;
   const int pos = P.pos[b];
   const size_t head_stride = (size_t)P.max_seq * D;
   const size_t kv_layer = (size_t)P.max_batch * P.nkv * head_stride;  // one of K or V, one layer
@@ -302,7 +321,6 @@ __device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, c
     // q or k: rows come in RoPE pairs (i, i + D/2) at packed positions (2i, 2i+1)
     const int pd = (rr < G * D) ? (rr % D) : (rr - G * D);
     const int i = pd >> 1, hi = pd & 1;
-    const float other = S.tot[tid ^ BM] * r;  // the RoPE partner row, same sequence
     const float2 cs = P.rope[(size_t)pos * half + i];
     float outv;
     int dim;
@@ -315,16 +333,25 @@ __device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, c
     }
     if (rr < G * D) {
       const int hq = grp * G + rr / D;
-      P.qbuf[((size_t)t.layer * P.B + b) * P.nq * D + (size_t)hq * D + dim] = outv;
+      P.qbuf[((size_t)layer * P.B + b) * P.nq * D + (size_t)hq * D + dim] = outv;
     } else {
-      uint16_t* kc = P.kv + ((size_t)t.layer * 2 + 0) * kv_layer + ((size_t)b * P.nkv + grp) * head_stride;
+      uint16_t* kc = P.kv + ((size_t)layer * 2 + 0) * kv_layer + ((size_t)b * P.nkv + grp) * head_stride;
       kc[(size_t)pos * D + dim] = f2bf(outv);
     }
   } else {
     const int dim = rr - (G + 1) * D;
-    uint16_t* vc = P.kv + ((size_t)t.layer * 2 + 1) * kv_layer + ((size_t)b * P.nkv + grp) * head_stride;
+    uint16_t* vc = P.kv + ((size_t)layer * 2 + 1) * kv_layer + ((size_t)b * P.nkv + grp) * head_stride;
     vc[(size_t)pos * D + dim] = f2bf(v);
   }
+}
+
+template <int BM>
+__device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, const Task& t, float r) {
+  const int tid = threadIdx.x;
+  const int b = tid % BM;
+  if (tid >= (int)t.nrows * BM || b >= P.nb) return;
+  // the RoPE partner row (R ^ 1) of the same sequence sits at tid ^ BM
+  qkv_out(P, t.layer, (int)t.row0 + tid / BM, b, S.tot[tid] * r, S.tot[tid ^ BM] * r);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -674,18 +701,289 @@ __device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, cons
 }
 
 // ---------------------------------------------------------------------------------------
+// Tensor-core projection task (batch width kTcBatch): D[128 rows x 32] = W_tile . [x_hi | x_lo]^T
+// over the task's K units, on tcgen05 with the accumulator in tensor memory.
+//
+// Operands.  A = a block of kTcRows x kTcUnitK bf16 weights straight from the ring stage (the
+// host stores every projection as such blocks, no-swizzle K-major core matrices: 8 rows x 16
+// bytes contiguous, 16 core matrices per 8-row group along K).  B = the activations of up to
+// 16 sequences times the norm gain, each split into a bf16 high part and a bf16 low part (the
+// rounding residual), so the product keeps about 16 mantissa bits of x; columns 0..15 are the
+// high parts, 16..31 the low parts.  D[r][b] + D[r][16 + b] is row r of sequence b.
+//
+// Split K.  An op's blocks (tile, K unit) are spread evenly over the SMs, so a tile's K range
+// can be covered by several tasks on several SMs.  Each task writes its partial [128][16] and
+// its per-sequence sum of x^2 to its own record; the last task of the tile to arrive (arrival
+// counter) sums the tile's records in slot order (deterministic), applies the fused norm
+// factor and runs the op's epilogue.  Every task notifies the op's event after it finishes,
+// so the event completes only after the last arriver's epilogue.
+constexpr uint32_t kTcIdesc = (1u << 4)                       // D: fp32
+                              | (1u << 7) | (1u << 10)        // A, B: bf16
+                              | ((uint32_t)(kTcN >> 3) << 17)   // N
+                              | ((uint32_t)(kTcRows >> 4) << 24);  // M (A and B K-major: bits 15, 16 = 0)
+
+__device__ __forceinline__ float bf2f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+__device__ __forceinline__ void warp_argmax(float& v, int& idx) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1)
+    argmax_merge(v, idx, __shfl_xor_sync(0xffffffffu, v, off), __shfl_xor_sync(0xffffffffu, idx, off));
+}
+
+__device__ __forceinline__ bool tc_task(const DecodeParams& P, DSmem& S, Pipe& pp, const uint8_t* ring,
+                                        uint8_t* bop, const Task& t, const LayerOff& lo, uint32_t task_id,
+                                        uint32_t& stall_ns, uint32_t& mma_phase, uint32_t tmem) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t lay = (size_t)t.layer * P.B;
+  const float* xs;
+  const uint16_t* gain = nullptr;
+  int K = P.H, xstride = P.H, rows;
+  switch (t.kind) {
+    case TK_QKV:
+      xs = P.x_in + lay * P.H;
+      gain = reinterpret_cast<const uint16_t*>(P.arena + lo.attn_norm);
+      rows = (P.nq + 2 * P.nkv) * P.D;
+      break;
+    case TK_OPROJ:
+      xs = P.obuf + lay * P.nq * P.D;
+      K = xstride = P.nq * P.D;
+      rows = P.H;
+      break;
+    case TK_GATEUP:
+      xs = P.x_mid + lay * P.H;
+      gain = reinterpret_cast<const uint16_t*>(P.arena + lo.mlp_norm);
+      rows = 2 * P.F;
+      break;
+    case TK_DOWN:
+      xs = P.hbuf + lay * P.F;
+      K = xstride = P.F;
+      rows = P.H;
+      break;
+    default:  // LM head
+      xs = P.x_in + (size_t)P.L * P.B * P.H;
+      gain = reinterpret_cast<const uint16_t*>(P.arena + P.off_fnorm);
+      rows = P.V;
+      break;
+  }
+  const int nK = (K + kTcUnitK - 1) / kTcUnitK;
+  const int tile = (int)t.row0 / nK, u0 = (int)t.row0 % nK, nu = (int)t.nrows;
+  const int k0 = u0 * kTcUnitK, ngroups = nu * (kTcUnitK / 8);
+
+  // 1. activation operand: warp w stages sequences w and w + 8, lane j the 8-element K groups
+  //    j, j + 32, ...; sequences outside the active batch and K past the end are zeros
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int b = warp + h * kWorkerWarps;
+    const bool act = b < P.nb;
+    const float* xb = xs + (size_t)b * xstride;
+    float ss = 0.f;
+    for (int j = lane; j < ngroups; j += 32) {
+      const int k = k0 + j * 8;
+      float x[8];
+      if (act && k < K) {
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(xb + k));
+        const float4 c = __ldcg(reinterpret_cast<const float4*>(xb + k + 4));
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+        if (gain) {
+          const uint4 g = __ldg(reinterpret_cast<const uint4*>(gain + k));
+          x[0] *= bf16lo(g.x); x[1] *= bf16hi(g.x);
+          x[2] *= bf16lo(g.y); x[3] *= bf16hi(g.y);
+          x[4] *= bf16lo(g.z); x[5] *= bf16hi(g.z);
+          x[6] *= bf16lo(g.w); x[7] *= bf16hi(g.w);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = 0.f;
+      }
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint16_t h0 = f2bf(x[2 * q]), h1 = f2bf(x[2 * q + 1]);
+        const uint16_t l0 = f2bf(x[2 * q] - bf2f(h0)), l1 = f2bf(x[2 * q + 1] - bf2f(h1));
+        hw[q] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+        lw[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+      }
+      const int hrow = b, lrow = kTcBatch + b;  // operand rows (MMA N index)
+      *reinterpret_cast<uint4*>(bop + (hrow >> 3) * kTcBopSbo + j * 128 + (hrow & 7) * 16) =
+          make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(bop + (lrow >> 3) * kTcBopSbo + j * 128 + (lrow & 7) * 16) =
+          make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (lane == 0) S.tss[b] = ss;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  worker_bar();
+  tc_fence_after();
+
+  // 2. one thread issues the MMAs of every K unit as its weight block lands; each stage is
+  //    released to the producer by a commit once its MMAs are done
+  if (tid == 0) {
+    const uint32_t b_base = smem_u32(bop);
+    for (int u = 0; u < nu; ++u) {
+      const uint64_t tw = P.trace ? globaltimer_ns() : 0;
+      if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
+        raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
+        S.cabort = 1u;
+        break;
+      }
+      if (P.trace) stall_ns += (uint32_t)(globaltimer_ns() - tw);
+      tc_fence_after();
+      const uint32_t a_base = smem_u32(ring + (size_t)pp.stage * kSlotBytes);
+#pragma unroll
+      for (int s = 0; s < kTcUnitK / 16; ++s) {
+        // K step s: core-matrix columns 2s, 2s + 1 (256 bytes) of the block / of unit u
+        const uint64_t ad = tc_smem_desc(a_base + s * 256, 128, (kTcUnitK / 8) * 128);
+        const uint64_t bd = tc_smem_desc(b_base + u * (kTcUnitK / 8) * 128 + s * 256, 128, kTcBopSbo);
+        tc_mma_f16(tmem, ad, bd, kTcIdesc, (u | s) != 0 ? 1u : 0u);
+      }
+      tc_commit(&S.empty[pp.stage]);
+      pp.advance();
+    }
+    tc_commit(&S.mma_done);
+  }
+  // 3. every worker waits for the MMAs (time-bounded only: they end within microseconds once
+  //    issued, and tensor memory must not be read or freed before)
+  if (!wait_bar(&S.mma_done, mma_phase, P.timeout_ns, nullptr)) {
+    raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
+    S.cabort = 1u;
+  }
+  mma_phase ^= 1u;
+  tc_fence_after();
+  worker_bar();
+  if (S.cabort) return false;
+
+  // 4. partial record: warps 0-3 read their 32 TMEM lanes (= rows), 32 columns each
+  float* rec = P.tpart + (size_t)t.index * kTcRecFloats;
+  if (warp < 4) {
+    float d[32];
+    tc_ld32(tmem + ((uint32_t)(warp * 32) << 16), d);
+    float4* dst = reinterpret_cast<float4*>(rec + (warp * 32 + lane) * kTcBatch);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_float4(d[4 * q] + d[kTcBatch + 4 * q], d[4 * q + 1] + d[kTcBatch + 4 * q + 1],
+                           d[4 * q + 2] + d[kTcBatch + 4 * q + 2], d[4 * q + 3] + d[kTcBatch + 4 * q + 3]);
+  }
+  if (tid < kTcBatch) rec[kTcRows * kTcBatch + tid] = S.tss[tid];
+  tc_fence_before();
+  worker_bar();
+  if (tid == 0) {
+    const uint32_t old = atom_acq_rel_gpu_add(&P.tcnt[t.pad1], 1u);
+    S.flag = (old + 1u == P.epoch * (uint32_t)t.pad0) ? 1u : 0u;
+  }
+  worker_bar();
+  if (!S.flag) return true;
+
+  // 5. last arriver: the tile's records in slot order
+  const float* rec0 = P.tpart + (size_t)(t.index - t.aux) * kTcRecFloats;
+  for (int e = tid; e < kTcRecFloats; e += kWorkerThreads) {
+    float v = 0.f;
+    for (int sl = 0; sl < (int)t.pad0; ++sl) v += __ldcg(rec0 + (size_t)sl * kTcRecFloats + e);
+    S.tile[e] = v;
+  }
+  worker_bar();
+  const float* ssum = S.tile + kTcRows * kTcBatch;
+
+  // 6. epilogue: thread tid handles (row, sequence) pairs e = tid + i * 256, e = row * 16 + b
+  if (t.kind == TK_LMHEAD) {
+    for (int e = tid; e < kTcRows * kTcBatch; e += kWorkerThreads) {
+      const int row = e / kTcBatch, b = e % kTcBatch, R = tile * kTcRows + row;
+      if (b < P.nb && R < rows)
+        P.logits[(size_t)b * P.V + R] = S.tile[e] / sqrtf(ssum[b] / (float)K + P.eps);
+    }
+    // per-sequence argmax over the tile: warp w takes sequences w and w + 8
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int b = warp + h * kWorkerWarps;
+      if (b < P.nb) {
+        const float r = 1.0f / sqrtf(ssum[b] / (float)K + P.eps);
+        float v = -INFINITY;
+        int idx = 0x7fffffff;
+        for (int row = lane; row < kTcRows; row += 32) {
+          const int R = tile * kTcRows + row;
+          if (R < rows) argmax_merge(v, idx, S.tile[row * kTcBatch + b] * r, R);
+        }
+        warp_argmax(v, idx);
+        if (lane == 0) {
+          P.lm_val[(size_t)tile * P.B + b] = v;
+          P.lm_idx[(size_t)tile * P.B + b] = idx;
+        }
+      }
+    }
+    worker_bar();
+    if (tid == 0) {
+      const uint32_t old = atom_acq_rel_gpu_add(&P.ev[P.ev_lm], 1u);
+      S.flag = (old + 1u == P.epoch * (uint32_t)P.n_lm) ? 1u : 0u;
+    }
+    worker_bar();
+    if (S.flag && P.next_tokens) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int b = warp + h * kWorkerWarps;
+        if (b < P.nb) {
+          float v = -INFINITY;
+          int idx = 0x7fffffff;
+          for (int i = lane; i < P.n_lm; i += 32)
+            argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
+          warp_argmax(v, idx);
+          if (lane == 0) P.next_tokens[b] = idx;
+        }
+      }
+    }
+    return true;
+  }
+  for (int e = tid; e < kTcRows * kTcBatch; e += kWorkerThreads) {
+    const int row = e / kTcBatch, b = e % kTcBatch, R = tile * kTcRows + row;
+    if (b >= P.nb || R >= rows) continue;
+    const float r = gain ? 1.0f / sqrtf(ssum[b] / (float)K + P.eps) : 1.f;
+    const float v = S.tile[e] * r;
+    switch (t.kind) {
+      case TK_QKV: qkv_out(P, t.layer, R, b, v, S.tile[e ^ kTcBatch] * r); break;  // partner row R ^ 1
+      case TK_OPROJ: {
+        const size_t at = (lay + b) * P.H + R;
+        P.x_mid[at] = __ldcg(P.x_in + at) + v;
+        break;
+      }
+      case TK_GATEUP:
+        if ((R & 1) == 0) {
+          const float uv = S.tile[e + kTcBatch] * r;
+          P.hbuf[(lay + b) * P.F + R / 2] = v / (1.f + expf(-v)) * uv;
+        }
+        break;
+      default: {  // down
+        const size_t at = (lay + b) * P.H + R;
+        P.x_in[P.B * P.H + at] = __ldcg(P.x_mid + at) + v;
+        break;
+      }
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------------------
 template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM>
 __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
+  constexpr bool TC = BM > kMaxDecodeBatch;  // tensor-core projection tiles
+  constexpr int BMC = TC ? 1 : BM;            // CUDA-core GEMV batch width (unused when TC)
+  constexpr int NST = ring_stages(TC);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  DSmem& S = *reinterpret_cast<DSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  uint8_t* const ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* const bop = ring + (size_t)NST * kSlotBytes;  // tensor-core activation operand
+  DSmem& S = *reinterpret_cast<DSmem*>(ring + ring_bytes(TC));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t qb = P.qbegin[blockIdx.x], qe = P.qbegin[blockIdx.x + 1];
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], kWorkerWarps);
+      mbar_init(&S.empty[s], TC ? 1 : kWorkerWarps);  // tensor-core stages: released by a commit
     }
+    mbar_init(&S.mma_done, 1);
     S.ready = 0;
     S.cabort = 0;
     S.abort = 0;
@@ -713,11 +1011,11 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
           la_row = 0;
           continue;
         }
-        const uint32_t rps = (la_t.kind == TK_DOWN) ? (uint32_t)RPS_F : (uint32_t)RPS_H;
+        const uint32_t rps = TC ? 1u : (la_t.kind == TK_DOWN) ? (uint32_t)RPS_F : (uint32_t)RPS_H;
         if (prefetch) {
           uint64_t off;
           uint32_t rb;
-          gemv_source(P, la_t, &off, &rb);
+          gemv_source<TC>(P, la_t, &off, &rb);
           const uint32_t nr = min(rps, la_t.nrows - la_row);
           prefetch_l2(P.arena + off + (uint64_t)(la_t.row0 + la_row) * rb, nr * rb);
         }
@@ -726,7 +1024,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
       }
       return false;
     };
-    Pipe pp{0, 0};
+    Pipe pp{0, 0, NST};
     int issued = 0;
     bool ok = true;
     for (uint32_t i = qb; i < qe && ok; ++i) {
@@ -734,8 +1032,8 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
       if (!is_gemv(t.kind)) continue;
       uint64_t off;
       uint32_t rb;
-      gemv_source(P, t, &off, &rb);
-      const int rps = (t.kind == TK_DOWN) ? RPS_F : RPS_H;
+      gemv_source<TC>(P, t, &off, &rb);
+      const int rps = TC ? 1 : (t.kind == TK_DOWN) ? RPS_F : RPS_H;
       const uint8_t* src = P.arena + off + (uint64_t)t.row0 * rb;
       uint64_t blocked = 0, first = 0;
       for (uint32_t r0 = 0; r0 < t.nrows; r0 += (uint32_t)rps) {
@@ -765,7 +1063,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
           if (r0 == 0) first = now;
         }
         mbar_arrive_expect_tx(&S.full[pp.stage], nr * rb);
-        bulk_g2s(S.ring[pp.stage], src + (uint64_t)r0 * rb, nr * rb, &S.full[pp.stage], pol);
+        bulk_g2s(ring + (size_t)pp.stage * kSlotBytes, src + (uint64_t)r0 * rb, nr * rb, &S.full[pp.stage], pol);
         ++issued;
         // the lookahead cursor stays at or in front of the next ring stage
         if (P.l2_ahead > 0) {
@@ -780,11 +1078,11 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
       }
     }
     // leave no copy in flight: wait (bounded) for the last issued stages to land
-    for (int k = 1; k <= (issued < kStages ? issued : kStages); ++k) {
+    for (int k = 1; k <= (issued < NST ? issued : NST); ++k) {
       int s = pp.stage - k;
       uint32_t ph = pp.phase;
       if (s < 0) {
-        s += kStages;
+        s += NST;
         ph ^= 1u;
       }
       wait_bar(&S.full[s], ph, P.timeout_ns, nullptr);
@@ -837,7 +1135,18 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
   }
 
   // --------------------------------- workers ---------------------------------
-  Pipe pp{0, 0};
+  Pipe pp{0, 0, NST};
+  uint32_t tmem = 0, mma_phase = 0;
+  if (TC) {  // one 32-column fp32 accumulator (128 lanes) for the whole kernel
+    if (warp == 0) {
+      tc_alloc(&S.tmem, kTcN);
+      tc_relinquish();
+    }
+    tc_fence_before();
+    worker_bar();
+    tc_fence_after();
+    tmem = S.tmem;
+  }
   // descriptor (and layer offsets) of the next task are loaded while the worker still waits
   // for that task's inputs, so only the activation loads remain after the release
   Task t_next = P.tasks[qb < qe ? qb : 0];
@@ -874,7 +1183,10 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     }
     const uint64_t t_ready = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     bool notify = true;
-    if (is_gemv(t.kind)) {
+    if (TC && is_gemv(t.kind)) {
+      if (!tc_task(P, S, pp, ring, bop, t, lo, i, stall, mma_phase, tmem)) goto out;
+      if (t.kind == TK_LMHEAD) notify = false;
+    } else if (is_gemv(t.kind)) {
       // operands of the task's GEMV: x source of sequence 0 and the stride to the next, norm
       // gain (null = no norm) and K
       const float* xs;
@@ -909,18 +1221,20 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
       uint32_t rb;
       {
         uint64_t off_unused;
-        gemv_source(P, t, &off_unused, &rb);
+        gemv_source<false>(P, t, &off_unused, &rb);
       }
       const bool ok = (t.kind == TK_DOWN)
-                          ? gemv_tile<NSEG_F, RPS_F, BM>(P, S, pp, xs, xstride, P.nb, gain, K, (int)t.nrows, rb, i, stall)
-                          : gemv_tile<NSEG_H, RPS_H, BM>(P, S, pp, xs, xstride, P.nb, gain, K, (int)t.nrows, rb, i, stall);
+                          ? gemv_tile<NSEG_F, RPS_F, BMC>(P, S, pp, ring, xs, xstride, P.nb, gain, K, (int)t.nrows, rb,
+                                                         i, stall)
+                          : gemv_tile<NSEG_H, RPS_H, BMC>(P, S, pp, ring, xs, xstride, P.nb, gain, K, (int)t.nrows, rb,
+                                                         i, stall);
       if (!ok) goto out;
       // this thread's (row, sequence) in the epilogues
-      const int eb = tid % BM, er = tid / BM;
+      const int eb = tid % BMC, er = tid / BMC;
       const bool mine = er < (int)t.nrows && eb < P.nb;
       const float r = gain ? norm_factor(S, K, P.eps, eb) : 1.f;
       switch (t.kind) {
-        case TK_QKV: epi_qkv<BM>(P, S, t, r); break;
+        case TK_QKV: epi_qkv<BMC>(P, S, t, r); break;
         case TK_OPROJ:
           if (mine) {
             const size_t at = (lay + eb) * P.H + t.row0 + er;
@@ -929,7 +1243,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
           break;
         case TK_GATEUP:
           if (mine && (er & 1) == 0) {
-            const float gv = S.tot[tid] * r, uv = S.tot[tid + BM] * r;
+            const float gv = S.tot[tid] * r, uv = S.tot[tid + BMC] * r;
             const float sg = gv / (1.f + expf(-gv));
             P.hbuf[(lay + eb) * P.F + (t.row0 + er) / 2] = sg * uv;
           }
@@ -946,7 +1260,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
           break;
         default:
           notify = false;
-          epi_lmhead<BM>(P, S, t, K);
+          epi_lmhead<BMC>(P, S, t, K);
           break;
       }
     } else if (t.kind == TK_EMBED) {
@@ -980,7 +1294,12 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     }
   }
 out:
-  return;
+  if (TC) {  // every worker thread arrives here together; no MMA is in flight
+    tc_fence_before();
+    worker_bar();
+    tc_fence_after();
+    if (warp == 0) tc_dealloc(tmem, kTcN);
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1010,12 +1329,15 @@ static const Variant kVariants[] = {
     MK_VARIANT(256, 768, 64, 4),      // tiny decoder, 2..4 sequences
     MK_VARIANT(2048, 4096, 128, 4),
     MK_VARIANT(256, 256, 64, 4),
+    {0, 1, 0, 1, 128, kTcBatch},      // tensor-core projection tiles, 5..16 sequences, any hidden / ffn
+    {0, 1, 0, 1, 64, kTcBatch},
 };
 static const void* kFns[] = {
     MK_KERNEL(4096, 14336, 128, 1), MK_KERNEL(4096, 11008, 128, 1), MK_KERNEL(256, 768, 64, 1),
     MK_KERNEL(4096, 4096, 128, 1),  MK_KERNEL(2048, 4096, 128, 1),  MK_KERNEL(256, 256, 64, 1),
     MK_KERNEL(4096, 4096, 128, 4),  MK_KERNEL(256, 768, 64, 4),     MK_KERNEL(2048, 4096, 128, 4),
     MK_KERNEL(256, 256, 64, 4),
+    (const void*)decode_kernel<1, 1, 1, 1, 128, kTcBatch>, (const void*)decode_kernel<1, 1, 1, 1, 64, kTcBatch>,
 };
 static_assert(sizeof(kVariants) / sizeof(kVariants[0]) == sizeof(kFns) / sizeof(kFns[0]), "variant table");
 
@@ -1031,9 +1353,14 @@ int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_d
 
 const void* decode_kernel_ptr(int variant) { return kFns[variant]; }
 
+size_t decode_smem_bytes(int variant) {
+  const bool tc = variant >= 0 && kVariants[variant].bm > kMaxDecodeBatch;
+  return ring_bytes(tc) + sizeof(DSmem) + 1024;  // + alignment of the ring to 1024 bytes
+}
+
 int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t stream, std::string* err) {
   const void* fn = kFns[variant];
-  const size_t smem = decode_smem_bytes();
+  const size_t smem = decode_smem_bytes(variant);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) {
     void* args[] = {const_cast<DecodeParams*>(&p)};

@@ -49,7 +49,12 @@ struct mk_ctx {
   int nseg_h = 0, rps_h = 0, nseg_f = 0, rps_f = 0;
   int bm = 1;              // batch width of the decode kernel (1, or 4 with masking)
   int kdc = 0, ndc = 1;    // down-projection K chunk and chunk count (ndc > 1 when bm > 1)
-  int task_rows = kTaskRows;  // rows per GEMV task (kTaskRows / bm)
+  int task_rows = kTaskRows;  // rows per GEMV task (kTaskRows / bm); tensor-core: K units per task
+  // tensor-core projection tiles (max_batch > 4): weights in kTcRows x kTcUnitK blocks
+  bool tc = false;
+  int tc_nk[8] = {0}, tc_tiles[8] = {0}, tc_tile_base[8] = {0};  // per task kind
+  int n_tile_ids = 0;         // tiles of one layer's projections plus the LM head's
+  size_t rec_cap = 0, n_recs = 0;  // partial records (workspace capacity, in use)
   // events
   int n_events = 0, ev_lm = 0;
   Graph g;
@@ -60,8 +65,8 @@ struct mk_ctx {
   // workspace layout
   size_t ws_tasks = 0, ws_qbegin = 0, ws_evcount = 0, ws_ev = 0, ws_acnt = 0, ws_err = 0, ws_loff = 0, ws_rope = 0,
          ws_xin = 0, ws_xmid = 0, ws_q = 0, ws_o = 0, ws_h = 0, ws_part = 0, ws_lmval = 0, ws_lmidx = 0,
-         ws_pf = 0, ws_bytes = 0;
-  size_t ev_bytes = 0, acnt_bytes = 0;
+         ws_pf = 0, ws_tpart = 0, ws_tcnt = 0, ws_bytes = 0;
+  size_t ev_bytes = 0, acnt_bytes = 0, tcnt_bytes = 0;
   int pf_rows = 0;
   size_t kv_bytes = 0;
   uint64_t weight_bytes_per_step = 0;
@@ -143,6 +148,29 @@ std::vector<std::vector<std::pair<int, int>>> partition_rows(int total, int gran
   return out;
 }
 
+// Tensor-core ops: the op's blocks (tile-major, K unit minor) split over the SMs in
+// contiguous ranges proportional to the per-SM weights; each range cut into tasks at tile
+// boundaries and after kTcUnitsMax units.  Returns per SM the (first block, blocks) pairs.
+std::vector<std::vector<std::pair<int, int>>> partition_blocks(int tiles, int nk, const std::vector<double>& w) {
+  const int n_sms = (int)w.size();
+  const long long total = (long long)tiles * nk;
+  std::vector<std::vector<std::pair<int, int>>> out(n_sms);
+  std::vector<double> cum(n_sms + 1, 0.0);
+  for (int s = 0; s < n_sms; ++s) cum[s + 1] = cum[s] + w[s];
+  auto bound = [&](int s) { return (long long)std::llround(total * (cum[s] / cum[n_sms])); };
+  for (int s = 0; s < n_sms; ++s) {
+    long long a = bound(s);
+    const long long b = bound(s + 1);
+    while (a < b) {
+      const long long tile_end = (a / nk + 1) * nk;
+      const long long e = std::min(std::min(b, tile_end), a + kTcUnitsMax);
+      out[s].push_back({(int)a, (int)(e - a)});
+      a = e;
+    }
+  }
+  return out;
+}
+
 Task make_task(uint8_t kind, int layer, int row0, int nrows) {
   Task t;
   std::memset(&t, 0, sizeof(t));
@@ -151,6 +179,10 @@ Task make_task(uint8_t kind, int layer, int row0, int nrows) {
   t.row0 = (uint32_t)row0;
   t.nrows = (uint32_t)nrows;
   return t;
+}
+
+bool is_gemv_kind(int k) {
+  return k == TK_QKV || k == TK_OPROJ || k == TK_GATEUP || k == TK_DOWN || k == TK_LMHEAD;
 }
 
 void add_wait(Task& t, int e) { t.wait[t.n_wait++] = (uint32_t)e; }
@@ -199,8 +231,18 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
         for (int k = 0; k < t.n_notify; ++k) produced[t.notify[k]]++;
       }
     }
-    for (const VTask& t : T)
-      if (t.kind == TK_LMHEAD) produced[c->ev_lm]++;
+    if (c->tc) {  // the last task of each LM tile counts
+      std::vector<char> seen((size_t)c->tc_tiles[TK_LMHEAD], 0);
+      for (const VTask& t : T)
+        if (t.kind == TK_LMHEAD && t.row0 >= 0 && t.row0 / c->tc_nk[TK_LMHEAD] < c->tc_tiles[TK_LMHEAD] &&
+            !seen[t.row0 / c->tc_nk[TK_LMHEAD]]) {
+          seen[t.row0 / c->tc_nk[TK_LMHEAD]] = 1;
+          produced[c->ev_lm]++;
+        }
+    } else {
+      for (const VTask& t : T)
+        if (t.kind == TK_LMHEAD) produced[c->ev_lm]++;
+    }
   }
   for (int e = 0; e < nE; ++e)
     if (produced[e] != cnt[e]) {
@@ -209,6 +251,7 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
     }
   // (c) every op's rows covered exactly once
   auto rows_of = [&](int kind) -> int {
+    if (c->tc && kind != TK_EMBED) return c->tc_tiles[kind] * c->tc_nk[kind];  // weight blocks
     switch (kind) {
       case TK_EMBED: return f.hidden;
       case TK_QKV: return c->rows_qkv;
@@ -233,7 +276,9 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
     int rows = rows_of(t.kind);
     if (t.nrows <= 0 || t.nrows > c->task_rows || t.row0 < 0 || t.row0 + t.nrows > rows)
       return fail(c, MK_ERR_INVALID_ARG, "task rows out of range");
-    if ((t.kind == TK_QKV || t.kind == TK_GATEUP) && ((t.row0 | t.nrows) & 1))
+    if (c->tc && t.kind != TK_EMBED && t.row0 / c->tc_nk[t.kind] != (t.row0 + t.nrows - 1) / c->tc_nk[t.kind])
+      return fail(c, MK_ERR_INVALID_ARG, "a tensor-core task spans two tiles");
+    if (!c->tc && (t.kind == TK_QKV || t.kind == TK_GATEUP) && ((t.row0 | t.nrows) & 1))
       return fail(c, MK_ERR_INVALID_ARG, "QKV/gate-up tasks must hold whole row pairs");
     int lay = (t.kind == TK_EMBED || t.kind == TK_LMHEAD) ? L : t.layer;
     auto& v = cover[(size_t)t.kind * (L + 1) + lay];
@@ -286,7 +331,13 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
     out.clear();
     out.push_back(cat_of(t.kind, t.layer));
     if (t.kind == TK_QKV) {
-      for (int g = t.row0 / rpg; g <= (t.row0 + t.nrows - 1) / rpg; ++g) out.push_back(cat_qkvg(t.layer, g));
+      int r0 = t.row0, r1 = t.row0 + t.nrows - 1;  // packed rows written (by the tile, for tensor-core tasks)
+      if (c->tc) {
+        const int tile = t.row0 / c->tc_nk[TK_QKV];
+        r0 = tile * kTcRows;
+        r1 = std::min(c->rows_qkv, r0 + kTcRows) - 1;
+      }
+      for (int g = r0 / rpg; g <= r1 / rpg; ++g) out.push_back(cat_qkvg(t.layer, g));
     }
   };
   std::vector<int> tmp;
@@ -438,17 +489,68 @@ int build_graph(mk_ctx* c) {
         q[s].push_back(t);
       }
   }
-  auto qkv_parts = partition_rows(c->rows_qkv, 2, c->sm_weights, c->task_rows);
-  auto o_parts = partition_rows(f.hidden, 1, c->sm_weights, c->task_rows);
-  auto gu_parts = partition_rows(c->rows_gu, 2, c->sm_weights, c->task_rows);
-  auto d_parts = partition_rows(f.hidden, 1, c->sm_weights, c->task_rows);
+  // GEMV ops.  CUDA-core tasks: row ranges (parts = (first row, rows)).  Tensor-core tasks:
+  // block ranges of one tile (parts = (first block, blocks)); the tile's tasks get slots in
+  // SM order, and its partial records are rec0[tile] + slot (the same for every layer).
+  struct Plan {
+    std::vector<std::vector<std::pair<int, int>>> parts;
+    std::vector<std::vector<int>> slot;  // tensor-core: per SM, per part
+    std::vector<int> nsplit, rec0;       // tensor-core: per tile
+  };
+  size_t rec_next = 0;
+  auto plan = [&](int kind, int rows, int gran) {
+    Plan pl;
+    if (!c->tc) {
+      pl.parts = partition_rows(rows, gran, c->sm_weights, c->task_rows);
+      return pl;
+    }
+    const int nk = c->tc_nk[kind], tiles = c->tc_tiles[kind];
+    pl.parts = partition_blocks(tiles, nk, c->sm_weights);
+    pl.nsplit.assign(tiles, 0);
+    pl.slot.resize(n);
+    for (int s = 0; s < n; ++s)
+      for (auto& p : pl.parts[s]) pl.slot[s].push_back(pl.nsplit[p.first / nk]++);
+    pl.rec0.assign(tiles, 0);
+    for (int t = 0; t < tiles; ++t) {
+      pl.rec0[t] = (int)rec_next;
+      rec_next += pl.nsplit[t];
+    }
+    return pl;
+  };
+  auto gemv_task = [&](int kind, int l, const Plan& pl, int s, int j) {
+    const auto& p = pl.parts[s][j];
+    Task t = make_task(kind, l, p.first, p.second);
+    if (c->tc) {
+      const int tile = p.first / c->tc_nk[kind];
+      t.aux = (uint16_t)pl.slot[s][j];
+      t.pad0 = (uint8_t)pl.nsplit[tile];
+      t.index = (uint32_t)(pl.rec0[tile] + pl.slot[s][j]);
+      t.pad1 = (uint32_t)((kind == TK_LMHEAD ? 0 : l) * c->n_tile_ids + c->tc_tile_base[kind] + tile);
+    }
+    return t;
+  };
+  if (c->tc)
+    for (int k : {TK_QKV, TK_OPROJ, TK_GATEUP, TK_DOWN, TK_LMHEAD})
+      if (c->tc_tiles[k] * c->tc_nk[k] > 0 && c->tc_nk[k] > 255)
+        return fail(c, MK_ERR_UNSUPPORTED, "K too large for the tensor-core tile split");
+  const Plan qkv_pl = plan(TK_QKV, c->rows_qkv, 2);
+  const Plan o_pl = plan(TK_OPROJ, f.hidden, 1);
+  const Plan gu_pl = plan(TK_GATEUP, c->rows_gu, 2);
+  const Plan d_pl = plan(TK_DOWN, f.hidden, 1);
+  const Plan lm_pl = plan(TK_LMHEAD, f.vocab, 1);
+  c->n_recs = rec_next;
   const int n_attn = B * nkv * c->nch;
   for (int l = 0; l < L; ++l) {
     for (int s = 0; s < n; ++s)
-      for (auto& p : qkv_parts[s]) {
-        Task t = make_task(TK_QKV, l, p.first, p.second);
+      for (int j = 0; j < (int)qkv_pl.parts[s].size(); ++j) {
+        Task t = gemv_task(TK_QKV, l, qkv_pl, s, j);
         add_wait(t, l == 0 ? ev_embed() : ev_down(c, l - 1));
-        int g0 = p.first / rpg, g1 = (p.first + p.second - 1) / rpg;
+        int r0 = (int)t.row0, r1 = (int)(t.row0 + t.nrows - 1);  // packed rows the task (or its tile) writes
+        if (c->tc) {
+          r0 = (int)t.row0 / c->tc_nk[TK_QKV] * kTcRows;
+          r1 = std::min(c->rows_qkv, r0 + kTcRows) - 1;
+        }
+        const int g0 = r0 / rpg, g1 = r1 / rpg;
         if (g1 - g0 > 1) return fail(c, MK_ERR_UNSUPPORTED, "QKV tile spans more than two KV groups");
         for (int g = g0; g <= g1; ++g) {
           add_notify(t, ev_qkv(c, l, g));
@@ -468,26 +570,26 @@ int build_graph(mk_ctx* c) {
     }
     evc[ev_attn(c, l)] = (uint32_t)(B * nkv);
     for (int s = 0; s < n; ++s)
-      for (auto& p : o_parts[s]) {
-        Task t = make_task(TK_OPROJ, l, p.first, p.second);
+      for (int j = 0; j < (int)o_pl.parts[s].size(); ++j) {
+        Task t = gemv_task(TK_OPROJ, l, o_pl, s, j);
         add_wait(t, ev_attn(c, l));
         add_notify(t, ev_o(c, l));
         evc[ev_o(c, l)]++;
         q[s].push_back(t);
       }
     for (int s = 0; s < n; ++s)
-      for (auto& p : gu_parts[s]) {
-        Task t = make_task(TK_GATEUP, l, p.first, p.second);
+      for (int j = 0; j < (int)gu_pl.parts[s].size(); ++j) {
+        Task t = gemv_task(TK_GATEUP, l, gu_pl, s, j);
         add_wait(t, ev_o(c, l));
         add_notify(t, ev_gu(c, l));
         evc[ev_gu(c, l)]++;
         q[s].push_back(t);
       }
     for (int s = 0; s < n; ++s)
-      for (auto& p : d_parts[s])
+      for (int j = 0; j < (int)d_pl.parts[s].size(); ++j)
         for (int kc = 0; kc < c->ndc; ++kc) {  // K chunks of the same rows run back to back
-          Task t = make_task(TK_DOWN, l, p.first, p.second);
-          t.aux = (uint16_t)kc;
+          Task t = gemv_task(TK_DOWN, l, d_pl, s, j);
+          t.aux = (uint16_t)(c->tc ? t.aux : kc);
           add_wait(t, ev_gu(c, l));
           add_notify(t, ev_down(c, l));
           evc[ev_down(c, l)]++;
@@ -495,18 +597,17 @@ int build_graph(mk_ctx* c) {
         }
   }
   {
-    auto parts = partition_rows(f.vocab, 1, c->sm_weights, c->task_rows);
     int idx = 0;
     for (int s = 0; s < n; ++s)
-      for (auto& p : parts[s]) {
-        Task t = make_task(TK_LMHEAD, L, p.first, p.second);
-        t.layer = (uint16_t)L;
+      for (int j = 0; j < (int)lm_pl.parts[s].size(); ++j) {
+        Task t = gemv_task(TK_LMHEAD, L, lm_pl, s, j);
         add_wait(t, ev_down(c, L - 1));
-        t.index = (uint32_t)idx++;
+        if (!c->tc) t.index = (uint32_t)idx;  // argmax partial slot (tensor-core: the tile's)
+        ++idx;
         q[s].push_back(t);
       }
-    c->n_lm = idx;
-    evc[c->ev_lm] = (uint32_t)idx;
+    c->n_lm = c->tc ? c->tc_tiles[TK_LMHEAD] : idx;
+    evc[c->ev_lm] = (uint32_t)c->n_lm;
   }
   c->g.tasks.clear();
   c->qbegin.assign(n + 1, 0);
@@ -515,6 +616,10 @@ int build_graph(mk_ctx* c) {
     c->qbegin[s] = (uint32_t)c->g.tasks.size();
     for (auto& t : q[s]) {
       c->g.tasks.push_back({t, s});
+      if (c->tc) {
+        if (is_gemv_kind(t.kind)) wbytes += (uint64_t)t.nrows * kSlotBytes;
+        continue;
+      }
       switch (t.kind) {
         case TK_QKV: case TK_OPROJ: case TK_GATEUP: case TK_LMHEAD: wbytes += (uint64_t)t.nrows * f.hidden * 2; break;
         case TK_DOWN: {
@@ -541,23 +646,28 @@ void layout(mk_ctx* c) {
   c->loff.resize(L);
   c->off_embed = o;
   o = align256(o + (uint64_t)f.vocab * H * 2);
+  // bytes of one projection: row-major, or whole kTcRows x kTcUnitK blocks (tensor-core)
+  auto mat = [&](int kind, int rows, int K) -> uint64_t {
+    if (c->tc) return (uint64_t)c->tc_tiles[kind] * c->tc_nk[kind] * kSlotBytes;
+    return (uint64_t)rows * K * 2;
+  };
   for (int l = 0; l < L; ++l) {
     LayerOff& lo = c->loff[l];
     lo.qkv = o;
-    o = align256(o + (uint64_t)c->rows_qkv * H * 2);
+    o = align256(o + mat(TK_QKV, c->rows_qkv, H));
     lo.o = o;
-    o = align256(o + (uint64_t)H * nq * D * 2);
+    o = align256(o + mat(TK_OPROJ, H, nq * D));
     lo.gu = o;
-    o = align256(o + (uint64_t)c->rows_gu * H * 2);
+    o = align256(o + mat(TK_GATEUP, c->rows_gu, H));
     lo.d = o;
-    o = align256(o + (uint64_t)H * F * 2);
+    o = align256(o + mat(TK_DOWN, H, F));
     lo.attn_norm = o;
     o = align256(o + (uint64_t)H * 2);
     lo.mlp_norm = o;
     o = align256(o + (uint64_t)H * 2);
   }
   c->off_lm = o;
-  o = align256(o + (uint64_t)f.vocab * H * 2);
+  o = align256(o + mat(TK_LMHEAD, f.vocab, H));
   c->off_fnorm = o;
   o = align256(o + (uint64_t)H * 2);
   c->arena_bytes = o;
@@ -589,6 +699,11 @@ void layout(mk_ctx* c) {
   c->ws_part = take((size_t)L * B * nq * c->nch * (D + 2) * 4);
   c->ws_lmval = take(c->lm_cap * B * 4);
   c->ws_lmidx = take(c->lm_cap * B * 4);
+  // tensor-core partial records and tile arrival counters
+  c->rec_cap = c->tc ? c->n_recs * 2 + (size_t)c->n_sms * 16 : 0;
+  c->ws_tpart = take(std::max<size_t>(c->rec_cap, 1) * kTcRecFloats * 4);
+  c->tcnt_bytes = c->tc ? (size_t)L * c->n_tile_ids * sizeof(uint32_t) : 4;
+  c->ws_tcnt = take(c->tcnt_bytes);
   // prefill scratch: X, XN, Y, Q, O, HH per row
   const long long ycols = std::max<long long>(std::max(c->rows_qkv, c->rows_gu), H);
   c->pf_rows = (int)std::min<long long>(1024, (long long)B * f.max_seq);
@@ -633,6 +748,26 @@ void rope_table(const mk_config& f, std::vector<float2>& out) {
   }
 }
 
+// Tensor-core weight layout of a [rows][K] bf16 matrix (row(i) = pointer to row i): blocks
+// of kTcRows x kTcUnitK, block (tile t, K unit u) at (t * nk + u) * kSlotBytes; inside a block,
+// core matrix (8-row group g, 8-element K group j) at (g * 16 + j) * 128 bytes and its row r at
+// r * 16 bytes.  Rows and K past the matrix are zeros.
+template <class RowFn>
+void pack_blocks(RowFn row, int rows, int K, std::vector<uint16_t>& out) {
+  const int tiles = (rows + kTcRows - 1) / kTcRows, nk = (K + kTcUnitK - 1) / kTcUnitK;
+  constexpr int kBlockElems = kTcRows * kTcUnitK;
+  out.assign((size_t)tiles * nk * kBlockElems, 0);
+  for (int i = 0; i < rows; ++i) {
+    const uint16_t* src = row(i);
+    const int t = i / kTcRows, g = (i % kTcRows) / 8, r = i % 8;
+    for (int k = 0; k < K; k += 8) {
+      const int u = k / kTcUnitK, j = (k % kTcUnitK) / 8;
+      uint16_t* dst = &out[(size_t)(t * nk + u) * kBlockElems + (size_t)(g * (kTcUnitK / 8) + j) * 64 + r * 8];
+      std::memcpy(dst, src + k, (size_t)std::min(8, K - k) * 2);
+    }
+  }
+}
+
 bool cuda_ok(mk_ctx* c, cudaError_t e, const char* what) {
   if (e == cudaSuccess) return true;
   fail(c, MK_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
@@ -652,7 +787,8 @@ int upload_graph(mk_ctx* c, uint8_t* W) {
                              cudaMemcpyHostToDevice),
                "event upload") ||
       !cuda_ok(c, cudaMemset(W + c->ws_ev, 0, c->ev_bytes), "counter reset") ||
-      !cuda_ok(c, cudaMemset(W + c->ws_acnt, 0, c->acnt_bytes), "counter reset"))
+      !cuda_ok(c, cudaMemset(W + c->ws_acnt, 0, c->acnt_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(W + c->ws_tcnt, 0, c->tcnt_bytes), "counter reset"))
     return MK_ERR_CUDA;
   c->epoch = 0;
   return MK_OK;
@@ -709,11 +845,13 @@ int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
     int by_len = std::max(1, (f.max_seq + 15) / 16);
     c->nch = std::min(std::min(per, by_len), kMaxChunks);
   }
-  // batch width: 1, or 4 (sequences beyond the active batch masked); with 4 the
-  // down projection runs in K chunks of kDownChunk so its activations fit in registers
-  c->bm = (f.max_batch > 1) ? 4 : 1;
-  c->task_rows = kTaskRows / c->bm;
-  c->kdc = (c->bm > 1) ? std::min(f.ffn, kDownChunk) : f.ffn;
+  // batch width: 1; or 4 (sequences beyond the active batch masked), where the down
+  // projection runs in K chunks of kDownChunk so its activations fit in registers; or, for
+  // more than 4 sequences, kTcBatch on the tensor cores
+  c->bm = (f.max_batch > kMaxDecodeBatch) ? kTcBatch : (f.max_batch > 1) ? 4 : 1;
+  c->tc = c->bm == kTcBatch;
+  c->task_rows = c->tc ? kTcUnitsMax : kTaskRows / c->bm;
+  c->kdc = (c->bm == 4) ? std::min(f.ffn, kDownChunk) : f.ffn;
   c->ndc = (f.ffn + c->kdc - 1) / c->kdc;
   c->nseg_h = (f.hidden + kSegElems - 1) / kSegElems;
   c->nseg_f = (c->kdc + kSegElems - 1) / kSegElems;
@@ -721,11 +859,32 @@ int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
   c->rps_f = pow2_floor(std::min(kRpsMax, kSlotBytes / (c->kdc * 2)));
   // the GEMV takes every segment but the last of a K chunk as full
   const bool ragged_chunk = c->ndc > 1 && f.ffn - (c->ndc - 1) * c->kdc < (c->nseg_f - 1) * kSegElems;
-  if ((f.max_batch == 1 && f.ffn * 2 > kSlotBytes) || f.hidden * 2 > kSlotBytes || ragged_chunk) {
+  if (!c->tc && ((f.max_batch == 1 && f.ffn * 2 > kSlotBytes) || f.hidden * 2 > kSlotBytes || ragged_chunk)) {
     delete c;
     return fail(nullptr, MK_ERR_UNSUPPORTED, "a weight row does not fit one ring stage");
   }
-  c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm);
+  if (c->tc) {
+    // tiles of kTcRows rows, K in units of kTcUnitK (rows and K past the end are zero padding)
+    const int H = f.hidden;
+    auto set = [&](int kind, int rows, int K) {
+      c->tc_tiles[kind] = (rows + kTcRows - 1) / kTcRows;
+      c->tc_nk[kind] = (K + kTcUnitK - 1) / kTcUnitK;
+    };
+    set(TK_QKV, c->rows_qkv, H);
+    set(TK_OPROJ, H, f.n_q_heads * f.head_dim);
+    set(TK_GATEUP, c->rows_gu, H);
+    set(TK_DOWN, H, f.ffn);
+    set(TK_LMHEAD, f.vocab, H);
+    int base = 0;
+    for (int k : {TK_QKV, TK_OPROJ, TK_GATEUP, TK_DOWN, TK_LMHEAD}) {
+      c->tc_tile_base[k] = base;
+      base += c->tc_tiles[k];
+    }
+    c->n_tile_ids = base;
+    c->variant = find_decode_variant(0, 1, 0, 1, f.head_dim, kTcBatch);
+  } else {
+    c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm);
+  }
   c->sm_weights.assign(c->n_sms, 1.0);
   rc = build_graph(c);
   if (rc) {
@@ -764,8 +923,15 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
   auto put = [&](uint64_t off, const void* src, size_t bytes) {
     return cuda_ok(c, cudaMemcpyAsync(A + off, src, bytes, cudaMemcpyHostToDevice, s), "weight copy");
   };
+  // tensor-core layout: each projection re-laid in blocks, copied synchronously (staging reused)
+  std::vector<uint16_t> blk;
+  auto put_blocks = [&](uint64_t off, const uint16_t* base, size_t stride, int rows, int K) {
+    pack_blocks([&](int i) { return base + (size_t)i * stride; }, rows, K, blk);
+    return cuda_ok(c, cudaMemcpy(A + off, blk.data(), blk.size() * 2, cudaMemcpyHostToDevice), "weight copy");
+  };
   if (!put(c->off_embed, w->embed, (size_t)f.vocab * H * 2)) return MK_ERR_CUDA;
-  if (!put(c->off_lm, w->lm_head, (size_t)f.vocab * H * 2)) return MK_ERR_CUDA;
+  if (c->tc ? !put_blocks(c->off_lm, w->lm_head, H, f.vocab, H) : !put(c->off_lm, w->lm_head, (size_t)f.vocab * H * 2))
+    return MK_ERR_CUDA;
   if (!put(c->off_fnorm, w->final_norm, (size_t)H * 2)) return MK_ERR_CUDA;
   std::vector<uint16_t> qkv((size_t)c->rows_qkv * H), gu((size_t)c->rows_gu * H);
   const int G = c->G, half = D / 2;
@@ -794,6 +960,14 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
       std::memcpy(&gu[(size_t)(2 * i + 1) * H], w->wu[l] + (size_t)i * H, (size_t)H * 2);
     }
     const LayerOff& lo = c->loff[l];
+    if (c->tc) {
+      if (!put_blocks(lo.qkv, qkv.data(), H, c->rows_qkv, H) || !put_blocks(lo.o, w->wo[l], nq * D, H, nq * D) ||
+          !put_blocks(lo.gu, gu.data(), H, c->rows_gu, H) || !put_blocks(lo.d, w->wd[l], F, H, F) ||
+          !put(lo.attn_norm, w->attn_norm[l], (size_t)H * 2) || !put(lo.mlp_norm, w->mlp_norm[l], (size_t)H * 2) ||
+          !cuda_ok(c, cudaStreamSynchronize(s), "weight copy"))
+        return MK_ERR_CUDA;
+      continue;
+    }
     // synchronous copies: the staging vectors are reused for the next layer
     if (!cuda_ok(c, cudaMemcpy(A + lo.qkv, qkv.data(), qkv.size() * 2, cudaMemcpyHostToDevice), "qkv copy"))
       return MK_ERR_CUDA;
@@ -830,6 +1004,7 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
                "rope upload") ||
       !cuda_ok(c, cudaMemset(W + c->ws_ev, 0, c->ev_bytes), "counter reset") ||
       !cuda_ok(c, cudaMemset(W + c->ws_acnt, 0, c->acnt_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(W + c->ws_tcnt, 0, c->tcnt_bytes), "counter reset") ||
       !cuda_ok(c, cudaMemset(W + c->ws_err, 0, 16), "error reset") ||
       !cuda_ok(c, cudaStreamSynchronize(s), "load sync"))
     return MK_ERR_CUDA;
@@ -878,6 +1053,7 @@ int mk_prefill(mk_ctx* c, const int32_t* tokens, int B, int T, void* kv_cache, f
   p.attn_scale = 1.0f / std::sqrt((float)f.head_dim);
   p.kdc = c->kdc;
   p.ndc = c->ndc;
+  p.blocked = c->tc ? 1 : 0;
   std::string err;
   int rc = run_prefill(p, tokens, B, T, last_logits, reinterpret_cast<cudaStream_t>(stream), &err);
   if (rc) return fail(c, rc, err);
@@ -958,6 +1134,8 @@ int mk_decode_step(mk_ctx* c, const int32_t* tokens, void* kv_cache, float* logi
   P.nb = c->B;
   P.kdc = c->kdc;
   P.ndc = c->ndc;
+  P.tpart = reinterpret_cast<float*>(W + c->ws_tpart);
+  P.tcnt = reinterpret_cast<uint32_t*>(W + c->ws_tcnt);
   P.epoch = c->epoch + 1;
   P.ev_lm = (uint32_t)c->ev_lm;
   P.drop_event = c->drop_event;
@@ -1024,9 +1202,11 @@ int mk_set_sm_weights(mk_ctx* c, const float* weights, int n, void* stream) {
   Graph old_g = c->g;
   std::vector<uint32_t> old_q = c->qbegin;
   const int old_lm = c->n_lm;
+  const size_t old_recs = c->n_recs;
+  const uint64_t old_wb = c->weight_bytes_per_step;
   c->sm_weights = w;
   int rc = build_graph(c);
-  if (rc == MK_OK && (c->g.tasks.size() > c->task_cap || (size_t)c->n_lm > c->lm_cap))
+  if (rc == MK_OK && (c->g.tasks.size() > c->task_cap || (size_t)c->n_lm > c->lm_cap || c->n_recs > c->rec_cap))
     rc = fail(c, MK_ERR_UNSUPPORTED, "re-partitioned graph exceeds the workspace reserve");
   if (rc != MK_OK) {
     std::string m = c->err;
@@ -1034,6 +1214,8 @@ int mk_set_sm_weights(mk_ctx* c, const float* weights, int n, void* stream) {
     c->g = old_g;
     c->qbegin = old_q;
     c->n_lm = old_lm;
+    c->n_recs = old_recs;
+    c->weight_bytes_per_step = old_wb;
     return fail(c, rc, m);
   }
   if (c->loaded && upload_graph(c, c->ws) != MK_OK) return MK_ERR_CUDA;
@@ -1063,7 +1245,7 @@ int mk_get_graph_info(const mk_ctx* c, mk_graph_info* out) {
   out->attn_chunks = c->nch;
   out->kernel_variant = c->variant;
   out->weight_bytes_per_step = c->weight_bytes_per_step;
-  out->smem_bytes = decode_smem_bytes();
+  out->smem_bytes = decode_smem_bytes(c->variant);
   return MK_OK;
 }
 

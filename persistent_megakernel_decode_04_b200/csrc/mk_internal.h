@@ -41,6 +41,19 @@ constexpr int kSlotBytes = MK_SLOT_KB * 1024;        // one ring stage
 constexpr int kStages = MK_STAGES;                   // ring depth (kStages x kSlotBytes per SM)
 constexpr int kMaxDecodeBatch = 4;                   // CUDA-core path: batch width 1 or 4
 constexpr int kDownChunk = 4096;                     // down-projection K chunk for batch width 4
+// Tensor-core projection tiles (batch width 5..16): a tile is kTcRows weight rows; a ring
+// stage is one block of kTcRows x kTcUnitK bf16 weights in the no-swizzle K-major core-matrix
+// layout; a task covers up to kTcUnitsMax blocks (K units) of one tile.
+constexpr int kTcBatch = 16;                         // sequences per tensor-core step (MMA N = 2 x 16)
+constexpr int kTcN = 2 * kTcBatch;                   // columns: bf16 high parts, then low parts
+constexpr int kTcRows = 128;                         // MMA M
+constexpr int kTcUnitK = 128;                        // K elements per ring stage
+constexpr int kTcUnitsMax = 8;                       // K units per task
+constexpr int kTcStages = 4;                         // ring depth of the tensor-core kernel
+constexpr int kTcBopSbo = kTcUnitsMax * kTcUnitK / 8 * 128;  // activation operand: bytes per 8-row group
+constexpr int kTcBopBytes = (kTcN / 8) * kTcBopSbo;  // 64 KB
+constexpr int kTcRecFloats = kTcRows * kTcBatch + kTcBatch;  // partial record: [row][seq] sums, seq sum of x^2
+static_assert(kTcRows * kTcUnitK * 2 == MK_SLOT_KB * 1024, "a weight block fills one ring stage");
 
 enum TaskKind : uint8_t {
   TK_EMBED = 1,   // x_0 = E[token] for a slice of rows
@@ -61,6 +74,9 @@ struct Task {
   uint32_t notify[2];   // ATTN: notify[0] is raised by the merging (last) chunk only
   uint32_t index;       // LMHEAD: ordinal among LM-head tasks (argmax partial slot)
   uint32_t pad1;
+  // Tensor-core tasks reuse the fields: row0 = first weight block (tile * K units + unit),
+  // nrows = blocks, index = partial record, aux = slot among the tile's tasks (the tile's
+  // records are index - aux ..), pad0 = tasks of the tile, pad1 = tile arrival counter.
 };
 static_assert(sizeof(Task) == 40, "Task layout");
 
@@ -104,6 +120,8 @@ struct DecodeParams {
   int l2_ahead;               // weight stages the producer prefetches into L2 beyond the ring
   int nb;                     // active sequences (<= the kernel's batch width)
   int kdc, ndc;               // down-projection K chunk and chunk count
+  float* tpart;               // tensor-core partial records [n_records][kTcRecFloats]
+  uint32_t* tcnt;             // tensor-core tile arrival counters
 };
 constexpr uint64_t kStallPrefetchNs = 1000;    // producer blocked this long: prefetch ahead into L2
 constexpr uint64_t kStallPrefetchGapNs = 100;   // then one more stage per this interval
@@ -133,7 +151,7 @@ struct Variant {
 };
 int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm);
 const void* decode_kernel_ptr(int variant);
-size_t decode_smem_bytes();
+size_t decode_smem_bytes(int variant);
 int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t stream, std::string* err);
 
 // Standalone attention (mk_attention.cu).
@@ -159,6 +177,7 @@ struct PrefillParams {
   int H, nq, nkv, D, F, V, L, max_seq, max_batch;
   float eps, attn_scale;
   int kdc, ndc;  // W_down stored in ndc chunk-major K chunks of kdc columns
+  int blocked;   // 1: projections in the tensor-core block layout (kTcRows x kTcUnitK blocks)
 };
 int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, float* last_logits,
                 cudaStream_t stream, std::string* err);

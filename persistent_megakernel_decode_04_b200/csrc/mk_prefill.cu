@@ -54,12 +54,22 @@ __global__ void rmsnorm(const float* X, const uint16_t* g, float* Y, int H, floa
   for (int i = threadIdx.x; i < H; i += blockDim.x) Y[(size_t)row * H + i] = x[i] * r * bf(g[i]);
 }
 
+// Element (r, k) of a [N][K] bf16 weight matrix: row-major, or (blocked) in the tensor-core
+// layout of kTcRows x kTcUnitK blocks of 8-row x 8-element core matrices.
+__device__ __forceinline__ size_t w_index(int r, int k, int K, int blocked) {
+  if (!blocked) return (size_t)r * K + k;
+  const int nk = (K + kTcUnitK - 1) / kTcUnitK;
+  const size_t blk = (size_t)(r / kTcRows) * nk + k / kTcUnitK;
+  return blk * (kTcRows * kTcUnitK) + (size_t)(((r % kTcRows) / 8) * (kTcUnitK / 8) + (k % kTcUnitK) / 8) * 64 +
+         (r % 8) * 8 + (k % 8);
+}
+
 // Y[n][N] (row stride ldy) (+)= A[n][K] (fp32, row stride lda) . W[N][K]^T (bf16), fp32
 // accumulation.  64 x 64 output tile per block, 256 threads x (4 x 4) outputs, K tile 32.
 constexpr int BM = 64, BN = 64, BK = 32;
 __global__ void __launch_bounds__(256) gemm(const float* __restrict__ A, const uint16_t* __restrict__ W,
                                             float* __restrict__ Y, int n, int N, int K, int lda, int ldy,
-                                            int accumulate) {
+                                            int accumulate, int blocked) {
   __shared__ float As[BK][BM + 4];
   __shared__ float Ws[BK][BN + 4];
   const int tid = threadIdx.x;
@@ -76,7 +86,7 @@ __global__ void __launch_bounds__(256) gemm(const float* __restrict__ A, const u
     for (int e = tid; e < BN * BK; e += 256) {
       const int r = e / BK, k = e % BK;
       const int gr = n0 + r, gk = k0 + k;
-      Ws[k][r] = (gr < N && gk < K) ? bf(W[(size_t)gr * K + gk]) : 0.f;
+      Ws[k][r] = (gr < N && gk < K) ? bf(W[w_index(gr, gk, K, blocked)]) : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -220,9 +230,9 @@ static bool ck(cudaError_t e, const char* what, std::string* err) {
 }
 
 static void gemm(const float* A, const uint16_t* W, float* Y, int n, int N, int K, int ldy, cudaStream_t s,
-                 int lda = -1, int accumulate = 0) {
+                 int blocked, int lda = -1, int accumulate = 0) {
   dim3 grid((N + pf::BN - 1) / pf::BN, (n + pf::BM - 1) / pf::BM);
-  pf::gemm<<<grid, 256, 0, s>>>(A, W, Y, n, N, K, lda < 0 ? K : lda, ldy, accumulate);
+  pf::gemm<<<grid, 256, 0, s>>>(A, W, Y, n, N, K, lda < 0 ? K : lda, ldy, accumulate, blocked);
 }
 
 int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, float* last_logits, cudaStream_t s,
@@ -247,20 +257,20 @@ int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, flo
       const uint16_t* an = reinterpret_cast<const uint16_t*>(p.arena + lo.attn_norm);
       const uint16_t* mn = reinterpret_cast<const uint16_t*>(p.arena + lo.mlp_norm);
       pf::rmsnorm<<<n, 256, 0, s>>>(p.X, an, p.XN, H, p.eps, 1, 0);
-      gemm(p.XN, reinterpret_cast<const uint16_t*>(p.arena + lo.qkv), p.Y, n, NQKV, H, NQKV, s);
+      gemm(p.XN, reinterpret_cast<const uint16_t*>(p.arena + lo.qkv), p.Y, n, NQKV, H, NQKV, s, p.blocked);
       pf::qkv_post<<<n, 256, 0, s>>>(p.Y, n, ct, t0, p.rope, p.Q, p.kv, l, nq, nkv, D, p.max_seq, p.max_batch);
       const size_t smem = (size_t)(t0 + ct) * sizeof(float);
       if (smem > 48 * 1024) cudaFuncSetAttribute(pf::attention, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       pf::attention<<<n * nq, 128, smem, s>>>(p.Q, p.kv, p.O, ct, t0, l, nq, nkv, D, p.max_seq, p.max_batch,
                                               p.attn_scale);
-      gemm(p.O, reinterpret_cast<const uint16_t*>(p.arena + lo.o), p.Y, n, H, nq * D, H, s);
+      gemm(p.O, reinterpret_cast<const uint16_t*>(p.arena + lo.o), p.Y, n, H, nq * D, H, s, p.blocked);
       pf::residual_add<<<256, 256, 0, s>>>(p.X, p.Y, (size_t)n * H);
       pf::rmsnorm<<<n, 256, 0, s>>>(p.X, mn, p.XN, H, p.eps, 1, 0);
-      gemm(p.XN, reinterpret_cast<const uint16_t*>(p.arena + lo.gu), p.Y, n, 2 * F, H, 2 * F, s);
+      gemm(p.XN, reinterpret_cast<const uint16_t*>(p.arena + lo.gu), p.Y, n, 2 * F, H, 2 * F, s, p.blocked);
       pf::swiglu<<<n, 256, 0, s>>>(p.Y, p.HH, F);
       for (int k = 0; k < p.ndc; ++k) {  // W_down in chunk-major K chunks (one chunk when unsplit)
         const int k0 = k * p.kdc, kc = (F - k0) < p.kdc ? (F - k0) : p.kdc;
-        gemm(p.HH + k0, reinterpret_cast<const uint16_t*>(p.arena + lo.d) + (size_t)H * k0, p.Y, n, H, kc, H, s, F, k);
+        gemm(p.HH + k0, reinterpret_cast<const uint16_t*>(p.arena + lo.d) + (size_t)H * k0, p.Y, n, H, kc, H, s, p.blocked, F, k);
       }
       pf::residual_add<<<256, 256, 0, s>>>(p.X, p.Y, (size_t)n * H);
     }
@@ -270,7 +280,7 @@ int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, flo
     // final norm of each sequence's last token (row b * last_ct + last_ct - 1), then the LM head
     const uint16_t* fn = reinterpret_cast<const uint16_t*>(p.arena + p.off_fnorm);
     pf::rmsnorm<<<B, 256, 0, s>>>(p.X, fn, p.XN, H, p.eps, last_ct, last_ct - 1);
-    gemm(p.XN, reinterpret_cast<const uint16_t*>(p.arena + p.off_lm), last_logits, B, p.V, H, p.V, s);
+    gemm(p.XN, reinterpret_cast<const uint16_t*>(p.arena + p.off_lm), last_logits, B, p.V, H, p.V, s, p.blocked);
   }
   (void)last_t0;
   if (!ck(cudaGetLastError(), "prefill", err)) return MK_ERR_CUDA;

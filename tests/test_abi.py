@@ -56,19 +56,23 @@ def test_decode_before_load_is_a_state_error():
         mk.mk_destroy(ctx)
 
 
-@pytest.fixture(params=["tiny", "llama3-8b", "chameleon-7b-b1", "tiny-b4", "llama3-8b-b4", "chameleon-7b-b4"])
+@pytest.fixture(params=["tiny", "llama3-8b", "chameleon-7b-b1", "tiny-b4", "llama3-8b-b4", "chameleon-7b-b4",
+                        "tiny-b16", "llama3-8b-b16", "chameleon-7b-b16"])
 def graph(request):
-    name, B = (request.param[:-3], 4) if request.param.endswith("-b4") else (request.param, 1)
+    name, B = request.param, 1
+    for suffix, b in (("-b4", 4), ("-b16", 16)):
+        if name.endswith(suffix):
+            name, B = name[: -len(suffix)], b
     shape, ms = {"tiny": (mi.TINY, 64), "llama3-8b": (mi.LLAMA8B, 1024),
                  "chameleon-7b-b1": (mi.CHAMELEON7B, 1280), "chameleon-7b": (mi.CHAMELEON7B, 1280)}[name]
     ctx = mk.mk_build_taskgraph(mk.Config.from_shape(shape, B, ms).c(), -1)
     tasks, counts = mk.mk_export_taskgraph(ctx)
-    yield ctx, tasks, counts, shape
+    yield ctx, tasks, counts, shape, B
     mk.mk_destroy(ctx)
 
 
 def test_built_graph_validates_and_balances_bytes(graph):
-    ctx, tasks, counts, shape = graph
+    ctx, tasks, counts, shape, B = graph
     assert mk.mk_validate_taskgraph(ctx, tasks, counts) == 0
     info = mk.mk_get_graph_info(ctx)
     # weight bytes streamed per step = every projection once (plain definition of the step)
@@ -76,15 +80,16 @@ def test_built_graph_validates_and_balances_bytes(graph):
     per_layer = ((s.n_q_heads + 2 * s.n_kv_heads) * s.head_dim * s.hidden + s.hidden * s.n_q_heads * s.head_dim
                  + 2 * s.ffn * s.hidden + s.hidden * s.ffn) * 2
     assert info["weight_bytes_per_step"] == s.n_layers * per_layer + s.vocab * s.hidden * 2
-    # each SM streams nearly the same number of weight bytes (within 3 %); with more than one
-    # sequence the down projection runs in K chunks, one task per chunk of the same rows
+    # each SM streams nearly the same number of weight bytes (within 3 %); with 2..4 sequences
+    # the down projection runs in K chunks, one task per chunk of the same rows; tensor-core
+    # tasks (more than 4 sequences) stream nrows whole 32 KB weight blocks
     down = tasks[tasks[:, 0] == 6]
     ndc = len(down) // len({(int(t[1]), int(t[3])) for t in down})
     K = {2: s.hidden, 4: s.hidden, 5: s.hidden, 6: s.ffn / ndc, 7: s.hidden}
     per_sm = np.zeros(info["n_sms"])
     for t in tasks:
         if t[0] in K:
-            per_sm[t[2]] += t[4] * K[t[0]] * 2
+            per_sm[t[2]] += t[4] * (32768 if B > 4 else K[t[0]] * 2)
     if s.hidden >= 4096:
         assert per_sm.max() / per_sm.mean() < 1.03
 
@@ -96,7 +101,7 @@ def _reject(ctx, tasks, counts, needle):
 
 
 def test_validator_rejects_a_dropped_notify(graph):
-    ctx, tasks, counts, _ = graph
+    ctx, tasks, counts, _, B = graph
     t = tasks.copy()
     i = int(np.nonzero(t[:, 0] == 4)[0][0])  # an O-projection task
     t[i, 8] = 0
@@ -104,7 +109,7 @@ def test_validator_rejects_a_dropped_notify(graph):
 
 
 def test_validator_rejects_a_missing_dependency(graph):
-    ctx, tasks, counts, _ = graph
+    ctx, tasks, counts, _, B = graph
     t = tasks.copy()
     i = int(np.nonzero(t[:, 0] == 3)[0][-1])  # an attention task loses its wait on QKV
     t[i, 5] = 0
@@ -112,28 +117,44 @@ def test_validator_rejects_a_missing_dependency(graph):
 
 
 def test_validator_rejects_a_queue_that_deadlocks(graph):
-    ctx, tasks, counts, _ = graph
+    ctx, tasks, counts, _, B = graph
     t = tasks.copy()
-    # move SM 0's first down-projection task in front of its first gate/up task
-    sm0 = np.nonzero(t[:, 2] == 0)[0]
-    gu = [i for i in sm0 if t[i, 0] == 5][0]
-    dn = [i for i in sm0 if t[i, 0] == 6][0]
+    # find a task that waits on an event an earlier task of the same SM raises, and move it
+    # in front of that producer: the SM then waits on itself
+    pick = None
+    for sm in range(int(t[:, 2].max()) + 1):
+        q = [int(i) for i in np.nonzero(t[:, 2] == sm)[0]]
+        for a_pos, a in enumerate(q):
+            raised = set(int(e) for e in t[a, 9 : 9 + t[a, 8]])
+            for b in q[a_pos + 1 :]:
+                if raised & set(int(e) for e in t[b, 6 : 6 + t[b, 5]]):
+                    pick = (a, b)
+                    break
+            if pick:
+                break
+        if pick:
+            break
+    assert pick is not None
+    a, b = pick
     order = list(range(len(t)))
-    order.remove(dn)
-    order.insert(order.index(gu), dn)
+    order.remove(b)
+    order.insert(order.index(a), b)
     _reject(ctx, t[order], counts, "deadlock")
 
 
 def test_validator_rejects_overlapping_rows(graph):
-    ctx, tasks, counts, _ = graph
+    ctx, tasks, counts, _, B = graph
     t = tasks.copy()
     i = int(np.nonzero(t[:, 0] == 7)[0][3])
-    t[i, 3] -= 2  # LM-head tile shifted onto its neighbour's rows
-    _reject(ctx, t, counts, "covered")
+    t[i, 3] -= 2  # LM-head tile shifted onto its neighbour's rows (or blocks)
+    rc = mk.mk_validate_taskgraph(ctx, t, counts)
+    assert rc == mk.MK_ERR_INVALID_ARG
+    msg = mk.mk_last_error(ctx)
+    assert "covered" in msg or "spans two tiles" in msg, msg
 
 
 def test_validator_rejects_a_wrong_threshold(graph):
-    ctx, tasks, counts, _ = graph
+    ctx, tasks, counts, _, B = graph
     c = counts.copy()
     c[1] += 1
     _reject(ctx, tasks, c, "threshold")

@@ -1,6 +1,7 @@
-"""Batched decode (2..4 sequences per step) against the CPU oracle, teacher-forced per
-sequence on the oracle's tokens: per-step logits of every sequence, argmax, the bf16 KV
-cache, masking of sequences outside the active batch and per-sequence positions."""
+"""Batched decode against the CPU oracle, teacher-forced per sequence on the oracle's tokens:
+2..4 sequences on the CUDA-core batch-4 kernel, 5..16 on the tensor-core kernel.  Per-step
+logits of every sequence, argmax, the bf16 KV cache, masking of sequences outside the active
+batch and per-sequence positions."""
 import numpy as np
 import pytest
 import torch
@@ -83,15 +84,39 @@ def test_tiny_batch4_ragged_positions():
         kv_close(got[:, :, b : b + 1, :, :n], want[:, :, b : b + 1, :, :n], f"kv cache seq {b}")
 
 
-def test_batch_beyond_kernel_width_is_rejected():
-    # 5..16 sequences need the tensor-core projection path; the CUDA-core kernel refuses them
+def test_tiny_batch16_tensor_core_prefill_and_12_steps():
+    # more than 4 sequences: the projections run as tcgen05 tiles (weights in block layout)
     w = mi.make_weights(mi.TINY, seed=8)
-    m = _model(w, 8, 16)
-    prompts = np.stack([mi.prompt(8, b, 4, w.shape.vocab) for b in range(8)])
-    m.prefill(torch.from_numpy(prompts.astype(np.int32)).to(DEV))
-    with pytest.raises(mk.MkError) as e:
-        m.decode(torch.zeros(8, dtype=torch.int32, device=DEV))
-    assert e.value.code == mk.MK_ERR_UNSUPPORTED
+    _teacher_forced_batch(w, B=16, max_batch=16, T=10, steps=12, max_seq=32, seed=8)
+
+
+@pytest.mark.parametrize("B", [5, 8])
+def test_tiny_tensor_core_partial_batch(B):
+    w = mi.make_weights(mi.TINY, seed=9)
+    _teacher_forced_batch(w, B=B, max_batch=16, T=7, steps=5, max_seq=16, seed=9 + B)
+
+
+def test_tiny_batch16_ragged_positions_and_random_gains():
+    # norm gains != 1 and a position per sequence, through the tensor-core path
+    w = mi.make_weights(mi.TINY, seed=12, sigma=0.05)
+    w.final_norm = mi.normal_bf16(12, 50, (w.shape.hidden,), sigma=0.3, mean=1.0)
+    for l in range(w.shape.n_layers):
+        w.attn_norm[l] = mi.normal_bf16(12, 51 + 2 * l, (w.shape.hidden,), sigma=0.3, mean=1.0)
+        w.mlp_norm[l] = mi.normal_bf16(12, 52 + 2 * l, (w.shape.hidden,), sigma=0.3, mean=1.0)
+    s = w.shape
+    L = 40
+    kv = mi.kv_cache_values(12, s, 16, L, sigma=1.0)
+    pos = [int(p) for p in 1 + (np.arange(16) * 7) % L]
+    ref = oracle.Decoder(w, 16, 48)
+    ref.set_cache(kv, L)
+    ref.set_positions(pos)
+    m = _model(w, 16, 48)
+    m.kv_view()[:, :, :16, :, :L, :] = torch.from_numpy(kv.view(np.int16)).to(DEV)
+    m.set_positions(pos)
+    toks = [int(t) for t in mi.prompt(12, 1, 16, s.vocab)]
+    for i in range(4):
+        toks = _step_both(ref, m, toks, f"step {i}")
+    assert m.sync_status() == mk.MK_OK
     m.close()
 
 
@@ -100,7 +125,7 @@ def w_chameleon():
     return mi.make_weights(mi.CHAMELEON7B, seed=0)
 
 
-@pytest.mark.parametrize("B", [1, 4])
+@pytest.mark.parametrize("B", [1, 4, 16])
 def test_chameleon7b_1024_context(w_chameleon, B):
     """Chameleon-7B-shaped MHA decoder, every sequence at 1024 cached positions (a seeded
     synthetic cache standing in for the 1024-token prompts), 2 decode steps."""
