@@ -90,8 +90,11 @@ size_t mk_kv_cache_bytes(const mk_ctx* ctx);
 
 /* Pack the host weights into tile order (QKV rows grouped per KV head with RoPE pairs
  * adjacent; gate/up rows interleaved) and copy them to `weight_arena`; upload the task
- * graph and RoPE table into `workspace` and zero its event counters.  Both buffers must
- * stay allocated and unmoved until mk_destroy.  Synchronises `stream` before returning. */
+ * graph and RoPE table into `workspace` and zero its event counters.  The packing depends
+ * on max_batch: row-major for 1 sequence; W_down in K chunks of 4096 columns for 2..4;
+ * every projection in 128 x 128 blocks of tensor-core core matrices for 5..16.  Both
+ * buffers must stay allocated and unmoved until mk_destroy.  Synchronises `stream` before
+ * returning. */
 int mk_load_weights(mk_ctx* ctx, const mk_host_weights* w, void* weight_arena, void* workspace, void* stream);
 
 /* Prefill (the hybrid arrangement of "Ada-MK: Adaptive MegaKernel Optimization via
@@ -111,7 +114,11 @@ int mk_get_positions(const mk_ctx* ctx, int32_t* host_pos, int capacity);
 /* One decode step of the active batch: one launch of the persistent megakernel.
  * tokens: device int32 [B], token b goes in at position pos[b]; logits: device fp32
  * [B][vocab]; next_tokens: device int32 [B] (greedy argmax, lowest index on ties) or NULL.
- * Appends K/V at pos[b] and advances every position by one. */
+ * Appends K/V at pos[b] and advances every position by one.  The kernel serves up to 1
+ * (max_batch 1), 4 (max_batch 2..4, CUDA-core GEMV) or 16 (max_batch 5..16, projections as
+ * tcgen05 tensor-core tiles) sequences; sequences past B are masked.  MK_ERR_INVALID_ARG if
+ * a sequence is full (pos = max_seq); MK_ERR_UNSUPPORTED if no kernel instantiation exists
+ * for the shape. */
 int mk_decode_step(mk_ctx* ctx, const int32_t* tokens, void* kv_cache, float* logits, int32_t* next_tokens,
                    void* stream);
 

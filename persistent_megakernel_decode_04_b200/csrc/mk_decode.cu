@@ -255,13 +255,12 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
               dot8(w, x2[0][s], acc[rr][0]);
             } else {
               const uint64_t wp[4] = {widen_bf16w(w.x), widen_bf16w(w.y), widen_bf16w(w.z), widen_bf16w(w.w)};
+              // sequences innermost: consecutive FMAs update different accumulators
 #pragma unroll
-              for (int b = 0; b < BM; ++b) {
-                if (b < nb) {
+              for (int j = 0; j < 4; ++j)
 #pragma unroll
-                  for (int j = 0; j < 4; ++j) fma2_pair(acc[rr][b], wp[j], x2[b][s][j]);
-                }
-              }
+                for (int b = 0; b < BM; ++b)
+                  if (b < nb) fma2_pair(acc[rr][b], wp[j], x2[b][s][j]);
             }
           }
         }
@@ -362,13 +361,17 @@ __device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, c
 // to arrive merges the partials into o (FlashDecoding-style online-softmax merge) and
 // notifies; with a single chunk in use that chunk writes o directly and nothing is merged.
 //
-// Latency: keys before the current position were written by earlier steps, so each warp
-// loads its first block of kAttnBlock keys (raw bf16 words in registers) before the task's
-// inputs are released (attn_preload); after the release only q and the key/value at the
-// current position are fetched.  Each lane holds DL = D/32 dims of every head; the KB x 4
-// (key, head) partial dot products of a block are summed across lanes with one transposed
-// butterfly (each exchange halves the live values) and broadcast back with shuffles.
+// Keys before the current position were written by earlier steps, so they stream through the
+// weight ring like weights: the producer copies the chunk's old K and V rows (kv_stage_keys
+// per stage, K rows then V rows) in queue order, ahead of the task's release, and the workers
+// read them from shared memory.  Only q and the key/value at the current position (written by
+// this step's QKV tasks) are loaded after the release.  Each lane holds DL = D/32 dims of
+// every head; the kAttnBlock x 4 (key, head) partial dot products of a block are summed
+// across lanes with one transposed butterfly (each exchange halves the live values) and
+// broadcast back with shuffles.
 constexpr int kAttnBlock = 8;  // keys per warp per block
+template <int D>
+__host__ __device__ constexpr int kv_stage_keys() { return kSlotBytes / (2 * D * 2); }
 
 struct AttnGeom {
   int b, g, c, Lk, nch_eff, j0, j1;
@@ -393,12 +396,6 @@ __device__ __forceinline__ AttnGeom attn_geom(const DecodeParams& P, const Task&
 }
 
 template <int D>
-struct AttnRegs {
-  static constexpr int W = D / 64;  // 32-bit words of K (or V) per lane per key: 2 (D=128) or 1
-  uint32_t k[kAttnBlock][W], v[kAttnBlock][W];
-};
-
-template <int D>
 __device__ __forceinline__ const uint16_t* attn_cache(const DecodeParams& P, const Task& t, const AttnGeom& a,
                                                        int kind) {
   const size_t head_stride = (size_t)P.max_seq * D;
@@ -420,27 +417,89 @@ __device__ __forceinline__ void attn_load_key(const uint16_t* kc, const uint16_t
   }
 }
 
-// Before the release: this warp's first block of keys, positions < pos only.
+// Online-softmax update of this warp's (m, l, acc) with one block of up to kAttnBlock keys
+// (K and V words kw/vw of this lane; key u counts if bit u of `valid` is set).
 template <int D>
-__device__ __forceinline__ void attn_preload(const DecodeParams& P, const Task& t, AttnRegs<D>& R) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const AttnGeom a = attn_geom(P, t);
-  if (warp >= kAttnWarps) return;
-  const uint16_t* kc = attn_cache<D>(P, t, a, 0);
-  const uint16_t* vc = attn_cache<D>(P, t, a, 1);
-  const int pos = a.Lk - 1;
+__device__ __forceinline__ void attn_block(const float (&qv)[4][D / 32], const uint32_t (&kw)[kAttnBlock][D / 64],
+                                           const uint32_t (&vw)[kAttnBlock][D / 64], uint32_t valid, int G,
+                                           float (&m)[4], float (&l)[4], float (&acc)[4][D / 32], int lane) {
+  constexpr int DL = D / 32;
+  constexpr int W = D / 64;
+  // partial dots of the block: slot u * 4 + h
+  float sc[kAttnBlock * 4];
 #pragma unroll
   for (int u = 0; u < kAttnBlock; ++u) {
-    const int j = a.j0 + warp + u * kAttnWarps;
-    if (j < a.j1 && j < pos) attn_load_key<D>(kc, vc, j, lane, R.k[u], R.v[u]);
+    float kf[DL];
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      kf[2 * w] = bf16lo(kw[u][w]);
+      kf[2 * w + 1] = bf16hi(kw[u][w]);
+    }
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float sv = 0.f;
+#pragma unroll
+      for (int i = 0; i < DL; ++i) sv = fmaf(qv[h][i], kf[i], sv);
+      sc[u * 4 + h] = sv;
+    }
+  }
+  // transposed butterfly: lane l ends with the warp's sum of slot l ...
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? sc[i] : sc[i + off];
+      const float keep = upper ? sc[i + off] : sc[i];
+      sc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  const float mine = sc[0];
+  // ... and every lane gets every slot back
+#pragma unroll
+  for (int i = 0; i < kAttnBlock * 4; ++i) sc[i] = __shfl_sync(0xffffffffu, mine, i);
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    if (h < G) {
+      float mx = m[h];
+#pragma unroll
+      for (int u = 0; u < kAttnBlock; ++u)
+        if ((valid >> u) & 1u) mx = fmaxf(mx, sc[u * 4 + h]);
+      const float alpha = __expf(m[h] - mx);  // 0 on the first block (m = -inf)
+      float ls = 0.f;
+#pragma unroll
+      for (int i = 0; i < DL; ++i) acc[h][i] *= alpha;
+#pragma unroll
+      for (int u = 0; u < kAttnBlock; ++u) {
+        if ((valid >> u) & 1u) {
+          const float p = __expf(sc[u * 4 + h] - mx);
+          ls += p;
+#pragma unroll
+          for (int w = 0; w < W; ++w) {
+            acc[h][2 * w] = fmaf(p, bf16lo(vw[u][w]), acc[h][2 * w]);
+            acc[h][2 * w + 1] = fmaf(p, bf16hi(vw[u][w]), acc[h][2 * w + 1]);
+          }
+        }
+      }
+      l[h] = l[h] * alpha + ls;
+      m[h] = mx;
+    }
   }
 }
 
+// Number of ring stages of an attention task: its old positions [j0, min(j1, pos)).
 template <int D>
-__device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, const Task& t, AttnRegs<D>& R,
-                                               uint32_t task_id) {
+__device__ __forceinline__ int attn_stage_span(const AttnGeom& a, int* jend) {
+  *jend = (a.c < a.nch_eff) ? min(a.j1, a.Lk - 1) : a.j0;
+  return *jend > a.j0 ? (*jend - a.j0 + kv_stage_keys<D>() - 1) / kv_stage_keys<D>() : 0;
+}
+
+template <int D, bool TC>
+__device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, Pipe& pp, const uint8_t* ring,
+                                               const Task& t, uint32_t task_id, uint32_t& stall_ns) {
   constexpr int DL = D / 32;
   constexpr int W = D / 64;
+  constexpr int KPS = kv_stage_keys<D>();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = P.nq / P.nkv;
   const AttnGeom a = attn_geom(P, t);
@@ -454,12 +513,6 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
 
   if (c < nch_eff) {  // uniform across the CTA
     float qv[4][DL], m[4], l[4], acc[4][DL];
-    // the key/value at the current position were written in this step: load them now
-#pragma unroll
-    for (int u = 0; u < kAttnBlock; ++u) {
-      const int j = a.j0 + warp + u * kAttnWarps;
-      if (warp < kAttnWarps && j == pos) attn_load_key<D>(kc, vc, j, lane, R.k[u], R.v[u]);
-    }
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       m[h] = -INFINITY;
@@ -470,74 +523,64 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
         acc[h][i] = 0.f;
       }
     }
-    for (int jb = a.j0 + warp; warp < kAttnWarps && jb < a.j1; jb += kAttnBlock * kAttnWarps) {
-      if (jb != a.j0 + warp) {  // later blocks (long chunks): load them now
+    uint32_t kw[kAttnBlock][W], vw[kAttnBlock][W];
+    // the key and value at the current position were written in this step: warp 0 fetches
+    // them together with q (one L2 round trip) and adds them after the ring stages
+    const bool has_cur = warp == 0 && pos >= a.j0 && pos < a.j1;
+    uint32_t kcur[W], vcur[W];
+    if (has_cur) attn_load_key<D>(kc, vc, pos, lane, kcur, vcur);
+    // old positions from the ring, kv_stage_keys per stage (K rows at 0, V rows at KPS * D)
+    int jend;
+    const int nst = attn_stage_span<D>(a, &jend);
+    for (int st = 0; st < nst; ++st) {
+      const int jj = a.j0 + st * KPS, nk = min(KPS, jend - jj);
+      const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
+      if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
+        raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
+        S.cabort = 1u;
+      }
+      if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
+      const uint8_t* kst = ring + (size_t)pp.stage * kSlotBytes;
+      const uint8_t* vst = kst + KPS * D * 2;
+#pragma unroll
+      for (int kb = 0; kb < KPS / (kAttnBlock * kAttnWarps); ++kb) {
+        uint32_t valid = 0;
 #pragma unroll
         for (int u = 0; u < kAttnBlock; ++u) {
-          const int j = jb + u * kAttnWarps;
-          if (j < a.j1) attn_load_key<D>(kc, vc, j, lane, R.k[u], R.v[u]);
-        }
-      }
-      // partial dots of the block: slot u * 4 + h
-      float sc[kAttnBlock * 4];
-#pragma unroll
-      for (int u = 0; u < kAttnBlock; ++u) {
-        float kf[DL];
-#pragma unroll
-        for (int w = 0; w < W; ++w) {
-          kf[2 * w] = bf16lo(R.k[u][w]);
-          kf[2 * w + 1] = bf16hi(R.k[u][w]);
-        }
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          float s = 0.f;
-#pragma unroll
-          for (int i = 0; i < DL; ++i) s = fmaf(qv[h][i], kf[i], s);
-          sc[u * 4 + h] = s;
-        }
-      }
-      // transposed butterfly: lane l ends with the warp's sum of slot l ...
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < off; ++i) {
-          const float send = upper ? sc[i] : sc[i + off];
-          const float keep = upper ? sc[i + off] : sc[i];
-          sc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-        }
-      }
-      const float mine = sc[0];
-      // ... and every lane gets every slot back
-#pragma unroll
-      for (int i = 0; i < kAttnBlock * 4; ++i) sc[i] = __shfl_sync(0xffffffffu, mine, i);
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        if (h < G) {
-          float mx = m[h];
-#pragma unroll
-          for (int u = 0; u < kAttnBlock; ++u)
-            if (jb + u * kAttnWarps < a.j1) mx = fmaxf(mx, sc[u * 4 + h]);
-          const float alpha = __expf(m[h] - mx);  // 0 on the first block (m = -inf)
-          float ls = 0.f;
-#pragma unroll
-          for (int i = 0; i < DL; ++i) acc[h][i] *= alpha;
-#pragma unroll
-          for (int u = 0; u < kAttnBlock; ++u) {
-            if (jb + u * kAttnWarps < a.j1) {
-              const float p = __expf(sc[u * 4 + h] - mx);
-              ls += p;
-#pragma unroll
-              for (int w = 0; w < W; ++w) {
-                acc[h][2 * w] = fmaf(p, bf16lo(R.v[u][w]), acc[h][2 * w]);
-                acc[h][2 * w + 1] = fmaf(p, bf16hi(R.v[u][w]), acc[h][2 * w + 1]);
-              }
+          const int idx = kb * kAttnBlock * kAttnWarps + warp + u * kAttnWarps;
+          if (idx < nk) {
+            valid |= 1u << u;
+            if (D == 128) {
+              const uint2 kk = *reinterpret_cast<const uint2*>(kst + idx * D * 2 + lane * 8);
+              const uint2 vv = *reinterpret_cast<const uint2*>(vst + idx * D * 2 + lane * 8);
+              kw[u][0] = kk.x; kw[u][W - 1] = kk.y;
+              vw[u][0] = vv.x; vw[u][W - 1] = vv.y;
+            } else {
+              kw[u][0] = *reinterpret_cast<const uint32_t*>(kst + idx * D * 2 + lane * 4);
+              vw[u][0] = *reinterpret_cast<const uint32_t*>(vst + idx * D * 2 + lane * 4);
             }
           }
-          l[h] = l[h] * alpha + ls;
-          m[h] = mx;
         }
+        if (valid) attn_block<D>(qv, kw, vw, valid, G, m, l, acc, lane);
       }
+      // release the stage: every warp's arrival (CUDA-core ring), or one after all warps
+      // (tensor-core ring, whose stages count a single release)
+      if (TC) {
+        worker_bar();
+        if (tid == 0) mbar_arrive(&S.empty[pp.stage]);
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
+      }
+      pp.advance();
+    }
+    if (has_cur) {
+#pragma unroll
+      for (int w = 0; w < W; ++w) {
+        kw[0][w] = kcur[w];
+        vw[0][w] = vcur[w];
+      }
+      attn_block<D>(qv, kw, vw, 1u, G, m, l, acc, lane);
     }
     // cross-warp merge of this chunk
 #pragma unroll
@@ -552,6 +595,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       }
     }
     worker_bar();
+    if (S.cabort) return false;  // a ring wait ran out (uniform: written before the barrier)
     for (int e = tid; e < G * D; e += kWorkerThreads) {
       const int h = e / D, d = e % D;
       float M = -INFINITY;
@@ -770,34 +814,45 @@ __device__ __forceinline__ bool tc_task(const DecodeParams& P, DSmem& S, Pipe& p
   const int k0 = u0 * kTcUnitK, ngroups = nu * (kTcUnitK / 8);
 
   // 1. activation operand: warp w stages sequences w and w + 8, lane j the 8-element K groups
-  //    j, j + 32, ...; sequences outside the active batch and K past the end are zeros
+  //    j, j + 32, ...; sequences outside the active batch and K past the end are zeros.  Every
+  //    load of the lane is issued before the first is used (one L2 round trip).
+  constexpr int kJ = kTcUnitsMax * kTcUnitK / 8 / 32;  // K groups per lane
+  float4 xv[2][kJ][2];
+  uint4 gv[kJ];
+#pragma unroll
+  for (int i = 0; i < kJ; ++i) {
+    const int j = lane + 32 * i, k = k0 + j * 8;
+    const bool in = j < ngroups && k < K;
+    gv[i] = (in && gain) ? __ldg(reinterpret_cast<const uint4*>(gain + k))
+                         : make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);  // bf16 1.0 pairs
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int b = warp + h * kWorkerWarps;
+      if (in && b < P.nb) {
+        const float* xb = xs + (size_t)b * xstride + k;
+        xv[h][i][0] = __ldcg(reinterpret_cast<const float4*>(xb));
+        xv[h][i][1] = __ldcg(reinterpret_cast<const float4*>(xb + 4));
+      } else {
+        xv[h][i][0] = xv[h][i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  }
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int b = warp + h * kWorkerWarps;
-    const bool act = b < P.nb;
-    const float* xb = xs + (size_t)b * xstride;
     float ss = 0.f;
-    for (int j = lane; j < ngroups; j += 32) {
-      const int k = k0 + j * 8;
-      float x[8];
-      if (act && k < K) {
-        const float4 a = __ldcg(reinterpret_cast<const float4*>(xb + k));
-        const float4 c = __ldcg(reinterpret_cast<const float4*>(xb + k + 4));
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-        x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
-        if (gain) {
-          const uint4 g = __ldg(reinterpret_cast<const uint4*>(gain + k));
-          x[0] *= bf16lo(g.x); x[1] *= bf16hi(g.x);
-          x[2] *= bf16lo(g.y); x[3] *= bf16hi(g.y);
-          x[4] *= bf16lo(g.z); x[5] *= bf16hi(g.z);
-          x[6] *= bf16lo(g.w); x[7] *= bf16hi(g.w);
-        }
-      } else {
+    for (int i = 0; i < kJ; ++i) {
+      const int j = lane + 32 * i;
+      if (j >= ngroups) continue;
+      const float4 a = xv[h][i][0], c = xv[h][i][1];
+      float x[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = 0.f;
-      }
+      for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+      x[0] *= bf16lo(gv[i].x); x[1] *= bf16hi(gv[i].x);
+      x[2] *= bf16lo(gv[i].y); x[3] *= bf16hi(gv[i].y);
+      x[4] *= bf16lo(gv[i].z); x[5] *= bf16hi(gv[i].z);
+      x[6] *= bf16lo(gv[i].w); x[7] *= bf16hi(gv[i].w);
       uint32_t hw[4], lw[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -846,6 +901,9 @@ __device__ __forceinline__ bool tc_task(const DecodeParams& P, DSmem& S, Pipe& p
       pp.advance();
     }
     tc_commit(&S.mma_done);
+  } else {
+    // the other workers keep the same ring cursor (attention tasks read the ring too)
+    for (int u = 0; u < nu; ++u) pp.advance();
   }
   // 3. every worker waits for the MMAs (time-bounded only: they end within microseconds once
   //    issued, and tensor memory must not be read or freed before)
@@ -858,8 +916,10 @@ __device__ __forceinline__ bool tc_task(const DecodeParams& P, DSmem& S, Pipe& p
   worker_bar();
   if (S.cabort) return false;
 
-  // 4. partial record: warps 0-3 read their 32 TMEM lanes (= rows), 32 columns each
-  float* rec = P.tpart + (size_t)t.index * kTcRecFloats;
+  // 4. partial record: warps 0-3 read their 32 TMEM lanes (= rows), 32 columns each.  A tile
+  //    covered by this task alone goes straight to shared memory and its epilogue.
+  const bool solo = t.pad0 == 1;
+  float* rec = solo ? S.tile : P.tpart + (size_t)t.index * kTcRecFloats;
   if (warp < 4) {
     float d[32];
     tc_ld32(tmem + ((uint32_t)(warp * 32) << 16), d);
@@ -872,21 +932,42 @@ __device__ __forceinline__ bool tc_task(const DecodeParams& P, DSmem& S, Pipe& p
   if (tid < kTcBatch) rec[kTcRows * kTcBatch + tid] = S.tss[tid];
   tc_fence_before();
   worker_bar();
-  if (tid == 0) {
-    const uint32_t old = atom_acq_rel_gpu_add(&P.tcnt[t.pad1], 1u);
-    S.flag = (old + 1u == P.epoch * (uint32_t)t.pad0) ? 1u : 0u;
+  if (!solo) {
+    if (tid == 0) {
+      const uint32_t old = atom_acq_rel_gpu_add(&P.tcnt[t.pad1], 1u);
+      S.flag = (old + 1u == P.epoch * (uint32_t)t.pad0) ? 1u : 0u;
+    }
+    worker_bar();
+    if (!S.flag) return true;
+    // 5. last arriver: the tile's records summed in slot order, four records per L2 round trip
+    const float* rec0 = P.tpart + (size_t)(t.index - t.aux) * kTcRecFloats;
+    constexpr int kE = (kTcRecFloats + kWorkerThreads - 1) / kWorkerThreads;
+    float v[kE];
+#pragma unroll
+    for (int i = 0; i < kE; ++i) v[i] = 0.f;
+    for (int sl0 = 0; sl0 < (int)t.pad0; sl0 += 4) {
+      float r[4][kE];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < kE; ++i) {
+          const int e = tid + i * kWorkerThreads;
+          r[q][i] = (sl0 + q < (int)t.pad0 && e < kTcRecFloats)
+                        ? __ldcg(rec0 + (size_t)(sl0 + q) * kTcRecFloats + e)
+                        : 0.f;
+        }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < kE; ++i) v[i] += r[q][i];
+    }
+#pragma unroll
+    for (int i = 0; i < kE; ++i) {
+      const int e = tid + i * kWorkerThreads;
+      if (e < kTcRecFloats) S.tile[e] = v[i];
+    }
+    worker_bar();
   }
-  worker_bar();
-  if (!S.flag) return true;
-
-  // 5. last arriver: the tile's records in slot order
-  const float* rec0 = P.tpart + (size_t)(t.index - t.aux) * kTcRecFloats;
-  for (int e = tid; e < kTcRecFloats; e += kWorkerThreads) {
-    float v = 0.f;
-    for (int sl = 0; sl < (int)t.pad0; ++sl) v += __ldcg(rec0 + (size_t)sl * kTcRecFloats + e);
-    S.tile[e] = v;
-  }
-  worker_bar();
   const float* ssum = S.tile + kTcRows * kTcBatch;
 
   // 6. epilogue: thread tid handles (row, sequence) pairs e = tid + i * 256, e = row * 16 + b
@@ -1029,6 +1110,30 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     bool ok = true;
     for (uint32_t i = qb; i < qe && ok; ++i) {
       const Task t = P.tasks[i];
+      if (t.kind == TK_ATTN) {
+        // old K/V rows of the chunk, kv_stage_keys<HD>() per stage: K rows, then V rows
+        const AttnGeom a = attn_geom(P, t);
+        int jend;
+        const int nst = attn_stage_span<HD>(a, &jend);
+        const uint16_t* kc = attn_cache<HD>(P, t, a, 0);
+        const uint16_t* vc = attn_cache<HD>(P, t, a, 1);
+        for (int st = 0; st < nst; ++st) {
+          const int jj = a.j0 + st * kv_stage_keys<HD>();
+          const uint32_t bytes = (uint32_t)min(kv_stage_keys<HD>(), jend - jj) * HD * 2u;
+          if (!wait_bar(&S.empty[pp.stage], pp.phase ^ 1u, P.timeout_ns, &S)) {
+            if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, i);
+            ok = false;
+            break;
+          }
+          uint8_t* dst = ring + (size_t)pp.stage * kSlotBytes;
+          mbar_arrive_expect_tx(&S.full[pp.stage], 2u * bytes);
+          bulk_g2s(dst, kc + (size_t)jj * HD, bytes, &S.full[pp.stage], pol);
+          bulk_g2s(dst + kv_stage_keys<HD>() * HD * 2, vc + (size_t)jj * HD, bytes, &S.full[pp.stage], pol);
+          ++issued;
+          pp.advance();
+        }
+        continue;
+      }
       if (!is_gemv(t.kind)) continue;
       uint64_t off;
       uint32_t rb;
@@ -1095,20 +1200,6 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     if (lane != 0) return;
     for (uint32_t i = qb; i < qe; ++i) {
       const Task t = P.tasks[i];
-      if (t.kind == TK_ATTN) {
-        // positions before pos were written by earlier steps: start their journey from HBM
-        // now, while this task still waits for the QKV tiles of its head group
-        const AttnGeom a = attn_geom(P, t);
-        const int j1 = min(a.j1, a.Lk - 1);  // old positions only
-        if (a.c < a.nch_eff && j1 > a.j0) {
-          const size_t head_stride = (size_t)P.max_seq * P.D;
-          const size_t kv_layer = (size_t)P.max_batch * P.nkv * head_stride;
-          const size_t off = ((size_t)a.b * P.nkv + a.g) * head_stride + (size_t)a.j0 * P.D;
-          const uint32_t bytes = (uint32_t)(j1 - a.j0) * (uint32_t)P.D * 2u;
-          prefetch_l2(P.kv + ((size_t)t.layer * 2 + 0) * kv_layer + off, bytes);
-          prefetch_l2(P.kv + ((size_t)t.layer * 2 + 1) * kv_layer + off, bytes);
-        }
-      }
       for (int w = 0; w < t.n_wait; ++w) {
         const uint32_t e = t.wait[w];
         const uint32_t target = P.epoch * P.ev_count[e];
@@ -1154,9 +1245,6 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     const Task t = t_next;
     const LayerOff lo = P.loff[t.layer < P.L ? t.layer : 0];
     if (i + 1 < qe) t_next = P.tasks[i + 1];
-    // attention: keys of earlier steps can be loaded before this step's q, k, v exist
-    AttnRegs<HD> ar;
-    if (t.kind == TK_ATTN) attn_preload<HD>(P, t, ar);
     const uint64_t t_wait = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     uint32_t stall = 0;
     // wait for the scheduler to release task i (bounded, abort-aware, then uniform decision)
@@ -1276,7 +1364,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
       }
     } else if (t.kind == TK_ATTN) {
       notify = false;  // the last chunk to arrive notifies
-      attention_task<HD>(P, S, t, ar, i);
+      if (!attention_task<HD, TC>(P, S, pp, ring, t, i, stall)) goto out;
     }
     if (P.trace && tid == 0) {
       uint64_t* rec = P.trace + (size_t)i * kTraceWords;
