@@ -241,43 +241,51 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
     }
     if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
     const uint8_t* base = ring + (size_t)pp.stage * kSlotBytes + tid * 16;
-    uint64_t acc[RPS][BM];  // per (row, sequence): (even, odd) partial sums
+    // rows in sub-blocks of RSUB (all of the stage's rows at batch width 1; two at width 4,
+    // which keeps 8 accumulator pairs live instead of 16)
+    constexpr int RSUB = (BM == 1) ? RPS : ((8 / BM) < RPS ? (8 / BM) : RPS);
 #pragma unroll
-    for (int rr = 0; rr < RPS; ++rr) {
+    for (int rs = 0; rs < RPS; rs += RSUB) {
+      uint64_t acc[RSUB][BM];  // per (row, sequence): (even, odd) partial sums
 #pragma unroll
-      for (int b = 0; b < BM; ++b) acc[rr][b] = 0ull;
-      if (RPS == 1 || r0 + rr < nrows) {
+      for (int rr = 0; rr < RSUB; ++rr) {
 #pragma unroll
-        for (int s = 0; s < NSEG; ++s) {
-          if (s < NSEG - 1 || last_ok) {
-            const uint4 w = *reinterpret_cast<const uint4*>(base + rr * row_bytes + s * kSegBytes);
-            if (BM == 1) {
-              dot8(w, x2[0][s], acc[rr][0]);
-            } else {
-              const uint64_t wp[4] = {widen_bf16w(w.x), widen_bf16w(w.y), widen_bf16w(w.z), widen_bf16w(w.w)};
-              // sequences innermost: consecutive FMAs update different accumulators
+        for (int b = 0; b < BM; ++b) acc[rr][b] = 0ull;
+        if (RPS == 1 || r0 + rs + rr < nrows) {
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
+          for (int s = 0; s < NSEG; ++s) {
+            if (s < NSEG - 1 || last_ok) {
+              const uint4 w = *reinterpret_cast<const uint4*>(base + (rs + rr) * row_bytes + s * kSegBytes);
+              if (BM == 1) {
+                dot8(w, x2[0][s], acc[rr][0]);
+              } else {
+                const uint64_t wp[4] = {widen_bf16w(w.x), widen_bf16w(w.y), widen_bf16w(w.z), widen_bf16w(w.w)};
+                // sequences innermost: consecutive FMAs update different accumulators
 #pragma unroll
-                for (int b = 0; b < BM; ++b)
-                  if (b < nb) fma2_pair(acc[rr][b], wp[j], x2[b][s][j]);
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                  for (int b = 0; b < BM; ++b)
+                    if (b < nb) fma2_pair(acc[rr][b], wp[j], x2[b][s][j]);
+              }
             }
           }
         }
       }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
-    pp.advance();
-    float a[RPS * BM];
-#pragma unroll
-    for (int rr = 0; rr < RPS; ++rr)
-#pragma unroll
-      for (int b = 0; b < BM; ++b) {
-        const float2 v = unpack2(acc[rr][b]);
-        a[rr * BM + b] = v.x + v.y;
+      if (rs + RSUB >= RPS) {  // the stage's last shared-memory read is done: release it
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
       }
-    warp_reduce_rows<RPS * BM>(a, red + r0 * BM, lane, (nrows - r0) * BM);
+      float a[RSUB * BM];
+#pragma unroll
+      for (int rr = 0; rr < RSUB; ++rr)
+#pragma unroll
+        for (int b = 0; b < BM; ++b) {
+          const float2 v = unpack2(acc[rr][b]);
+          a[rr * BM + b] = v.x + v.y;
+        }
+      warp_reduce_rows<RSUB * BM>(a, red + (r0 + rs) * BM, lane, (nrows - r0 - rs) * BM);
+    }
+    pp.advance();
   }
 #pragma unroll
   for (int b = 0; b < BM; ++b) {
@@ -418,15 +426,18 @@ __device__ __forceinline__ void attn_load_key(const uint16_t* kc, const uint16_t
 }
 
 // Online-softmax update of this warp's (m, l, acc) with one block of up to kAttnBlock keys
-// (K and V words kw/vw of this lane; key u counts if bit u of `valid` is set).
-template <int D>
+// (K and V words kw/vw of this lane; key u counts if bit u of `valid` is set) for the GW
+// (1, 2 or 4, a power of two >= G) query heads of the KV head.  The kAttnBlock x GW partial
+// dots (slot u * GW + h) are summed across lanes by warp_reduce_rows, which leaves slot r on
+// the lanes l with l % (32 / slots) == 0, and are then broadcast to every lane.
+template <int D, int GW>
 __device__ __forceinline__ void attn_block(const float (&qv)[4][D / 32], const uint32_t (&kw)[kAttnBlock][D / 64],
                                            const uint32_t (&vw)[kAttnBlock][D / 64], uint32_t valid, int G,
                                            float (&m)[4], float (&l)[4], float (&acc)[4][D / 32], int lane) {
   constexpr int DL = D / 32;
   constexpr int W = D / 64;
-  // partial dots of the block: slot u * 4 + h
-  float sc[kAttnBlock * 4];
+  constexpr int NS = kAttnBlock * GW;  // slots
+  float sc[NS];
 #pragma unroll
   for (int u = 0; u < kAttnBlock; ++u) {
     float kf[DL];
@@ -436,35 +447,44 @@ __device__ __forceinline__ void attn_block(const float (&qv)[4][D / 32], const u
       kf[2 * w + 1] = bf16hi(kw[u][w]);
     }
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
+    for (int h = 0; h < GW; ++h) {
       float sv = 0.f;
 #pragma unroll
       for (int i = 0; i < DL; ++i) sv = fmaf(qv[h][i], kf[i], sv);
-      sc[u * 4 + h] = sv;
+      sc[u * GW + h] = sv;
     }
   }
-  // transposed butterfly: lane l ends with the warp's sum of slot l ...
+  // transposed butterfly (each exchange halves the live values), then a plain one
+  constexpr int LV = ilog2(NS);
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) {
+  for (int k = 0; k < LV; ++k) {
+    const int off = 16 >> k, half = (NS >> k) >> 1;
     const bool upper = (lane & off) != 0;
 #pragma unroll
-    for (int i = 0; i < off; ++i) {
-      const float send = upper ? sc[i] : sc[i + off];
-      const float keep = upper ? sc[i + off] : sc[i];
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? sc[i] : sc[i + half];
+      const float keep = upper ? sc[i + half] : sc[i];
       sc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
     }
   }
+#pragma unroll
+  for (int off = 16 >> LV; off >= 1; off >>= 1) sc[0] += __shfl_xor_sync(0xffffffffu, sc[0], off);
+  // slot r sits on lane src(r): the bits of r, most significant first, at lane bits 4, 3, ..
   const float mine = sc[0];
-  // ... and every lane gets every slot back
 #pragma unroll
-  for (int i = 0; i < kAttnBlock * 4; ++i) sc[i] = __shfl_sync(0xffffffffu, mine, i);
+  for (int r = 0; r < NS; ++r) {
+    int src = 0;
 #pragma unroll
-  for (int h = 0; h < 4; ++h) {
+    for (int k = 0; k < LV; ++k) src |= ((r >> (LV - 1 - k)) & 1) << (4 - k);
+    sc[r] = __shfl_sync(0xffffffffu, mine, src);
+  }
+#pragma unroll
+  for (int h = 0; h < GW; ++h) {
     if (h < G) {
       float mx = m[h];
 #pragma unroll
       for (int u = 0; u < kAttnBlock; ++u)
-        if ((valid >> u) & 1u) mx = fmaxf(mx, sc[u * 4 + h]);
+        if ((valid >> u) & 1u) mx = fmaxf(mx, sc[u * GW + h]);
       const float alpha = __expf(m[h] - mx);  // 0 on the first block (m = -inf)
       float ls = 0.f;
 #pragma unroll
@@ -472,7 +492,7 @@ __device__ __forceinline__ void attn_block(const float (&qv)[4][D / 32], const u
 #pragma unroll
       for (int u = 0; u < kAttnBlock; ++u) {
         if ((valid >> u) & 1u) {
-          const float p = __expf(sc[u * 4 + h] - mx);
+          const float p = __expf(sc[u * GW + h] - mx);
           ls += p;
 #pragma unroll
           for (int w = 0; w < W; ++w) {
@@ -485,6 +505,15 @@ __device__ __forceinline__ void attn_block(const float (&qv)[4][D / 32], const u
       m[h] = mx;
     }
   }
+}
+
+template <int D>
+__device__ __forceinline__ void attn_block_g(const float (&qv)[4][D / 32], const uint32_t (&kw)[kAttnBlock][D / 64],
+                                             const uint32_t (&vw)[kAttnBlock][D / 64], uint32_t valid, int G,
+                                             float (&m)[4], float (&l)[4], float (&acc)[4][D / 32], int lane) {
+  if (G == 1) attn_block<D, 1>(qv, kw, vw, valid, G, m, l, acc, lane);
+  else if (G == 2) attn_block<D, 2>(qv, kw, vw, valid, G, m, l, acc, lane);
+  else attn_block<D, 4>(qv, kw, vw, valid, G, m, l, acc, lane);
 }
 
 // Number of ring stages of an attention task: its old positions [j0, min(j1, pos)).
@@ -561,7 +590,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
             }
           }
         }
-        if (valid) attn_block<D>(qv, kw, vw, valid, G, m, l, acc, lane);
+        if (valid) attn_block_g<D>(qv, kw, vw, valid, G, m, l, acc, lane);
       }
       // release the stage: every warp's arrival (CUDA-core ring), or one after all warps
       // (tensor-core ring, whose stages count a single release)
@@ -580,7 +609,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
         kw[0][w] = kcur[w];
         vw[0][w] = vcur[w];
       }
-      attn_block<D>(qv, kw, vw, 1u, G, m, l, acc, lane);
+      attn_block_g<D>(qv, kw, vw, 1u, G, m, l, acc, lane);
     }
     // cross-warp merge of this chunk
 #pragma unroll
