@@ -46,11 +46,15 @@ struct DSmem {
   float mm[4 * kMaxChunks], ll[4 * kMaxChunks], ww[4 * kMaxChunks];  // split-KV merge
   float lmv[kWorkerWarps];
   int lmi[kWorkerWarps];
-  float tss[kTcBatch];       // tensor-core task: per-sequence sum of x^2 over its K range
+  float tss[2][kTcBatch];    // tensor-core tasks (by parity): per-sequence sum of x^2 over the K range
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t mma_done;         // tensor-core task: its MMAs completed
-  uint32_t tmem;             // tensor-memory accumulator address
+  uint64_t bop_full[2];      // tensor-core operand buffer staged (one arrival per worker warp)
+  uint64_t bop_free[2];      // ... and read by its MMAs (tcgen05.commit)
+  uint64_t acc_full[2];      // tensor-core accumulator complete (tcgen05.commit)
+  uint64_t acc_free[2];      // ... and read back (one arrival per reading warp)
+  uint64_t mma_done;         // every MMA issued so far completed (issuer drain at exit)
+  uint32_t tmem;             // tensor-memory accumulators (2 x kTcN columns)
   uint32_t ready;            // tasks [0, ready) of this queue have their inputs
   uint32_t cabort;           // worker-role abort: written before, read after a worker barrier
   volatile uint32_t abort;   // any role gave up: stop waiting
@@ -454,8 +458,11 @@ __device__ __forceinline__ void attn_block(const float (&qv)[4][D / 32], const u
       sc[u * GW + h] = sv;
     }
   }
-  // transposed butterfly (each exchange halves the live values), then a plain one
+  // transposed butterfly (each exchange halves the live values), then a plain one: lane l
+  // ends with the warp total of slot r = l >> SH (key u = r / GW, head h = r % GW)
   constexpr int LV = ilog2(NS);
+  constexpr int SH = 5 - LV;  // log2(lanes per slot)
+  constexpr int LG = ilog2(GW);
 #pragma unroll
   for (int k = 0; k < LV; ++k) {
     const int off = 16 >> k, half = (NS >> k) >> 1;
@@ -469,40 +476,48 @@ __device__ __forceinline__ void attn_block(const float (&qv)[4][D / 32], const u
   }
 #pragma unroll
   for (int off = 16 >> LV; off >= 1; off >>= 1) sc[0] += __shfl_xor_sync(0xffffffffu, sc[0], off);
-  // slot r sits on lane src(r): the bits of r, most significant first, at lane bits 4, 3, ..
-  const float mine = sc[0];
+  // online softmax with one exponential per lane: each lane owns its slot's score
+  const int r = lane >> SH, u_me = r >> LG, h_me = r & (GW - 1);
+  const bool v_me = ((valid >> u_me) & 1u) && h_me < G;
+  const float s_me = v_me ? sc[0] : -INFINITY;
+  float mx = s_me;  // block maximum of head h_me: over the key bits of the slot index
 #pragma unroll
-  for (int r = 0; r < NS; ++r) {
-    int src = 0;
+  for (int k = 0; k < 3; ++k) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1 << (SH + LG + k)));
+  float M[GW], alpha[GW];
 #pragma unroll
-    for (int k = 0; k < LV; ++k) src |= ((r >> (LV - 1 - k)) & 1) << (4 - k);
-    sc[r] = __shfl_sync(0xffffffffu, mine, src);
+  for (int h = 0; h < GW; ++h) {
+    const float bm = __shfl_sync(0xffffffffu, mx, h << SH);  // key 0's lanes hold head h's maximum
+    M[h] = fmaxf(m[h], bm);
+    alpha[h] = (h < G) ? __expf(m[h] - M[h]) : 0.f;  // 0 on the first block (m = -inf)
   }
+  const float p_me = v_me ? __expf(s_me - M[h_me]) : 0.f;
+  float ps = p_me;  // block sum of head h_me
+#pragma unroll
+  for (int k = 0; k < 3; ++k) ps += __shfl_xor_sync(0xffffffffu, ps, 1 << (SH + LG + k));
 #pragma unroll
   for (int h = 0; h < GW; ++h) {
     if (h < G) {
-      float mx = m[h];
+      const float bs = __shfl_sync(0xffffffffu, ps, h << SH);
+      l[h] = l[h] * alpha[h] + bs;
+      m[h] = M[h];
 #pragma unroll
-      for (int u = 0; u < kAttnBlock; ++u)
-        if ((valid >> u) & 1u) mx = fmaxf(mx, sc[u * GW + h]);
-      const float alpha = __expf(m[h] - mx);  // 0 on the first block (m = -inf)
-      float ls = 0.f;
+      for (int i = 0; i < DL; ++i) acc[h][i] *= alpha[h];
+    }
+  }
+  // P.V: every lane takes each slot's probability from that slot's lanes (the V words of a
+  // key outside the block are stale or unset, so they are skipped rather than weighted by 0)
 #pragma unroll
-      for (int i = 0; i < DL; ++i) acc[h][i] *= alpha;
+  for (int u = 0; u < kAttnBlock; ++u) {
 #pragma unroll
-      for (int u = 0; u < kAttnBlock; ++u) {
-        if ((valid >> u) & 1u) {
-          const float p = __expf(sc[u * GW + h] - mx);
-          ls += p;
+    for (int h = 0; h < GW; ++h) {
+      const float p = __shfl_sync(0xffffffffu, p_me, (u * GW + h) << SH);
+      if (h < G && ((valid >> u) & 1u)) {
 #pragma unroll
-          for (int w = 0; w < W; ++w) {
-            acc[h][2 * w] = fmaf(p, bf16lo(vw[u][w]), acc[h][2 * w]);
-            acc[h][2 * w + 1] = fmaf(p, bf16hi(vw[u][w]), acc[h][2 * w + 1]);
-          }
+        for (int w = 0; w < W; ++w) {
+          acc[h][2 * w] = fmaf(p, bf16lo(vw[u][w]), acc[h][2 * w]);
+          acc[h][2 * w + 1] = fmaf(p, bf16hi(vw[u][w]), acc[h][2 * w + 1]);
         }
       }
-      l[h] = l[h] * alpha + ls;
-      m[h] = mx;
     }
   }
 }
@@ -553,9 +568,14 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       }
     }
     uint32_t kw[kAttnBlock][W], vw[kAttnBlock][W];
-    // the key and value at the current position were written in this step: warp 0 fetches
-    // them together with q (one L2 round trip) and adds them after the ring stages
-    const bool has_cur = warp == 0 && pos >= a.j0 && pos < a.j1;
+    // the key and value at the current position were written in this step: the warp that
+    // owns its slot fetches them together with q (one L2 round trip).  It takes the free slot
+    // after the old keys of the last ring stage, or (no free slot) one extra block of warp 0.
+    const int cur_rel = pos - a.j0;
+    const bool has_pos = pos >= a.j0 && pos < a.j1;
+    const bool cur_in_stage = has_pos && (cur_rel % KPS) != 0;
+    const int cur_warp = cur_in_stage ? (cur_rel % KPS) % kAttnWarps : 0;
+    const bool has_cur = has_pos && warp == cur_warp;
     uint32_t kcur[W], vcur[W];
     if (has_cur) attn_load_key<D>(kc, vc, pos, lane, kcur, vcur);
     // old positions from the ring, kv_stage_keys per stage (K rows at 0, V rows at KPS * D)
@@ -577,7 +597,14 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
 #pragma unroll
         for (int u = 0; u < kAttnBlock; ++u) {
           const int idx = kb * kAttnBlock * kAttnWarps + warp + u * kAttnWarps;
-          if (idx < nk) {
+          if (cur_in_stage && st == nst - 1 && idx == nk) {  // the current key's slot
+            valid |= 1u << u;
+#pragma unroll
+            for (int w = 0; w < W; ++w) {
+              kw[u][w] = kcur[w];
+              vw[u][w] = vcur[w];
+            }
+          } else if (idx < nk) {
             valid |= 1u << u;
             if (D == 128) {
               const uint2 kk = *reinterpret_cast<const uint2*>(kst + idx * D * 2 + lane * 8);
@@ -603,7 +630,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       }
       pp.advance();
     }
-    if (has_cur) {
+    if (has_cur && !cur_in_stage) {
 #pragma unroll
       for (int w = 0; w < W; ++w) {
         kw[0][w] = kcur[w];
@@ -803,62 +830,85 @@ __device__ __forceinline__ void warp_argmax(float& v, int& idx) {
     argmax_merge(v, idx, __shfl_xor_sync(0xffffffffu, v, off), __shfl_xor_sync(0xffffffffu, idx, off));
 }
 
-__device__ __forceinline__ bool tc_task(const DecodeParams& P, DSmem& S, Pipe& pp, const uint8_t* ring,
-                                        uint8_t* bop, const Task& t, const LayerOff& lo, uint32_t task_id,
-                                        uint32_t& stall_ns, uint32_t& mma_phase, uint32_t tmem) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const size_t lay = (size_t)t.layer * P.B;
+// Operands of a tensor-core task's op: x of sequence 0 and the stride to the next, norm gain
+// (null = none), K and the op's row count.
+struct TcOp {
   const float* xs;
-  const uint16_t* gain = nullptr;
-  int K = P.H, xstride = P.H, rows;
+  const uint16_t* gain;
+  int K, xstride, rows;
+};
+
+__device__ __forceinline__ TcOp tc_op(const DecodeParams& P, const Task& t, const LayerOff& lo) {
+  const size_t lay = (size_t)t.layer * P.B;
+  TcOp o;
+  o.gain = nullptr;
+  o.K = o.xstride = P.H;
   switch (t.kind) {
     case TK_QKV:
-      xs = P.x_in + lay * P.H;
-      gain = reinterpret_cast<const uint16_t*>(P.arena + lo.attn_norm);
-      rows = (P.nq + 2 * P.nkv) * P.D;
+      o.xs = P.x_in + lay * P.H;
+      o.gain = reinterpret_cast<const uint16_t*>(P.arena + lo.attn_norm);
+      o.rows = (P.nq + 2 * P.nkv) * P.D;
       break;
     case TK_OPROJ:
-      xs = P.obuf + lay * P.nq * P.D;
-      K = xstride = P.nq * P.D;
-      rows = P.H;
+      o.xs = P.obuf + lay * P.nq * P.D;
+      o.K = o.xstride = P.nq * P.D;
+      o.rows = P.H;
       break;
     case TK_GATEUP:
-      xs = P.x_mid + lay * P.H;
-      gain = reinterpret_cast<const uint16_t*>(P.arena + lo.mlp_norm);
-      rows = 2 * P.F;
+      o.xs = P.x_mid + lay * P.H;
+      o.gain = reinterpret_cast<const uint16_t*>(P.arena + lo.mlp_norm);
+      o.rows = 2 * P.F;
       break;
     case TK_DOWN:
-      xs = P.hbuf + lay * P.F;
-      K = xstride = P.F;
-      rows = P.H;
+      o.xs = P.hbuf + lay * P.F;
+      o.K = o.xstride = P.F;
+      o.rows = P.H;
       break;
     default:  // LM head
-      xs = P.x_in + (size_t)P.L * P.B * P.H;
-      gain = reinterpret_cast<const uint16_t*>(P.arena + P.off_fnorm);
-      rows = P.V;
+      o.xs = P.x_in + (size_t)P.L * P.B * P.H;
+      o.gain = reinterpret_cast<const uint16_t*>(P.arena + P.off_fnorm);
+      o.rows = P.V;
       break;
   }
-  const int nK = (K + kTcUnitK - 1) / kTcUnitK;
-  const int tile = (int)t.row0 / nK, u0 = (int)t.row0 % nK, nu = (int)t.nrows;
-  const int k0 = u0 * kTcUnitK, ngroups = nu * (kTcUnitK / 8);
+  return o;
+}
 
-  // 1. activation operand: warp w stages sequences w and w + 8, lane j the 8-element K groups
-  //    j, j + 32, ...; sequences outside the active batch and K past the end are zeros.  Every
-  //    load of the lane is issued before the first is used (one L2 round trip).
-  constexpr int kJ = kTcUnitsMax * kTcUnitK / 8 / 32;  // K groups per lane
+// Stage activation segment sg (kTcSegUnits K units) of task t into operand buffer gseg & 1,
+// after the MMAs that last read that buffer are done.  Warp w stages sequences w and w + 8,
+// lane j the 8-element K groups j, j + 32; sequences outside the active batch and K past the
+// end are zeros.  Every load of the lane is issued before the first is used.  The sums of x^2
+// of the task's K range accumulate in S.tss[tsb].  Each warp arrives on bop_full once its
+// stores are visible to the tensor cores.  False if the wait ran out (the caller aborts).
+__device__ __forceinline__ bool tc_stage(const DecodeParams& P, DSmem& S, uint8_t* bop, const Task& t,
+                                         const LayerOff& lo, int sg, uint32_t gseg, int tsb, uint32_t task_id) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const TcOp op = tc_op(P, t, lo);
+  const int nK = (op.K + kTcUnitK - 1) / kTcUnitK;
+  const int u0 = (int)t.row0 % nK, nu = (int)t.nrows;
+  const int su = min(kTcSegUnits, nu - sg * kTcSegUnits);
+  const int k0 = (u0 + sg * kTcSegUnits) * kTcUnitK, ngroups = su * (kTcUnitK / 8);
+  const uint32_t buf = gseg & 1u, use = gseg >> 1;
+  bool ok = wait_bar(&S.bop_free[buf], (use & 1u) ^ 1u, P.timeout_ns, &S);
+  if (!ok) {
+    raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
+    S.cabort = 1u;
+  }
+  tc_fence_after();
+  uint8_t* ob = bop + buf * kTcBopBuf;
+  constexpr int kJ = kTcSegUnits * kTcUnitK / 8 / 32;  // K groups per lane
   float4 xv[2][kJ][2];
   uint4 gv[kJ];
 #pragma unroll
   for (int i = 0; i < kJ; ++i) {
     const int j = lane + 32 * i, k = k0 + j * 8;
-    const bool in = j < ngroups && k < K;
-    gv[i] = (in && gain) ? __ldg(reinterpret_cast<const uint4*>(gain + k))
-                         : make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);  // bf16 1.0 pairs
+    const bool in = j < ngroups && k < op.K;
+    gv[i] = (in && op.gain) ? __ldg(reinterpret_cast<const uint4*>(op.gain + k))
+                            : make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);  // bf16 1.0 pairs
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int b = warp + h * kWorkerWarps;
       if (in && b < P.nb) {
-        const float* xb = xs + (size_t)b * xstride + k;
+        const float* xb = op.xs + (size_t)b * op.xstride + k;
         xv[h][i][0] = __ldcg(reinterpret_cast<const float4*>(xb));
         xv[h][i][1] = __ldcg(reinterpret_cast<const float4*>(xb + 4));
       } else {
@@ -891,56 +941,108 @@ __device__ __forceinline__ bool tc_task(const DecodeParams& P, DSmem& S, Pipe& p
         lw[q] = (uint32_t)l0 | ((uint32_t)l1 << 16);
       }
       const int hrow = b, lrow = kTcBatch + b;  // operand rows (MMA N index)
-      *reinterpret_cast<uint4*>(bop + (hrow >> 3) * kTcBopSbo + j * 128 + (hrow & 7) * 16) =
+      *reinterpret_cast<uint4*>(ob + (hrow >> 3) * kTcBopSbo + j * 128 + (hrow & 7) * 16) =
           make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(bop + (lrow >> 3) * kTcBopSbo + j * 128 + (lrow & 7) * 16) =
+      *reinterpret_cast<uint4*>(ob + (lrow >> 3) * kTcBopSbo + j * 128 + (lrow & 7) * 16) =
           make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if (lane == 0) S.tss[b] = ss;
+    if (lane == 0) S.tss[tsb][b] = (sg == 0) ? ss : S.tss[tsb][b] + ss;
   }
   fence_proxy_async_smem();
-  tc_fence_before();
-  worker_bar();
-  tc_fence_after();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&S.bop_full[buf]);
+  return ok;
+}
 
-  // 2. one thread issues the MMAs of every K unit as its weight block lands; each stage is
-  //    released to the producer by a commit once its MMAs are done
-  if (tid == 0) {
-    const uint32_t b_base = smem_u32(bop);
-    for (int u = 0; u < nu; ++u) {
-      const uint64_t tw = P.trace ? globaltimer_ns() : 0;
-      if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
-        raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
-        S.cabort = 1u;
+// MMA issuer (one thread of the tensor-core kernel's issuer warp): walks the queue like the
+// workers; for each tensor-core task waits for a free accumulator, then per segment for the
+// staged operand, and issues 8 tcgen05.mma per weight block as the block lands.  Each ring
+// stage is released by a commit once its MMAs are done, each operand buffer after its
+// segment's MMAs, and the accumulator is announced full after the task's last MMA.
+// Attention stages of the ring belong to the workers: the cursor only steps over them.
+template <int HD>
+__device__ __forceinline__ void tc_issuer(const DecodeParams& P, DSmem& S, const uint8_t* ring, const uint8_t* bop,
+                                          uint32_t qb, uint32_t qe, uint32_t tmem) {
+  Pipe pp{0, 0, kTcStages};
+  uint32_t gseg = 0, gtask = 0;
+  const uint32_t b_base0 = smem_u32(bop);
+  for (uint32_t i = qb; i < qe; ++i) {
+    const Task t = P.tasks[i];
+    if (t.kind == TK_ATTN) {
+      int jend;
+      const int nst = attn_stage_span<HD>(attn_geom(P, t), &jend);
+      for (int st = 0; st < nst; ++st) pp.advance();
+      continue;
+    }
+    if (!is_gemv(t.kind)) continue;
+    const uint32_t ab = gtask & 1u, av = gtask >> 1;
+    if (!wait_bar(&S.acc_free[ab], (av & 1u) ^ 1u, P.timeout_ns, &S)) {
+      if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, i);
+      break;
+    }
+    tc_fence_after();
+    const uint32_t d_tmem = tmem + ab * kTcN;
+    const int nu = (int)t.nrows, nseg = (nu + kTcSegUnits - 1) / kTcSegUnits;
+    bool ok = true;
+    for (int sg = 0; sg < nseg && ok; ++sg) {
+      const uint32_t buf = gseg & 1u, use = gseg >> 1;
+      if (!wait_bar(&S.bop_full[buf], use & 1u, P.timeout_ns, &S)) {
+        if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, i);
+        ok = false;
         break;
       }
-      if (P.trace) stall_ns += (uint32_t)(globaltimer_ns() - tw);
       tc_fence_after();
-      const uint32_t a_base = smem_u32(ring + (size_t)pp.stage * kSlotBytes);
+      const uint32_t b_base = b_base0 + buf * kTcBopBuf;
+      const int su = min(kTcSegUnits, nu - sg * kTcSegUnits);
+      for (int u = 0; u < su; ++u) {
+        if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
+          if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, i);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(ring + (size_t)pp.stage * kSlotBytes);
 #pragma unroll
-      for (int s = 0; s < kTcUnitK / 16; ++s) {
-        // K step s: core-matrix columns 2s, 2s + 1 (256 bytes) of the block / of unit u
-        const uint64_t ad = tc_smem_desc(a_base + s * 256, 128, (kTcUnitK / 8) * 128);
-        const uint64_t bd = tc_smem_desc(b_base + u * (kTcUnitK / 8) * 128 + s * 256, 128, kTcBopSbo);
-        tc_mma_f16(tmem, ad, bd, kTcIdesc, (u | s) != 0 ? 1u : 0u);
+        for (int s = 0; s < kTcUnitK / 16; ++s) {
+          // K step s: core-matrix columns 2s, 2s + 1 (256 bytes) of the block / of unit u
+          const uint64_t ad = tc_smem_desc(a_base + s * 256, 128, (kTcUnitK / 8) * 128);
+          const uint64_t bd = tc_smem_desc(b_base + u * (kTcUnitK / 8) * 128 + s * 256, 128, kTcBopSbo);
+          tc_mma_f16(d_tmem, ad, bd, kTcIdesc, (sg | u | s) != 0 ? 1u : 0u);
+        }
+        tc_commit(&S.empty[pp.stage]);
+        pp.advance();
       }
-      tc_commit(&S.empty[pp.stage]);
-      pp.advance();
+      tc_commit(&S.bop_free[buf]);
+      ++gseg;
     }
-    tc_commit(&S.mma_done);
-  } else {
-    // the other workers keep the same ring cursor (attention tasks read the ring too)
-    for (int u = 0; u < nu; ++u) pp.advance();
+    if (!ok) break;
+    tc_commit(&S.acc_full[ab]);
+    ++gtask;
   }
-  // 3. every worker waits for the MMAs (time-bounded only: they end within microseconds once
-  //    issued, and tensor memory must not be read or freed before)
-  if (!wait_bar(&S.mma_done, mma_phase, P.timeout_ns, nullptr)) {
+  // leave no MMA in flight: tensor memory is freed after this
+  tc_commit(&S.mma_done);
+  wait_bar(&S.mma_done, 0, P.timeout_ns, nullptr);
+}
+
+// Worker side of a tensor-core task after its segments were staged: wait for the accumulator,
+// read it back, then the partial record / tile epilogue.  False (for every worker alike) if a
+// wait ran out.
+__device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const Task& t, const LayerOff& lo,
+                                          uint32_t tmem, uint32_t gtask, int tsb, uint32_t task_id) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t lay = (size_t)t.layer * P.B;
+  const TcOp op = tc_op(P, t, lo);
+  const uint16_t* gain = op.gain;
+  const int K = op.K, rows = op.rows;
+  const int nK = (K + kTcUnitK - 1) / kTcUnitK;
+  const int tile = (int)t.row0 / nK;
+  const uint32_t ab = gtask & 1u, av = gtask >> 1;
+  if (!wait_bar(&S.acc_full[ab], av & 1u, P.timeout_ns, &S)) {
     raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
     S.cabort = 1u;
   }
-  mma_phase ^= 1u;
   tc_fence_after();
   worker_bar();
   if (S.cabort) return false;
@@ -951,14 +1053,17 @@ __device__ __forceinline__ bool tc_task(const DecodeParams& P, DSmem& S, Pipe& p
   float* rec = solo ? S.tile : P.tpart + (size_t)t.index * kTcRecFloats;
   if (warp < 4) {
     float d[32];
-    tc_ld32(tmem + ((uint32_t)(warp * 32) << 16), d);
+    tc_ld32(tmem + ab * kTcN + ((uint32_t)(warp * 32) << 16), d);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.acc_free[ab]);  // the issuer may reuse the accumulator
     float4* dst = reinterpret_cast<float4*>(rec + (warp * 32 + lane) * kTcBatch);
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       dst[q] = make_float4(d[4 * q] + d[kTcBatch + 4 * q], d[4 * q + 1] + d[kTcBatch + 4 * q + 1],
                            d[4 * q + 2] + d[kTcBatch + 4 * q + 2], d[4 * q + 3] + d[kTcBatch + 4 * q + 3]);
   }
-  if (tid < kTcBatch) rec[kTcRows * kTcBatch + tid] = S.tss[tid];
+  if (tid < kTcBatch) rec[kTcRows * kTcBatch + tid] = S.tss[tsb][tid];
   tc_fence_before();
   worker_bar();
   if (!solo) {
@@ -1077,7 +1182,8 @@ __device__ __forceinline__ bool tc_task(const DecodeParams& P, DSmem& S, Pipe& p
 
 // ---------------------------------------------------------------------------------------
 template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM>
-__global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
+__global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBlockThreads, 1)
+    decode_kernel(const __grid_constant__ DecodeParams P) {
   constexpr bool TC = BM > kMaxDecodeBatch;  // tensor-core projection tiles
   constexpr int BMC = TC ? 1 : BM;            // CUDA-core GEMV batch width (unused when TC)
   constexpr int NST = ring_stages(TC);
@@ -1094,13 +1200,34 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
       mbar_init(&S.empty[s], TC ? 1 : kWorkerWarps);  // tensor-core stages: released by a commit
     }
     mbar_init(&S.mma_done, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.bop_full[b], kWorkerWarps);
+      mbar_init(&S.bop_free[b], 1);
+      mbar_init(&S.acc_full[b], 1);
+      mbar_init(&S.acc_free[b], 4);
+    }
     S.ready = 0;
     S.cabort = 0;
     S.abort = 0;
     S.flag = 0;
     fence_mbar_init();
   }
+  if (TC && warp == 0) {  // two 32-column fp32 accumulators (128 lanes) for the whole kernel
+    tc_alloc(&S.tmem, 2 * kTcN);
+    tc_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = TC ? S.tmem : 0u;
+
+  if (TC && warp == kIssuerWarp) {
+    // ------------------------------- MMA issuer ------------------------------
+    if (lane == 0) tc_issuer<HD>(P, S, ring, bop, qb, qe, tmem);
+    __syncwarp();
+    named_bar_sync(2, kWorkerThreads + 32);  // with the workers, before tensor memory is freed
+    return;
+  }
 
   if (warp == kProducerWarp) {
     // ------------------------------- producer -------------------------------
@@ -1256,17 +1383,10 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
 
   // --------------------------------- workers ---------------------------------
   Pipe pp{0, 0, NST};
-  uint32_t tmem = 0, mma_phase = 0;
-  if (TC) {  // one 32-column fp32 accumulator (128 lanes) for the whole kernel
-    if (warp == 0) {
-      tc_alloc(&S.tmem, kTcN);
-      tc_relinquish();
-    }
-    tc_fence_before();
-    worker_bar();
-    tc_fence_after();
-    tmem = S.tmem;
-  }
+  // tensor-core pipeline (workers): operand segments staged and tasks finished so far, and
+  // whether the next task's first segment was staged ahead
+  uint32_t gseg = 0, gtask = 0;
+  bool staged_ahead = false;
   // descriptor (and layer offsets) of the next task are loaded while the worker still waits
   // for that task's inputs, so only the activation loads remain after the release
   Task t_next = P.tasks[qb < qe ? qb : 0];
@@ -1301,7 +1421,40 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     const uint64_t t_ready = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     bool notify = true;
     if (TC && is_gemv(t.kind)) {
-      if (!tc_task(P, S, pp, ring, bop, t, lo, i, stall, mma_phase, tmem)) goto out;
+      const int nu = (int)t.nrows, nseg = (nu + kTcSegUnits - 1) / kTcSegUnits;
+      const int tsb = (int)(gtask & 1u);
+      bool ok = true;
+      for (int sg = staged_ahead ? 1 : 0; sg < nseg; ++sg) ok &= tc_stage(P, S, bop, t, lo, sg, gseg++, tsb, i);
+      staged_ahead = false;
+      // the next task of the same op has this task's inputs: stage its first segment now, so
+      // the tensor cores go on with it while this task is read back and finished
+      if (ok && i + 1 < qe && t_next.kind == t.kind && t_next.layer == t.layer) {
+        uint64_t t0 = 0;
+        for (uint32_t n = 1;; ++n) {  // its release (immediate: same events as this task)
+          if (ld_acquire_cta_shared(&S.ready) > i + 1 - qb) break;
+          if ((n & 63u) == 0) {
+            if (S.abort) {
+              ok = false;
+              break;
+            }
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > P.timeout_ns + 1000000000ull) {
+              raise_error(P, S, DEV_ERR_WAIT_READY, blockIdx.x, i + 1);
+              ok = false;
+              break;
+            }
+          }
+        }
+        if (ok) {
+          ok = tc_stage(P, S, bop, t_next, lo, 0, gseg++, (int)((gtask + 1) & 1u), i + 1);
+          staged_ahead = true;
+        }
+      }
+      if (!ok) S.cabort = 1u;
+      for (int u = 0; u < nu; ++u) pp.advance();  // the task's weight blocks go to the issuer
+      if (!tc_finish(P, S, t, lo, tmem, gtask, tsb, i)) goto out;
+      ++gtask;
       if (t.kind == TK_LMHEAD) notify = false;
     } else if (is_gemv(t.kind)) {
       // operands of the task's GEMV: x source of sequence 0 and the stride to the next, norm
@@ -1411,11 +1564,11 @@ __global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel(const __grid_c
     }
   }
 out:
-  if (TC) {  // every worker thread arrives here together; no MMA is in flight
+  if (TC) {  // every worker thread and the issuer warp (which drained its MMAs) meet here
     tc_fence_before();
-    worker_bar();
+    named_bar_sync(2, kWorkerThreads + 32);
     tc_fence_after();
-    if (warp == 0) tc_dealloc(tmem, kTcN);
+    if (warp == 0) tc_dealloc(tmem, 2 * kTcN);
   }
 }
 
@@ -1481,7 +1634,8 @@ int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t str
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess) {
     void* args[] = {const_cast<DecodeParams*>(&p)};
-    e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(kBlockThreads), args, smem, stream);
+    const bool tc = kVariants[variant].bm > kMaxDecodeBatch;
+    e = cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(tc ? kTcBlockThreads : kBlockThreads), args, smem, stream);
   }
   if (e != cudaSuccess) {
     *err = std::string("decode launch: ") + cudaGetErrorString(e);

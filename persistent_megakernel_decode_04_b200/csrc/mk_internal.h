@@ -26,6 +26,8 @@ constexpr int kWorkerThreads = kWorkerWarps * 32;    // 256
 constexpr int kProducerWarp = kWorkerWarps;          // TMA weight streaming
 constexpr int kSchedWarp = kWorkerWarps + 1;         // event polling (the "scheduler" role)
 constexpr int kBlockThreads = (kWorkerWarps + 2) * 32;
+constexpr int kIssuerWarp = kWorkerWarps + 2;        // tensor-core kernel: tcgen05.mma issue
+constexpr int kTcBlockThreads = (kWorkerWarps + 3) * 32;
 constexpr int kSegElems = kWorkerThreads * 8;        // K elements one pass of all workers covers
 constexpr int kSegBytes = kSegElems * 2;
 constexpr int kTaskRows = 256;                       // rows per GEMV task (one per worker thread)
@@ -43,15 +45,18 @@ constexpr int kMaxDecodeBatch = 4;                   // CUDA-core path: batch wi
 constexpr int kDownChunk = 4096;                     // down-projection K chunk for batch width 4
 // Tensor-core projection tiles (batch width 5..16): a tile is kTcRows weight rows; a ring
 // stage is one block of kTcRows x kTcUnitK bf16 weights in the no-swizzle K-major core-matrix
-// layout; a task covers up to kTcUnitsMax blocks (K units) of one tile.
+// layout; a task covers up to kTcUnitsMax blocks (K units) of one tile.  Activations are
+// staged kTcSegUnits units at a time into one of two operand buffers.
 constexpr int kTcBatch = 16;                         // sequences per tensor-core step (MMA N = 2 x 16)
 constexpr int kTcN = 2 * kTcBatch;                   // columns: bf16 high parts, then low parts
 constexpr int kTcRows = 128;                         // MMA M
 constexpr int kTcUnitK = 128;                        // K elements per ring stage
-constexpr int kTcUnitsMax = 8;                       // K units per task
+constexpr int kTcUnitsMax = 64;                      // K units per task
+constexpr int kTcSegUnits = 4;                       // K units per activation segment
 constexpr int kTcStages = 4;                         // ring depth of the tensor-core kernel
-constexpr int kTcBopSbo = kTcUnitsMax * kTcUnitK / 8 * 128;  // activation operand: bytes per 8-row group
-constexpr int kTcBopBytes = (kTcN / 8) * kTcBopSbo;  // 64 KB
+constexpr int kTcBopSbo = kTcSegUnits * kTcUnitK / 8 * 128;  // operand buffer: bytes per 8-row group
+constexpr int kTcBopBuf = (kTcN / 8) * kTcBopSbo;   // one operand buffer (32 KB)
+constexpr int kTcBopBytes = 2 * kTcBopBuf;          // two buffers
 constexpr int kTcRecFloats = kTcRows * kTcBatch + kTcBatch;  // partial record: [row][seq] sums, seq sum of x^2
 static_assert(kTcRows * kTcUnitK * 2 == MK_SLOT_KB * 1024, "a weight block fills one ring stage");
 
