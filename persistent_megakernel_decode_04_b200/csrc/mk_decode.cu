@@ -1387,13 +1387,15 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
   // whether the next task's first segment was staged ahead
   uint32_t gseg = 0, gtask = 0;
   bool staged_ahead = false;
-  // descriptor (and layer offsets) of the next task are loaded while the worker still waits
-  // for that task's inputs, so only the activation loads remain after the release
+  // batch width 1: the next task's descriptor is loaded during the current task, so only the
+  // activation loads remain after its release; wider kernels load it at the top of its own
+  // iteration instead, which keeps 10 registers free across the GEMV
+  constexpr bool kHoist = (BM == 1);
   Task t_next = P.tasks[qb < qe ? qb : 0];
   for (uint32_t i = qb; i < qe; ++i) {
-    const Task t = t_next;
+    const Task t = kHoist ? t_next : P.tasks[i];
     const LayerOff lo = P.loff[t.layer < P.L ? t.layer : 0];
-    if (i + 1 < qe) t_next = P.tasks[i + 1];
+    if (kHoist && i + 1 < qe) t_next = P.tasks[i + 1];
     const uint64_t t_wait = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     uint32_t stall = 0;
     // wait for the scheduler to release task i (bounded, abort-aware, then uniform decision)
@@ -1428,7 +1430,8 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       staged_ahead = false;
       // the next task of the same op has this task's inputs: stage its first segment now, so
       // the tensor cores go on with it while this task is read back and finished
-      if (ok && i + 1 < qe && t_next.kind == t.kind && t_next.layer == t.layer) {
+      const Task tn = P.tasks[i + 1 < qe ? i + 1 : i];
+      if (ok && i + 1 < qe && tn.kind == t.kind && tn.layer == t.layer) {
         uint64_t t0 = 0;
         for (uint32_t n = 1;; ++n) {  // its release (immediate: same events as this task)
           if (ld_acquire_cta_shared(&S.ready) > i + 1 - qb) break;
@@ -1447,7 +1450,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
           }
         }
         if (ok) {
-          ok = tc_stage(P, S, bop, t_next, lo, 0, gseg++, (int)((gtask + 1) & 1u), i + 1);
+          ok = tc_stage(P, S, bop, tn, lo, 0, gseg++, (int)((gtask + 1) & 1u), i + 1);
           staged_ahead = true;
         }
       }

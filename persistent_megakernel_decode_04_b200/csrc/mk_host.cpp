@@ -80,7 +80,7 @@ struct mk_ctx {
   uint64_t timeout_ns = 2000000000ull;
   int drop_event = -1;
   uint64_t* trace = nullptr;
-  int l2_ahead = 0;
+  int l2_ahead = 8;  // L2 lookahead stages while the ring is full (mk_set_l2_prefetch)
   std::vector<double> sm_weights;  // relative streaming speed per SM (partition weights)
   size_t task_cap = 0, lm_cap = 0; // workspace capacity for re-partitioned graphs
   std::string err;
