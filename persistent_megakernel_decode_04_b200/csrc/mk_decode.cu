@@ -619,15 +619,9 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
         }
         if (valid) attn_block_g<D>(qv, kw, vw, valid, G, m, l, acc, lane);
       }
-      // release the stage: every warp's arrival (CUDA-core ring), or one after all warps
-      // (tensor-core ring, whose stages count a single release)
-      if (TC) {
-        worker_bar();
-        if (tid == 0) mbar_arrive(&S.empty[pp.stage]);
-      } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
-      }
+      // release the stage: one arrival per warp once its reads are done
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
       pp.advance();
     }
     if (has_cur && !cur_in_stage) {
@@ -1011,7 +1005,10 @@ __device__ __forceinline__ void tc_issuer(const DecodeParams& P, DSmem& S, const
           const uint64_t bd = tc_smem_desc(b_base + u * (kTcUnitK / 8) * 128 + s * 256, 128, kTcBopSbo);
           tc_mma_f16(d_tmem, ad, bd, kTcIdesc, (sg | u | s) != 0 ? 1u : 0u);
         }
-        tc_commit(&S.empty[pp.stage]);
+        // the stage's release counts one arrival per worker warp (attention stages are released
+        // warp by warp): the issuer's commit arrives as all of them once its MMAs are done
+#pragma unroll
+        for (int k = 0; k < kWorkerWarps; ++k) tc_commit(&S.empty[pp.stage]);
         pp.advance();
       }
       tc_commit(&S.bop_free[buf]);
@@ -1197,7 +1194,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
   if (tid == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], TC ? 1 : kWorkerWarps);  // tensor-core stages: released by a commit
+      mbar_init(&S.empty[s], kWorkerWarps);  // one release per worker warp (tensor-core: 8 commits)
     }
     mbar_init(&S.mma_done, 1);
     for (int b = 0; b < 2; ++b) {
