@@ -175,8 +175,12 @@ typedef struct mk_graph_info {
 int mk_get_graph_info(const mk_ctx* ctx, mk_graph_info* out);
 
 /* Flat copy of the task graph: per task {kind, layer, sm, row0, nrows, n_wait, wait0,
- * wait1, n_notify, notify0, notify1} as 11 int32; per event its per-step count.  Returns
- * the number of tasks (or a negative error); either buffer may be NULL to query sizes. */
+ * wait1, n_notify, notify0, notify1} as 11 int32; per event its per-step count.  For an
+ * attention task row0 = sequence * n_kv_heads + KV head and nrows = its split-KV chunk; for a
+ * projection task of a tensor-core context (max_batch > 4) row0 = its first 128 x 128 weight
+ * block (tile * K blocks + K block) and nrows = its block count; otherwise row0/nrows are
+ * packed weight rows.  Returns the number of tasks (or a negative error); either buffer may
+ * be NULL to query sizes. */
 int mk_export_taskgraph(const mk_ctx* ctx, int32_t* tasks, int task_capacity, int32_t* event_counts,
                         int event_capacity);
 
