@@ -48,6 +48,7 @@ WORKLOADS = {
     "chameleon7b-b1": ("CHAMELEON7B", 1, 1024),
     "chameleon7b-b4": ("CHAMELEON7B", 4, 1024),
     "chameleon7b-b16": ("CHAMELEON7B", 16, 1024),
+    "attention": (None, 0, 0),  # the standalone decode-attention op, Mirage size
 }
 WORKLOAD_TEXT = {
     "llama8b": "llama3-8b-shape decode, batch 1, 39-token prompt, greedy",
@@ -56,6 +57,8 @@ WORKLOAD_TEXT = {
     "chameleon7b-b4": "chameleon-7b-shape MHA decode, batch 4, 1024 cached positions each (synthetic), greedy",
     "chameleon7b-b16": "chameleon-7b-shape MHA decode, batch 16 (tensor-core projections), 1024 cached positions "
                        "each (synthetic), greedy",
+    "attention": "standalone decode attention O = softmax(Q.K).V, fp16 Q [64,1,128], K^T [64,128,4096], "
+                 "V [64,4096,128], fp32 out, 3 rotating input copies",
 }
 
 
@@ -257,6 +260,83 @@ def run_reference(args, rank, world):
     print(json.dumps(out), flush=True)
 
 
+def run_attention(args, rank, world, local):
+    """The standalone decode-attention op at the Mirage size: one call per step, inputs rotated
+    over three seeded copies (3 x 134 MB > L2) so no call finds its K/V in L2."""
+    import torch
+    import mk_inputs as mi
+    import persistent_megakernel_decode_04_b200 as mk
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    BH, D, L = 64, 128, 4096
+    sets = []
+    for c in range(3):
+        q, kt, v = (torch.from_numpy(mi.normal_f16(c, i + 1, shape).view(np.int16)).to(dev)
+                    for i, shape in enumerate(((BH, D), (BH, D, L), (BH, L, D))))
+        sets.append((q, kt, v))
+    o = torch.empty((BH, D), dtype=torch.float32, device=dev)
+    ws = torch.zeros(mk.mk_attention_workspace_bytes(BH, D, L), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for i in range(args.warmup):
+        q, kt, v = sets[i % 3]
+        mk.mk_attention_decode(q, kt, v, o, BH, D, L, 1.0, ws)
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(uuid) as clk:
+        start.record(stream)
+        for i, (a, b) in enumerate(ev):
+            q, kt, v = sets[i % 3]
+            a.record(stream)
+            mk.mk_attention_decode(q, kt, v, o, BH, D, L, 1.0, ws)
+            b.record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if mk.mk_attention_status(ws, BH, D, L) != mk.MK_OK:
+        raise SystemExit("attention reported an error status")
+    us = np.array([a.elapsed_time(b) for a, b in ev]) * 1e3
+    total_us = start.elapsed_time(stop) * 1e3 / args.steps
+    alg = BH * L * D * 2 * 2 + BH * D * 2 + BH * D * 4  # K and V once, q, o
+    peak, peak_kind = measured_peaks()
+    achieved = alg / (us.mean() * 1e-6) / 1e9
+    # end to end: host inputs (pinned) copied in and o copied out every call
+    hq, hk, hv = (t.cpu().pin_memory() for t in sets[0])
+    ho = torch.empty_like(o, device="cpu").pin_memory()
+    q, kt, v = sets[0]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, min(args.e2e_steps, 16))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        q.copy_(hq, non_blocking=True)
+        kt.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        mk.mk_attention_decode(q, kt, v, o, BH, D, L, 1.0, ws)
+        ho.copy_(o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if rank == 0:
+        out = {"metric": "standalone decode attention us/call + achieved HBM GB/s, Mirage size, 1 B200",
+               "value": float(us.mean()), "unit": "us/call", "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": float(us.mean()) / 1e3, "higher_is_better": False,
+               "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic (seeded N(0,1))",
+               "config": {"workload": WORKLOAD_TEXT["attention"], "BH": BH, "head_dim": D, "keys": L,
+                          "l2": "3 rotating input copies (402 MB > L2)"},
+               "us_p50": float(np.median(us)), "us_per_call_back_to_back": total_us,
+               "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                            "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                            "algorithmic_bytes_per_launch": alg},
+               "e2e": {"value": e0.elapsed_time(e1) * 1e3 / n_e2e, "unit": "us/call",
+                       "h2d_bytes_per_step": (BH * D + 2 * BH * L * D) * 2, "d2h_bytes_per_step": BH * D * 4,
+                       "steps": n_e2e},
+               "gpu_launches": args.steps, "clocks": clk.summary()}
+        print(json.dumps(out), flush=True)
+
+
 def run_mk(args, rank, world, local):
     import torch
     import torch.distributed as dist
@@ -424,6 +504,8 @@ def main():
         sys.exit(2)
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.workload == "attention":
+        run_attention(args, rank, world, local)
     else:
         run_mk(args, rank, world, local)
 

@@ -122,6 +122,19 @@ int mk_get_positions(const mk_ctx* ctx, int32_t* host_pos, int capacity);
 int mk_decode_step(mk_ctx* ctx, const int32_t* tokens, void* kv_cache, float* logits, int32_t* next_tokens,
                    void* stream);
 
+/* Several greedy decode steps in ONE launch of the persistent megakernel (the token picked
+ * by step s, lowest index on ties, is the input of step s + 1 without leaving the device).
+ * tokens: device int32 [B] for the first step; tokens_out: device int32 [n_steps][max_batch]
+ * (row s, entries b < B: the token picked by step s; required); logits: device fp32
+ * [B][vocab], left holding the
+ * last step's.  1 <= n_steps <= MK_MAX_STEPS and pos[b] + n_steps <= max_seq, else
+ * MK_ERR_INVALID_ARG.  The result equals n_steps mk_decode_step calls fed with their own
+ * picks.  Inside the launch, cache rows written by its earlier steps are read from memory
+ * after their producers finished, not streamed ahead. */
+#define MK_MAX_STEPS 4096
+int mk_decode_steps(mk_ctx* ctx, const int32_t* tokens, int n_steps, void* kv_cache, float* logits,
+                    int32_t* tokens_out, void* stream);
+
 /* Synchronise `stream` and report the device status of the steps run on it:
  * MK_OK, or MK_ERR_DEVICE_TIMEOUT (the event counters are then reset so the context
  * stays usable; the cache contents of the failed step are undefined). */

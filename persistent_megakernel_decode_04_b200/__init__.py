@@ -76,6 +76,7 @@ _SIGS = {
     "mk_set_positions": ([_vp, _vp, _i32], _i32),
     "mk_get_positions": ([_vp, _vp, _i32], _i32),
     "mk_decode_step": ([_vp, _vp, _vp, _vp, _vp, _vp], _i32),
+    "mk_decode_steps": ([_vp, _vp, _i32, _vp, _vp, _vp, _vp], _i32),
     "mk_sync_status": ([_vp, _vp], _i32),
     "mk_set_wait_timeout_ns": ([_vp, _u64], _i32),
     "mk_debug_drop_notify": ([_vp, _i32, _i32], _i32),
@@ -192,6 +193,11 @@ def mk_get_positions(ctx, capacity: int = MK_MAX_BATCH):
 def mk_decode_step(ctx, tokens, kv_cache, logits, next_tokens=None, stream=None):
     _check(_lib.mk_decode_step(ctx, _ptr(tokens), _ptr(kv_cache), _ptr(logits), _ptr(next_tokens),
                                _stream(stream)), ctx)
+
+
+def mk_decode_steps(ctx, tokens, n_steps: int, kv_cache, logits, tokens_out, stream=None):
+    _check(_lib.mk_decode_steps(ctx, _ptr(tokens), int(n_steps), _ptr(kv_cache), _ptr(logits), _ptr(tokens_out),
+                                _stream(stream)), ctx)
 
 
 def mk_sync_status(ctx, stream=None) -> int:
@@ -341,6 +347,15 @@ class Megakernel:
         B = tokens.shape[0]
         mk_decode_step(self.ctx, tokens, self.kv, self.logits, self.next_tokens, self.stream)
         return self.logits[:B], self.next_tokens[:B]
+
+    def decode_steps(self, tokens, n_steps: int):
+        """n_steps greedy decode steps in one launch, starting from tokens (int32 CUDA [B]);
+        returns (logits of the last step [B, vocab], picked tokens [n_steps, B])."""
+        import torch
+        B = tokens.shape[0]
+        out = torch.empty((n_steps, self.cfg.max_batch), dtype=torch.int32, device=tokens.device)
+        mk_decode_steps(self.ctx, tokens, n_steps, self.kv, self.logits, out, self.stream)
+        return self.logits[:B], out[:, :B]
 
     def calibrate(self, tokens, steps: int = 2, rounds: int = 3):
         """Measure each SM's busy time on the projection tasks over `steps` traced decode steps

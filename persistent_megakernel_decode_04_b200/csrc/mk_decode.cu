@@ -321,11 +321,12 @@ __device__ __forceinline__ float norm_factor(const DSmem& S, int K, float eps, i
 // GEMV total is S.tot[e] (sequences b >= nb are skipped).
 // Packed QKV row R of sequence b (value v; other = its RoPE partner row R ^ 1): q rows go to
 // qbuf after RoPE, k rows after RoPE and v rows as they are into the bf16 cache at pos[b].
-__device__ __forceinline__ void qkv_out(const DecodeParams& P, int layer, int R, int b, float v, float other) {
+__device__ __forceinline__ void qkv_out(const DecodeParams& P, int layer, int R, int b, float v, float other,
+                                        int st) {
   const int D = P.D, G = P.nq / P.nkv, half = D / 2;
   const int rpg = (G + 2) * D;
   const int grp = R / rpg, rr = R % rpg;
-  const int pos = P.pos[b];
+  const int pos = P.pos[b] + st;  // step st of the launch
   const size_t head_stride = (size_t)P.max_seq * D;
   const size_t kv_layer = (size_t)P.max_batch * P.nkv * head_stride;  // one of K or V, one layer
   if (rr < (G + 1) * D) {
@@ -357,12 +358,12 @@ __device__ __forceinline__ void qkv_out(const DecodeParams& P, int layer, int R,
 }
 
 template <int BM>
-__device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, const Task& t, float r) {
+__device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, const Task& t, float r, int st) {
   const int tid = threadIdx.x;
   const int b = tid % BM;
   if (tid >= (int)t.nrows * BM || b >= P.nb) return;
   // the RoPE partner row (R ^ 1) of the same sequence sits at tid ^ BM
-  qkv_out(P, t.layer, (int)t.row0 + tid / BM, b, S.tot[tid] * r, S.tot[tid ^ BM] * r);
+  qkv_out(P, t.layer, (int)t.row0 + tid / BM, b, S.tot[tid] * r, S.tot[tid ^ BM] * r, st);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -386,15 +387,19 @@ template <int D>
 __host__ __device__ constexpr int kv_stage_keys() { return kSlotBytes / (2 * D * 2); }
 
 struct AttnGeom {
-  int b, g, c, Lk, nch_eff, j0, j1;
+  int b, g, c, Lk, nch_eff, j0, j1, pos0;
 };
 
-__device__ __forceinline__ AttnGeom attn_geom(const DecodeParams& P, const Task& t) {
+// Chunk of an attention task at step st of the launch: keys [j0, j1) of Lk = pos + 1; pos0 is
+// the sequence's position at the launch's first step (rows at or past it are written during
+// this launch).
+__device__ __forceinline__ AttnGeom attn_geom(const DecodeParams& P, const Task& t, int st) {
   AttnGeom a;
   a.b = (int)t.row0 / P.nkv;
   a.g = (int)t.row0 % P.nkv;
   a.c = t.aux;
-  a.Lk = P.pos[a.b] + 1;
+  a.pos0 = P.pos[a.b];
+  a.Lk = P.pos[a.b] + st + 1;
   if (a.b >= P.nb) {  // sequence not in the active batch: its tasks only count their arrival
     a.nch_eff = 0;
     a.j0 = a.j1 = 0;
@@ -531,22 +536,23 @@ __device__ __forceinline__ void attn_block_g(const float (&qv)[4][D / 32], const
   else attn_block<D, 4>(qv, kw, vw, valid, G, m, l, acc, lane);
 }
 
-// Number of ring stages of an attention task: its old positions [j0, min(j1, pos)).
+// Number of ring stages of an attention task: its rows written before the launch,
+// [j0, min(j1, pos0)) (the producer runs ahead and must not read rows of this launch).
 template <int D>
 __device__ __forceinline__ int attn_stage_span(const AttnGeom& a, int* jend) {
-  *jend = (a.c < a.nch_eff) ? min(a.j1, a.Lk - 1) : a.j0;
+  *jend = (a.c < a.nch_eff) ? max(a.j0, min(a.j1, a.pos0)) : a.j0;
   return *jend > a.j0 ? (*jend - a.j0 + kv_stage_keys<D>() - 1) / kv_stage_keys<D>() : 0;
 }
 
 template <int D, bool TC>
 __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, Pipe& pp, const uint8_t* ring,
-                                               const Task& t, uint32_t task_id, uint32_t& stall_ns) {
+                                               const Task& t, uint32_t task_id, uint32_t& stall_ns, int st) {
   constexpr int DL = D / 32;
   constexpr int W = D / 64;
   constexpr int KPS = kv_stage_keys<D>();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = P.nq / P.nkv;
-  const AttnGeom a = attn_geom(P, t);
+  const AttnGeom a = attn_geom(P, t, st);
   const int g = a.g, b = a.b, c = a.c, nch_eff = a.nch_eff, pos = a.Lk - 1;
   const uint16_t* kc = attn_cache<D>(P, t, a, 0);
   const uint16_t* vc = attn_cache<D>(P, t, a, 1);
@@ -571,8 +577,11 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
     // the key and value at the current position were written in this step: the warp that
     // owns its slot fetches them together with q (one L2 round trip).  It takes the free slot
     // after the old keys of the last ring stage, or (no free slot) one extra block of warp 0.
+    // (In a multi-step launch, the rows its earlier steps wrote are "fresh" too: they are
+    // read from global memory in blocks after the ring stages.)
+    const int jf0 = max(a.j0, a.pos0), nf = max(0, a.j1 - jf0);  // rows of this launch
     const int cur_rel = pos - a.j0;
-    const bool has_pos = pos >= a.j0 && pos < a.j1;
+    const bool has_pos = pos >= a.j0 && pos < a.j1 && nf == 1;  // the current key is the only fresh row
     const bool cur_in_stage = has_pos && (cur_rel % KPS) != 0;
     const int cur_warp = cur_in_stage ? (cur_rel % KPS) % kAttnWarps : 0;
     const bool has_cur = has_pos && warp == cur_warp;
@@ -632,6 +641,20 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       }
       attn_block_g<D>(qv, kw, vw, 1u, G, m, l, acc, lane);
     }
+    if (nf > 1) {  // several rows written during this launch: blocks of kAttnBlock keys per warp
+      for (int fb = 0; fb < nf; fb += kAttnBlock * kAttnWarps) {
+        uint32_t valid = 0;
+#pragma unroll
+        for (int u = 0; u < kAttnBlock; ++u) {
+          const int idx = fb + warp + u * kAttnWarps;
+          if (idx < nf) {
+            valid |= 1u << u;
+            attn_load_key<D>(kc, vc, jf0 + idx, lane, kw[u], vw[u]);
+          }
+        }
+        if (valid) attn_block_g<D>(qv, kw, vw, valid, G, m, l, acc, lane);
+      }
+    }
     // cross-warp merge of this chunk
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
@@ -676,7 +699,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
   if (tid == 0) {
     uint32_t* cnt = P.acnt + ((size_t)t.layer * P.B + b) * P.nkv + g;
     const uint32_t old = atom_acq_rel_gpu_add(cnt, 1u);
-    S.flag = (old + 1u == P.epoch * (uint32_t)P.nch) ? 1u : 0u;
+    S.flag = (old + 1u == (P.epoch + (uint32_t)st) * (uint32_t)P.nch) ? 1u : 0u;
   }
   worker_bar();
   if (S.flag && nch_eff > 1) {
@@ -757,8 +780,15 @@ __device__ __forceinline__ void block_argmax(DSmem& S, float& v, int& idx) {
     for (int w = 1; w < kWorkerWarps; ++w) argmax_merge(v, idx, S.lmv[w], S.lmi[w]);
 }
 
+// The token pick of step st: greedy tokens to next_tokens[st][b]; then the event the next
+// step's embedding waits for.
+__device__ __forceinline__ void announce_tokens(const DecodeParams& P, DSmem& S) {
+  worker_bar();
+  if (threadIdx.x == 0) red_release_gpu_add(&P.ev[P.ev_tok], 1u);
+}
+
 template <int BM>
-__device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, const Task& t, int K) {
+__device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, const Task& t, int K, int st) {
   const int tid = threadIdx.x;
   for (int b = 0; b < P.nb; ++b) {
     const float r = norm_factor(S, K, P.eps, b);
@@ -778,19 +808,22 @@ __device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, cons
   }
   if (tid == 0) {
     const uint32_t old = atom_acq_rel_gpu_add(&P.ev[P.ev_lm], 1u);
-    S.flag = (old + 1u == P.epoch * (uint32_t)P.n_lm) ? 1u : 0u;
+    S.flag = (old + 1u == (P.epoch + (uint32_t)st) * (uint32_t)P.n_lm) ? 1u : 0u;
   }
   worker_bar();
-  if (S.flag && P.next_tokens) {
-    for (int b = 0; b < P.nb; ++b) {
-      float v = -INFINITY;
-      int idx = 0x7fffffff;
-      for (int i = tid; i < P.n_lm; i += kWorkerThreads)
-        argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
-      block_argmax(S, v, idx);
-      if (tid == 0) P.next_tokens[b] = idx;
-      worker_bar();
+  if (S.flag) {
+    if (P.next_tokens) {
+      for (int b = 0; b < P.nb; ++b) {
+        float v = -INFINITY;
+        int idx = 0x7fffffff;
+        for (int i = tid; i < P.n_lm; i += kWorkerThreads)
+          argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
+        block_argmax(S, v, idx);
+        if (tid == 0) P.next_tokens[(size_t)st * P.B + b] = idx;
+        worker_bar();
+      }
     }
+    announce_tokens(P, S);
   }
 }
 
@@ -962,11 +995,13 @@ __device__ __forceinline__ void tc_issuer(const DecodeParams& P, DSmem& S, const
   Pipe pp{0, 0, kTcStages};
   uint32_t gseg = 0, gtask = 0;
   const uint32_t b_base0 = smem_u32(bop);
+  bool ok = true;
+  for (int st = 0; st < P.n_steps && ok; ++st)
   for (uint32_t i = qb; i < qe; ++i) {
     const Task t = P.tasks[i];
     if (t.kind == TK_ATTN) {
       int jend;
-      const int nst = attn_stage_span<HD>(attn_geom(P, t), &jend);
+      const int nst = attn_stage_span<HD>(attn_geom(P, t, st), &jend);
       for (int st = 0; st < nst; ++st) pp.advance();
       continue;
     }
@@ -974,12 +1009,12 @@ __device__ __forceinline__ void tc_issuer(const DecodeParams& P, DSmem& S, const
     const uint32_t ab = gtask & 1u, av = gtask >> 1;
     if (!wait_bar(&S.acc_free[ab], (av & 1u) ^ 1u, P.timeout_ns, &S)) {
       if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, i);
+      ok = false;
       break;
     }
     tc_fence_after();
     const uint32_t d_tmem = tmem + ab * kTcN;
     const int nu = (int)t.nrows, nseg = (nu + kTcSegUnits - 1) / kTcSegUnits;
-    bool ok = true;
     for (int sg = 0; sg < nseg && ok; ++sg) {
       const uint32_t buf = gseg & 1u, use = gseg >> 1;
       if (!wait_bar(&S.bop_full[buf], use & 1u, P.timeout_ns, &S)) {
@@ -1027,7 +1062,7 @@ __device__ __forceinline__ void tc_issuer(const DecodeParams& P, DSmem& S, const
 // read it back, then the partial record / tile epilogue.  False (for every worker alike) if a
 // wait ran out.
 __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const Task& t, const LayerOff& lo,
-                                          uint32_t tmem, uint32_t gtask, int tsb, uint32_t task_id) {
+                                          uint32_t tmem, uint32_t gtask, int tsb, uint32_t task_id, int st) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t lay = (size_t)t.layer * P.B;
   const TcOp op = tc_op(P, t, lo);
@@ -1066,7 +1101,7 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
   if (!solo) {
     if (tid == 0) {
       const uint32_t old = atom_acq_rel_gpu_add(&P.tcnt[t.pad1], 1u);
-      S.flag = (old + 1u == P.epoch * (uint32_t)t.pad0) ? 1u : 0u;
+      S.flag = (old + 1u == (P.epoch + (uint32_t)st) * (uint32_t)t.pad0) ? 1u : 0u;
     }
     worker_bar();
     if (!S.flag) return true;
@@ -1130,22 +1165,25 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
     worker_bar();
     if (tid == 0) {
       const uint32_t old = atom_acq_rel_gpu_add(&P.ev[P.ev_lm], 1u);
-      S.flag = (old + 1u == P.epoch * (uint32_t)P.n_lm) ? 1u : 0u;
+      S.flag = (old + 1u == (P.epoch + (uint32_t)st) * (uint32_t)P.n_lm) ? 1u : 0u;
     }
     worker_bar();
-    if (S.flag && P.next_tokens) {
+    if (S.flag) {
+      if (P.next_tokens) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int b = warp + h * kWorkerWarps;
-        if (b < P.nb) {
-          float v = -INFINITY;
-          int idx = 0x7fffffff;
-          for (int i = lane; i < P.n_lm; i += 32)
-            argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
-          warp_argmax(v, idx);
-          if (lane == 0) P.next_tokens[b] = idx;
+        for (int h = 0; h < 2; ++h) {
+          const int b = warp + h * kWorkerWarps;
+          if (b < P.nb) {
+            float v = -INFINITY;
+            int idx = 0x7fffffff;
+            for (int i = lane; i < P.n_lm; i += 32)
+              argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
+            warp_argmax(v, idx);
+            if (lane == 0) P.next_tokens[(size_t)st * P.B + b] = idx;
+          }
         }
       }
+      announce_tokens(P, S);
     }
     return true;
   }
@@ -1155,7 +1193,7 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
     const float r = gain ? 1.0f / sqrtf(ssum[b] / (float)K + P.eps) : 1.f;
     const float v = S.tile[e] * r;
     switch (t.kind) {
-      case TK_QKV: qkv_out(P, t.layer, R, b, v, S.tile[e ^ kTcBatch] * r); break;  // partner row R ^ 1
+      case TK_QKV: qkv_out(P, t.layer, R, b, v, S.tile[e ^ kTcBatch] * r, st); break;  // partner row R ^ 1
       case TK_OPROJ: {
         const size_t at = (lay + b) * P.H + R;
         P.x_mid[at] = __ldcg(P.x_in + at) + v;
@@ -1261,11 +1299,18 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
     Pipe pp{0, 0, NST};
     int issued = 0;
     bool ok = true;
+    for (int st = 0; st < P.n_steps && ok; ++st) {
+    if (st > 0) {  // the lookahead restarts with the step's queue
+      la_task = qb;
+      la_row = 0;
+      la_lead = 0;
+      la_t = P.tasks[qb < qe ? qb : 0];
+    }
     for (uint32_t i = qb; i < qe && ok; ++i) {
       const Task t = P.tasks[i];
       if (t.kind == TK_ATTN) {
         // old K/V rows of the chunk, kv_stage_keys<HD>() per stage: K rows, then V rows
-        const AttnGeom a = attn_geom(P, t);
+        const AttnGeom a = attn_geom(P, t, st);
         int jend;
         const int nst = attn_stage_span<HD>(a, &jend);
         const uint16_t* kc = attn_cache<HD>(P, t, a, 0);
@@ -1335,6 +1380,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
         P.trace[(size_t)i * kTraceWords + 5] = first;
       }
     }
+    }
     // leave no copy in flight: wait (bounded) for the last issued stages to land
     for (int k = 1; k <= (issued < NST ? issued : NST); ++k) {
       int s = pp.stage - k;
@@ -1351,11 +1397,16 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
   if (warp == kSchedWarp) {
     // ------------------------------- scheduler ------------------------------
     if (lane != 0) return;
+    const uint32_t nq = qe - qb;
+    for (int st = 0; st < P.n_steps; ++st)
     for (uint32_t i = qb; i < qe; ++i) {
       const Task t = P.tasks[i];
-      for (int w = 0; w < t.n_wait; ++w) {
-        const uint32_t e = t.wait[w];
-        const uint32_t target = P.epoch * P.ev_count[e];
+      // a later step's embedding also waits for the previous step's token pick
+      const int n_wait = t.n_wait + ((t.kind == TK_EMBED && st > 0) ? 1 : 0);
+      for (int w = 0; w < n_wait; ++w) {
+        const bool tok = w == t.n_wait;
+        const uint32_t e = tok ? P.ev_tok : t.wait[w];
+        const uint32_t target = tok ? P.epoch + (uint32_t)st - 1u : (P.epoch + (uint32_t)st) * P.ev_count[e];
         uint64_t t0 = 0;
         for (uint32_t n = 1;; ++n) {
           if ((int32_t)(ld_acquire_gpu(&P.ev[e]) - target) >= 0) break;
@@ -1373,7 +1424,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
           }
         }
       }
-      st_release_cta_shared(&S.ready, i - qb + 1u);
+      st_release_cta_shared(&S.ready, (uint32_t)st * nq + (i - qb) + 1u);
     }
     return;
   }
@@ -1389,17 +1440,21 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
   // iteration instead, which keeps 10 registers free across the GEMV
   constexpr bool kHoist = (BM == 1);
   Task t_next = P.tasks[qb < qe ? qb : 0];
-  for (uint32_t i = qb; i < qe; ++i) {
+  // the queue once per step of the launch: k counts released tasks over all steps
+  const uint32_t nq = qe - qb, nk = nq * (uint32_t)P.n_steps;
+  for (uint32_t k = 0; k < nk; ++k) {
+    const int st = (int)(k / nq);
+    const uint32_t i = qb + k % nq;
     const Task t = kHoist ? t_next : P.tasks[i];
     const LayerOff lo = P.loff[t.layer < P.L ? t.layer : 0];
-    if (kHoist && i + 1 < qe) t_next = P.tasks[i + 1];
+    if (kHoist && k + 1 < nk) t_next = P.tasks[qb + (k + 1) % nq];
     const uint64_t t_wait = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     uint32_t stall = 0;
     // wait for the scheduler to release task i (bounded, abort-aware, then uniform decision)
     {
       uint64_t t0 = 0;
       for (uint32_t n = 1;; ++n) {
-        if (ld_acquire_cta_shared(&S.ready) > i - qb) break;
+        if (ld_acquire_cta_shared(&S.ready) > k) break;
         if ((n & 63u) == 0) {
           if (S.abort) {
             S.cabort = 1u;
@@ -1431,7 +1486,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       if (ok && i + 1 < qe && tn.kind == t.kind && tn.layer == t.layer) {
         uint64_t t0 = 0;
         for (uint32_t n = 1;; ++n) {  // its release (immediate: same events as this task)
-          if (ld_acquire_cta_shared(&S.ready) > i + 1 - qb) break;
+          if (ld_acquire_cta_shared(&S.ready) > k + 1) break;
           if ((n & 63u) == 0) {
             if (S.abort) {
               ok = false;
@@ -1453,7 +1508,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       }
       if (!ok) S.cabort = 1u;
       for (int u = 0; u < nu; ++u) pp.advance();  // the task's weight blocks go to the issuer
-      if (!tc_finish(P, S, t, lo, tmem, gtask, tsb, i)) goto out;
+      if (!tc_finish(P, S, t, lo, tmem, gtask, tsb, i, st)) goto out;
       ++gtask;
       if (t.kind == TK_LMHEAD) notify = false;
     } else if (is_gemv(t.kind)) {
@@ -1504,7 +1559,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       const bool mine = er < (int)t.nrows && eb < P.nb;
       const float r = gain ? norm_factor(S, K, P.eps, eb) : 1.f;
       switch (t.kind) {
-        case TK_QKV: epi_qkv<BMC>(P, S, t, r); break;
+        case TK_QKV: epi_qkv<BMC>(P, S, t, r, st); break;
         case TK_OPROJ:
           if (mine) {
             const size_t at = (lay + eb) * P.H + t.row0 + er;
@@ -1530,12 +1585,13 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
           break;
         default:
           notify = false;
-          epi_lmhead<BMC>(P, S, t, K);
+          epi_lmhead<BMC>(P, S, t, K, st);
           break;
       }
     } else if (t.kind == TK_EMBED) {
       for (int b = 0; b < P.nb; ++b) {
-        int tok = __ldcg(P.tokens + b);
+        // step 0: the caller's tokens; later steps: the previous step's greedy pick
+        int tok = (st == 0) ? __ldcg(P.tokens + b) : __ldcg(P.next_tokens + (size_t)(st - 1) * P.B + b);
         if (tok < 0 || tok >= P.V) {  // never read outside the table: record and use row 0
           if (tid == 0 && t.row0 == 0) atomicCAS(&P.err[ERR_CODE], 0u, (uint32_t)DEV_ERR_BAD_TOKEN);
           tok = 0;
@@ -1546,7 +1602,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       }
     } else if (t.kind == TK_ATTN) {
       notify = false;  // the last chunk to arrive notifies
-      if (!attention_task<HD, TC>(P, S, pp, ring, t, i, stall)) goto out;
+      if (!attention_task<HD, TC>(P, S, pp, ring, t, i, stall, st)) goto out;
     }
     if (P.trace && tid == 0) {
       uint64_t* rec = P.trace + (size_t)i * kTraceWords;

@@ -56,7 +56,7 @@ struct mk_ctx {
   int n_tile_ids = 0;         // tiles of one layer's projections plus the LM head's
   size_t rec_cap = 0, n_recs = 0;  // partial records (workspace capacity, in use)
   // events
-  int n_events = 0, ev_lm = 0;
+  int n_events = 0, ev_lm = 0, ev_tok = 0;
   Graph g;
   std::vector<uint32_t> qbegin;
   // arena layout
@@ -243,6 +243,7 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
       for (const VTask& t : T)
         if (t.kind == TK_LMHEAD) produced[c->ev_lm]++;
     }
+    if (c->ev_tok < nE) produced[c->ev_tok] = 1;  // raised once per step by the token pick
   }
   for (int e = 0; e < nE; ++e)
     if (produced[e] != cnt[e]) {
@@ -472,8 +473,9 @@ int build_graph(mk_ctx* c) {
   const mk_config& f = c->cfg;
   const int L = f.n_layers, nkv = f.n_kv_heads, D = f.head_dim, n = c->n_sms;
   const int B = f.max_batch;
-  c->n_events = 1 + L * (nkv + 4) + 1;
-  c->ev_lm = c->n_events - 1;
+  c->n_events = 1 + L * (nkv + 4) + 2;
+  c->ev_lm = c->n_events - 2;
+  c->ev_tok = c->n_events - 1;  // tokens picked: a later step of a multi-step launch waits on it
   std::vector<uint32_t> evc(c->n_events, 0);
   std::vector<std::vector<Task>> q(n);
   const int rpg = (c->G + 2) * D;
@@ -608,6 +610,7 @@ int build_graph(mk_ctx* c) {
       }
     c->n_lm = c->tc ? c->tc_tiles[TK_LMHEAD] : idx;
     evc[c->ev_lm] = (uint32_t)c->n_lm;
+    evc[c->ev_tok] = 1u;
   }
   c->g.tasks.clear();
   c->qbegin.assign(n + 1, 0);
@@ -1078,17 +1081,21 @@ int mk_get_positions(const mk_ctx* c, int32_t* host_pos, int capacity) {
   return c->B;
 }
 
-int mk_decode_step(mk_ctx* c, const int32_t* tokens, void* kv_cache, float* logits, int32_t* next_tokens,
-                   void* stream) {
+namespace {
+// One launch of the persistent kernel running n_steps greedy decode steps.
+int decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache, float* logits,
+                  int32_t* next_tokens, void* stream) {
   if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
   if (!c->loaded) return fail(c, MK_ERR_STATE, "weights not loaded");
   if (c->B < 1) return fail(c, MK_ERR_STATE, "no active batch (call mk_prefill or mk_set_positions)");
   if (!tokens || !kv_cache || !logits) return fail(c, MK_ERR_INVALID_ARG, "NULL tokens, cache or logits");
+  if (n_steps < 1 || n_steps > MK_MAX_STEPS) return fail(c, MK_ERR_INVALID_ARG, "n_steps out of range");
+  if (n_steps > 1 && !next_tokens) return fail(c, MK_ERR_INVALID_ARG, "a multi-step launch needs tokens_out");
   if (c->variant < 0 || c->B > c->bm)
     return fail(c, MK_ERR_UNSUPPORTED, "no decode kernel instantiation for this shape / batch");
   const mk_config& f = c->cfg;
   for (int b = 0; b < c->B; ++b)
-    if (c->pos[b] >= f.max_seq) return fail(c, MK_ERR_INVALID_ARG, "sequence is full (max_seq reached)");
+    if (c->pos[b] + n_steps > f.max_seq) return fail(c, MK_ERR_INVALID_ARG, "sequence is full (max_seq reached)");
   DecodeParams P;
   std::memset(&P, 0, sizeof(P));
   uint8_t* W = c->ws;
@@ -1138,6 +1145,8 @@ int mk_decode_step(mk_ctx* c, const int32_t* tokens, void* kv_cache, float* logi
   P.tcnt = reinterpret_cast<uint32_t*>(W + c->ws_tcnt);
   P.epoch = c->epoch + 1;
   P.ev_lm = (uint32_t)c->ev_lm;
+  P.ev_tok = (uint32_t)c->ev_tok;
+  P.n_steps = n_steps;
   P.drop_event = c->drop_event;
   P.timeout_ns = c->timeout_ns;
   P.trace = c->trace;
@@ -1145,9 +1154,20 @@ int mk_decode_step(mk_ctx* c, const int32_t* tokens, void* kv_cache, float* logi
   std::string err;
   int rc = launch_decode(c->variant, P, c->n_sms, reinterpret_cast<cudaStream_t>(stream), &err);
   if (rc) return fail(c, rc, err);
-  c->epoch += 1;
-  for (int b = 0; b < c->B; ++b) c->pos[b] += 1;
+  c->epoch += (uint32_t)n_steps;
+  for (int b = 0; b < c->B; ++b) c->pos[b] += n_steps;
   return MK_OK;
+}
+}  // namespace
+
+int mk_decode_step(mk_ctx* c, const int32_t* tokens, void* kv_cache, float* logits, int32_t* next_tokens,
+                   void* stream) {
+  return decode_launch(c, tokens, 1, kv_cache, logits, next_tokens, stream);
+}
+
+int mk_decode_steps(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache, float* logits,
+                    int32_t* tokens_out, void* stream) {
+  return decode_launch(c, tokens, n_steps, kv_cache, logits, tokens_out, stream);
 }
 
 int mk_sync_status(mk_ctx* c, void* stream) {

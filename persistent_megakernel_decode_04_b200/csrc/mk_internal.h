@@ -113,7 +113,7 @@ struct DecodeParams {
   int32_t* lm_idx;            // [n_lm][B]
   const int32_t* tokens;      // [B]
   float* logits;              // [B][V]
-  int32_t* next_tokens;       // [B] or null
+  int32_t* next_tokens;       // [n_steps][B] greedy tokens of every step (null: not kept, 1 step only)
   int pos[MK_MAX_BATCH];
   int B, H, nq, nkv, D, F, V, L, nch, max_seq, max_batch, n_lm;
   float eps, attn_scale;
@@ -127,6 +127,8 @@ struct DecodeParams {
   int kdc, ndc;               // down-projection K chunk and chunk count
   float* tpart;               // tensor-core partial records [n_records][kTcRecFloats]
   uint32_t* tcnt;             // tensor-core tile arrival counters
+  int n_steps;                // greedy decode steps in this launch (step s: epoch + s, pos + s)
+  uint32_t ev_tok;            // event: the step's tokens are picked (the next step's embedding waits)
 };
 constexpr uint64_t kStallPrefetchNs = 1000;    // producer blocked this long: prefetch ahead into L2
 constexpr uint64_t kStallPrefetchGapNs = 100;   // then one more stage per this interval
