@@ -574,22 +574,24 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       }
     }
     uint32_t kw[kAttnBlock][W], vw[kAttnBlock][W];
-    // the key and value at the current position were written in this step: the warp that
-    // owns its slot fetches them together with q (one L2 round trip).  It takes the free slot
-    // after the old keys of the last ring stage, or (no free slot) one extra block of warp 0.
-    // (In a multi-step launch, the rows its earlier steps wrote are "fresh" too: they are
-    // read from global memory in blocks after the ring stages.)
-    const int jf0 = max(a.j0, a.pos0), nf = max(0, a.j1 - jf0);  // rows of this launch
-    const int cur_rel = pos - a.j0;
-    const bool has_pos = pos >= a.j0 && pos < a.j1 && nf == 1;  // the current key is the only fresh row
-    const bool cur_in_stage = has_pos && (cur_rel % KPS) != 0;
-    const int cur_warp = cur_in_stage ? (cur_rel % KPS) % kAttnWarps : 0;
-    const bool has_cur = has_pos && warp == cur_warp;
-    uint32_t kcur[W], vcur[W];
-    if (has_cur) attn_load_key<D>(kc, vc, pos, lane, kcur, vcur);
-    // old positions from the ring, kv_stage_keys per stage (K rows at 0, V rows at KPS * D)
+    // Rows of this chunk written during the launch ("fresh": the current position and, in a
+    // multi-step launch, those of its earlier steps) cannot come through the ring.  They take
+    // the free slots after the old rows of the last ring stage; each warp fetches up to
+    // kFreshPre of its fresh slots together with q (one L2 round trip) and any others when the
+    // stage is processed.  Fresh rows that do not fit (no stage, or no free slot) follow in
+    // blocks of kAttnBlock keys per warp read from memory.
+    constexpr int kFreshPre = 2;
+    const int jf0 = max(a.j0, a.pos0), nf = max(0, a.j1 - jf0);
     int jend;
     const int nst = attn_stage_span<D>(a, &jend);
+    const int nl = (nst > 0) ? (jend - a.j0) - (nst - 1) * KPS : 0;  // old rows in the last stage
+    const int n_in = (nst > 0) ? min(nf, KPS - nl) : 0;              // fresh rows in its free slots
+    const int f_first = ((warp - nl) % kAttnWarps + kAttnWarps) % kAttnWarps;  // this warp's first fresh slot
+    uint32_t kpre[kFreshPre][W], vpre[kFreshPre][W];
+#pragma unroll
+    for (int j = 0; j < kFreshPre; ++j)
+      if (f_first + kAttnWarps * j < n_in) attn_load_key<D>(kc, vc, jf0 + f_first + kAttnWarps * j, lane, kpre[j], vpre[j]);
+    // old positions from the ring, kv_stage_keys per stage (K rows at 0, V rows at KPS * D)
     for (int st = 0; st < nst; ++st) {
       const int jj = a.j0 + st * KPS, nk = min(KPS, jend - jj);
       const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
@@ -600,20 +602,14 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
       const uint8_t* kst = ring + (size_t)pp.stage * kSlotBytes;
       const uint8_t* vst = kst + KPS * D * 2;
+      const bool last = st == nst - 1;
 #pragma unroll
       for (int kb = 0; kb < KPS / (kAttnBlock * kAttnWarps); ++kb) {
         uint32_t valid = 0;
 #pragma unroll
         for (int u = 0; u < kAttnBlock; ++u) {
           const int idx = kb * kAttnBlock * kAttnWarps + warp + u * kAttnWarps;
-          if (cur_in_stage && st == nst - 1 && idx == nk) {  // the current key's slot
-            valid |= 1u << u;
-#pragma unroll
-            for (int w = 0; w < W; ++w) {
-              kw[u][w] = kcur[w];
-              vw[u][w] = vcur[w];
-            }
-          } else if (idx < nk) {
+          if (idx < nk) {
             valid |= 1u << u;
             if (D == 128) {
               const uint2 kk = *reinterpret_cast<const uint2*>(kst + idx * D * 2 + lane * 8);
@@ -624,6 +620,18 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
               kw[u][0] = *reinterpret_cast<const uint32_t*>(kst + idx * D * 2 + lane * 4);
               vw[u][0] = *reinterpret_cast<const uint32_t*>(vst + idx * D * 2 + lane * 4);
             }
+          } else if (last && idx - nk < n_in) {  // a fresh row in a free slot
+            const int f = idx - nk, j = (f - f_first) / kAttnWarps;
+            valid |= 1u << u;
+            if (j < kFreshPre) {
+#pragma unroll
+              for (int w = 0; w < W; ++w) {
+                kw[u][w] = kpre[j < kFreshPre ? j : 0][w];
+                vw[u][w] = vpre[j < kFreshPre ? j : 0][w];
+              }
+            } else {
+              attn_load_key<D>(kc, vc, jf0 + f, lane, kw[u], vw[u]);
+            }
           }
         }
         if (valid) attn_block_g<D>(qv, kw, vw, valid, G, m, l, acc, lane);
@@ -633,27 +641,18 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
       pp.advance();
     }
-    if (has_cur && !cur_in_stage) {
+    // fresh rows that found no free slot: blocks read from memory
+    for (int fb = n_in; fb < nf; fb += kAttnBlock * kAttnWarps) {
+      uint32_t valid = 0;
 #pragma unroll
-      for (int w = 0; w < W; ++w) {
-        kw[0][w] = kcur[w];
-        vw[0][w] = vcur[w];
-      }
-      attn_block_g<D>(qv, kw, vw, 1u, G, m, l, acc, lane);
-    }
-    if (nf > 1) {  // several rows written during this launch: blocks of kAttnBlock keys per warp
-      for (int fb = 0; fb < nf; fb += kAttnBlock * kAttnWarps) {
-        uint32_t valid = 0;
-#pragma unroll
-        for (int u = 0; u < kAttnBlock; ++u) {
-          const int idx = fb + warp + u * kAttnWarps;
-          if (idx < nf) {
-            valid |= 1u << u;
-            attn_load_key<D>(kc, vc, jf0 + idx, lane, kw[u], vw[u]);
-          }
+      for (int u = 0; u < kAttnBlock; ++u) {
+        const int idx = fb + warp + u * kAttnWarps;
+        if (idx < nf) {
+          valid |= 1u << u;
+          attn_load_key<D>(kc, vc, jf0 + idx, lane, kw[u], vw[u]);
         }
-        if (valid) attn_block_g<D>(qv, kw, vw, valid, G, m, l, acc, lane);
       }
+      if (valid) attn_block_g<D>(qv, kw, vw, valid, G, m, l, acc, lane);
     }
     // cross-warp merge of this chunk
 #pragma unroll
