@@ -86,6 +86,16 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(x: float, dev, world: int) -> float:
+    """The largest of every rank's x (the slowest replica's time); x itself on one rank."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -411,11 +421,9 @@ def run_mk(args, rank, world, local):
         raise SystemExit(f"decode reported status {status}: {mk.mk_last_error(m.ctx)}")
     elapsed_ms = start.elapsed_time(stop)
     step_ms = np.array([a.elapsed_time(b) for a, b in ev])
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    max_ms = max_over_ranks(elapsed_ms, dev, world)
     if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
         dist.barrier()
-    max_ms = float(t.item())
 
     # end to end through the C ABI with host buffers: token in from pinned host memory,
     # logits and next token back to pinned host memory, every step
@@ -441,11 +449,7 @@ def run_mk(args, rank, world, local):
         host_tok.copy_(host_next)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_max = float(te.item())
+    e2e_max = max_over_ranks(e0.elapsed_time(e1), dev, world)
     if m.sync_status() != mk.MK_OK:
         raise SystemExit("decode reported an error in the end-to-end loop")
 
