@@ -160,6 +160,13 @@ int mk_debug_drop_notify(mk_ctx* ctx, int event_id, int on);
  * does not fit the workspace reserve (the old graph then stays). */
 int mk_set_sm_weights(mk_ctx* ctx, const float* weights, int n, void* stream);
 
+/* The same for one projection only: op_kind 2 (QKV), 4 (O), 5 (gate/up), 6 (down) or 7 (LM
+ * head) takes its rows by `weights`, the other projections keep theirs (an SM can be slow in
+ * one phase only, e.g. where it also runs attention).  mk_set_sm_weights resets every
+ * projection to its weights.  Errors as mk_set_sm_weights; MK_ERR_INVALID_ARG for another
+ * op_kind. */
+int mk_set_op_sm_weights(mk_ctx* ctx, int op_kind, const float* weights, int n, void* stream);
+
 /* Weight prefetch depth: besides the shared-memory ring (6 stages of 32 KB per SM), an SM's
  * producer that has been blocked on a full ring for over a microsecond (its workers wait for a
  * dependency, e.g. during attention) prefetches up to `stages` further weight stages of its

@@ -82,6 +82,7 @@ _SIGS = {
     "mk_debug_drop_notify": ([_vp, _i32, _i32], _i32),
     "mk_set_l2_prefetch": ([_vp, _i32], _i32),
     "mk_set_sm_weights": ([_vp, _vp, _i32, _vp], _i32),
+    "mk_set_op_sm_weights": ([_vp, _i32, _vp, _i32, _vp], _i32),
     "mk_set_trace": ([_vp, _vp], _i32),
     "mk_get_graph_info": ([_vp, ctypes.POINTER(mk_graph_info)], _i32),
     "mk_export_taskgraph": ([_vp, _vp, _i32, _vp, _i32], _i32),
@@ -222,6 +223,12 @@ def mk_set_sm_weights(ctx, weights, stream=None):
     _check(_lib.mk_set_sm_weights(ctx, w.ctypes.data, w.size, _stream(stream)), ctx)
 
 
+def mk_set_op_sm_weights(ctx, op_kind: int, weights, stream=None):
+    import numpy as np
+    w = np.ascontiguousarray(weights, dtype=np.float32)
+    _check(_lib.mk_set_op_sm_weights(ctx, int(op_kind), w.ctypes.data, w.size, _stream(stream)), ctx)
+
+
 def mk_set_l2_prefetch(ctx, stages: int):
     _check(_lib.mk_set_l2_prefetch(ctx, int(stages)), ctx)
 
@@ -358,32 +365,37 @@ class Megakernel:
         return self.logits[:B], out[:, :B]
 
     def calibrate(self, tokens, steps: int = 2, rounds: int = 3):
-        """Measure each SM's busy time on the projection tasks over `steps` traced decode steps
-        (decoding `tokens`, which advances the positions) and re-partition the rows so that
-        every SM finishes together; `rounds` measure/re-partition passes.  Returns the weights."""
+        """Measure each SM's busy time on each projection (QKV, O, gate/up, down, LM head) over
+        `steps` traced decode steps (decoding `tokens`, which advances the positions) and
+        re-partition that projection's rows so that every SM finishes it together; `rounds`
+        measure/re-partition passes.  Returns the weights, one row per projection kind."""
         import numpy as np
         import torch
         info = self.info()
         n = info["n_sms"]
-        w = np.ones(n)
+        kinds = (2, 4, 5, 6, 7)
+        w = {k: np.ones(n) for k in kinds}
         trace = torch.zeros(info["task_capacity"] * 6, dtype=torch.int64, device=tokens.device)
         for _ in range(rounds):
             tasks, _ = mk_export_taskgraph(self.ctx)
             mk_set_trace(self.ctx, trace)
-            busy = np.zeros(n)
+            busy = {k: np.zeros(n) for k in kinds}
             for _ in range(steps):
                 self.decode(tokens)
                 self.sync_status()
                 T = trace[: tasks.shape[0] * 6].view(-1, 6).cpu().numpy()
-                gemv = np.isin(tasks[:, 0], (2, 4, 5, 6, 7))
-                np.add.at(busy, tasks[gemv, 2], (T[gemv, 2] - T[gemv, 1]).astype(np.float64))
+                for k in kinds:
+                    sel = tasks[:, 0] == k
+                    np.add.at(busy[k], tasks[sel, 2], (T[sel, 2] - T[sel, 1]).astype(np.float64))
             mk_set_trace(self.ctx, None)
-            if busy.min() <= 0:
-                break
-            w = w * busy.mean() / busy  # slower SMs (more busy time) get fewer rows
-            w = w / w.mean()
-            mk_set_sm_weights(self.ctx, w, self.stream)
-        return w
+            for k in kinds:
+                b = busy[k]
+                if b.min() <= 0:  # an SM without tasks of this kind: keep its weights
+                    continue
+                w[k] = w[k] * b.mean() / b  # slower SMs (more busy time) get fewer rows
+                w[k] = w[k] / w[k].mean()
+                mk_set_op_sm_weights(self.ctx, k, w[k], self.stream)
+        return np.stack([w[k] for k in kinds])
 
     def set_positions(self, positions):
         mk_set_positions(self.ctx, positions)

@@ -82,6 +82,7 @@ struct mk_ctx {
   uint64_t* trace = nullptr;
   int l2_ahead = 8;  // L2 lookahead stages while the ring is full (mk_set_l2_prefetch)
   std::vector<double> sm_weights;  // relative streaming speed per SM (partition weights)
+  std::vector<double> op_weights[8];  // per projection kind; empty = sm_weights
   size_t task_cap = 0, lm_cap = 0; // workspace capacity for re-partitioned graphs
   std::string err;
 };
@@ -500,14 +501,17 @@ int build_graph(mk_ctx* c) {
     std::vector<int> nsplit, rec0;       // tensor-core: per tile
   };
   size_t rec_next = 0;
+  auto op_w = [&](int kind) -> const std::vector<double>& {
+    return c->op_weights[kind].empty() ? c->sm_weights : c->op_weights[kind];
+  };
   auto plan = [&](int kind, int rows, int gran) {
     Plan pl;
     if (!c->tc) {
-      pl.parts = partition_rows(rows, gran, c->sm_weights, c->task_rows);
+      pl.parts = partition_rows(rows, gran, op_w(kind), c->task_rows);
       return pl;
     }
     const int nk = c->tc_nk[kind], tiles = c->tc_tiles[kind];
-    pl.parts = partition_blocks(tiles, nk, c->sm_weights);
+    pl.parts = partition_blocks(tiles, nk, op_w(kind));
     pl.nsplit.assign(tiles, 0);
     pl.slot.resize(n);
     for (int s = 0; s < n; ++s)
@@ -1207,8 +1211,12 @@ int mk_debug_drop_notify(mk_ctx* c, int event_id, int on) {
   return MK_OK;
 }
 
-int mk_set_sm_weights(mk_ctx* c, const float* weights, int n, void* stream) {
+namespace {
+// Re-partition with new per-SM weights for one projection kind (op > 0) or for all (op = 0).
+int set_weights(mk_ctx* c, int op, const float* weights, int n, void* stream) {
   if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (op != 0 && op != TK_QKV && op != TK_OPROJ && op != TK_GATEUP && op != TK_DOWN && op != TK_LMHEAD)
+    return fail(c, MK_ERR_INVALID_ARG, "op must be 0 or a projection task kind");
   if (!weights || n != c->n_sms) return fail(c, MK_ERR_INVALID_ARG, "need one weight per SM");
   std::vector<double> w(n);
   for (int i = 0; i < n; ++i) {
@@ -1219,18 +1227,26 @@ int mk_set_sm_weights(mk_ctx* c, const float* weights, int n, void* stream) {
   if (c->loaded && !cuda_ok(c, cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "stream sync"))
     return MK_ERR_CUDA;
   std::vector<double> old = c->sm_weights;
+  std::vector<double> old_op[8];
+  for (int k = 0; k < 8; ++k) old_op[k] = c->op_weights[k];
   Graph old_g = c->g;
   std::vector<uint32_t> old_q = c->qbegin;
   const int old_lm = c->n_lm;
   const size_t old_recs = c->n_recs;
   const uint64_t old_wb = c->weight_bytes_per_step;
-  c->sm_weights = w;
+  if (op == 0) {
+    c->sm_weights = w;
+    for (int k = 0; k < 8; ++k) c->op_weights[k].clear();
+  } else {
+    c->op_weights[op] = w;
+  }
   int rc = build_graph(c);
   if (rc == MK_OK && (c->g.tasks.size() > c->task_cap || (size_t)c->n_lm > c->lm_cap || c->n_recs > c->rec_cap))
     rc = fail(c, MK_ERR_UNSUPPORTED, "re-partitioned graph exceeds the workspace reserve");
   if (rc != MK_OK) {
     std::string m = c->err;
     c->sm_weights = old;
+    for (int k = 0; k < 8; ++k) c->op_weights[k] = old_op[k];
     c->g = old_g;
     c->qbegin = old_q;
     c->n_lm = old_lm;
@@ -1240,6 +1256,16 @@ int mk_set_sm_weights(mk_ctx* c, const float* weights, int n, void* stream) {
   }
   if (c->loaded && upload_graph(c, c->ws) != MK_OK) return MK_ERR_CUDA;
   return MK_OK;
+}
+}  // namespace
+
+int mk_set_sm_weights(mk_ctx* c, const float* weights, int n, void* stream) {
+  return set_weights(c, 0, weights, n, stream);
+}
+
+int mk_set_op_sm_weights(mk_ctx* c, int op_kind, const float* weights, int n, void* stream) {
+  if (op_kind == 0) return fail(c, MK_ERR_INVALID_ARG, "op_kind must be a projection task kind");
+  return set_weights(c, op_kind, weights, n, stream);
 }
 
 int mk_set_l2_prefetch(mk_ctx* c, int stages) {

@@ -185,3 +185,28 @@ def test_weighted_partition_follows_the_sm_weights():
             mk.mk_set_sm_weights(ctx, np.ones(n - 1, dtype=np.float32))
     finally:
         mk.mk_destroy(ctx)
+
+
+def test_per_op_weights_repartition_only_that_op():
+    ctx = mk.mk_build_taskgraph(mk.Config.from_shape(mi.LLAMA8B, 1, 1024).c(), -1)
+    try:
+        n = mk.mk_get_graph_info(ctx)["n_sms"]
+        before, _ = mk.mk_export_taskgraph(ctx)
+        w = np.random.default_rng(1).uniform(0.6, 1.4, n).astype(np.float32)
+        mk.mk_set_op_sm_weights(ctx, 5, w)  # gate/up only
+        tasks, counts = mk.mk_export_taskgraph(ctx)
+        assert mk.mk_validate_taskgraph(ctx, tasks, counts) == 0
+        per_sm = np.zeros(n)
+        for t in tasks:
+            if t[0] == 5:
+                per_sm[t[2]] += t[4]
+        assert np.allclose(per_sm / per_sm.sum(), w / w.sum(), rtol=0.03)
+        for k in (2, 4, 6, 7):  # the other projections keep their partition
+            assert np.array_equal(before[before[:, 0] == k][:, 2:5], tasks[tasks[:, 0] == k][:, 2:5])
+        with pytest.raises(mk.MkError):
+            mk.mk_set_op_sm_weights(ctx, 3, w)  # attention is not a projection
+        mk.mk_set_sm_weights(ctx, np.ones(n, dtype=np.float32))  # resets every projection
+        again, _ = mk.mk_export_taskgraph(ctx)
+        assert np.array_equal(again, before)
+    finally:
+        mk.mk_destroy(ctx)

@@ -136,7 +136,7 @@ def test_calibrated_schedule_keeps_parity():
     weights = m.calibrate(torch.tensor([tok], dtype=torch.int32, device=DEV), steps=1, rounds=2)
     for _ in range(2):
         ref.decode(np.array([tok], dtype=np.int32))
-    assert weights.shape[0] == m.info()["n_sms"]
+    assert weights.shape == (5, m.info()["n_sms"])  # one row per projection kind
     for i in range(4):
         rl = ref.decode(np.array([tok], dtype=np.int32))[0]
         gl, _ = m.decode(torch.tensor([tok], dtype=torch.int32, device=DEV))
