@@ -113,6 +113,7 @@ class Shape:
     vocab: int
     rms_eps: float
     rope_theta: float
+    qk_norm: bool = False  # LayerNorm on every query and key head before RoPE (Chameleon)
 
     def with_layers(self, n: int) -> "Shape":
         d = dict(self.__dict__)
@@ -124,6 +125,8 @@ class Shape:
 TINY = Shape("tiny", 2, 256, 4, 2, 64, 768, 1024, 1e-6, 1e4)
 LLAMA8B = Shape("llama3-8b", 32, 4096, 32, 8, 128, 14336, 128256, 1e-5, 5e5)
 CHAMELEON7B = Shape("chameleon-7b", 32, 4096, 32, 32, 128, 11008, 65536, 1e-5, 1e4)
+CHAMELEON7B_QK = Shape("chameleon-7b-qknorm", 32, 4096, 32, 32, 128, 11008, 65536, 1e-5, 1e4, qk_norm=True)
+TINY_QK = Shape("tiny-qknorm", 2, 256, 4, 2, 64, 768, 1024, 1e-5, 1e4, qk_norm=True)
 
 # tensor ids: one stream per tensor so any subset can be regenerated independently
 TID_EMBED, TID_LM_HEAD = 1, 2
@@ -135,7 +138,7 @@ def _layer_tid(layer: int, which: int) -> int:
     return 1000 + 16 * layer + which
 
 
-W_Q, W_K, W_V, W_O, W_G, W_U, W_D = range(7)
+W_Q, W_K, W_V, W_O, W_G, W_U, W_D, W_QN_G, W_QN_B, W_KN_G, W_KN_B = range(11)
 
 
 @dataclass
@@ -154,9 +157,16 @@ class Weights:
     wg: list = field(default_factory=list)
     wu: list = field(default_factory=list)
     wd: list = field(default_factory=list)
+    # QK-norm models only: LayerNorm gain and bias per head, [heads * head_dim] each
+    q_norm_w: list = field(default_factory=list)
+    q_norm_b: list = field(default_factory=list)
+    k_norm_w: list = field(default_factory=list)
+    k_norm_b: list = field(default_factory=list)
 
 
-def make_weights(s: Shape, seed: int = 0, sigma: float = 0.02) -> Weights:
+def make_weights(s: Shape, seed: int = 0, sigma: float = 0.02, norm_sigma: float = 0.2) -> Weights:
+    """Weights of shape `s`; for a QK-norm shape the norm gains are 1 + N(0, norm_sigma^2) and
+    the biases N(0, norm_sigma^2), per head and element."""
     H, F, D = s.hidden, s.ffn, s.head_dim
     w = Weights(s, normal_bf16(seed, TID_EMBED, (s.vocab, H), sigma),
                 normal_bf16(seed, TID_LM_HEAD, (s.vocab, H), sigma), const_bf16((H,), 1.0))
@@ -170,6 +180,12 @@ def make_weights(s: Shape, seed: int = 0, sigma: float = 0.02) -> Weights:
         w.wg.append(normal_bf16(seed, _layer_tid(l, W_G), (F, H), sigma))
         w.wu.append(normal_bf16(seed, _layer_tid(l, W_U), (F, H), sigma))
         w.wd.append(normal_bf16(seed, _layer_tid(l, W_D), (H, F), sigma))
+        if s.qk_norm:
+            nq, nkv = s.n_q_heads * D, s.n_kv_heads * D
+            w.q_norm_w.append(normal_bf16(seed, _layer_tid(l, W_QN_G), (nq,), norm_sigma, mean=1.0))
+            w.q_norm_b.append(normal_bf16(seed, _layer_tid(l, W_QN_B), (nq,), norm_sigma))
+            w.k_norm_w.append(normal_bf16(seed, _layer_tid(l, W_KN_G), (nkv,), norm_sigma, mean=1.0))
+            w.k_norm_b.append(normal_bf16(seed, _layer_tid(l, W_KN_B), (nkv,), norm_sigma))
     return w
 
 

@@ -43,7 +43,8 @@ _PP = ctypes.POINTER(ctypes.c_void_p)
 class _Weights(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("lm_head", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
                 ("attn_norm", _PP), ("wq", _PP), ("wk", _PP), ("wv", _PP), ("wo", _PP),
-                ("mlp_norm", _PP), ("wg", _PP), ("wu", _PP), ("wd", _PP)]
+                ("mlp_norm", _PP), ("wg", _PP), ("wu", _PP), ("wd", _PP),
+                ("q_norm_w", _PP), ("q_norm_b", _PP), ("k_norm_w", _PP), ("k_norm_b", _PP)]
 
 
 def lib():
@@ -64,6 +65,9 @@ def lib():
         L.or_set_positions.argtypes = [vp, vp]
         L.or_position.argtypes = [vp, i32]
         L.or_argmax.argtypes = [vp, i32]
+        L.or_get_qk.argtypes = [vp, i32, vp, vp]
+        L.or_layernorm.argtypes = [vp, vp, vp, i32, dbl, vp]
+        L.or_layernorm.restype = None
         L.or_rmsnorm.argtypes = [vp, vp, i32, dbl, vp]
         L.or_rmsnorm.restype = None
         L.or_matvec_bf16.argtypes = [vp, vp, i32, i32, vp]
@@ -113,7 +117,10 @@ class Decoder:
 
         self._arrs = []
         fields = {}
-        for name in ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "wg", "wu", "wd"):
+        names = ["attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "wg", "wu", "wd"]
+        if getattr(weights, "q_norm_w", None):  # QK-norm model
+            names += ["q_norm_w", "q_norm_b", "k_norm_w", "k_norm_b"]
+        for name in names:
             p, a = arr(getattr(weights, name))
             self._arrs.append(a)
             fields[name] = p
@@ -174,6 +181,16 @@ class Decoder:
     def position(self, b: int = 0) -> int:
         return lib().or_position(self._h, b)
 
+    def get_qk(self, layer: int):
+        """q [batch, n_q_heads*head_dim] and k [batch, n_kv_heads*head_dim] of layer `layer` for the
+        last token of the last call (after QK-norm and RoPE, before the cache's bf16 rounding)."""
+        s = self.shape
+        q = np.empty((self.batch, s.n_q_heads * s.head_dim), dtype=np.float64)
+        k = np.empty((self.batch, s.n_kv_heads * s.head_dim), dtype=np.float64)
+        if lib().or_get_qk(self._h, int(layer), _ptr(q), _ptr(k)) != 0:
+            raise ValueError("or_get_qk rejected its arguments")
+        return q, k
+
 
 def argmax(logits: np.ndarray) -> int:
     x = _c(logits, np.float32)
@@ -184,6 +201,13 @@ def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
     x, g = _c(x, np.float64), _c(g, np.float64)
     y = np.empty_like(x)
     lib().or_rmsnorm(_ptr(x), _ptr(g), x.size, eps, _ptr(y))
+    return y
+
+
+def layernorm(x: np.ndarray, g: np.ndarray, b: np.ndarray, eps: float) -> np.ndarray:
+    x, g, b = _c(x, np.float64), _c(g, np.float64), _c(b, np.float64)
+    y = np.empty_like(x)
+    lib().or_layernorm(_ptr(x), _ptr(g), _ptr(b), x.size, eps, _ptr(y))
     return y
 
 

@@ -10,6 +10,8 @@
 //   per layer:
 //     xn  = RMSNorm(x; g_attn)                                (Mirage, "Case 1: Normalization + Linear")
 //     q,k,v = Wq xn, Wk xn, Wv xn                             (matmul, Mirage attention example)
+//     q,k = LayerNorm per head (QK-norm models only)          (Mirage, "Case 4.1: Attention with
+//                                                              Query-Key Normalization")
 //     q,k = RoPE(q,k; pos)                                    (rotate-half pairing, reading below)
 //     cache[pos] = k, v  (bf16-rounded when kv_round)         (KV-cache append)
 //     o_h = sum_j softmax_j(q_h . k_j * scale) v_j,  j = 0..pos,  kv head of q head h = h*nkv/nq
@@ -22,6 +24,9 @@
 //   * RMSNorm: y = x * (mean(x^2) + eps)^(-1/2) * g, the sum of squares in double.
 //   * RoPE: pairs (i, i + d/2) of each head; angle = pos * theta^(-2i/d) in double; in the
 //     fp32 mode cos and sin are rounded once to fp32 before use.
+//   * QK-norm: a LayerNorm over the head_dim values of each query head and each key head,
+//     with a gain and a bias per head and element, applied to the projections before RoPE
+//     (so the cache holds normalised, rotated keys), eps = the model's rms_eps.
 //   * scale = 1/sqrt(head_dim) in the decoder; the standalone op takes it as an argument
 //     (1.0 for the Mirage example, which applies no scaling).
 //   * GQA: contiguous groups, q head h reads kv head floor(h * nkv / nq).
@@ -135,6 +140,19 @@ void rmsnorm(const T* x, const uint16_t* g, int n, double eps, T* y) {
   for (int i = 0; i < n; ++i) y[i] = (T)((double)x[i] * r * bf16_to_double(g[i]));
 }
 
+// LayerNorm (QK-norm, Mirage "Case 4.1"): y = (x - mean) / sqrt(var + eps) * g + b, the
+// mean and the mean squared deviation in double.  In place is allowed (x == y).
+template <class T>
+void layernorm(const T* x, const uint16_t* g, const uint16_t* b, int n, double eps, T* y) {
+  double sum = 0;
+  for (int i = 0; i < n; ++i) sum += (double)x[i];
+  const double mean = sum / n;
+  double sq = 0;
+  for (int i = 0; i < n; ++i) sq += ((double)x[i] - mean) * ((double)x[i] - mean);
+  const double r = 1.0 / std::sqrt(sq / n + eps);
+  for (int i = 0; i < n; ++i) y[i] = (T)(((double)x[i] - mean) * r * bf16_to_double(g[i]) + bf16_to_double(b[i]));
+}
+
 // Rotary angle table entry for pair i at position pos (reading: rotate-half, theta^(-2i/d)).
 inline void rope_angle(int head_dim, int pos, double theta, int i, double* c, double* s) {
   double inv_freq = std::pow(theta, -2.0 * (double)i / (double)head_dim);
@@ -192,6 +210,7 @@ struct StateBase {
   or_weights w;
   int batch, max_seq, kv_round;
   std::vector<int> pos;
+  std::vector<double> last_q, last_k;  // [layer][batch][heads*head_dim] of the last token
   virtual ~StateBase() {}
   virtual int forward(const int32_t* tokens, int T, float* logits_f32, double* logits_f64, bool all_logits) = 0;
   virtual void set_cache(const uint16_t* kv, int length) = 0;
@@ -265,12 +284,30 @@ struct State : StateBase {
       linear(w.wq[l], nq * D, H, xn.data(), N, q.data());
       linear(w.wk[l], nkv * D, H, xn.data(), N, k.data());
       linear(w.wv[l], nkv * D, H, xn.data(), N, v.data());
+      if (w.q_norm_w) {
+        for (int n = 0; n < N; ++n) {
+          for (int h = 0; h < nq; ++h) {
+            T* qh = &q[((size_t)n * nq + h) * D];
+            layernorm(qh, w.q_norm_w[l] + (size_t)h * D, w.q_norm_b[l] + (size_t)h * D, D, c.rms_eps, qh);
+          }
+          for (int h = 0; h < nkv; ++h) {
+            T* kh = &k[((size_t)n * nkv + h) * D];
+            layernorm(kh, w.k_norm_w[l] + (size_t)h * D, w.k_norm_b[l] + (size_t)h * D, D, c.rms_eps, kh);
+          }
+        }
+      }
       for (int b = 0; b < batch; ++b)
         for (int t = 0; t < T_; ++t) {
           int n = b * T_ + t, p = pos[b] + t;
           for (int h = 0; h < nq; ++h) rope_head(&q[((size_t)n * nq + h) * D], D, p, c.rope_theta, f32_table);
+          for (int h = 0; h < nkv; ++h) rope_head(&k[((size_t)n * nkv + h) * D], D, p, c.rope_theta, f32_table);
+          if (t == T_ - 1) {
+            for (int e = 0; e < nq * D; ++e)
+              last_q[((size_t)l * batch + b) * nq * D + e] = (double)q[(size_t)n * nq * D + e];
+            for (int e = 0; e < nkv * D; ++e)
+              last_k[((size_t)l * batch + b) * nkv * D + e] = (double)k[(size_t)n * nkv * D + e];
+          }
           for (int h = 0; h < nkv; ++h) {
-            rope_head(&k[((size_t)n * nkv + h) * D], D, p, c.rope_theta, f32_table);
             for (int e = 0; e < D; ++e) {
               cache[cidx(l, 0, b, h, p) + e] = kv_store((double)k[((size_t)n * nkv + h) * D + e]);
               cache[cidx(l, 1, b, h, p) + e] = kv_store((double)v[((size_t)n * nkv + h) * D + e]);
@@ -325,6 +362,9 @@ void or_set_threads(int n) { g_threads = n; }
 
 or_state* or_create(const or_config* cfg, const or_weights* w, int batch, int max_seq, int f64, int kv_round) {
   if (!cfg || !w || batch < 1 || max_seq < 1) return nullptr;
+  if ((w->q_norm_w || w->q_norm_b || w->k_norm_w || w->k_norm_b) &&
+      !(w->q_norm_w && w->q_norm_b && w->k_norm_w && w->k_norm_b))
+    return nullptr;  // QK-norm needs all four arrays
   if (cfg->n_layers < 1 || cfg->hidden < 1 || cfg->n_q_heads < 1 || cfg->n_kv_heads < 1 || cfg->head_dim < 2 ||
       (cfg->head_dim & 1) || cfg->ffn < 1 || cfg->vocab < 1 || cfg->n_q_heads % cfg->n_kv_heads)
     return nullptr;
@@ -344,6 +384,8 @@ or_state* or_create(const or_config* cfg, const or_weights* w, int batch, int ma
   s->max_seq = max_seq;
   s->kv_round = kv_round;
   s->pos.assign(batch, 0);
+  s->last_q.assign((size_t)cfg->n_layers * batch * cfg->n_q_heads * cfg->head_dim, 0.0);
+  s->last_k.assign((size_t)cfg->n_layers * batch * cfg->n_kv_heads * cfg->head_dim, 0.0);
   return new or_state{s};
 }
 
@@ -393,6 +435,16 @@ int or_position(const or_state* s, int b) {
   return s->impl->pos[b];
 }
 
+int or_get_qk(const or_state* s, int layer, double* q, double* k) {
+  if (!s || !q || !k || layer < 0 || layer >= s->impl->c.n_layers) return -1;
+  const StateBase* b = s->impl;
+  const size_t nq = (size_t)b->batch * b->c.n_q_heads * b->c.head_dim;
+  const size_t nk = (size_t)b->batch * b->c.n_kv_heads * b->c.head_dim;
+  std::memcpy(q, b->last_q.data() + (size_t)layer * nq, nq * sizeof(double));
+  std::memcpy(k, b->last_k.data() + (size_t)layer * nk, nk * sizeof(double));
+  return 0;
+}
+
 int or_argmax(const float* logits, int n) {
   int best = 0;
   for (int i = 1; i < n; ++i)
@@ -405,6 +457,16 @@ void or_rmsnorm(const double* x, const double* g, int n, double eps, double* y) 
   for (int i = 0; i < n; ++i) ss += x[i] * x[i];
   double r = 1.0 / std::sqrt(ss / n + eps);
   for (int i = 0; i < n; ++i) y[i] = x[i] * r * g[i];
+}
+
+void or_layernorm(const double* x, const double* g, const double* b, int n, double eps, double* y) {
+  double sum = 0;
+  for (int i = 0; i < n; ++i) sum += x[i];
+  const double mean = sum / n;
+  double sq = 0;
+  for (int i = 0; i < n; ++i) sq += (x[i] - mean) * (x[i] - mean);
+  const double r = 1.0 / std::sqrt(sq / n + eps);
+  for (int i = 0; i < n; ++i) y[i] = (x[i] - mean) * r * g[i] + b[i];
 }
 
 void or_matvec_bf16(const uint16_t* W, const double* x, int rows, int cols, double* y) {

@@ -12,7 +12,9 @@
  *   - RMSNorm + linear and the gated MLP: Mirage article (iaiol.com), "Case 1:
  *     Normalization + Linear" and "Case 3: Gated MLP";
  *   - attention O = softmax(Q K) V: Mirage article, the attention example (Q [64,1,128],
- *     K [64,128,4096], V [64,4096,128], fp16).
+ *     K [64,128,4096], V [64,4096,128], fp16);
+ *   - optional QK-norm: a LayerNorm on every query and key head before attention, Mirage
+ *     article, "Case 4.1: Attention with Query-Key Normalization" (Chameleon, ViT-22B).
  * Where the pages are silent (RoPE pairing, scale, GQA grouping, precision), the
  * readings are stated next to each function in oracle.cpp.
  *
@@ -52,6 +54,12 @@ typedef struct or_weights {
   const uint16_t* const* wg;  /* [ffn, hidden] */
   const uint16_t* const* wu;  /* [ffn, hidden] */
   const uint16_t* const* wd;  /* [hidden, ffn] */
+  /* QK-norm (NULL arrays = the model has none): LayerNorm gain and bias of every query head
+   * ([n_q_heads*head_dim], head h at h*head_dim) and key head ([n_kv_heads*head_dim]). */
+  const uint16_t* const* q_norm_w;
+  const uint16_t* const* q_norm_b;
+  const uint16_t* const* k_norm_w;
+  const uint16_t* const* k_norm_b;
 } or_weights;
 
 typedef struct or_state or_state;
@@ -80,9 +88,15 @@ int or_set_positions(or_state* s, const int32_t* pos);
 int or_position(const or_state* s, int b);
 /* Greedy pick: index of the largest logit, the lowest index among equal values. */
 int or_argmax(const float* logits, int n);
+/* The query and key vectors (after QK-norm, if any, and RoPE; before the bf16 rounding of the
+ * cache) that layer `layer` computed for the last token of each sequence in the last
+ * prefill or decode call: q [batch][n_q_heads*head_dim], k [batch][n_kv_heads*head_dim]. */
+int or_get_qk(const or_state* s, int layer, double* q, double* k);
 
 /* ---- single operations (the pieces the decoder step is made of), fp64 I/O ---- */
 void or_rmsnorm(const double* x, const double* g, int n, double eps, double* y);
+/* LayerNorm: y = (x - mean(x)) / sqrt(var(x) + eps) * g + b, var the mean squared deviation. */
+void or_layernorm(const double* x, const double* g, const double* b, int n, double eps, double* y);
 void or_matvec_bf16(const uint16_t* W, const double* x, int rows, int cols, double* y);
 void or_rope(double* v, int head_dim, int pos, double theta);
 void or_rope_cos_sin(int head_dim, int pos, double theta, float* cos_out, float* sin_out);

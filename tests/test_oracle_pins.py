@@ -362,3 +362,156 @@ def test_thread_count_does_not_change_results(tiny_weights):
     b = oracle.Decoder(w, 1, 8).prefill(toks)
     oracle.set_threads(0)
     assert np.array_equal(a, b)
+
+
+# ---------------------------------------------------------------- QK-norm (Chameleon)
+# Mirage article, "Case 4.1: Attention with Query-Key Normalization": a LayerNorm on the
+# query and key vectors before attention.
+
+def test_layernorm_closed_form_and_torch():
+    # [1, 2, 3, 4]: mean 2.5, mean squared deviation 1.25 -> (x - 2.5) / sqrt(1.25) = (2x - 5) / sqrt(5)
+    x = np.array([1.0, 2.0, 3.0, 4.0])
+    y = oracle.layernorm(x, np.ones(4), np.zeros(4), 0.0)
+    assert np.allclose(y, (2 * x - 5) / math.sqrt(5), rtol=1e-15, atol=1e-15)
+    g, b = np.array([2.0, -1.0, 0.5, 3.0]), np.array([0.25, 0.0, -1.0, 4.0])
+    assert np.allclose(oracle.layernorm(x, g, b, 0.0), (2 * x - 5) / math.sqrt(5) * g + b, rtol=1e-15, atol=1e-15)
+    # eps enters next to the variance: constant input -> b exactly; eps shrinks the spread
+    assert np.array_equal(oracle.layernorm(np.full(8, 7.0), np.full(8, 3.0), np.arange(8.0), 1e-5), np.arange(8.0))
+    assert np.allclose(oracle.layernorm(x, np.ones(4), np.zeros(4), 1.25), (x - 2.5) / math.sqrt(2.5), rtol=1e-15)
+    rng = np.random.default_rng(7)
+    x, g, b = rng.normal(size=128) * 3 + 1, rng.normal(size=128), rng.normal(size=128)
+    ref = torch.nn.functional.layer_norm(torch.tensor(x), (128,), torch.tensor(g), torch.tensor(b), eps=1e-5).numpy()
+    assert np.allclose(oracle.layernorm(x, g, b, 1e-5), ref, rtol=1e-12, atol=1e-13)
+
+
+@pytest.fixture(scope="module")
+def tiny_qk_weights():
+    return _random_gains(mi.make_weights(mi.TINY_QK, seed=3, sigma=0.05))
+
+
+def _hf_chameleon(w):
+    """transformers' Chameleon text decoder (independent implementation; LayerNorm over each
+    query / key head with per-head gain and bias, eps 1e-5, before RoPE), float64."""
+    from transformers import ChameleonConfig, ChameleonForConditionalGeneration
+    s = w.shape
+    assert s.rms_eps == 1e-5  # the transformers model fixes the QK LayerNorm eps at 1e-5
+    vq = dict(embed_dim=32, num_embeddings=16, double_latent=False, latent_channels=32, resolution=16,
+              in_channels=3, base_channels=32, channel_multiplier=[1], num_res_blocks=1, attn_resolutions=[],
+              attn_type="vanilla", dropout=0.0)  # unused image tokenizer, kept small
+    cfg = ChameleonConfig(vocab_size=s.vocab, hidden_size=s.hidden, intermediate_size=s.ffn,
+                          num_hidden_layers=s.n_layers, num_attention_heads=s.n_q_heads,
+                          num_key_value_heads=s.n_kv_heads, rms_norm_eps=s.rms_eps, rope_theta=s.rope_theta,
+                          max_position_embeddings=4096, tie_word_embeddings=False, attention_bias=False,
+                          vq_config=vq, vocabulary_map={"<image>": s.vocab + 5})
+    cfg._attn_implementation = "eager"
+    m = ChameleonForConditionalGeneration(cfg).to(torch.float64).eval()
+    assert not cfg.swin_norm
+
+    def t(a):
+        return torch.tensor(mi.bf16_to_f32(a), dtype=torch.float64)
+
+    D = s.head_dim
+    with torch.no_grad():
+        m.model.embed_tokens.weight.copy_(t(w.embed))
+        m.lm_head.weight.copy_(t(w.lm_head))
+        m.model.norm.weight.copy_(t(w.final_norm))
+        for l, layer in enumerate(m.model.layers):
+            layer.input_layernorm.weight.copy_(t(w.attn_norm[l]))
+            layer.post_attention_layernorm.weight.copy_(t(w.mlp_norm[l]))
+            a = layer.self_attn
+            a.q_proj.weight.copy_(t(w.wq[l]))
+            a.k_proj.weight.copy_(t(w.wk[l]))
+            a.v_proj.weight.copy_(t(w.wv[l]))
+            a.o_proj.weight.copy_(t(w.wo[l]))
+            a.q_norm.weight.copy_(t(w.q_norm_w[l]).reshape(s.n_q_heads, D))
+            a.q_norm.bias.copy_(t(w.q_norm_b[l]).reshape(s.n_q_heads, D))
+            a.k_norm.weight.copy_(t(w.k_norm_w[l]).reshape(s.n_kv_heads, D))
+            a.k_norm.bias.copy_(t(w.k_norm_b[l]).reshape(s.n_kv_heads, D))
+            layer.mlp.gate_proj.weight.copy_(t(w.wg[l]))
+            layer.mlp.up_proj.weight.copy_(t(w.wu[l]))
+            layer.mlp.down_proj.weight.copy_(t(w.wd[l]))
+    return m
+
+
+def test_qk_norm_decoder_matches_transformers_chameleon(tiny_qk_weights):
+    w = tiny_qk_weights
+    T = 11
+    toks = mi.prompt(3, 0, T + 3, w.shape.vocab)
+    m = _hf_chameleon(w)
+    with torch.no_grad():
+        ref = m(input_ids=torch.tensor(toks[None].astype(np.int64)), use_cache=False).logits[0].numpy()
+    d = oracle.Decoder(w, 1, 64, f64=True, kv_round=False)
+    got = [d.prefill(toks[:T])[0]]
+    for t in range(T, T + 3):
+        got.append(d.decode_f64(toks[t:t + 1])[0])
+    got, want = np.stack(got), ref[T - 1:]
+    assert np.max(np.abs(got - want)) < 2e-5 * np.max(np.abs(want))
+    # and the norm matters: the same weights without QK-norm give other logits
+    import copy
+    w0 = copy.copy(w)
+    w0.q_norm_w = []
+    plain = oracle.Decoder(w0, 1, 64, f64=True, kv_round=False).prefill(toks[:T])[0]
+    assert np.max(np.abs(plain - want[0])) > 1e-2 * np.max(np.abs(want[0]))
+
+
+def _unrotate(v, pos, theta, D):
+    # inverse RoPE of every head: rotation by -pos (RoPE pinned above as a plane rotation per pair)
+    return np.concatenate([oracle.rope(h, -pos, theta) for h in v.reshape(-1, D)])
+
+
+@pytest.mark.parametrize("T", [1, 6])
+def test_qk_norm_heads_are_layer_normed_before_rope(tiny_qk_weights, T):
+    # Every query and key head of the last token, rotated back, is g * z + b with z of mean 0
+    # and mean square var/(var+eps) ~ 1: a dropped mean, a gain or bias of another head, or
+    # RoPE applied before the norm all break it (T = 1: position 0, no rotation at all).
+    w = tiny_qk_weights
+    s = w.shape
+    D = s.head_dim
+    d = oracle.Decoder(w, 2, 16, f64=True)
+    d.prefill(np.stack([mi.prompt(3, 1, T, s.vocab), mi.prompt(3, 2, T, s.vocab)]))
+    for l in range(s.n_layers):
+        q, k = d.get_qk(l)
+        for vec, gw, gb in ((q, w.q_norm_w[l], w.q_norm_b[l]), (k, w.k_norm_w[l], w.k_norm_b[l])):
+            g = mi.bf16_to_f32(gw).astype(np.float64)
+            b = mi.bf16_to_f32(gb).astype(np.float64)
+            for row in vec:
+                z = ((_unrotate(row, T - 1, s.rope_theta, D) - b) / g).reshape(-1, D)
+                assert np.max(np.abs(z.mean(axis=1))) < 1e-10
+                assert np.max(np.abs((z * z).mean(axis=1) - 1.0)) < 1e-3
+    # the cache holds the normalised, rotated keys (bf16-rounded)
+    kv = d.get_cache(T)
+    _, k = d.get_qk(s.n_layers - 1)
+    got = mi.bf16_to_f32(kv[s.n_layers - 1, 0, :, :, T - 1, :]).reshape(2, -1)
+    assert np.allclose(got, k, rtol=2 ** -8, atol=1e-6)
+
+
+def test_qk_norm_absorbs_a_per_head_scale(tiny_qk_weights):
+    # LayerNorm(a x) = LayerNorm(x) up to eps: scaling the W_q rows of one query head by 4 and
+    # the W_k rows of one key head by 2 (exact in bf16) leaves the logits unchanged with
+    # QK-norm and changes them without.
+    w = tiny_qk_weights
+    s = w.shape
+    D = s.head_dim
+    import copy
+
+    def scaled(src):
+        w2 = copy.copy(src)
+        w2.wq, w2.wk = list(src.wq), list(src.wk)
+        for l in range(s.n_layers):
+            q = mi.bf16_to_f32(src.wq[l]).copy()
+            q[D:2 * D] *= 4.0
+            k = mi.bf16_to_f32(src.wk[l]).copy()
+            k[:D] *= 2.0
+            w2.wq[l] = (q.view(np.uint32) >> 16).astype(np.uint16)
+            w2.wk[l] = (k.view(np.uint32) >> 16).astype(np.uint16)
+        return w2
+
+    toks = mi.prompt(3, 3, 9, s.vocab)
+    a = oracle.Decoder(w, 1, 16, f64=True, kv_round=False).prefill(toks)[0]
+    b = oracle.Decoder(scaled(w), 1, 16, f64=True, kv_round=False).prefill(toks)[0]
+    assert np.max(np.abs(a - b)) < 1e-4 * np.max(np.abs(a))
+    w0 = copy.copy(w)
+    w0.q_norm_w = []
+    a0 = oracle.Decoder(w0, 1, 16, f64=True, kv_round=False).prefill(toks)[0]
+    b0 = oracle.Decoder(scaled(w0), 1, 16, f64=True, kv_round=False).prefill(toks)[0]
+    assert np.max(np.abs(a0 - b0)) > 1e-2 * np.max(np.abs(a0))
