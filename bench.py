@@ -10,9 +10,9 @@ W=8, K=504 is the 512-step run of that workload).  The weights stream from HBM e
 
 Other workloads of the same decoder family (`--workload`, each printing its own line; the
 default is the one above): `llama8b-ctx4096` (8B shape, batch 1, every step attending over
-4096+ cached positions) and `chameleon7b-b1` / `-b4` / `-b16` (Chameleon-7B-shaped MHA
+4096+ cached positions), `chameleon7b-b1` / `-b4` / `-b16` (Chameleon-7B-shaped MHA
 decoder, 1, 4 or 16 sequences each at 1024+ cached positions; 16 sequences run the
-projections on the tensor cores).  Their caches are seeded synthetic values standing in for
+projections on the tensor cores) and `chameleon7b-qk-b1` / `-b16` (the same with QK-norm).  Their caches are seeded synthetic values standing in for
 the prefilled prompts.
 
 Multi-GPU (torchrun, one process per GPU): independent replicas, no collective on the data
@@ -48,6 +48,8 @@ WORKLOADS = {
     "chameleon7b-b1": ("CHAMELEON7B", 1, 1024),
     "chameleon7b-b4": ("CHAMELEON7B", 4, 1024),
     "chameleon7b-b16": ("CHAMELEON7B", 16, 1024),
+    "chameleon7b-qk-b1": ("CHAMELEON7B_QK", 1, 1024),
+    "chameleon7b-qk-b16": ("CHAMELEON7B_QK", 16, 1024),
     "attention": (None, 0, 0),  # the standalone decode-attention op, Mirage size
 }
 WORKLOAD_TEXT = {
@@ -57,6 +59,10 @@ WORKLOAD_TEXT = {
     "chameleon7b-b4": "chameleon-7b-shape MHA decode, batch 4, 1024 cached positions each (synthetic), greedy",
     "chameleon7b-b16": "chameleon-7b-shape MHA decode, batch 16 (tensor-core projections), 1024 cached positions "
                        "each (synthetic), greedy",
+    "chameleon7b-qk-b1": "chameleon-7b-shape MHA decode with QK-norm (LayerNorm per q/k head before RoPE), "
+                         "batch 1, 1024 cached positions (synthetic), greedy",
+    "chameleon7b-qk-b16": "chameleon-7b-shape MHA decode with QK-norm, batch 16 (tensor-core projections), "
+                          "1024 cached positions each (synthetic), greedy",
     "attention": "standalone decode attention O = softmax(Q.K).V, fp16 Q [64,1,128], K^T [64,128,4096], "
                  "V [64,4096,128], fp32 out, 3 rotating input copies",
 }
@@ -108,11 +114,14 @@ def measured_peaks():
 
 def algorithmic_bytes(shape, positions):
     """Bytes one decode step must read from HBM: every weight once (projections, norms, LM
-    head), one embedding row, and the K/V actually attended (positions 0..p inclusive)."""
+    head, QK-norm gains and biases), one embedding row, and the K/V actually attended
+    (positions 0..p inclusive)."""
     s = shape
     D = s.head_dim
     per_layer = ((s.n_q_heads + 2 * s.n_kv_heads) * D * s.hidden + s.hidden * s.n_q_heads * D
                  + 2 * s.ffn * s.hidden + s.hidden * s.ffn + 2 * s.hidden) * 2
+    if getattr(s, "qk_norm", False):
+        per_layer += 2 * (s.n_q_heads + s.n_kv_heads) * D * 2
     weights = s.n_layers * per_layer + (s.vocab * s.hidden + s.hidden) * 2 + s.hidden * 2
     kv = [s.n_layers * 2 * s.n_kv_heads * (p + 1) * D * 2 for p in positions]
     return weights, kv

@@ -44,12 +44,19 @@ extern "C" {
  * MPK decode benchmark, "Valeur cle de MPK"; Chameleon-7B / Llama-3-8B shapes in the Mirage
  * article's end-to-end figure).  Requirements checked by mk_build_taskgraph:
  * hidden == n_q_heads * head_dim; n_q_heads % n_kv_heads == 0; head_dim in {64, 128};
- * hidden and ffn multiples of 8; max_batch in [1, MK_MAX_BATCH]; tie_embeddings == 0. */
+ * hidden and ffn multiples of 8; max_batch in [1, MK_MAX_BATCH]; tie_embeddings == 0;
+ * qk_norm in {0, 1}. */
 typedef struct mk_config {
   int n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab;
   float rms_eps, rope_theta;
   int max_batch, max_seq;
   int tie_embeddings; /* must be 0: separate LM-head matrix */
+  /* 1: QK-norm (Mirage article, "Case 4.1: Attention with Query-Key Normalization", as in
+   * Chameleon): every query head and key head of the QKV projection goes through a LayerNorm
+   * over its head_dim values (mean and mean squared deviation, eps = rms_eps) with a gain and
+   * a bias per head and element, before RoPE; the cache holds the normalised, rotated keys.
+   * 0: none. */
+  int qk_norm;
 } mk_config;
 
 #define MK_MAX_BATCH 16
@@ -69,6 +76,12 @@ typedef struct mk_host_weights {
   const uint16_t* const* wg;  /* [ffn, hidden] */
   const uint16_t* const* wu;  /* [ffn, hidden] */
   const uint16_t* const* wd;  /* [hidden, ffn] */
+  /* QK-norm gains and biases (required when cfg.qk_norm, ignored otherwise):
+   * q_norm_* [n_q_heads*head_dim] (head h at h*head_dim), k_norm_* [n_kv_heads*head_dim]. */
+  const uint16_t* const* q_norm_w;
+  const uint16_t* const* q_norm_b;
+  const uint16_t* const* k_norm_w;
+  const uint16_t* const* k_norm_b;
 } mk_host_weights;
 
 typedef struct mk_ctx mk_ctx; /* opaque, library-owned host object */

@@ -47,7 +47,8 @@ class mk_config(ctypes.Structure):
     _fields_ = [("n_layers", ctypes.c_int), ("hidden", ctypes.c_int), ("n_q_heads", ctypes.c_int),
                 ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("ffn", ctypes.c_int),
                 ("vocab", ctypes.c_int), ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
-                ("max_batch", ctypes.c_int), ("max_seq", ctypes.c_int), ("tie_embeddings", ctypes.c_int)]
+                ("max_batch", ctypes.c_int), ("max_seq", ctypes.c_int), ("tie_embeddings", ctypes.c_int),
+                ("qk_norm", ctypes.c_int)]
 
 
 _PP = ctypes.POINTER(ctypes.c_void_p)
@@ -56,7 +57,8 @@ _PP = ctypes.POINTER(ctypes.c_void_p)
 class mk_host_weights(ctypes.Structure):
     _fields_ = [("embed", ctypes.c_void_p), ("lm_head", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
                 ("attn_norm", _PP), ("wq", _PP), ("wk", _PP), ("wv", _PP), ("wo", _PP),
-                ("mlp_norm", _PP), ("wg", _PP), ("wu", _PP), ("wd", _PP)]
+                ("mlp_norm", _PP), ("wg", _PP), ("wu", _PP), ("wd", _PP),
+                ("q_norm_w", _PP), ("q_norm_b", _PP), ("k_norm_w", _PP), ("k_norm_b", _PP)]
 
 
 class mk_graph_info(ctypes.Structure):
@@ -158,15 +160,19 @@ def _host_weights(w, n_layers):
         keep.append(a)
         return ctypes.cast(a, _PP)
 
+    qk = [arr(getattr(w, name)) if getattr(w, "q_norm_w", None) else None
+          for name in ("q_norm_w", "q_norm_b", "k_norm_w", "k_norm_b")]
     hw = mk_host_weights(_ptr(w.embed), _ptr(w.lm_head), _ptr(w.final_norm),
                          arr(w.attn_norm), arr(w.wq), arr(w.wk), arr(w.wv), arr(w.wo),
-                         arr(w.mlp_norm), arr(w.wg), arr(w.wu), arr(w.wd))
+                         arr(w.mlp_norm), arr(w.wg), arr(w.wu), arr(w.wd), *qk)
     return hw, keep
 
 
 def mk_load_weights(ctx, weights, weight_arena, workspace, stream=None, n_layers: int | None = None):
     """``weights``: object with bf16 (uint16) host arrays embed, lm_head, final_norm and per-layer
-    lists attn_norm, wq, wk, wv, wo, mlp_norm, wg, wu, wd (canonical [out, in] row-major)."""
+    lists attn_norm, wq, wk, wv, wo, mlp_norm, wg, wu, wd (canonical [out, in] row-major); for a
+    QK-norm model also q_norm_w, q_norm_b ([n_q_heads*head_dim]) and k_norm_w, k_norm_b
+    ([n_kv_heads*head_dim])."""
     n = n_layers if n_layers is not None else len(weights.wq)
     hw, keep = _host_weights(weights, n)
     _check(_lib.mk_load_weights(ctx, ctypes.byref(hw), _ptr(weight_arena), _ptr(workspace), _stream(stream)), ctx)
@@ -305,15 +311,18 @@ class Config:
     rope_theta: float
     max_batch: int = 1
     max_seq: int = 1024
+    qk_norm: bool = False
 
     @classmethod
     def from_shape(cls, shape, max_batch: int = 1, max_seq: int = 1024) -> "Config":
         return cls(shape.n_layers, shape.hidden, shape.n_q_heads, shape.n_kv_heads, shape.head_dim, shape.ffn,
-                   shape.vocab, shape.rms_eps, shape.rope_theta, max_batch, max_seq)
+                   shape.vocab, shape.rms_eps, shape.rope_theta, max_batch, max_seq,
+                   bool(getattr(shape, "qk_norm", False)))
 
     def c(self) -> mk_config:
         return mk_config(self.n_layers, self.hidden, self.n_q_heads, self.n_kv_heads, self.head_dim, self.ffn,
-                         self.vocab, self.rms_eps, self.rope_theta, self.max_batch, self.max_seq, 0)
+                         self.vocab, self.rms_eps, self.rope_theta, self.max_batch, self.max_seq, 0,
+                         int(self.qk_norm))
 
 
 class Megakernel:

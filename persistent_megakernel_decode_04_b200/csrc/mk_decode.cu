@@ -47,6 +47,7 @@ struct DSmem {
   float lmv[kWorkerWarps];
   int lmi[kWorkerWarps];
   float tss[2][kTcBatch];    // tensor-core tasks (by parity): per-sequence sum of x^2 over the K range
+  float qn[4 * 128];         // QK-norm: the normed, rotated q heads of an attention task's group
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t bop_full[2];      // tensor-core operand buffer staged (one arrival per worker warp)
@@ -65,6 +66,10 @@ __host__ __device__ constexpr int ring_stages(bool tc) { return tc ? kTcStages :
 __host__ __device__ constexpr size_t ring_bytes(bool tc) {
   return (size_t)ring_stages(tc) * kSlotBytes + (tc ? (size_t)kTcBopBytes : 0);
 }
+
+static_assert(ring_bytes(false) + sizeof(DSmem) + 1024 <= 227 * 1024 &&
+                  ring_bytes(true) + sizeof(DSmem) + 1024 <= 227 * 1024,
+              "dynamic shared memory of a CTA exceeds 227 KB");
 
 __device__ __forceinline__ void worker_bar() { named_bar_sync(1, kWorkerThreads); }
 
@@ -120,6 +125,8 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
   u += 0x7fffu + ((u >> 16) & 1u);
   return (uint16_t)(u >> 16);
 }
+
+__device__ __forceinline__ float bf2f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
 // Which stream a GEMV task reads: arena offset and row length (bytes) for the task's op.  A
 // tensor-core task streams whole weight blocks: row0 counts blocks of kSlotBytes.
@@ -321,6 +328,9 @@ __device__ __forceinline__ float norm_factor(const DSmem& S, int K, float eps, i
 // GEMV total is S.tot[e] (sequences b >= nb are skipped).
 // Packed QKV row R of sequence b (value v; other = its RoPE partner row R ^ 1): q rows go to
 // qbuf after RoPE, k rows after RoPE and v rows as they are into the bf16 cache at pos[b].
+// With QK-norm the q and k rows are stored as they are (qbuf, kraw; natural dim order): the
+// LayerNorm needs a whole head, which the attention task of its KV head holds, so the norm
+// and RoPE of q and of the new key happen there.
 __device__ __forceinline__ void qkv_out(const DecodeParams& P, int layer, int R, int b, float v, float other,
                                         int st) {
   const int D = P.D, G = P.nq / P.nkv, half = D / 2;
@@ -333,6 +343,14 @@ __device__ __forceinline__ void qkv_out(const DecodeParams& P, int layer, int R,
     // q or k: rows come in RoPE pairs (i, i + D/2) at packed positions (2i, 2i+1)
     const int pd = (rr < G * D) ? (rr % D) : (rr - G * D);
     const int i = pd >> 1, hi = pd & 1;
+    if (P.qk_norm) {
+      const int dim = hi ? i + half : i;
+      if (rr < G * D)
+        P.qbuf[((size_t)layer * P.B + b) * P.nq * D + (size_t)(grp * G + rr / D) * D + dim] = v;
+      else
+        P.kraw[((size_t)layer * P.B + b) * P.nkv * D + (size_t)grp * D + dim] = v;
+      return;
+    }
     const float2 cs = P.rope[(size_t)pos * half + i];
     float outv;
     int dim;
@@ -378,7 +396,8 @@ __device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, c
 // weight ring like weights: the producer copies the chunk's old K and V rows (kv_stage_keys
 // per stage, K rows then V rows) in queue order, ahead of the task's release, and the workers
 // read them from shared memory.  Only q and the key/value at the current position (written by
-// this step's QKV tasks) are loaded after the release.  Each lane holds DL = D/32 dims of
+// this step's QKV tasks) are loaded after the release; with QK-norm the task also normalises
+// and rotates q and that key (qk_norm_rope).  Each lane holds DL = D/32 dims of
 // every head; the kAttnBlock x 4 (key, head) partial dot products of a block are summed
 // across lanes with one transposed butterfly (each exchange halves the live values) and
 // broadcast back with shuffles.
@@ -432,6 +451,80 @@ __device__ __forceinline__ void attn_load_key(const uint16_t* kc, const uint16_t
     kw[0] = __ldcg(reinterpret_cast<const unsigned int*>(kc + (size_t)j * D + lane * 2));
     vw[0] = __ldcg(reinterpret_cast<const unsigned int*>(vc + (size_t)j * D + lane * 2));
   }
+}
+
+// QK-norm (Mirage article, "Case 4.1: Attention with Query-Key Normalization"): LayerNorm of
+// one head held by a warp (lane l holds dims l*DL .. l*DL + DL-1), with this lane's gains g and
+// biases bi of the head, then RoPE with this lane's angles cs of the position.  The
+// rotate-half partner of dim d < D/2 is d + D/2, held by lane l ^ 16 at the same register
+// index.  Warp-uniform.
+template <int D>
+__device__ __forceinline__ void qk_norm_rope(float (&v)[D / 32], const float (&g)[D / 32], const float (&bi)[D / 32],
+                                             const float2 (&cs)[D / 32], float eps, int lane) {
+  constexpr int DL = D / 32;
+  float sum = 0.f;
+#pragma unroll
+  for (int i = 0; i < DL; ++i) sum += v[i];
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  const float mean = sum * (1.0f / D);
+  float sq = 0.f;
+#pragma unroll
+  for (int i = 0; i < DL; ++i) {
+    v[i] -= mean;
+    sq = fmaf(v[i], v[i], sq);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+  const float r = 1.0f / sqrtf(sq * (1.0f / D) + eps);
+#pragma unroll
+  for (int i = 0; i < DL; ++i) v[i] = fmaf(v[i] * r, g[i], bi[i]);
+  const bool hi = lane >= 16;
+#pragma unroll
+  for (int i = 0; i < DL; ++i) {
+    const float o = __shfl_xor_sync(0xffffffffu, v[i], 16);
+    v[i] = hi ? fmaf(v[i], cs[i].x, o * cs[i].y) : fmaf(v[i], cs[i].x, -(o * cs[i].y));
+  }
+}
+
+// QK-norm gains and biases of a layer: q gain [nq*D], q bias [nq*D], k gain [nkv*D], k bias [nkv*D].
+__device__ __forceinline__ const uint16_t* qk_norm_params(const DecodeParams& P, int layer) {
+  return reinterpret_cast<const uint16_t*>(P.arena + P.loff[layer].qkn);
+}
+
+// This lane's DL gains (or biases) of head row `head` of a QK-norm parameter array.
+template <int D>
+__device__ __forceinline__ void qk_param_load(const uint16_t* base, int head, int lane, float (&out)[D / 32]) {
+  const uint16_t* p = base + (size_t)head * D + lane * (D / 32);
+  if constexpr (D == 128) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    out[0] = __uint_as_float(u.x << 16);
+    out[1] = __uint_as_float(u.x & 0xffff0000u);
+    out[2] = __uint_as_float(u.y << 16);
+    out[3] = __uint_as_float(u.y & 0xffff0000u);
+  } else {
+    const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(p));
+    out[0] = __uint_as_float(u << 16);
+    out[1] = __uint_as_float(u & 0xffff0000u);
+  }
+}
+
+// Before an attention task's release (its inputs need not exist yet): bring this lane's QK-norm
+// gains, biases and RoPE angles into L1, so the norm after the release finds them there.
+template <int D>
+__device__ __forceinline__ void qk_norm_prefetch(const DecodeParams& P, const Task& t, int st, int lane) {
+  const AttnGeom a = attn_geom(P, t, st);
+  if (a.c >= a.nch_eff) return;
+  const int G = P.nq / P.nkv;
+  const uint16_t* nb = qk_norm_params(P, t.layer);
+  const int off = lane * (D / 32);
+  for (int h = 0; h < G; ++h) {
+    prefetch_l1(nb + (size_t)(a.g * G + h) * D + off);
+    prefetch_l1(nb + (size_t)(P.nq + a.g * G + h) * D + off);
+  }
+  prefetch_l1(nb + (size_t)(2 * P.nq + a.g) * D + off);
+  prefetch_l1(nb + (size_t)(2 * P.nq + P.nkv + a.g) * D + off);
+  prefetch_l1(P.rope + (size_t)(a.Lk - 1) * (D / 2) + (lane & 15) * (D / 32));
 }
 
 // Online-softmax update of this warp's (m, l, acc) with one block of up to kAttnBlock keys
@@ -544,7 +637,8 @@ __device__ __forceinline__ int attn_stage_span(const AttnGeom& a, int* jend) {
   return *jend > a.j0 ? (*jend - a.j0 + kv_stage_keys<D>() - 1) / kv_stage_keys<D>() : 0;
 }
 
-template <int D, bool TC>
+// QKN: the model has QK-norm (a separate instantiation, so the plain path keeps its registers).
+template <int D, bool TC, bool QKN>
 __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, Pipe& pp, const uint8_t* ring,
                                                const Task& t, uint32_t task_id, uint32_t& stall_ns, int st) {
   constexpr int DL = D / 32;
@@ -563,13 +657,52 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
 
   if (c < nch_eff) {  // uniform across the CTA
     float qv[4][DL], m[4], l[4], acc[4][DL];
+    const float* qsrc_n = qsrc;  // where this task's q heads are read from
+    if (QKN) {
+      // QK-norm: q and the key of the current position arrive as raw projections (qbuf, kraw).
+      // Warp h < G normalises and rotates q head h into S.qn; in the one chunk holding the
+      // current position, the last warp does the same for that key and writes it, in bf16, to
+      // its cache row.  After one barrier every warp reads q from S.qn and the key row from the
+      // cache like any other row.  The gains and angles were prefetched into L1 before the
+      // release.
+      const uint16_t* nb = qk_norm_params(P, t.layer);
+      const bool key_here = a.j0 <= pos && pos < a.j1;  // uniform across the CTA
+      const int head = warp < G ? g * G + warp : (warp == kAttnWarps - 1 && key_here) ? 2 * P.nq + g : -1;
+      if (head >= 0) {  // warp-uniform
+        float v[DL], gn[DL], bn[DL];
+        float2 cs[DL];
+        const float* src = warp < G ? qsrc + warp * D : P.kraw + ((size_t)t.layer * P.B + b) * P.nkv * D + (size_t)g * D;
+#pragma unroll
+        for (int i = 0; i < DL; ++i) {
+          v[i] = __ldcg(src + lane * DL + i);
+          cs[i] = P.rope[(size_t)pos * (D / 2) + (lane & 15) * DL + i];
+        }
+        qk_param_load<D>(nb, head, lane, gn);
+        qk_param_load<D>(nb, warp < G ? P.nq + head : head + P.nkv, lane, bn);
+        qk_norm_rope<D>(v, gn, bn, cs, P.eps, lane);
+        if (warp < G) {
+#pragma unroll
+          for (int i = 0; i < DL; ++i) S.qn[warp * D + lane * DL + i] = v[i];
+        } else {
+          uint16_t* kdst = const_cast<uint16_t*>(kc) + (size_t)pos * D + lane * DL;
+          if constexpr (D == 128)
+            *reinterpret_cast<uint2*>(kdst) = make_uint2((uint32_t)f2bf(v[0]) | ((uint32_t)f2bf(v[1]) << 16),
+                                                         (uint32_t)f2bf(v[2]) | ((uint32_t)f2bf(v[3]) << 16));
+          else
+            *reinterpret_cast<uint32_t*>(kdst) = (uint32_t)f2bf(v[0]) | ((uint32_t)f2bf(v[1]) << 16);
+        }
+      }
+      worker_bar();
+      qsrc_n = S.qn;
+    }
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       m[h] = -INFINITY;
       l[h] = 0.f;
 #pragma unroll
       for (int i = 0; i < DL; ++i) {
-        qv[h][i] = (h < G) ? __ldcg(qsrc + h * D + lane * DL + i) * P.attn_scale : 0.f;
+        qv[h][i] = (h < G) ? (QKN ? qsrc_n[h * D + lane * DL + i] : __ldcg(qsrc + h * D + lane * DL + i)) * P.attn_scale
+                           : 0.f;
         acc[h][i] = 0.f;
       }
     }
@@ -590,7 +723,8 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
     uint32_t kpre[kFreshPre][W], vpre[kFreshPre][W];
 #pragma unroll
     for (int j = 0; j < kFreshPre; ++j)
-      if (f_first + kAttnWarps * j < n_in) attn_load_key<D>(kc, vc, jf0 + f_first + kAttnWarps * j, lane, kpre[j], vpre[j]);
+      if (f_first + kAttnWarps * j < n_in)
+        attn_load_key<D>(kc, vc, jf0 + f_first + kAttnWarps * j, lane, kpre[j], vpre[j]);
     // old positions from the ring, kv_stage_keys per stage (K rows at 0, V rows at KPS * D)
     for (int st = 0; st < nst; ++st) {
       const int jj = a.j0 + st * KPS, nk = min(KPS, jend - jj);
@@ -848,7 +982,6 @@ constexpr uint32_t kTcIdesc = (1u << 4)                       // D: fp32
                               | ((uint32_t)(kTcN >> 3) << 17)   // N
                               | ((uint32_t)(kTcRows >> 4) << 24);  // M (A and B K-major: bits 15, 16 = 0)
 
-__device__ __forceinline__ float bf2f(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
 __device__ __forceinline__ void warp_argmax(float& v, int& idx) {
 #pragma unroll
@@ -1215,7 +1348,8 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
 }
 
 // ---------------------------------------------------------------------------------------
-template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM>
+// QKN: the model has QK-norm (its own instantiations, so the plain kernels keep their registers).
+template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM, bool QKN>
 __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBlockThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams P) {
   constexpr bool TC = BM > kMaxDecodeBatch;  // tensor-core projection tiles
@@ -1449,6 +1583,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
     if (kHoist && k + 1 < nk) t_next = P.tasks[qb + (k + 1) % nq];
     const uint64_t t_wait = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     uint32_t stall = 0;
+    if (QKN && t.kind == TK_ATTN) qk_norm_prefetch<HD>(P, t, st, lane);
     // wait for the scheduler to release task i (bounded, abort-aware, then uniform decision)
     {
       uint64_t t0 = 0;
@@ -1601,7 +1736,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       }
     } else if (t.kind == TK_ATTN) {
       notify = false;  // the last chunk to arrive notifies
-      if (!attention_task<HD, TC>(P, S, pp, ring, t, i, stall, st)) goto out;
+      if (!attention_task<HD, TC, QKN>(P, S, pp, ring, t, i, stall, st)) goto out;
     }
     if (P.trace && tid == 0) {
       uint64_t* rec = P.trace + (size_t)i * kTraceWords;
@@ -1639,38 +1774,51 @@ __host__ __device__ constexpr int stage_rows(int K) {
 // Batch width 1 streams W_down whole (K = ffn); batch width 4 streams it in K chunks of
 // kDownChunk columns, so the K = ffn class is the chunk's.
 __host__ __device__ constexpr int down_k(int F, int BM) { return BM == 1 ? F : (F < kDownChunk ? F : kDownChunk); }
-#define MK_VARIANT(H, F, D, BM) {seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, BM}
-#define MK_KERNEL(H, F, D, BM)                                                                                   \
+#define MK_VARIANT(H, F, D, BM, QK) \
+  {seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, BM, QK}
+#define MK_KERNEL(H, F, D, BM, QK)                                                                               \
   (const void*)decode_kernel<seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, \
-                             BM>
+                             BM, QK>
 static const Variant kVariants[] = {
-    MK_VARIANT(4096, 14336, 128, 1),  // Llama-3-8B shape
-    MK_VARIANT(4096, 11008, 128, 1),  // Chameleon-7B shape
-    MK_VARIANT(256, 768, 64, 1),      // tiny decoder
-    MK_VARIANT(4096, 4096, 128, 1),
-    MK_VARIANT(2048, 4096, 128, 1),
-    MK_VARIANT(256, 256, 64, 1),
-    MK_VARIANT(4096, 4096, 128, 4),   // hidden 4096, any ffn >= 4096 (Llama-3-8B, Chameleon-7B), 2..4 sequences
-    MK_VARIANT(256, 768, 64, 4),      // tiny decoder, 2..4 sequences
-    MK_VARIANT(2048, 4096, 128, 4),
-    MK_VARIANT(256, 256, 64, 4),
-    {0, 1, 0, 1, 128, kTcBatch},      // tensor-core projection tiles, 5..16 sequences, any hidden / ffn
-    {0, 1, 0, 1, 64, kTcBatch},
+    MK_VARIANT(4096, 14336, 128, 1, 0),  // Llama-3-8B shape
+    MK_VARIANT(4096, 11008, 128, 1, 0),  // Chameleon-7B shape
+    MK_VARIANT(256, 768, 64, 1, 0),      // tiny decoder
+    MK_VARIANT(4096, 4096, 128, 1, 0),
+    MK_VARIANT(2048, 4096, 128, 1, 0),
+    MK_VARIANT(256, 256, 64, 1, 0),
+    MK_VARIANT(4096, 4096, 128, 4, 0),   // hidden 4096, any ffn >= 4096 (Llama-3-8B, Chameleon-7B), 2..4 sequences
+    MK_VARIANT(256, 768, 64, 4, 0),      // tiny decoder, 2..4 sequences
+    MK_VARIANT(2048, 4096, 128, 4, 0),
+    MK_VARIANT(256, 256, 64, 4, 0),
+    {0, 1, 0, 1, 128, kTcBatch, 0},      // tensor-core projection tiles, 5..16 sequences, any hidden / ffn
+    {0, 1, 0, 1, 64, kTcBatch, 0},
+    // QK-norm models: Chameleon-7B shape and the tiny decoder, every batch width
+    MK_VARIANT(4096, 11008, 128, 1, 1),
+    MK_VARIANT(256, 768, 64, 1, 1),
+    MK_VARIANT(4096, 4096, 128, 4, 1),
+    MK_VARIANT(256, 768, 64, 4, 1),
+    {0, 1, 0, 1, 128, kTcBatch, 1},
+    {0, 1, 0, 1, 64, kTcBatch, 1},
 };
 static const void* kFns[] = {
-    MK_KERNEL(4096, 14336, 128, 1), MK_KERNEL(4096, 11008, 128, 1), MK_KERNEL(256, 768, 64, 1),
-    MK_KERNEL(4096, 4096, 128, 1),  MK_KERNEL(2048, 4096, 128, 1),  MK_KERNEL(256, 256, 64, 1),
-    MK_KERNEL(4096, 4096, 128, 4),  MK_KERNEL(256, 768, 64, 4),     MK_KERNEL(2048, 4096, 128, 4),
-    MK_KERNEL(256, 256, 64, 4),
-    (const void*)decode_kernel<1, 1, 1, 1, 128, kTcBatch>, (const void*)decode_kernel<1, 1, 1, 1, 64, kTcBatch>,
+    MK_KERNEL(4096, 14336, 128, 1, false), MK_KERNEL(4096, 11008, 128, 1, false), MK_KERNEL(256, 768, 64, 1, false),
+    MK_KERNEL(4096, 4096, 128, 1, false),  MK_KERNEL(2048, 4096, 128, 1, false),  MK_KERNEL(256, 256, 64, 1, false),
+    MK_KERNEL(4096, 4096, 128, 4, false),  MK_KERNEL(256, 768, 64, 4, false),     MK_KERNEL(2048, 4096, 128, 4, false),
+    MK_KERNEL(256, 256, 64, 4, false),
+    (const void*)decode_kernel<1, 1, 1, 1, 128, kTcBatch, false>,
+    (const void*)decode_kernel<1, 1, 1, 1, 64, kTcBatch, false>,
+    MK_KERNEL(4096, 11008, 128, 1, true),  MK_KERNEL(256, 768, 64, 1, true),
+    MK_KERNEL(4096, 4096, 128, 4, true),   MK_KERNEL(256, 768, 64, 4, true),
+    (const void*)decode_kernel<1, 1, 1, 1, 128, kTcBatch, true>,
+    (const void*)decode_kernel<1, 1, 1, 1, 64, kTcBatch, true>,
 };
 static_assert(sizeof(kVariants) / sizeof(kVariants[0]) == sizeof(kFns) / sizeof(kFns[0]), "variant table");
 
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm) {
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn) {
   for (int i = 0; i < (int)(sizeof(kVariants) / sizeof(kVariants[0])); ++i) {
     const Variant& v = kVariants[i];
     if (v.nseg_h == nseg_h && v.rps_h == rps_h && v.nseg_f == nseg_f && v.rps_f == rps_f && v.head_dim == head_dim &&
-        v.bm == bm)
+        v.bm == bm && v.qkn == qkn)
       return i;
   }
   return -1;

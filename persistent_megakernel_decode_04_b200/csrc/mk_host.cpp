@@ -65,7 +65,7 @@ struct mk_ctx {
   // workspace layout
   size_t ws_tasks = 0, ws_qbegin = 0, ws_evcount = 0, ws_ev = 0, ws_acnt = 0, ws_err = 0, ws_loff = 0, ws_rope = 0,
          ws_xin = 0, ws_xmid = 0, ws_q = 0, ws_o = 0, ws_h = 0, ws_part = 0, ws_lmval = 0, ws_lmidx = 0,
-         ws_pf = 0, ws_tpart = 0, ws_tcnt = 0, ws_bytes = 0;
+         ws_pf = 0, ws_tpart = 0, ws_tcnt = 0, ws_kraw = 0, ws_bytes = 0;
   size_t ev_bytes = 0, acnt_bytes = 0, tcnt_bytes = 0;
   int pf_rows = 0;
   size_t kv_bytes = 0;
@@ -672,6 +672,8 @@ void layout(mk_ctx* c) {
     o = align256(o + (uint64_t)H * 2);
     lo.mlp_norm = o;
     o = align256(o + (uint64_t)H * 2);
+    lo.qkn = o;  // QK-norm gains and biases (0 bytes without QK-norm)
+    o = align256(o + (f.qk_norm ? (uint64_t)2 * (nq + nkv) * D * 2 : 0));
   }
   c->off_lm = o;
   o = align256(o + mat(TK_LMHEAD, f.vocab, H));
@@ -701,6 +703,7 @@ void layout(mk_ctx* c) {
   c->ws_xin = take((size_t)(L + 1) * B * H * 4);
   c->ws_xmid = take((size_t)L * B * H * 4);
   c->ws_q = take((size_t)L * B * nq * D * 4);
+  c->ws_kraw = take(f.qk_norm ? (size_t)L * B * nkv * D * 4 : 4);
   c->ws_o = take((size_t)L * B * nq * D * 4);
   c->ws_h = take((size_t)L * B * F * 4);
   c->ws_part = take((size_t)L * B * nq * c->nch * (D + 2) * 4);
@@ -738,6 +741,7 @@ int check_config(const mk_config* f, std::string* why) {
   if (f->max_batch < 1 || f->max_batch > MK_MAX_BATCH) return bad("max_batch out of range");
   if (f->max_seq < 1 || f->max_seq > (1 << 20)) return bad("max_seq out of range");
   if (f->tie_embeddings != 0) return bad("tied embeddings are not supported");
+  if (f->qk_norm != 0 && f->qk_norm != 1) return bad("qk_norm must be 0 or 1");
   if (f->hidden > 4 * kSegElems || f->ffn > 8 * kSegElems) return bad("hidden or ffn too large");
   return MK_OK;
 }
@@ -888,9 +892,9 @@ int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
       base += c->tc_tiles[k];
     }
     c->n_tile_ids = base;
-    c->variant = find_decode_variant(0, 1, 0, 1, f.head_dim, kTcBatch);
+    c->variant = find_decode_variant(0, 1, 0, 1, f.head_dim, kTcBatch, f.qk_norm);
   } else {
-    c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm);
+    c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm, f.qk_norm);
   }
   c->sm_weights.assign(c->n_sms, 1.0);
   rc = build_graph(c);
@@ -924,6 +928,13 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
     if (!w->attn_norm[l] || !w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->mlp_norm[l] || !w->wg[l] ||
         !w->wu[l] || !w->wd[l])
       return fail(c, MK_ERR_INVALID_ARG, "a per-layer weight pointer is NULL");
+  if (f.qk_norm) {
+    if (!w->q_norm_w || !w->q_norm_b || !w->k_norm_w || !w->k_norm_b)
+      return fail(c, MK_ERR_INVALID_ARG, "a QK-norm model needs q_norm_w, q_norm_b, k_norm_w and k_norm_b");
+    for (int l = 0; l < L; ++l)
+      if (!w->q_norm_w[l] || !w->q_norm_b[l] || !w->k_norm_w[l] || !w->k_norm_b[l])
+        return fail(c, MK_ERR_INVALID_ARG, "a per-layer QK-norm pointer is NULL");
+  }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (!cuda_ok(c, cudaSetDevice(c->device), "cudaSetDevice")) return MK_ERR_CUDA;
   uint8_t* A = static_cast<uint8_t*>(weight_arena);
@@ -967,6 +978,12 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
       std::memcpy(&gu[(size_t)(2 * i + 1) * H], w->wu[l] + (size_t)i * H, (size_t)H * 2);
     }
     const LayerOff& lo = c->loff[l];
+    if (f.qk_norm) {
+      const size_t qb = (size_t)nq * D * 2, kb = (size_t)nkv * D * 2;
+      if (!put(lo.qkn, w->q_norm_w[l], qb) || !put(lo.qkn + qb, w->q_norm_b[l], qb) ||
+          !put(lo.qkn + 2 * qb, w->k_norm_w[l], kb) || !put(lo.qkn + 2 * qb + kb, w->k_norm_b[l], kb))
+        return MK_ERR_CUDA;
+    }
     if (c->tc) {
       if (!put_blocks(lo.qkv, qkv.data(), H, c->rows_qkv, H) || !put_blocks(lo.o, w->wo[l], nq * D, H, nq * D) ||
           !put_blocks(lo.gu, gu.data(), H, c->rows_gu, H) || !put_blocks(lo.d, w->wd[l], F, H, F) ||
@@ -1061,6 +1078,7 @@ int mk_prefill(mk_ctx* c, const int32_t* tokens, int B, int T, void* kv_cache, f
   p.kdc = c->kdc;
   p.ndc = c->ndc;
   p.blocked = c->tc ? 1 : 0;
+  p.qk_norm = f.qk_norm;
   std::string err;
   int rc = run_prefill(p, tokens, B, T, last_logits, reinterpret_cast<cudaStream_t>(stream), &err);
   if (rc) return fail(c, rc, err);
@@ -1119,6 +1137,8 @@ int decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache,
   P.x_in = reinterpret_cast<float*>(W + c->ws_xin);
   P.x_mid = reinterpret_cast<float*>(W + c->ws_xmid);
   P.qbuf = reinterpret_cast<float*>(W + c->ws_q);
+  P.kraw = reinterpret_cast<float*>(W + c->ws_kraw);
+  P.qk_norm = f.qk_norm;
   P.obuf = reinterpret_cast<float*>(W + c->ws_o);
   P.hbuf = reinterpret_cast<float*>(W + c->ws_h);
   P.part = reinterpret_cast<float*>(W + c->ws_part);

@@ -89,6 +89,7 @@ static_assert(sizeof(Task) == 40, "Task layout");
 struct LayerOff {
   uint64_t qkv, o, gu, d;   // packed matrices
   uint64_t attn_norm, mlp_norm;
+  uint64_t qkn;             // QK-norm: q gain [nq*D], q bias [nq*D], k gain [nkv*D], k bias [nkv*D]
 };
 
 struct DecodeParams {
@@ -105,7 +106,8 @@ struct DecodeParams {
   uint16_t* kv;               // [L][2][max_batch][nkv][max_seq][D]
   float* x_in;                // [L+1][B][H]
   float* x_mid;               // [L][B][H]
-  float* qbuf;                // [L][B][nq*D]
+  float* qbuf;                // [L][B][nq*D] (QK-norm: before the norm and RoPE)
+  float* kraw;                // QK-norm: [L][B][nkv*D] k before the norm and RoPE
   float* obuf;                // [L][B][nq*D]
   float* hbuf;                // [L][B][F]
   float* part;                // [L][B][nq][nch][D+2]
@@ -129,6 +131,7 @@ struct DecodeParams {
   uint32_t* tcnt;             // tensor-core tile arrival counters
   int n_steps;                // greedy decode steps in this launch (step s: epoch + s, pos + s)
   uint32_t ev_tok;            // event: the step's tokens are picked (the next step's embedding waits)
+  int qk_norm;                // 1: LayerNorm of every q and k head before RoPE, in the attention task
 };
 constexpr uint64_t kStallPrefetchNs = 1000;    // producer blocked this long: prefetch ahead into L2
 constexpr uint64_t kStallPrefetchGapNs = 100;   // then one more stage per this interval
@@ -154,9 +157,9 @@ TensorMapEncodeFn get_tensor_map_encoder();
 
 // Kernel variants: one instantiation per (segments, rows per stage) of the two K sizes.
 struct Variant {
-  int nseg_h, rps_h, nseg_f, rps_f, head_dim, bm;
+  int nseg_h, rps_h, nseg_f, rps_f, head_dim, bm, qkn;
 };
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm);
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn);
 const void* decode_kernel_ptr(int variant);
 size_t decode_smem_bytes(int variant);
 int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t stream, std::string* err);
@@ -185,6 +188,7 @@ struct PrefillParams {
   float eps, attn_scale;
   int kdc, ndc;  // W_down stored in ndc chunk-major K chunks of kdc columns
   int blocked;   // 1: projections in the tensor-core block layout (kTcRows x kTcUnitK blocks)
+  int qk_norm;   // 1: LayerNorm of every q and k head before RoPE
 };
 int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, float* last_logits,
                 cudaStream_t stream, std::string* err);

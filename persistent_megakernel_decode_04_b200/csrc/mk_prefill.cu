@@ -116,6 +116,34 @@ __global__ void __launch_bounds__(256) gemm(const float* __restrict__ A, const u
   }
 }
 
+// QK-norm (Mirage article, "Case 4.1: Attention with Query-Key Normalization"): LayerNorm of
+// every q and k head of a packed QKV output row, in place, before RoPE.  One block per row, one
+// warp per head; a head's D values sit at packed positions 2i (dim i) and 2i + 1 (dim i + D/2).
+// Gains and biases: q gain [nq*D], q bias [nq*D], k gain [nkv*D], k bias [nkv*D].
+__global__ void qk_norm(float* Yq, const uint16_t* nb, int nq, int nkv, int D, float eps) {
+  const int G = nq / nkv, rpg = (G + 2) * D, NQKV = (nq + 2 * nkv) * D, half = D / 2;
+  const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  float* y = Yq + (size_t)blockIdx.x * NQKV;
+  for (int h = threadIdx.x >> 5; h < nq + nkv; h += nw) {  // heads 0..nq-1: q; then k
+    const int grp = h < nq ? h / G : h - nq;
+    float* v = y + (size_t)grp * rpg + (h < nq ? (h % G) * D : G * D);
+    const uint16_t* g = nb + (h < nq ? (size_t)h * D : (size_t)2 * nq * D + (size_t)(h - nq) * D);
+    const uint16_t* b = g + (h < nq ? (size_t)nq * D : (size_t)nkv * D);
+    float sum = 0.f;
+    for (int e = lane; e < D; e += 32) sum += v[e];
+    for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    const float mean = sum / D;
+    float sq = 0.f;
+    for (int e = lane; e < D; e += 32) sq += (v[e] - mean) * (v[e] - mean);
+    for (int off = 16; off >= 1; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    const float r = 1.0f / sqrtf(sq / D + eps);
+    for (int e = lane; e < D; e += 32) {
+      const int dim = (e & 1) ? (e >> 1) + half : (e >> 1);
+      v[e] = (v[e] - mean) * r * bf(g[dim]) + bf(b[dim]);
+    }
+  }
+}
+
 // Packed QKV output row -> RoPE'd q (natural head/dim order) and bf16 K/V cache entries.
 __global__ void qkv_post(const float* Yq, int n, int ct, int t0, const float2* rope, float* Q, uint16_t* kv,
                          int layer, int nq, int nkv, int D, int max_seq, int max_batch) {
@@ -258,6 +286,8 @@ int run_prefill(const PrefillParams& p, const int32_t* tokens, int B, int T, flo
       const uint16_t* mn = reinterpret_cast<const uint16_t*>(p.arena + lo.mlp_norm);
       pf::rmsnorm<<<n, 256, 0, s>>>(p.X, an, p.XN, H, p.eps, 1, 0);
       gemm(p.XN, reinterpret_cast<const uint16_t*>(p.arena + lo.qkv), p.Y, n, NQKV, H, NQKV, s, p.blocked);
+      if (p.qk_norm)
+        pf::qk_norm<<<n, 256, 0, s>>>(p.Y, reinterpret_cast<const uint16_t*>(p.arena + lo.qkn), nq, nkv, D, p.eps);
       pf::qkv_post<<<n, 256, 0, s>>>(p.Y, n, ct, t0, p.rope, p.Q, p.kv, l, nq, nkv, D, p.max_seq, p.max_batch);
       const size_t smem = (size_t)(t0 + ct) * sizeof(float);
       if (smem > 48 * 1024) cudaFuncSetAttribute(pf::attention, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

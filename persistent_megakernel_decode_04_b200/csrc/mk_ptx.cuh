@@ -94,6 +94,11 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// Bring the line holding a global address into L1 (and L2).
+__device__ __forceinline__ void prefetch_l1(const void* src) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(src) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }

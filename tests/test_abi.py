@@ -34,11 +34,34 @@ def _cfg(**kw):
 
 
 @pytest.mark.parametrize("field,value", [("head_dim", 96), ("hidden", 250), ("n_kv_heads", 3), ("max_batch", 0),
-                                         ("max_batch", 17), ("max_seq", 0), ("rms_eps", 0.0), ("vocab", 1)])
+                                         ("max_batch", 17), ("max_seq", 0), ("rms_eps", 0.0), ("vocab", 1),
+                                         ("qk_norm", 2)])
 def test_bad_configs_are_rejected(field, value):
     with pytest.raises(mk.MkError) as e:
         mk.mk_build_taskgraph(_cfg(**{field: value}).c(), -1)
     assert e.value.code == mk.MK_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("max_batch", [1, 4, 16])
+def test_qk_norm_config_sizes(max_batch):
+    # QK-norm adds the per-layer gains and biases to the arena (q and k heads, gain + bias, bf16)
+    # and a raw-key buffer [layer][batch][n_kv_heads*head_dim] fp32 to the workspace
+    s = mi.TINY_QK
+    sizes = []
+    for qk in (False, True):
+        c = mk.Config.from_shape(s, max_batch, 64)
+        c.qk_norm = qk
+        ctx = mk.mk_build_taskgraph(c.c(), -1)
+        try:
+            sizes.append((mk.mk_weight_arena_bytes(ctx), mk.mk_workspace_bytes(ctx), mk.mk_kv_cache_bytes(ctx)))
+        finally:
+            mk.mk_destroy(ctx)
+    (a0, w0, k0), (a1, w1, k1) = sizes
+    per_layer = 2 * (s.n_q_heads + s.n_kv_heads) * s.head_dim * 2
+    assert a1 - a0 >= s.n_layers * per_layer and a1 - a0 < s.n_layers * (per_layer + 256)
+    assert w1 - w0 >= s.n_layers * max_batch * s.n_kv_heads * s.head_dim * 4 - 256
+    assert k1 == k0
+    assert mk.Config.from_shape(s, 1, 8).qk_norm and not mk.Config.from_shape(mi.TINY, 1, 8).qk_norm
 
 
 def test_null_context_calls_fail_cleanly():
