@@ -43,11 +43,15 @@ struct DSmem {
   float ssw[kWorkerWarps][kMaxDecodeBatch];  // per-warp sums of x^2 per sequence
   float am[kAttnWarps][4];
   float al[kAttnWarps][4];
-  float mm[4 * kMaxChunks], ll[4 * kMaxChunks], ww[4 * kMaxChunks];  // split-KV merge
+  union {
+    struct {
+      float mm[4 * kMaxChunks], ll[4 * kMaxChunks];  // split-KV merge of the last arriver (after the key loop)
+    } mg;
+    float qn[4 * 128];  // QK-norm: an attention task's normed, rotated q heads (read before its key loop)
+  };
   float lmv[kWorkerWarps];
   int lmi[kWorkerWarps];
   float tss[2][kTcBatch];    // tensor-core tasks (by parity): per-sequence sum of x^2 over the K range
-  float qn[4 * 128];         // QK-norm: the normed, rotated q heads of an attention task's group
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t bop_full[2];      // tensor-core operand buffer staged (one arrival per worker warp)
@@ -857,13 +861,13 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
         for (int e = tid; e < G * nch_eff; e += kWorkerThreads) {
           const int h = e / nch_eff, cc = e % nch_eff;
           const float* pc = part_base + ((size_t)(g * G + h) * P.nch + cc) * (D + 2);
-          S.mm[e] = __ldcg(pc);
-          S.ll[e] = __ldcg(pc + 1);
+          S.mg.mm[e] = __ldcg(pc);
+          S.mg.ll[e] = __ldcg(pc + 1);
         }
         worker_bar();
       }
-      const float* mm0 = S.mm + (has0 ? h0 : 0) * nch_eff;
-      const float* mm1 = S.mm + (has1 ? h1 : 0) * nch_eff;
+      const float* mm0 = S.mg.mm + (has0 ? h0 : 0) * nch_eff;
+      const float* mm1 = S.mg.mm + (has1 ? h1 : 0) * nch_eff;
       float M0 = -INFINITY, M1 = -INFINITY;
       for (int cc = 0; cc < nch_eff; ++cc) {
         M0 = fmaxf(M0, mm0[cc]);
@@ -876,9 +880,9 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
           const float w0 = (mm0[cc] == -INFINITY) ? 0.f : __expf(mm0[cc] - M0);
           const float w1 = (mm1[cc] == -INFINITY) ? 0.f : __expf(mm1[cc] - M1);
           num0 = fmaf(w0, v0[k], num0);
-          den0 = fmaf(w0, S.ll[(has0 ? h0 : 0) * nch_eff + cc], den0);
+          den0 = fmaf(w0, S.mg.ll[(has0 ? h0 : 0) * nch_eff + cc], den0);
           num1 = fmaf(w1, v1[k], num1);
-          den1 = fmaf(w1, S.ll[(has1 ? h1 : 0) * nch_eff + cc], den1);
+          den1 = fmaf(w1, S.mg.ll[(has1 ? h1 : 0) * nch_eff + cc], den1);
         }
       }
     }
