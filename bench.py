@@ -79,6 +79,10 @@ def parse():
     p.add_argument("--no-calibrate", action="store_true",
                    help="keep equal rows per SM instead of the schedule calibrated during warm-up")
     p.add_argument("--workload", default="llama8b", choices=sorted(WORKLOADS))
+    p.add_argument("--dispatch", default="static", choices=["static", "claim"],
+                   help="scheduling variant: fixed per-SM queues (default), or projection tasks claimed "
+                        "at run time from per-op pools (batch-1 kernel only)")
+    p.add_argument("--tasks-per-sm", type=int, default=2, help="pool tasks per SM and projection (--dispatch claim)")
     p.add_argument("--layers", type=int, default=0,
                    help="truncate the decoder to this many layers (profiling captures of a small case); "
                         "0 = the full 32-layer workload")
@@ -397,7 +401,9 @@ def run_mk(args, rank, world, local):
         tok = torch.from_numpy(mi.prompt(0, 0, B, shape.vocab).astype(np.int32)).to(dev)
     warm = args.warmup
     calibrated = False
-    if not args.no_calibrate and warm >= 6:
+    if args.dispatch == "claim":  # pools are cut in equal shares: no per-SM calibration
+        m.set_dispatch(mk.MK_DISPATCH_CLAIM, args.tasks_per_sm)
+    elif not args.no_calibrate and warm >= 6:
         # measure per-SM streaming speed on warm-up steps and re-partition rows (3 rounds x 2 steps)
         m.calibrate(tok, steps=2, rounds=3)
         warm -= 6
@@ -469,7 +475,8 @@ def run_mk(args, rank, world, local):
         mean_ms = float(step_ms.mean())
         peak, peak_kind = measured_peaks()
         achieved = alg / (mean_ms * 1e-3) / 1e9
-        traffic, traffic_note = profiled_traffic(alg) if args.workload == "llama8b" else (None, "no ncu summary")
+        traffic, traffic_note = (profiled_traffic(alg) if args.workload == "llama8b" and args.dispatch == "static"
+                                 else (None, "no ncu summary"))
         # whole job: slowest rank's time over all ranks' steps (replicas decode concurrently)
         value = max_ms / (args.steps * world)
         out = {
@@ -482,7 +489,9 @@ def run_mk(args, rank, world, local):
                        "prompt_len": PROMPT_LEN if ctx0 == 0 else None, "cached_positions": ctx0 or None,
                        "decode_positions": [pos0, pos0 + args.steps - 1], "batch_per_gpu": B,
                        "global_batch": world * B, "parallelism": "replicas", "weights": "bf16",
-                       "schedule": "calibrated per-SM rows" if calibrated else "equal rows per SM",
+                       "schedule": (f"run-time claims from per-op pools, {args.tasks_per_sm} tasks per SM"
+                                    if args.dispatch == "claim" else
+                                    "calibrated per-SM rows" if calibrated else "equal rows per SM"),
                        "l2": "inputs larger than L2 (15 GB of weights streamed per step)"},
             "ms_per_step_p50": float(np.median(step_ms)), "tokens_per_s": 1e3 / (max_ms / args.steps) * world * B,
             "hbm_gbs": achieved, "hbm_frac_of_measured": achieved / peak, "hbm_frac_of_8tbs": achieved / NOMINAL_HBM_GBS,

@@ -180,6 +180,20 @@ int mk_set_sm_weights(mk_ctx* ctx, const float* weights, int n, void* stream);
  * op_kind. */
 int mk_set_op_sm_weights(mk_ctx* ctx, int op_kind, const float* weights, int n, void* stream);
 
+/* Scheduling variant (MPK's run-time dispatch vs the static schedule of "Ada-MK: Adaptive
+ * MegaKernel Optimization via Automated DAG-based Search for LLM Inference", section 2).
+ * MK_DISPATCH_STATIC (default): every task has a fixed SM and queue position, chosen at
+ * lowering time.  MK_DISPATCH_CLAIM: every projection of every layer becomes a pool of
+ * tasks_per_sm * n_sms equal tasks (1..4); each SM's queue holds one entry per pool, where the
+ * SM claims tasks from the pool's counter (one atomic add per claim) until it is empty, so
+ * faster SMs take more; attention, embedding and LM-head tasks stay static.  The graph is
+ * validated with the pools' tasks dealt round-robin.  Only the batch-1 kernel of the Llama-3-8B
+ * and tiny shapes has a run-time-claim instantiation: MK_ERR_UNSUPPORTED otherwise.  Rebuilds
+ * and re-uploads the graph (synchronises `stream` first if weights are loaded). */
+#define MK_DISPATCH_STATIC 0
+#define MK_DISPATCH_CLAIM 1
+int mk_set_dispatch(mk_ctx* ctx, int mode, int tasks_per_sm, void* stream);
+
 /* Weight prefetch depth: besides the shared-memory ring (6 stages of 32 KB per SM), an SM's
  * producer that has been blocked on a full ring for over a microsecond (its workers wait for a
  * dependency, e.g. during attention) prefetches up to `stages` further weight stages of its

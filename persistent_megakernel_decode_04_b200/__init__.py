@@ -33,8 +33,10 @@ MK_ERR_NOT_RESIDENT = -4
 MK_ERR_STATE = -5
 MK_ERR_UNSUPPORTED = -6
 MK_MAX_BATCH = 16
+MK_DISPATCH_STATIC = 0
+MK_DISPATCH_CLAIM = 1
 
-TASK_KINDS = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead"}
+TASK_KINDS = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead", 8: "pool"}
 
 
 class MkError(RuntimeError):
@@ -83,6 +85,7 @@ _SIGS = {
     "mk_set_wait_timeout_ns": ([_vp, _u64], _i32),
     "mk_debug_drop_notify": ([_vp, _i32, _i32], _i32),
     "mk_set_l2_prefetch": ([_vp, _i32], _i32),
+    "mk_set_dispatch": ([_vp, _i32, _i32, _vp], _i32),
     "mk_set_sm_weights": ([_vp, _vp, _i32, _vp], _i32),
     "mk_set_op_sm_weights": ([_vp, _i32, _vp, _i32, _vp], _i32),
     "mk_set_trace": ([_vp, _vp], _i32),
@@ -237,6 +240,12 @@ def mk_set_op_sm_weights(ctx, op_kind: int, weights, stream=None):
 
 def mk_set_l2_prefetch(ctx, stages: int):
     _check(_lib.mk_set_l2_prefetch(ctx, int(stages)), ctx)
+
+
+def mk_set_dispatch(ctx, mode: int, tasks_per_sm: int = 2, stream=None):
+    """MK_DISPATCH_STATIC (fixed per-SM queues) or MK_DISPATCH_CLAIM (projection tasks claimed at
+    run time from per-op pools of tasks_per_sm * n_sms tasks)."""
+    _check(_lib.mk_set_dispatch(ctx, int(mode), int(tasks_per_sm), _stream(stream)), ctx)
 
 
 def mk_set_trace(ctx, device_buffer):
@@ -417,6 +426,10 @@ class Megakernel:
 
     def info(self) -> dict:
         return mk_get_graph_info(self.ctx)
+
+    def set_dispatch(self, mode: int, tasks_per_sm: int = 2):
+        """Scheduling variant: MK_DISPATCH_STATIC or MK_DISPATCH_CLAIM (see mk_set_dispatch)."""
+        mk_set_dispatch(self.ctx, mode, tasks_per_sm, self.stream)
 
     def close(self):
         if getattr(self, "ctx", None):

@@ -64,6 +64,11 @@ struct DSmem {
   uint32_t cabort;           // worker-role abort: written before, read after a worker barrier
   volatile uint32_t abort;   // any role gave up: stop waiting
   uint32_t flag;             // worker broadcast (last-arriver decisions)
+  // run-time claims: task FIFO from the producer (which claims) to the scheduler and workers
+  uint32_t dq_id[kDynQ];
+  uint16_t dq_st[kDynQ];
+  uint32_t dq_n;             // entries pushed
+  uint32_t wdone;            // entries the workers finished (their slots can be reused)
 };
 
 __host__ __device__ constexpr int ring_stages(bool tc) { return tc ? kTcStages : kStages; }
@@ -919,8 +924,16 @@ __device__ __forceinline__ void block_argmax(DSmem& S, float& v, int& idx) {
 
 // The token pick of step st: greedy tokens to next_tokens[st][b]; then the event the next
 // step's embedding waits for.
-__device__ __forceinline__ void announce_tokens(const DecodeParams& P, DSmem& S) {
+// The step's tokens are picked.  With run-time claims this also zeroes the claim counters of
+// the step two ahead (every SM finished its claims of two steps back: each ends its step with
+// a static LM-head task, and this is the step's last LM-head task), published by the release.
+__device__ __forceinline__ void announce_tokens(const DecodeParams& P, DSmem& S, int st) {
   worker_bar();
+  if (P.dyn) {
+    uint32_t* row = P.pcnt + (size_t)((P.epoch + (uint32_t)st + 2u) & 3u) * P.n_pools;
+    for (int p = threadIdx.x; p < P.n_pools; p += kWorkerThreads) row[p] = 0u;
+    worker_bar();
+  }
   if (threadIdx.x == 0) red_release_gpu_add(&P.ev[P.ev_tok], 1u);
 }
 
@@ -960,7 +973,7 @@ __device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, cons
         worker_bar();
       }
     }
-    announce_tokens(P, S);
+    announce_tokens(P, S, st);
   }
 }
 
@@ -1319,7 +1332,7 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
           }
         }
       }
-      announce_tokens(P, S);
+      announce_tokens(P, S, st);
     }
     return true;
   }
@@ -1353,7 +1366,8 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
 
 // ---------------------------------------------------------------------------------------
 // QKN: the model has QK-norm (its own instantiations, so the plain kernels keep their registers).
-template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM, bool QKN>
+// DYN: run-time claims (projection tasks taken from per-op pools; TK_POOL queue entries).
+template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM, bool QKN, bool DYN>
 __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBlockThreads, 1)
     decode_kernel(const __grid_constant__ DecodeParams P) {
   constexpr bool TC = BM > kMaxDecodeBatch;  // tensor-core projection tiles
@@ -1379,6 +1393,8 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       mbar_init(&S.acc_free[b], 4);
     }
     S.ready = 0;
+    S.dq_n = 0;
+    S.wdone = 0;
     S.cabort = 0;
     S.abort = 0;
     S.flag = 0;
@@ -1436,6 +1452,77 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
     Pipe pp{0, 0, NST};
     int issued = 0;
     bool ok = true;
+    // run-time claims: hand task `id` of step st to the scheduler and workers (FIFO entry),
+    // after the workers freed its slot (bounded wait)
+    uint32_t dq_count = 0;
+    auto dyn_push = [&](uint32_t id, int st) -> bool {
+      uint64_t t0 = 0;
+      for (uint32_t n = 1;; ++n) {
+        if (dq_count - ld_acquire_cta_shared(&S.wdone) < (uint32_t)kDynQ) break;
+        if ((n & 63u) == 0) {
+          if (S.abort) return false;
+          const uint64_t now = globaltimer_ns();
+          if (t0 == 0) t0 = now;
+          else if (now - t0 > P.timeout_ns) {
+            raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, id);
+            return false;
+          }
+        }
+      }
+      S.dq_id[dq_count % kDynQ] = id;
+      S.dq_st[dq_count % kDynQ] = (uint16_t)st;
+      st_release_cta_shared(&S.dq_n, ++dq_count);
+      return true;
+    };
+    // a projection task's weight rows through the ring (i: its task index, for the trace)
+    auto stream_gemv = [&](const Task& t, uint32_t i) -> bool {
+      uint64_t off;
+      uint32_t rb;
+      gemv_source<TC>(P, t, &off, &rb);
+      const int rps = TC ? 1 : (t.kind == TK_DOWN) ? RPS_F : RPS_H;
+      const uint8_t* src = P.arena + off + (uint64_t)t.row0 * rb;
+      uint64_t blocked = 0, first = 0;
+      for (uint32_t r0 = 0; r0 < t.nrows; r0 += (uint32_t)rps) {
+        const uint32_t nr = min((uint32_t)rps, t.nrows - r0);
+        const uint64_t tw = (P.trace || P.l2_ahead > 0) ? globaltimer_ns() : 0;
+        if (P.l2_ahead > 0 && !mbar_test_now(&S.empty[pp.stage], pp.phase ^ 1u)) {
+          // blocked: after kStallPrefetchNs, prefetch while still blocked
+          uint64_t t0 = tw;
+          for (uint32_t n = 1;; ++n) {
+            if (mbar_test(&S.empty[pp.stage], pp.phase ^ 1u)) break;
+            const uint64_t now = globaltimer_ns();
+            if (now - t0 > kStallPrefetchNs && la_lead < P.l2_ahead && la_advance(true)) {
+              ++la_lead;
+              t0 = now - kStallPrefetchNs + kStallPrefetchGapNs;  // next prefetch after a short gap
+            }
+            if ((n & 127u) == 0 && (S.abort || now - tw > P.timeout_ns)) break;
+          }
+        }
+        if (!wait_bar(&S.empty[pp.stage], pp.phase ^ 1u, P.timeout_ns, &S)) {
+          if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, i);
+          return false;
+        }
+        if (P.trace) {
+          const uint64_t now = globaltimer_ns();
+          blocked += now - tw;
+          if (r0 == 0) first = now;
+        }
+        mbar_arrive_expect_tx(&S.full[pp.stage], nr * rb);
+        bulk_g2s(ring + (size_t)pp.stage * kSlotBytes, src + (uint64_t)r0 * rb, nr * rb, &S.full[pp.stage], pol);
+        ++issued;
+        // the lookahead cursor stays at or in front of the next ring stage
+        if (P.l2_ahead > 0) {
+          if (la_lead > 0) --la_lead;
+          else la_advance(false);
+        }
+        pp.advance();
+      }
+      if (P.trace) {
+        P.trace[(size_t)i * kTraceWords + 4] = blocked;
+        P.trace[(size_t)i * kTraceWords + 5] = first;
+      }
+      return true;
+    };
     for (int st = 0; st < P.n_steps && ok; ++st) {
     if (st > 0) {  // the lookahead restarts with the step's queue
       la_task = qb;
@@ -1443,8 +1530,56 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       la_lead = 0;
       la_t = P.tasks[qb < qe ? qb : 0];
     }
+    bool gated = false;
     for (uint32_t i = qb; i < qe && ok; ++i) {
       const Task t = P.tasks[i];
+      if constexpr (DYN) {
+        if (t.kind == TK_POOL) {
+          // this step's claim counters were zeroed by the token pick of the step two back
+          if (!gated && st >= 2) {
+            const uint32_t target = P.epoch + (uint32_t)st - 2u;
+            uint64_t t0 = 0;
+            for (uint32_t n = 1;; ++n) {
+              if ((int32_t)(ld_acquire_gpu(&P.ev[P.ev_tok]) - target) >= 0) break;
+              if ((n & 63u) == 0) {
+                if (S.abort || *(volatile uint32_t*)&P.err[ERR_ABORT]) {
+                  S.abort = 1u;
+                  ok = false;
+                  break;
+                }
+                const uint64_t now = globaltimer_ns();
+                if (t0 == 0) t0 = now;
+                else if (now - t0 > P.timeout_ns) {
+                  raise_error(P, S, DEV_ERR_WAIT_EVENT, P.ev_tok, i);
+                  ok = false;
+                  break;
+                }
+              }
+            }
+            gated = true;
+            if (!ok) break;
+          }
+          // claim until the pool is empty; the next claim is in flight while a task streams
+          const uint2 pl = P.pools[t.index];
+          uint32_t* ctr = P.pcnt + (size_t)((P.epoch + (uint32_t)st) & 3u) * P.n_pools + t.index;
+          uint32_t c = atomicAdd(ctr, 1u);
+          while (ok && c < pl.y) {
+            const uint32_t id = pl.x + c;
+            if (!dyn_push(id, st)) {
+              ok = false;
+              break;
+            }
+            const uint32_t cn = atomicAdd(ctr, 1u);
+            ok = stream_gemv(P.tasks[id], id);
+            c = cn;
+          }
+          continue;
+        }
+        if (!dyn_push(i, st)) {
+          ok = false;
+          break;
+        }
+      }
       if (t.kind == TK_ATTN) {
         // old K/V rows of the chunk, kv_stage_keys<HD>() per stage: K rows, then V rows
         const AttnGeom a = attn_geom(P, t, st);
@@ -1470,54 +1605,10 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
         continue;
       }
       if (!is_gemv(t.kind)) continue;
-      uint64_t off;
-      uint32_t rb;
-      gemv_source<TC>(P, t, &off, &rb);
-      const int rps = TC ? 1 : (t.kind == TK_DOWN) ? RPS_F : RPS_H;
-      const uint8_t* src = P.arena + off + (uint64_t)t.row0 * rb;
-      uint64_t blocked = 0, first = 0;
-      for (uint32_t r0 = 0; r0 < t.nrows; r0 += (uint32_t)rps) {
-        const uint32_t nr = min((uint32_t)rps, t.nrows - r0);
-        const uint64_t tw = (P.trace || P.l2_ahead > 0) ? globaltimer_ns() : 0;
-        if (P.l2_ahead > 0 && !mbar_test_now(&S.empty[pp.stage], pp.phase ^ 1u)) {
-          // blocked: after kStallPrefetchNs, prefetch while still blocked
-          uint64_t t0 = tw;
-          for (uint32_t n = 1;; ++n) {
-            if (mbar_test(&S.empty[pp.stage], pp.phase ^ 1u)) break;
-            const uint64_t now = globaltimer_ns();
-            if (now - t0 > kStallPrefetchNs && la_lead < P.l2_ahead && la_advance(true)) {
-              ++la_lead;
-              t0 = now - kStallPrefetchNs + kStallPrefetchGapNs;  // next prefetch after a short gap
-            }
-            if ((n & 127u) == 0 && (S.abort || now - tw > P.timeout_ns)) break;
-          }
-        }
-        if (!wait_bar(&S.empty[pp.stage], pp.phase ^ 1u, P.timeout_ns, &S)) {
-          if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, i);
-          ok = false;
-          break;
-        }
-        if (P.trace) {
-          const uint64_t now = globaltimer_ns();
-          blocked += now - tw;
-          if (r0 == 0) first = now;
-        }
-        mbar_arrive_expect_tx(&S.full[pp.stage], nr * rb);
-        bulk_g2s(ring + (size_t)pp.stage * kSlotBytes, src + (uint64_t)r0 * rb, nr * rb, &S.full[pp.stage], pol);
-        ++issued;
-        // the lookahead cursor stays at or in front of the next ring stage
-        if (P.l2_ahead > 0) {
-          if (la_lead > 0) --la_lead;
-          else la_advance(false);
-        }
-        pp.advance();
-      }
-      if (P.trace) {
-        P.trace[(size_t)i * kTraceWords + 4] = blocked;
-        P.trace[(size_t)i * kTraceWords + 5] = first;
-      }
+      ok = stream_gemv(t, i);
     }
     }
+    if (DYN && ok) dyn_push(kDynEnd, 0);
     // leave no copy in flight: wait (bounded) for the last issued stages to land
     for (int k = 1; k <= (issued < NST ? issued : NST); ++k) {
       int s = pp.stage - k;
@@ -1535,8 +1626,36 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
     // ------------------------------- scheduler ------------------------------
     if (lane != 0) return;
     const uint32_t nq = qe - qb;
-    for (int st = 0; st < P.n_steps; ++st)
-    for (uint32_t i = qb; i < qe; ++i) {
+    // static queues: entry r is task qb + r % nq of step r / nq; run-time claims: the
+    // producer's FIFO entry r (bounded wait for it), up to the end marker
+    const uint32_t nr = DYN ? 0xffffffffu : nq * (uint32_t)P.n_steps;
+    for (uint32_t r = 0; r < nr; ++r) {
+      int st;
+      uint32_t i;
+      if constexpr (DYN) {
+        uint64_t t0 = 0;
+        for (uint32_t n = 1;; ++n) {
+          if (ld_acquire_cta_shared(&S.dq_n) > r) break;
+          if ((n & 63u) == 0) {
+            if (S.abort || *(volatile uint32_t*)&P.err[ERR_ABORT]) {
+              S.abort = 1u;
+              return;
+            }
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > P.timeout_ns) {
+              raise_error(P, S, DEV_ERR_WAIT_READY, blockIdx.x, r);
+              return;
+            }
+          }
+        }
+        i = S.dq_id[r % kDynQ];
+        if (i == kDynEnd) return;
+        st = S.dq_st[r % kDynQ];
+      } else {
+        st = (int)(r / nq);
+        i = qb + r % nq;
+      }
       const Task t = P.tasks[i];
       // a later step's embedding also waits for the previous step's token pick
       const int n_wait = t.n_wait + ((t.kind == TK_EMBED && st > 0) ? 1 : 0);
@@ -1561,7 +1680,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
           }
         }
       }
-      st_release_cta_shared(&S.ready, (uint32_t)st * nq + (i - qb) + 1u);
+      st_release_cta_shared(&S.ready, r + 1u);
     }
     return;
   }
@@ -1575,13 +1694,42 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
   // batch width 1: the next task's descriptor is loaded during the current task, so only the
   // activation loads remain after its release; wider kernels load it at the top of its own
   // iteration instead, which keeps 10 registers free across the GEMV
-  constexpr bool kHoist = (BM == 1);
+  constexpr bool kHoist = (BM == 1) && !DYN;
   Task t_next = P.tasks[qb < qe ? qb : 0];
-  // the queue once per step of the launch: k counts released tasks over all steps
-  const uint32_t nq = qe - qb, nk = nq * (uint32_t)P.n_steps;
+  // the queue once per step of the launch: k counts released tasks over all steps (run-time
+  // claims: the producer's FIFO entries, up to the end marker)
+  const uint32_t nq = qe - qb, nk = DYN ? 0xffffffffu : nq * (uint32_t)P.n_steps;
   for (uint32_t k = 0; k < nk; ++k) {
-    const int st = (int)(k / nq);
-    const uint32_t i = qb + k % nq;
+    int st;
+    uint32_t i;
+    if constexpr (DYN) {
+      // the producer's entry k (bounded, abort-aware, then uniform decision)
+      uint64_t t0 = 0;
+      for (uint32_t n = 1;; ++n) {
+        if (ld_acquire_cta_shared(&S.dq_n) > k) break;
+        if ((n & 63u) == 0) {
+          if (S.abort) {
+            S.cabort = 1u;
+            break;
+          }
+          const uint64_t now = globaltimer_ns();
+          if (t0 == 0) t0 = now;
+          else if (now - t0 > P.timeout_ns + 1000000000ull) {  // the producer reports first
+            raise_error(P, S, DEV_ERR_WAIT_READY, blockIdx.x, k);
+            S.cabort = 1u;
+            break;
+          }
+        }
+      }
+      worker_bar();
+      if (S.cabort) break;
+      i = S.dq_id[k % kDynQ];
+      if (i == kDynEnd) break;
+      st = S.dq_st[k % kDynQ];
+    } else {
+      st = (int)(k / nq);
+      i = qb + k % nq;
+    }
     const Task t = kHoist ? t_next : P.tasks[i];
     const LayerOff lo = P.loff[t.layer < P.L ? t.layer : 0];
     if (kHoist && k + 1 < nk) t_next = P.tasks[qb + (k + 1) % nq];
@@ -1756,6 +1904,10 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
           if ((int)t.notify[k] != P.drop_event) red_release_gpu_add(&P.ev[t.notify[k]], 1u);
       }
     }
+    if constexpr (DYN) {  // every worker read FIFO entry k: its slot can be reused
+      worker_bar();
+      if (tid == 0) st_release_cta_shared(&S.wdone, k + 1u);
+    }
   }
 out:
   if (TC) {  // every worker thread and the issuer warp (which drained its MMAs) meet here
@@ -1778,51 +1930,55 @@ __host__ __device__ constexpr int stage_rows(int K) {
 // Batch width 1 streams W_down whole (K = ffn); batch width 4 streams it in K chunks of
 // kDownChunk columns, so the K = ffn class is the chunk's.
 __host__ __device__ constexpr int down_k(int F, int BM) { return BM == 1 ? F : (F < kDownChunk ? F : kDownChunk); }
-#define MK_VARIANT(H, F, D, BM, QK) \
-  {seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, BM, QK}
-#define MK_KERNEL(H, F, D, BM, QK)                                                                               \
+#define MK_VARIANT(H, F, D, BM, QK, DY) \
+  {seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, BM, QK, DY}
+#define MK_KERNEL(H, F, D, BM, QK, DY)                                                                           \
   (const void*)decode_kernel<seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, \
-                             BM, QK>
+                             BM, QK, DY>
 static const Variant kVariants[] = {
-    MK_VARIANT(4096, 14336, 128, 1, 0),  // Llama-3-8B shape
-    MK_VARIANT(4096, 11008, 128, 1, 0),  // Chameleon-7B shape
-    MK_VARIANT(256, 768, 64, 1, 0),      // tiny decoder
-    MK_VARIANT(4096, 4096, 128, 1, 0),
-    MK_VARIANT(2048, 4096, 128, 1, 0),
-    MK_VARIANT(256, 256, 64, 1, 0),
-    MK_VARIANT(4096, 4096, 128, 4, 0),   // hidden 4096, any ffn >= 4096 (Llama-3-8B, Chameleon-7B), 2..4 sequences
-    MK_VARIANT(256, 768, 64, 4, 0),      // tiny decoder, 2..4 sequences
-    MK_VARIANT(2048, 4096, 128, 4, 0),
-    MK_VARIANT(256, 256, 64, 4, 0),
-    {0, 1, 0, 1, 128, kTcBatch, 0},      // tensor-core projection tiles, 5..16 sequences, any hidden / ffn
-    {0, 1, 0, 1, 64, kTcBatch, 0},
+    MK_VARIANT(4096, 14336, 128, 1, 0, 0),  // Llama-3-8B shape
+    MK_VARIANT(4096, 11008, 128, 1, 0, 0),  // Chameleon-7B shape
+    MK_VARIANT(256, 768, 64, 1, 0, 0),      // tiny decoder
+    MK_VARIANT(4096, 4096, 128, 1, 0, 0),
+    MK_VARIANT(2048, 4096, 128, 1, 0, 0),
+    MK_VARIANT(256, 256, 64, 1, 0, 0),
+    MK_VARIANT(4096, 4096, 128, 4, 0, 0),   // hidden 4096, any ffn >= 4096 (Llama-3-8B, Chameleon-7B), 2..4 sequences
+    MK_VARIANT(256, 768, 64, 4, 0, 0),      // tiny decoder, 2..4 sequences
+    MK_VARIANT(2048, 4096, 128, 4, 0, 0),
+    MK_VARIANT(256, 256, 64, 4, 0, 0),
+    {0, 1, 0, 1, 128, kTcBatch, 0, 0},      // tensor-core projection tiles, 5..16 sequences, any hidden / ffn
+    {0, 1, 0, 1, 64, kTcBatch, 0, 0},
     // QK-norm models: Chameleon-7B shape and the tiny decoder, every batch width
-    MK_VARIANT(4096, 11008, 128, 1, 1),
-    MK_VARIANT(256, 768, 64, 1, 1),
-    MK_VARIANT(4096, 4096, 128, 4, 1),
-    MK_VARIANT(256, 768, 64, 4, 1),
-    {0, 1, 0, 1, 128, kTcBatch, 1},
-    {0, 1, 0, 1, 64, kTcBatch, 1},
+    MK_VARIANT(4096, 11008, 128, 1, 1, 0),
+    MK_VARIANT(256, 768, 64, 1, 1, 0),
+    MK_VARIANT(4096, 4096, 128, 4, 1, 0),
+    MK_VARIANT(256, 768, 64, 4, 1, 0),
+    {0, 1, 0, 1, 128, kTcBatch, 1, 0},
+    {0, 1, 0, 1, 64, kTcBatch, 1, 0},
+    // run-time claims (scheduling variant): batch 1, Llama-3-8B shape and the tiny decoder
+    MK_VARIANT(4096, 14336, 128, 1, 0, 1),
+    MK_VARIANT(256, 768, 64, 1, 0, 1),
 };
 static const void* kFns[] = {
-    MK_KERNEL(4096, 14336, 128, 1, false), MK_KERNEL(4096, 11008, 128, 1, false), MK_KERNEL(256, 768, 64, 1, false),
-    MK_KERNEL(4096, 4096, 128, 1, false),  MK_KERNEL(2048, 4096, 128, 1, false),  MK_KERNEL(256, 256, 64, 1, false),
-    MK_KERNEL(4096, 4096, 128, 4, false),  MK_KERNEL(256, 768, 64, 4, false),     MK_KERNEL(2048, 4096, 128, 4, false),
-    MK_KERNEL(256, 256, 64, 4, false),
-    (const void*)decode_kernel<1, 1, 1, 1, 128, kTcBatch, false>,
-    (const void*)decode_kernel<1, 1, 1, 1, 64, kTcBatch, false>,
-    MK_KERNEL(4096, 11008, 128, 1, true),  MK_KERNEL(256, 768, 64, 1, true),
-    MK_KERNEL(4096, 4096, 128, 4, true),   MK_KERNEL(256, 768, 64, 4, true),
-    (const void*)decode_kernel<1, 1, 1, 1, 128, kTcBatch, true>,
-    (const void*)decode_kernel<1, 1, 1, 1, 64, kTcBatch, true>,
+    MK_KERNEL(4096, 14336, 128, 1, false, false), MK_KERNEL(4096, 11008, 128, 1, false, false), MK_KERNEL(256, 768, 64, 1, false, false),
+    MK_KERNEL(4096, 4096, 128, 1, false, false),  MK_KERNEL(2048, 4096, 128, 1, false, false),  MK_KERNEL(256, 256, 64, 1, false, false),
+    MK_KERNEL(4096, 4096, 128, 4, false, false),  MK_KERNEL(256, 768, 64, 4, false, false),     MK_KERNEL(2048, 4096, 128, 4, false, false),
+    MK_KERNEL(256, 256, 64, 4, false, false),
+    (const void*)decode_kernel<1, 1, 1, 1, 128, kTcBatch, false, false>,
+    (const void*)decode_kernel<1, 1, 1, 1, 64, kTcBatch, false, false>,
+    MK_KERNEL(4096, 11008, 128, 1, true, false),  MK_KERNEL(256, 768, 64, 1, true, false),
+    MK_KERNEL(4096, 4096, 128, 4, true, false),   MK_KERNEL(256, 768, 64, 4, true, false),
+    (const void*)decode_kernel<1, 1, 1, 1, 128, kTcBatch, true, false>,
+    (const void*)decode_kernel<1, 1, 1, 1, 64, kTcBatch, true, false>,
+    MK_KERNEL(4096, 14336, 128, 1, false, true), MK_KERNEL(256, 768, 64, 1, false, true),
 };
 static_assert(sizeof(kVariants) / sizeof(kVariants[0]) == sizeof(kFns) / sizeof(kFns[0]), "variant table");
 
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn) {
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn, int dyn) {
   for (int i = 0; i < (int)(sizeof(kVariants) / sizeof(kVariants[0])); ++i) {
     const Variant& v = kVariants[i];
     if (v.nseg_h == nseg_h && v.rps_h == rps_h && v.nseg_f == nseg_f && v.rps_f == rps_f && v.head_dim == head_dim &&
-        v.bm == bm && v.qkn == qkn)
+        v.bm == bm && v.qkn == qkn && v.dyn == dyn)
       return i;
   }
   return -1;

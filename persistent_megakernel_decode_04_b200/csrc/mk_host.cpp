@@ -65,8 +65,13 @@ struct mk_ctx {
   // workspace layout
   size_t ws_tasks = 0, ws_qbegin = 0, ws_evcount = 0, ws_ev = 0, ws_acnt = 0, ws_err = 0, ws_loff = 0, ws_rope = 0,
          ws_xin = 0, ws_xmid = 0, ws_q = 0, ws_o = 0, ws_h = 0, ws_part = 0, ws_lmval = 0, ws_lmidx = 0,
-         ws_pf = 0, ws_tpart = 0, ws_tcnt = 0, ws_kraw = 0, ws_bytes = 0;
-  size_t ev_bytes = 0, acnt_bytes = 0, tcnt_bytes = 0;
+         ws_pf = 0, ws_tpart = 0, ws_tcnt = 0, ws_kraw = 0, ws_pools = 0, ws_pcnt = 0, ws_bytes = 0;
+  size_t ev_bytes = 0, acnt_bytes = 0, tcnt_bytes = 0, pcnt_bytes = 0;
+  // run-time claims (mk_set_dispatch): 0 = static queues; 1 = every projection of every layer
+  // is a pool of n_sms * dyn_split tasks claimed at run time
+  int dyn = 0, dyn_split = 2;
+  std::vector<uint32_t> pool_first, pool_count;  // per pool: first task index, task count
+  int pool_cap = 0;
   int pf_rows = 0;
   size_t kv_bytes = 0;
   uint64_t weight_bytes_per_step = 0;
@@ -480,6 +485,12 @@ int build_graph(mk_ctx* c) {
   std::vector<uint32_t> evc(c->n_events, 0);
   std::vector<std::vector<Task>> q(n);
   const int rpg = (c->G + 2) * D;
+  // Run-time claims (mk_set_dispatch): a projection of a layer is a pool of tasks cut for
+  // n_sms * dyn_split equal shares; every SM's queue holds one TK_POOL entry for it, where the
+  // SM claims tasks until the pool is empty.  qv is the validation view: the pool's tasks
+  // dealt round-robin over the SMs at that queue position (one assignment the claims can give).
+  const bool dyn = c->dyn != 0;
+  std::vector<std::vector<Task>> qv(n);
 
   // embedding slices
   {
@@ -490,6 +501,7 @@ int build_graph(mk_ctx* c) {
         add_notify(t, ev_embed());
         evc[ev_embed()]++;
         q[s].push_back(t);
+        if (dyn) qv[s].push_back(t);
       }
   }
   // GEMV ops.  CUDA-core tasks: row ranges (parts = (first row, rows)).  Tensor-core tasks:
@@ -546,7 +558,46 @@ int build_graph(mk_ctx* c) {
   const Plan lm_pl = plan(TK_LMHEAD, f.vocab, 1);
   c->n_recs = rec_next;
   const int n_attn = B * nkv * c->nch;
+  std::vector<Task> pool_tasks;
+  c->pool_first.clear();
+  c->pool_count.clear();
+  auto push_static = [&](int s, const Task& t) {
+    q[s].push_back(t);
+    if (dyn) qv[s].push_back(t);
+  };
+  auto add_pool = [&](int kind, int l, int rows, int gran, auto&& finish) -> int {
+    const auto parts = partition_rows(rows, gran, std::vector<double>((size_t)n * c->dyn_split, 1.0), c->task_rows);
+    const uint32_t p = (uint32_t)c->pool_first.size();
+    c->pool_first.push_back((uint32_t)pool_tasks.size());
+    uint32_t cnt = 0;
+    for (const auto& v : parts)
+      for (const auto& pr : v) {
+        Task t = make_task(kind, l, pr.first, pr.second);
+        if (int rc = finish(t)) return rc;
+        pool_tasks.push_back(t);
+        qv[cnt % n].push_back(t);
+        ++cnt;
+      }
+    c->pool_count.push_back(cnt);
+    Task e = make_task(TK_POOL, l, 0, 0);
+    e.index = p;
+    for (int s2 = 0; s2 < n; ++s2) q[s2].push_back(e);
+    return MK_OK;
+  };
   for (int l = 0; l < L; ++l) {
+    auto qkv_edges = [&](Task& t) -> int {
+      add_wait(t, l == 0 ? ev_embed() : ev_down(c, l - 1));
+      const int g0 = (int)t.row0 / rpg, g1 = (int)(t.row0 + t.nrows - 1) / rpg;
+      if (g1 - g0 > 1) return fail(c, MK_ERR_UNSUPPORTED, "QKV task spans more than two KV groups");
+      for (int g = g0; g <= g1; ++g) {
+        add_notify(t, ev_qkv(c, l, g));
+        evc[ev_qkv(c, l, g)]++;
+      }
+      return MK_OK;
+    };
+    if (dyn) {
+      if (int rc = add_pool(TK_QKV, l, c->rows_qkv, 2, qkv_edges)) return rc;
+    } else
     for (int s = 0; s < n; ++s)
       for (int j = 0; j < (int)qkv_pl.parts[s].size(); ++j) {
         Task t = gemv_task(TK_QKV, l, qkv_pl, s, j);
@@ -572,9 +623,33 @@ int build_graph(mk_ctx* c) {
       add_wait(t, ev_qkv(c, l, g));
       add_notify(t, ev_attn(c, l));
       const int s = (int)(((long long)idx * n / n_attn + (long long)l * 37) % n);
-      q[s].push_back(t);
+      push_static(s, t);
     }
     evc[ev_attn(c, l)] = (uint32_t)(B * nkv);
+    if (dyn) {
+      auto o_edges = [&](Task& t) -> int {
+        add_wait(t, ev_attn(c, l));
+        add_notify(t, ev_o(c, l));
+        evc[ev_o(c, l)]++;
+        return MK_OK;
+      };
+      auto gu_edges = [&](Task& t) -> int {
+        add_wait(t, ev_o(c, l));
+        add_notify(t, ev_gu(c, l));
+        evc[ev_gu(c, l)]++;
+        return MK_OK;
+      };
+      auto d_edges = [&](Task& t) -> int {
+        add_wait(t, ev_gu(c, l));
+        add_notify(t, ev_down(c, l));
+        evc[ev_down(c, l)]++;
+        return MK_OK;
+      };
+      if (int rc = add_pool(TK_OPROJ, l, f.hidden, 1, o_edges)) return rc;
+      if (int rc = add_pool(TK_GATEUP, l, c->rows_gu, 2, gu_edges)) return rc;
+      if (int rc = add_pool(TK_DOWN, l, f.hidden, 1, d_edges)) return rc;
+      continue;
+    }
     for (int s = 0; s < n; ++s)
       for (int j = 0; j < (int)o_pl.parts[s].size(); ++j) {
         Task t = gemv_task(TK_OPROJ, l, o_pl, s, j);
@@ -610,15 +685,33 @@ int build_graph(mk_ctx* c) {
         add_wait(t, ev_down(c, L - 1));
         if (!c->tc) t.index = (uint32_t)idx;  // argmax partial slot (tensor-core: the tile's)
         ++idx;
-        q[s].push_back(t);
+        push_static(s, t);
       }
     c->n_lm = c->tc ? c->tc_tiles[TK_LMHEAD] : idx;
     evc[c->ev_lm] = (uint32_t)c->n_lm;
     evc[c->ev_tok] = 1u;
   }
+  if (dyn) {
+    // every SM ends its step with a static LM-head task (the claim counters of a step are
+    // recycled by the token pick, which needs every SM's claims of two steps back done)
+    for (int s = 0; s < n; ++s)
+      if (q[s].empty() || q[s].back().kind != TK_LMHEAD)
+        return fail(c, MK_ERR_UNSUPPORTED, "run-time claims need an LM-head task on every SM");
+    // validate the round-robin view with the ordinary checks
+    c->g.tasks.clear();
+    for (int s = 0; s < n; ++s)
+      for (auto& t : qv[s]) c->g.tasks.push_back({t, s});
+    if (int rc = validate(c, to_vtasks(c->g), evc)) return rc;
+  }
   c->g.tasks.clear();
   c->qbegin.assign(n + 1, 0);
   uint64_t wbytes = 0;
+  for (auto& t : pool_tasks) {
+    switch (t.kind) {
+      case TK_QKV: case TK_OPROJ: case TK_GATEUP: wbytes += (uint64_t)t.nrows * f.hidden * 2; break;
+      case TK_DOWN: wbytes += (uint64_t)t.nrows * f.ffn * 2; break;
+    }
+  }
   for (int s = 0; s < n; ++s) {
     c->qbegin[s] = (uint32_t)c->g.tasks.size();
     for (auto& t : q[s]) {
@@ -641,6 +734,11 @@ int build_graph(mk_ctx* c) {
   c->g.ev_count = evc;
   c->g.n_sms = n;
   c->weight_bytes_per_step = wbytes;
+  if (dyn) {  // the pools' tasks follow the queues (SM -1: whoever claims them)
+    for (auto& fi : c->pool_first) fi += c->qbegin[n];
+    for (auto& t : pool_tasks) c->g.tasks.push_back({t, -1});
+    return MK_OK;
+  }
   return validate(c, to_vtasks(c->g), evc);
 }
 
@@ -690,7 +788,13 @@ void layout(mk_ctx* c) {
   // room for re-partitioned graphs (mk_set_sm_weights) without changing the workspace size
   c->task_cap = c->g.tasks.size() * 2 + (size_t)c->n_sms * 16;
   c->lm_cap = (size_t)c->n_lm * 2 + (size_t)c->n_sms * 4;
+  // run-time claims: queue entries (one per SM and pool) plus pools of up to 4 tasks per SM
+  c->pool_cap = 4 * L;
+  c->task_cap = std::max(c->task_cap, c->g.tasks.size() + (size_t)c->n_sms * c->pool_cap * 5);
   c->ws_tasks = take(c->task_cap * sizeof(Task));
+  c->ws_pools = take((size_t)c->pool_cap * 2 * sizeof(uint32_t));
+  c->pcnt_bytes = (size_t)4 * c->pool_cap * sizeof(uint32_t);
+  c->ws_pcnt = take(c->pcnt_bytes);
   c->ws_qbegin = take((c->n_sms + 1) * sizeof(uint32_t));
   c->ws_evcount = take(c->n_events * sizeof(uint32_t));
   c->ev_bytes = c->n_events * sizeof(uint32_t);
@@ -799,8 +903,18 @@ int upload_graph(mk_ctx* c, uint8_t* W) {
                "event upload") ||
       !cuda_ok(c, cudaMemset(W + c->ws_ev, 0, c->ev_bytes), "counter reset") ||
       !cuda_ok(c, cudaMemset(W + c->ws_acnt, 0, c->acnt_bytes), "counter reset") ||
-      !cuda_ok(c, cudaMemset(W + c->ws_tcnt, 0, c->tcnt_bytes), "counter reset"))
+      !cuda_ok(c, cudaMemset(W + c->ws_tcnt, 0, c->tcnt_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(W + c->ws_pcnt, 0, c->pcnt_bytes), "counter reset"))
     return MK_ERR_CUDA;
+  if (!c->pool_first.empty()) {
+    std::vector<uint32_t> pl;
+    for (size_t p = 0; p < c->pool_first.size(); ++p) {
+      pl.push_back(c->pool_first[p]);
+      pl.push_back(c->pool_count[p]);
+    }
+    if (!cuda_ok(c, cudaMemcpy(W + c->ws_pools, pl.data(), pl.size() * 4, cudaMemcpyHostToDevice), "pool upload"))
+      return MK_ERR_CUDA;
+  }
   c->epoch = 0;
   return MK_OK;
 }
@@ -892,9 +1006,9 @@ int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
       base += c->tc_tiles[k];
     }
     c->n_tile_ids = base;
-    c->variant = find_decode_variant(0, 1, 0, 1, f.head_dim, kTcBatch, f.qk_norm);
+    c->variant = find_decode_variant(0, 1, 0, 1, f.head_dim, kTcBatch, f.qk_norm, 0);
   } else {
-    c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm, f.qk_norm);
+    c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm, f.qk_norm, 0);
   }
   c->sm_weights.assign(c->n_sms, 1.0);
   rc = build_graph(c);
@@ -1029,6 +1143,7 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
       !cuda_ok(c, cudaMemset(W + c->ws_ev, 0, c->ev_bytes), "counter reset") ||
       !cuda_ok(c, cudaMemset(W + c->ws_acnt, 0, c->acnt_bytes), "counter reset") ||
       !cuda_ok(c, cudaMemset(W + c->ws_tcnt, 0, c->tcnt_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(W + c->ws_pcnt, 0, c->pcnt_bytes), "counter reset") ||
       !cuda_ok(c, cudaMemset(W + c->ws_err, 0, 16), "error reset") ||
       !cuda_ok(c, cudaStreamSynchronize(s), "load sync"))
     return MK_ERR_CUDA;
@@ -1138,6 +1253,10 @@ int decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache,
   P.x_mid = reinterpret_cast<float*>(W + c->ws_xmid);
   P.qbuf = reinterpret_cast<float*>(W + c->ws_q);
   P.kraw = reinterpret_cast<float*>(W + c->ws_kraw);
+  P.pools = reinterpret_cast<const uint2*>(W + c->ws_pools);
+  P.pcnt = reinterpret_cast<uint32_t*>(W + c->ws_pcnt);
+  P.n_pools = (int)c->pool_first.size();
+  P.dyn = c->dyn;
   P.qk_norm = f.qk_norm;
   P.obuf = reinterpret_cast<float*>(W + c->ws_o);
   P.hbuf = reinterpret_cast<float*>(W + c->ws_h);
@@ -1174,7 +1293,7 @@ int decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache,
   P.drop_event = c->drop_event;
   P.timeout_ns = c->timeout_ns;
   P.trace = c->trace;
-  P.l2_ahead = c->l2_ahead;
+  P.l2_ahead = c->dyn ? 0 : c->l2_ahead;  // the lookahead walks static queues only
   std::string err;
   int rc = launch_decode(c->variant, P, c->n_sms, reinterpret_cast<cudaStream_t>(stream), &err);
   if (rc) return fail(c, rc, err);
@@ -1212,6 +1331,8 @@ int mk_sync_status(mk_ctx* c, void* stream) {
   // reset counters so the context stays usable
   if (!cuda_ok(c, cudaMemset(c->ws + c->ws_ev, 0, c->ev_bytes), "counter reset") ||
       !cuda_ok(c, cudaMemset(c->ws + c->ws_acnt, 0, c->acnt_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(c->ws + c->ws_tcnt, 0, c->tcnt_bytes), "counter reset") ||
+      !cuda_ok(c, cudaMemset(c->ws + c->ws_pcnt, 0, c->pcnt_bytes), "counter reset") ||
       !cuda_ok(c, cudaMemset(c->ws + c->ws_err, 0, 16), "error reset") ||
       !cuda_ok(c, cudaDeviceSynchronize(), "reset sync"))
     return MK_ERR_CUDA;
@@ -1286,6 +1407,49 @@ int mk_set_sm_weights(mk_ctx* c, const float* weights, int n, void* stream) {
 int mk_set_op_sm_weights(mk_ctx* c, int op_kind, const float* weights, int n, void* stream) {
   if (op_kind == 0) return fail(c, MK_ERR_INVALID_ARG, "op_kind must be a projection task kind");
   return set_weights(c, op_kind, weights, n, stream);
+}
+
+int mk_set_dispatch(mk_ctx* c, int mode, int tasks_per_sm, void* stream) {
+  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (mode != MK_DISPATCH_STATIC && mode != MK_DISPATCH_CLAIM) return fail(c, MK_ERR_INVALID_ARG, "unknown mode");
+  if (mode == MK_DISPATCH_CLAIM && (tasks_per_sm < 1 || tasks_per_sm > 4))
+    return fail(c, MK_ERR_INVALID_ARG, "tasks_per_sm must be in [1, 4]");
+  const mk_config& f = c->cfg;
+  int variant = c->variant;
+  if (mode == MK_DISPATCH_CLAIM) {
+    if (c->tc || c->bm != 1)
+      return fail(c, MK_ERR_UNSUPPORTED, "run-time claims are built for the batch-1 kernel only");
+    variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm, f.qk_norm, 1);
+  } else if (!c->tc) {
+    variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm, f.qk_norm, 0);
+  }
+  if (variant < 0) return fail(c, MK_ERR_UNSUPPORTED, "no kernel instantiation for this shape and dispatch mode");
+  if (c->loaded && !cuda_ok(c, cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "stream sync"))
+    return MK_ERR_CUDA;
+  const int old_dyn = c->dyn, old_split = c->dyn_split, old_variant = c->variant;
+  Graph old_g = c->g;
+  std::vector<uint32_t> old_q = c->qbegin, old_pf = c->pool_first, old_pc = c->pool_count;
+  const uint64_t old_wb = c->weight_bytes_per_step;
+  c->dyn = mode;
+  c->dyn_split = mode == MK_DISPATCH_CLAIM ? tasks_per_sm : c->dyn_split;
+  int rc = build_graph(c);
+  if (rc == MK_OK && (c->g.tasks.size() > c->task_cap || (int)c->pool_first.size() > c->pool_cap))
+    rc = fail(c, MK_ERR_UNSUPPORTED, "graph exceeds the workspace reserve");
+  if (rc != MK_OK) {
+    std::string m = c->err;
+    c->dyn = old_dyn;
+    c->dyn_split = old_split;
+    c->g = old_g;
+    c->qbegin = old_q;
+    c->pool_first = old_pf;
+    c->pool_count = old_pc;
+    c->weight_bytes_per_step = old_wb;
+    return fail(c, rc, m);
+  }
+  c->variant = variant;
+  (void)old_variant;
+  if (c->loaded && upload_graph(c, c->ws) != MK_OK) return MK_ERR_CUDA;
+  return MK_OK;
 }
 
 int mk_set_l2_prefetch(mk_ctx* c, int stages) {

@@ -68,6 +68,7 @@ enum TaskKind : uint8_t {
   TK_GATEUP = 5,  // h = silu(W_g xn) * (W_u xn), rows interleaved (g_i, u_i)
   TK_DOWN = 6,    // x_next = x_mid + W_d h
   TK_LMHEAD = 7,  // logits rows of W_lm . RMSNorm(x); per-task argmax partial
+  TK_POOL = 8,    // queue entry (run-time claims): claim tasks of pool `index` until it is empty
 };
 
 struct Task {
@@ -132,7 +133,15 @@ struct DecodeParams {
   int n_steps;                // greedy decode steps in this launch (step s: epoch + s, pos + s)
   uint32_t ev_tok;            // event: the step's tokens are picked (the next step's embedding waits)
   int qk_norm;                // 1: LayerNorm of every q and k head before RoPE, in the attention task
+  // run-time claims: pools[p] = (first task, task count); pcnt[4][n_pools] claim counters, one
+  // row per step (epoch mod 4), the row of step e + 2 zeroed by step e's token pick
+  const uint2* pools;
+  uint32_t* pcnt;
+  int n_pools;
+  int dyn;
 };
+constexpr int kDynQ = 64;                 // run-time claims: task FIFO from the producer to the other roles
+constexpr uint32_t kDynEnd = 0xffffffffu;  // FIFO entry: no more tasks in this launch
 constexpr uint64_t kStallPrefetchNs = 1000;    // producer blocked this long: prefetch ahead into L2
 constexpr uint64_t kStallPrefetchGapNs = 100;   // then one more stage per this interval
 #ifndef MK_MIN_CHUNK_KEYS
@@ -157,9 +166,9 @@ TensorMapEncodeFn get_tensor_map_encoder();
 
 // Kernel variants: one instantiation per (segments, rows per stage) of the two K sizes.
 struct Variant {
-  int nseg_h, rps_h, nseg_f, rps_f, head_dim, bm, qkn;
+  int nseg_h, rps_h, nseg_f, rps_f, head_dim, bm, qkn, dyn;
 };
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn);
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn, int dyn);
 const void* decode_kernel_ptr(int variant);
 size_t decode_smem_bytes(int variant);
 int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t stream, std::string* err);

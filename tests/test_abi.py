@@ -233,3 +233,69 @@ def test_per_op_weights_repartition_only_that_op():
         assert np.array_equal(again, before)
     finally:
         mk.mk_destroy(ctx)
+
+
+# ---------------------------------------------------------------- run-time claims (scheduling variant)
+
+def _rows(shape, kind):
+    D = shape.head_dim
+    return {2: (shape.n_q_heads + 2 * shape.n_kv_heads) * D, 4: shape.hidden, 5: 2 * shape.ffn, 6: shape.hidden}[kind]
+
+
+@pytest.mark.parametrize("shape,tps", [(mi.TINY, 1), (mi.TINY, 2), (mi.LLAMA8B.with_layers(3), 2),
+                                       (mi.LLAMA8B.with_layers(2), 4)])
+def test_claim_dispatch_pools_cover_every_projection(shape, tps):
+    ctx = mk.mk_build_taskgraph(mk.Config.from_shape(shape, 1, 256).c(), -1)
+    try:
+        n0 = mk.mk_get_graph_info(ctx)["n_tasks"]
+        mk.mk_set_dispatch(ctx, mk.MK_DISPATCH_CLAIM, tps)
+        tasks, counts = mk.mk_export_taskgraph(ctx)
+        n_sms = mk.mk_get_graph_info(ctx)["n_sms"]
+        L = shape.n_layers
+        entries = tasks[tasks[:, 0] == 8]
+        pooled = tasks[tasks[:, 2] == -1]
+        # one claim entry per SM for each projection of each layer, on every SM
+        assert len(entries) == n_sms * 4 * L
+        assert sorted(set(entries[:, 2].tolist())) == list(range(n_sms))
+        assert set(pooled[:, 0].tolist()) == {2, 4, 5, 6}
+        for kind in (2, 4, 5, 6):
+            for l in range(L):
+                sel = pooled[(pooled[:, 0] == kind) & (pooled[:, 1] == l)]
+                cover = np.zeros(_rows(shape, kind), dtype=np.int32)
+                for t in sel:
+                    cover[t[3]:t[3] + t[4]] += 1
+                assert (cover == 1).all(), f"kind {kind} layer {l}: rows not covered exactly once"
+                assert len(sel) <= n_sms * tps
+                # each task notifies the op's event; the event's count is the pool's task count
+                if kind != 2:
+                    assert counts[sel[0, 9]] == len(sel)
+        # static tasks stay on their SMs: embedding, attention and the LM head
+        static = tasks[(tasks[:, 2] >= 0) & (tasks[:, 0] != 8)]
+        assert set(static[:, 0].tolist()) == {1, 3, 7}
+        mk.mk_set_dispatch(ctx, mk.MK_DISPATCH_STATIC)
+        assert mk.mk_get_graph_info(ctx)["n_tasks"] == n0
+        assert not (mk.mk_export_taskgraph(ctx)[0][:, 0] == 8).any()
+    finally:
+        mk.mk_destroy(ctx)
+
+
+def test_claim_dispatch_rejections():
+    for shape, b in ((mi.TINY, 4), (mi.TINY, 16), (mi.CHAMELEON7B.with_layers(1), 1)):
+        ctx = mk.mk_build_taskgraph(mk.Config.from_shape(shape, b, 64).c(), -1)
+        try:
+            with pytest.raises(mk.MkError) as e:
+                mk.mk_set_dispatch(ctx, mk.MK_DISPATCH_CLAIM, 2)
+            assert e.value.code == mk.MK_ERR_UNSUPPORTED
+        finally:
+            mk.mk_destroy(ctx)
+    ctx = mk.mk_build_taskgraph(_cfg().c(), -1)
+    try:
+        for mode, tps in ((mk.MK_DISPATCH_CLAIM, 0), (mk.MK_DISPATCH_CLAIM, 5), (7, 1)):
+            with pytest.raises(mk.MkError) as e:
+                mk.mk_set_dispatch(ctx, mode, tps)
+            assert e.value.code == mk.MK_ERR_INVALID_ARG
+        n0 = mk.mk_get_graph_info(ctx)["n_tasks"]
+        mk.mk_set_dispatch(ctx, mk.MK_DISPATCH_CLAIM, 1)
+        assert mk.mk_get_graph_info(ctx)["n_tasks"] > n0
+    finally:
+        mk.mk_destroy(ctx)
