@@ -79,7 +79,7 @@ def parse():
     p.add_argument("--no-calibrate", action="store_true",
                    help="keep equal rows per SM instead of the schedule calibrated during warm-up")
     p.add_argument("--workload", default="llama8b", choices=sorted(WORKLOADS))
-    p.add_argument("--dispatch", default="static", choices=["static", "claim"],
+    p.add_argument("--dispatch", default="static", choices=["static", "claim", "claim-paced"],
                    help="scheduling variant: fixed per-SM queues (default), or projection tasks claimed "
                         "at run time from per-op pools (batch-1 kernel only)")
     p.add_argument("--tasks-per-sm", type=int, default=2, help="pool tasks per SM and projection (--dispatch claim)")
@@ -401,8 +401,9 @@ def run_mk(args, rank, world, local):
         tok = torch.from_numpy(mi.prompt(0, 0, B, shape.vocab).astype(np.int32)).to(dev)
     warm = args.warmup
     calibrated = False
-    if args.dispatch == "claim":  # pools are cut in equal shares: no per-SM calibration
-        m.set_dispatch(mk.MK_DISPATCH_CLAIM, args.tasks_per_sm)
+    if args.dispatch != "static":  # pools are cut in equal shares: no per-SM calibration
+        m.set_dispatch(mk.MK_DISPATCH_CLAIM if args.dispatch == "claim" else mk.MK_DISPATCH_CLAIM_PACED,
+                       args.tasks_per_sm)
     elif not args.no_calibrate and warm >= 6:
         # measure per-SM streaming speed on warm-up steps and re-partition rows (3 rounds x 2 steps)
         m.calibrate(tok, steps=2, rounds=3)
@@ -490,7 +491,8 @@ def run_mk(args, rank, world, local):
                        "decode_positions": [pos0, pos0 + args.steps - 1], "batch_per_gpu": B,
                        "global_batch": world * B, "parallelism": "replicas", "weights": "bf16",
                        "schedule": (f"run-time claims from per-op pools, {args.tasks_per_sm} tasks per SM"
-                                    if args.dispatch == "claim" else
+                                    + (", paced by the workers" if args.dispatch == "claim-paced" else "")
+                                    if args.dispatch != "static" else
                                     "calibrated per-SM rows" if calibrated else "equal rows per SM"),
                        "l2": "inputs larger than L2 (15 GB of weights streamed per step)"},
             "ms_per_step_p50": float(np.median(step_ms)), "tokens_per_s": 1e3 / (max_ms / args.steps) * world * B,

@@ -187,11 +187,14 @@ int mk_set_op_sm_weights(mk_ctx* ctx, int op_kind, const float* weights, int n, 
  * tasks_per_sm * n_sms equal tasks (1..4); each SM's queue holds one entry per pool, where the
  * SM claims tasks from the pool's counter (one atomic add per claim) until it is empty, so
  * faster SMs take more; attention, embedding and LM-head tasks stay static.  The graph is
- * validated with the pools' tasks dealt round-robin.  Only the batch-1 kernel of the Llama-3-8B
+ * validated with the pools' tasks dealt round-robin.  MK_DISPATCH_CLAIM_PACED: the same, but an
+ * SM claims its next task only once its workers finished every task but the last one handed
+ * to them (at most one unstarted claimed task per SM).  Only the batch-1 kernel of the Llama-3-8B
  * and tiny shapes has a run-time-claim instantiation: MK_ERR_UNSUPPORTED otherwise.  Rebuilds
  * and re-uploads the graph (synchronises `stream` first if weights are loaded). */
 #define MK_DISPATCH_STATIC 0
 #define MK_DISPATCH_CLAIM 1
+#define MK_DISPATCH_CLAIM_PACED 2
 int mk_set_dispatch(mk_ctx* ctx, int mode, int tasks_per_sm, void* stream);
 
 /* Weight prefetch depth: besides the shared-memory ring (6 stages of 32 KB per SM), an SM's

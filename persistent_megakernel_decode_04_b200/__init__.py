@@ -35,6 +35,7 @@ MK_ERR_UNSUPPORTED = -6
 MK_MAX_BATCH = 16
 MK_DISPATCH_STATIC = 0
 MK_DISPATCH_CLAIM = 1
+MK_DISPATCH_CLAIM_PACED = 2
 
 TASK_KINDS = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead", 8: "pool"}
 
@@ -243,8 +244,9 @@ def mk_set_l2_prefetch(ctx, stages: int):
 
 
 def mk_set_dispatch(ctx, mode: int, tasks_per_sm: int = 2, stream=None):
-    """MK_DISPATCH_STATIC (fixed per-SM queues) or MK_DISPATCH_CLAIM (projection tasks claimed at
-    run time from per-op pools of tasks_per_sm * n_sms tasks)."""
+    """MK_DISPATCH_STATIC (fixed per-SM queues), MK_DISPATCH_CLAIM (projection tasks claimed at
+    run time from per-op pools of tasks_per_sm * n_sms tasks) or MK_DISPATCH_CLAIM_PACED (claims
+    paced by the SM's workers)."""
     _check(_lib.mk_set_dispatch(ctx, int(mode), int(tasks_per_sm), _stream(stream)), ctx)
 
 

@@ -1559,9 +1559,31 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
             gated = true;
             if (!ok) break;
           }
-          // claim until the pool is empty; the next claim is in flight while a task streams
+          // claim until the pool is empty; the next claim is in flight while a task streams.
+          // Paced (dyn == 2): a claim waits until the workers have finished every task but the
+          // last one handed to them, so an SM holds at most one unstarted task.
           const uint2 pl = P.pools[t.index];
           uint32_t* ctr = P.pcnt + (size_t)((P.epoch + (uint32_t)st) & 3u) * P.n_pools + t.index;
+          auto paced = [&]() -> bool {
+            if (P.dyn != 2 || dq_count == 0) return true;
+            uint64_t t0 = 0;
+            for (uint32_t n = 1;; ++n) {
+              if (ld_acquire_cta_shared(&S.wdone) + 1u >= dq_count) return true;
+              if ((n & 63u) == 0) {
+                if (S.abort) return false;
+                const uint64_t now = globaltimer_ns();
+                if (t0 == 0) t0 = now;
+                else if (now - t0 > P.timeout_ns) {
+                  raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, i);
+                  return false;
+                }
+              }
+            }
+          };
+          if (!paced()) {
+            ok = false;
+            break;
+          }
           uint32_t c = atomicAdd(ctr, 1u);
           while (ok && c < pl.y) {
             const uint32_t id = pl.x + c;
@@ -1569,8 +1591,13 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
               ok = false;
               break;
             }
-            const uint32_t cn = atomicAdd(ctr, 1u);
+            uint32_t cn = 0xffffffffu;
+            if (P.dyn != 2) cn = atomicAdd(ctr, 1u);
             ok = stream_gemv(P.tasks[id], id);
+            if (ok && P.dyn == 2) {
+              ok = paced();
+              if (ok) cn = atomicAdd(ctr, 1u);
+            }
             c = cn;
           }
           continue;

@@ -1411,12 +1411,14 @@ int mk_set_op_sm_weights(mk_ctx* c, int op_kind, const float* weights, int n, vo
 
 int mk_set_dispatch(mk_ctx* c, int mode, int tasks_per_sm, void* stream) {
   if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
-  if (mode != MK_DISPATCH_STATIC && mode != MK_DISPATCH_CLAIM) return fail(c, MK_ERR_INVALID_ARG, "unknown mode");
-  if (mode == MK_DISPATCH_CLAIM && (tasks_per_sm < 1 || tasks_per_sm > 4))
+  if (mode != MK_DISPATCH_STATIC && mode != MK_DISPATCH_CLAIM && mode != MK_DISPATCH_CLAIM_PACED)
+    return fail(c, MK_ERR_INVALID_ARG, "unknown mode");
+  const bool claim = mode != MK_DISPATCH_STATIC;
+  if (claim && (tasks_per_sm < 1 || tasks_per_sm > 4))
     return fail(c, MK_ERR_INVALID_ARG, "tasks_per_sm must be in [1, 4]");
   const mk_config& f = c->cfg;
   int variant = c->variant;
-  if (mode == MK_DISPATCH_CLAIM) {
+  if (claim) {
     if (c->tc || c->bm != 1)
       return fail(c, MK_ERR_UNSUPPORTED, "run-time claims are built for the batch-1 kernel only");
     variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm, f.qk_norm, 1);
@@ -1431,7 +1433,7 @@ int mk_set_dispatch(mk_ctx* c, int mode, int tasks_per_sm, void* stream) {
   std::vector<uint32_t> old_q = c->qbegin, old_pf = c->pool_first, old_pc = c->pool_count;
   const uint64_t old_wb = c->weight_bytes_per_step;
   c->dyn = mode;
-  c->dyn_split = mode == MK_DISPATCH_CLAIM ? tasks_per_sm : c->dyn_split;
+  c->dyn_split = claim ? tasks_per_sm : c->dyn_split;
   int rc = build_graph(c);
   if (rc == MK_OK && (c->g.tasks.size() > c->task_cap || (int)c->pool_first.size() > c->pool_cap))
     rc = fail(c, MK_ERR_UNSUPPORTED, "graph exceeds the workspace reserve");

@@ -15,19 +15,20 @@ pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
 
 
-def _model(w, max_seq, tps=None):
+def _model(w, max_seq, tps=None, mode=mk.MK_DISPATCH_CLAIM):
     m = mk.Megakernel(mk.Config.from_shape(w.shape, 1, max_seq), w, 0)
     if tps:
-        m.set_dispatch(mk.MK_DISPATCH_CLAIM, tps)
+        m.set_dispatch(mode, tps)
     return m
 
 
-@pytest.mark.parametrize("tps", [1, 2, 4])
-def test_claims_match_the_oracle(tps):
+@pytest.mark.parametrize("tps,mode", [(1, mk.MK_DISPATCH_CLAIM), (2, mk.MK_DISPATCH_CLAIM), (4, mk.MK_DISPATCH_CLAIM),
+                                      (2, mk.MK_DISPATCH_CLAIM_PACED)])
+def test_claims_match_the_oracle(tps, mode):
     w = mi.make_weights(mi.TINY, seed=40)
     prompt = mi.prompt(40, 0, 14, w.shape.vocab)
     ref = oracle.Decoder(w, 1, 64)
-    m = _model(w, 64, tps)
+    m = _model(w, 64, tps, mode)
     rl = ref.prefill(prompt)[0]
     m.prefill(torch.from_numpy(prompt[None].astype(np.int32)).to(DEV))
     tok = oracle.argmax(rl)
@@ -42,8 +43,8 @@ def test_claims_match_the_oracle(tps):
     m.close()
 
 
-def _run(w, max_seq, tps, prompt_or_cache, steps, multi):
-    m = _model(w, max_seq, tps)
+def _run(w, max_seq, tps, prompt_or_cache, steps, multi, mode=mk.MK_DISPATCH_CLAIM):
+    m = _model(w, max_seq, tps, mode)
     if isinstance(prompt_or_cache, tuple):
         kv, L = prompt_or_cache
         m.kv_view()[:, :, :1, :, :L, :] = torch.from_numpy(kv.view(np.int16)).to(DEV)
@@ -75,8 +76,8 @@ def test_claims_equal_static_schedule_tiny(multi):
     w = mi.make_weights(mi.TINY, seed=42)
     prompt = mi.prompt(42, 0, 10, w.shape.vocab)
     a = _run(w, 32, None, prompt, 9, multi)
-    for tps in (1, 3):
-        b = _run(w, 32, tps, prompt, 9, multi)
+    for tps, mode in ((1, mk.MK_DISPATCH_CLAIM), (3, mk.MK_DISPATCH_CLAIM), (2, mk.MK_DISPATCH_CLAIM_PACED)):
+        b = _run(w, 32, tps, prompt, 9, multi, mode)
         assert np.array_equal(a[0], b[0])
         assert np.abs(a[1] - b[1]).max() <= 1e-3
 
@@ -89,7 +90,8 @@ def test_claims_equal_static_schedule_llama8b_two_layers():
     a = _run(w, L + 16, None, (kv, L), 5, True)
     b = _run(w, L + 16, 2, (kv, L), 5, True)
     c = _run(w, L + 16, 2, (kv, L), 5, False)
-    for r in (b, c):
+    d = _run(w, L + 16, 2, (kv, L), 5, True, mk.MK_DISPATCH_CLAIM_PACED)
+    for r in (b, c, d):
         assert np.array_equal(a[0], r[0])
         assert np.abs(a[1] - r[1]).max() <= 1e-3
 
