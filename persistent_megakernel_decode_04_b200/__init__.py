@@ -388,7 +388,9 @@ class Megakernel:
         """Measure each SM's busy time on each projection (QKV, O, gate/up, down, LM head) over
         `steps` traced decode steps (decoding `tokens`, which advances the positions) and
         re-partition that projection's rows so that every SM finishes it together; `rounds`
-        measure/re-partition passes.  Returns the weights, one row per projection kind."""
+        measure/re-partition passes.  Returns the weights, one row per projection kind.  (With
+        run-time claims the pools stay cut in equal shares: the weights apply once the static
+        schedule is selected again.)"""
         import numpy as np
         import torch
         info = self.info()
@@ -404,9 +406,10 @@ class Megakernel:
                 self.decode(tokens)
                 self.sync_status()
                 T = trace[: tasks.shape[0] * 6].view(-1, 6).cpu().numpy()
+                sm = (T[:, 3].astype(np.uint64) >> np.uint64(32)).astype(np.int64)  # the SM that ran it
                 for k in kinds:
                     sel = tasks[:, 0] == k
-                    np.add.at(busy[k], tasks[sel, 2], (T[sel, 2] - T[sel, 1]).astype(np.float64))
+                    np.add.at(busy[k], sm[sel], (T[sel, 2] - T[sel, 1]).astype(np.float64))
             mk_set_trace(self.ctx, None)
             for k in kinds:
                 b = busy[k]
