@@ -68,7 +68,8 @@ struct mk_ctx {
          ws_pf = 0, ws_tpart = 0, ws_tcnt = 0, ws_kraw = 0, ws_pools = 0, ws_pcnt = 0, ws_bytes = 0;
   size_t ev_bytes = 0, acnt_bytes = 0, tcnt_bytes = 0, pcnt_bytes = 0;
   // run-time claims (mk_set_dispatch): 0 = static queues; 1 = every projection of every layer
-  // is a pool of n_sms * dyn_split tasks claimed at run time
+  // is a pool of n_sms * dyn_split tasks claimed at run time; 2 = the same, claims paced by
+  // the SM's workers
   int dyn = 0, dyn_split = 2;
   std::vector<uint32_t> pool_first, pool_count;  // per pool: first task index, task count
   int pool_cap = 0;
@@ -1428,7 +1429,7 @@ int mk_set_dispatch(mk_ctx* c, int mode, int tasks_per_sm, void* stream) {
   if (variant < 0) return fail(c, MK_ERR_UNSUPPORTED, "no kernel instantiation for this shape and dispatch mode");
   if (c->loaded && !cuda_ok(c, cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "stream sync"))
     return MK_ERR_CUDA;
-  const int old_dyn = c->dyn, old_split = c->dyn_split, old_variant = c->variant;
+  const int old_dyn = c->dyn, old_split = c->dyn_split;
   Graph old_g = c->g;
   std::vector<uint32_t> old_q = c->qbegin, old_pf = c->pool_first, old_pc = c->pool_count;
   const uint64_t old_wb = c->weight_bytes_per_step;
@@ -1449,7 +1450,6 @@ int mk_set_dispatch(mk_ctx* c, int mode, int tasks_per_sm, void* stream) {
     return fail(c, rc, m);
   }
   c->variant = variant;
-  (void)old_variant;
   if (c->loaded && upload_graph(c, c->ws) != MK_OK) return MK_ERR_CUDA;
   return MK_OK;
 }
