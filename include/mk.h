@@ -119,7 +119,8 @@ int mk_prefill(mk_ctx* ctx, const int32_t* tokens, int B, int T, void* kv_cache,
                void* stream);
 
 /* Declare that the caller filled the cache itself: sequence b (b < B) has host_pos[b]
- * valid positions.  Sets the active batch to B. */
+ * valid positions.  Sets the active batch to B.  The cache holds keys as the decoder stores
+ * them: rotated by RoPE and, with qk_norm, normalised before that. */
 int mk_set_positions(mk_ctx* ctx, const int32_t* host_pos, int B);
 /* Current positions of the active batch (host copy kept by the library); returns B. */
 int mk_get_positions(const mk_ctx* ctx, int32_t* host_pos, int capacity);

@@ -299,3 +299,25 @@ def test_claim_dispatch_rejections():
         assert mk.mk_get_graph_info(ctx)["n_tasks"] > n0
     finally:
         mk.mk_destroy(ctx)
+
+
+def test_claim_dispatch_survives_repartitioning():
+    # per-SM weights re-partition the static tasks; with run-time claims the pools stay whole
+    ctx = mk.mk_build_taskgraph(mk.Config.from_shape(mi.TINY, 1, 64).c(), -1)
+    try:
+        mk.mk_set_dispatch(ctx, mk.MK_DISPATCH_CLAIM, 2)
+        n_sms = mk.mk_get_graph_info(ctx)["n_sms"]
+        before = mk.mk_export_taskgraph(ctx)[0]
+        w = np.linspace(0.5, 1.5, n_sms).astype(np.float32)
+        mk.mk_set_sm_weights(ctx, w)
+        after, counts = mk.mk_export_taskgraph(ctx)
+        pooled_b, pooled_a = before[before[:, 2] == -1], after[after[:, 2] == -1]
+        assert np.array_equal(pooled_b, pooled_a)
+        assert (after[:, 0] == 8).sum() == (before[:, 0] == 8).sum()
+        # the static part (embedding, LM head) follows the weights: more rows on faster SMs
+        lm = after[after[:, 0] == 7]
+        rows = np.zeros(n_sms)
+        np.add.at(rows, lm[:, 2], lm[:, 4])
+        assert rows[-1] > rows[0]
+    finally:
+        mk.mk_destroy(ctx)
