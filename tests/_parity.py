@@ -2,12 +2,19 @@
 
 Tolerances for the decoder follow the targets stated for this build: per-step logits
 max|diff| <= 2e-2 and relative L2 <= 5e-3; argmax equal wherever the oracle's top-2 margin
-exceeds 0.1.  "K/V cache within 1e-2" is read normwise: for every layer and for K and V
-separately, max|diff| <= 1e-2 * max(1, max|ref|).  An absolute 1e-2 is below bf16 storage
-precision (one ulp at |v| in [2, 4) is 0.0156), and an elementwise relative bound fails even
-between two correct CPU oracles at 8B depth (fp32 vs fp64 activations: 5 of 2.75M entries in
-the deepest layers, because 32 random layers amplify last-bit differences).  The elementwise
-count is still reported.
+exceeds 0.1.
+
+"K/V cache within 1e-2" is read elementwise as |diff| <= 1e-2 * max(1, |ref|) for every entry
+(an absolute 1e-2 is below bf16 storage precision: one ulp at |v| in [2, 4) is 0.0156; the
+relative form is always above one bf16 ulp of the reference, so two correct implementations
+whose pre-rounding values differ by a hair and round to neighbouring bf16 values still pass).
+This is asserted for every entry of every model shallower than KV_DEEP_LAYERS.
+
+For the 32-layer models the same elementwise bound fails even between two correct CPU oracles
+(fp32 vs fp64 activations: 5 of 2.75M entries of the 8B cache, in the deepest layers, because
+32 random layers amplify last-bit differences until a few entries sit near a rounding
+boundary).  There every layer's K and V must satisfy max|diff| <= 1e-2 * max(1, max|ref|) and
+the fraction of entries outside the elementwise bound must stay at or below KV_DEEP_FRAC.
 """
 import numpy as np
 
@@ -15,6 +22,8 @@ LOGIT_MAX_ABS = 2e-2
 LOGIT_REL_L2 = 5e-3
 KV_REL = 1e-2
 ARGMAX_MARGIN = 0.1
+KV_DEEP_LAYERS = 16
+KV_DEEP_FRAC = 2e-4
 
 
 def logits_close(got, ref, what=""):
@@ -41,14 +50,27 @@ def argmax_agrees(got_logits, ref_logits, got_token=None):
 
 
 def kv_close(got_bits, ref_bits, what=""):
-    """got/ref: bf16 bits [layer][K|V][...]; returns the elementwise-violation fraction."""
+    """got/ref: bf16 bits [layer][K|V][...].  Elementwise bound on every entry for models
+    shallower than KV_DEEP_LAYERS; for deeper ones the per-layer normwise bound plus a cap on
+    the fraction of entries outside the elementwise bound.  Returns that fraction."""
     import mk_inputs as mi
     g = mi.bf16_to_f32(np.asarray(got_bits).view(np.uint16)).astype(np.float64)
     r = mi.bf16_to_f32(np.asarray(ref_bits).view(np.uint16)).astype(np.float64)
+    assert g.shape == r.shape, f"{what}: shapes {g.shape} vs {r.shape}"
     assert np.isfinite(g).all(), f"{what}: non-finite K/V entries"
+    diff = np.abs(g - r)
+    viol = diff > KV_REL * np.maximum(1.0, np.abs(r))
+    frac = float(viol.mean()) if viol.size else 0.0
+    if r.shape[0] < KV_DEEP_LAYERS:
+        if viol.any():
+            idx = np.unravel_index(int(np.argmax(np.where(viol, diff, -1.0))), r.shape)
+            raise AssertionError(f"{what}: {int(viol.sum())} of {viol.size} entries outside 1e-2*max(1,|ref|); "
+                                 f"worst at {idx}: got {g[idx]:.6g}, oracle {r[idx]:.6g}")
+        return frac
     for l in range(r.shape[0]):
         for kind in range(2):
-            d = np.abs(g[l, kind] - r[l, kind]).max()
+            d = diff[l, kind].max()
             bound = KV_REL * max(1.0, np.abs(r[l, kind]).max())
             assert d <= bound, f"{what}: layer {l} {'KV'[kind]}: max|diff| {d:.4g} > {bound:.4g}"
-    return float((np.abs(g - r) > KV_REL * np.maximum(1.0, np.abs(r))).mean())
+    assert frac <= KV_DEEP_FRAC, f"{what}: {frac:.3e} of the entries outside the elementwise bound > {KV_DEEP_FRAC}"
+    return frac
