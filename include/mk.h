@@ -241,6 +241,51 @@ int mk_export_taskgraph(const mk_ctx* ctx, int32_t* tasks, int task_capacity, in
 int mk_validate_taskgraph(mk_ctx* ctx, const int32_t* tasks, int n_tasks, const int32_t* event_counts,
                           int n_events);
 
+/* Tensor parallel (the pages' multi-GPU scheme: "Compiler des LLM en MegaKernel ...", Part 1,
+ * where a matmul followed by an all-reduce is lowered into tile tasks that start the reduction
+ * on partial results, and "Valeur cle de MPK", overlap of computation and communication).
+ * Rank r of n_ranks holds 1/n_ranks of the query and KV heads, of the ffn rows and of the
+ * vocabulary: QKV, gate/up and the LM head are split by output rows (column parallel), O and
+ * down by input columns (row parallel).  Each O or down task stores its partial output rows
+ * into EVERY rank's receive buffer (peer stores) and raises the op's event on every rank
+ * (remote-signal edges); a rank's next op waits for all ranks' tasks and adds the ranks'
+ * partials in rank order, so the replicated residual stream is bitwise the same on every rank.
+ * The LM head's argmax is exchanged the same way, so every rank picks the same token.
+ *
+ * mk_build_taskgraph_tp builds an EMULATED tensor-parallel context: all n_ranks ranks on one
+ * device, in one persistent launch of n_ranks x (SMs / n_ranks) CTAs, CTA b serving rank
+ * b / (SMs / n_ranks), each rank's peer buffers in the same device memory.  Requirements:
+ * n_ranks in [2, 4]; max_batch == 1; qk_norm == 0; n_kv_heads, ffn / 8 and vocab divisible by
+ * n_ranks; a compiled instantiation for the shard shape (the tiny decoder over 2 ranks, the
+ * Llama-3-8B shape over 2 or 4) else MK_ERR_UNSUPPORTED.  The graph of every rank is validated
+ * together (mk_validate_taskgraph_tp).  The context is used with the ordinary calls:
+ * mk_weight_arena_bytes / mk_workspace_bytes / mk_kv_cache_bytes (the ranks' regions one after
+ * another; the cache is [rank][layer][K|V][1][n_kv_heads / n_ranks][max_seq][head_dim]),
+ * mk_load_weights (the whole model's host weights; each rank's shard is cut from them),
+ * mk_set_positions (a prompt is fed as decode steps from position 0, or the caller fills the
+ * cache), mk_decode_step / mk_decode_steps (logits [1][vocab] whole: each rank writes its
+ * vocabulary slice), mk_sync_status, mk_set_wait_timeout_ns, mk_debug_drop_notify (the event id
+ * on every rank), mk_get_graph_info, mk_destroy.  mk_prefill, mk_set_sm_weights,
+ * mk_set_op_sm_weights, mk_set_dispatch, mk_set_trace and mk_export_taskgraph return
+ * MK_ERR_UNSUPPORTED for it. */
+int mk_build_taskgraph_tp(const mk_config* cfg, int n_ranks, int device, mk_ctx** out);
+
+/* The tensor-parallel task graph of every rank: per task 15 int32 {rank, kind, layer, sm (global:
+ * rank r's SM s is r * (SMs / n_ranks) + s), row0, nrows (attention: chunk), n_wait, wait0, wait1,
+ * n_notify, notify0, notify1, remote (1: the notifies go to the event on every rank), row_lo,
+ * row_hi (gate/up: the rows of the residual sum x_mid this task writes; else 0)};
+ * event_counts: one rank's per-step thresholds (every rank has the same).  Returns the number
+ * of tasks; either buffer may be NULL to query sizes. */
+int mk_export_taskgraph_tp(const mk_ctx* ctx, int32_t* tasks, int task_capacity, int32_t* event_counts,
+                           int event_capacity);
+/* Validate an exported-and-edited tensor-parallel graph: per rank, thresholds equal the
+ * producers that reach that rank's counter (remote signals included); every op's rows,
+ * attention chunks and residual rows covered once; and, with every rank's queues simulated
+ * together, no deadlock and no task reading data before its producers on any rank.  MK_OK or
+ * MK_ERR_INVALID_ARG with the reason in mk_last_error(ctx). */
+int mk_validate_taskgraph_tp(mk_ctx* ctx, const int32_t* tasks, int n_tasks, const int32_t* event_counts,
+                             int n_events);
+
 /* Standalone decode attention in the Mirage article's example form (attention code sample:
  * Q [64,1,128], K [64,128,4096] pre-transposed, V [64,4096,128], fp16, O = softmax(Q K) V):
  *   q [BH][d], k_t [BH][d][L] (key index fastest), v [BH][L][d]: fp16 device arrays;
@@ -265,14 +310,32 @@ int mk_attention_status(void* workspace, int BH, int d, int L, void* stream);
  * arithmetic and result as mk_attention_decode; the scratch is a fixed 4 MiB array inside
  * the library that every GPU loading the library keeps until the process exits.  Sizes whose
  * scratch (mk_attention_workspace_bytes(BH, d, L)) exceeds 4 MiB are rejected with
- * MK_ERR_INVALID_ARG and a message.  The first call on a device looks up the array's device
- * address (once, with that device current); make that first call before any stream capture.
- * The call allocates nothing (no cudaMalloc, cudaFree or allocating library routine); it
- * zeroes the array's arrival counts and error word on `stream` before the kernel.  All calls
- * share the one array, so calls that overlap on the GPU (other streams, other threads) race:
- * order them on one stream. */
+ * MK_ERR_INVALID_ARG and a message; a device index of 64 or more with MK_ERR_UNSUPPORTED.
+ * The first call on a device looks up the array's device address (once, with that device
+ * current); make that first call before any stream capture.  The call allocates nothing (no
+ * cudaMalloc, cudaFree or allocating library routine); it zeroes the array's arrival counts on
+ * `stream` before the kernel.  A device wait that runs out is recorded in an error word at the
+ * end of the array, which keeps the first such event until mk_attention_noalloc_status reads
+ * it.  All calls share the one array, so calls that overlap on the GPU (other streams, other
+ * threads) race: order them on one stream. */
 int mk_attention_decode_noalloc(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d,
                                 int L, float scale, void* stream);
+/* Synchronise `stream` and report whether any mk_attention_decode_noalloc call on the current
+ * device since the previous mk_attention_noalloc_status had a device wait run out
+ * (MK_ERR_DEVICE_TIMEOUT: that call's output is undefined; the error word is cleared) or not
+ * (MK_OK).  Allocates nothing: the word is read and cleared with cudaMemcpyFromSymbol /
+ * cudaMemcpyToSymbol of 4 bytes. */
+int mk_attention_noalloc_status(void* stream);
+
+/* Limit, in nanoseconds, of every device-side wait of mk_attention_decode and
+ * mk_attention_decode_noalloc calls issued after this one (process-wide; default 2e9).  Must
+ * be > 0. */
+int mk_attention_set_wait_timeout_ns(uint64_t ns);
+/* Test hook for failure detection (process-wide): while unit >= 0, the split-KV attention
+ * kernels launched afterwards never load the 64-key unit with that global index (head h's units
+ * are h * ceil(L/64) ..), so the compute warp waiting for it runs out of time and the call's
+ * status reports MK_ERR_DEVICE_TIMEOUT.  Nothing faults or traps.  unit < 0 switches it off. */
+int mk_attention_debug_drop_unit(int unit);
 
 /* Last error text for ctx (or the thread's last context-free error when ctx is NULL). */
 const char* mk_last_error(const mk_ctx* ctx);

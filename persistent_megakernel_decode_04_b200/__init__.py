@@ -93,10 +93,16 @@ _SIGS = {
     "mk_get_graph_info": ([_vp, ctypes.POINTER(mk_graph_info)], _i32),
     "mk_export_taskgraph": ([_vp, _vp, _i32, _vp, _i32], _i32),
     "mk_validate_taskgraph": ([_vp, _vp, _i32, _vp, _i32], _i32),
+    "mk_build_taskgraph_tp": ([ctypes.POINTER(mk_config), _i32, _i32, ctypes.POINTER(_vp)], _i32),
+    "mk_export_taskgraph_tp": ([_vp, _vp, _i32, _vp, _i32], _i32),
+    "mk_validate_taskgraph_tp": ([_vp, _vp, _i32, _vp, _i32], _i32),
     "mk_attention_workspace_bytes": ([_i32, _i32, _i32], _sz),
     "mk_attention_decode": ([_vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.c_float, _vp, _vp], _i32),
     "mk_attention_status": ([_vp, _i32, _i32, _i32, _vp], _i32),
     "mk_attention_decode_noalloc": ([_vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.c_float, _vp], _i32),
+    "mk_attention_noalloc_status": ([_vp], _i32),
+    "mk_attention_set_wait_timeout_ns": ([_u64], _i32),
+    "mk_attention_debug_drop_unit": ([_i32], _i32),
     "mk_last_error": ([_vp], ctypes.c_char_p),
     "mk_destroy": ([_vp], None),
 }
@@ -278,6 +284,36 @@ def mk_validate_taskgraph(ctx, tasks, counts) -> int:
     return _lib.mk_validate_taskgraph(ctx, tasks.ctypes.data, tasks.shape[0], counts.ctypes.data, counts.size)
 
 
+def mk_build_taskgraph_tp(cfg: mk_config, n_ranks: int, device: int) -> int:
+    h = _vp()
+    _check(_lib.mk_build_taskgraph_tp(ctypes.byref(cfg), int(n_ranks), int(device), ctypes.byref(h)))
+    return h.value
+
+
+TP_FIELDS = ("rank", "kind", "layer", "sm", "row0", "nrows", "n_wait", "wait0", "wait1", "n_notify", "notify0",
+             "notify1", "remote", "row_lo", "row_hi")
+
+
+def mk_export_taskgraph_tp(ctx):
+    """Returns (tasks int32 [n, 15] with the columns TP_FIELDS, event_counts int32 [n_events])."""
+    import numpy as np
+    n = _lib.mk_export_taskgraph_tp(ctx, None, 0, None, 0)
+    if n < 0:
+        raise MkError(n, "mk_export_taskgraph_tp")
+    info = mk_get_graph_info(ctx)
+    tasks = np.zeros((n, 15), dtype=np.int32)
+    counts = np.zeros(info["n_events"], dtype=np.int32)
+    _lib.mk_export_taskgraph_tp(ctx, tasks.ctypes.data, n, counts.ctypes.data, counts.size)
+    return tasks, counts
+
+
+def mk_validate_taskgraph_tp(ctx, tasks, counts) -> int:
+    import numpy as np
+    tasks = np.ascontiguousarray(tasks, dtype=np.int32)
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    return _lib.mk_validate_taskgraph_tp(ctx, tasks.ctypes.data, tasks.shape[0], counts.ctypes.data, counts.size)
+
+
 def mk_attention_workspace_bytes(BH: int, d: int, L: int) -> int:
     return _lib.mk_attention_workspace_bytes(int(BH), int(d), int(L))
 
@@ -296,6 +332,20 @@ def mk_attention_decode_noalloc(q, k_t, v, o, BH: int, d: int, L: int, scale: fl
 
 def mk_attention_status(workspace, BH: int, d: int, L: int, stream=None) -> int:
     return _lib.mk_attention_status(_ptr(workspace), int(BH), int(d), int(L), _stream(stream))
+
+
+def mk_attention_noalloc_status(stream=None) -> int:
+    """MK_OK, or MK_ERR_DEVICE_TIMEOUT if a no-alloc call since the last status call had a device
+    wait run out (returned, not raised)."""
+    return _lib.mk_attention_noalloc_status(_stream(stream))
+
+
+def mk_attention_set_wait_timeout_ns(ns: int):
+    _check(_lib.mk_attention_set_wait_timeout_ns(int(ns)))
+
+
+def mk_attention_debug_drop_unit(unit: int):
+    _check(_lib.mk_attention_debug_drop_unit(int(unit)))
 
 
 def mk_last_error(ctx=None) -> str:
@@ -339,11 +389,15 @@ class Config:
 class Megakernel:
     """One model instance: task graph + torch-allocated weight arena, workspace and KV cache."""
 
-    def __init__(self, cfg: Config, weights=None, device: int = 0, stream=None):
+    def __init__(self, cfg: Config, weights=None, device: int = 0, stream=None, tp_ranks: int = 1):
+        """tp_ranks > 1: an emulated tensor-parallel model (mk_build_taskgraph_tp), every rank on
+        this device; kv_view() then has a leading rank axis."""
         import torch
         self.cfg = cfg
         self.device = device
-        self.ctx = mk_build_taskgraph(cfg.c(), device)
+        self.tp_ranks = tp_ranks
+        self.ctx = mk_build_taskgraph_tp(cfg.c(), tp_ranks, device) if tp_ranks > 1 else \
+            mk_build_taskgraph(cfg.c(), device)
         dev = torch.device("cuda", device)
         self.arena = torch.empty(mk_weight_arena_bytes(self.ctx), dtype=torch.uint8, device=dev)
         self.workspace = torch.zeros(mk_workspace_bytes(self.ctx), dtype=torch.uint8, device=dev)
@@ -358,8 +412,14 @@ class Megakernel:
         mk_load_weights(self.ctx, weights, self.arena, self.workspace, self.stream, self.cfg.n_layers)
 
     def kv_view(self):
-        """The cache as int16 bf16 bits [layer][K|V][max_batch][n_kv][max_seq][head_dim]."""
+        """The cache as int16 bf16 bits [layer][K|V][max_batch][n_kv][max_seq][head_dim]; with
+        tensor parallelism [rank][layer][K|V][1][n_kv / ranks][max_seq][head_dim]."""
         c = self.cfg
+        if self.tp_ranks > 1:
+            R = self.tp_ranks
+            per = c.n_layers * 2 * c.max_batch * (c.n_kv_heads // R) * c.max_seq * c.head_dim
+            return self.kv.view(-1)[: R * per].view(R, c.n_layers, 2, c.max_batch, c.n_kv_heads // R, c.max_seq,
+                                                   c.head_dim)
         return self.kv.view(c.n_layers, 2, c.max_batch, c.n_kv_heads, c.max_seq, c.head_dim)
 
     def prefill(self, tokens):

@@ -7,10 +7,14 @@
 //
 // Work split: the keys of all heads form BH * ceil(L/64) units of 64 keys; CTA c of G takes
 // units [c*U/G, (c+1)*U/G), so every SM streams the same number of bytes.  A TMA producer
-// warp keeps a 6-stage ring of (K^T tile [d][64], V tile [64][d]) fp16 tiles full; eight
-// compute warps turn each tile into scores, update a running (max, sum, acc) and, when a
-// head's units end inside the CTA, write one partial.  The last CTA to finish a head
-// (atomic arrival count) merges that head's partials and resets the count to zero.
+// warp keeps a 6-stage ring of (K^T tile [d][64], V tile [64][d]) fp16 tiles full, in unit
+// order.  The eight compute warps work independently: warp w takes the CTA's units of a head
+// round-robin (the head's first unit in the CTA, then every eighth), each with its own running
+// (max, sum, acc) -- lane l scores keys 2l and 2l+1 over all d, then owns d/32 output dims in
+// P.V -- and releases the stage it read.  Only at the end of a head's units in the CTA do the
+// warps meet: their partials are combined in shared memory into one partial per (CTA, head);
+// a head inside one CTA is written out directly, otherwise the last CTA to finish the head
+// (atomic arrival count) merges the CTAs' partials and resets the count to zero.
 //
 // L % 8 != 0 cannot be described to TMA (row stride must be a multiple of 16 bytes); those
 // shapes take a plain-load kernel (attention_plain) that needs no workspace.
@@ -20,6 +24,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <climits>
 #include <mutex>
 
 #include "mk_internal.h"
@@ -28,21 +34,22 @@
 namespace mk {
 namespace attn {
 
-constexpr int kUnit = 64;             // keys per unit
+constexpr int kUnit = 64;             // keys per unit (one ring stage)
 constexpr int kStages = 6;
 constexpr int kComputeWarps = 8;
 constexpr int kThreads = (kComputeWarps + 1) * 32;  // + producer warp
 constexpr int kMaxD = 128;
 
 struct Params {
-  const __half_raw* q;  // [BH][d]
+  const uint16_t* q;    // [BH][d] fp16
   float* o;             // [BH][d]
-  float* part;          // [BH][maxc][d + 2]
+  float* part;          // [BH][maxc][d + 2]: per-(head, CTA) partials (m, l, acc[d])
   uint32_t* cnt;        // [BH] arrival counts, zero between calls
-  uint32_t* err;        // error word: 0 = ok, else 1 + stage of the wait that ran out
+  uint32_t* err;        // error word: 0 = ok, else 1 + role of the first wait that ran out
   int BH, d, L, nu, U, G, maxc;
   float scale;
   uint64_t timeout_ns;
+  int drop_unit;        // test hook: the producer never loads this unit (-1 = none)
 };
 
 __host__ __device__ inline int unit_begin(int c, int U, int G) { return (int)(((long long)c * U) / G); }
@@ -61,17 +68,23 @@ __device__ __forceinline__ float h2f(uint16_t h) {
   return __half2float(__half(r));
 }
 
+__device__ __forceinline__ float2 h2f2(uint32_t w) {
+  __half2_raw r;
+  r.x = (unsigned short)(w & 0xffffu);
+  r.y = (unsigned short)(w >> 16);
+  return __half22float2(__half2(r));
+}
+
 struct Smem {
   alignas(128) uint16_t kt[kStages][kMaxD * kUnit];  // [d][64]
   alignas(128) uint16_t v[kStages][kUnit * kMaxD];   // [64][d]
-  float red[kComputeWarps][kUnit];                   // partial scores per warp
-  float p[kUnit];                                    // probabilities of the current tile
-  float acc_red[2048];                               // final per-key-group accumulators [VKG][d]
-  float alpha;                                       // rescale factor of the current tile
-  float m, l;                                        // running max / sum (warp 0 owns)
-  uint32_t last;                                     // this CTA merges head `last` when set
+  alignas(16) float qs[kComputeWarps][kMaxD];        // each warp's scaled q of its current head
+  alignas(16) float ps[kComputeWarps][kUnit];        // each warp's probabilities of its current unit
+  float wacc[kComputeWarps][kMaxD];                  // per-warp partial outputs at a head's end
+  float wm[kComputeWarps], wl[kComputeWarps];
+  uint32_t last;                                     // this CTA merges the head when set
   volatile uint32_t abort;                           // a wait ran out: every role stops waiting
-  uint32_t cabort;  // compute-role copy: written only before, and read only after, a compute barrier
+  int abort_epoch;  // first compute-barrier epoch whose barrier follows an abort (INT_MAX: none)
   alignas(8) uint64_t full[kStages];
   alignas(8) uint64_t empty[kStages];
 };
@@ -96,6 +109,17 @@ __device__ __forceinline__ void report_timeout(uint32_t* err, uint32_t code, vol
   atomicCAS(err, 0u, code);
 }
 
+// Compute-warp barrier.  Every compute warp passes the same sequence of barriers; `epoch`
+// counts them.  A warp whose wait ran out records (atomicMin) the epoch of the next barrier it
+// will reach; after barrier e every warp leaves iff the recorded epoch is <= e.  A value <= e
+// can only have been written before barrier e, so the decision is the same in every warp.
+__device__ __forceinline__ bool compute_bar(Smem& S, int& epoch) {
+  named_bar_sync(1, kComputeWarps * 32);
+  const bool stop = S.abort_epoch <= epoch;
+  ++epoch;
+  return stop;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_split_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
@@ -109,10 +133,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], kComputeWarps);
+      mbar_init(&S.empty[s], 1);  // the one warp that read the stage releases it
     }
     S.abort = 0;
-    S.cabort = 0;
+    S.abort_epoch = INT_MAX;
     fence_mbar_init();
   }
   __syncthreads();
@@ -132,9 +156,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           report_timeout(P.err, 1u, &S.abort);
           break;
         }
-        mbar_arrive_expect_tx(&S.full[stage], 2u * D * kUnit * 2u);
-        tma_load_3d(S.kt[stage], &map_k, j0, 0, h, &S.full[stage], pol);
-        tma_load_3d(S.v[stage], &map_v, 0, j0, h, &S.full[stage], pol);
+        if (u != P.drop_unit) {
+          mbar_arrive_expect_tx(&S.full[stage], 2u * D * kUnit * 2u);
+          tma_load_3d(S.kt[stage], &map_k, j0, 0, h, &S.full[stage], pol);
+          tma_load_3d(S.v[stage], &map_v, 0, j0, h, &S.full[stage], pol);
+        }
         ++issued;
         if (++stage == kStages) {
           stage = 0;
@@ -155,181 +181,167 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---------------- compute warps ----------------
-  constexpr int DG = D / 32;  // dims per thread in the score phase (4 or 2)
-  const int kg = tid & 7;     // score phase: 8-key group
-  const int dg = tid >> 3;    // score phase: dim group (0..31)
-  const int vdg = tid & (D / 8 - 1);  // PV phase: 8-dim group
-  const int vkg = tid / (D / 8);      // PV phase: key group
-  constexpr int VKG = 256 / (D / 8);  // key groups in PV phase (16 or 32)
-  constexpr int VK = kUnit / VKG;     // keys per thread in PV phase (4 or 2)
-
-  float qreg[DG];
-  float acc[8];
-  int stage = 0;
-  uint32_t phase = 0;
-  int cur_h = -1;
-
-  auto begin_head = [&](int h) {
-    cur_h = h;
+  constexpr int DL = D / 32;  // output dims per lane in P.V
+  int epoch = 0;
+  bool failed = false;  // this warp saw a wait run out (warp-uniform)
+  float* qs = S.qs[warp];
+  float* ps = S.ps[warp];
+  for (int hu0 = u0; hu0 < u1;) {
+    const int h = hu0 / P.nu;
+    const int hu1 = min(u1, (h + 1) * P.nu);  // this CTA's units of head h: [hu0, hu1)
+    // the warp's own copy of q (scaled), read back as broadcasts
+    {
+      const uint16_t* qh = P.q + (size_t)h * D + lane * DL;
 #pragma unroll
-    for (int i = 0; i < DG; ++i) qreg[i] = h2f(((const uint16_t*)P.q)[(size_t)h * D + dg * DG + i]) * P.scale;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    if (tid == 0) {
-      S.m = -INFINITY;
-      S.l = 0.f;
+      for (int i = 0; i < DL; ++i) qs[lane * DL + i] = h2f(__ldg(qh + i)) * P.scale;
     }
-  };
-
-  auto finish_head = [&]() {
-    // reduce acc over key groups, write this CTA's partial for head cur_h, count arrival
+    __syncwarp();
+    float m = -INFINITY, l = 0.f, acc[DL];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) S.acc_red[vkg * D + vdg * 8 + i] = acc[i];
-    named_bar_sync(1, 256);
-    const int h = cur_h;
-    const int cf = unit_owner(h * P.nu, P.U, P.G);
-    const int slot = c - cf;
-    float* part = P.part + ((size_t)h * P.maxc + slot) * (D + 2);
+    for (int i = 0; i < DL; ++i) acc[i] = 0.f;
+    for (int u = hu0 + warp; u < hu1; u += kComputeWarps) {
+      const int idx = u - u0, stage = idx % kStages;
+      const uint32_t parity = (uint32_t)(idx / kStages) & 1u;
+      bool ok = !failed && wait_bar(&S.full[stage], parity, P.timeout_ns, &S.abort);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (!failed && lane == 0) {
+          report_timeout(P.err, 2u, &S.abort);
+          atomicMin(&S.abort_epoch, epoch);
+        }
+        failed = true;
+        continue;
+      }
+      const int valid = min(kUnit, P.L - (u % P.nu) * kUnit);
+      // scores: lane owns keys 2*lane, 2*lane+1; row dd of the K^T tile holds 64 keys
+      const uint32_t* kt = reinterpret_cast<const uint32_t*>(S.kt[stage]) + lane;
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int dd = 0; dd < D; dd += 4) {
+        const float4 q4 = *reinterpret_cast<const float4*>(qs + dd);
+        const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 k2 = h2f2(kt[(dd + e) * (kUnit / 2)]);
+          sa[e] = fmaf(qv[e], k2.x, sa[e]);
+          sb[e] = fmaf(qv[e], k2.y, sb[e]);
+        }
+      }
+      float s0 = (sa[0] + sa[1]) + (sa[2] + sa[3]);
+      float s1 = (sb[0] + sb[1]) + (sb[2] + sb[3]);
+      if (2 * lane >= valid) s0 = -INFINITY;
+      if (2 * lane + 1 >= valid) s1 = -INFINITY;
+      float bm = fmaxf(s0, s1);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+      const float m_new = fmaxf(m, bm);  // finite: the unit holds at least one key
+      const float alpha = __expf(m - m_new);  // 0 on the first unit (m = -inf)
+      const float p0 = __expf(s0 - m_new), p1 = __expf(s1 - m_new);
+      float psum = p0 + p1;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+      l = fmaf(l, alpha, psum);
+      m = m_new;
+#pragma unroll
+      for (int i = 0; i < DL; ++i) acc[i] *= alpha;
+      *reinterpret_cast<float2*>(ps + 2 * lane) = make_float2(p0, p1);
+      __syncwarp();
+      // P.V: lane owns dims lane*DL .. lane*DL + DL - 1 (keys past L have p = 0 and zero rows)
+      const uint16_t* vt = S.v[stage] + lane * DL;
+#pragma unroll 4
+      for (int k = 0; k < kUnit; k += 4) {
+        const float4 p4 = *reinterpret_cast<const float4*>(ps + k);
+        const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if constexpr (DL == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(vt + (k + e) * D);
+            const float2 a = h2f2(w.x), b = h2f2(w.y);
+            acc[0] = fmaf(pv[e], a.x, acc[0]);
+            acc[1] = fmaf(pv[e], a.y, acc[1]);
+            acc[2] = fmaf(pv[e], b.x, acc[2]);
+            acc[3] = fmaf(pv[e], b.y, acc[3]);
+          } else {
+            const float2 a = h2f2(*reinterpret_cast<const uint32_t*>(vt + (k + e) * D));
+            acc[0] = fmaf(pv[e], a.x, acc[0]);
+            acc[1] = fmaf(pv[e], a.y, acc[1]);
+          }
+        }
+      }
+      __syncwarp();  // every lane's reads of the stage and of ps are done
+      if (lane == 0) mbar_arrive(&S.empty[stage]);
+    }
+    // end of the head's units in this CTA: combine the warps' partials
+    if (lane == 0) {
+      S.wm[warp] = m;
+      S.wl[warp] = l;
+    }
+#pragma unroll
+    for (int i = 0; i < DL; ++i) S.wacc[warp][lane * DL + i] = acc[i];
+    if (compute_bar(S, epoch)) return;
+    const int cf = unit_owner(h * P.nu, P.U, P.G), cl = unit_owner((h + 1) * P.nu - 1, P.U, P.G);
     if (tid < D) {
-      float s = 0.f;
-      for (int g = 0; g < VKG; ++g) s += S.acc_red[g * D + tid];
-      part[2 + tid] = s;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, S.wm[w]);
+      float ls = 0.f, as = 0.f;
+#pragma unroll
+      for (int w = 0; w < kComputeWarps; ++w) {
+        const float f = (S.wm[w] == -INFINITY) ? 0.f : __expf(S.wm[w] - M);  // warps without units add 0
+        ls = fmaf(f, S.wl[w], ls);
+        as = fmaf(f, S.wacc[w][tid], as);
+      }
+      if (cf == cl) {
+        P.o[(size_t)h * D + tid] = as / ls;  // the head lies inside this CTA
+      } else {
+        float* part = P.part + ((size_t)h * P.maxc + (c - cf)) * (D + 2);
+        part[2 + tid] = as;
+        if (tid == 0) {
+          part[0] = M;
+          part[1] = ls;
+        }
+      }
     }
-    if (tid == 0) {
-      part[0] = S.m;
-      part[1] = S.l;
-    }
-    named_bar_sync(1, 256);
-    if (tid == 0) {
-      __threadfence();
-      const int cl = unit_owner((h + 1) * P.nu - 1, P.U, P.G);
-      const uint32_t n = (uint32_t)(cl - cf + 1);
-      const uint32_t old = atom_acq_rel_gpu_add(&P.cnt[h], 1u);
-      S.last = (old + 1 == n) ? n : 0u;
-      if (old + 1 == n) P.cnt[h] = 0u;  // self-cleaning for the next call
-    }
-    named_bar_sync(1, 256);
-    if (S.last) {
-      __threadfence();
-      const int n = (int)S.last;
-      const float* base = P.part + (size_t)h * P.maxc * (D + 2);
-      if (tid < D) {
+    if (cf != cl) {
+      if (compute_bar(S, epoch)) return;
+      if (tid == 0) {
+        __threadfence();
+        const uint32_t n = (uint32_t)(cl - cf + 1);
+        const uint32_t old = atom_acq_rel_gpu_add(&P.cnt[h], 1u);
+        S.last = (old + 1 == n) ? n : 0u;
+        if (old + 1 == n) P.cnt[h] = 0u;  // self-cleaning for the next call
+      }
+      if (compute_bar(S, epoch)) return;
+      if (S.last && tid < D) {
+        __threadfence();
+        const int n = (int)S.last;
+        const float* base = P.part + (size_t)h * P.maxc * (D + 2);
         float M = -INFINITY;
         for (int i = 0; i < n; ++i) M = fmaxf(M, __ldcg(base + (size_t)i * (D + 2)));
         float num = 0.f, den = 0.f;
-        for (int i = 0; i < n; ++i) {
-          const float* pi = base + (size_t)i * (D + 2);
-          const float w = expf(__ldcg(pi) - M);
-          den += w * __ldcg(pi + 1);
-          num += w * __ldcg(pi + 2 + tid);
+        for (int i0 = 0; i0 < n; i0 += 8) {  // eight partials per L2 round trip
+          float mv[8], lv[8], av[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const bool in = i0 + k < n;
+            const float* pi = base + (size_t)(in ? i0 + k : 0) * (D + 2);
+            mv[k] = in ? __ldcg(pi) : -INFINITY;
+            lv[k] = in ? __ldcg(pi + 1) : 0.f;
+            av[k] = in ? __ldcg(pi + 2 + tid) : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float w = (mv[k] == -INFINITY) ? 0.f : __expf(mv[k] - M);
+            den = fmaf(w, lv[k], den);
+            num = fmaf(w, av[k], num);
+          }
         }
         P.o[(size_t)h * D + tid] = num / den;
       }
     }
-    named_bar_sync(1, 256);
-  };
-
-  for (int u = u0; u < u1; ++u) {
-    const int h = u / P.nu, j0 = (u % P.nu) * kUnit;
-    if (h != cur_h) {
-      if (cur_h >= 0) finish_head();
-      begin_head(h);
-    }
-    const int valid = min(kUnit, P.L - j0);
-    if (!wait_bar(&S.full[stage], phase, P.timeout_ns, &S.abort)) {
-      report_timeout(P.err, 2u, &S.abort);
-      S.cabort = 1u;  // every compute thread reaches the barrier below, then all leave together
-    }
-    // scores: thread (kg, dg) covers keys kg*8..+8 over dims dg*DG..+DG
-    const uint16_t* kt = S.kt[stage];
-    float sc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) sc[j] = 0.f;
-#pragma unroll
-    for (int i = 0; i < DG; ++i) {
-      const uint4 w = *reinterpret_cast<const uint4*>(kt + (dg * DG + i) * kUnit + kg * 8);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        __half2_raw hr;
-        hr.x = (unsigned short)(ws[j] & 0xffffu);
-        hr.y = (unsigned short)(ws[j] >> 16);
-        const float2 f = __half22float2(__half2(hr));
-        sc[2 * j] = fmaf(qreg[i], f.x, sc[2 * j]);
-        sc[2 * j + 1] = fmaf(qreg[i], f.y, sc[2 * j + 1]);
-      }
-    }
-    // reduce over the 4 dim groups inside the warp (lanes differing in bits 3,4)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      sc[j] += __shfl_xor_sync(0xffffffffu, sc[j], 8);
-      sc[j] += __shfl_xor_sync(0xffffffffu, sc[j], 16);
-    }
-    if (lane < 8) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) S.red[warp][lane * 8 + j] = sc[j];
-    }
-    named_bar_sync(1, 256);
-    if (S.cabort) return;  // uniform: cabort only changes before this barrier
-    if (warp == 0) {
-      // lane owns keys lane and lane+32
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int w = 0; w < kComputeWarps; ++w) {
-        s0 += S.red[w][lane];
-        s1 += S.red[w][lane + 32];
-      }
-      if (lane >= valid) s0 = -INFINITY;
-      if (lane + 32 >= valid) s1 = -INFINITY;
-      float mx = fmaxf(s0, s1);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_old = S.m;
-      const float m_new = fmaxf(m_old, mx);
-      const float p0 = expf(s0 - m_new), p1 = expf(s1 - m_new);
-      float ps = p0 + p1;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-      S.p[lane] = p0;
-      S.p[lane + 32] = p1;
-      __syncwarp();
-      if (lane == 0) {
-        const float a = expf(m_old - m_new);  // 0 on the first tile (m_old = -inf)
-        S.alpha = a;
-        S.l = S.l * a + ps;
-        S.m = m_new;
-      }
-    }
-    named_bar_sync(1, 256);
-    // PV: thread (vkg, vdg) covers keys vkg*VK..+VK over dims vdg*8..+8
-    const float a = S.alpha;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] *= a;
-    const uint16_t* vt = S.v[stage];
-#pragma unroll
-    for (int jj = 0; jj < VK; ++jj) {
-      const int j = vkg * VK + jj;
-      const float p = S.p[j];
-      const uint4 w = *reinterpret_cast<const uint4*>(vt + j * D + vdg * 8);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        __half2_raw hr;
-        hr.x = (unsigned short)(ws[e] & 0xffffu);
-        hr.y = (unsigned short)(ws[e] >> 16);
-        const float2 f = __half22float2(__half2(hr));
-        acc[2 * e] = fmaf(p, f.x, acc[2 * e]);
-        acc[2 * e + 1] = fmaf(p, f.y, acc[2 * e + 1]);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S.empty[stage]);
-    if (++stage == kStages) {
-      stage = 0;
-      phase ^= 1;
-    }
+    if (compute_bar(S, epoch)) return;  // S.wacc / S.last are reused by the next head
+    hu0 = hu1;
   }
-  if (cur_h >= 0) finish_head();
 }
 
 // Plain-load path for any L: one CTA per head, scores staged in shared memory in chunks.
@@ -436,8 +448,16 @@ static bool encode_map(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+std::atomic<uint64_t> g_attn_timeout_ns{2000000000ull};  // limit of every device wait
+std::atomic<int> g_attn_drop_unit{-1};                   // test hook (see mk_attention_debug_drop_unit)
+}  // namespace
+
+void attention_set_wait_timeout_ns(uint64_t ns) { g_attn_timeout_ns.store(ns); }
+void attention_debug_drop_unit(int unit) { g_attn_drop_unit.store(unit); }
+
 int attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d, int L,
-                     float scale, void* workspace, cudaStream_t stream, int n_sms, uint64_t timeout_ns,
+                     float scale, void* workspace, cudaStream_t stream, int n_sms, uint32_t* err_word,
                      std::string* err) {
   if (L % 8 != 0) {
     attn::attention_plain<<<BH, 256, 0, stream>>>(q, k_t, v, o, d, L, scale);
@@ -455,15 +475,16 @@ int attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, 
   int nu, U, G, maxc;
   attn_geometry(BH, d, L, n_sms, &nu, &U, &G, &maxc);
   attn::Params P;
-  P.q = reinterpret_cast<const __half_raw*>(q);
+  P.q = q;
   P.o = o;
   P.part = reinterpret_cast<float*>(workspace);
-  size_t part = (size_t)BH * maxc * (d + 2) * sizeof(float);
-  part = (part + 255) & ~(size_t)255;
-  P.cnt = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(workspace) + part);
-  P.err = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(workspace) +
-                                      attention_error_word_offset(BH, d, L, n_sms));
-  P.timeout_ns = timeout_ns;
+  P.cnt = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(workspace) +
+                                      attention_counter_offset(BH, d, L, n_sms));
+  P.err = err_word ? err_word
+                   : reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(workspace) +
+                                                 attention_error_word_offset(BH, d, L, n_sms));
+  P.timeout_ns = g_attn_timeout_ns.load();
+  P.drop_unit = g_attn_drop_unit.load();
   P.BH = BH;
   P.d = d;
   P.L = L;
@@ -503,10 +524,12 @@ int attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, 
 // Allocation-free variant.  Some callers may not call cudaMalloc: a serving process whose own
 // allocator reserved the device memory up front (a library allocation would fail or fragment
 // it), or a latency-critical loop where cudaMalloc/cudaFree would block and synchronise the
-// device.  For them the scratch of the split-KV attention (per-head partials, arrival counts,
-// error word) lives in one fixed array in the library's device image instead of a caller
-// buffer.  Every GPU that loads the library holds the array until the process exits.
+// device.  For them the scratch of the split-KV attention (per-head partials, arrival counts)
+// lives in one fixed array in the library's device image instead of a caller buffer, and the
+// error word in the array's last 256 bytes.  Every GPU that loads the library holds the array
+// until the process exits.
 constexpr size_t kNoAllocScratchBytes = 4u << 20;  // 4 MiB
+constexpr size_t kNoAllocErrOffset = kNoAllocScratchBytes - 256;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
@@ -520,11 +543,18 @@ size_t attention_noalloc_capacity() { return kNoAllocScratchBytes; }
 int attention_decode_noalloc(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d,
                              int L, float scale, cudaStream_t stream, std::string* err) {
   int dev = 0, n_sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices ||
+  if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&n_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
     *err = "no usable CUDA device";
     return MK_ERR_CUDA;
   }
+  if (dev < 0 || dev >= kNoAllocMaxDevices) {
+    *err = "mk_attention_decode_noalloc: device index " + std::to_string(dev) +
+           " exceeds the per-device address table (" + std::to_string(kNoAllocMaxDevices) + " devices)";
+    return MK_ERR_UNSUPPORTED;
+  }
+  // the per-call scratch ends with its own 256-byte error slot, which this variant does not
+  // use (its error word sits at a fixed place): it fits iff need <= the array's size
   const size_t need = attention_workspace_bytes(BH, d, L, n_sms);
   if (need > kNoAllocScratchBytes) {
     *err = "mk_attention_decode_noalloc: these sizes need " + std::to_string(need) +
@@ -548,16 +578,38 @@ int attention_decode_noalloc(const uint16_t* q, const uint16_t* k_t, const uint1
     }
     scratch = g_noalloc_ptr[dev];
   }
+  uint8_t* base = static_cast<uint8_t*>(scratch);
   if (L % 8 == 0) {
-    // the array keeps the previous call's contents: zero the arrival counts and error word
+    // the array keeps the previous call's contents: zero the arrival counts (the error word
+    // keeps the first timeout until attention_noalloc_status reads it)
     const size_t counters = attention_counter_offset(BH, d, L, n_sms);
-    const cudaError_t e = cudaMemsetAsync(static_cast<uint8_t*>(scratch) + counters, 0, need - counters, stream);
+    const cudaError_t e = cudaMemsetAsync(base + counters, 0, need - 256 - counters, stream);
     if (e != cudaSuccess) {
       *err = std::string("clearing the noalloc counters: ") + cudaGetErrorString(e);
       return MK_ERR_CUDA;
     }
   }
-  return attention_decode(q, k_t, v, o, BH, d, L, scale, scratch, stream, n_sms, 2000000000ull, err);
+  return attention_decode(q, k_t, v, o, BH, d, L, scale, scratch, stream, n_sms,
+                          reinterpret_cast<uint32_t*>(base + kNoAllocErrOffset), err);
+}
+
+int attention_noalloc_status(cudaStream_t stream, std::string* err) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  uint32_t word = 0;
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&word, g_noalloc_scratch, 4, kNoAllocErrOffset, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && word != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_noalloc_scratch, &zero, 4, kNoAllocErrOffset, cudaMemcpyHostToDevice);
+  }
+  if (e != cudaSuccess) {
+    *err = std::string("reading the noalloc error word: ") + cudaGetErrorString(e);
+    return MK_ERR_CUDA;
+  }
+  if (word != 0) {
+    *err = "mk_attention_decode_noalloc: a device wait timed out (its output is undefined)";
+    return MK_ERR_DEVICE_TIMEOUT;
+  }
+  return MK_OK;
 }
 
 }  // namespace mk

@@ -26,6 +26,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <cstring>
+
 #include "mk_internal.h"
 #include "mk_ptx.cuh"
 
@@ -155,7 +157,7 @@ __device__ __forceinline__ void gemv_source(const DecodeParams& P, const Task& t
   }
   switch (t.kind) {
     case TK_QKV: *off = lo.qkv; *row_bytes = (uint32_t)P.H * 2u; break;
-    case TK_OPROJ: *off = lo.o; *row_bytes = (uint32_t)P.H * 2u; break;
+    case TK_OPROJ: *off = lo.o; *row_bytes = (uint32_t)(P.nq * P.D) * 2u; break;  // K = the heads' width
     case TK_GATEUP: *off = lo.gu; *row_bytes = (uint32_t)P.H * 2u; break;
     case TK_DOWN: {  // K chunk t.aux of W_down: chunk-major, rows of kc = min(kdc, F - k0) weights
       const uint32_t k0 = (uint32_t)t.aux * (uint32_t)P.kdc;
@@ -210,11 +212,25 @@ __device__ __forceinline__ void warp_reduce_rows(float (&a)[V], float* out, int 
 // across lanes right away into S.red[warp][row * BM + b], and across warps at the end into
 // S.tot.  Also leaves the per-warp sums of x_b^2 in S.ssw for the fused norm.  Returns false
 // (for every worker thread alike) if a wait ran out.
-template <int NSEG, int RPS, int BM>
+// Tensor-parallel input of a GEMV: x = xsrc + add[0] + add[stride] + ... (n ranks' partial
+// rows) + add2[0] + add2[stride] + ... (n2 more), added in that order so every rank gets the
+// same bits; the sum's elements [mlo, mhi) (multiples of 8) are also stored to mat.
+struct XAdd {
+  const float* add;
+  int n;
+  const float* add2;
+  int n2;
+  size_t stride;
+  float* mat;
+  int mlo, mhi;
+};
+
+template <int NSEG, int RPS, int BM, bool TPX = false>
 __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe& pp, const uint8_t* ring,
                                           const float* __restrict__ xsrc,
                                           int xstride, int nb, const uint16_t* __restrict__ gain, int K, int nrows,
-                                          uint32_t row_bytes, uint32_t task_id, uint32_t& stall_ns) {
+                                          uint32_t row_bytes, uint32_t task_id, uint32_t& stall_ns,
+                                          const XAdd& xa = XAdd{nullptr, 0, nullptr, 0, 0, nullptr, 0, 0}) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // only the last segment can be partial or empty: K > (NSEG - 2) * kSegElems by construction
   const bool last_ok = (NSEG - 1) * kSegElems + tid * 8 < K;
@@ -229,8 +245,21 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
       float x[8];
       if ((s < NSEG - 1 || last_ok) && (BM == 1 || b < nb)) {
         const float* xb = xsrc + (size_t)b * xstride;
-        const float4 a = __ldcg(reinterpret_cast<const float4*>(xb + k));
-        const float4 c = __ldcg(reinterpret_cast<const float4*>(xb + k + 4));
+        float4 a = __ldcg(reinterpret_cast<const float4*>(xb + k));
+        float4 c = __ldcg(reinterpret_cast<const float4*>(xb + k + 4));
+        if constexpr (TPX) {
+          for (int r = 0; r < xa.n + xa.n2; ++r) {
+            const float* ad = (r < xa.n ? xa.add + (size_t)r * xa.stride : xa.add2 + (size_t)(r - xa.n) * xa.stride) + k;
+            const float4 u = __ldcg(reinterpret_cast<const float4*>(ad));
+            const float4 w = __ldcg(reinterpret_cast<const float4*>(ad + 4));
+            a.x += u.x; a.y += u.y; a.z += u.z; a.w += u.w;
+            c.x += w.x; c.y += w.y; c.z += w.z; c.w += w.w;
+          }
+          if (xa.mat && k >= xa.mlo && k < xa.mhi) {
+            *reinterpret_cast<float4*>(xa.mat + k) = a;
+            *reinterpret_cast<float4*>(xa.mat + k + 4) = c;
+          }
+        }
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
         x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
 #pragma unroll
@@ -937,17 +966,58 @@ __device__ __forceinline__ void announce_tokens(const DecodeParams& P, DSmem& S,
   if (threadIdx.x == 0) red_release_gpu_add(&P.ev[P.ev_tok], 1u);
 }
 
-template <int BM>
-__device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, const Task& t, int K, int st) {
+// Tensor parallel: every rank's best (value, vocab index) of the step, exchanged through the
+// ranks' slot arrays; each rank waits (bounded) for all of them and picks the same token.
+// False (for every worker alike) if the wait ran out.
+__device__ __forceinline__ bool tp_exchange_argmax(const DecodeParams& P, DSmem& S, int b, float& v, int& idx,
+                                                   int st) {
   const int tid = threadIdx.x;
+  if (tid == 0) {
+    const uint64_t w = ((uint64_t)__float_as_uint(v) << 32) | (uint32_t)idx;
+    for (int d = 0; d < P.tp_ranks; ++d) P.tp_lmx[d][(size_t)P.tp_rank * P.B + b] = w;
+    for (int d = 0; d < P.tp_ranks; ++d) red_release_sys_add(P.tp_ev[d] + P.ev_lmx, 1u);
+    // each rank raises the counter once per (step, sequence): sequence b of step e is complete
+    // at ((e - 1) * nb + b + 1) * ranks
+    const uint32_t target =
+        (((P.epoch + (uint32_t)st - 1u) * (uint32_t)P.nb) + (uint32_t)b + 1u) * (uint32_t)P.tp_ranks;
+    uint64_t t0 = 0;
+    for (uint32_t n = 1;; ++n) {
+      if ((int32_t)(ld_acquire_sys(&P.ev[P.ev_lmx]) - target) >= 0) break;
+      if ((n & 63u) == 0) {
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        else if (S.abort || now - t0 > P.timeout_ns) {
+          raise_error(P, S, DEV_ERR_WAIT_EVENT, P.ev_lmx, 0u);
+          S.cabort = 1u;
+          break;
+        }
+      }
+    }
+    if (!S.cabort) {
+      v = -INFINITY;
+      idx = 0x7fffffff;
+      for (int r = 0; r < P.tp_ranks; ++r) {
+        const uint64_t w2 = ld_acquire_sys_u64(P.tp_lmx[P.tp_rank] + (size_t)r * P.B + b);
+        argmax_merge(v, idx, __uint_as_float((uint32_t)(w2 >> 32)), (int)(uint32_t)w2);
+      }
+    }
+  }
+  worker_bar();
+  return !S.cabort;
+}
+
+template <int BM, bool TP>
+__device__ __forceinline__ bool epi_lmhead(const DecodeParams& P, DSmem& S, const Task& t, int K, int st) {
+  const int tid = threadIdx.x;
+  const int vs = TP ? P.tp_vfull : P.V, vb = TP ? P.tp_vbase : 0;  // logits stride, this shard's first row
   for (int b = 0; b < P.nb; ++b) {
     const float r = norm_factor(S, K, P.eps, b);
     float v = -INFINITY;
     int idx = 0x7fffffff;
     for (int i = tid; i < (int)t.nrows; i += kWorkerThreads) {
       const float lv = S.tot[i * BM + b] * r;
-      P.logits[(size_t)b * P.V + t.row0 + i] = lv;
-      argmax_merge(v, idx, lv, (int)t.row0 + i);
+      P.logits[(size_t)b * vs + vb + t.row0 + i] = lv;
+      argmax_merge(v, idx, lv, vb + (int)t.row0 + i);
     }
     block_argmax(S, v, idx);
     if (tid == 0) {
@@ -962,19 +1032,22 @@ __device__ __forceinline__ void epi_lmhead(const DecodeParams& P, DSmem& S, cons
   }
   worker_bar();
   if (S.flag) {
-    if (P.next_tokens) {
+    // every step exchanges (tensor parallel), even without next_tokens, so the counters stay in step
+    if (P.next_tokens || TP) {
       for (int b = 0; b < P.nb; ++b) {
         float v = -INFINITY;
         int idx = 0x7fffffff;
         for (int i = tid; i < P.n_lm; i += kWorkerThreads)
           argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
         block_argmax(S, v, idx);
-        if (tid == 0) P.next_tokens[(size_t)st * P.B + b] = idx;
+        if (TP && !tp_exchange_argmax(P, S, b, v, idx, st)) return false;
+        if (tid == 0 && P.next_tokens) P.next_tokens[(size_t)st * P.B + b] = idx;
         worker_bar();
       }
     }
     announce_tokens(P, S, st);
   }
+  return true;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1367,9 +1440,9 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
 // ---------------------------------------------------------------------------------------
 // QKN: the model has QK-norm (its own instantiations, so the plain kernels keep their registers).
 // DYN: run-time claims (projection tasks taken from per-op pools; TK_POOL queue entries).
-template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM, bool QKN, bool DYN>
-__global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBlockThreads, 1)
-    decode_kernel(const __grid_constant__ DecodeParams P) {
+// TP: tensor-parallel view (batch width 1, static queues): see DecodeParams.
+template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM, bool QKN, bool DYN, bool TP>
+__device__ __forceinline__ void decode_body(const DecodeParams& P) {
   constexpr bool TC = BM > kMaxDecodeBatch;  // tensor-core projection tiles
   constexpr int BMC = TC ? 1 : BM;            // CUDA-core GEMV batch width (unused when TC)
   constexpr int NST = ring_stages(TC);
@@ -1692,7 +1765,7 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
         const uint32_t target = tok ? P.epoch + (uint32_t)st - 1u : (P.epoch + (uint32_t)st) * P.ev_count[e];
         uint64_t t0 = 0;
         for (uint32_t n = 1;; ++n) {
-          if ((int32_t)(ld_acquire_gpu(&P.ev[e]) - target) >= 0) break;
+          if ((int32_t)((TP ? ld_acquire_sys(&P.ev[e]) : ld_acquire_gpu(&P.ev[e])) - target) >= 0) break;
           if ((n & 63u) == 0) {
             if (S.abort || *(volatile uint32_t*)&P.err[ERR_ABORT]) {
               S.abort = 1u;
@@ -1831,18 +1904,43 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       const uint16_t* gain = nullptr;
       int K = P.H, xstride = P.H;
       const size_t lay = (size_t)t.layer * P.B;
+      // tensor parallel: the residual stream is the last materialised copy plus every rank's
+      // partial rows of the projection that followed it
+      XAdd xa{nullptr, 0, nullptr, 0, (size_t)P.B * P.H, nullptr, 0, 0};
+      auto recv_of = [&](float* const* bufs, int layer) {
+        return bufs[P.tp_rank] + (size_t)layer * P.tp_ranks * P.B * P.H;
+      };
       switch (t.kind) {
         case TK_QKV:
           xs = P.x_in + lay * P.H;
           gain = reinterpret_cast<const uint16_t*>(P.arena + lo.attn_norm);
+          if (TP && t.layer > 0) {  // x_in[l] = x_mid[l-1] + the ranks' down rows of layer l-1
+            xs = P.x_mid + (lay - P.B) * P.H;
+            xa.add = recv_of(P.tp_recv_d, t.layer - 1);
+            xa.n = P.tp_ranks;
+          }
           break;
         case TK_OPROJ:
           xs = P.obuf + lay * P.nq * P.D;
-          xstride = P.nq * P.D;
+          K = xstride = P.nq * P.D;
           break;
         case TK_GATEUP:
           xs = P.x_mid + lay * P.H;
           gain = reinterpret_cast<const uint16_t*>(P.arena + lo.mlp_norm);
+          if (TP) {  // x_mid[l] = x_in[l] + the ranks' O rows, x_in[l] formed as in QKV; written here
+            if (t.layer > 0) {
+              xs = P.x_mid + (lay - P.B) * P.H;
+              xa.add = recv_of(P.tp_recv_d, t.layer - 1);
+              xa.n = P.tp_ranks;
+            } else {
+              xs = P.x_in;  // the embedding
+            }
+            xa.add2 = recv_of(P.tp_recv_o, t.layer);
+            xa.n2 = P.tp_ranks;
+            xa.mat = P.x_mid + lay * P.H;
+            xa.mlo = (int)t.index;
+            xa.mhi = (int)t.pad1;
+          }
           break;
         case TK_DOWN: {
           const int k0 = (int)t.aux * P.kdc;  // K chunk of the down projection
@@ -1854,6 +1952,11 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
         default:  // LM head
           xs = P.x_in + (size_t)P.L * P.B * P.H;
           gain = reinterpret_cast<const uint16_t*>(P.arena + P.off_fnorm);
+          if (TP) {
+            xs = P.x_mid + (size_t)(P.L - 1) * P.B * P.H;
+            xa.add = recv_of(P.tp_recv_d, P.L - 1);
+            xa.n = P.tp_ranks;
+          }
           break;
       }
       uint32_t rb;
@@ -1864,8 +1967,8 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
       const bool ok = (t.kind == TK_DOWN)
                           ? gemv_tile<NSEG_F, RPS_F, BMC>(P, S, pp, ring, xs, xstride, P.nb, gain, K, (int)t.nrows, rb,
                                                          i, stall)
-                          : gemv_tile<NSEG_H, RPS_H, BMC>(P, S, pp, ring, xs, xstride, P.nb, gain, K, (int)t.nrows, rb,
-                                                         i, stall);
+                          : gemv_tile<NSEG_H, RPS_H, BMC, TP>(P, S, pp, ring, xs, xstride, P.nb, gain, K, (int)t.nrows,
+                                                             rb, i, stall, xa);
       if (!ok) goto out;
       // this thread's (row, sequence) in the epilogues
       const int eb = tid % BMC, er = tid / BMC;
@@ -1875,8 +1978,13 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
         case TK_QKV: epi_qkv<BMC>(P, S, t, r, st); break;
         case TK_OPROJ:
           if (mine) {
-            const size_t at = (lay + eb) * P.H + t.row0 + er;
-            P.x_mid[at] = __ldcg(P.x_in + at) + S.tot[tid];
+            if constexpr (TP) {  // this rank's partial rows to every rank's receive buffer
+              const size_t at = (((size_t)t.layer * P.tp_ranks + P.tp_rank) * P.B + eb) * P.H + t.row0 + er;
+              for (int d = 0; d < P.tp_ranks; ++d) P.tp_recv_o[d][at] = S.tot[tid];
+            } else {
+              const size_t at = (lay + eb) * P.H + t.row0 + er;
+              P.x_mid[at] = __ldcg(P.x_in + at) + S.tot[tid];
+            }
           }
           break;
         case TK_GATEUP:
@@ -1887,7 +1995,10 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
           }
           break;
         case TK_DOWN:
-          if (mine) {
+          if (TP && mine) {
+            const size_t at = (((size_t)t.layer * P.tp_ranks + P.tp_rank) * P.B + eb) * P.H + t.row0 + er;
+            for (int d = 0; d < P.tp_ranks; ++d) P.tp_recv_d[d][at] = S.tot[tid];
+          } else if (mine) {
             // K chunk 0 starts from the residual; later chunks of the same rows ran earlier
             // in this queue, on this thread, and add to what it stored
             const size_t at = (lay + eb) * P.H + t.row0 + er;
@@ -1898,14 +2009,14 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
           break;
         default:
           notify = false;
-          epi_lmhead<BMC>(P, S, t, K, st);
+          if (!epi_lmhead<BMC, TP>(P, S, t, K, st)) goto out;
           break;
       }
     } else if (t.kind == TK_EMBED) {
       for (int b = 0; b < P.nb; ++b) {
         // step 0: the caller's tokens; later steps: the previous step's greedy pick
         int tok = (st == 0) ? __ldcg(P.tokens + b) : __ldcg(P.next_tokens + (size_t)(st - 1) * P.B + b);
-        if (tok < 0 || tok >= P.V) {  // never read outside the table: record and use row 0
+        if (tok < 0 || tok >= (TP ? P.tp_vfull : P.V)) {  // never read outside the table: record, use row 0
           if (tid == 0 && t.row0 == 0) atomicCAS(&P.err[ERR_CODE], 0u, (uint32_t)DEV_ERR_BAD_TOKEN);
           tok = 0;
         }
@@ -1927,8 +2038,14 @@ __global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBloc
     if (notify) {
       worker_bar();
       if (tid == 0) {
-        for (int k = 0; k < t.n_notify; ++k)
-          if ((int)t.notify[k] != P.drop_event) red_release_gpu_add(&P.ev[t.notify[k]], 1u);
+        for (int k = 0; k < t.n_notify; ++k) {
+          if ((int)t.notify[k] == P.drop_event) continue;
+          if (TP && (t.pad0 & 1u)) {  // remote-signal edge: the event on every rank
+            for (int d = 0; d < P.tp_ranks; ++d) red_release_sys_add(P.tp_ev[d] + t.notify[k], 1u);
+          } else {
+            red_release_gpu_add(&P.ev[t.notify[k]], 1u);
+          }
+        }
       }
     }
     if constexpr (DYN) {  // every worker read FIFO entry k: its slot can be reused
@@ -1945,6 +2062,20 @@ out:
   }
 }
 
+template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD, int BM, bool QKN, bool DYN>
+__global__ void __launch_bounds__(BM > kMaxDecodeBatch ? kTcBlockThreads : kBlockThreads, 1)
+    decode_kernel(const __grid_constant__ DecodeParams P) {
+  decode_body<NSEG_H, RPS_H, NSEG_F, RPS_F, HD, BM, QKN, DYN, false>(P);
+}
+
+// Several tensor-parallel ranks in one launch on one GPU: CTA b runs rank b / sms_per_rank's
+// queue with that rank's view.  On separate GPUs each rank would launch decode_body with its
+// own view, its peers' buffers reached through peer mappings.
+template <int NSEG_H, int RPS_H, int NSEG_F, int RPS_F, int HD>
+__global__ void __launch_bounds__(kBlockThreads, 1) decode_kernel_tp(const __grid_constant__ DecodeParamsTP T) {
+  decode_body<NSEG_H, RPS_H, NSEG_F, RPS_F, HD, 1, false, false, true>(T.r[blockIdx.x / T.sms_per_rank]);
+}
+
 // ---------------------------------------------------------------------------------------
 // Instantiations: (segments, rows per stage) for K = hidden and K = ffn.
 // One instantiation per weight-row shape class: (segments, rows per ring stage) of the
@@ -1958,10 +2089,14 @@ __host__ __device__ constexpr int stage_rows(int K) {
 // kDownChunk columns, so the K = ffn class is the chunk's.
 __host__ __device__ constexpr int down_k(int F, int BM) { return BM == 1 ? F : (F < kDownChunk ? F : kDownChunk); }
 #define MK_VARIANT(H, F, D, BM, QK, DY) \
-  {seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, BM, QK, DY}
+  {seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, BM, QK, DY, 0}
 #define MK_KERNEL(H, F, D, BM, QK, DY)                                                                           \
   (const void*)decode_kernel<seg_count(H), stage_rows(H), seg_count(down_k(F, BM)), stage_rows(down_k(F, BM)), D, \
                              BM, QK, DY>
+// tensor-parallel instantiations: F is one rank's share of the ffn
+#define MK_VARIANT_TP(H, F, D) {seg_count(H), stage_rows(H), seg_count(F), stage_rows(F), D, 1, 0, 0, 1}
+#define MK_KERNEL_TP(H, F, D) \
+  (const void*)decode_kernel_tp<seg_count(H), stage_rows(H), seg_count(F), stage_rows(F), D>
 static const Variant kVariants[] = {
     MK_VARIANT(4096, 14336, 128, 1, 0, 0),  // Llama-3-8B shape
     MK_VARIANT(4096, 11008, 128, 1, 0, 0),  // Chameleon-7B shape
@@ -1973,18 +2108,22 @@ static const Variant kVariants[] = {
     MK_VARIANT(256, 768, 64, 4, 0, 0),      // tiny decoder, 2..4 sequences
     MK_VARIANT(2048, 4096, 128, 4, 0, 0),
     MK_VARIANT(256, 256, 64, 4, 0, 0),
-    {0, 1, 0, 1, 128, kTcBatch, 0, 0},      // tensor-core projection tiles, 5..16 sequences, any hidden / ffn
-    {0, 1, 0, 1, 64, kTcBatch, 0, 0},
+    {0, 1, 0, 1, 128, kTcBatch, 0, 0, 0},   // tensor-core projection tiles, 5..16 sequences, any hidden / ffn
+    {0, 1, 0, 1, 64, kTcBatch, 0, 0, 0},
     // QK-norm models: Chameleon-7B shape and the tiny decoder, every batch width
     MK_VARIANT(4096, 11008, 128, 1, 1, 0),
     MK_VARIANT(256, 768, 64, 1, 1, 0),
     MK_VARIANT(4096, 4096, 128, 4, 1, 0),
     MK_VARIANT(256, 768, 64, 4, 1, 0),
-    {0, 1, 0, 1, 128, kTcBatch, 1, 0},
-    {0, 1, 0, 1, 64, kTcBatch, 1, 0},
+    {0, 1, 0, 1, 128, kTcBatch, 1, 0, 0},
+    {0, 1, 0, 1, 64, kTcBatch, 1, 0, 0},
     // run-time claims (scheduling variant): batch 1, Llama-3-8B shape and the tiny decoder
     MK_VARIANT(4096, 14336, 128, 1, 0, 1),
     MK_VARIANT(256, 768, 64, 1, 0, 1),
+    // tensor parallel, batch 1: the tiny decoder over 2 ranks, the Llama-3-8B shape over 2 and 4
+    MK_VARIANT_TP(256, 384, 64),
+    MK_VARIANT_TP(4096, 7168, 128),
+    MK_VARIANT_TP(4096, 3584, 128),
 };
 static const void* kFns[] = {
     MK_KERNEL(4096, 14336, 128, 1, false, false), MK_KERNEL(4096, 11008, 128, 1, false, false), MK_KERNEL(256, 768, 64, 1, false, false),
@@ -1998,14 +2137,15 @@ static const void* kFns[] = {
     (const void*)decode_kernel<1, 1, 1, 1, 128, kTcBatch, true, false>,
     (const void*)decode_kernel<1, 1, 1, 1, 64, kTcBatch, true, false>,
     MK_KERNEL(4096, 14336, 128, 1, false, true), MK_KERNEL(256, 768, 64, 1, false, true),
+    MK_KERNEL_TP(256, 384, 64), MK_KERNEL_TP(4096, 7168, 128), MK_KERNEL_TP(4096, 3584, 128),
 };
 static_assert(sizeof(kVariants) / sizeof(kVariants[0]) == sizeof(kFns) / sizeof(kFns[0]), "variant table");
 
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn, int dyn) {
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn, int dyn, int tp) {
   for (int i = 0; i < (int)(sizeof(kVariants) / sizeof(kVariants[0])); ++i) {
     const Variant& v = kVariants[i];
     if (v.nseg_h == nseg_h && v.rps_h == rps_h && v.nseg_f == nseg_f && v.rps_f == rps_f && v.head_dim == head_dim &&
-        v.bm == bm && v.qkn == qkn && v.dyn == dyn)
+        v.bm == bm && v.qkn == qkn && v.dyn == dyn && v.tp == tp)
       return i;
   }
   return -1;
@@ -2029,6 +2169,30 @@ int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t str
   }
   if (e != cudaSuccess) {
     *err = std::string("decode launch: ") + cudaGetErrorString(e);
+    return e == cudaErrorCooperativeLaunchTooLarge ? MK_ERR_NOT_RESIDENT : MK_ERR_CUDA;
+  }
+  return MK_OK;
+}
+
+int launch_decode_tp(int variant, const DecodeParams* views, int n_ranks, int sms_per_rank, cudaStream_t stream,
+                     std::string* err) {
+  if (variant < 0 || !kVariants[variant].tp || n_ranks < 1 || n_ranks > kMaxTpRanks || sms_per_rank < 1) {
+    *err = "no tensor-parallel kernel instantiation for this launch";
+    return MK_ERR_UNSUPPORTED;
+  }
+  DecodeParamsTP T;  // copied by the launch
+  std::memset(&T, 0, sizeof(T));
+  for (int r = 0; r < n_ranks; ++r) T.r[r] = views[r];
+  T.sms_per_rank = sms_per_rank;
+  const void* fn = kFns[variant];
+  const size_t smem = decode_smem_bytes(variant);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) {
+    void* args[] = {&T};
+    e = cudaLaunchCooperativeKernel(fn, dim3(n_ranks * sms_per_rank), dim3(kBlockThreads), args, smem, stream);
+  }
+  if (e != cudaSuccess) {
+    *err = std::string("tensor-parallel decode launch: ") + cudaGetErrorString(e);
     return e == cudaErrorCooperativeLaunchTooLarge ? MK_ERR_NOT_RESIDENT : MK_ERR_CUDA;
   }
   return MK_OK;

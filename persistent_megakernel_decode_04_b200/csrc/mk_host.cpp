@@ -91,6 +91,24 @@ struct mk_ctx {
   std::vector<double> op_weights[8];  // per projection kind; empty = sm_weights
   size_t task_cap = 0, lm_cap = 0; // workspace capacity for re-partitioned graphs
   std::string err;
+  // Tensor parallel.  A shard context (tp_ranks > 1, no tp_shards) is rank tp_rank's part of
+  // the model: 1/tp_ranks of the query and KV heads, of the ffn rows and of the vocabulary,
+  // the whole hidden size.  An emulated tensor-parallel context (tp_shards non-empty) hosts
+  // every rank's shard on one device in one launch; it owns the shards.
+  int tp_ranks = 1, tp_rank = 0;
+  int tp_vbase = 0, tp_vfull = 0;   // shard: first vocab row of the LM-head slice; full vocab
+  int ev_lmx = -1;                  // shard: the argmax-exchange event
+  size_t ws_recv_o = 0, ws_recv_d = 0, ws_lmx = 0, recv_o_bytes = 0;
+  std::vector<mk_ctx*> tp_shards;
+  int tp_sms = 0;                   // emulated: SMs per rank
+  std::vector<size_t> tp_arena_off, tp_ws_off, tp_kv_off;
+  size_t tp_ws_tasks = 0, tp_ws_qbegin = 0;  // emulated: the combined queues
+  std::vector<Task> tp_tasks;       // emulated: every rank's tasks, rank 0's SMs first
+  std::vector<int> tp_task_sm;      // their (global) SMs
+  std::vector<uint32_t> tp_qbegin;
+  ~mk_ctx() {
+    for (mk_ctx* sh : tp_shards) delete sh;
+  }
 };
 
 namespace {
@@ -476,13 +494,318 @@ std::vector<VTask> to_vtasks(const Graph& g) {
 }
 
 // ---------------------------------------------------------------------------------------
+// Validation of a tensor-parallel graph (every rank's tasks; used when an emulated
+// tensor-parallel context is built and by mk_validate_taskgraph_tp).  A task's events live on
+// its own rank; a remote-signal edge (remote = 1) raises the notified event on every rank.
+// Checks, per rank: thresholds equal the producers that reach the rank's counter; every op's
+// rows and every attention chunk covered once; the summed residual rows written once per
+// layer (gate/up writes x_mid); and, simulating every rank's
+// queues together, no deadlock and no task reading data before its producers -- on its own
+// rank or, for the receive buffers of the row-parallel projections, on every rank.
+struct TVTask {
+  int rank, kind, layer, sm, row0, nrows, n_wait, wait[2], n_notify, notify[2], remote, mlo, mhi;
+};
+
+int validate_tp(mk_ctx* c, const std::vector<TVTask>& T, const std::vector<uint32_t>& cnt) {
+  const mk_ctx* sh = c->tp_shards[0];
+  const mk_config& f = sh->cfg;  // one rank's shapes
+  const int R = c->tp_ranks, S = c->tp_sms, L = f.n_layers, nkv = f.n_kv_heads, B = f.max_batch, H = f.hidden;
+  const int nE = (int)cnt.size();
+  const int rpg = sh->rows_qkv / nkv;
+  char buf[256];
+  if (nE != sh->n_events) return fail(c, MK_ERR_INVALID_ARG, "event count array has the wrong length");
+  for (size_t i = 0; i < T.size(); ++i) {
+    const TVTask& t = T[i];
+    if (t.rank < 0 || t.rank >= R || t.sm < t.rank * S || t.sm >= (t.rank + 1) * S || t.n_wait < 0 || t.n_wait > 2 ||
+        t.n_notify < 0 || t.n_notify > 2 || t.layer < 0 || t.layer > L || (t.remote != 0 && t.remote != 1))
+      return fail(c, MK_ERR_INVALID_ARG, "task " + std::to_string(i) + ": field out of range");
+    for (int k = 0; k < t.n_wait; ++k)
+      if (t.wait[k] < 0 || t.wait[k] >= nE) return fail(c, MK_ERR_INVALID_ARG, "task wait event out of range");
+    for (int k = 0; k < t.n_notify; ++k)
+      if (t.notify[k] < 0 || t.notify[k] >= nE) return fail(c, MK_ERR_INVALID_ARG, "task notify event out of range");
+  }
+  // (b) thresholds, per rank
+  std::vector<uint32_t> produced((size_t)R * nE, 0);
+  {
+    std::vector<char> seen((size_t)R * nE * L * B * nkv + 1, 0);
+    for (const TVTask& t : T) {
+      for (int k = 0; k < t.n_notify; ++k) {
+        if (t.kind == TK_ATTN) {  // a (sequence, KV head) group notifies once, from its merge
+          if (t.layer >= L || t.row0 < 0 || t.row0 >= B * nkv) continue;
+          const size_t key = (((size_t)t.rank * nE + t.notify[k]) * L + t.layer) * B * nkv + t.row0;
+          if (seen[key]) continue;
+          seen[key] = 1;
+        }
+        for (int d = 0; d < R; ++d)
+          if (t.remote || d == t.rank) produced[(size_t)d * nE + t.notify[k]]++;
+      }
+      if (t.kind == TK_LMHEAD) produced[(size_t)t.rank * nE + sh->ev_lm]++;
+    }
+    for (int r = 0; r < R; ++r) {
+      produced[(size_t)r * nE + sh->ev_tok] = 1;                    // the rank's token pick
+      produced[(size_t)r * nE + sh->ev_lmx] = (uint32_t)(R * B);  // every rank's argmax exchange
+    }
+  }
+  for (int r = 0; r < R; ++r)
+    for (int e = 0; e < nE; ++e)
+      if (produced[(size_t)r * nE + e] != cnt[e]) {
+        snprintf(buf, sizeof buf, "rank %d event %d: threshold %u but %u producers per step", r, e, cnt[e],
+                 produced[(size_t)r * nE + e]);
+        return fail(c, MK_ERR_INVALID_ARG, buf);
+      }
+  // (c) coverage per rank: op rows, attention chunks, materialised residual rows
+  auto rows_of = [&](int kind) -> int {
+    switch (kind) {
+      case TK_EMBED: return H;
+      case TK_QKV: return sh->rows_qkv;
+      case TK_OPROJ: return H;
+      case TK_GATEUP: return sh->rows_gu;
+      case TK_DOWN: return H;
+      case TK_LMHEAD: return f.vocab;
+    }
+    return 0;
+  };
+  for (int r = 0; r < R; ++r) {
+    std::vector<std::vector<int>> cover((size_t)8 * (L + 1)), mat((size_t)L);
+    std::vector<std::vector<int>> attn_cover((size_t)L * B * nkv);
+    for (const TVTask& t : T) {
+      if (t.rank != r) continue;
+      if (t.kind == TK_ATTN) {
+        if (t.row0 < 0 || t.row0 >= B * nkv || t.layer >= L)
+          return fail(c, MK_ERR_INVALID_ARG, "attention task outside the (sequence, KV head) range");
+        attn_cover[(size_t)t.layer * B * nkv + t.row0].push_back(t.nrows);
+        continue;
+      }
+      if (t.kind < TK_EMBED || t.kind > TK_LMHEAD) return fail(c, MK_ERR_INVALID_ARG, "unknown task kind");
+      const int rows = rows_of(t.kind);
+      if (t.nrows <= 0 || t.nrows > sh->task_rows || t.row0 < 0 || t.row0 + t.nrows > rows)
+        return fail(c, MK_ERR_INVALID_ARG, "task rows out of range");
+      if ((t.kind == TK_QKV || t.kind == TK_GATEUP) && ((t.row0 | t.nrows) & 1))
+        return fail(c, MK_ERR_INVALID_ARG, "QKV/gate-up tasks must hold whole row pairs");
+      const int lay = (t.kind == TK_EMBED || t.kind == TK_LMHEAD) ? L : t.layer;
+      auto& v = cover[(size_t)t.kind * (L + 1) + lay];
+      if (v.empty()) v.assign(rows, 0);
+      for (int x = t.row0; x < t.row0 + t.nrows; ++x) v[x]++;
+      if (t.kind == TK_GATEUP) {
+        if (t.mlo < 0 || t.mhi < t.mlo || t.mhi > H || ((t.mlo | t.mhi) & 7))
+          return fail(c, MK_ERR_INVALID_ARG, "residual slice out of range or not a multiple of 8");
+        auto& m = mat[t.layer];
+        if (m.empty()) m.assign(H, 0);
+        for (int x = t.mlo; x < t.mhi; ++x) m[x]++;
+      }
+    }
+    for (int kind = TK_EMBED; kind <= TK_LMHEAD; ++kind) {
+      if (kind == TK_ATTN) continue;
+      for (int l = 0; l <= L; ++l) {
+        const bool per_layer = !(kind == TK_EMBED || kind == TK_LMHEAD);
+        if (per_layer == (l == L)) continue;
+        auto& v = cover[(size_t)kind * (L + 1) + l];
+        if ((int)v.size() != rows_of(kind)) return fail(c, MK_ERR_INVALID_ARG, "an op has no tasks on a rank");
+        for (int x = 0; x < (int)v.size(); ++x)
+          if (v[x] != 1) {
+            snprintf(buf, sizeof buf, "rank %d op kind %d layer %d: row %d covered %d times", r, kind, l, x, v[x]);
+            return fail(c, MK_ERR_INVALID_ARG, buf);
+          }
+      }
+    }
+    for (int l = 0; l < L; ++l) {
+      const auto& m = mat[l];
+      for (int x = 0; x < H; ++x)
+        if ((m.empty() ? 0 : m[x]) != 1) {
+          snprintf(buf, sizeof buf, "rank %d layer %d: residual row %d of x_mid written %d times", r, l, x,
+                   m.empty() ? 0 : m[x]);
+          return fail(c, MK_ERR_INVALID_ARG, buf);
+        }
+    }
+    for (int l = 0; l < L; ++l)
+      for (int bg = 0; bg < B * nkv; ++bg) {
+        auto v = attn_cover[(size_t)l * B * nkv + bg];
+        std::sort(v.begin(), v.end());
+        bool ok = (int)v.size() == sh->nch;
+        for (int i = 0; ok && i < (int)v.size(); ++i) ok = v[i] == i;
+        if (!ok) return fail(c, MK_ERR_INVALID_ARG, "attention chunks of a (sequence, KV head) incomplete");
+      }
+  }
+  // (d) + (e): every rank's queues together; categories and events per rank
+  const int CPL = nkv + 5, NC = 2 + L * CPL, NCA = R * NC, W = (NCA + 63) / 64;
+  auto cat_qkvg = [&](int r, int l, int g) { return r * NC + 1 + l * CPL + g; };
+  auto cat_of = [&](int r, int kind, int l) {
+    switch (kind) {
+      case TK_QKV: return r * NC + 1 + l * CPL + nkv;
+      case TK_ATTN: return r * NC + 1 + l * CPL + nkv + 1;
+      case TK_OPROJ: return r * NC + 1 + l * CPL + nkv + 2;
+      case TK_GATEUP: return r * NC + 1 + l * CPL + nkv + 3;
+      case TK_DOWN: return r * NC + 1 + l * CPL + nkv + 4;
+      case TK_LMHEAD: return r * NC + 1 + L * CPL;
+    }
+    return r * NC;  // embedding
+  };
+  std::vector<int> cat_size(NCA, 0), tmp;
+  auto cats_of_task = [&](const TVTask& t, std::vector<int>& out) {
+    out.clear();
+    out.push_back(cat_of(t.rank, t.kind, t.layer));
+    if (t.kind == TK_QKV)
+      for (int g = t.row0 / rpg; g <= (t.row0 + t.nrows - 1) / rpg; ++g) out.push_back(cat_qkvg(t.rank, t.layer, g));
+  };
+  for (const TVTask& t : T) {
+    cats_of_task(t, tmp);
+    for (int x : tmp) cat_size[x]++;
+  }
+  const int NS = R * S;
+  std::vector<std::vector<int>> q(NS);
+  for (size_t i = 0; i < T.size(); ++i) q[T[i].sm].push_back((int)i);
+  std::vector<size_t> head(NS, 0);
+  std::vector<uint32_t> ctr((size_t)R * nE, 0);
+  std::vector<uint64_t> Gb(W, 0), Fe((size_t)R * nE * W, 0);
+  std::vector<int> ev_ncat((size_t)R * nE * NCA, 0);
+  std::vector<int> attn_arrive((size_t)R * L * B * nkv, 0);
+  std::vector<uint64_t> attn_acc((size_t)R * L * B * nkv * W, 0);
+  std::vector<std::vector<uint64_t>> smG(NS, std::vector<uint64_t>(W, 0));
+  auto setbit = [&](uint64_t* bs, int x) { bs[x >> 6] |= 1ull << (x & 63); };
+  auto hasbit = [&](const uint64_t* bs, int x) { return (bs[x >> 6] >> (x & 63)) & 1ull; };
+  auto fire = [&](int r, int e, const uint64_t* contrib, const std::vector<int>& cats_done) {
+    const size_t ge = (size_t)r * nE + e;
+    ctr[ge]++;
+    for (int w = 0; w < W; ++w) Fe[ge * W + w] |= contrib[w];
+    for (int x : cats_done)
+      if (++ev_ncat[ge * NCA + x] == cat_size[x]) setbit(&Fe[ge * W], x);
+  };
+  size_t executed = 0;
+  bool progress = true;
+  while (progress) {
+    progress = false;
+    for (int sm = 0; sm < NS; ++sm) {
+      while (head[sm] < q[sm].size()) {
+        const int i = q[sm][head[sm]];
+        const TVTask& t = T[i];
+        const int r = t.rank, l = t.layer;
+        bool ready = true;
+        for (int k = 0; k < t.n_wait; ++k)
+          if (ctr[(size_t)r * nE + t.wait[k]] < cnt[t.wait[k]]) ready = false;
+        if (!ready) break;
+        for (int w = 0; w < W; ++w) Gb[w] = smG[sm][w];
+        for (int k = 0; k < t.n_wait; ++k)
+          for (int w = 0; w < W; ++w) Gb[w] |= Fe[((size_t)r * nE + t.wait[k]) * W + w];
+        std::vector<int> need;
+        auto all_ranks = [&](int kind, int layer) {
+          for (int d = 0; d < R; ++d) need.push_back(cat_of(d, kind, layer));
+        };
+        switch (t.kind) {
+          case TK_QKV:
+            if (l == 0) {
+              need.push_back(cat_of(r, TK_EMBED, 0));
+            } else {
+              all_ranks(TK_DOWN, l - 1);                    // the ranks' down rows
+              need.push_back(cat_of(r, TK_GATEUP, l - 1));  // x_mid[l-1], materialised by this rank
+            }
+            break;
+          case TK_ATTN: need.push_back(cat_qkvg(r, l, t.row0 % nkv)); break;
+          case TK_OPROJ: need.push_back(cat_of(r, TK_ATTN, l)); break;
+          case TK_GATEUP:
+            all_ranks(TK_OPROJ, l);  // the ranks' O rows
+            if (l == 0) {
+              need.push_back(cat_of(r, TK_EMBED, 0));
+            } else {                                        // x_in[l], formed as in QKV
+              all_ranks(TK_DOWN, l - 1);
+              need.push_back(cat_of(r, TK_GATEUP, l - 1));
+            }
+            break;
+          case TK_DOWN: need.push_back(cat_of(r, TK_GATEUP, l)); break;
+          case TK_LMHEAD:
+            all_ranks(TK_DOWN, L - 1);
+            need.push_back(cat_of(r, TK_GATEUP, L - 1));
+            break;
+        }
+        for (int x : need)
+          if (!hasbit(Gb.data(), x)) {
+            snprintf(buf, sizeof buf, "rank %d task %d (kind %d layer %d) may read data before its producers finish",
+                     r, i, t.kind, l);
+            return fail(c, MK_ERR_INVALID_ARG, buf);
+          }
+        cats_of_task(t, tmp);
+        if (t.kind == TK_ATTN) {
+          const size_t key = ((size_t)r * L + l) * B * nkv + t.row0;
+          uint64_t* acc = &attn_acc[key * W];
+          for (int w = 0; w < W; ++w) acc[w] |= Gb[w];
+          if (++attn_arrive[key] == sh->nch) {
+            std::vector<int> done(sh->nch, cat_of(r, TK_ATTN, l));
+            for (int k = 0; k < t.n_notify; ++k)
+              for (int d = 0; d < R; ++d)
+                if (t.remote || d == r) fire(d, t.notify[k], acc, done);
+          }
+        } else {
+          for (int k = 0; k < t.n_notify; ++k)
+            for (int d = 0; d < R; ++d)
+              if (t.remote || d == r) fire(d, t.notify[k], Gb.data(), tmp);
+        }
+        for (int w = 0; w < W; ++w) smG[sm][w] = Gb[w];
+        head[sm]++;
+        executed++;
+        progress = true;
+      }
+    }
+  }
+  if (executed != T.size()) {
+    for (int sm = 0; sm < NS; ++sm)
+      if (head[sm] < q[sm].size()) {
+        snprintf(buf, sizeof buf, "deadlock: SM %d (rank %d) blocked at its task %zu", sm, sm / S, head[sm]);
+        return fail(c, MK_ERR_INVALID_ARG, buf);
+      }
+  }
+  return MK_OK;
+}
+
+std::vector<TVTask> tp_vtasks(const mk_ctx* c) {
+  std::vector<TVTask> v;
+  for (size_t i = 0; i < c->tp_tasks.size(); ++i) {
+    const Task& t = c->tp_tasks[i];
+    const int sm = c->tp_task_sm[i];
+    TVTask x;
+    x.rank = sm / c->tp_sms;
+    x.kind = t.kind;
+    x.layer = t.layer;
+    x.sm = sm;
+    x.row0 = (int)t.row0;
+    x.nrows = t.kind == TK_ATTN ? (int)t.aux : (int)t.nrows;
+    x.n_wait = t.n_wait;
+    x.wait[0] = (int)t.wait[0];
+    x.wait[1] = (int)t.wait[1];
+    x.n_notify = t.n_notify;
+    x.notify[0] = (int)t.notify[0];
+    x.notify[1] = (int)t.notify[1];
+    x.remote = (t.kind == TK_OPROJ || t.kind == TK_DOWN) ? (t.pad0 & 1) : 0;
+    x.mlo = t.kind == TK_GATEUP ? (int)t.index : 0;
+    x.mhi = t.kind == TK_GATEUP ? (int)t.pad1 : 0;
+    v.push_back(x);
+  }
+  return v;
+}
+
+// Tensor parallel: the tasks of op `kind` in layer l (queue order, SM 0 first) share out the
+// rows [0, H) of the residual sum they form, each writing its slice [index, pad1) (multiples
+// of 8, so whole 8-element groups of a GEMV thread's input).
+void share_rows(std::vector<std::vector<Task>>& q, int kind, int l, int H) {
+  std::vector<Task*> ts;
+  for (auto& v : q)
+    for (auto& t : v)
+      if (t.kind == kind && t.layer == l) ts.push_back(&t);
+  const int n = (int)ts.size();
+  for (int j = 0; j < n; ++j) {
+    ts[j]->index = (uint32_t)((long long)H * j / n / 8 * 8);
+    ts[j]->pad1 = (uint32_t)(j + 1 == n ? H : (long long)H * (j + 1) / n / 8 * 8);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
 int build_graph(mk_ctx* c) {
   const mk_config& f = c->cfg;
   const int L = f.n_layers, nkv = f.n_kv_heads, D = f.head_dim, n = c->n_sms;
   const int B = f.max_batch;
-  c->n_events = 1 + L * (nkv + 4) + 2;
-  c->ev_lm = c->n_events - 2;
-  c->ev_tok = c->n_events - 1;  // tokens picked: a later step of a multi-step launch waits on it
+  const bool tp = c->tp_ranks > 1;
+  c->n_events = 1 + L * (nkv + 4) + 2 + (tp ? 1 : 0);
+  c->ev_lm = 1 + L * (nkv + 4);
+  c->ev_tok = c->ev_lm + 1;  // tokens picked: a later step of a multi-step launch waits on it
+  c->ev_lmx = tp ? c->ev_lm + 2 : -1;  // tensor parallel: every rank's argmax partial arrived
   std::vector<uint32_t> evc(c->n_events, 0);
   std::vector<std::vector<Task>> q(n);
   const int rpg = (c->G + 2) * D;
@@ -656,7 +979,8 @@ int build_graph(mk_ctx* c) {
         Task t = gemv_task(TK_OPROJ, l, o_pl, s, j);
         add_wait(t, ev_attn(c, l));
         add_notify(t, ev_o(c, l));
-        evc[ev_o(c, l)]++;
+        if (tp) t.pad0 = 1;  // remote-signal edge: the partial rows go to every rank
+        evc[ev_o(c, l)] += tp ? (uint32_t)c->tp_ranks : 1u;
         q[s].push_back(t);
       }
     for (int s = 0; s < n; ++s)
@@ -667,6 +991,7 @@ int build_graph(mk_ctx* c) {
         evc[ev_gu(c, l)]++;
         q[s].push_back(t);
       }
+    if (tp) share_rows(q, TK_GATEUP, l, f.hidden);  // each task writes a slice of x_mid[l]
     for (int s = 0; s < n; ++s)
       for (int j = 0; j < (int)d_pl.parts[s].size(); ++j)
         for (int kc = 0; kc < c->ndc; ++kc) {  // K chunks of the same rows run back to back
@@ -674,7 +999,8 @@ int build_graph(mk_ctx* c) {
           t.aux = (uint16_t)(c->tc ? t.aux : kc);
           add_wait(t, ev_gu(c, l));
           add_notify(t, ev_down(c, l));
-          evc[ev_down(c, l)]++;
+          if (tp) t.pad0 = 1;
+          evc[ev_down(c, l)] += tp ? (uint32_t)c->tp_ranks : 1u;
           q[s].push_back(t);
         }
   }
@@ -691,6 +1017,7 @@ int build_graph(mk_ctx* c) {
     c->n_lm = c->tc ? c->tc_tiles[TK_LMHEAD] : idx;
     evc[c->ev_lm] = (uint32_t)c->n_lm;
     evc[c->ev_tok] = 1u;
+    if (tp) evc[c->ev_lmx] = (uint32_t)(c->tp_ranks * f.max_batch);  // one exchange per rank and sequence
   }
   if (dyn) {
     // every SM ends its step with a static LM-head task (the claim counters of a step are
@@ -740,6 +1067,7 @@ int build_graph(mk_ctx* c) {
     for (auto& t : pool_tasks) c->g.tasks.push_back({t, -1});
     return MK_OK;
   }
+  if (tp) return MK_OK;  // a shard is validated together with the other ranks (validate_tp)
   return validate(c, to_vtasks(c->g), evc);
 }
 
@@ -751,7 +1079,7 @@ void layout(mk_ctx* c) {
   uint64_t o = 0;
   c->loff.resize(L);
   c->off_embed = o;
-  o = align256(o + (uint64_t)f.vocab * H * 2);
+  o = align256(o + (uint64_t)(c->tp_ranks > 1 ? c->tp_vfull : f.vocab) * H * 2);  // the whole table on every rank
   // bytes of one projection: row-major, or whole kTcRows x kTcUnitK blocks (tensor-core)
   auto mat = [&](int kind, int rows, int K) -> uint64_t {
     if (c->tc) return (uint64_t)c->tc_tiles[kind] * c->tc_nk[kind] * kSlotBytes;
@@ -824,6 +1152,13 @@ void layout(mk_ctx* c) {
   c->pf_rows = (int)std::min<long long>(1024, (long long)B * f.max_seq);
   const long long per_row = (long long)H * 2 + ycols + (long long)nq * D * 2 + F;
   c->ws_pf = take((size_t)c->pf_rows * per_row * 4);
+  if (c->tp_ranks > 1) {
+    // receive buffers of the row-parallel projections [L][ranks][B][H] and the argmax slots
+    c->recv_o_bytes = (size_t)L * c->tp_ranks * B * H * 4;
+    c->ws_recv_o = take(c->recv_o_bytes);
+    c->ws_recv_d = take(c->recv_o_bytes);
+    c->ws_lmx = take((size_t)c->tp_ranks * B * 8);
+  }
   c->ws_bytes = w;
   c->kv_bytes = (size_t)L * 2 * B * nkv * f.max_seq * D * 2;
 }
@@ -920,47 +1255,10 @@ int upload_graph(mk_ctx* c, uint8_t* W) {
   return MK_OK;
 }
 
-}  // namespace
-
-namespace mk {
-TensorMapEncodeFn get_tensor_map_encoder() {
-  static TensorMapEncodeFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<TensorMapEncodeFn>(p);
-  }
-  return fn;
-}
-}  // namespace mk
-
-// =========================================================================================
-extern "C" {
-
-int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
-  if (!out) return fail(nullptr, MK_ERR_INVALID_ARG, "out is NULL");
-  *out = nullptr;
-  std::string why;
-  int rc = check_config(cfg, &why);
-  if (rc) return fail(nullptr, rc, why);
-  mk_ctx* c = new mk_ctx();
-  c->cfg = *cfg;
-  c->device = device;
-  if (device >= 0) {
-    int n = 0;
-    cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
-    if (e != cudaSuccess) {
-      delete c;
-      return fail(nullptr, MK_ERR_CUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
-    }
-    c->n_sms = n;
-  } else {
-    c->n_sms = 148;  // planning without a device: a B200's SM count
-  }
+// Everything after the config, device and SM count are set: kernel geometry, the task
+// graph and the arena / workspace layout.  Tensor-parallel shards also come here (their
+// tp_* fields set first).
+int init_ctx(mk_ctx* c) {
   const mk_config& f = c->cfg;
   c->G = f.n_q_heads / f.n_kv_heads;
   c->rows_qkv = (f.n_q_heads + 2 * f.n_kv_heads) * f.head_dim;
@@ -985,10 +1283,8 @@ int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
   c->rps_f = pow2_floor(std::min(kRpsMax, kSlotBytes / (c->kdc * 2)));
   // the GEMV takes every segment but the last of a K chunk as full
   const bool ragged_chunk = c->ndc > 1 && f.ffn - (c->ndc - 1) * c->kdc < (c->nseg_f - 1) * kSegElems;
-  if (!c->tc && ((f.max_batch == 1 && f.ffn * 2 > kSlotBytes) || f.hidden * 2 > kSlotBytes || ragged_chunk)) {
-    delete c;
-    return fail(nullptr, MK_ERR_UNSUPPORTED, "a weight row does not fit one ring stage");
-  }
+  if (!c->tc && ((f.max_batch == 1 && f.ffn * 2 > kSlotBytes) || f.hidden * 2 > kSlotBytes || ragged_chunk))
+    return fail(c, MK_ERR_UNSUPPORTED, "a weight row does not fit one ring stage");
   if (c->tc) {
     // tiles of kTcRows rows, K in units of kTcUnitK (rows and K past the end are zero padding)
     const int H = f.hidden;
@@ -1009,17 +1305,152 @@ int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
     c->n_tile_ids = base;
     c->variant = find_decode_variant(0, 1, 0, 1, f.head_dim, kTcBatch, f.qk_norm, 0);
   } else {
-    c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm, f.qk_norm, 0);
+    c->variant = find_decode_variant(c->nseg_h, c->rps_h, c->nseg_f, c->rps_f, f.head_dim, c->bm, f.qk_norm, 0,
+                                     c->tp_ranks > 1 ? 1 : 0);
   }
   c->sm_weights.assign(c->n_sms, 1.0);
-  rc = build_graph(c);
+  if (int rc = build_graph(c)) return rc;
+  layout(c);
+  c->pos.assign(f.max_batch, 0);
+  return MK_OK;
+}
+
+}  // namespace
+
+namespace mk {
+TensorMapEncodeFn get_tensor_map_encoder() {
+  static TensorMapEncodeFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<TensorMapEncodeFn>(p);
+  }
+  return fn;
+}
+}  // namespace mk
+
+
+namespace {
+// Emulated tensor parallel: each rank's shard of the host weights (heads, ffn rows, vocab rows;
+// the O and down projections' column slices copied out), loaded into its arena and workspace
+// regions; then every rank's queues into the combined arrays the kernel walks.
+int tp_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, void* workspace, void* stream) {
+  const mk_config& f = c->cfg;
+  const int R = c->tp_ranks, L = f.n_layers, H = f.hidden, D = f.head_dim;
+  const int nq_l = f.n_q_heads / R, nkv_l = f.n_kv_heads / R, F_l = f.ffn / R, V_l = f.vocab / R;
+  if (!w->embed || !w->lm_head || !w->final_norm || !w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo ||
+      !w->mlp_norm || !w->wg || !w->wu || !w->wd)
+    return fail(c, MK_ERR_INVALID_ARG, "a weight pointer is NULL");
+  if ((reinterpret_cast<uintptr_t>(weight_arena) | reinterpret_cast<uintptr_t>(workspace)) & 255)
+    return fail(c, MK_ERR_INVALID_ARG, "arena and workspace must be 256-byte aligned");
+  uint8_t* A = static_cast<uint8_t*>(weight_arena);
+  uint8_t* W = static_cast<uint8_t*>(workspace);
+  for (int r = 0; r < R; ++r) {
+    std::vector<const uint16_t*> wq(L), wk(L), wv(L), wo(L), wg(L), wu(L), wd(L);
+    std::vector<std::vector<uint16_t>> wo_s(L), wd_s(L);
+    for (int l = 0; l < L; ++l) {
+      if (!w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->wg[l] || !w->wu[l] || !w->wd[l])
+        return fail(c, MK_ERR_INVALID_ARG, "a per-layer weight pointer is NULL");
+      wq[l] = w->wq[l] + (size_t)r * nq_l * D * H;   // rows of this rank's query heads
+      wk[l] = w->wk[l] + (size_t)r * nkv_l * D * H;  // ... KV heads
+      wv[l] = w->wv[l] + (size_t)r * nkv_l * D * H;
+      wg[l] = w->wg[l] + (size_t)r * F_l * H;        // ffn rows
+      wu[l] = w->wu[l] + (size_t)r * F_l * H;
+      wo_s[l].resize((size_t)H * nq_l * D);          // columns of this rank's heads
+      wd_s[l].resize((size_t)H * F_l);               // columns of its ffn rows
+      for (int i = 0; i < H; ++i) {
+        std::memcpy(&wo_s[l][(size_t)i * nq_l * D], w->wo[l] + (size_t)i * f.n_q_heads * D + (size_t)r * nq_l * D,
+                    (size_t)nq_l * D * 2);
+        std::memcpy(&wd_s[l][(size_t)i * F_l], w->wd[l] + (size_t)i * f.ffn + (size_t)r * F_l, (size_t)F_l * 2);
+      }
+      wo[l] = wo_s[l].data();
+      wd[l] = wd_s[l].data();
+    }
+    mk_host_weights hw = *w;
+    hw.lm_head = w->lm_head + (size_t)r * V_l * H;  // this rank's vocab rows; the embedding stays whole
+    hw.wq = wq.data();
+    hw.wk = wk.data();
+    hw.wv = wv.data();
+    hw.wo = wo.data();
+    hw.wg = wg.data();
+    hw.wu = wu.data();
+    hw.wd = wd.data();
+    mk_ctx* sh = c->tp_shards[r];
+    if (int rc = mk_load_weights(sh, &hw, A + c->tp_arena_off[r], W + c->tp_ws_off[r], stream))
+      return fail(c, rc, "rank " + std::to_string(r) + ": " + sh->err);
+  }
+  if (!cuda_ok(c, cudaMemcpy(W + c->tp_ws_tasks, c->tp_tasks.data(), c->tp_tasks.size() * sizeof(Task),
+                             cudaMemcpyHostToDevice), "task upload") ||
+      !cuda_ok(c, cudaMemcpy(W + c->tp_ws_qbegin, c->tp_qbegin.data(), c->tp_qbegin.size() * 4,
+                             cudaMemcpyHostToDevice), "queue upload"))
+    return MK_ERR_CUDA;
+  c->arena = A;
+  c->ws = W;
+  c->loaded = true;
+  c->epoch = 0;
+  return MK_OK;
+}
+
+// Every rank's counters back to zero (the epoch restarts); the error word is rank 0's.
+int tp_reset_counters(mk_ctx* c) {
+  for (mk_ctx* sh : c->tp_shards)
+    if (!cuda_ok(c, cudaMemset(sh->ws + sh->ws_ev, 0, sh->ev_bytes), "counter reset") ||
+        !cuda_ok(c, cudaMemset(sh->ws + sh->ws_acnt, 0, sh->acnt_bytes), "counter reset") ||
+        !cuda_ok(c, cudaMemset(sh->ws + sh->ws_err, 0, 16), "error reset"))
+      return MK_ERR_CUDA;
+  if (!cuda_ok(c, cudaDeviceSynchronize(), "reset sync")) return MK_ERR_CUDA;
+  c->epoch = 0;
+  return MK_OK;
+}
+
+int tp_sync_status(mk_ctx* c) {
+  mk_ctx* s0 = c->tp_shards[0];
+  uint32_t e[4];
+  if (!cuda_ok(c, cudaMemcpy(e, s0->ws + s0->ws_err, 16, cudaMemcpyDeviceToHost), "error read")) return MK_ERR_CUDA;
+  if (e[ERR_CODE] == 0) return MK_OK;
+  if (e[ERR_CODE] == DEV_ERR_BAD_TOKEN && e[ERR_ABORT] == 0) {
+    cudaMemset(s0->ws + s0->ws_err, 0, 16);
+    return fail(c, MK_ERR_INVALID_ARG, "a token id was outside [0, vocab); row 0 was used");
+  }
+  char buf[160];
+  snprintf(buf, sizeof buf, "device wait timed out (kind %u, at %u, task %u)", e[ERR_CODE], e[ERR_WHERE], e[ERR_TASK]);
+  if (int rc = tp_reset_counters(c)) return rc;
+  return fail(c, MK_ERR_DEVICE_TIMEOUT, buf);
+}
+}  // namespace
+// =========================================================================================
+extern "C" {
+
+int mk_build_taskgraph(const mk_config* cfg, int device, mk_ctx** out) {
+  if (!out) return fail(nullptr, MK_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  std::string why;
+  int rc = check_config(cfg, &why);
+  if (rc) return fail(nullptr, rc, why);
+  mk_ctx* c = new mk_ctx();
+  c->cfg = *cfg;
+  c->device = device;
+  if (device >= 0) {
+    int n = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
+    if (e != cudaSuccess) {
+      delete c;
+      return fail(nullptr, MK_ERR_CUDA, std::string("cudaDeviceGetAttribute: ") + cudaGetErrorString(e));
+    }
+    c->n_sms = n;
+  } else {
+    c->n_sms = 148;  // planning without a device: a B200's SM count
+  }
+  rc = init_ctx(c);
   if (rc) {
     std::string m = c->err;
     delete c;
     return fail(nullptr, rc, m);
   }
-  layout(c);
-  c->pos.assign(f.max_batch, 0);
   *out = c;
   return MK_OK;
 }
@@ -1031,6 +1462,7 @@ size_t mk_kv_cache_bytes(const mk_ctx* c) { return c ? c->kv_bytes : 0; }
 int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, void* workspace, void* stream) {
   if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
   if (!w || !weight_arena || !workspace) return fail(c, MK_ERR_INVALID_ARG, "NULL weights or buffers");
+  if (!c->tp_shards.empty()) return tp_load_weights(c, w, weight_arena, workspace, stream);
   if (c->device < 0) return fail(c, MK_ERR_STATE, "context was planned without a device");
   if ((reinterpret_cast<uintptr_t>(weight_arena) | reinterpret_cast<uintptr_t>(workspace)) & 255)
     return fail(c, MK_ERR_INVALID_ARG, "arena and workspace must be 256-byte aligned");
@@ -1062,7 +1494,7 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
     pack_blocks([&](int i) { return base + (size_t)i * stride; }, rows, K, blk);
     return cuda_ok(c, cudaMemcpy(A + off, blk.data(), blk.size() * 2, cudaMemcpyHostToDevice), "weight copy");
   };
-  if (!put(c->off_embed, w->embed, (size_t)f.vocab * H * 2)) return MK_ERR_CUDA;
+  if (!put(c->off_embed, w->embed, (size_t)(c->tp_ranks > 1 ? c->tp_vfull : f.vocab) * H * 2)) return MK_ERR_CUDA;
   if (c->tc ? !put_blocks(c->off_lm, w->lm_head, H, f.vocab, H) : !put(c->off_lm, w->lm_head, (size_t)f.vocab * H * 2))
     return MK_ERR_CUDA;
   if (!put(c->off_fnorm, w->final_norm, (size_t)H * 2)) return MK_ERR_CUDA;
@@ -1157,6 +1589,8 @@ int mk_load_weights(mk_ctx* c, const mk_host_weights* w, void* weight_arena, voi
 
 int mk_prefill(mk_ctx* c, const int32_t* tokens, int B, int T, void* kv_cache, float* last_logits, void* stream) {
   if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!c->tp_shards.empty())
+    return fail(c, MK_ERR_UNSUPPORTED, "tensor-parallel contexts take the prompt as decode steps (or a filled cache)");
   if (!c->loaded) return fail(c, MK_ERR_STATE, "weights not loaded");
   if (!tokens || !kv_cache) return fail(c, MK_ERR_INVALID_ARG, "NULL tokens or cache");
   if (B < 1 || B > c->cfg.max_batch || T < 1 || T > c->cfg.max_seq)
@@ -1220,21 +1654,11 @@ int mk_get_positions(const mk_ctx* c, int32_t* host_pos, int capacity) {
 }
 
 namespace {
-// One launch of the persistent kernel running n_steps greedy decode steps.
-int decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache, float* logits,
-                  int32_t* next_tokens, void* stream) {
-  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
-  if (!c->loaded) return fail(c, MK_ERR_STATE, "weights not loaded");
-  if (c->B < 1) return fail(c, MK_ERR_STATE, "no active batch (call mk_prefill or mk_set_positions)");
-  if (!tokens || !kv_cache || !logits) return fail(c, MK_ERR_INVALID_ARG, "NULL tokens, cache or logits");
-  if (n_steps < 1 || n_steps > MK_MAX_STEPS) return fail(c, MK_ERR_INVALID_ARG, "n_steps out of range");
-  if (n_steps > 1 && !next_tokens) return fail(c, MK_ERR_INVALID_ARG, "a multi-step launch needs tokens_out");
-  if (c->variant < 0 || c->B > c->bm)
-    return fail(c, MK_ERR_UNSUPPORTED, "no decode kernel instantiation for this shape / batch");
+// The kernel's view of context c (a whole model, or one tensor-parallel shard) for a launch of
+// n_steps decode steps; `run` holds the positions, active batch, epoch and test settings.
+void make_params(const mk_ctx* c, const mk_ctx* run, const int32_t* tokens, int n_steps, void* kv_cache,
+                 float* logits, int32_t* next_tokens, DecodeParams& P) {
   const mk_config& f = c->cfg;
-  for (int b = 0; b < c->B; ++b)
-    if (c->pos[b] + n_steps > f.max_seq) return fail(c, MK_ERR_INVALID_ARG, "sequence is full (max_seq reached)");
-  DecodeParams P;
   std::memset(&P, 0, sizeof(P));
   uint8_t* W = c->ws;
   P.tasks = reinterpret_cast<const Task*>(W + c->ws_tasks);
@@ -1267,7 +1691,7 @@ int decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache,
   P.tokens = tokens;
   P.logits = logits;
   P.next_tokens = next_tokens;
-  for (int b = 0; b < c->B; ++b) P.pos[b] = c->pos[b];
+  for (int b = 0; b < run->B; ++b) P.pos[b] = run->pos[b];
   P.B = f.max_batch;  // buffer strides use the capacity; the kernel serves sequence 0.. of it
   P.H = f.hidden;
   P.nq = f.n_q_heads;
@@ -1282,21 +1706,78 @@ int decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache,
   P.n_lm = c->n_lm;
   P.eps = f.rms_eps;
   P.attn_scale = 1.0f / std::sqrt((float)f.head_dim);
-  P.nb = c->B;
+  P.nb = run->B;
   P.kdc = c->kdc;
   P.ndc = c->ndc;
   P.tpart = reinterpret_cast<float*>(W + c->ws_tpart);
   P.tcnt = reinterpret_cast<uint32_t*>(W + c->ws_tcnt);
-  P.epoch = c->epoch + 1;
+  P.epoch = run->epoch + 1;
   P.ev_lm = (uint32_t)c->ev_lm;
   P.ev_tok = (uint32_t)c->ev_tok;
   P.n_steps = n_steps;
-  P.drop_event = c->drop_event;
-  P.timeout_ns = c->timeout_ns;
-  P.trace = c->trace;
-  P.l2_ahead = c->dyn ? 0 : c->l2_ahead;  // the lookahead walks static queues only
+  P.drop_event = run->drop_event;
+  P.timeout_ns = run->timeout_ns;
+  P.trace = run->trace;
+  P.l2_ahead = c->dyn ? 0 : run->l2_ahead;  // the lookahead walks static queues only
+  P.tp_ranks = 1;
+}
+
+int tp_decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache, float* logits,
+                     int32_t* next_tokens, void* stream);
+
+// One launch of the persistent kernel running n_steps greedy decode steps.
+int decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache, float* logits,
+                  int32_t* next_tokens, void* stream) {
+  if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!c->loaded) return fail(c, MK_ERR_STATE, "weights not loaded");
+  if (c->B < 1) return fail(c, MK_ERR_STATE, "no active batch (call mk_prefill or mk_set_positions)");
+  if (!tokens || !kv_cache || !logits) return fail(c, MK_ERR_INVALID_ARG, "NULL tokens, cache or logits");
+  if (n_steps < 1 || n_steps > MK_MAX_STEPS) return fail(c, MK_ERR_INVALID_ARG, "n_steps out of range");
+  if (n_steps > 1 && !next_tokens) return fail(c, MK_ERR_INVALID_ARG, "a multi-step launch needs tokens_out");
+  if (c->variant < 0 || c->B > c->bm)
+    return fail(c, MK_ERR_UNSUPPORTED, "no decode kernel instantiation for this shape / batch");
+  const mk_config& f = c->cfg;
+  for (int b = 0; b < c->B; ++b)
+    if (c->pos[b] + n_steps > f.max_seq) return fail(c, MK_ERR_INVALID_ARG, "sequence is full (max_seq reached)");
+  if (!c->tp_shards.empty()) return tp_decode_launch(c, tokens, n_steps, kv_cache, logits, next_tokens, stream);
+  DecodeParams P;
+  make_params(c, c, tokens, n_steps, kv_cache, logits, next_tokens, P);
   std::string err;
   int rc = launch_decode(c->variant, P, c->n_sms, reinterpret_cast<cudaStream_t>(stream), &err);
+  if (rc) return fail(c, rc, err);
+  c->epoch += (uint32_t)n_steps;
+  for (int b = 0; b < c->B; ++b) c->pos[b] += n_steps;
+  return MK_OK;
+}
+
+// Emulated tensor parallel: one launch, every rank's view (see mk_build_taskgraph_tp).
+int tp_decode_launch(mk_ctx* c, const int32_t* tokens, int n_steps, void* kv_cache, float* logits,
+                     int32_t* next_tokens, void* stream) {
+  const int R = c->tp_ranks;
+  DecodeParams views[kMaxTpRanks];
+  for (int r = 0; r < R; ++r) {
+    const mk_ctx* sh = c->tp_shards[r];
+    DecodeParams& P = views[r];
+    make_params(sh, c, tokens, n_steps, static_cast<uint8_t*>(kv_cache) + c->tp_kv_off[r], logits, next_tokens, P);
+    P.tasks = reinterpret_cast<const Task*>(c->ws + c->tp_ws_tasks);  // every rank's queues
+    P.qbegin = reinterpret_cast<const uint32_t*>(c->ws + c->tp_ws_qbegin);
+    P.err = reinterpret_cast<uint32_t*>(c->tp_shards[0]->ws + c->tp_shards[0]->ws_err);  // one error word
+    P.trace = nullptr;
+    P.tp_rank = r;
+    P.tp_ranks = R;
+    P.tp_vbase = sh->tp_vbase;
+    P.tp_vfull = sh->tp_vfull;
+    P.ev_lmx = (uint32_t)sh->ev_lmx;
+    for (int d = 0; d < R; ++d) {
+      mk_ctx* pd = c->tp_shards[d];
+      P.tp_recv_o[d] = reinterpret_cast<float*>(pd->ws + pd->ws_recv_o);
+      P.tp_recv_d[d] = reinterpret_cast<float*>(pd->ws + pd->ws_recv_d);
+      P.tp_ev[d] = reinterpret_cast<uint32_t*>(pd->ws + pd->ws_ev);
+      P.tp_lmx[d] = reinterpret_cast<uint64_t*>(pd->ws + pd->ws_lmx);
+    }
+  }
+  std::string err;
+  int rc = launch_decode_tp(c->variant, views, R, c->tp_sms, reinterpret_cast<cudaStream_t>(stream), &err);
   if (rc) return fail(c, rc, err);
   c->epoch += (uint32_t)n_steps;
   for (int b = 0; b < c->B; ++b) c->pos[b] += n_steps;
@@ -1319,6 +1800,7 @@ int mk_sync_status(mk_ctx* c, void* stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (!cuda_ok(c, cudaStreamSynchronize(s), "stream sync")) return MK_ERR_CUDA;
   if (!c->loaded) return MK_OK;
+  if (!c->tp_shards.empty()) return tp_sync_status(c);
   uint32_t e[4];
   if (!cuda_ok(c, cudaMemcpy(e, c->ws + c->ws_err, 16, cudaMemcpyDeviceToHost), "error read")) return MK_ERR_CUDA;
   if (e[ERR_CODE] == 0) return MK_OK;
@@ -1357,6 +1839,7 @@ namespace {
 // Re-partition with new per-SM weights for one projection kind (op > 0) or for all (op = 0).
 int set_weights(mk_ctx* c, int op, const float* weights, int n, void* stream) {
   if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!c->tp_shards.empty()) return fail(c, MK_ERR_UNSUPPORTED, "tensor-parallel graphs keep equal rows per SM");
   if (op != 0 && op != TK_QKV && op != TK_OPROJ && op != TK_GATEUP && op != TK_DOWN && op != TK_LMHEAD)
     return fail(c, MK_ERR_INVALID_ARG, "op must be 0 or a projection task kind");
   if (!weights || n != c->n_sms) return fail(c, MK_ERR_INVALID_ARG, "need one weight per SM");
@@ -1412,6 +1895,7 @@ int mk_set_op_sm_weights(mk_ctx* c, int op_kind, const float* weights, int n, vo
 
 int mk_set_dispatch(mk_ctx* c, int mode, int tasks_per_sm, void* stream) {
   if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!c->tp_shards.empty()) return fail(c, MK_ERR_UNSUPPORTED, "tensor-parallel graphs use static queues");
   if (mode != MK_DISPATCH_STATIC && mode != MK_DISPATCH_CLAIM && mode != MK_DISPATCH_CLAIM_PACED)
     return fail(c, MK_ERR_INVALID_ARG, "unknown mode");
   const bool claim = mode != MK_DISPATCH_STATIC;
@@ -1462,6 +1946,7 @@ int mk_set_l2_prefetch(mk_ctx* c, int stages) {
 
 int mk_set_trace(mk_ctx* c, void* device_buffer) {
   if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
+  if (!c->tp_shards.empty()) return fail(c, MK_ERR_UNSUPPORTED, "no tracing of tensor-parallel launches");
   if (device_buffer && (reinterpret_cast<uintptr_t>(device_buffer) & 7))
     return fail(c, MK_ERR_INVALID_ARG, "trace buffer must be 8-byte aligned");
   c->trace = static_cast<uint64_t*>(device_buffer);
@@ -1473,6 +1958,10 @@ int mk_get_graph_info(const mk_ctx* c, mk_graph_info* out) {
   out->n_sms = c->n_sms;
   out->n_tasks = (int)c->g.tasks.size();
   out->task_capacity = (int)c->task_cap;
+  if (!c->tp_shards.empty()) {  // emulated tensor parallel: every rank's tasks, rank 0's SMs first
+    out->n_sms = c->tp_ranks * c->tp_sms;
+    out->n_tasks = out->task_capacity = (int)c->tp_tasks.size();
+  }
   out->n_events = c->n_events;
   out->attn_chunks = c->nch;
   out->kernel_variant = c->variant;
@@ -1484,6 +1973,7 @@ int mk_get_graph_info(const mk_ctx* c, mk_graph_info* out) {
 int mk_export_taskgraph(const mk_ctx* c, int32_t* tasks, int task_capacity, int32_t* event_counts,
                         int event_capacity) {
   if (!c) return MK_ERR_INVALID_ARG;
+  if (!c->tp_shards.empty()) return MK_ERR_UNSUPPORTED;  // mk_export_taskgraph_tp
   std::vector<VTask> v = to_vtasks(c->g);
   if (tasks)
     for (int i = 0; i < (int)v.size() && i < task_capacity; ++i) {
@@ -1525,7 +2015,7 @@ int mk_attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* 
     return fail(nullptr, MK_ERR_CUDA, "no CUDA device");
   std::string err;
   int rc = attention_decode(q, k_t, v, o, BH, d, L, scale, workspace, reinterpret_cast<cudaStream_t>(stream), n,
-                            2000000000ull, &err);
+                            nullptr, &err);
   if (rc) return fail(nullptr, rc, err);
   return MK_OK;
 }
@@ -1558,6 +2048,153 @@ int mk_attention_status(void* workspace, int BH, int d, int L, void* stream) {
   cudaMemset(workspace, 0, bytes);
   cudaDeviceSynchronize();
   return fail(nullptr, MK_ERR_DEVICE_TIMEOUT, "attention wait timed out");
+}
+
+int mk_attention_noalloc_status(void* stream) {
+  std::string err;
+  const int rc = attention_noalloc_status(reinterpret_cast<cudaStream_t>(stream), &err);
+  if (rc) return fail(nullptr, rc, err);
+  return MK_OK;
+}
+
+int mk_attention_set_wait_timeout_ns(uint64_t ns) {
+  if (ns == 0) return fail(nullptr, MK_ERR_INVALID_ARG, "the wait limit must be > 0");
+  attention_set_wait_timeout_ns(ns);
+  return MK_OK;
+}
+
+int mk_attention_debug_drop_unit(int unit) {
+  attention_debug_drop_unit(unit < 0 ? -1 : unit);
+  return MK_OK;
+}
+
+int mk_build_taskgraph_tp(const mk_config* cfg, int n_ranks, int device, mk_ctx** out) {
+  if (!out) return fail(nullptr, MK_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  std::string why;
+  int rc = check_config(cfg, &why);
+  if (rc) return fail(nullptr, rc, why);
+  const mk_config& f = *cfg;
+  const int R = n_ranks;
+  if (R < 2 || R > kMaxTpRanks) return fail(nullptr, MK_ERR_INVALID_ARG, "n_ranks must be in [2, 4]");
+  if (f.max_batch != 1) return fail(nullptr, MK_ERR_UNSUPPORTED, "tensor parallel serves one sequence (max_batch 1)");
+  if (f.qk_norm) return fail(nullptr, MK_ERR_UNSUPPORTED, "no tensor-parallel QK-norm");
+  if (f.n_kv_heads % R || f.ffn % (8 * R) || f.vocab % R)
+    return fail(nullptr, MK_ERR_INVALID_ARG, "n_kv_heads, ffn / 8 and vocab must divide by n_ranks");
+  mk_ctx* c = new mk_ctx();
+  c->cfg = f;
+  c->device = device;
+  if (device >= 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+      delete c;
+      return fail(nullptr, MK_ERR_CUDA, "cudaDeviceGetAttribute failed");
+    }
+    c->n_sms = n;
+  } else {
+    c->n_sms = 148;
+  }
+  c->tp_ranks = R;
+  c->tp_sms = c->n_sms / R;
+  for (int r = 0; r < R; ++r) {
+    mk_ctx* sh = new mk_ctx();
+    c->tp_shards.push_back(sh);
+    sh->cfg = f;
+    sh->cfg.n_q_heads /= R;
+    sh->cfg.n_kv_heads /= R;
+    sh->cfg.ffn /= R;
+    sh->cfg.vocab /= R;
+    sh->device = device;
+    sh->n_sms = c->tp_sms;
+    sh->tp_ranks = R;
+    sh->tp_rank = r;
+    sh->tp_vbase = r * sh->cfg.vocab;
+    sh->tp_vfull = f.vocab;
+    rc = init_ctx(sh);
+    if (rc == MK_OK && sh->variant < 0)
+      rc = fail(sh, MK_ERR_UNSUPPORTED, "no tensor-parallel kernel instantiation for this shape");
+    if (rc) {
+      std::string m = "rank " + std::to_string(r) + ": " + sh->err;
+      delete c;
+      return fail(nullptr, rc, m);
+    }
+  }
+  // every rank's queues, rank r's SM s at global SM r * tp_sms + s
+  c->tp_qbegin.assign((size_t)R * c->tp_sms + 1, 0);
+  for (int r = 0; r < R; ++r) {
+    const mk_ctx* sh = c->tp_shards[r];
+    for (int s2 = 0; s2 < sh->n_sms; ++s2) {
+      c->tp_qbegin[(size_t)r * c->tp_sms + s2] = (uint32_t)c->tp_tasks.size();
+      for (uint32_t i = sh->qbegin[s2]; i < sh->qbegin[s2 + 1]; ++i) {
+        c->tp_tasks.push_back(sh->g.tasks[i].t);
+        c->tp_task_sm.push_back(r * c->tp_sms + s2);
+      }
+    }
+    c->weight_bytes_per_step += sh->weight_bytes_per_step;
+  }
+  c->tp_qbegin[(size_t)R * c->tp_sms] = (uint32_t)c->tp_tasks.size();
+  c->n_events = c->tp_shards[0]->n_events;
+  rc = validate_tp(c, tp_vtasks(c), c->tp_shards[0]->g.ev_count);
+  if (rc) {
+    std::string m = c->err;
+    delete c;
+    return fail(nullptr, rc, m);
+  }
+  // buffers: the ranks' regions one after another
+  for (int r = 0; r < R; ++r) {
+    const mk_ctx* sh = c->tp_shards[r];
+    c->tp_arena_off.push_back(c->arena_bytes);
+    c->arena_bytes = align256(c->arena_bytes + sh->arena_bytes);
+    c->tp_kv_off.push_back(c->kv_bytes);
+    c->kv_bytes = align256(c->kv_bytes + sh->kv_bytes);
+  }
+  size_t ws = 0;
+  c->tp_ws_tasks = ws;
+  ws = align256(ws + c->tp_tasks.size() * sizeof(Task));
+  c->tp_ws_qbegin = ws;
+  ws = align256(ws + c->tp_qbegin.size() * 4);
+  for (int r = 0; r < R; ++r) {
+    c->tp_ws_off.push_back(ws);
+    ws = align256(ws + c->tp_shards[r]->ws_bytes);
+  }
+  c->ws_bytes = ws;
+  c->variant = c->tp_shards[0]->variant;
+  c->nch = c->tp_shards[0]->nch;
+  c->bm = 1;
+  c->pos.assign(1, 0);
+  *out = c;
+  return MK_OK;
+}
+
+int mk_export_taskgraph_tp(const mk_ctx* c, int32_t* tasks, int task_capacity, int32_t* event_counts,
+                           int event_capacity) {
+  if (!c || c->tp_shards.empty()) return MK_ERR_INVALID_ARG;
+  const std::vector<TVTask> v = tp_vtasks(c);
+  if (tasks)
+    for (int i = 0; i < (int)v.size() && i < task_capacity; ++i) {
+      const TVTask& t = v[i];
+      int32_t* o = tasks + (size_t)i * 15;
+      o[0] = t.rank; o[1] = t.kind; o[2] = t.layer; o[3] = t.sm; o[4] = t.row0; o[5] = t.nrows; o[6] = t.n_wait;
+      o[7] = t.wait[0]; o[8] = t.wait[1]; o[9] = t.n_notify; o[10] = t.notify[0]; o[11] = t.notify[1];
+      o[12] = t.remote; o[13] = t.mlo; o[14] = t.mhi;
+    }
+  const auto& cnt = c->tp_shards[0]->g.ev_count;
+  if (event_counts)
+    for (int e = 0; e < (int)cnt.size() && e < event_capacity; ++e) event_counts[e] = (int32_t)cnt[e];
+  return (int)v.size();
+}
+
+int mk_validate_taskgraph_tp(mk_ctx* c, const int32_t* tasks, int n_tasks, const int32_t* event_counts, int n_events) {
+  if (!c || c->tp_shards.empty() || !tasks || !event_counts || n_tasks < 0)
+    return fail(c, MK_ERR_INVALID_ARG, "bad arguments to mk_validate_taskgraph_tp");
+  std::vector<TVTask> v(n_tasks);
+  for (int i = 0; i < n_tasks; ++i) {
+    const int32_t* o = tasks + (size_t)i * 15;
+    v[i] = TVTask{o[0], o[1], o[2], o[3], o[4], o[5], o[6], {o[7], o[8]}, o[9], {o[10], o[11]}, o[12], o[13], o[14]};
+  }
+  std::vector<uint32_t> cnt(n_events);
+  for (int e = 0; e < n_events; ++e) cnt[e] = (uint32_t)std::max(0, event_counts[e]);
+  return validate_tp(c, v, cnt);
 }
 
 const char* mk_last_error(const mk_ctx* c) { return c ? c->err.c_str() : g_err.c_str(); }

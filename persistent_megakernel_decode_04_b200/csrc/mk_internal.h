@@ -33,6 +33,7 @@ constexpr int kSegBytes = kSegElems * 2;
 constexpr int kTaskRows = 256;                       // rows per GEMV task (one per worker thread)
 constexpr int kRpsMax = 8;                           // rows per ring stage (unrolled in the GEMV loop)
 constexpr int kMaxChunks = 64;                       // split-KV chunks per (sequence, KV head)
+constexpr int kMaxTpRanks = 4;                       // tensor-parallel ranks one launch can host
 #ifndef MK_SLOT_KB
 #define MK_SLOT_KB 32
 #endif
@@ -80,6 +81,9 @@ struct Task {
   uint32_t notify[2];   // ATTN: notify[0] is raised by the merging (last) chunk only
   uint32_t index;       // LMHEAD: ordinal among LM-head tasks (argmax partial slot)
   uint32_t pad1;
+  // Tensor-parallel graphs: pad0 = 1 marks a remote-signal edge (the task's notifies go to the
+  // event of that id on every rank); gate/up tasks also write the rows [index, pad1) of the
+  // residual sum x_mid they form (each rank keeps its copy, shared out over its tasks).
   // Tensor-core tasks reuse the fields: row0 = first weight block (tile * K units + unit),
   // nrows = blocks, index = partial record, aux = slot among the tile's tasks (the tile's
   // records are index - aux ..), pad0 = tasks of the tile, pad1 = tile arrival counter.
@@ -139,6 +143,28 @@ struct DecodeParams {
   uint32_t* pcnt;
   int n_pools;
   int dyn;
+  // Tensor parallel (the TP instantiation only; "Compiler des LLM en MegaKernel ...", Part 1:
+  // a matmul followed by an all-reduce lowered into tile tasks).  This view is rank tp_rank of
+  // tp_ranks; its weights, KV cache and activations are its shard.  The row-parallel O and down
+  // tasks store their partial rows into EVERY rank's receive buffer (peer stores) and raise the
+  // op's event on every rank (remote signals); consumers add the ranks' partials in rank order,
+  // so the replicated residual stream is bitwise the same on every rank.  Only x_mid[l] is
+  // stored (by the gate/up tasks); QKV, gate/up and the LM head form x_in[l] = x_mid[l-1] +
+  // the ranks' down rows of layer l-1 as they load it.
+  int tp_rank, tp_ranks;
+  int tp_vbase, tp_vfull;          // LM head: this rank's first vocab row; the full vocab (logits stride)
+  float* tp_recv_o[kMaxTpRanks];   // rank d's O-projection receive buffer [L][ranks][B][H]
+  float* tp_recv_d[kMaxTpRanks];   // rank d's down-projection receive buffer [L][ranks][B][H]
+  uint32_t* tp_ev[kMaxTpRanks];    // rank d's event counters
+  uint64_t* tp_lmx[kMaxTpRanks];   // rank d's argmax slots [ranks][B]: value bits << 32 | vocab index
+  uint32_t ev_lmx;                 // event: every rank's argmax partial of the step arrived
+};
+
+// One launch hosting several tensor-parallel ranks on one GPU (CTA b serves rank
+// b / sms_per_rank): the ranks' views, each pointing at its own shard.
+struct DecodeParamsTP {
+  DecodeParams r[kMaxTpRanks];
+  int sms_per_rank;
 };
 constexpr int kDynQ = 64;                 // run-time claims: task FIFO from the producer to the other roles
 constexpr uint32_t kDynEnd = 0xffffffffu;  // FIFO entry: no more tasks in this launch
@@ -166,23 +192,32 @@ TensorMapEncodeFn get_tensor_map_encoder();
 
 // Kernel variants: one instantiation per (segments, rows per stage) of the two K sizes.
 struct Variant {
-  int nseg_h, rps_h, nseg_f, rps_f, head_dim, bm, qkn, dyn;
+  int nseg_h, rps_h, nseg_f, rps_f, head_dim, bm, qkn, dyn, tp;
 };
-int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn, int dyn);
+int find_decode_variant(int nseg_h, int rps_h, int nseg_f, int rps_f, int head_dim, int bm, int qkn, int dyn,
+                        int tp = 0);
 const void* decode_kernel_ptr(int variant);
 size_t decode_smem_bytes(int variant);
 int launch_decode(int variant, const DecodeParams& p, int grid, cudaStream_t stream, std::string* err);
+// The tensor-parallel instantiation: n_ranks views, grid = n_ranks * sms_per_rank CTAs.
+int launch_decode_tp(int variant, const DecodeParams* views, int n_ranks, int sms_per_rank, cudaStream_t stream,
+                     std::string* err);
 
-// Standalone attention (mk_attention.cu).
+// Standalone attention (mk_attention.cu).  err_word: where the kernel records a wait that
+// ran out (null: the workspace's own error word).  The wait limit and the drop-unit test hook
+// are process-wide settings.
 size_t attention_workspace_bytes(int BH, int d, int L, int n_sms);
 size_t attention_error_word_offset(int BH, int d, int L, int n_sms);
 int attention_decode(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d, int L,
-                     float scale, void* workspace, cudaStream_t stream, int n_sms, uint64_t timeout_ns,
+                     float scale, void* workspace, cudaStream_t stream, int n_sms, uint32_t* err_word,
                      std::string* err);
 size_t attention_counter_offset(int BH, int d, int L, int n_sms);
 size_t attention_noalloc_capacity();
 int attention_decode_noalloc(const uint16_t* q, const uint16_t* k_t, const uint16_t* v, float* o, int BH, int d,
                              int L, float scale, cudaStream_t stream, std::string* err);
+int attention_noalloc_status(cudaStream_t stream, std::string* err);
+void attention_set_wait_timeout_ns(uint64_t ns);
+void attention_debug_drop_unit(int unit);
 
 // Prefill (mk_prefill.cu).
 struct PrefillParams {

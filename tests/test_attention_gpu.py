@@ -65,3 +65,29 @@ def test_single_key_returns_v():
     v = mi.normal_f16(9, 3, (BH, 1, d))
     outs, _ = run(BH, d, 1, seed=9)
     assert np.allclose(outs[0], mi.f16_to_f32(v)[:, 0, :], atol=1e-6)
+
+
+def test_wait_that_runs_out_is_reported_and_the_workspace_recovers():
+    """A tile the producer never loads (test hook) makes its compute warp give up after the wait
+    limit: the status reports MK_ERR_DEVICE_TIMEOUT (and re-zeroes the workspace), nothing faults,
+    and the next call with the same workspace is correct."""
+    BH, d, L = 6, 128, 2048
+    q = mi.normal_f16(4, 1, (BH, d))
+    kt = mi.normal_f16(4, 2, (BH, d, L))
+    v = mi.normal_f16(4, 3, (BH, L, d))
+    dev = torch.device("cuda", 0)
+    tq, tk, tv = (torch.from_numpy(a.view(np.int16)).to(dev) for a in (q, kt, v))
+    o = torch.zeros((BH, d), dtype=torch.float32, device=dev)
+    ws = torch.zeros(mk.mk_attention_workspace_bytes(BH, d, L), dtype=torch.uint8, device=dev)
+    mk.mk_attention_set_wait_timeout_ns(50_000_000)
+    try:
+        mk.mk_attention_debug_drop_unit(70)  # head 2, keys 384..447
+        mk.mk_attention_decode(tq, tk, tv, o, BH, d, L, 1.0, ws)
+        assert mk.mk_attention_status(ws, BH, d, L) == mk.MK_ERR_DEVICE_TIMEOUT
+    finally:
+        mk.mk_attention_debug_drop_unit(-1)
+        mk.mk_attention_set_wait_timeout_ns(2_000_000_000)
+    o.fill_(float("nan"))
+    mk.mk_attention_decode(tq, tk, tv, o, BH, d, L, 1.0, ws)
+    assert mk.mk_attention_status(ws, BH, d, L) == mk.MK_OK
+    check(o.cpu().numpy(), oracle.attention_decode_f16(q, kt, v, 1.0))
