@@ -81,7 +81,7 @@ def parse():
                    help="keep equal rows per SM instead of the schedule calibrated on untimed steps before "
                         "the warm-up")
     p.add_argument("--workload", default="llama8b", choices=sorted(WORKLOADS))
-    p.add_argument("--dispatch", default="static", choices=["static", "claim", "claim-paced"],
+    p.add_argument("--dispatch", default="static", choices=["static", "claim", "claim-paced", "claim-priority"],
                    help="scheduling variant: fixed per-SM queues (default), or projection tasks claimed "
                         "at run time from per-op pools (batch-1 kernel only)")
     p.add_argument("--tasks-per-sm", type=int, default=2, help="pool tasks per SM and projection (--dispatch claim)")
@@ -398,8 +398,8 @@ def run_mk(args, rank, world, local):
         tok = torch.from_numpy(mi.prompt(0, 0, B, shape.vocab).astype(np.int32)).to(dev)
     calibrated = False
     if args.dispatch != "static":  # pools are cut in equal shares: no per-SM calibration
-        m.set_dispatch(mk.MK_DISPATCH_CLAIM if args.dispatch == "claim" else mk.MK_DISPATCH_CLAIM_PACED,
-                       args.tasks_per_sm)
+        m.set_dispatch({"claim": mk.MK_DISPATCH_CLAIM, "claim-paced": mk.MK_DISPATCH_CLAIM_PACED,
+                        "claim-priority": mk.MK_DISPATCH_CLAIM_PRIORITY}[args.dispatch], args.tasks_per_sm)
     elif calib_steps:
         # the schedule: per-SM streaming speed measured on untimed traced decode steps
         # (3 rounds x 2 steps) and every projection's rows re-partitioned, before the warm-up
@@ -488,6 +488,8 @@ def run_mk(args, rank, world, local):
                        "global_batch": world * B, "parallelism": "replicas", "weights": "bf16",
                        "schedule": (f"run-time claims from per-op pools, {args.tasks_per_sm} tasks per SM"
                                     + (", paced by the workers" if args.dispatch == "claim-paced" else "")
+                                    + (", attention chunks claimed first (priority)"
+                                       if args.dispatch == "claim-priority" else "")
                                     if args.dispatch != "static" else
                                     f"calibrated per-SM rows ({calib_steps} untimed calibration steps "
                                     f"before the warm-up)" if calibrated else "equal rows per SM"),

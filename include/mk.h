@@ -196,6 +196,12 @@ int mk_set_op_sm_weights(mk_ctx* ctx, int op_kind, const float* weights, int n, 
 #define MK_DISPATCH_STATIC 0
 #define MK_DISPATCH_CLAIM 1
 #define MK_DISPATCH_CLAIM_PACED 2
+/* Priority dispatch ("Orientations futures" of the MPK summary: scheduling by priority): as
+ * MK_DISPATCH_CLAIM, and the critical path's tasks -- every layer's attention chunks, on which the
+ * O projection of every SM waits -- are a pool too, placed right after the QKV pool in every SM's
+ * queue, so the SMs that finish their QKV claims first take them instead of chunks fixed to SMs
+ * that may still be streaming QKV rows. */
+#define MK_DISPATCH_CLAIM_PRIORITY 3
 int mk_set_dispatch(mk_ctx* ctx, int mode, int tasks_per_sm, void* stream);
 
 /* Weight prefetch depth: besides the shared-memory ring (6 stages of 32 KB per SM), an SM's

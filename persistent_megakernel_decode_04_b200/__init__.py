@@ -36,6 +36,7 @@ MK_MAX_BATCH = 16
 MK_DISPATCH_STATIC = 0
 MK_DISPATCH_CLAIM = 1
 MK_DISPATCH_CLAIM_PACED = 2
+MK_DISPATCH_CLAIM_PRIORITY = 3
 
 TASK_KINDS = {1: "embed", 2: "qkv", 3: "attn", 4: "oproj", 5: "gateup", 6: "down", 7: "lmhead", 8: "pool"}
 

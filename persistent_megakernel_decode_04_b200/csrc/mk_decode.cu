@@ -1596,6 +1596,30 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
       }
       return true;
     };
+    // an attention chunk's old K/V rows through the ring, kv_stage_keys<HD>() per stage: K rows,
+    // then V rows (i: its task index, for error reports)
+    auto stream_attn = [&](const Task& t, uint32_t i, int st) -> bool {
+      const AttnGeom a = attn_geom(P, t, st);
+      int jend;
+      const int nst = attn_stage_span<HD>(a, &jend);
+      const uint16_t* kc = attn_cache<HD>(P, t, a, 0);
+      const uint16_t* vc = attn_cache<HD>(P, t, a, 1);
+      for (int k = 0; k < nst; ++k) {
+        const int jj = a.j0 + k * kv_stage_keys<HD>();
+        const uint32_t bytes = (uint32_t)min(kv_stage_keys<HD>(), jend - jj) * HD * 2u;
+        if (!wait_bar(&S.empty[pp.stage], pp.phase ^ 1u, P.timeout_ns, &S)) {
+          if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, i);
+          return false;
+        }
+        uint8_t* dst = ring + (size_t)pp.stage * kSlotBytes;
+        mbar_arrive_expect_tx(&S.full[pp.stage], 2u * bytes);
+        bulk_g2s(dst, kc + (size_t)jj * HD, bytes, &S.full[pp.stage], pol);
+        bulk_g2s(dst + kv_stage_keys<HD>() * HD * 2, vc + (size_t)jj * HD, bytes, &S.full[pp.stage], pol);
+        ++issued;
+        pp.advance();
+      }
+      return true;
+    };
     for (int st = 0; st < P.n_steps && ok; ++st) {
     if (st > 0) {  // the lookahead restarts with the step's queue
       la_task = qb;
@@ -1666,7 +1690,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
             }
             uint32_t cn = 0xffffffffu;
             if (P.dyn != 2) cn = atomicAdd(ctr, 1u);
-            ok = stream_gemv(P.tasks[id], id);
+            {
+              const Task tc2 = P.tasks[id];  // a projection tile, or (priority claims) an attention chunk
+              ok = tc2.kind == TK_ATTN ? stream_attn(tc2, id, st) : stream_gemv(tc2, id);
+            }
             if (ok && P.dyn == 2) {
               ok = paced();
               if (ok) cn = atomicAdd(ctr, 1u);
@@ -1681,27 +1708,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
         }
       }
       if (t.kind == TK_ATTN) {
-        // old K/V rows of the chunk, kv_stage_keys<HD>() per stage: K rows, then V rows
-        const AttnGeom a = attn_geom(P, t, st);
-        int jend;
-        const int nst = attn_stage_span<HD>(a, &jend);
-        const uint16_t* kc = attn_cache<HD>(P, t, a, 0);
-        const uint16_t* vc = attn_cache<HD>(P, t, a, 1);
-        for (int st = 0; st < nst; ++st) {
-          const int jj = a.j0 + st * kv_stage_keys<HD>();
-          const uint32_t bytes = (uint32_t)min(kv_stage_keys<HD>(), jend - jj) * HD * 2u;
-          if (!wait_bar(&S.empty[pp.stage], pp.phase ^ 1u, P.timeout_ns, &S)) {
-            if (!S.abort) raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, i);
-            ok = false;
-            break;
-          }
-          uint8_t* dst = ring + (size_t)pp.stage * kSlotBytes;
-          mbar_arrive_expect_tx(&S.full[pp.stage], 2u * bytes);
-          bulk_g2s(dst, kc + (size_t)jj * HD, bytes, &S.full[pp.stage], pol);
-          bulk_g2s(dst + kv_stage_keys<HD>() * HD * 2, vc + (size_t)jj * HD, bytes, &S.full[pp.stage], pol);
-          ++issued;
-          pp.advance();
-        }
+        ok = stream_attn(t, i, st);
         continue;
       }
       if (!is_gemv(t.kind)) continue;

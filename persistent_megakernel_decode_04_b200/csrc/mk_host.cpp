@@ -939,6 +939,11 @@ int build_graph(mk_ctx* c) {
         }
         q[s].push_back(t);
       }
+    // priority claims: the attention chunks (the critical path between QKV and O) become a pool
+    // right after the QKV pool, taken by whichever SMs finish their QKV claims first
+    const bool attn_pool = dyn && c->dyn == MK_DISPATCH_CLAIM_PRIORITY;
+    const uint32_t attn_p = (uint32_t)c->pool_first.size();
+    if (attn_pool) c->pool_first.push_back((uint32_t)pool_tasks.size());
     for (int idx = 0; idx < n_attn; ++idx) {
       const int bg = idx / c->nch, ch = idx % c->nch;
       const int g = bg % nkv;
@@ -946,8 +951,19 @@ int build_graph(mk_ctx* c) {
       t.aux = (uint16_t)ch;
       add_wait(t, ev_qkv(c, l, g));
       add_notify(t, ev_attn(c, l));
+      if (attn_pool) {
+        pool_tasks.push_back(t);
+        qv[idx % n].push_back(t);
+        continue;
+      }
       const int s = (int)(((long long)idx * n / n_attn + (long long)l * 37) % n);
       push_static(s, t);
+    }
+    if (attn_pool) {
+      c->pool_count.push_back((uint32_t)n_attn);
+      Task e = make_task(TK_POOL, l, 0, 0);
+      e.index = attn_p;
+      for (int s2 = 0; s2 < n; ++s2) q[s2].push_back(e);
     }
     evc[ev_attn(c, l)] = (uint32_t)(B * nkv);
     if (dyn) {
@@ -1118,7 +1134,7 @@ void layout(mk_ctx* c) {
   c->task_cap = c->g.tasks.size() * 2 + (size_t)c->n_sms * 16;
   c->lm_cap = (size_t)c->n_lm * 2 + (size_t)c->n_sms * 4;
   // run-time claims: queue entries (one per SM and pool) plus pools of up to 4 tasks per SM
-  c->pool_cap = 4 * L;
+  c->pool_cap = 5 * L;  // QKV, attention (priority claims), O, gate/up, down
   c->task_cap = std::max(c->task_cap, c->g.tasks.size() + (size_t)c->n_sms * c->pool_cap * 5);
   c->ws_tasks = take(c->task_cap * sizeof(Task));
   c->ws_pools = take((size_t)c->pool_cap * 2 * sizeof(uint32_t));
@@ -1896,7 +1912,8 @@ int mk_set_op_sm_weights(mk_ctx* c, int op_kind, const float* weights, int n, vo
 int mk_set_dispatch(mk_ctx* c, int mode, int tasks_per_sm, void* stream) {
   if (!c) return fail(nullptr, MK_ERR_INVALID_ARG, "ctx is NULL");
   if (!c->tp_shards.empty()) return fail(c, MK_ERR_UNSUPPORTED, "tensor-parallel graphs use static queues");
-  if (mode != MK_DISPATCH_STATIC && mode != MK_DISPATCH_CLAIM && mode != MK_DISPATCH_CLAIM_PACED)
+  if (mode != MK_DISPATCH_STATIC && mode != MK_DISPATCH_CLAIM && mode != MK_DISPATCH_CLAIM_PACED &&
+      mode != MK_DISPATCH_CLAIM_PRIORITY)
     return fail(c, MK_ERR_INVALID_ARG, "unknown mode");
   const bool claim = mode != MK_DISPATCH_STATIC;
   if (claim && (tasks_per_sm < 1 || tasks_per_sm > 4))

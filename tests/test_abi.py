@@ -279,6 +279,35 @@ def test_claim_dispatch_pools_cover_every_projection(shape, tps):
         mk.mk_destroy(ctx)
 
 
+@pytest.mark.parametrize("shape", [mi.TINY, mi.LLAMA8B.with_layers(2)])
+def test_priority_dispatch_pools_the_attention_chunks(shape):
+    # priority claims: every layer's attention chunks form a pool right after its QKV pool
+    ctx = mk.mk_build_taskgraph(mk.Config.from_shape(shape, 1, 256).c(), -1)
+    try:
+        info = mk.mk_get_graph_info(ctx)
+        mk.mk_set_dispatch(ctx, mk.MK_DISPATCH_CLAIM_PRIORITY, 2)
+        tasks, counts = mk.mk_export_taskgraph(ctx)
+        n_sms, L = info["n_sms"], shape.n_layers
+        entries = tasks[tasks[:, 0] == 8]
+        assert len(entries) == n_sms * 5 * L  # QKV, attention, O, gate/up, down
+        pooled = tasks[tasks[:, 2] == -1]
+        assert set(pooled[:, 0].tolist()) == {2, 3, 4, 5, 6}
+        for l in range(L):
+            attn = pooled[(pooled[:, 0] == 3) & (pooled[:, 1] == l)]
+            assert len(attn) == shape.n_kv_heads * info["attn_chunks"]
+            # every (sequence, KV head) has each chunk once
+            seen = {(int(t[3]), int(t[4])) for t in attn}
+            assert len(seen) == len(attn)
+        static = tasks[(tasks[:, 2] >= 0) & (tasks[:, 0] != 8)]
+        assert set(static[:, 0].tolist()) == {1, 7}  # only the embedding and the LM head stay fixed
+        # on every SM the layer's attention entry comes right after its QKV entry
+        sm0 = tasks[tasks[:, 2] == 0]
+        kinds = [int(t[0]) for t in sm0]
+        assert kinds.count(8) == 5 * L
+    finally:
+        mk.mk_destroy(ctx)
+
+
 def test_claim_dispatch_rejections():
     for shape, b in ((mi.TINY, 4), (mi.TINY, 16), (mi.CHAMELEON7B.with_layers(1), 1)):
         ctx = mk.mk_build_taskgraph(mk.Config.from_shape(shape, b, 64).c(), -1)
@@ -290,7 +319,7 @@ def test_claim_dispatch_rejections():
             mk.mk_destroy(ctx)
     ctx = mk.mk_build_taskgraph(_cfg().c(), -1)
     try:
-        for mode, tps in ((mk.MK_DISPATCH_CLAIM, 0), (mk.MK_DISPATCH_CLAIM, 5), (7, 1)):
+        for mode, tps in ((mk.MK_DISPATCH_CLAIM, 0), (mk.MK_DISPATCH_CLAIM, 5), (7, 1), (-1, 1)):
             with pytest.raises(mk.MkError) as e:
                 mk.mk_set_dispatch(ctx, mode, tps)
             assert e.value.code == mk.MK_ERR_INVALID_ARG

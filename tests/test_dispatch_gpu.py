@@ -1,5 +1,5 @@
-"""Scheduling variant: projection tasks claimed at run time from per-op pools (MK_DISPATCH_CLAIM)
-instead of fixed per-SM queues.  The result must not depend on which SM ran which task: parity
+"""Scheduling variant: projection tasks claimed at run time from per-op pools (MK_DISPATCH_CLAIM;
+paced; with priority to the attention chunks of the critical path) instead of fixed per-SM queues.  The result must not depend on which SM ran which task: parity
 with the oracle, with the static schedule (one-step and multi-step launches, where the claim
 counters of a step are recycled two steps later), and clean timeouts."""
 import numpy as np
@@ -23,7 +23,7 @@ def _model(w, max_seq, tps=None, mode=mk.MK_DISPATCH_CLAIM):
 
 
 @pytest.mark.parametrize("tps,mode", [(1, mk.MK_DISPATCH_CLAIM), (2, mk.MK_DISPATCH_CLAIM), (4, mk.MK_DISPATCH_CLAIM),
-                                      (2, mk.MK_DISPATCH_CLAIM_PACED)])
+                                      (2, mk.MK_DISPATCH_CLAIM_PACED), (2, mk.MK_DISPATCH_CLAIM_PRIORITY)])
 def test_claims_match_the_oracle(tps, mode):
     w = mi.make_weights(mi.TINY, seed=40)
     prompt = mi.prompt(40, 0, 14, w.shape.vocab)
@@ -76,7 +76,8 @@ def test_claims_equal_static_schedule_tiny(multi):
     w = mi.make_weights(mi.TINY, seed=42)
     prompt = mi.prompt(42, 0, 10, w.shape.vocab)
     a = _run(w, 32, None, prompt, 9, multi)
-    for tps, mode in ((1, mk.MK_DISPATCH_CLAIM), (3, mk.MK_DISPATCH_CLAIM), (2, mk.MK_DISPATCH_CLAIM_PACED)):
+    for tps, mode in ((1, mk.MK_DISPATCH_CLAIM), (3, mk.MK_DISPATCH_CLAIM), (2, mk.MK_DISPATCH_CLAIM_PACED),
+                      (2, mk.MK_DISPATCH_CLAIM_PRIORITY)):
         b = _run(w, 32, tps, prompt, 9, multi, mode)
         assert np.array_equal(a[0], b[0])
         assert np.abs(a[1] - b[1]).max() <= 1e-3
@@ -91,7 +92,8 @@ def test_claims_equal_static_schedule_llama8b_two_layers():
     b = _run(w, L + 16, 2, (kv, L), 5, True)
     c = _run(w, L + 16, 2, (kv, L), 5, False)
     d = _run(w, L + 16, 2, (kv, L), 5, True, mk.MK_DISPATCH_CLAIM_PACED)
-    for r in (b, c, d):
+    e = _run(w, L + 16, 2, (kv, L), 5, True, mk.MK_DISPATCH_CLAIM_PRIORITY)
+    for r in (b, c, d, e):
         assert np.array_equal(a[0], r[0])
         assert np.abs(a[1] - r[1]).max() <= 1e-3
 
