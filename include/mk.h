@@ -211,6 +211,13 @@ int mk_set_dispatch(mk_ctx* ctx, int mode, int tasks_per_sm, void* stream);
  * than 0 = off on the 8B batch-1 decode); at most 64. */
 int mk_set_l2_prefetch(mk_ctx* ctx, int stages);
 
+/* Split-KV chunk length floor: at attention length Lk, a (sequence, KV head) uses
+ * min(chunks, ceil(Lk / keys)) chunks, each on its own SM, whose partials the last one to finish
+ * merges (FlashDecoding, named in the Mirage article's attention example).  Fewer, longer chunks
+ * save the arrival atomic and the merge on the critical path; more, shorter ones spread the keys
+ * over more SMs.  Default 64; must be in [1, 2^20].  Results do not depend on it beyond rounding. */
+int mk_set_attn_chunk_keys(mk_ctx* ctx, int keys);
+
 /* Tracing (per-task timing of the next decode steps).  device_buffer: n_tasks * 6 uint64
  * records (n_tasks from mk_get_graph_info), or NULL to switch tracing off.  Record of task i
  * (global-timer ns): [0] worker starts waiting for the task's inputs, [1] inputs released by

@@ -87,6 +87,7 @@ _SIGS = {
     "mk_set_wait_timeout_ns": ([_vp, _u64], _i32),
     "mk_debug_drop_notify": ([_vp, _i32, _i32], _i32),
     "mk_set_l2_prefetch": ([_vp, _i32], _i32),
+    "mk_set_attn_chunk_keys": ([_vp, _i32], _i32),
     "mk_set_dispatch": ([_vp, _i32, _i32, _vp], _i32),
     "mk_set_sm_weights": ([_vp, _vp, _i32, _vp], _i32),
     "mk_set_op_sm_weights": ([_vp, _i32, _vp, _i32, _vp], _i32),
@@ -248,6 +249,10 @@ def mk_set_op_sm_weights(ctx, op_kind: int, weights, stream=None):
 
 def mk_set_l2_prefetch(ctx, stages: int):
     _check(_lib.mk_set_l2_prefetch(ctx, int(stages)), ctx)
+
+
+def mk_set_attn_chunk_keys(ctx, keys: int):
+    _check(_lib.mk_set_attn_chunk_keys(ctx, int(keys)), ctx)
 
 
 def mk_set_dispatch(ctx, mode: int, tasks_per_sm: int = 2, stream=None):

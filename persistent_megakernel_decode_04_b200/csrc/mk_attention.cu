@@ -85,6 +85,11 @@ struct Smem {
   uint32_t last;                                     // this CTA merges the head when set
   volatile uint32_t abort;                           // a wait ran out: every role stops waiting
   int abort_epoch;  // first compute-barrier epoch whose barrier follows an abort (INT_MAX: none)
+  // unit whose tiles the producer armed stage s for.  Eight warps take units round-robin over
+  // six stages, so a warp can reach a stage's next use before the previous use's tiles have
+  // landed; a parity wait cannot tell those phases apart.  A warp first waits until its stage
+  // is armed for its unit (the previous use is then complete), then on the stage's phase.
+  uint32_t armed[kStages];
   alignas(8) uint64_t full[kStages];
   alignas(8) uint64_t empty[kStages];
 };
@@ -97,6 +102,21 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_
     if (mbar_test(bar, parity)) return true;
     if ((n & 255u) == 0) {
       if (abort && *abort) return false;
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > limit_ns) return false;
+    }
+  }
+}
+
+// Bounded wait until the producer armed a stage for unit u: false once `limit_ns` passed or
+// another role aborted.
+__device__ __forceinline__ bool wait_armed(uint32_t* armed, uint32_t u, uint64_t limit_ns, volatile uint32_t* abort) {
+  uint64_t t0 = 0;
+  for (uint32_t n = 1;; ++n) {
+    if (ld_acquire_cta_shared(armed) == u) return true;
+    if ((n & 255u) == 0) {
+      if (*abort) return false;
       const uint64_t now = globaltimer_ns();
       if (t0 == 0) t0 = now;
       else if (now - t0 > limit_ns) return false;
@@ -137,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     S.abort = 0;
     S.abort_epoch = INT_MAX;
+    for (int s = 0; s < kStages; ++s) S.armed[s] = 0xffffffffu;
     fence_mbar_init();
   }
   __syncthreads();
@@ -160,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(&S.full[stage], 2u * D * kUnit * 2u);
           tma_load_3d(S.kt[stage], &map_k, j0, 0, h, &S.full[stage], pol);
           tma_load_3d(S.v[stage], &map_v, 0, j0, h, &S.full[stage], pol);
+          st_release_cta_shared(&S.armed[stage], (uint32_t)u);  // the stage's previous use is released
         }
         ++issued;
         if (++stage == kStages) {
@@ -202,7 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = hu0 + warp; u < hu1; u += kComputeWarps) {
       const int idx = u - u0, stage = idx % kStages;
       const uint32_t parity = (uint32_t)(idx / kStages) & 1u;
-      bool ok = !failed && wait_bar(&S.full[stage], parity, P.timeout_ns, &S.abort);
+      bool ok = !failed && wait_armed(&S.armed[stage], (uint32_t)u, P.timeout_ns, &S.abort) &&
+                wait_bar(&S.full[stage], parity, P.timeout_ns, &S.abort);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (!failed && lane == 0) {

@@ -31,6 +31,10 @@
 #include "mk_internal.h"
 #include "mk_ptx.cuh"
 
+#ifndef MK_GEMV_PIPE
+#define MK_GEMV_PIPE 1  // batch width 1: software-pipelined stage loop (0: the plain loop)
+#endif
+
 namespace mk {
 
 // Dynamic shared memory: the weight ring (nst stages of kSlotBytes, 1024-aligned), then for
@@ -232,8 +236,11 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
                                           uint32_t row_bytes, uint32_t task_id, uint32_t& stall_ns,
                                           const XAdd& xa = XAdd{nullptr, 0, nullptr, 0, 0, nullptr, 0, 0}) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // only the last segment can be partial or empty: K > (NSEG - 2) * kSegElems by construction
+  // only the last segment can be partial or empty: K > (NSEG - 2) * kSegElems by construction,
+  // except in a tensor-parallel shard, where the O projection's K (the rank's heads) can end
+  // inside an earlier segment: there every segment is checked
   const bool last_ok = (NSEG - 1) * kSegElems + tid * 8 < K;
+  auto seg_ok = [&](int s) { return TPX ? (s * kSegElems + tid * 8 < K) : (s < NSEG - 1 || last_ok); };
   uint64_t x2[BM][NSEG][4];
   float ss[BM];
 #pragma unroll
@@ -243,7 +250,7 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
     for (int s = 0; s < NSEG; ++s) {
       const int k = s * kSegElems + tid * 8;
       float x[8];
-      if ((s < NSEG - 1 || last_ok) && (BM == 1 || b < nb)) {
+      if (seg_ok(s) && (BM == 1 || b < nb)) {
         const float* xb = xsrc + (size_t)b * xstride;
         float4 a = __ldcg(reinterpret_cast<const float4*>(xb + k));
         float4 c = __ldcg(reinterpret_cast<const float4*>(xb + k + 4));
@@ -281,6 +288,52 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
   }
   float* red = S.red[warp];
   bool ok = true;
+#if MK_GEMV_PIPE
+  if constexpr (BM == 1) {
+    // Batch width 1, software-pipelined: the cross-lane reduction of stage i-1's partial sums
+    // (a chain of shuffles) is issued between stage i's shared-memory loads and its FMAs, so
+    // the shuffle latency overlaps the load latency instead of following the FMAs.  Every
+    // stage computes all RPS rows (rows past nrows read stale but in-bounds ring bytes; their
+    // sums are never stored), so the stage body has no branches.
+    float ap[RPS];
+    int rp = -1;  // first row of the partial sums in ap (-1: none yet)
+    for (int r0 = 0; r0 < nrows; r0 += RPS) {
+      const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
+      if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
+        if (ok) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
+        ok = false;
+        S.cabort = 1u;
+      }
+      if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
+      const uint8_t* base = ring + (size_t)pp.stage * kSlotBytes + tid * 16;
+      uint4 w[RPS][NSEG];
+#pragma unroll
+      for (int rr = 0; rr < RPS; ++rr)
+#pragma unroll
+        for (int s = 0; s < NSEG; ++s)
+          w[rr][s] = seg_ok(s) ? *reinterpret_cast<const uint4*>(base + rr * row_bytes + s * kSegBytes)
+                               : make_uint4(0u, 0u, 0u, 0u);
+      if (rp >= 0) warp_reduce_rows<RPS>(ap, red + rp, lane, nrows - rp);
+      uint64_t acc[RPS];
+#pragma unroll
+      for (int rr = 0; rr < RPS; ++rr) {
+        acc[rr] = 0ull;
+#pragma unroll
+        for (int s = 0; s < NSEG; ++s) dot8(w[rr][s], x2[0][s], acc[rr]);
+      }
+      __syncwarp();  // every lane's reads of the stage are done: release it
+      if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
+#pragma unroll
+      for (int rr = 0; rr < RPS; ++rr) {
+        const float2 v = unpack2(acc[rr]);
+        ap[rr] = v.x + v.y;
+      }
+      rp = r0;
+      pp.advance();
+    }
+    if (rp >= 0) warp_reduce_rows<RPS>(ap, red + rp, lane, nrows - rp);
+  } else
+#endif
   for (int r0 = 0; r0 < nrows; r0 += RPS) {
     const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
@@ -303,7 +356,7 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
         if (RPS == 1 || r0 + rs + rr < nrows) {
 #pragma unroll
           for (int s = 0; s < NSEG; ++s) {
-            if (s < NSEG - 1 || last_ok) {
+            if (seg_ok(s)) {
               const uint4 w = *reinterpret_cast<const uint4*>(base + (rs + rr) * row_bytes + s * kSegBytes);
               if (BM == 1) {
                 dot8(w, x2[0][s], acc[rr][0]);
@@ -425,7 +478,7 @@ __device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, c
 // ---------------------------------------------------------------------------------------
 // Split-KV attention chunk for one (sequence, KV head): scores of its G query heads over the
 // chunk's keys, per-warp online softmax, merged across warps into one partial (m, l, acc).
-// At the current length only nch_eff = ceil(L / kMinChunkKeys) (at most nch) chunks hold keys;
+// At the current length only nch_eff = ceil(L / min_chunk_keys) (at most nch) chunks hold keys;
 // the other chunk tasks only count their arrival.  The last task of the (sequence, KV head)
 // to arrive merges the partials into o (FlashDecoding-style online-softmax merge) and
 // notifies; with a single chunk in use that chunk writes o directly and nothing is merged.
@@ -462,7 +515,7 @@ __device__ __forceinline__ AttnGeom attn_geom(const DecodeParams& P, const Task&
     a.j0 = a.j1 = 0;
     return a;
   }
-  a.nch_eff = max(1, min(P.nch, (a.Lk + kMinChunkKeys - 1) / kMinChunkKeys));
+  a.nch_eff = max(1, min(P.nch, (a.Lk + P.min_chunk_keys - 1) / P.min_chunk_keys));
   const int cl = (a.Lk + a.nch_eff - 1) / a.nch_eff;
   a.j0 = a.c * cl;
   a.j1 = (a.c < a.nch_eff) ? min(a.Lk, a.j0 + cl) : a.j0;

@@ -87,6 +87,7 @@ struct mk_ctx {
   int drop_event = -1;
   uint64_t* trace = nullptr;
   int l2_ahead = 8;  // L2 lookahead stages while the ring is full (mk_set_l2_prefetch)
+  int min_chunk_keys = kMinChunkKeysDefault;  // split-KV chunk length floor (mk_set_attn_chunk_keys)
   std::vector<double> sm_weights;  // relative streaming speed per SM (partition weights)
   std::vector<double> op_weights[8];  // per projection kind; empty = sm_weights
   size_t task_cap = 0, lm_cap = 0; // workspace capacity for re-partitioned graphs
@@ -1735,6 +1736,7 @@ void make_params(const mk_ctx* c, const mk_ctx* run, const int32_t* tokens, int 
   P.timeout_ns = run->timeout_ns;
   P.trace = run->trace;
   P.l2_ahead = c->dyn ? 0 : run->l2_ahead;  // the lookahead walks static queues only
+  P.min_chunk_keys = run->min_chunk_keys;
   P.tp_ranks = 1;
 }
 
@@ -1958,6 +1960,12 @@ int mk_set_dispatch(mk_ctx* c, int mode, int tasks_per_sm, void* stream) {
 int mk_set_l2_prefetch(mk_ctx* c, int stages) {
   if (!c || stages < 0 || stages > 64) return fail(c, MK_ERR_INVALID_ARG, "stages must be in [0, 64]");
   c->l2_ahead = stages;
+  return MK_OK;
+}
+
+int mk_set_attn_chunk_keys(mk_ctx* c, int keys) {
+  if (!c || keys < 1 || keys > (1 << 20)) return fail(c, MK_ERR_INVALID_ARG, "keys must be in [1, 2^20]");
+  c->min_chunk_keys = keys;
   return MK_OK;
 }
 
