@@ -5,16 +5,17 @@
 // fp16) with FlashDecoding-style split-KV, which the same article names among the designs
 // its search covers.  fp32 accumulation and softmax.
 //
-// Work split: the keys of all heads form BH * ceil(L/64) units of 64 keys; CTA c of G takes
+// Work split: the keys of all heads form BH * ceil(L/128) units of 128 keys; CTA c of G takes
 // units [c*U/G, (c+1)*U/G), so every SM streams the same number of bytes.  A TMA producer
-// warp keeps a 6-stage ring of (K^T tile [d][64], V tile [64][d]) fp16 tiles full, in unit
-// order.  The eight compute warps work independently: warp w takes the CTA's units of a head
-// round-robin (the head's first unit in the CTA, then every eighth), each with its own running
-// (max, sum, acc) -- lane l scores keys 2l and 2l+1 over all d, then owns d/32 output dims in
-// P.V -- and releases the stage it read.  Only at the end of a head's units in the CTA do the
-// warps meet: their partials are combined in shared memory into one partial per (CTA, head);
-// a head inside one CTA is written out directly, otherwise the last CTA to finish the head
-// (atomic arrival count) merges the CTAs' partials and resets the count to zero.
+// warp keeps a 3-stage ring of (K^T tile [d][128], V tile [128][d]) fp16 tiles full, in unit
+// order (a K^T tile is d rows of 256 contiguous bytes).  The eight compute warps work
+// independently and never wait for each other: warp w takes units u0 + w, u0 + w + 8, ..., each
+// with its own running (max, sum, acc) -- lane l scores keys 4l .. 4l+3 over all d, then owns
+// d/32 output dims in P.V -- and releases the stage it read.  At the end of its units of a
+// head a warp leaves its partial in a shared-memory slot of the head and goes on (it already
+// loaded the next head's q); the last of the head's warps to arrive combines the slot into one
+// partial per (CTA, head), written out directly if the head lies inside the CTA, else merged by
+// the last CTA to finish the head (atomic arrival count, reset to zero by that CTA).
 //
 // L % 8 != 0 cannot be described to TMA (row stride must be a multiple of 16 bytes); those
 // shapes take a plain-load kernel (attention_plain) that needs no workspace.
@@ -34,8 +35,8 @@
 namespace mk {
 namespace attn {
 
-constexpr int kUnit = 64;             // keys per unit (one ring stage)
-constexpr int kStages = 6;
+constexpr int kUnit = 128;            // keys per unit (one ring stage): 256-byte K^T rows
+constexpr int kStages = 3;
 constexpr int kComputeWarps = 8;
 constexpr int kThreads = (kComputeWarps + 1) * 32;  // + producer warp
 constexpr int kMaxD = 128;
@@ -45,7 +46,8 @@ struct Params {
   float* o;             // [BH][d]
   float* part;          // [BH][maxc][d + 2]: per-(head, CTA) partials (m, l, acc[d])
   uint32_t* cnt;        // [BH] arrival counts, zero between calls
-  uint32_t* err;        // error word: 0 = ok, else 1 + role of the first wait that ran out
+  uint32_t* err;        // error word: 0 = ok, else the role of the first wait that ran out
+                        // (1 producer slot, 2 tile arrival, 3 combine slot)
   int BH, d, L, nu, U, G, maxc;
   float scale;
   uint64_t timeout_ns;
@@ -76,19 +78,21 @@ __device__ __forceinline__ float2 h2f2(uint32_t w) {
 }
 
 struct Smem {
-  alignas(128) uint16_t kt[kStages][kMaxD * kUnit];  // [d][64]
-  alignas(128) uint16_t v[kStages][kUnit * kMaxD];   // [64][d]
+  alignas(128) uint16_t kt[kStages][kMaxD * kUnit];  // [d][128 keys]
+  alignas(128) uint16_t v[kStages][kUnit * kMaxD];   // [128 keys][d]
   alignas(16) float qs[kComputeWarps][kMaxD];        // each warp's scaled q of its current head
   alignas(16) float ps[kComputeWarps][kUnit];        // each warp's probabilities of its current unit
-  float wacc[kComputeWarps][kMaxD];                  // per-warp partial outputs at a head's end
-  float wm[kComputeWarps], wl[kComputeWarps];
-  uint32_t last;                                     // this CTA merges the head when set
-  volatile uint32_t abort;                           // a wait ran out: every role stops waiting
-  int abort_epoch;  // first compute-barrier epoch whose barrier follows an abort (INT_MAX: none)
+  // per-head combine slots (double-buffered by head parity): every warp that took units of the
+  // head leaves its (m, l, acc) here; the last one to arrive combines them
+  float cm[2][kComputeWarps], cl[2][kComputeWarps];
+  alignas(16) float cacc[2][kComputeWarps][kMaxD];
+  uint32_t ccount[2];    // warps that left their partial in the slot
+  int cowner[2];         // head that owns the slot (-1: free)
+  volatile uint32_t abort;  // a wait ran out: every role stops waiting
   // unit whose tiles the producer armed stage s for.  Eight warps take units round-robin over
-  // six stages, so a warp can reach a stage's next use before the previous use's tiles have
-  // landed; a parity wait cannot tell those phases apart.  A warp first waits until its stage
-  // is armed for its unit (the previous use is then complete), then on the stage's phase.
+  // the ring's stages, so a warp can reach a stage's next use before the previous use's tiles
+  // have landed; a parity wait cannot tell those phases apart.  A warp first waits until its
+  // stage is armed for its unit (the previous use is then complete), then on the stage's phase.
   uint32_t armed[kStages];
   alignas(8) uint64_t full[kStages];
   alignas(8) uint64_t empty[kStages];
@@ -109,12 +113,12 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_
   }
 }
 
-// Bounded wait until the producer armed a stage for unit u: false once `limit_ns` passed or
-// another role aborted.
-__device__ __forceinline__ bool wait_armed(uint32_t* armed, uint32_t u, uint64_t limit_ns, volatile uint32_t* abort) {
+// Bounded wait until *word == want (acquire): false once `limit_ns` passed or another role
+// aborted.
+__device__ __forceinline__ bool wait_word(uint32_t* word, uint32_t want, uint64_t limit_ns, volatile uint32_t* abort) {
   uint64_t t0 = 0;
   for (uint32_t n = 1;; ++n) {
-    if (ld_acquire_cta_shared(armed) == u) return true;
+    if (ld_acquire_cta_shared(word) == want) return true;
     if ((n & 255u) == 0) {
       if (*abort) return false;
       const uint64_t now = globaltimer_ns();
@@ -129,15 +133,126 @@ __device__ __forceinline__ void report_timeout(uint32_t* err, uint32_t code, vol
   atomicCAS(err, 0u, code);
 }
 
-// Compute-warp barrier.  Every compute warp passes the same sequence of barriers; `epoch`
-// counts them.  A warp whose wait ran out records (atomicMin) the epoch of the next barrier it
-// will reach; after barrier e every warp leaves iff the recorded epoch is <= e.  A value <= e
-// can only have been written before barrier e, so the decision is the same in every warp.
-__device__ __forceinline__ bool compute_bar(Smem& S, int& epoch) {
-  named_bar_sync(1, kComputeWarps * 32);
-  const bool stop = S.abort_epoch <= epoch;
-  ++epoch;
-  return stop;
+// End of a warp's units of head h in this CTA: leave its partial in the head's combine slot.
+// The last of the head's contributing warps (nw of them, the first being warp w0) combines the
+// slot into one partial per (CTA, head): written out directly if the head lies inside this CTA,
+// else stored for the cross-CTA merge, which the last CTA to finish the head performs.  Warp-
+// uniform; false if the slot wait ran out.
+template <int D>
+__device__ __forceinline__ bool flush_head(const Params& P, Smem& S, int h, int c, int w0, int nw, float m, float l,
+                                           const float (&acc)[D / 32], int warp, int lane) {
+  constexpr int DL = D / 32;
+  const int sl = h & 1;
+  // claim the slot for head h (free, or already claimed by another warp of this head)
+  {
+    uint64_t t0 = 0;
+    for (uint32_t n = 1;; ++n) {
+      int own = -1;
+      if (lane == 0) {
+        own = atomicCAS(&S.cowner[sl], -1, h);
+      }
+      own = __shfl_sync(0xffffffffu, own, 0);
+      if (own == -1 || own == h) {
+        __threadfence_block();  // the previous owner's reset of the count is seen
+        break;
+      }
+      if ((n & 15u) == 0) {
+        if (S.abort) return false;
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > P.timeout_ns) return false;
+      }
+    }
+  }
+  if (lane == 0) {
+    S.cm[sl][warp] = m;
+    S.cl[sl][warp] = l;
+  }
+#pragma unroll
+  for (int i = 0; i < DL; ++i) S.cacc[sl][warp][lane * DL + i] = acc[i];
+  __syncwarp();
+  uint32_t arrived = 0;
+  if (lane == 0) {
+    __threadfence_block();
+    arrived = atomicAdd(&S.ccount[sl], 1u) + 1u;
+  }
+  arrived = __shfl_sync(0xffffffffu, arrived, 0);
+  if (arrived != (uint32_t)nw) return true;
+  // this warp combines: every contributing warp's writes are visible (fence + atomic)
+  __threadfence_block();
+  float M = -INFINITY;
+  for (int k = 0; k < nw; ++k) M = fmaxf(M, S.cm[sl][(w0 + k) & (kComputeWarps - 1)]);
+  float ls = 0.f, as[DL];
+#pragma unroll
+  for (int i = 0; i < DL; ++i) as[i] = 0.f;
+  for (int k = 0; k < nw; ++k) {
+    const int w = (w0 + k) & (kComputeWarps - 1);
+    const float f = __expf(S.cm[sl][w] - M);
+    ls = fmaf(f, S.cl[sl][w], ls);
+#pragma unroll
+    for (int i = 0; i < DL; ++i) as[i] = fmaf(f, S.cacc[sl][w][lane * DL + i], as[i]);
+  }
+  // the slot is read: free it for head h + 2
+  __syncwarp();
+  if (lane == 0) {
+    S.ccount[sl] = 0u;
+    __threadfence_block();
+    atomicExch(&S.cowner[sl], -1);
+  }
+  const int cf = unit_owner(h * P.nu, P.U, P.G), cl = unit_owner((h + 1) * P.nu - 1, P.U, P.G);
+  if (cf == cl) {  // the head lies inside this CTA
+#pragma unroll
+    for (int i = 0; i < DL; ++i) P.o[(size_t)h * D + lane * DL + i] = as[i] / ls;
+    return true;
+  }
+  float* part = P.part + ((size_t)h * P.maxc + (c - cf)) * (D + 2);
+#pragma unroll
+  for (int i = 0; i < DL; ++i) part[2 + lane * DL + i] = as[i];
+  if (lane == 0) {
+    part[0] = M;
+    part[1] = ls;
+  }
+  __syncwarp();
+  uint32_t last = 0;
+  const uint32_t n = (uint32_t)(cl - cf + 1);
+  if (lane == 0) {
+    __threadfence();
+    const uint32_t old = atom_acq_rel_gpu_add(&P.cnt[h], 1u);
+    last = (old + 1 == n) ? 1u : 0u;
+    if (last) P.cnt[h] = 0u;  // self-cleaning for the next call
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return true;
+  // the last CTA of the head merges every CTA's partial, eight per L2 round trip
+  __threadfence();
+  const float* base = P.part + (size_t)h * P.maxc * (D + 2);
+  float M2 = -INFINITY;
+  for (int i = 0; i < (int)n; ++i) M2 = fmaxf(M2, __ldcg(base + (size_t)i * (D + 2)));
+  float num[DL], den = 0.f;
+#pragma unroll
+  for (int i = 0; i < DL; ++i) num[i] = 0.f;
+  for (int i0 = 0; i0 < (int)n; i0 += 8) {
+    float mv[8], lv[8], av[8][DL];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const bool in = i0 + k < (int)n;
+      const float* pi = base + (size_t)(in ? i0 + k : 0) * (D + 2);
+      mv[k] = in ? __ldcg(pi) : -INFINITY;
+      lv[k] = in ? __ldcg(pi + 1) : 0.f;
+#pragma unroll
+      for (int i = 0; i < DL; ++i) av[k][i] = in ? __ldcg(pi + 2 + lane * DL + i) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float f = (mv[k] == -INFINITY) ? 0.f : __expf(mv[k] - M2);
+      den = fmaf(f, lv[k], den);
+#pragma unroll
+      for (int i = 0; i < DL; ++i) num[i] = fmaf(f, av[k][i], num[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < DL; ++i) P.o[(size_t)h * D + lane * DL + i] = num[i] / den;
+  return true;
 }
 
 template <int D>
@@ -154,10 +269,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);  // the one warp that read the stage releases it
+      S.armed[s] = 0xffffffffu;
+    }
+    for (int s = 0; s < 2; ++s) {
+      S.ccount[s] = 0u;
+      S.cowner[s] = -1;
     }
     S.abort = 0;
-    S.abort_epoch = INT_MAX;
-    for (int s = 0; s < kStages; ++s) S.armed[s] = 0xffffffffu;
     fence_mbar_init();
   }
   __syncthreads();
@@ -203,168 +321,132 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---------------- compute warps ----------------
+  // Warp w takes units u0 + w, u0 + w + 8, ... (heads in order), each with its own running
+  // (max, sum, acc); at the end of its units of a head it leaves its partial in the head's
+  // combine slot (flush_head) and goes on.  No compute-warp barrier: a wait that runs out
+  // makes the warp skip its remaining work.
   constexpr int DL = D / 32;  // output dims per lane in P.V
-  int epoch = 0;
-  bool failed = false;  // this warp saw a wait run out (warp-uniform)
+  constexpr int KPL = kUnit / 32;  // keys per lane in the scores (4)
   float* qs = S.qs[warp];
   float* ps = S.ps[warp];
-  for (int hu0 = u0; hu0 < u1;) {
-    const int h = hu0 / P.nu;
-    const int hu1 = min(u1, (h + 1) * P.nu);  // this CTA's units of head h: [hu0, hu1)
-    // the warp's own copy of q (scaled), read back as broadcasts
-    {
-      const uint16_t* qh = P.q + (size_t)h * D + lane * DL;
-#pragma unroll
-      for (int i = 0; i < DL; ++i) qs[lane * DL + i] = h2f(__ldg(qh + i)) * P.scale;
+  bool alive = true;
+  int cur_h = -1;
+  float m = -INFINITY, l = 0.f, acc[DL];
+  float qn[DL];  // the next head's q (prefetched)
+  auto flush = [&](int h) {
+    const int a = max(u0, h * P.nu), b = min(u1, (h + 1) * P.nu);  // the head's units in this CTA
+    const int nw = min(kComputeWarps, b - a), w0 = (a - u0) & (kComputeWarps - 1);
+    if (alive && !flush_head<D>(P, S, h, c, w0, nw, m, l, acc, warp, lane)) {
+      if (lane == 0) report_timeout(P.err, 3u, &S.abort);
+      alive = false;
     }
-    __syncwarp();
-    float m = -INFINITY, l = 0.f, acc[DL];
+  };
+  for (int u = u0 + warp; u < u1 && alive; u += kComputeWarps) {
+    const int h = u / P.nu;
+    if (h != cur_h) {
+      if (cur_h >= 0) flush(cur_h);
+      if (cur_h < 0) {  // the first head's q (later heads were prefetched)
+        const uint16_t* qh = P.q + (size_t)h * D + lane * DL;
 #pragma unroll
-    for (int i = 0; i < DL; ++i) acc[i] = 0.f;
-    for (int u = hu0 + warp; u < hu1; u += kComputeWarps) {
-      const int idx = u - u0, stage = idx % kStages;
-      const uint32_t parity = (uint32_t)(idx / kStages) & 1u;
-      bool ok = !failed && wait_armed(&S.armed[stage], (uint32_t)u, P.timeout_ns, &S.abort) &&
-                wait_bar(&S.full[stage], parity, P.timeout_ns, &S.abort);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        if (!failed && lane == 0) {
-          report_timeout(P.err, 2u, &S.abort);
-          atomicMin(&S.abort_epoch, epoch);
-        }
-        failed = true;
-        continue;
+        for (int i = 0; i < DL; ++i) qn[i] = h2f(__ldg(qh + i)) * P.scale;
       }
-      const int valid = min(kUnit, P.L - (u % P.nu) * kUnit);
-      // scores: lane owns keys 2*lane, 2*lane+1; row dd of the K^T tile holds 64 keys
-      const uint32_t* kt = reinterpret_cast<const uint32_t*>(S.kt[stage]) + lane;
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-      for (int dd = 0; dd < D; dd += 4) {
-        const float4 q4 = *reinterpret_cast<const float4*>(qs + dd);
-        const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 k2 = h2f2(kt[(dd + e) * (kUnit / 2)]);
-          sa[e] = fmaf(qv[e], k2.x, sa[e]);
-          sb[e] = fmaf(qv[e], k2.y, sb[e]);
-        }
-      }
-      float s0 = (sa[0] + sa[1]) + (sa[2] + sa[3]);
-      float s1 = (sb[0] + sb[1]) + (sb[2] + sb[3]);
-      if (2 * lane >= valid) s0 = -INFINITY;
-      if (2 * lane + 1 >= valid) s1 = -INFINITY;
-      float bm = fmaxf(s0, s1);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-      const float m_new = fmaxf(m, bm);  // finite: the unit holds at least one key
-      const float alpha = __expf(m - m_new);  // 0 on the first unit (m = -inf)
-      const float p0 = __expf(s0 - m_new), p1 = __expf(s1 - m_new);
-      float psum = p0 + p1;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
-      l = fmaf(l, alpha, psum);
-      m = m_new;
-#pragma unroll
-      for (int i = 0; i < DL; ++i) acc[i] *= alpha;
-      *reinterpret_cast<float2*>(ps + 2 * lane) = make_float2(p0, p1);
+      for (int i = 0; i < DL; ++i) qs[lane * DL + i] = qn[i];
       __syncwarp();
-      // P.V: lane owns dims lane*DL .. lane*DL + DL - 1 (keys past L have p = 0 and zero rows)
-      const uint16_t* vt = S.v[stage] + lane * DL;
+      // the q of the head after this one, loaded while this one runs
+      {
+        const int hn = min(h + 1, P.BH - 1);
+        const uint16_t* qh = P.q + (size_t)hn * D + lane * DL;
+#pragma unroll
+        for (int i = 0; i < DL; ++i) qn[i] = h2f(__ldg(qh + i)) * P.scale;
+      }
+      cur_h = h;
+      m = -INFINITY;
+      l = 0.f;
+#pragma unroll
+      for (int i = 0; i < DL; ++i) acc[i] = 0.f;
+    }
+    const int idx = u - u0, stage = idx % kStages;
+    const uint32_t parity = (uint32_t)(idx / kStages) & 1u;
+    bool ok = wait_word(&S.armed[stage], (uint32_t)u, P.timeout_ns, &S.abort) &&
+              wait_bar(&S.full[stage], parity, P.timeout_ns, &S.abort);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) {
+      if (lane == 0) report_timeout(P.err, 2u, &S.abort);
+      alive = false;
+      break;
+    }
+    const int valid = min(kUnit, P.L - (u % P.nu) * kUnit);
+    // scores: lane owns keys KPL*lane .. KPL*lane + KPL-1; row dd of the K^T tile holds 128 keys
+    const uint16_t* kt = S.kt[stage] + lane * KPL;
+    float sa[KPL], sb[KPL];
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) sa[k] = sb[k] = 0.f;
 #pragma unroll 4
-      for (int k = 0; k < kUnit; k += 4) {
-        const float4 p4 = *reinterpret_cast<const float4*>(ps + k);
-        const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+    for (int dd = 0; dd < D; dd += 4) {
+      const float4 q4 = *reinterpret_cast<const float4*>(qs + dd);
+      const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if constexpr (DL == 4) {
-            const uint2 w = *reinterpret_cast<const uint2*>(vt + (k + e) * D);
-            const float2 a = h2f2(w.x), b = h2f2(w.y);
-            acc[0] = fmaf(pv[e], a.x, acc[0]);
-            acc[1] = fmaf(pv[e], a.y, acc[1]);
-            acc[2] = fmaf(pv[e], b.x, acc[2]);
-            acc[3] = fmaf(pv[e], b.y, acc[3]);
-          } else {
-            const float2 a = h2f2(*reinterpret_cast<const uint32_t*>(vt + (k + e) * D));
-            acc[0] = fmaf(pv[e], a.x, acc[0]);
-            acc[1] = fmaf(pv[e], a.y, acc[1]);
-          }
+      for (int e = 0; e < 4; ++e) {
+        const uint2 w = *reinterpret_cast<const uint2*>(kt + (dd + e) * kUnit);
+        const float2 k01 = h2f2(w.x), k23 = h2f2(w.y);
+        float* s = (e & 1) ? sb : sa;
+        s[0] = fmaf(qv[e], k01.x, s[0]);
+        s[1] = fmaf(qv[e], k01.y, s[1]);
+        s[2] = fmaf(qv[e], k23.x, s[2]);
+        s[3] = fmaf(qv[e], k23.y, s[3]);
+      }
+    }
+    float sc[KPL], bm = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+      sc[k] = (lane * KPL + k < valid) ? sa[k] + sb[k] : -INFINITY;
+      bm = fmaxf(bm, sc[k]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+    const float m_new = fmaxf(m, bm);  // finite: the unit holds at least one key
+    const float alpha = __expf(m - m_new);  // 0 on the head's first unit (m = -inf)
+    float p[KPL], psum = 0.f;
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+      p[k] = __expf(sc[k] - m_new);
+      psum += p[k];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+    l = fmaf(l, alpha, psum);
+    m = m_new;
+#pragma unroll
+    for (int i = 0; i < DL; ++i) acc[i] *= alpha;
+    *reinterpret_cast<float4*>(ps + KPL * lane) = make_float4(p[0], p[1], p[2], p[3]);
+    __syncwarp();
+    // P.V: lane owns dims lane*DL .. lane*DL + DL - 1 (keys past L have p = 0 and zero rows)
+    const uint16_t* vt = S.v[stage] + lane * DL;
+#pragma unroll 4
+    for (int k = 0; k < kUnit; k += 4) {
+      const float4 p4 = *reinterpret_cast<const float4*>(ps + k);
+      const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if constexpr (DL == 4) {
+          const uint2 w = *reinterpret_cast<const uint2*>(vt + (k + e) * D);
+          const float2 a = h2f2(w.x), b = h2f2(w.y);
+          acc[0] = fmaf(pv[e], a.x, acc[0]);
+          acc[1] = fmaf(pv[e], a.y, acc[1]);
+          acc[2] = fmaf(pv[e], b.x, acc[2]);
+          acc[3] = fmaf(pv[e], b.y, acc[3]);
+        } else {
+          const float2 a = h2f2(*reinterpret_cast<const uint32_t*>(vt + (k + e) * D));
+          acc[0] = fmaf(pv[e], a.x, acc[0]);
+          acc[1] = fmaf(pv[e], a.y, acc[1]);
         }
       }
-      __syncwarp();  // every lane's reads of the stage and of ps are done
-      if (lane == 0) mbar_arrive(&S.empty[stage]);
     }
-    // end of the head's units in this CTA: combine the warps' partials
-    if (lane == 0) {
-      S.wm[warp] = m;
-      S.wl[warp] = l;
-    }
-#pragma unroll
-    for (int i = 0; i < DL; ++i) S.wacc[warp][lane * DL + i] = acc[i];
-    if (compute_bar(S, epoch)) return;
-    const int cf = unit_owner(h * P.nu, P.U, P.G), cl = unit_owner((h + 1) * P.nu - 1, P.U, P.G);
-    if (tid < D) {
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, S.wm[w]);
-      float ls = 0.f, as = 0.f;
-#pragma unroll
-      for (int w = 0; w < kComputeWarps; ++w) {
-        const float f = (S.wm[w] == -INFINITY) ? 0.f : __expf(S.wm[w] - M);  // warps without units add 0
-        ls = fmaf(f, S.wl[w], ls);
-        as = fmaf(f, S.wacc[w][tid], as);
-      }
-      if (cf == cl) {
-        P.o[(size_t)h * D + tid] = as / ls;  // the head lies inside this CTA
-      } else {
-        float* part = P.part + ((size_t)h * P.maxc + (c - cf)) * (D + 2);
-        part[2 + tid] = as;
-        if (tid == 0) {
-          part[0] = M;
-          part[1] = ls;
-        }
-      }
-    }
-    if (cf != cl) {
-      if (compute_bar(S, epoch)) return;
-      if (tid == 0) {
-        __threadfence();
-        const uint32_t n = (uint32_t)(cl - cf + 1);
-        const uint32_t old = atom_acq_rel_gpu_add(&P.cnt[h], 1u);
-        S.last = (old + 1 == n) ? n : 0u;
-        if (old + 1 == n) P.cnt[h] = 0u;  // self-cleaning for the next call
-      }
-      if (compute_bar(S, epoch)) return;
-      if (S.last && tid < D) {
-        __threadfence();
-        const int n = (int)S.last;
-        const float* base = P.part + (size_t)h * P.maxc * (D + 2);
-        float M = -INFINITY;
-        for (int i = 0; i < n; ++i) M = fmaxf(M, __ldcg(base + (size_t)i * (D + 2)));
-        float num = 0.f, den = 0.f;
-        for (int i0 = 0; i0 < n; i0 += 8) {  // eight partials per L2 round trip
-          float mv[8], lv[8], av[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const bool in = i0 + k < n;
-            const float* pi = base + (size_t)(in ? i0 + k : 0) * (D + 2);
-            mv[k] = in ? __ldcg(pi) : -INFINITY;
-            lv[k] = in ? __ldcg(pi + 1) : 0.f;
-            av[k] = in ? __ldcg(pi + 2 + tid) : 0.f;
-          }
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const float w = (mv[k] == -INFINITY) ? 0.f : __expf(mv[k] - M);
-            den = fmaf(w, lv[k], den);
-            num = fmaf(w, av[k], num);
-          }
-        }
-        P.o[(size_t)h * D + tid] = num / den;
-      }
-    }
-    if (compute_bar(S, epoch)) return;  // S.wacc / S.last are reused by the next head
-    hu0 = hu1;
+    __syncwarp();  // every lane's reads of the stage and of ps are done
+    if (lane == 0) mbar_arrive(&S.empty[stage]);
   }
+  if (alive && cur_h >= 0) flush(cur_h);
 }
 
 // Plain-load path for any L: one CTA per head, scores staged in shared memory in chunks.

@@ -31,10 +31,6 @@
 #include "mk_internal.h"
 #include "mk_ptx.cuh"
 
-#ifndef MK_GEMV_PIPE
-#define MK_GEMV_PIPE 1  // batch width 1: software-pipelined stage loop (0: the plain loop)
-#endif
-
 namespace mk {
 
 // Dynamic shared memory: the weight ring (nst stages of kSlotBytes, 1024-aligned), then for
@@ -44,6 +40,8 @@ struct DSmem {
     float red[kWorkerWarps][kTaskRows];  // GEMV: per-warp sums of the current task, [row][seq]
     float aacc[kAttnWarps][4][128];      // attention: per-warp partial outputs
     float tile[kTcRecFloats];            // tensor-core tile: summed partial records
+    float wp[kAttnWarps][512];           // wide attention: a warp's probabilities [head][key] (warp w
+                                         // uses only row w, which its own aacc row overlays)
   };
   float tot[kTaskRows];                  // totals of the current task, [row][seq]
   float ssw[kWorkerWarps][kMaxDecodeBatch];  // per-warp sums of x^2 per sequence
@@ -67,6 +65,10 @@ struct DSmem {
   uint64_t mma_done;         // every MMA issued so far completed (issuer drain at exit)
   uint32_t tmem;             // tensor-memory accumulators (2 x kTcN columns)
   uint32_t ready;            // tasks [0, ready) of this queue have their inputs
+  // ring stage s holds the stage with this launch-wide sequence number (published by the
+  // producer once armed): a warp that takes stages out of order (wide attention) first waits
+  // for its stage's number, so a parity wait is never a phase ahead
+  uint32_t armed[kStages];
   uint32_t cabort;           // worker-role abort: written before, read after a worker barrier
   volatile uint32_t abort;   // any role gave up: stop waiting
   uint32_t flag;             // worker broadcast (last-arriver decisions)
@@ -116,8 +118,10 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, uint64_
 struct Pipe {
   int stage;
   uint32_t phase;
-  int nst;  // ring depth
+  int nst;       // ring depth
+  uint32_t seq;  // launch-wide number of the next stage
   __device__ __forceinline__ void advance() {
+    ++seq;
     if (++stage == nst) {
       stage = 0;
       phase ^= 1u;
@@ -288,52 +292,6 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
   }
   float* red = S.red[warp];
   bool ok = true;
-#if MK_GEMV_PIPE
-  if constexpr (BM == 1) {
-    // Batch width 1, software-pipelined: the cross-lane reduction of stage i-1's partial sums
-    // (a chain of shuffles) is issued between stage i's shared-memory loads and its FMAs, so
-    // the shuffle latency overlaps the load latency instead of following the FMAs.  Every
-    // stage computes all RPS rows (rows past nrows read stale but in-bounds ring bytes; their
-    // sums are never stored), so the stage body has no branches.
-    float ap[RPS];
-    int rp = -1;  // first row of the partial sums in ap (-1: none yet)
-    for (int r0 = 0; r0 < nrows; r0 += RPS) {
-      const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
-      if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
-        if (ok) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
-        ok = false;
-        S.cabort = 1u;
-      }
-      if (P.trace && tid == 0) stall_ns += (uint32_t)(globaltimer_ns() - tw);
-      const uint8_t* base = ring + (size_t)pp.stage * kSlotBytes + tid * 16;
-      uint4 w[RPS][NSEG];
-#pragma unroll
-      for (int rr = 0; rr < RPS; ++rr)
-#pragma unroll
-        for (int s = 0; s < NSEG; ++s)
-          w[rr][s] = seg_ok(s) ? *reinterpret_cast<const uint4*>(base + rr * row_bytes + s * kSegBytes)
-                               : make_uint4(0u, 0u, 0u, 0u);
-      if (rp >= 0) warp_reduce_rows<RPS>(ap, red + rp, lane, nrows - rp);
-      uint64_t acc[RPS];
-#pragma unroll
-      for (int rr = 0; rr < RPS; ++rr) {
-        acc[rr] = 0ull;
-#pragma unroll
-        for (int s = 0; s < NSEG; ++s) dot8(w[rr][s], x2[0][s], acc[rr]);
-      }
-      __syncwarp();  // every lane's reads of the stage are done: release it
-      if (lane == 0) mbar_arrive(&S.empty[pp.stage]);
-#pragma unroll
-      for (int rr = 0; rr < RPS; ++rr) {
-        const float2 v = unpack2(acc[rr]);
-        ap[rr] = v.x + v.y;
-      }
-      rp = r0;
-      pp.advance();
-    }
-    if (rp >= 0) warp_reduce_rows<RPS>(ap, red + rp, lane, nrows - rp);
-  } else
-#endif
   for (int r0 = 0; r0 < nrows; r0 += RPS) {
     const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
     if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
@@ -728,6 +686,177 @@ __device__ __forceinline__ int attn_stage_span(const AttnGeom& a, int* jend) {
   return *jend > a.j0 ? (*jend - a.j0 + kv_stage_keys<D>() - 1) / kv_stage_keys<D>() : 0;
 }
 
+// Wide attention (long chunks): warp w takes ring stages w, w + 8, ... of the chunk's cached keys,
+// each whole, with its own online softmax.  Lane l scores keys l*KPL .. l*KPL + KPL-1 of the
+// stage over every dim (reading its K words in the rotated order (t + l) mod (D/2), so the 32
+// lanes hit 32 banks, and the matching q words of the scaled q in S.qn), then owns D/32 output
+// dims of P.V, with the stage's probabilities read back as broadcasts from its row of S.wp.
+// Stages are taken out of order, so a warp first waits until its stage is armed with its
+// launch-wide number (S.armed), then on the stage's phase; it releases the stage for every
+// worker warp at once.  False if a wait ran out (the warp then skips its remaining stages).
+constexpr int kWideMinStages = 3;
+
+template <int D, int GW>
+__device__ __forceinline__ bool attn_wide(const DecodeParams& P, DSmem& S, const Pipe& pp, const uint8_t* ring,
+                                          const AttnGeom& a, int jend, int nst, int G, float (&m)[4], float (&l)[4],
+                                          float (&acc)[4][D / 32], int lane, int warp, uint32_t task_id,
+                                          uint32_t& stall_ns) {
+  constexpr int KPS = kv_stage_keys<D>();  // keys per stage: 64 (D = 128) or 128 (D = 64)
+  constexpr int W2 = D / 2;                 // 32-bit words (bf16 pairs) per K row
+  constexpr int KPL = KPS / 32;             // keys a lane scores
+  constexpr int DL = D / 32;
+  float* pw = S.wp[warp];  // [GW][KPS]
+  const float* qs = S.qn;  // [G][D], scaled
+  bool ok = true;
+  for (int i = warp; i < nst; i += kAttnWarps) {
+    int pos = pp.stage + i;
+    uint32_t ph = pp.phase;
+    while (pos >= pp.nst) {
+      pos -= pp.nst;
+      ph ^= 1u;
+    }
+    const uint32_t seq = pp.seq + (uint32_t)i;
+    const uint64_t tw = (P.trace && lane == 0 && warp == 0) ? globaltimer_ns() : 0;
+    bool got = ok;
+    if (got) {  // bounded: the stage armed with this number, then its phase
+      uint64_t t0 = 0;
+      for (uint32_t n = 1;; ++n) {
+        if (ld_acquire_cta_shared(&S.armed[pos]) == seq) break;
+        if ((n & 127u) == 0) {
+          if (S.abort) {
+            got = false;
+            break;
+          }
+          const uint64_t now = globaltimer_ns();
+          if (t0 == 0) t0 = now;
+          else if (now - t0 > P.timeout_ns) {
+            got = false;
+            break;
+          }
+        }
+      }
+    }
+    got = got && wait_bar(&S.full[pos], ph, P.timeout_ns, &S);
+    got = __all_sync(0xffffffffu, got);
+    if (tw) stall_ns += (uint32_t)(globaltimer_ns() - tw);
+    if (!got) {
+      if (ok && lane == 0) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
+      ok = false;
+      continue;
+    }
+    const uint8_t* kst = ring + (size_t)pos * kSlotBytes;
+    const uint16_t* vst = reinterpret_cast<const uint16_t*>(kst + KPS * D * 2);
+    const int nk = min(KPS, jend - (a.j0 + i * KPS));
+    // scores of this lane's keys for every head
+    float sc[KPL][GW];
+#pragma unroll
+    for (int k = 0; k < KPL; ++k)
+#pragma unroll
+      for (int h = 0; h < GW; ++h) sc[k][h] = 0.f;
+    const uint32_t* kwr = reinterpret_cast<const uint32_t*>(kst) + lane * KPL * W2;
+#pragma unroll 4
+    for (int t = 0; t < W2; ++t) {
+      const int tr = (t + lane) & (W2 - 1);
+      float2 q2[GW];
+#pragma unroll
+      for (int h = 0; h < GW; ++h)
+        q2[h] = (h < G) ? *reinterpret_cast<const float2*>(qs + h * D + 2 * tr) : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < KPL; ++k) {
+        const uint32_t w = kwr[k * W2 + tr];
+        const float k0 = bf16lo(w), k1 = bf16hi(w);
+#pragma unroll
+        for (int h = 0; h < GW; ++h) sc[k][h] = fmaf(q2[h].y, k1, fmaf(q2[h].x, k0, sc[k][h]));
+      }
+    }
+    // online softmax of each head over the stage's keys
+#pragma unroll
+    for (int h = 0; h < GW; ++h) {
+      if (h >= G) continue;
+      float bm = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < KPL; ++k) {
+        if (lane * KPL + k >= nk) sc[k][h] = -INFINITY;
+        bm = fmaxf(bm, sc[k][h]);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+      const float m_new = fmaxf(m[h], bm);  // finite: the stage holds at least one key
+      const float alpha = __expf(m[h] - m_new);
+      float psum = 0.f;
+#pragma unroll
+      for (int k = 0; k < KPL; ++k) {
+        const float p = (lane * KPL + k < nk) ? __expf(sc[k][h] - m_new) : 0.f;
+        pw[h * KPS + lane * KPL + k] = p;
+        psum += p;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+      l[h] = fmaf(l[h], alpha, psum);
+      m[h] = m_new;
+#pragma unroll
+      for (int d = 0; d < DL; ++d) acc[h][d] *= alpha;
+    }
+    __syncwarp();
+    // P.V: lane owns dims lane*DL .. lane*DL + DL-1; keys past nk are skipped (their V bytes are
+    // stale, so they are not weighted by 0)
+    const uint16_t* vl = vst + lane * DL;
+    const int n4 = nk & ~3;
+    for (int k0 = 0; k0 < n4; k0 += 4) {
+      float4 p4[GW];
+#pragma unroll
+      for (int h = 0; h < GW; ++h) p4[h] = *reinterpret_cast<const float4*>(pw + h * KPS + k0);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v[DL];
+        if constexpr (DL == 4) {
+          const uint2 u = *reinterpret_cast<const uint2*>(vl + (k0 + e) * D);
+          v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+        } else {
+          const uint32_t u = *reinterpret_cast<const uint32_t*>(vl + (k0 + e) * D);
+          v[0] = bf16lo(u); v[1] = bf16hi(u);
+        }
+#pragma unroll
+        for (int h = 0; h < GW; ++h) {
+          const float p = e == 0 ? p4[h].x : e == 1 ? p4[h].y : e == 2 ? p4[h].z : p4[h].w;
+#pragma unroll
+          for (int d = 0; d < DL; ++d) acc[h][d] = fmaf(p, v[d], acc[h][d]);
+        }
+      }
+    }
+    for (int k = n4; k < nk; ++k) {
+      float v[DL];
+      if constexpr (DL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(vl + k * D);
+        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+      } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(vl + k * D);
+        v[0] = bf16lo(u); v[1] = bf16hi(u);
+      }
+#pragma unroll
+      for (int h = 0; h < GW; ++h) {
+        if (h >= G) continue;
+        const float p = pw[h * KPS + k];
+#pragma unroll
+        for (int d = 0; d < DL; ++d) acc[h][d] = fmaf(p, v[d], acc[h][d]);
+      }
+    }
+    __syncwarp();  // every lane's reads of the stage and of pw are done
+    if (lane == 0) mbar_arrive_cnt(&S.empty[pos], kWorkerWarps);
+  }
+  return ok;
+}
+
+template <int D>
+__device__ __forceinline__ bool attn_wide_g(const DecodeParams& P, DSmem& S, const Pipe& pp, const uint8_t* ring,
+                                            const AttnGeom& a, int jend, int nst, int G, float (&m)[4], float (&l)[4],
+                                            float (&acc)[4][D / 32], int lane, int warp, uint32_t task_id,
+                                            uint32_t& stall_ns) {
+  if (G == 1) return attn_wide<D, 1>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+  if (G == 2) return attn_wide<D, 2>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+  return attn_wide<D, 4>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+}
+
 // QKN: the model has QK-norm (a separate instantiation, so the plain path keeps its registers).
 template <int D, bool TC, bool QKN>
 __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, Pipe& pp, const uint8_t* ring,
@@ -808,16 +937,27 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
     const int jf0 = max(a.j0, a.pos0), nf = max(0, a.j1 - jf0);
     int jend;
     const int nst = attn_stage_span<D>(a, &jend);
+    const bool wide = nst >= kWideMinStages;  // long chunk: whole stages per warp (attn_wide)
     const int nl = (nst > 0) ? (jend - a.j0) - (nst - 1) * KPS : 0;  // old rows in the last stage
-    const int n_in = (nst > 0) ? min(nf, KPS - nl) : 0;              // fresh rows in its free slots
+    const int n_in = (nst > 0 && !wide) ? min(nf, KPS - nl) : 0;     // fresh rows in its free slots
     const int f_first = ((warp - nl) % kAttnWarps + kAttnWarps) % kAttnWarps;  // this warp's first fresh slot
     uint32_t kpre[kFreshPre][W], vpre[kFreshPre][W];
 #pragma unroll
     for (int j = 0; j < kFreshPre; ++j)
       if (f_first + kAttnWarps * j < n_in)
         attn_load_key<D>(kc, vc, jf0 + f_first + kAttnWarps * j, lane, kpre[j], vpre[j]);
+    if (wide) {
+      // the scaled q of the group's heads in shared memory, read rotated by every lane (with
+      // QK-norm S.qn already holds q, which every warp has first read into its registers)
+      if (QKN) worker_bar();
+      for (int e = tid; e < G * D; e += kWorkerThreads)
+        S.qn[e] = (QKN ? S.qn[e] : __ldcg(qsrc + e)) * P.attn_scale;
+      worker_bar();
+      if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns)) S.cabort = 1u;
+      for (int k = 0; k < nst; ++k) pp.advance();
+    }
     // old positions from the ring, kv_stage_keys per stage (K rows at 0, V rows at KPS * D)
-    for (int st = 0; st < nst; ++st) {
+    for (int st = 0; st < (wide ? 0 : nst); ++st) {
       const int jj = a.j0 + st * KPS, nk = min(KPS, jend - jj);
       const uint64_t tw = (P.trace && tid == 0) ? globaltimer_ns() : 0;
       if (!wait_bar(&S.full[pp.stage], pp.phase, P.timeout_ns, &S)) {
@@ -1267,7 +1407,7 @@ __device__ __forceinline__ bool tc_stage(const DecodeParams& P, DSmem& S, uint8_
 template <int HD>
 __device__ __forceinline__ void tc_issuer(const DecodeParams& P, DSmem& S, const uint8_t* ring, const uint8_t* bop,
                                           uint32_t qb, uint32_t qe, uint32_t tmem) {
-  Pipe pp{0, 0, kTcStages};
+  Pipe pp{0, 0, kTcStages, 0};
   uint32_t gseg = 0, gtask = 0;
   const uint32_t b_base0 = smem_u32(bop);
   bool ok = true;
@@ -1519,6 +1659,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
       mbar_init(&S.acc_free[b], 4);
     }
     S.ready = 0;
+    for (int s = 0; s < NST; ++s) S.armed[s] = 0xffffffffu;
     S.dq_n = 0;
     S.wdone = 0;
     S.cabort = 0;
@@ -1575,7 +1716,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
       }
       return false;
     };
-    Pipe pp{0, 0, NST};
+    Pipe pp{0, 0, NST, 0};
     int issued = 0;
     bool ok = true;
     // run-time claims: hand task `id` of step st to the scheduler and workers (FIFO entry),
@@ -1635,6 +1776,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
         }
         mbar_arrive_expect_tx(&S.full[pp.stage], nr * rb);
         bulk_g2s(ring + (size_t)pp.stage * kSlotBytes, src + (uint64_t)r0 * rb, nr * rb, &S.full[pp.stage], pol);
+        st_release_cta_shared(&S.armed[pp.stage], pp.seq);
         ++issued;
         // the lookahead cursor stays at or in front of the next ring stage
         if (P.l2_ahead > 0) {
@@ -1668,6 +1810,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
         mbar_arrive_expect_tx(&S.full[pp.stage], 2u * bytes);
         bulk_g2s(dst, kc + (size_t)jj * HD, bytes, &S.full[pp.stage], pol);
         bulk_g2s(dst + kv_stage_keys<HD>() * HD * 2, vc + (size_t)jj * HD, bytes, &S.full[pp.stage], pol);
+        st_release_cta_shared(&S.armed[pp.stage], pp.seq);
         ++issued;
         pp.advance();
       }
@@ -1846,7 +1989,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
   }
 
   // --------------------------------- workers ---------------------------------
-  Pipe pp{0, 0, NST};
+  Pipe pp{0, 0, NST, 0};
   // tensor-core pipeline (workers): operand segments staged and tasks finished so far, and
   // whether the next task's first segment was staged ahead
   uint32_t gseg = 0, gtask = 0;

@@ -81,7 +81,7 @@ def test_wait_that_runs_out_is_reported_and_the_workspace_recovers():
     ws = torch.zeros(mk.mk_attention_workspace_bytes(BH, d, L), dtype=torch.uint8, device=dev)
     mk.mk_attention_set_wait_timeout_ns(50_000_000)
     try:
-        mk.mk_attention_debug_drop_unit(70)  # head 2, keys 384..447
+        mk.mk_attention_debug_drop_unit(70)  # head 4, keys 768..895 (units of 128 keys)
         mk.mk_attention_decode(tq, tk, tv, o, BH, d, L, 1.0, ws)
         assert mk.mk_attention_status(ws, BH, d, L) == mk.MK_ERR_DEVICE_TIMEOUT
     finally:
