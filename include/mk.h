@@ -204,11 +204,12 @@ int mk_set_op_sm_weights(mk_ctx* ctx, int op_kind, const float* weights, int n, 
 #define MK_DISPATCH_CLAIM_PRIORITY 3
 int mk_set_dispatch(mk_ctx* ctx, int mode, int tasks_per_sm, void* stream);
 
-/* Weight prefetch depth: besides the shared-memory ring (6 stages of 32 KB per SM), an SM's
- * producer that has been blocked on a full ring for over a microsecond (its workers wait for a
+/* Prefetch depth: besides the shared-memory ring (6 stages of 32 KB per SM), an SM's producer
+ * that has been blocked on a full ring for over a microsecond (its workers wait for a
  * dependency, e.g. during attention) prefetches up to `stages` further weight stages of its
- * queue into L2, so HBM keeps streaming.  Default 8 (measured fastest on B200, 0.7 % faster
- * than 0 = off on the 8B batch-1 decode); at most 64. */
+ * queue into L2, so HBM keeps streaming.  (Attention K/V rows are not prefetched: requesting
+ * them into L2 ahead of the ring made the 16-sequence step 4 % slower on B200.)  Default 8 (measured fastest on B200, 0.7 % faster than 0 = off on the 8B batch-1 decode);
+ * at most 64. */
 int mk_set_l2_prefetch(mk_ctx* ctx, int stages);
 
 /* Split-KV chunk length floor: at attention length Lk, a (sequence, KV head) uses
@@ -217,6 +218,14 @@ int mk_set_l2_prefetch(mk_ctx* ctx, int stages);
  * save the arrival atomic and the merge on the critical path; more, shorter ones spread the keys
  * over more SMs.  Default 64; must be in [1, 2^20].  Results do not depend on it beyond rounding. */
 int mk_set_attn_chunk_keys(mk_ctx* ctx, int keys);
+
+/* Head mode of the decode attention: while the attention length Lk is at most `keys` (and the
+ * model has G > 1 query heads per KV head and at least G chunk tasks per group), chunk task
+ * c < G of a (sequence, KV head) computes query head c over all Lk keys and stores its output
+ * directly; no partial is written or merged, so the arrival atomic and the merge leave the
+ * critical path.  Longer lengths split the keys (mk_set_attn_chunk_keys).  0 turns head mode
+ * off.  Default 640; must be in [0, 2^20].  Results do not depend on it beyond rounding. */
+int mk_set_attn_head_keys(mk_ctx* ctx, int keys);
 
 /* Tracing (per-task timing of the next decode steps).  device_buffer: n_tasks * 6 uint64
  * records (n_tasks from mk_get_graph_info), or NULL to switch tracing off.  Record of task i

@@ -88,6 +88,7 @@ _SIGS = {
     "mk_debug_drop_notify": ([_vp, _i32, _i32], _i32),
     "mk_set_l2_prefetch": ([_vp, _i32], _i32),
     "mk_set_attn_chunk_keys": ([_vp, _i32], _i32),
+    "mk_set_attn_head_keys": ([_vp, _i32], _i32),
     "mk_set_dispatch": ([_vp, _i32, _i32, _vp], _i32),
     "mk_set_sm_weights": ([_vp, _vp, _i32, _vp], _i32),
     "mk_set_op_sm_weights": ([_vp, _i32, _vp, _i32, _vp], _i32),
@@ -253,6 +254,10 @@ def mk_set_l2_prefetch(ctx, stages: int):
 
 def mk_set_attn_chunk_keys(ctx, keys: int):
     _check(_lib.mk_set_attn_chunk_keys(ctx, int(keys)), ctx)
+
+
+def mk_set_attn_head_keys(ctx, keys: int):
+    _check(_lib.mk_set_attn_head_keys(ctx, int(keys)), ctx)
 
 
 def mk_set_dispatch(ctx, mode: int, tasks_per_sm: int = 2, stream=None):

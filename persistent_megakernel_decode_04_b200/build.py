@@ -7,6 +7,7 @@ is written next to the library as libmk.ptxas.txt.
 from __future__ import annotations
 
 import glob
+import time
 import os
 import subprocess
 import sys
@@ -43,6 +44,7 @@ def build(force: bool = False, verbose: bool = False, csrc: str | None = None, o
     objdir = os.path.join(os.path.dirname(so), "_build")
     os.makedirs(objdir, exist_ok=True)
     objs, report = [], []
+    t_start = time.time()  # sources edited while this build runs must leave the library stale
     common = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include"), "-I", src_dir]
     common += [f"-D{d}" for d in defines]
     srcs = sorted(glob.glob(os.path.join(src_dir, "*.cu")) + glob.glob(os.path.join(src_dir, "*.cpp")))
@@ -60,11 +62,12 @@ def build(force: bool = False, verbose: bool = False, csrc: str | None = None, o
     tmp = so + ".tmp"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lrt", "-lpthread"])
     os.replace(tmp, so)
+    os.utime(so, (t_start, t_start))
     with open(os.path.join(os.path.dirname(so), "libmk.ptxas.txt"), "w") as f:
         f.write("\n".join(report))
     if verbose:
         print("\n".join(report))
-    return SO
+    return so
 
 
 if __name__ == "__main__":

@@ -380,8 +380,19 @@ __device__ __forceinline__ float norm_factor(const DSmem& S, int K, float eps, i
 // With QK-norm the q and k rows are stored as they are (qbuf, kraw; natural dim order): the
 // LayerNorm needs a whole head, which the attention task of its KV head holds, so the norm
 // and RoPE of q and of the new key happen there.
+// RoPE angle (cos, sin) that packed QKV row R of sequence b takes at step st: (1, 0) for v rows
+// and with QK-norm (whose RoPE runs in the attention task).  A constant table: callers may load
+// it before the task's inputs exist.
+__device__ __forceinline__ float2 qkv_rope_angle(const DecodeParams& P, int R, int b, int st) {
+  const int D = P.D, G = P.nq / P.nkv;
+  const int rr = R % ((G + 2) * D);
+  if (P.qk_norm || rr >= (G + 1) * D) return make_float2(1.f, 0.f);
+  const int pd = (rr < G * D) ? (rr % D) : (rr - G * D);
+  return __ldg(P.rope + (size_t)(P.pos[b] + st) * (D / 2) + (pd >> 1));
+}
+
 __device__ __forceinline__ void qkv_out(const DecodeParams& P, int layer, int R, int b, float v, float other,
-                                        int st) {
+                                        int st, float2 cs) {
   const int D = P.D, G = P.nq / P.nkv, half = D / 2;
   const int rpg = (G + 2) * D;
   const int grp = R / rpg, rr = R % rpg;
@@ -400,7 +411,6 @@ __device__ __forceinline__ void qkv_out(const DecodeParams& P, int layer, int R,
         P.kraw[((size_t)layer * P.B + b) * P.nkv * D + (size_t)grp * D + dim] = v;
       return;
     }
-    const float2 cs = P.rope[(size_t)pos * half + i];
     float outv;
     int dim;
     if (hi == 0) {
@@ -425,12 +435,13 @@ __device__ __forceinline__ void qkv_out(const DecodeParams& P, int layer, int R,
 }
 
 template <int BM>
-__device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, const Task& t, float r, int st) {
+__device__ __forceinline__ void epi_qkv(const DecodeParams& P, const DSmem& S, const Task& t, float r, int st,
+                                        float2 cs) {
   const int tid = threadIdx.x;
   const int b = tid % BM;
   if (tid >= (int)t.nrows * BM || b >= P.nb) return;
   // the RoPE partner row (R ^ 1) of the same sequence sits at tid ^ BM
-  qkv_out(P, t.layer, (int)t.row0 + tid / BM, b, S.tot[tid] * r, S.tot[tid ^ BM] * r, st);
+  qkv_out(P, t.layer, (int)t.row0 + tid / BM, b, S.tot[tid] * r, S.tot[tid ^ BM] * r, st, cs);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -454,25 +465,51 @@ constexpr int kAttnBlock = 8;  // keys per warp per block
 template <int D>
 __host__ __device__ constexpr int kv_stage_keys() { return kSlotBytes / (2 * D * 2); }
 
+// How the chunk tasks of a (sequence, KV head) share the work at one step.
+enum AttnMode : int {
+  AM_SPLIT = 0,     // chunk c takes keys [j0, j1) for all G heads; the last to arrive merges
+  AM_HEAD = 1,      // short length: chunk c < G takes query head c over every key, no merge
+  AM_INACTIVE = 2,  // sequence outside the active batch: nothing to compute
+};
+
 struct AttnGeom {
   int b, g, c, Lk, nch_eff, j0, j1, pos0;
+  int mode;  // AttnMode
+  int h0;    // first query head of the task within the group (head mode: c)
+  int gh;    // query heads the task computes (G, or 1 in head mode)
 };
 
 // Chunk of an attention task at step st of the launch: keys [j0, j1) of Lk = pos + 1; pos0 is
 // the sequence's position at the launch's first step (rows at or past it are written during
-// this launch).
+// this launch).  Up to head_keys keys (and with G > 1 query heads per KV head, at least G
+// chunks) the group runs in head mode: every key of one query head per chunk, so no partial
+// is merged; the chunks c >= G have no work.  Longer lengths split the keys.
 __device__ __forceinline__ AttnGeom attn_geom(const DecodeParams& P, const Task& t, int st) {
   AttnGeom a;
+  const int G = P.nq / P.nkv;
   a.b = (int)t.row0 / P.nkv;
   a.g = (int)t.row0 % P.nkv;
   a.c = t.aux;
   a.pos0 = P.pos[a.b];
   a.Lk = P.pos[a.b] + st + 1;
+  a.h0 = 0;
+  a.gh = G;
   if (a.b >= P.nb) {  // sequence not in the active batch: its tasks only count their arrival
+    a.mode = AM_INACTIVE;
     a.nch_eff = 0;
     a.j0 = a.j1 = 0;
     return a;
   }
+  if (G > 1 && P.nch >= G && a.Lk <= P.head_keys) {
+    a.mode = AM_HEAD;
+    a.nch_eff = G;
+    a.h0 = a.c < G ? a.c : 0;
+    a.gh = 1;
+    a.j0 = 0;
+    a.j1 = a.c < G ? a.Lk : 0;
+    return a;
+  }
+  a.mode = AM_SPLIT;
   a.nch_eff = max(1, min(P.nch, (a.Lk + P.min_chunk_keys - 1) / P.min_chunk_keys));
   const int cl = (a.Lk + a.nch_eff - 1) / a.nch_eff;
   a.j0 = a.c * cl;
@@ -868,12 +905,13 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
   const int G = P.nq / P.nkv;
   const AttnGeom a = attn_geom(P, t, st);
   const int g = a.g, b = a.b, c = a.c, nch_eff = a.nch_eff, pos = a.Lk - 1;
+  const int Gt = a.gh, hb = g * G + a.h0;  // the task's query heads: hb .. hb + Gt - 1
   const uint16_t* kc = attn_cache<D>(P, t, a, 0);
   const uint16_t* vc = attn_cache<D>(P, t, a, 1);
-  const float* qsrc = P.qbuf + ((size_t)t.layer * P.B + b) * P.nq * D + (size_t)g * G * D;
+  const float* qsrc = P.qbuf + ((size_t)t.layer * P.B + b) * P.nq * D + (size_t)hb * D;
   // partial of (head h, chunk cc) of this sequence at part_base + (h * nch + cc) * (D + 2)
   float* part_base = P.part + ((size_t)t.layer * P.B + b) * P.nq * (size_t)P.nch * (D + 2);
-  float* o = P.obuf + ((size_t)t.layer * P.B + b) * P.nq * D + (size_t)g * G * D;
+  float* o = P.obuf + ((size_t)t.layer * P.B + b) * P.nq * D + (size_t)hb * D;
 
   if (c < nch_eff) {  // uniform across the CTA
     float qv[4][DL], m[4], l[4], acc[4][DL];
@@ -887,20 +925,20 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       // release.
       const uint16_t* nb = qk_norm_params(P, t.layer);
       const bool key_here = a.j0 <= pos && pos < a.j1;  // uniform across the CTA
-      const int head = warp < G ? g * G + warp : (warp == kAttnWarps - 1 && key_here) ? 2 * P.nq + g : -1;
+      const int head = warp < Gt ? hb + warp : (warp == kAttnWarps - 1 && key_here) ? 2 * P.nq + g : -1;
       if (head >= 0) {  // warp-uniform
         float v[DL], gn[DL], bn[DL];
         float2 cs[DL];
-        const float* src = warp < G ? qsrc + warp * D : P.kraw + ((size_t)t.layer * P.B + b) * P.nkv * D + (size_t)g * D;
+        const float* src = warp < Gt ? qsrc + warp * D : P.kraw + ((size_t)t.layer * P.B + b) * P.nkv * D + (size_t)g * D;
 #pragma unroll
         for (int i = 0; i < DL; ++i) {
           v[i] = __ldcg(src + lane * DL + i);
           cs[i] = P.rope[(size_t)pos * (D / 2) + (lane & 15) * DL + i];
         }
         qk_param_load<D>(nb, head, lane, gn);
-        qk_param_load<D>(nb, warp < G ? P.nq + head : head + P.nkv, lane, bn);
+        qk_param_load<D>(nb, warp < Gt ? P.nq + head : head + P.nkv, lane, bn);
         qk_norm_rope<D>(v, gn, bn, cs, P.eps, lane);
-        if (warp < G) {
+        if (warp < Gt) {
 #pragma unroll
           for (int i = 0; i < DL; ++i) S.qn[warp * D + lane * DL + i] = v[i];
         } else {
@@ -921,7 +959,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       l[h] = 0.f;
 #pragma unroll
       for (int i = 0; i < DL; ++i) {
-        qv[h][i] = (h < G) ? (QKN ? qsrc_n[h * D + lane * DL + i] : __ldcg(qsrc + h * D + lane * DL + i)) * P.attn_scale
+        qv[h][i] = (h < Gt) ? (QKN ? qsrc_n[h * D + lane * DL + i] : __ldcg(qsrc + h * D + lane * DL + i)) * P.attn_scale
                            : 0.f;
         acc[h][i] = 0.f;
       }
@@ -950,10 +988,10 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       // the scaled q of the group's heads in shared memory, read rotated by every lane (with
       // QK-norm S.qn already holds q, which every warp has first read into its registers)
       if (QKN) worker_bar();
-      for (int e = tid; e < G * D; e += kWorkerThreads)
+      for (int e = tid; e < Gt * D; e += kWorkerThreads)
         S.qn[e] = (QKN ? S.qn[e] : __ldcg(qsrc + e)) * P.attn_scale;
       worker_bar();
-      if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns)) S.cabort = 1u;
+      if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, Gt, m, l, acc, lane, warp, task_id, stall_ns)) S.cabort = 1u;
       for (int k = 0; k < nst; ++k) pp.advance();
     }
     // old positions from the ring, kv_stage_keys per stage (K rows at 0, V rows at KPS * D)
@@ -999,7 +1037,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
             }
           }
         }
-        if (valid) attn_block_g<D>(qv, kw, vw, valid, G, m, l, acc, lane);
+        if (valid) attn_block_g<D>(qv, kw, vw, valid, Gt, m, l, acc, lane);
       }
       // release the stage: one arrival per warp once its reads are done
       __syncwarp();
@@ -1017,12 +1055,12 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
           attn_load_key<D>(kc, vc, jf0 + idx, lane, kw[u], vw[u]);
         }
       }
-      if (valid) attn_block_g<D>(qv, kw, vw, valid, G, m, l, acc, lane);
+      if (valid) attn_block_g<D>(qv, kw, vw, valid, Gt, m, l, acc, lane);
     }
     // cross-warp merge of this chunk
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      if (h < G && warp < kAttnWarps) {
+      if (h < Gt && warp < kAttnWarps) {
         if (lane == 0) {
           S.am[warp][h] = m[h];
           S.al[warp][h] = l[h];
@@ -1033,7 +1071,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
     }
     worker_bar();
     if (S.cabort) return false;  // a ring wait ran out (uniform: written before the barrier)
-    for (int e = tid; e < G * D; e += kWorkerThreads) {
+    for (int e = tid; e < Gt * D; e += kWorkerThreads) {
       const int h = e / D, d = e % D;
       float M = -INFINITY;
 #pragma unroll
@@ -1047,8 +1085,8 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
           as += f * S.aacc[w][h][d];
         }
       }
-      if (nch_eff == 1) {
-        o[(size_t)h * D + d] = as / ls;  // the only chunk in use: final output, nothing to merge
+      if (nch_eff == 1 || a.mode == AM_HEAD) {
+        o[(size_t)h * D + d] = as / ls;  // the head's only chunk: final output, nothing to merge
       } else {
         float* pc = part_base + ((size_t)(g * G + h) * P.nch + c) * (D + 2);
         pc[2 + d] = as;
@@ -1060,6 +1098,20 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
     }
   }
   worker_bar();
+  if (a.mode == AM_HEAD) {
+    // No merge: the group's event count (nch per group and step) comes from every head task (1
+    // each, once its output is stored) and from chunk G for the chunks without work (nch - G).
+    // The arrival counter of split-mode steps advances by nch as if every chunk had arrived (one
+    // chunk adds it, before its release, which orders it for later steps).
+    if (tid == 0) {
+      const int c_cnt = P.nch > G ? G : 0;
+      if (c == c_cnt) red_relaxed_gpu_add(P.acnt + ((size_t)t.layer * P.B + b) * P.nkv + g, (uint32_t)P.nch);
+      const uint32_t add = c < G ? 1u : (c == G ? (uint32_t)(P.nch - G) : 0u);
+      if (add && (int)t.notify[0] != P.drop_event) red_release_gpu_add(&P.ev[t.notify[0]], add);
+    }
+    (void)task_id;
+    return true;
+  }
   if (tid == 0) {
     uint32_t* cnt = P.acnt + ((size_t)t.layer * P.B + b) * P.nkv + g;
     const uint32_t old = atom_acq_rel_gpu_add(cnt, 1u);
@@ -1117,7 +1169,8 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
     if (has1) o[(size_t)h1 * D + d1] = num1 / den1;
     worker_bar();
   }
-  if (S.flag && tid == 0 && (int)t.notify[0] != P.drop_event) red_release_gpu_add(&P.ev[t.notify[0]], 1u);
+  // the merge stands for every chunk of the group: nch counts of the event
+  if (S.flag && tid == 0 && (int)t.notify[0] != P.drop_event) red_release_gpu_add(&P.ev[t.notify[0]], (uint32_t)P.nch);
   (void)task_id;
   return true;
 }
@@ -1608,7 +1661,7 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
     const float r = gain ? 1.0f / sqrtf(ssum[b] / (float)K + P.eps) : 1.f;
     const float v = S.tile[e] * r;
     switch (t.kind) {
-      case TK_QKV: qkv_out(P, t.layer, R, b, v, S.tile[e ^ kTcBatch] * r, st); break;  // partner row R ^ 1
+      case TK_QKV: qkv_out(P, t.layer, R, b, v, S.tile[e ^ kTcBatch] * r, st, qkv_rope_angle(P, R, b, st)); break;  // partner row R ^ 1
       case TK_OPROJ: {
         const size_t at = (lay + b) * P.H + R;
         P.x_mid[at] = __ldcg(P.x_in + at) + v;
@@ -2167,26 +2220,35 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
         uint64_t off_unused;
         gemv_source<false>(P, t, &off_unused, &rb);
       }
+      // this thread's (row, sequence) in the epilogues, and the epilogue's other operand, loaded
+      // now so that its round trip overlaps the activation loads and the GEMV instead of
+      // following them: the residual (O projection, first down chunk), this thread's own sum of
+      // the earlier down chunks, or the RoPE angle of its QKV row
+      const int eb = tid % BMC, er = tid / BMC;
+      const bool mine = er < (int)t.nrows && eb < P.nb;
+      float2 e_op = make_float2(1.f, 0.f);  // QKV: (cos, sin); O, down: (residual, -)
+      if (mine) {
+        const size_t at = (lay + eb) * P.H + t.row0 + er;
+        if (t.kind == TK_QKV) e_op = qkv_rope_angle(P, (int)t.row0 + er, eb, st);
+        else if (!TP && t.kind == TK_OPROJ) e_op.x = __ldcg(P.x_in + at);
+        else if (!TP && t.kind == TK_DOWN) e_op.x = (t.aux == 0) ? __ldcg(P.x_mid + at) : P.x_in[P.B * P.H + at];
+      }
       const bool ok = (t.kind == TK_DOWN)
                           ? gemv_tile<NSEG_F, RPS_F, BMC>(P, S, pp, ring, xs, xstride, P.nb, gain, K, (int)t.nrows, rb,
                                                          i, stall)
                           : gemv_tile<NSEG_H, RPS_H, BMC, TP>(P, S, pp, ring, xs, xstride, P.nb, gain, K, (int)t.nrows,
                                                              rb, i, stall, xa);
       if (!ok) goto out;
-      // this thread's (row, sequence) in the epilogues
-      const int eb = tid % BMC, er = tid / BMC;
-      const bool mine = er < (int)t.nrows && eb < P.nb;
       const float r = gain ? norm_factor(S, K, P.eps, eb) : 1.f;
       switch (t.kind) {
-        case TK_QKV: epi_qkv<BMC>(P, S, t, r, st); break;
+        case TK_QKV: epi_qkv<BMC>(P, S, t, r, st, e_op); break;
         case TK_OPROJ:
           if (mine) {
             if constexpr (TP) {  // this rank's partial rows to every rank's receive buffer
               const size_t at = (((size_t)t.layer * P.tp_ranks + P.tp_rank) * P.B + eb) * P.H + t.row0 + er;
               for (int d = 0; d < P.tp_ranks; ++d) P.tp_recv_o[d][at] = S.tot[tid];
             } else {
-              const size_t at = (lay + eb) * P.H + t.row0 + er;
-              P.x_mid[at] = __ldcg(P.x_in + at) + S.tot[tid];
+              P.x_mid[(lay + eb) * P.H + t.row0 + er] = e_op.x + S.tot[tid];
             }
           }
           break;
@@ -2203,11 +2265,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
             for (int d = 0; d < P.tp_ranks; ++d) P.tp_recv_d[d][at] = S.tot[tid];
           } else if (mine) {
             // K chunk 0 starts from the residual; later chunks of the same rows ran earlier
-            // in this queue, on this thread, and add to what it stored
-            const size_t at = (lay + eb) * P.H + t.row0 + er;
-            float* dst = P.x_in + P.B * P.H + at;
-            const float base = (t.aux == 0) ? __ldcg(P.x_mid + at) : *dst;
-            *dst = base + S.tot[tid];
+            // in this queue, on this thread, and add to what it stored (both in e_op.x)
+            P.x_in[P.B * P.H + (lay + eb) * P.H + t.row0 + er] = e_op.x + S.tot[tid];
           }
           break;
         default:

@@ -88,6 +88,7 @@ struct mk_ctx {
   uint64_t* trace = nullptr;
   int l2_ahead = 8;  // L2 lookahead stages while the ring is full (mk_set_l2_prefetch)
   int min_chunk_keys = kMinChunkKeysDefault;  // split-KV chunk length floor (mk_set_attn_chunk_keys)
+  int head_keys = kHeadKeysDefault;           // head-mode attention up to this length (mk_set_attn_head_keys)
   std::vector<double> sm_weights;  // relative streaming speed per SM (partition weights)
   std::vector<double> op_weights[8];  // per projection kind; empty = sm_weights
   size_t task_cap = 0, lm_cap = 0; // workspace capacity for re-partitioned graphs
@@ -238,25 +239,12 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
       if (t.notify[k] < 0 || t.notify[k] >= nE)
         return fail(c, MK_ERR_INVALID_ARG, "task notify event out of range");
   }
-  // (b) thresholds equal producer counts (an attention group notifies once, from its merge)
+  // (b) thresholds equal producer counts (every attention chunk task counts once per step,
+  // whether its group's merge adds the counts of all its chunks or each head task its own)
   std::vector<uint32_t> produced(nE, 0);
   {
-    std::vector<std::vector<char>> seen(nE);
-    for (const VTask& t : T) {
-      if (t.kind == TK_ATTN) {
-        for (int k = 0; k < t.n_notify; ++k) {
-          auto& s = seen[t.notify[k]];
-          size_t key = (size_t)t.layer * B * nkv + t.row0;
-          if (s.size() <= key) s.resize(key + 1, 0);
-          if (!s[key]) {
-            s[key] = 1;
-            produced[t.notify[k]]++;
-          }
-        }
-      } else {
-        for (int k = 0; k < t.n_notify; ++k) produced[t.notify[k]]++;
-      }
-    }
+    for (const VTask& t : T)
+      for (int k = 0; k < t.n_notify; ++k) produced[t.notify[k]]++;
     if (c->tc) {  // the last task of each LM tile counts
       std::vector<char> seen((size_t)c->tc_tiles[TK_LMHEAD], 0);
       for (const VTask& t : T)
@@ -448,10 +436,12 @@ int validate(mk_ctx* c, const std::vector<VTask>& T, const std::vector<uint32_t>
           for (int w = 0; w < W; ++w) acc[w] |= gi[w];
           if (++attn_arrive[key] == c->nch) {
             // the merge runs after every chunk of the group: all their views hold, and the
-            // group's chunks are done
-            std::vector<int> done_cats;
+            // group's chunks are done; it adds one count per chunk (head mode adds the same
+            // counts from the chunks themselves, the last of them after every head's output)
+            std::vector<int> done_cats, none;
             for (int r = 0; r < c->nch; ++r) done_cats.push_back(cat_of(TK_ATTN, l));
-            for (int k = 0; k < t.n_notify; ++k) fire(t.notify[k], acc, done_cats);
+            for (int k = 0; k < t.n_notify; ++k)
+              for (int r = 0; r < c->nch; ++r) fire(t.notify[k], acc, r == 0 ? done_cats : none);
           }
         } else {
           for (int k = 0; k < t.n_notify; ++k) fire(t.notify[k], gi, tmp);
@@ -528,15 +518,9 @@ int validate_tp(mk_ctx* c, const std::vector<TVTask>& T, const std::vector<uint3
   // (b) thresholds, per rank
   std::vector<uint32_t> produced((size_t)R * nE, 0);
   {
-    std::vector<char> seen((size_t)R * nE * L * B * nkv + 1, 0);
     for (const TVTask& t : T) {
       for (int k = 0; k < t.n_notify; ++k) {
-        if (t.kind == TK_ATTN) {  // a (sequence, KV head) group notifies once, from its merge
-          if (t.layer >= L || t.row0 < 0 || t.row0 >= B * nkv) continue;
-          const size_t key = (((size_t)t.rank * nE + t.notify[k]) * L + t.layer) * B * nkv + t.row0;
-          if (seen[key]) continue;
-          seen[key] = 1;
-        }
+        // every attention chunk task counts once per step (see the single-device check)
         for (int d = 0; d < R; ++d)
           if (t.remote || d == t.rank) produced[(size_t)d * nE + t.notify[k]]++;
       }
@@ -729,10 +713,11 @@ int validate_tp(mk_ctx* c, const std::vector<TVTask>& T, const std::vector<uint3
           uint64_t* acc = &attn_acc[key * W];
           for (int w = 0; w < W; ++w) acc[w] |= Gb[w];
           if (++attn_arrive[key] == sh->nch) {
-            std::vector<int> done(sh->nch, cat_of(r, TK_ATTN, l));
+            std::vector<int> done(sh->nch, cat_of(r, TK_ATTN, l)), none;
             for (int k = 0; k < t.n_notify; ++k)
               for (int d = 0; d < R; ++d)
-                if (t.remote || d == r) fire(d, t.notify[k], acc, done);
+                if (t.remote || d == r)
+                  for (int x = 0; x < sh->nch; ++x) fire(d, t.notify[k], acc, x == 0 ? done : none);
           }
         } else {
           for (int k = 0; k < t.n_notify; ++k)
@@ -966,7 +951,9 @@ int build_graph(mk_ctx* c) {
       e.index = attn_p;
       for (int s2 = 0; s2 < n; ++s2) q[s2].push_back(e);
     }
-    evc[ev_attn(c, l)] = (uint32_t)(B * nkv);
+    // one count per chunk task and step: a split-mode merge adds its group's nch at once; in
+    // head mode each head task adds its own and one chunk adds those of the chunks without work
+    evc[ev_attn(c, l)] = (uint32_t)(B * nkv * c->nch);
     if (dyn) {
       auto o_edges = [&](Task& t) -> int {
         add_wait(t, ev_attn(c, l));
@@ -1737,6 +1724,7 @@ void make_params(const mk_ctx* c, const mk_ctx* run, const int32_t* tokens, int 
   P.trace = run->trace;
   P.l2_ahead = c->dyn ? 0 : run->l2_ahead;  // the lookahead walks static queues only
   P.min_chunk_keys = run->min_chunk_keys;
+  P.head_keys = run->head_keys;
   P.tp_ranks = 1;
 }
 
@@ -1966,6 +1954,12 @@ int mk_set_l2_prefetch(mk_ctx* c, int stages) {
 int mk_set_attn_chunk_keys(mk_ctx* c, int keys) {
   if (!c || keys < 1 || keys > (1 << 20)) return fail(c, MK_ERR_INVALID_ARG, "keys must be in [1, 2^20]");
   c->min_chunk_keys = keys;
+  return MK_OK;
+}
+
+int mk_set_attn_head_keys(mk_ctx* c, int keys) {
+  if (!c || keys < 0 || keys > (1 << 20)) return fail(c, MK_ERR_INVALID_ARG, "keys must be in [0, 2^20]");
+  c->head_keys = keys;
   return MK_OK;
 }
 

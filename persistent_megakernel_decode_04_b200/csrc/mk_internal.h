@@ -131,6 +131,7 @@ struct DecodeParams {
   uint64_t* trace;            // optional [n_tasks][kTraceWords] timing records (null = off)
   int l2_ahead;               // weight stages the producer prefetches into L2 beyond the ring
   int min_chunk_keys;         // split-KV: a chunk in use holds at least this many keys
+  int head_keys;              // up to this attention length a chunk takes one query head, no merge
   int nb;                     // active sequences (<= the kernel's batch width)
   int kdc, ndc;               // down-projection K chunk and chunk count
   float* tpart;               // tensor-core partial records [n_records][kTcRecFloats]
@@ -171,6 +172,7 @@ constexpr int kDynQ = 64;                 // run-time claims: task FIFO from the
 constexpr uint32_t kDynEnd = 0xffffffffu;  // FIFO entry: no more tasks in this launch
 constexpr uint64_t kStallPrefetchNs = 1000;    // producer blocked this long: prefetch ahead into L2
 constexpr uint64_t kStallPrefetchGapNs = 100;   // then one more stage per this interval
+constexpr int kHeadKeysDefault = 640;     // head-mode attention up to this length (mk_set_attn_head_keys)
 constexpr int kMinChunkKeysDefault = 64;  // split-KV chunks hold at least this many keys (mk_set_attn_chunk_keys)
 
 // Trace record per task (global-timer ns): worker start of the wait for inputs, inputs

@@ -43,15 +43,18 @@ def step_both(ref, m, tok, label):
     return oracle.argmax(rl)
 
 
-@pytest.mark.parametrize("shape,ranks", [(mi.TINY, 2), (mi.LLAMA8B.with_layers(2), 2),
-                                         (mi.LLAMA8B.with_layers(2), 4)])
-def test_tp_decode_over_a_filled_cache(shape, ranks):
+@pytest.mark.parametrize("shape,ranks,head_keys", [(mi.TINY, 2, 256), (mi.LLAMA8B.with_layers(2), 2, 256),
+                                                   (mi.LLAMA8B.with_layers(2), 2, 0),
+                                                   (mi.LLAMA8B.with_layers(2), 4, 256)])
+def test_tp_decode_over_a_filled_cache(shape, ranks, head_keys):
+    # head_keys 256: the attention of every step in head mode; 0: the keys split and merged
     w = mi.make_weights(shape, seed=31)
     L0, steps, max_seq = 100, 4, 128
     kv = mi.kv_cache_values(31, shape, 1, L0, sigma=1.0)
     ref = oracle.Decoder(w, 1, max_seq)
     ref.set_cache(kv, L0)
     m = tp_model(w, ranks, max_seq)
+    mk.mk_set_attn_head_keys(m.ctx, head_keys)
     fill_cache(m, kv, L0, ranks)
     m.set_positions([L0])
     tok = int(mi.prompt(31, 0, 1, shape.vocab)[0])
