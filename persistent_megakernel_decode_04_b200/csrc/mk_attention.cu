@@ -227,7 +227,7 @@ __device__ __forceinline__ bool flush_head(const Params& P, Smem& S, int h, int 
   __threadfence();
   const float* base = P.part + (size_t)h * P.maxc * (D + 2);
   float M2 = -INFINITY;
-  for (int i = 0; i < (int)n; ++i) M2 = fmaxf(M2, __ldcg(base + (size_t)i * (D + 2)));
+  for (int i = 0; i < (int)n; ++i) M2 = fmaxf(M2, ldcg_f32(base + (size_t)i * (D + 2)));
   float num[DL], den = 0.f;
 #pragma unroll
   for (int i = 0; i < DL; ++i) num[i] = 0.f;
@@ -237,10 +237,10 @@ __device__ __forceinline__ bool flush_head(const Params& P, Smem& S, int h, int 
     for (int k = 0; k < 8; ++k) {
       const bool in = i0 + k < (int)n;
       const float* pi = base + (size_t)(in ? i0 + k : 0) * (D + 2);
-      mv[k] = in ? __ldcg(pi) : -INFINITY;
-      lv[k] = in ? __ldcg(pi + 1) : 0.f;
+      mv[k] = in ? ldcg_f32(pi) : -INFINITY;
+      lv[k] = in ? ldcg_f32(pi + 1) : 0.f;
 #pragma unroll
-      for (int i = 0; i < DL; ++i) av[k][i] = in ? __ldcg(pi + 2 + lane * DL + i) : 0.f;
+      for (int i = 0; i < DL; ++i) av[k][i] = in ? ldcg_f32(pi + 2 + lane * DL + i) : 0.f;
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) {

@@ -256,13 +256,13 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
       float x[8];
       if (seg_ok(s) && (BM == 1 || b < nb)) {
         const float* xb = xsrc + (size_t)b * xstride;
-        float4 a = __ldcg(reinterpret_cast<const float4*>(xb + k));
-        float4 c = __ldcg(reinterpret_cast<const float4*>(xb + k + 4));
+        float4 a = ldcg_f4(xb + k);
+        float4 c = ldcg_f4(xb + k + 4);
         if constexpr (TPX) {
           for (int r = 0; r < xa.n + xa.n2; ++r) {
             const float* ad = (r < xa.n ? xa.add + (size_t)r * xa.stride : xa.add2 + (size_t)(r - xa.n) * xa.stride) + k;
-            const float4 u = __ldcg(reinterpret_cast<const float4*>(ad));
-            const float4 w = __ldcg(reinterpret_cast<const float4*>(ad + 4));
+            const float4 u = ldcg_f4(ad);
+            const float4 w = ldcg_f4(ad + 4);
             a.x += u.x; a.y += u.y; a.z += u.z; a.w += u.w;
             c.x += w.x; c.y += w.y; c.z += w.z; c.w += w.w;
           }
@@ -289,6 +289,14 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
 #pragma unroll
       for (int j = 0; j < 4; ++j) x2[b][s][j] = pack2(x[2 * j], x[2 * j + 1]);
     }
+  }
+  // the per-warp sums of x^2 for the fused norm, stored before the stage loop so that they do
+  // not stay live across it (read after the task's last worker barrier)
+#pragma unroll
+  for (int b = 0; b < BM; ++b) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss[b] += __shfl_xor_sync(0xffffffffu, ss[b], off);
+    if (lane == 0) S.ssw[warp][b] = ss[b];
   }
   float* red = S.red[warp];
   bool ok = true;
@@ -346,12 +354,6 @@ __device__ __forceinline__ bool gemv_tile(const DecodeParams& P, DSmem& S, Pipe&
       warp_reduce_rows<RSUB * BM>(a, red + (r0 + rs) * BM, lane, (nrows - r0 - rs) * BM);
     }
     pp.advance();
-  }
-#pragma unroll
-  for (int b = 0; b < BM; ++b) {
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) ss[b] += __shfl_xor_sync(0xffffffffu, ss[b], off);
-    if (lane == 0) S.ssw[warp][b] = ss[b];
   }
   worker_bar();
   if (S.cabort) return false;
@@ -529,13 +531,13 @@ template <int D>
 __device__ __forceinline__ void attn_load_key(const uint16_t* kc, const uint16_t* vc, int j, int lane,
                                               uint32_t (&kw)[D / 64], uint32_t (&vw)[D / 64]) {
   if (D == 128) {
-    const uint2 a = __ldcg(reinterpret_cast<const uint2*>(kc + (size_t)j * D + lane * 4));
-    const uint2 b = __ldcg(reinterpret_cast<const uint2*>(vc + (size_t)j * D + lane * 4));
+    const uint2 a = ldcg_u2(kc + (size_t)j * D + lane * 4);
+    const uint2 b = ldcg_u2(vc + (size_t)j * D + lane * 4);
     kw[0] = a.x; kw[(D / 64) - 1] = a.y;
     vw[0] = b.x; vw[(D / 64) - 1] = b.y;
   } else {
-    kw[0] = __ldcg(reinterpret_cast<const unsigned int*>(kc + (size_t)j * D + lane * 2));
-    vw[0] = __ldcg(reinterpret_cast<const unsigned int*>(vc + (size_t)j * D + lane * 2));
+    kw[0] = ldcg_u32(kc + (size_t)j * D + lane * 2);
+    vw[0] = ldcg_u32(vc + (size_t)j * D + lane * 2);
   }
 }
 
@@ -932,7 +934,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
         const float* src = warp < Gt ? qsrc + warp * D : P.kraw + ((size_t)t.layer * P.B + b) * P.nkv * D + (size_t)g * D;
 #pragma unroll
         for (int i = 0; i < DL; ++i) {
-          v[i] = __ldcg(src + lane * DL + i);
+          v[i] = ldcg_f32(src + lane * DL + i);
           cs[i] = P.rope[(size_t)pos * (D / 2) + (lane & 15) * DL + i];
         }
         qk_param_load<D>(nb, head, lane, gn);
@@ -959,7 +961,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       l[h] = 0.f;
 #pragma unroll
       for (int i = 0; i < DL; ++i) {
-        qv[h][i] = (h < Gt) ? (QKN ? qsrc_n[h * D + lane * DL + i] : __ldcg(qsrc + h * D + lane * DL + i)) * P.attn_scale
+        qv[h][i] = (h < Gt) ? (QKN ? qsrc_n[h * D + lane * DL + i] : ldcg_f32(qsrc + h * D + lane * DL + i)) * P.attn_scale
                            : 0.f;
         acc[h][i] = 0.f;
       }
@@ -989,7 +991,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       // QK-norm S.qn already holds q, which every warp has first read into its registers)
       if (QKN) worker_bar();
       for (int e = tid; e < Gt * D; e += kWorkerThreads)
-        S.qn[e] = (QKN ? S.qn[e] : __ldcg(qsrc + e)) * P.attn_scale;
+        S.qn[e] = (QKN ? S.qn[e] : ldcg_f32(qsrc + e)) * P.attn_scale;
       worker_bar();
       if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, Gt, m, l, acc, lane, warp, task_id, stall_ns)) S.cabort = 1u;
       for (int k = 0; k < nst; ++k) pp.advance();
@@ -1133,15 +1135,15 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
 #pragma unroll
       for (int k = 0; k < 16; ++k) {
         const bool ok = c0 + k < nch_eff;
-        v0[k] = (ok && has0) ? __ldcg(ph0 + (size_t)(c0 + k) * (D + 2)) : 0.f;
-        v1[k] = (ok && has1) ? __ldcg(ph1 + (size_t)(c0 + k) * (D + 2)) : 0.f;
+        v0[k] = (ok && has0) ? ldcg_f32(ph0 + (size_t)(c0 + k) * (D + 2)) : 0.f;
+        v1[k] = (ok && has1) ? ldcg_f32(ph1 + (size_t)(c0 + k) * (D + 2)) : 0.f;
       }
       if (c0 == 0) {
         for (int e = tid; e < G * nch_eff; e += kWorkerThreads) {
           const int h = e / nch_eff, cc = e % nch_eff;
           const float* pc = part_base + ((size_t)(g * G + h) * P.nch + cc) * (D + 2);
-          S.mg.mm[e] = __ldcg(pc);
-          S.mg.ll[e] = __ldcg(pc + 1);
+          S.mg.mm[e] = ldcg_f32(pc);
+          S.mg.ll[e] = ldcg_f32(pc + 1);
         }
         worker_bar();
       }
@@ -1284,7 +1286,7 @@ __device__ __forceinline__ bool epi_lmhead(const DecodeParams& P, DSmem& S, cons
         float v = -INFINITY;
         int idx = 0x7fffffff;
         for (int i = tid; i < P.n_lm; i += kWorkerThreads)
-          argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
+          argmax_merge(v, idx, ldcg_f32(P.lm_val + (size_t)i * P.B + b), ldcg_i32(P.lm_idx + (size_t)i * P.B + b));
         block_argmax(S, v, idx);
         if (TP && !tp_exchange_argmax(P, S, b, v, idx, st)) return false;
         if (tid == 0 && P.next_tokens) P.next_tokens[(size_t)st * P.B + b] = idx;
@@ -1404,8 +1406,8 @@ __device__ __forceinline__ bool tc_stage(const DecodeParams& P, DSmem& S, uint8_
       const int b = warp + h * kWorkerWarps;
       if (in && b < P.nb) {
         const float* xb = op.xs + (size_t)b * op.xstride + k;
-        xv[h][i][0] = __ldcg(reinterpret_cast<const float4*>(xb));
-        xv[h][i][1] = __ldcg(reinterpret_cast<const float4*>(xb + 4));
+        xv[h][i][0] = ldcg_f4(xb);
+        xv[h][i][1] = ldcg_f4(xb + 4);
       } else {
         xv[h][i][0] = xv[h][i][1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
@@ -1587,7 +1589,7 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
         for (int i = 0; i < kE; ++i) {
           const int e = tid + i * kWorkerThreads;
           r[q][i] = (sl0 + q < (int)t.pad0 && e < kTcRecFloats)
-                        ? __ldcg(rec0 + (size_t)(sl0 + q) * kTcRecFloats + e)
+                        ? ldcg_f32(rec0 + (size_t)(sl0 + q) * kTcRecFloats + e)
                         : 0.f;
         }
 #pragma unroll
@@ -1645,7 +1647,7 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
             float v = -INFINITY;
             int idx = 0x7fffffff;
             for (int i = lane; i < P.n_lm; i += 32)
-              argmax_merge(v, idx, __ldcg(P.lm_val + (size_t)i * P.B + b), __ldcg(P.lm_idx + (size_t)i * P.B + b));
+              argmax_merge(v, idx, ldcg_f32(P.lm_val + (size_t)i * P.B + b), ldcg_i32(P.lm_idx + (size_t)i * P.B + b));
             warp_argmax(v, idx);
             if (lane == 0) P.next_tokens[(size_t)st * P.B + b] = idx;
           }
@@ -1664,7 +1666,7 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
       case TK_QKV: qkv_out(P, t.layer, R, b, v, S.tile[e ^ kTcBatch] * r, st, qkv_rope_angle(P, R, b, st)); break;  // partner row R ^ 1
       case TK_OPROJ: {
         const size_t at = (lay + b) * P.H + R;
-        P.x_mid[at] = __ldcg(P.x_in + at) + v;
+        P.x_mid[at] = ldcg_f32(P.x_in + at) + v;
         break;
       }
       case TK_GATEUP:
@@ -1675,7 +1677,7 @@ __device__ __forceinline__ bool tc_finish(const DecodeParams& P, DSmem& S, const
         break;
       default: {  // down
         const size_t at = (lay + b) * P.H + R;
-        P.x_in[P.B * P.H + at] = __ldcg(P.x_mid + at) + v;
+        P.x_in[P.B * P.H + at] = ldcg_f32(P.x_mid + at) + v;
         break;
       }
     }
@@ -2230,8 +2232,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
       if (mine) {
         const size_t at = (lay + eb) * P.H + t.row0 + er;
         if (t.kind == TK_QKV) e_op = qkv_rope_angle(P, (int)t.row0 + er, eb, st);
-        else if (!TP && t.kind == TK_OPROJ) e_op.x = __ldcg(P.x_in + at);
-        else if (!TP && t.kind == TK_DOWN) e_op.x = (t.aux == 0) ? __ldcg(P.x_mid + at) : P.x_in[P.B * P.H + at];
+        else if (!TP && t.kind == TK_OPROJ) e_op.x = ldcg_f32(P.x_in + at);
+        else if (!TP && t.kind == TK_DOWN) e_op.x = (t.aux == 0) ? ldcg_f32(P.x_mid + at) : P.x_in[P.B * P.H + at];
       }
       const bool ok = (t.kind == TK_DOWN)
                           ? gemv_tile<NSEG_F, RPS_F, BMC>(P, S, pp, ring, xs, xstride, P.nb, gain, K, (int)t.nrows, rb,
@@ -2277,7 +2279,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
     } else if (t.kind == TK_EMBED) {
       for (int b = 0; b < P.nb; ++b) {
         // step 0: the caller's tokens; later steps: the previous step's greedy pick
-        int tok = (st == 0) ? __ldcg(P.tokens + b) : __ldcg(P.next_tokens + (size_t)(st - 1) * P.B + b);
+        int tok = (st == 0) ? ldcg_i32(P.tokens + b) : ldcg_i32(P.next_tokens + (size_t)(st - 1) * P.B + b);
         if (tok < 0 || tok >= (TP ? P.tp_vfull : P.V)) {  // never read outside the table: record, use row 0
           if (tid == 0 && t.row0 == 0) atomicCAS(&P.err[ERR_CODE], 0u, (uint32_t)DEV_ERR_BAD_TOKEN);
           tok = 0;
