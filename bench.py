@@ -48,6 +48,7 @@ WORKLOADS = {
     "llama8b-ctx4096": ("LLAMA8B", 1, 4096),
     "chameleon7b-b1": ("CHAMELEON7B", 1, 1024),
     "chameleon7b-b4": ("CHAMELEON7B", 4, 1024),
+    "chameleon7b-b4-cuda": ("CHAMELEON7B", 4, 1024),  # the same on the width-4 CUDA-core GEMV
     "chameleon7b-b16": ("CHAMELEON7B", 16, 1024),
     "chameleon7b-qk-b1": ("CHAMELEON7B_QK", 1, 1024),
     "chameleon7b-qk-b16": ("CHAMELEON7B_QK", 16, 1024),
@@ -57,7 +58,10 @@ WORKLOAD_TEXT = {
     "llama8b": "llama3-8b-shape decode, batch 1, 39-token prompt, greedy",
     "llama8b-ctx4096": "llama3-8b-shape decode, batch 1, 4096 cached positions (synthetic), greedy",
     "chameleon7b-b1": "chameleon-7b-shape MHA decode, batch 1, 1024 cached positions (synthetic), greedy",
-    "chameleon7b-b4": "chameleon-7b-shape MHA decode, batch 4, 1024 cached positions each (synthetic), greedy",
+    "chameleon7b-b4": "chameleon-7b-shape MHA decode, batch 4 (tensor-core projections), 1024 cached positions "
+                      "each (synthetic), greedy",
+    "chameleon7b-b4-cuda": "chameleon-7b-shape MHA decode, batch 4 (width-4 CUDA-core GEMV), 1024 cached positions "
+                           "each (synthetic), greedy",
     "chameleon7b-b16": "chameleon-7b-shape MHA decode, batch 16 (tensor-core projections), 1024 cached positions "
                        "each (synthetic), greedy",
     "chameleon7b-qk-b1": "chameleon-7b-shape MHA decode with QK-norm (LayerNorm per q/k head before RoPE), "
@@ -376,7 +380,10 @@ def run_mk(args, rank, world, local):
     os.environ.setdefault("MK_INPUT_THREADS", str(max(1, (os.cpu_count() or 1) // max(1, world))))
     weights = mi.make_weights(shape, seed=0)
     stream = torch.cuda.current_stream(dev)
-    m = mk.Megakernel(mk.Config.from_shape(shape, B, max_seq), weights, local, stream=stream)
+    cfg = mk.Config.from_shape(shape, B, max_seq)
+    if args.workload.endswith("-cuda"):
+        cfg.tc_min_batch = 5  # batches up to 4 on the CUDA-core GEMV
+    m = mk.Megakernel(cfg, weights, local, stream=stream)
     info = m.info()
     cpu_baseline = rank == 0 and not args.no_cpu_baseline and args.workload == "llama8b"
     if not cpu_baseline:

@@ -57,6 +57,12 @@ typedef struct mk_config {
    * a bias per head and element, before RoPE; the cache holds the normalised, rotated keys.
    * 0: none. */
   int qk_norm;
+  /* Smallest max_batch served by the tensor-core instantiation (the projections as 128-row
+   * tcgen05 tiles over N = 32 columns: 16 sequences' high and low bf16 parts, unused ones
+   * zero); smaller batches take the CUDA-core GEMV (width 1, or width 4 for 2..4 sequences).
+   * 2..5, or 0 for the default 2: every batched width on the tensor cores (on B200 batch 4
+   * runs 20 % faster there than on the width-4 GEMV).  5 keeps batches 2..4 on CUDA cores. */
+  int tc_min_batch;
 } mk_config;
 
 #define MK_MAX_BATCH 16

@@ -52,7 +52,7 @@ class mk_config(ctypes.Structure):
                 ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("ffn", ctypes.c_int),
                 ("vocab", ctypes.c_int), ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
                 ("max_batch", ctypes.c_int), ("max_seq", ctypes.c_int), ("tie_embeddings", ctypes.c_int),
-                ("qk_norm", ctypes.c_int)]
+                ("qk_norm", ctypes.c_int), ("tc_min_batch", ctypes.c_int)]
 
 
 _PP = ctypes.POINTER(ctypes.c_void_p)
@@ -384,6 +384,7 @@ class Config:
     max_batch: int = 1
     max_seq: int = 1024
     qk_norm: bool = False
+    tc_min_batch: int = 0  # 0: default (every batched width on the tensor cores); 5: CUDA-core GEMV up to 4
 
     @classmethod
     def from_shape(cls, shape, max_batch: int = 1, max_seq: int = 1024) -> "Config":
@@ -394,7 +395,7 @@ class Config:
     def c(self) -> mk_config:
         return mk_config(self.n_layers, self.hidden, self.n_q_heads, self.n_kv_heads, self.head_dim, self.ffn,
                          self.vocab, self.rms_eps, self.rope_theta, self.max_batch, self.max_seq, 0,
-                         int(self.qk_norm))
+                         int(self.qk_norm), int(self.tc_min_batch))
 
 
 class Megakernel:

@@ -1186,6 +1186,8 @@ int check_config(const mk_config* f, std::string* why) {
   if (f->max_seq < 1 || f->max_seq > (1 << 20)) return bad("max_seq out of range");
   if (f->tie_embeddings != 0) return bad("tied embeddings are not supported");
   if (f->qk_norm != 0 && f->qk_norm != 1) return bad("qk_norm must be 0 or 1");
+  if (f->tc_min_batch != 0 && (f->tc_min_batch < 2 || f->tc_min_batch > kMaxDecodeBatch + 1))
+    return bad("tc_min_batch must be 0 or in [2, 5]");
   if (f->hidden > 4 * kSegElems || f->ffn > 8 * kSegElems) return bad("hidden or ffn too large");
   return MK_OK;
 }
@@ -1276,7 +1278,10 @@ int init_ctx(mk_ctx* c) {
   // batch width: 1; or 4 (sequences beyond the active batch masked), where the down
   // projection runs in K chunks of kDownChunk so its activations fit in registers; or, for
   // more than 4 sequences, kTcBatch on the tensor cores
-  c->bm = (f.max_batch > kMaxDecodeBatch) ? kTcBatch : (f.max_batch > 1) ? 4 : 1;
+  {
+    const int tc_min = f.tc_min_batch ? f.tc_min_batch : kTcMinBatchDefault;
+    c->bm = (f.max_batch >= tc_min) ? kTcBatch : (f.max_batch > 1) ? 4 : 1;
+  }
   c->tc = c->bm == kTcBatch;
   c->task_rows = c->tc ? kTcUnitsMax : kTaskRows / c->bm;
   c->kdc = (c->bm == 4) ? std::min(f.ffn, kDownChunk) : f.ffn;

@@ -172,6 +172,7 @@ constexpr int kDynQ = 64;                 // run-time claims: task FIFO from the
 constexpr uint32_t kDynEnd = 0xffffffffu;  // FIFO entry: no more tasks in this launch
 constexpr uint64_t kStallPrefetchNs = 1000;    // producer blocked this long: prefetch ahead into L2
 constexpr uint64_t kStallPrefetchGapNs = 100;   // then one more stage per this interval
+constexpr int kTcMinBatchDefault = 2;    // max_batch from which the tensor-core instantiation runs
 constexpr int kHeadKeysDefault = 640;     // head-mode attention up to this length (mk_set_attn_head_keys)
 constexpr int kMinChunkKeysDefault = 64;  // split-KV chunks hold at least this many keys (mk_set_attn_chunk_keys)
 

@@ -35,7 +35,7 @@ def _cfg(**kw):
 
 @pytest.mark.parametrize("field,value", [("head_dim", 96), ("hidden", 250), ("n_kv_heads", 3), ("max_batch", 0),
                                          ("max_batch", 17), ("max_seq", 0), ("rms_eps", 0.0), ("vocab", 1),
-                                         ("qk_norm", 2)])
+                                         ("qk_norm", 2), ("tc_min_batch", 1), ("tc_min_batch", 6)])
 def test_bad_configs_are_rejected(field, value):
     with pytest.raises(mk.MkError) as e:
         mk.mk_build_taskgraph(_cfg(**{field: value}).c(), -1)

@@ -1,5 +1,6 @@
 """Batched decode against the CPU oracle, teacher-forced per sequence on the oracle's tokens:
-2..4 sequences on the CUDA-core batch-4 kernel, 5..16 on the tensor-core kernel.  Per-step
+2..16 sequences on the tensor-core kernel (the default), and 2..4 also on the CUDA-core
+batch-4 kernel (tc_min_batch = 5).  Per-step
 logits of every sequence, argmax, the bf16 KV cache, masking of sequences outside the active
 batch and per-sequence positions."""
 import numpy as np
@@ -15,8 +16,10 @@ pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda", 0)
 
 
-def _model(weights, max_batch, max_seq):
-    return mk.Megakernel(mk.Config.from_shape(weights.shape, max_batch, max_seq), weights, 0)
+def _model(weights, max_batch, max_seq, tc_min=0):
+    cfg = mk.Config.from_shape(weights.shape, max_batch, max_seq)
+    cfg.tc_min_batch = tc_min
+    return mk.Megakernel(cfg, weights, 0)
 
 
 def _step_both(ref, m, toks, label):
@@ -31,10 +34,10 @@ def _step_both(ref, m, toks, label):
     return [oracle.argmax(rl[b]) for b in range(B)]
 
 
-def _teacher_forced_batch(w, B, max_batch, T, steps, max_seq, seed):
+def _teacher_forced_batch(w, B, max_batch, T, steps, max_seq, seed, tc_min=0):
     prompts = np.stack([mi.prompt(seed, b, T, w.shape.vocab) for b in range(B)])
     ref = oracle.Decoder(w, B, max_seq)
-    m = _model(w, max_batch, max_seq)
+    m = _model(w, max_batch, max_seq, tc_min)
     rl = ref.prefill(prompts)
     gl = m.prefill(torch.from_numpy(prompts.astype(np.int32)).to(DEV)).cpu().numpy()
     for b in range(B):
@@ -48,19 +51,22 @@ def _teacher_forced_batch(w, B, max_batch, T, steps, max_seq, seed):
     m.close()
 
 
-def test_tiny_batch4_prefill_and_16_steps():
+@pytest.mark.parametrize("tc_min", [0, 5], ids=["tensor-core", "cuda-core"])
+def test_tiny_batch4_prefill_and_16_steps(tc_min):
     w = mi.make_weights(mi.TINY, seed=5)
-    _teacher_forced_batch(w, B=4, max_batch=4, T=12, steps=16, max_seq=64, seed=5)
+    _teacher_forced_batch(w, B=4, max_batch=4, T=12, steps=16, max_seq=64, seed=5, tc_min=tc_min)
 
 
+@pytest.mark.parametrize("tc_min", [0, 5], ids=["tensor-core", "cuda-core"])
 @pytest.mark.parametrize("B", [1, 2, 3])
-def test_tiny_partial_batch_is_masked(B):
-    # the batch-4 kernel serving fewer sequences: the unused slots compute nothing visible
+def test_tiny_partial_batch_is_masked(B, tc_min):
+    # a batched kernel serving fewer sequences: the unused slots compute nothing visible
     w = mi.make_weights(mi.TINY, seed=6)
-    _teacher_forced_batch(w, B=B, max_batch=4, T=9, steps=6, max_seq=32, seed=6 + B)
+    _teacher_forced_batch(w, B=B, max_batch=4, T=9, steps=6, max_seq=32, seed=6 + B, tc_min=tc_min)
 
 
-def test_tiny_batch4_ragged_positions():
+@pytest.mark.parametrize("tc_min", [0, 5], ids=["tensor-core", "cuda-core"])
+def test_tiny_batch4_ragged_positions(tc_min):
     # every sequence at its own position: RoPE angle, cache slot and attention length per sequence
     w = mi.make_weights(mi.TINY, seed=7)
     s = w.shape
@@ -70,7 +76,7 @@ def test_tiny_batch4_ragged_positions():
     ref = oracle.Decoder(w, 4, 64)
     ref.set_cache(kv, L)
     ref.set_positions(pos)
-    m = _model(w, 4, 64)
+    m = _model(w, 4, 64, tc_min)
     m.kv_view()[:, :, :4, :, :L, :] = torch.from_numpy(kv.view(np.int16)).to(DEV)
     m.set_positions(pos)
     toks = [3, 99, 512, 1000]
