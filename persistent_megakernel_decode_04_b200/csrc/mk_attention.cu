@@ -9,9 +9,10 @@
 // units [c*U/G, (c+1)*U/G), so every SM streams the same number of bytes.  A TMA producer
 // warp keeps a 3-stage ring of (K^T tile [d][128], V tile [128][d]) fp16 tiles full, in unit
 // order (a K^T tile is d rows of 256 contiguous bytes).  The eight compute warps work
-// independently and never wait for each other: warp w takes units u0 + w, u0 + w + 8, ..., each
-// with its own running (max, sum, acc) -- lane l scores keys 4l .. 4l+3 over all d, then owns
-// d/32 output dims in P.V -- and releases the stage it read.  At the end of its units of a
+// independently and never wait for each other: warp pair p takes units u0 + p, u0 + p + 4, ...,
+// warp 2p + h the unit's key half h, each warp with its own running (max, sum, acc) -- lane l
+// scores keys 64h + 2l, 64h + 2l + 1 over all d, then owns d/32 output dims in P.V -- and
+// both warps of the pair release the stage they read.  At the end of its units of a
 // head a warp leaves its partial in a shared-memory slot of the head and goes on (it already
 // loaded the next head's q); the last of the head's warps to arrive combines the slot into one
 // partial per (CTA, head), written out directly if the head lies inside the CTA, else merged by
@@ -268,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], 1);  // the one warp that read the stage releases it
+      mbar_init(&S.empty[s], 2);  // the warp pair that read the stage releases it
       S.armed[s] = 0xffffffffu;
     }
     for (int s = 0; s < 2; ++s) {
@@ -321,12 +322,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // ---------------- compute warps ----------------
-  // Warp w takes units u0 + w, u0 + w + 8, ... (heads in order), each with its own running
-  // (max, sum, acc); at the end of its units of a head it leaves its partial in the head's
-  // combine slot (flush_head) and goes on.  No compute-warp barrier: a wait that runs out
-  // makes the warp skip its remaining work.
+  // Warp pair p (warps 2p, 2p + 1) takes units u0 + p, u0 + p + 4, ... (heads in order); warp
+  // 2p + h takes key half h of each, with its own running (max, sum, acc), so a stage is held
+  // for half the time one warp would need.  At the end of its units of a head a warp leaves
+  // its partial in the head's combine slot (flush_head) and goes on.  No compute-warp barrier:
+  // a wait that runs out makes the warp skip its remaining work.
   constexpr int DL = D / 32;  // output dims per lane in P.V
-  constexpr int KPL = kUnit / 32;  // keys per lane in the scores (4)
+  constexpr int KPW = kUnit / 2;  // keys per warp (half a unit)
+  constexpr int KPL = KPW / 32;   // keys per lane in the scores (2)
+  constexpr int kPairs = kComputeWarps / 2;
+  const int kb = (warp & 1) * KPW;  // this warp's first key of a unit
   float* qs = S.qs[warp];
   float* ps = S.ps[warp];
   bool alive = true;
@@ -335,13 +340,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   float qn[DL];  // the next head's q (prefetched)
   auto flush = [&](int h) {
     const int a = max(u0, h * P.nu), b = min(u1, (h + 1) * P.nu);  // the head's units in this CTA
-    const int nw = min(kComputeWarps, b - a), w0 = (a - u0) & (kComputeWarps - 1);
+    // the head's warps: both warps of every pair that took one of its units
+    const int nw = 2 * min(kPairs, b - a), w0 = 2 * ((a - u0) & (kPairs - 1));
     if (alive && !flush_head<D>(P, S, h, c, w0, nw, m, l, acc, warp, lane)) {
       if (lane == 0) report_timeout(P.err, 3u, &S.abort);
       alive = false;
     }
   };
-  for (int u = u0 + warp; u < u1 && alive; u += kComputeWarps) {
+  for (int u = u0 + (warp >> 1); u < u1 && alive; u += kPairs) {
     const int h = u / P.nu;
     if (h != cur_h) {
       if (cur_h >= 0) flush(cur_h);
@@ -376,9 +382,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       alive = false;
       break;
     }
-    const int valid = min(kUnit, P.L - (u % P.nu) * kUnit);
-    // scores: lane owns keys KPL*lane .. KPL*lane + KPL-1; row dd of the K^T tile holds 128 keys
-    const uint16_t* kt = S.kt[stage] + lane * KPL;
+    const int valid = min(KPW, min(kUnit, P.L - (u % P.nu) * kUnit) - kb);  // this warp's keys
+    if (valid <= 0) {  // warp-uniform: the unit's second half lies past L
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[stage]);
+      continue;
+    }
+    // scores: lane owns keys kb + KPL*lane .. + KPL-1; row dd of the K^T tile holds 128 keys
+    const uint16_t* kt = S.kt[stage] + kb + lane * KPL;
     float sa[KPL], sb[KPL];
 #pragma unroll
     for (int k = 0; k < KPL; ++k) sa[k] = sb[k] = 0.f;
@@ -388,13 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const uint2 w = *reinterpret_cast<const uint2*>(kt + (dd + e) * kUnit);
-        const float2 k01 = h2f2(w.x), k23 = h2f2(w.y);
+        const float2 k01 = h2f2(*reinterpret_cast<const uint32_t*>(kt + (dd + e) * kUnit));
         float* s = (e & 1) ? sb : sa;
         s[0] = fmaf(qv[e], k01.x, s[0]);
         s[1] = fmaf(qv[e], k01.y, s[1]);
-        s[2] = fmaf(qv[e], k23.x, s[2]);
-        s[3] = fmaf(qv[e], k23.y, s[3]);
       }
     }
     float sc[KPL], bm = -INFINITY;
@@ -405,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-    const float m_new = fmaxf(m, bm);  // finite: the unit holds at least one key
+    const float m_new = fmaxf(m, bm);  // finite: the warp's half holds at least one key
     const float alpha = __expf(m - m_new);  // 0 on the head's first unit (m = -inf)
     float p[KPL], psum = 0.f;
 #pragma unroll
@@ -419,12 +427,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     m = m_new;
 #pragma unroll
     for (int i = 0; i < DL; ++i) acc[i] *= alpha;
-    *reinterpret_cast<float4*>(ps + KPL * lane) = make_float4(p[0], p[1], p[2], p[3]);
+    *reinterpret_cast<float2*>(ps + KPL * lane) = make_float2(p[0], p[1]);
     __syncwarp();
     // P.V: lane owns dims lane*DL .. lane*DL + DL - 1 (keys past L have p = 0 and zero rows)
-    const uint16_t* vt = S.v[stage] + lane * DL;
+    const uint16_t* vt = S.v[stage] + (size_t)kb * D + lane * DL;
 #pragma unroll 4
-    for (int k = 0; k < kUnit; k += 4) {
+    for (int k = 0; k < KPW; k += 4) {
       const float4 p4 = *reinterpret_cast<const float4*>(ps + k);
       const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll

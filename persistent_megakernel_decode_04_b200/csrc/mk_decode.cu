@@ -725,29 +725,35 @@ __device__ __forceinline__ int attn_stage_span(const AttnGeom& a, int* jend) {
   return *jend > a.j0 ? (*jend - a.j0 + kv_stage_keys<D>() - 1) / kv_stage_keys<D>() : 0;
 }
 
-// Wide attention (long chunks): warp w takes ring stages w, w + 8, ... of the chunk's cached keys,
-// each whole, with its own online softmax.  Lane l scores keys l*KPL .. l*KPL + KPL-1 of the
-// stage over every dim (reading its K words in the rotated order (t + l) mod (D/2), so the 32
-// lanes hit 32 banks, and the matching q words of the scaled q in S.qn), then owns D/32 output
-// dims of P.V, with the stage's probabilities read back as broadcasts from its row of S.wp.
-// Stages are taken out of order, so a warp first waits until its stage is armed with its
-// launch-wide number (S.armed), then on the stage's phase; it releases the stage for every
-// worker warp at once.  False if a wait ran out (the warp then skips its remaining stages).
+// Wide attention (long chunks): WPS warps share a stage.  With WPS = 1 warp w takes ring stages
+// w, w + 8, ... whole; with WPS = 2 the warp pair (2p, 2p + 1) takes stages p, p + 4, ..., warp
+// 2p + h the stage's key half h (the stage is held half as long, so the ring turns over faster,
+// at the price of loading q once per key instead of once per two).  Each warp keeps its own
+// online softmax.
+// Lane l scores keys l*KPL .. l*KPL + KPL-1 of its half over every dim (reading its K words in
+// the rotated order (t + l) mod (D/2), so the 32 lanes hit 32 banks, and the matching q words
+// of the scaled q in S.qn), then owns D/32 output dims of P.V, with its half's probabilities
+// read back as broadcasts from its row of S.wp.  Stages are taken out of order, so a warp first
+// waits until its stage is armed with its launch-wide number (S.armed), then on the stage's
+// phase; each warp sharing a stage releases it for 1/WPS of the worker warps.  False if a
+// wait ran out (the warp then skips its remaining stages).
 constexpr int kWideMinStages = 3;
 
-template <int D, int GW>
+template <int D, int GW, int WPS>
 __device__ __forceinline__ bool attn_wide(const DecodeParams& P, DSmem& S, const Pipe& pp, const uint8_t* ring,
                                           const AttnGeom& a, int jend, int nst, int G, float (&m)[4], float (&l)[4],
                                           float (&acc)[4][D / 32], int lane, int warp, uint32_t task_id,
                                           uint32_t& stall_ns) {
   constexpr int KPS = kv_stage_keys<D>();  // keys per stage: 64 (D = 128) or 128 (D = 64)
+  constexpr int KPW = KPS / WPS;            // keys per warp
   constexpr int W2 = D / 2;                 // 32-bit words (bf16 pairs) per K row
-  constexpr int KPL = KPS / 32;             // keys a lane scores
+  constexpr int KPL = KPW / 32;             // keys a lane scores
   constexpr int DL = D / 32;
-  float* pw = S.wp[warp];  // [GW][KPS]
+  float* pw = S.wp[warp];  // [GW][KPW]
   const float* qs = S.qn;  // [G][D], scaled
+  const int kb = (warp % WPS) * KPW;  // this warp's first key in a stage
   bool ok = true;
-  for (int i = warp; i < nst; i += kAttnWarps) {
+  for (int i = warp / WPS; i < nst; i += kAttnWarps / WPS) {
     int pos = pp.stage + i;
     uint32_t ph = pp.phase;
     while (pos >= pp.nst) {
@@ -785,14 +791,19 @@ __device__ __forceinline__ bool attn_wide(const DecodeParams& P, DSmem& S, const
     }
     const uint8_t* kst = ring + (size_t)pos * kSlotBytes;
     const uint16_t* vst = reinterpret_cast<const uint16_t*>(kst + KPS * D * 2);
-    const int nk = min(KPS, jend - (a.j0 + i * KPS));
+    const int nk = min(KPW, min(KPS, jend - (a.j0 + i * KPS)) - kb);  // this warp's keys (none if <= 0)
+    if (nk <= 0) {  // warp-uniform: an empty second half
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cnt(&S.empty[pos], kWorkerWarps / WPS);
+      continue;
+    }
     // scores of this lane's keys for every head
     float sc[KPL][GW];
 #pragma unroll
     for (int k = 0; k < KPL; ++k)
 #pragma unroll
       for (int h = 0; h < GW; ++h) sc[k][h] = 0.f;
-    const uint32_t* kwr = reinterpret_cast<const uint32_t*>(kst) + lane * KPL * W2;
+    const uint32_t* kwr = reinterpret_cast<const uint32_t*>(kst) + (kb + lane * KPL) * W2;
 #pragma unroll 4
     for (int t = 0; t < W2; ++t) {
       const int tr = (t + lane) & (W2 - 1);
@@ -826,7 +837,7 @@ __device__ __forceinline__ bool attn_wide(const DecodeParams& P, DSmem& S, const
 #pragma unroll
       for (int k = 0; k < KPL; ++k) {
         const float p = (lane * KPL + k < nk) ? __expf(sc[k][h] - m_new) : 0.f;
-        pw[h * KPS + lane * KPL + k] = p;
+        pw[h * KPW + lane * KPL + k] = p;
         psum += p;
       }
 #pragma unroll
@@ -839,12 +850,12 @@ __device__ __forceinline__ bool attn_wide(const DecodeParams& P, DSmem& S, const
     __syncwarp();
     // P.V: lane owns dims lane*DL .. lane*DL + DL-1; keys past nk are skipped (their V bytes are
     // stale, so they are not weighted by 0)
-    const uint16_t* vl = vst + lane * DL;
+    const uint16_t* vl = vst + (size_t)kb * D + lane * DL;
     const int n4 = nk & ~3;
     for (int k0 = 0; k0 < n4; k0 += 4) {
       float4 p4[GW];
 #pragma unroll
-      for (int h = 0; h < GW; ++h) p4[h] = *reinterpret_cast<const float4*>(pw + h * KPS + k0);
+      for (int h = 0; h < GW; ++h) p4[h] = *reinterpret_cast<const float4*>(pw + h * KPW + k0);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float v[DL];
@@ -875,25 +886,33 @@ __device__ __forceinline__ bool attn_wide(const DecodeParams& P, DSmem& S, const
 #pragma unroll
       for (int h = 0; h < GW; ++h) {
         if (h >= G) continue;
-        const float p = pw[h * KPS + k];
+        const float p = pw[h * KPW + k];
 #pragma unroll
         for (int d = 0; d < DL; ++d) acc[h][d] = fmaf(p, v[d], acc[h][d]);
       }
     }
     __syncwarp();  // every lane's reads of the stage and of pw are done
-    if (lane == 0) mbar_arrive_cnt(&S.empty[pos], kWorkerWarps);
+    if (lane == 0) mbar_arrive_cnt(&S.empty[pos], kWorkerWarps / WPS);
   }
   return ok;
 }
 
+// wps: warps per stage (1 or 2).  Head mode keeps whole stages per warp (its chunks are few
+// and the weight ring is deep enough); split chunks and the tensor-core kernel's 4-stage ring
+// turn over faster with warp pairs (measured on B200).
 template <int D>
 __device__ __forceinline__ bool attn_wide_g(const DecodeParams& P, DSmem& S, const Pipe& pp, const uint8_t* ring,
-                                            const AttnGeom& a, int jend, int nst, int G, float (&m)[4], float (&l)[4],
-                                            float (&acc)[4][D / 32], int lane, int warp, uint32_t task_id,
-                                            uint32_t& stall_ns) {
-  if (G == 1) return attn_wide<D, 1>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
-  if (G == 2) return attn_wide<D, 2>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
-  return attn_wide<D, 4>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+                                            const AttnGeom& a, int jend, int nst, int G, int wps, float (&m)[4],
+                                            float (&l)[4], float (&acc)[4][D / 32], int lane, int warp,
+                                            uint32_t task_id, uint32_t& stall_ns) {
+  if (wps == 2) {
+    if (G == 1) return attn_wide<D, 1, 2>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+    if (G == 2) return attn_wide<D, 2, 2>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+    return attn_wide<D, 4, 2>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+  }
+  if (G == 1) return attn_wide<D, 1, 1>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+  if (G == 2) return attn_wide<D, 2, 1>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+  return attn_wide<D, 4, 1>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
 }
 
 // QKN: the model has QK-norm (a separate instantiation, so the plain path keeps its registers).
@@ -993,7 +1012,9 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       for (int e = tid; e < Gt * D; e += kWorkerThreads)
         S.qn[e] = (QKN ? S.qn[e] : ldcg_f32(qsrc + e)) * P.attn_scale;
       worker_bar();
-      if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, Gt, m, l, acc, lane, warp, task_id, stall_ns)) S.cabort = 1u;
+      if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, Gt, (a.mode == AM_HEAD && !TC) ? 1 : 2, m, l, acc, lane,
+                          warp, task_id, stall_ns))
+        S.cabort = 1u;
       for (int k = 0; k < nst; ++k) pp.advance();
     }
     // old positions from the ring, kv_stage_keys per stage (K rows at 0, V rows at KPS * D)
