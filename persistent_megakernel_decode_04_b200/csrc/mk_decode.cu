@@ -991,20 +991,29 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
     // the free slots after the old rows of the last ring stage; each warp fetches up to
     // kFreshPre of its fresh slots together with q (one L2 round trip) and any others when the
     // stage is processed.  Fresh rows that do not fit (no stage, or no free slot) follow in
-    // blocks of kAttnBlock keys per warp read from memory.
+    // blocks of kAttnBlock keys per warp read from memory.  With whole stages per warp (wide)
+    // the fresh rows start at the first warp after those of the stages (an idle warp while
+    // the stages take fewer than all warps, else one of the first stages, which are in the ring
+    // at the release), and that warp fetches its first kFreshPre of them with q.
     constexpr int kFreshPre = 2;
     const int jf0 = max(a.j0, a.pos0), nf = max(0, a.j1 - jf0);
     int jend;
     const int nst = attn_stage_span<D>(a, &jend);
     const bool wide = nst >= kWideMinStages;  // long chunk: whole stages per warp (attn_wide)
+    const int wps = (a.mode == AM_HEAD && !TC) ? 1 : 2;  // wide: warps per stage
     const int nl = (nst > 0) ? (jend - a.j0) - (nst - 1) * KPS : 0;  // old rows in the last stage
     const int n_in = (nst > 0 && !wide) ? min(nf, KPS - nl) : 0;     // fresh rows in its free slots
     const int f_first = ((warp - nl) % kAttnWarps + kAttnWarps) % kAttnWarps;  // this warp's first fresh slot
+    // this warp's index in the blocks of fresh rows read from memory
+    const int fwarp = wide ? ((warp - wps * nst) % kAttnWarps + kAttnWarps) % kAttnWarps : warp;
     uint32_t kpre[kFreshPre][W], vpre[kFreshPre][W];
 #pragma unroll
-    for (int j = 0; j < kFreshPre; ++j)
+    for (int j = 0; j < kFreshPre; ++j) {
       if (f_first + kAttnWarps * j < n_in)
         attn_load_key<D>(kc, vc, jf0 + f_first + kAttnWarps * j, lane, kpre[j], vpre[j]);
+      else if (wide && fwarp + kAttnWarps * j < nf)
+        attn_load_key<D>(kc, vc, jf0 + fwarp + kAttnWarps * j, lane, kpre[j], vpre[j]);
+    }
     if (wide) {
       // the scaled q of the group's heads in shared memory, read rotated by every lane (with
       // QK-norm S.qn already holds q, which every warp has first read into its registers)
@@ -1012,8 +1021,7 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       for (int e = tid; e < Gt * D; e += kWorkerThreads)
         S.qn[e] = (QKN ? S.qn[e] : ldcg_f32(qsrc + e)) * P.attn_scale;
       worker_bar();
-      if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, Gt, (a.mode == AM_HEAD && !TC) ? 1 : 2, m, l, acc, lane,
-                          warp, task_id, stall_ns))
+      if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, Gt, wps, m, l, acc, lane, warp, task_id, stall_ns))
         S.cabort = 1u;
       for (int k = 0; k < nst; ++k) pp.advance();
     }
@@ -1072,10 +1080,18 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       uint32_t valid = 0;
 #pragma unroll
       for (int u = 0; u < kAttnBlock; ++u) {
-        const int idx = fb + warp + u * kAttnWarps;
+        const int idx = fb + fwarp + u * kAttnWarps;
         if (idx < nf) {
           valid |= 1u << u;
-          attn_load_key<D>(kc, vc, jf0 + idx, lane, kw[u], vw[u]);
+          if (wide && fb == 0 && u < kFreshPre) {  // fetched with q
+#pragma unroll
+            for (int w = 0; w < W; ++w) {
+              kw[u][w] = kpre[u < kFreshPre ? u : 0][w];
+              vw[u][w] = vpre[u < kFreshPre ? u : 0][w];
+            }
+          } else {
+            attn_load_key<D>(kc, vc, jf0 + idx, lane, kw[u], vw[u]);
+          }
         }
       }
       if (valid) attn_block_g<D>(qv, kw, vw, valid, Gt, m, l, acc, lane);

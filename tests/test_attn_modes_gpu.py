@@ -123,3 +123,40 @@ def test_head_keys_argument_checks():
         mk.mk_set_attn_head_keys(m.ctx, (1 << 20) + 1)
     mk.mk_set_attn_head_keys(m.ctx, 0)
     m.close()
+
+
+@pytest.mark.parametrize("head_keys,L0", [(1 << 20, 300), (0, 2400)], ids=["head", "split"])
+def test_llama8b_two_layers_whole_stage_chunks_with_fresh_rows(head_keys, L0):
+    """Chunks of three or more ring stages (whole stages per warp or warp pair) while a 12-step
+    launch writes fresh rows: the fresh rows go to the warps after those of the stages, the
+    first two of each such warp fetched with q.  Picks and logits against one-step launches, and
+    every step's logits against the oracle fed the same tokens."""
+    shape = mi.LLAMA8B.with_layers(2)
+    w = mi.make_weights(shape, seed=45)
+    steps, max_seq = 12, L0 + 16
+    tok0 = int(mi.prompt(45, 0, 1, shape.vocab)[0])
+    a, kv = _filled(w, L0, max_seq, head_keys, 45)
+    tok = torch.tensor([tok0], dtype=torch.int32, device=DEV)
+    picks, logits = [], []
+    for _ in range(steps):
+        lg, nt = a.decode(tok)
+        tok = nt.clone()
+        picks.append(int(tok.item()))
+        logits.append(lg[0].cpu().numpy().copy())
+    assert a.sync_status() == mk.MK_OK
+    a.close()
+    b, _ = _filled(w, L0, max_seq, head_keys, 45)
+    lg_b, out = b.decode_steps(torch.tensor([tok0], dtype=torch.int32, device=DEV), steps)
+    assert b.sync_status() == mk.MK_OK
+    assert np.array_equal(out.cpu().numpy()[:, 0], np.array(picks)), "multi-step picks differ from one-step launches"
+    assert np.abs(lg_b[0].cpu().numpy() - logits[-1]).max() <= 1e-3
+    n = L0 + steps
+    got_kv = b.kv_view()[:, :, :1, :, L0:n, :].cpu().numpy()
+    b.close()
+    ref = oracle.Decoder(w, 1, max_seq)
+    ref.set_cache(kv, L0)
+    for i, t in enumerate([tok0] + picks[:-1]):
+        rl = ref.decode(np.array([t], dtype=np.int32))[0]
+        logits_close(logits[i], rl, f"head_keys={head_keys} step {i}")
+        assert argmax_agrees(logits[i], rl, picks[i]), f"step {i}: pick is not the oracle's argmax with a clear margin"
+    kv_close(got_kv, ref.get_cache(n)[:, :, :, :, L0:n], "rows written inside the launch")
