@@ -63,6 +63,8 @@ struct DSmem {
   uint64_t acc_full[2];      // tensor-core accumulator complete (tcgen05.commit)
   uint64_t acc_free[2];      // ... and read back (one arrival per reading warp)
   uint64_t mma_done;         // every MMA issued so far completed (issuer drain at exit)
+  uint64_t kv_full[2];       // tensor-core attention: K/V stage loaded into operand buffer b
+  uint64_t kv_empty[2];      // ... and read by both warps of the last warp pair
   uint32_t tmem;             // tensor-memory accumulators (2 x kTcN columns)
   uint32_t ready;            // tasks [0, ready) of this queue have their inputs
   // ring stage s holds the stage with this launch-wide sequence number (published by the
@@ -739,21 +741,140 @@ __device__ __forceinline__ int attn_stage_span(const AttnGeom& a, int* jend) {
 // wait ran out (the warp then skips its remaining stages).
 constexpr int kWideMinStages = 3;
 
+// One whole stage (or its key half kb .. kb + KPW - 1) of wide attention: kst holds the stage's
+// K rows, then its V rows at KPS * D; nk (> 0) keys of this warp.  See attn_wide.
+template <int D, int GW, int WPS>
+__device__ __forceinline__ void attn_wide_stage(DSmem& S, const uint8_t* kst, int nk, int G, float (&m)[4],
+                                                float (&l)[4], float (&acc)[4][D / 32], int lane, int warp) {
+  constexpr int KPS = kv_stage_keys<D>();
+  constexpr int KPW = KPS / WPS;
+  constexpr int W2 = D / 2;
+  constexpr int KPL = KPW / 32;
+  constexpr int DL = D / 32;
+  float* pw = S.wp[warp];  // [GW][KPW]
+  const float* qs = S.qn;  // [G][D], scaled
+  const int kb = (warp % WPS) * KPW;
+  const uint16_t* vst = reinterpret_cast<const uint16_t*>(kst + KPS * D * 2);
+  // scores of this lane's keys for every head
+  float sc[KPL][GW];
+#pragma unroll
+  for (int k = 0; k < KPL; ++k)
+#pragma unroll
+    for (int h = 0; h < GW; ++h) sc[k][h] = 0.f;
+  const uint32_t* kwr = reinterpret_cast<const uint32_t*>(kst) + (kb + lane * KPL) * W2;
+#pragma unroll 4
+  for (int t = 0; t < W2; ++t) {
+    const int tr = (t + lane) & (W2 - 1);
+    float2 q2[GW];
+#pragma unroll
+    for (int h = 0; h < GW; ++h)
+      q2[h] = (h < G) ? *reinterpret_cast<const float2*>(qs + h * D + 2 * tr) : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+      const uint32_t w = kwr[k * W2 + tr];
+      const float k0 = bf16lo(w), k1 = bf16hi(w);
+#pragma unroll
+      for (int h = 0; h < GW; ++h) sc[k][h] = fmaf(q2[h].y, k1, fmaf(q2[h].x, k0, sc[k][h]));
+    }
+  }
+  // online softmax of each head over the stage's keys
+#pragma unroll
+  for (int h = 0; h < GW; ++h) {
+    if (h >= G) continue;
+    float bm = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+      if (lane * KPL + k >= nk) sc[k][h] = -INFINITY;
+      bm = fmaxf(bm, sc[k][h]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+    const float m_new = fmaxf(m[h], bm);  // finite: the stage holds at least one key
+    const float alpha = __expf(m[h] - m_new);
+    float psum = 0.f;
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+      const float p = (lane * KPL + k < nk) ? __expf(sc[k][h] - m_new) : 0.f;
+      pw[h * KPW + lane * KPL + k] = p;
+      psum += p;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+    l[h] = fmaf(l[h], alpha, psum);
+    m[h] = m_new;
+#pragma unroll
+    for (int d = 0; d < DL; ++d) acc[h][d] *= alpha;
+  }
+  __syncwarp();
+  // P.V: lane owns dims lane*DL .. lane*DL + DL-1; keys past nk are skipped (their V bytes are
+  // stale, so they are not weighted by 0)
+  const uint16_t* vl = vst + (size_t)kb * D + lane * DL;
+  const int n4 = nk & ~3;
+  for (int k0 = 0; k0 < n4; k0 += 4) {
+    float4 p4[GW];
+#pragma unroll
+    for (int h = 0; h < GW; ++h) p4[h] = *reinterpret_cast<const float4*>(pw + h * KPW + k0);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float v[DL];
+      if constexpr (DL == 4) {
+        const uint2 u = *reinterpret_cast<const uint2*>(vl + (k0 + e) * D);
+        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+      } else {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(vl + (k0 + e) * D);
+        v[0] = bf16lo(u); v[1] = bf16hi(u);
+      }
+#pragma unroll
+      for (int h = 0; h < GW; ++h) {
+        const float p = e == 0 ? p4[h].x : e == 1 ? p4[h].y : e == 2 ? p4[h].z : p4[h].w;
+#pragma unroll
+        for (int d = 0; d < DL; ++d) acc[h][d] = fmaf(p, v[d], acc[h][d]);
+      }
+    }
+  }
+  for (int k = n4; k < nk; ++k) {
+    float v[DL];
+    if constexpr (DL == 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(vl + k * D);
+      v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+    } else {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(vl + k * D);
+      v[0] = bf16lo(u); v[1] = bf16hi(u);
+    }
+#pragma unroll
+    for (int h = 0; h < GW; ++h) {
+      if (h >= G) continue;
+      const float p = pw[h * KPW + k];
+#pragma unroll
+      for (int d = 0; d < DL; ++d) acc[h][d] = fmaf(p, v[d], acc[h][d]);
+    }
+  }
+}
+
+// Tensor-core kernel: the last third of a whole-stage chunk's K/V stages are not streamed
+// through the ring but loaded into the two activation operand buffers, which attention tasks
+// leave idle, by the last warp pair itself (two stages in flight); the other pairs take the
+// ring stages.  That is 6 instead of 4 stages in flight per SM.
+static_assert(kTcBopBuf >= kSlotBytes, "a K/V ring stage fits one operand buffer");
+template <bool TC>
+__device__ __forceinline__ int attn_kv_op_stages(int nst) {
+  return (TC && nst >= kWideMinStages) ? nst / 3 : 0;
+}
+
 template <int D, int GW, int WPS>
 __device__ __forceinline__ bool attn_wide(const DecodeParams& P, DSmem& S, const Pipe& pp, const uint8_t* ring,
                                           const AttnGeom& a, int jend, int nst, int G, float (&m)[4], float (&l)[4],
                                           float (&acc)[4][D / 32], int lane, int warp, uint32_t task_id,
-                                          uint32_t& stall_ns) {
+                                          uint32_t& stall_ns, int nb, uint8_t* kvb, uint32_t kvn,
+                                          const uint16_t* kc, const uint16_t* vc) {
   constexpr int KPS = kv_stage_keys<D>();  // keys per stage: 64 (D = 128) or 128 (D = 64)
   constexpr int KPW = KPS / WPS;            // keys per warp
-  constexpr int W2 = D / 2;                 // 32-bit words (bf16 pairs) per K row
-  constexpr int KPL = KPW / 32;             // keys a lane scores
-  constexpr int DL = D / 32;
-  float* pw = S.wp[warp];  // [GW][KPW]
-  const float* qs = S.qn;  // [G][D], scaled
   const int kb = (warp % WPS) * KPW;  // this warp's first key in a stage
+  const int nr = nst - nb;            // ring stages; operand-buffer stages nr .. nst - 1
+  const int np = kAttnWarps / WPS - (nb > 0 ? 1 : 0);  // warp groups on ring stages
   bool ok = true;
-  for (int i = warp / WPS; i < nst; i += kAttnWarps / WPS) {
+  if (warp / WPS < np) {
+  for (int i = warp / WPS; i < nr; i += np) {
     int pos = pp.stage + i;
     uint32_t ph = pp.phase;
     while (pos >= pp.nst) {
@@ -790,110 +911,67 @@ __device__ __forceinline__ bool attn_wide(const DecodeParams& P, DSmem& S, const
       continue;
     }
     const uint8_t* kst = ring + (size_t)pos * kSlotBytes;
-    const uint16_t* vst = reinterpret_cast<const uint16_t*>(kst + KPS * D * 2);
     const int nk = min(KPW, min(KPS, jend - (a.j0 + i * KPS)) - kb);  // this warp's keys (none if <= 0)
-    if (nk <= 0) {  // warp-uniform: an empty second half
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cnt(&S.empty[pos], kWorkerWarps / WPS);
-      continue;
-    }
-    // scores of this lane's keys for every head
-    float sc[KPL][GW];
-#pragma unroll
-    for (int k = 0; k < KPL; ++k)
-#pragma unroll
-      for (int h = 0; h < GW; ++h) sc[k][h] = 0.f;
-    const uint32_t* kwr = reinterpret_cast<const uint32_t*>(kst) + (kb + lane * KPL) * W2;
-#pragma unroll 4
-    for (int t = 0; t < W2; ++t) {
-      const int tr = (t + lane) & (W2 - 1);
-      float2 q2[GW];
-#pragma unroll
-      for (int h = 0; h < GW; ++h)
-        q2[h] = (h < G) ? *reinterpret_cast<const float2*>(qs + h * D + 2 * tr) : make_float2(0.f, 0.f);
-#pragma unroll
-      for (int k = 0; k < KPL; ++k) {
-        const uint32_t w = kwr[k * W2 + tr];
-        const float k0 = bf16lo(w), k1 = bf16hi(w);
-#pragma unroll
-        for (int h = 0; h < GW; ++h) sc[k][h] = fmaf(q2[h].y, k1, fmaf(q2[h].x, k0, sc[k][h]));
-      }
-    }
-    // online softmax of each head over the stage's keys
-#pragma unroll
-    for (int h = 0; h < GW; ++h) {
-      if (h >= G) continue;
-      float bm = -INFINITY;
-#pragma unroll
-      for (int k = 0; k < KPL; ++k) {
-        if (lane * KPL + k >= nk) sc[k][h] = -INFINITY;
-        bm = fmaxf(bm, sc[k][h]);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-      const float m_new = fmaxf(m[h], bm);  // finite: the stage holds at least one key
-      const float alpha = __expf(m[h] - m_new);
-      float psum = 0.f;
-#pragma unroll
-      for (int k = 0; k < KPL; ++k) {
-        const float p = (lane * KPL + k < nk) ? __expf(sc[k][h] - m_new) : 0.f;
-        pw[h * KPW + lane * KPL + k] = p;
-        psum += p;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
-      l[h] = fmaf(l[h], alpha, psum);
-      m[h] = m_new;
-#pragma unroll
-      for (int d = 0; d < DL; ++d) acc[h][d] *= alpha;
-    }
-    __syncwarp();
-    // P.V: lane owns dims lane*DL .. lane*DL + DL-1; keys past nk are skipped (their V bytes are
-    // stale, so they are not weighted by 0)
-    const uint16_t* vl = vst + (size_t)kb * D + lane * DL;
-    const int n4 = nk & ~3;
-    for (int k0 = 0; k0 < n4; k0 += 4) {
-      float4 p4[GW];
-#pragma unroll
-      for (int h = 0; h < GW; ++h) p4[h] = *reinterpret_cast<const float4*>(pw + h * KPW + k0);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v[DL];
-        if constexpr (DL == 4) {
-          const uint2 u = *reinterpret_cast<const uint2*>(vl + (k0 + e) * D);
-          v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-        } else {
-          const uint32_t u = *reinterpret_cast<const uint32_t*>(vl + (k0 + e) * D);
-          v[0] = bf16lo(u); v[1] = bf16hi(u);
-        }
-#pragma unroll
-        for (int h = 0; h < GW; ++h) {
-          const float p = e == 0 ? p4[h].x : e == 1 ? p4[h].y : e == 2 ? p4[h].z : p4[h].w;
-#pragma unroll
-          for (int d = 0; d < DL; ++d) acc[h][d] = fmaf(p, v[d], acc[h][d]);
-        }
-      }
-    }
-    for (int k = n4; k < nk; ++k) {
-      float v[DL];
-      if constexpr (DL == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(vl + k * D);
-        v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-      } else {
-        const uint32_t u = *reinterpret_cast<const uint32_t*>(vl + k * D);
-        v[0] = bf16lo(u); v[1] = bf16hi(u);
-      }
-#pragma unroll
-      for (int h = 0; h < GW; ++h) {
-        if (h >= G) continue;
-        const float p = pw[h * KPW + k];
-#pragma unroll
-        for (int d = 0; d < DL; ++d) acc[h][d] = fmaf(p, v[d], acc[h][d]);
-      }
-    }
+    if (nk > 0) attn_wide_stage<D, GW, WPS>(S, kst, nk, G, m, l, acc, lane, warp);  // warp-uniform
     __syncwarp();  // every lane's reads of the stage and of pw are done
     if (lane == 0) mbar_arrive_cnt(&S.empty[pos], kWorkerWarps / WPS);
   }
+  return ok;
+  }
+  // the last warp group: operand-buffer stages.  Stage b of the chunk's nb is the CTA's
+  // operand-buffer load kvn + b, into buffer (kvn + b) & 1; its first warp's lane 0 issues the
+  // loads (the next one into a buffer once both warps released it) and every warp of the
+  // group waits for them, so none is left in flight when the task returns.
+  const bool lead = (warp % WPS) == 0;  // the group's first warp: its lane 0 issues, it drains
+  const uint64_t pol = policy_evict_first();
+  auto issue = [&](int b) {
+    const uint32_t g = kvn + (uint32_t)b, buf = g & 1u;
+    const int jj = a.j0 + (nr + b) * KPS;
+    const uint32_t bytes = (uint32_t)min(KPS, jend - jj) * D * 2u;
+    uint8_t* dst = kvb + (size_t)buf * kTcBopBuf;
+    fence_proxy_async_smem();  // after the generic accesses of the buffer's previous use
+    mbar_arrive_expect_tx(&S.kv_full[buf], 2u * bytes);
+    bulk_g2s(dst, kc + (size_t)jj * D, bytes, &S.kv_full[buf], pol);
+    bulk_g2s(dst + KPS * D * 2, vc + (size_t)jj * D, bytes, &S.kv_full[buf], pol);
+  };
+  int issued = nb < 2 ? nb : 2;  // loads issued (kept by the lead warp)
+  if (lead && lane == 0)
+    for (int b = 0; b < issued; ++b) issue(b);
+  int done = 0;  // stages whose load this warp saw land
+  for (int b = 0; b < nb && ok; ++b) {
+    const uint32_t g = kvn + (uint32_t)b, buf = g & 1u;
+    const bool got = __all_sync(0xffffffffu, wait_bar(&S.kv_full[buf], (g >> 1) & 1u, P.timeout_ns, &S));
+    if (!got) {
+      if (lane == 0) raise_error(P, S, DEV_ERR_WAIT_FULL, blockIdx.x, task_id);
+      ok = false;
+      break;
+    }
+    done = b + 1;
+    const int nk = min(KPW, min(KPS, jend - (a.j0 + (nr + b) * KPS)) - kb);
+    if (nk > 0) attn_wide_stage<D, GW, WPS>(S, kvb + (size_t)buf * kTcBopBuf, nk, G, m, l, acc, lane, warp);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.kv_empty[buf]);
+    if (lead && b + 2 < nb) {
+      // the buffer's next load, once both warps of the group released it (bounded)
+      int fok = 1;
+      if (lane == 0) {
+        fok = wait_bar(&S.kv_empty[buf], (g >> 1) & 1u, P.timeout_ns, &S) ? 1 : 0;
+        if (fok) issue(b + 2);
+        else raise_error(P, S, DEV_ERR_WAIT_EMPTY, blockIdx.x, task_id);
+      }
+      if (!__shfl_sync(0xffffffffu, fok, 0)) {
+        ok = false;
+        break;
+      }
+      issued = b + 3;
+    }
+  }
+  // after a wait that ran out: wait (bounded) for the loads issued but not seen landing
+  if (lead)
+    for (int b = done; b < issued; ++b) {
+      const uint32_t g = kvn + (uint32_t)b;
+      wait_bar(&S.kv_full[g & 1u], (g >> 1) & 1u, P.timeout_ns, nullptr);
+    }
   return ok;
 }
 
@@ -904,21 +982,26 @@ template <int D>
 __device__ __forceinline__ bool attn_wide_g(const DecodeParams& P, DSmem& S, const Pipe& pp, const uint8_t* ring,
                                             const AttnGeom& a, int jend, int nst, int G, int wps, float (&m)[4],
                                             float (&l)[4], float (&acc)[4][D / 32], int lane, int warp,
-                                            uint32_t task_id, uint32_t& stall_ns) {
+                                            uint32_t task_id, uint32_t& stall_ns, int nb, uint8_t* kvb,
+                                            uint32_t kvn, const uint16_t* kc, const uint16_t* vc) {
+#define MK_ATTN_WIDE(GW_, WPS_) \
+  attn_wide<D, GW_, WPS_>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns, nb, kvb, kvn, kc, vc)
   if (wps == 2) {
-    if (G == 1) return attn_wide<D, 1, 2>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
-    if (G == 2) return attn_wide<D, 2, 2>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
-    return attn_wide<D, 4, 2>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+    if (G == 1) return MK_ATTN_WIDE(1, 2);
+    if (G == 2) return MK_ATTN_WIDE(2, 2);
+    return MK_ATTN_WIDE(4, 2);
   }
-  if (G == 1) return attn_wide<D, 1, 1>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
-  if (G == 2) return attn_wide<D, 2, 1>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
-  return attn_wide<D, 4, 1>(P, S, pp, ring, a, jend, nst, G, m, l, acc, lane, warp, task_id, stall_ns);
+  if (G == 1) return MK_ATTN_WIDE(1, 1);
+  if (G == 2) return MK_ATTN_WIDE(2, 1);
+  return MK_ATTN_WIDE(4, 1);
+#undef MK_ATTN_WIDE
 }
 
 // QKN: the model has QK-norm (a separate instantiation, so the plain path keeps its registers).
 template <int D, bool TC, bool QKN>
 __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, Pipe& pp, const uint8_t* ring,
-                                               const Task& t, uint32_t task_id, uint32_t& stall_ns, int st) {
+                                               const Task& t, uint32_t task_id, uint32_t& stall_ns, int st,
+                                               uint8_t* kvb, uint32_t& kvn) {
   constexpr int DL = D / 32;
   constexpr int W = D / 64;
   constexpr int KPS = kv_stage_keys<D>();
@@ -1021,9 +1104,12 @@ __device__ __forceinline__ bool attention_task(const DecodeParams& P, DSmem& S, 
       for (int e = tid; e < Gt * D; e += kWorkerThreads)
         S.qn[e] = (QKN ? S.qn[e] : ldcg_f32(qsrc + e)) * P.attn_scale;
       worker_bar();
-      if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, Gt, wps, m, l, acc, lane, warp, task_id, stall_ns))
+      const int nb = attn_kv_op_stages<TC>(nst);  // stages loaded into the operand buffers
+      if (!attn_wide_g<D>(P, S, pp, ring, a, jend, nst, Gt, wps, m, l, acc, lane, warp, task_id, stall_ns, nb, kvb,
+                          kvn, kc, vc))
         S.cabort = 1u;
-      for (int k = 0; k < nst; ++k) pp.advance();
+      kvn += (uint32_t)nb;
+      for (int k = 0; k < nst - nb; ++k) pp.advance();
     }
     // old positions from the ring, kv_stage_keys per stage (K rows at 0, V rows at KPS * D)
     for (int st = 0; st < (wide ? 0 : nst); ++st) {
@@ -1509,7 +1595,7 @@ __device__ __forceinline__ void tc_issuer(const DecodeParams& P, DSmem& S, const
     if (t.kind == TK_ATTN) {
       int jend;
       const int nst = attn_stage_span<HD>(attn_geom(P, t, st), &jend);
-      for (int st = 0; st < nst; ++st) pp.advance();
+      for (int k = 0; k < nst - attn_kv_op_stages<true>(nst); ++k) pp.advance();  // its ring stages
       continue;
     }
     if (!is_gemv(t.kind)) continue;
@@ -1749,6 +1835,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
       mbar_init(&S.bop_free[b], 1);
       mbar_init(&S.acc_full[b], 1);
       mbar_init(&S.acc_free[b], 4);
+      mbar_init(&S.kv_full[b], 1);
+      mbar_init(&S.kv_empty[b], 2);
     }
     S.ready = 0;
     for (int s = 0; s < NST; ++s) S.armed[s] = 0xffffffffu;
@@ -1891,7 +1979,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
       const int nst = attn_stage_span<HD>(a, &jend);
       const uint16_t* kc = attn_cache<HD>(P, t, a, 0);
       const uint16_t* vc = attn_cache<HD>(P, t, a, 1);
-      for (int k = 0; k < nst; ++k) {
+      for (int k = 0; k < nst - attn_kv_op_stages<TC>(nst); ++k) {  // the ring's stages of the chunk
         const int jj = a.j0 + k * kv_stage_keys<HD>();
         const uint32_t bytes = (uint32_t)min(kv_stage_keys<HD>(), jend - jj) * HD * 2u;
         if (!wait_bar(&S.empty[pp.stage], pp.phase ^ 1u, P.timeout_ns, &S)) {
@@ -2086,6 +2174,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
   // whether the next task's first segment was staged ahead
   uint32_t gseg = 0, gtask = 0;
   bool staged_ahead = false;
+  uint32_t kvn = 0;  // K/V stages loaded into the operand buffers so far (tensor-core attention)
   // batch width 1: the next task's descriptor is loaded during the current task, so only the
   // activation loads remain after its release; wider kernels load it at the top of its own
   // iteration instead, which keeps 10 registers free across the GEMV
@@ -2327,7 +2416,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& P) {
       }
     } else if (t.kind == TK_ATTN) {
       notify = false;  // the last chunk to arrive notifies
-      if (!attention_task<HD, TC, QKN>(P, S, pp, ring, t, i, stall, st)) goto out;
+      if (!attention_task<HD, TC, QKN>(P, S, pp, ring, t, i, stall, st, bop, kvn)) goto out;
     }
     if (P.trace && tid == 0) {
       uint64_t* rec = P.trace + (size_t)i * kTraceWords;

@@ -153,3 +153,51 @@ def test_chameleon7b_1024_context(w_chameleon, B):
     got = m.kv_view()[:, :, :B, :, L:n, :].cpu().numpy()
     kv_close(got, ref.get_cache(n)[:, :, :, :, L:n], "kv cache (appended positions)")
     m.close()
+
+
+@pytest.mark.parametrize("L0", [400, 1000])
+def test_chameleon7b_two_layers_tensor_core_long_chunks_multistep(L0):
+    """Tensor-core kernel, 4 sequences, chunks of 7 and 16 ring stages: the last third of each
+    chunk's K/V stages is loaded into the idle operand buffers by the last warp pair (1000
+    positions reload each buffer), the rest comes through the ring.  A 6-step launch against
+    one-step launches (same picks, last logits within 1e-3), every step's logits against the
+    oracle fed the same tokens, and the rows written inside the launch."""
+    s = mi.CHAMELEON7B.with_layers(2)
+    w = mi.make_weights(s, seed=46)
+    B, steps, max_seq = 4, 6, L0 + 8
+    kv = mi.kv_cache_values(46, s, B, L0, sigma=1.0)
+    toks0 = [int(t) for t in mi.prompt(46, 0, B, s.vocab)]
+
+    def filled():
+        m = _model(w, B, max_seq)
+        m.kv_view()[:, :, :B, :, :L0, :] = torch.from_numpy(kv.view(np.int16)).to(DEV)
+        m.set_positions([L0] * B)
+        return m
+
+    a = filled()
+    tok = torch.tensor(toks0, dtype=torch.int32, device=DEV)
+    picks, logits = [], []
+    for _ in range(steps):
+        lg, nt = a.decode(tok)
+        tok = nt.clone()
+        picks.append(tok.cpu().numpy().copy())
+        logits.append(lg[:B].cpu().numpy().copy())
+    assert a.sync_status() == mk.MK_OK
+    a.close()
+    b = filled()
+    lg_b, out = b.decode_steps(torch.tensor(toks0, dtype=torch.int32, device=DEV), steps)
+    assert b.sync_status() == mk.MK_OK
+    assert np.array_equal(out.cpu().numpy()[:, :B], np.stack(picks)), "multi-step picks differ from one-step launches"
+    assert np.abs(lg_b[:B].cpu().numpy() - logits[-1]).max() <= 1e-3
+    n = L0 + steps
+    got_kv = b.kv_view()[:, :, :B, :, L0:n, :].cpu().numpy()
+    b.close()
+    ref = oracle.Decoder(w, B, max_seq)
+    ref.set_cache(kv, L0)
+    feed = [np.array(toks0, dtype=np.int32)] + [p.astype(np.int32) for p in picks[:-1]]
+    for i, t in enumerate(feed):
+        rl = ref.decode(t)
+        for q in range(B):
+            logits_close(logits[i][q], rl[q], f"step {i} sequence {q}")
+            assert argmax_agrees(logits[i][q], rl[q], int(picks[i][q])), f"step {i} sequence {q}: argmax"
+    kv_close(got_kv, ref.get_cache(n)[:, :, :, :, L0:n], "rows written inside the launch")
