@@ -157,9 +157,9 @@ def test_chameleon7b_1024_context(w_chameleon, B):
 
 @pytest.mark.parametrize("L0", [400, 1000])
 def test_chameleon7b_two_layers_tensor_core_long_chunks_multistep(L0):
-    """Tensor-core kernel, 4 sequences, chunks of 7 and 16 ring stages: the last third of each
-    chunk's K/V stages is loaded into the idle operand buffers by the last warp pair (1000
-    positions reload each buffer), the rest comes through the ring.  A 6-step launch against
+    """Tensor-core kernel, 4 sequences, chunks of 7 and 16 stages: the last quarter of each
+    chunk's K/V stages is loaded into the idle operand buffers by the last warp pair (at 1000
+    positions each buffer is loaded twice), the rest comes through the ring.  A 6-step launch against
     one-step launches (same picks, last logits within 1e-3), every step's logits against the
     oracle fed the same tokens, and the rows written inside the launch."""
     s = mi.CHAMELEON7B.with_layers(2)
